@@ -1,0 +1,260 @@
+/*
+ * pkv_oracle.c -- plain, slow, fp64 CPU oracle for one paged decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's
+ * CPU-baseline leg are the only callers. It shares no code, header, table or
+ * constant with the CUDA library; the two meet only through the seeded inputs
+ * that both consume.
+ *
+ * What it computes, and where the pages fix it:
+ *
+ *  - The KV cache is split into fixed-size blocks that need not be contiguous;
+ *    a per-sequence block table maps logical block j to a physical block, and
+ *    several requests may share physical blocks ("DeepSeek复刻vLLM反超原版",
+ *    section "vLLM：大模型推理的加速引擎与挑战"; "nano-vllm：轻量级大模型推理引擎的
+ *    技术探索与实践", section "PagedAttention 原理回顾"). The result is therefore
+ *    ordinary attention over each sequence's tokens in logical order:
+ *    out = softmax(scale * q K^T) V, evaluated here directly, in fp64, with no
+ *    blocking, splitting or online rescaling.
+ *  - The FP8 cache stores E4M3 codes ("nano-vllm-lite：深入理解LLM推理机制的教育级
+ *    开源项目", section 核心技术改进 3 "FP8 KV Cache量化"). The code set is the
+ *    OCP 8-bit floating point format, E4M3 variant: exponent bias 7, three
+ *    mantissa bits, subnormals at exponent field 0, S.1111.111 the only NaN,
+ *    no infinities, largest finite magnitude 448.
+ *
+ * Readings where the pages are silent (the same ones the CUDA library takes):
+ *  - pool layout [num_blocks][num_kv_heads][block_size][head_dim]; slot s is
+ *    block s / block_size, offset s % block_size;
+ *  - query head h reads KV head h / (num_q_heads / num_kv_heads);
+ *  - slot -1 means "do not write";
+ *  - FP8 store: y = x / scale[h] as one IEEE binary32 division, then the
+ *    nearest E4M3 value, ties to the even code, magnitudes beyond 448 clamped
+ *    to 448 (NaN stays NaN);
+ *  - FP8 read: code value times the head's scale, both exact in fp64.
+ *
+ * Every function here is pinned by a CPU test (brute force against a
+ * library softmax, invariants, closed forms, the OCP format points and a
+ * library FP8 cast); none is "parity unpinned".
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fopenmp -shared -fPIC.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_BOUNDS 5
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+double orc_bf16_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Value of one E4M3 code, from the format definition. */
+double orc_e4m3_to_double(uint8_t code)
+{
+    int sign = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double mag;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6); /* subnormal: 0.mmm * 2^(1-7) */
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7); /* normal: 1.mmm * 2^(e-7) */
+    return sign ? -mag : mag;
+}
+
+/*
+ * Nearest E4M3 code to y: codes 0x00..0x7E have increasing magnitude, so a
+ * binary search finds the code just below |y|; the nearer neighbour wins and
+ * an exact midpoint goes to the even code. Saturating: |y| >= 448 gives 448.
+ */
+uint8_t orc_e4m3_from_float(float y)
+{
+    uint8_t sign;
+    double a;
+    int lo, hi;
+    if (isnan(y))
+        return 0x7F;
+    sign = signbit(y) ? 0x80 : 0x00;
+    a = fabs((double)y);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    lo = 0;
+    hi = 0x7E;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (orc_e4m3_to_double((uint8_t)mid) <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    if (lo < 0x7E) {
+        double below = orc_e4m3_to_double((uint8_t)lo);
+        double above = orc_e4m3_to_double((uint8_t)(lo + 1));
+        double d_lo = a - below, d_hi = above - a;
+        if (d_hi < d_lo || (d_hi == d_lo && (lo & 1)))
+            lo += 1;
+    }
+    return sign | (uint8_t)lo;
+}
+
+/* Pool element index of (block, kv head, offset, dim) in the HND layout. */
+static int64_t pool_index(int64_t blk, int h, int off, int i, int nkv, int bs, int d)
+{
+    return ((blk * nkv + h) * bs + off) * (int64_t)d + i;
+}
+
+/*
+ * store_kvcache: write token t's K and V rows (all KV heads) into the pool
+ * slot slot_mapping[t]; slot -1 is skipped. Pools hold bf16 bit patterns
+ * (fp8 == 0) or E4M3 codes (fp8 != 0). A slot beyond the pool is not
+ * written and the call reports ORC_ERR_BOUNDS.
+ */
+int orc_store_kvcache(const uint16_t *k, const uint16_t *v, void *k_cache, void *v_cache,
+                      const int32_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                      int head_dim, int block_size, int64_t num_blocks, int fp8,
+                      const float *k_scale, const float *v_scale)
+{
+    int status = ORC_OK;
+    int64_t t;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping || num_tokens < 0 || num_kv_heads < 1 ||
+        head_dim < 1 || block_size < 1 || num_blocks < 1 || (fp8 && (!k_scale || !v_scale)))
+        return ORC_ERR_ARG;
+    for (t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        int64_t blk;
+        int off, h, i;
+        if (slot < 0)
+            continue;
+        if (slot >= num_blocks * (int64_t)block_size) {
+            status = ORC_ERR_BOUNDS;
+            continue;
+        }
+        blk = slot / block_size;
+        off = (int)(slot % block_size);
+        for (h = 0; h < num_kv_heads; ++h) {
+            for (i = 0; i < head_dim; ++i) {
+                int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim + i;
+                int64_t dst = pool_index(blk, h, off, i, num_kv_heads, block_size, head_dim);
+                if (fp8) {
+                    float kx = (float)orc_bf16_to_double(k[src]);
+                    float vx = (float)orc_bf16_to_double(v[src]);
+                    float ky = kx / k_scale[h];
+                    float vy = vx / v_scale[h];
+                    ((uint8_t *)k_cache)[dst] = orc_e4m3_from_float(ky);
+                    ((uint8_t *)v_cache)[dst] = orc_e4m3_from_float(vy);
+                } else {
+                    ((uint16_t *)k_cache)[dst] = k[src];
+                    ((uint16_t *)v_cache)[dst] = v[src];
+                }
+            }
+        }
+    }
+    return status;
+}
+
+/* One cached element as an exact fp64 value (bf16 bits, or code * scale). */
+static double cache_value(const void *cache, int64_t idx, int fp8, const float *scale, int h)
+{
+    if (fp8)
+        return orc_e4m3_to_double(((const uint8_t *)cache)[idx]) * (double)scale[h];
+    return orc_bf16_to_double(((const uint16_t *)cache)[idx]);
+}
+
+/*
+ * paged_attention_decode: for each of the S sequences (row s of q,
+ * block_tables and context_lens) and each query head h, attend over the
+ * context_lens[s] tokens whose K/V the block table locates, and write the
+ * fp64 result to out[s][h][:]. A sequence whose length or block ids fall
+ * outside the pool gets zeros and the call reports ORC_ERR_BOUNDS.
+ * num_threads > 1 spreads sequences over OpenMP threads (no change in the
+ * arithmetic of any one output).
+ */
+int orc_paged_attention_decode(const uint16_t *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_tables, int max_blocks_per_seq,
+                               const int32_t *context_lens, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                               float scale, int fp8, const float *k_scale, const float *v_scale,
+                               double *out, int num_threads)
+{
+    int status = ORC_OK;
+    int group, s;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || num_seqs < 0 ||
+        num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads || head_dim < 1 ||
+        block_size < 1 || num_blocks < 1 || max_blocks_per_seq < 1 ||
+        (fp8 && (!k_scale || !v_scale)))
+        return ORC_ERR_ARG;
+    group = num_q_heads / num_kv_heads;
+    if (num_threads < 1)
+        num_threads = 1;
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads) reduction(| : status)
+    for (s = 0; s < num_seqs; ++s) {
+        const int32_t *table = block_tables + (int64_t)s * max_blocks_per_seq;
+        double *out_s = out + (int64_t)s * num_q_heads * head_dim;
+        int ctx = context_lens[s];
+        int bad = (ctx < 1 || ctx > max_blocks_per_seq * block_size);
+        double *score, *w, *acc;
+        int h, t, i;
+        for (t = 0; !bad && t < ctx; t += block_size)
+            bad = (table[t / block_size] < 0 || table[t / block_size] >= num_blocks);
+        if (bad) {
+            memset(out_s, 0, sizeof(double) * (size_t)num_q_heads * head_dim);
+            status |= ORC_ERR_BOUNDS;
+            continue;
+        }
+        score = (double *)malloc(sizeof(double) * (size_t)ctx);
+        w = (double *)malloc(sizeof(double) * (size_t)ctx);
+        acc = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        for (h = 0; h < num_q_heads; ++h) {
+            int g = h / group;
+            const uint16_t *q_h = q + ((int64_t)s * num_q_heads + h) * head_dim;
+            double m = -INFINITY, z = 0.0;
+            for (t = 0; t < ctx; ++t) {
+                int64_t blk = table[t / block_size];
+                int off = t % block_size;
+                double dot = 0.0;
+                for (i = 0; i < head_dim; ++i) {
+                    int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
+                    dot += orc_bf16_to_double(q_h[i]) * cache_value(k_cache, idx, fp8, k_scale, g);
+                }
+                score[t] = (double)scale * dot;
+                if (score[t] > m)
+                    m = score[t];
+            }
+            for (t = 0; t < ctx; ++t) {
+                w[t] = exp(score[t] - m);
+                z += w[t];
+            }
+            /* out_i = sum_t w_t V[t][i] / z, summed in increasing t. */
+            for (i = 0; i < head_dim; ++i)
+                acc[i] = 0.0;
+            for (t = 0; t < ctx; ++t) {
+                int64_t blk = table[t / block_size];
+                int off = t % block_size;
+                for (i = 0; i < head_dim; ++i) {
+                    int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
+                    acc[i] += w[t] * cache_value(v_cache, idx, fp8, v_scale, g);
+                }
+            }
+            for (i = 0; i < head_dim; ++i)
+                out_s[(int64_t)h * head_dim + i] = acc[i] / z;
+        }
+        free(score);
+        free(w);
+        free(acc);
+    }
+    return status;
+}

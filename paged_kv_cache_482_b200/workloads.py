@@ -1,0 +1,294 @@
+"""Seeded synthetic inputs for one paged decode-attention step.
+
+This module only draws random numbers and lays out the bookkeeping that an
+engine's block manager would hand to the kernels: context lengths, block
+tables, the slot of every cached token, and the per-KV-head FP8 scales. It
+holds none of the attention arithmetic. Both the CUDA path and the CPU checker
+consume exactly what it returns, so neither can see the other's results.
+
+Workload shapes follow the benchmark the pages describe: many sequences with
+lengths drawn uniformly at random ("Nano-vLLM：轻量高效的大模型推理框架",
+section 五 "使用方法", the ``bench.py`` run over 256 sequences; "DeepSeek复刻vLLM
+反超原版", section "性能对决", 256 and 1024 sequences with lengths sampled
+between 100 and 1024 tokens). No dataset is involved: Q/K/V are N(0, 1) draws
+rounded to bf16, which stands in for real activations.
+
+Layout conventions shared with the C-ABI (they are readings, not page text):
+
+* KV pool ``[num_blocks, num_kv_heads, block_size, head_dim]`` (HND); a token
+  in slot ``s`` lives in block ``s // block_size`` at offset
+  ``s % block_size``.
+* ``context_lens[i]`` counts the new token of step i; it is the last token of
+  the sequence and is written by ``store_kvcache`` right before the decode.
+* ``slot_mapping == -1`` marks a token that must not be written (its block is
+  a shared prefix block that already holds it).
+* unused tail entries of a block table row are ``-1``.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+# Pool fill patterns for slots that no token was written to. A bf16 quiet NaN
+# and the E4M3 NaN code: any read of such a slot poisons the output.
+CANARY_BF16 = 0x7FC0
+CANARY_FP8 = 0x7F
+
+CACHE_BF16 = "bf16"
+CACHE_FP8 = "fp8_e4m3"
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    """Shape of one decode step over a paged KV cache.
+
+    ``ctx_lo``/``ctx_hi`` bound the uniform (inclusive) context length. When
+    ``prefix_tokens`` > 0 they bound the private suffix instead, and every
+    sequence's context is ``prefix_tokens + suffix``.
+    """
+
+    name: str
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    ctx_lo: int
+    ctx_hi: int
+    cache_dtype: str = CACHE_BF16
+    prefix_tokens: int = 0
+    pool_blocks: int | None = None  # None: blocks in use plus 10 %
+    scale: float | None = None  # None: 1/sqrt(head_dim)
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.head_dim)
+
+    @property
+    def max_context(self) -> int:
+        return self.prefix_tokens + self.ctx_hi
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return -(-self.max_context // self.block_size)
+
+    def with_(self, **kw) -> "DecodeConfig":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return DecodeConfig(**d)
+
+
+# The five workloads of the tier, by what they are.
+CONFIGS: dict[str, DecodeConfig] = {
+    c.name: c
+    for c in (
+        DecodeConfig("tiny", 4, 2, 1, 64, 16, 1, 300, pool_blocks=128, scale=1.0 / 8.0),
+        DecodeConfig("qwen3_0.6b", 256, 16, 8, 128, 256, 100, 2048),
+        DecodeConfig("qwen3_8b", 1024, 32, 8, 128, 256, 100, 2048),
+        DecodeConfig("prefix_shared", 512, 32, 8, 128, 256, 0, 512, prefix_tokens=1024),
+        DecodeConfig("long_fp8", 64, 32, 8, 128, 16, 16384, 32768, cache_dtype=CACHE_FP8),
+    )
+}
+
+
+@dataclass
+class Workload:
+    """All inputs of one decode step plus the history that fills the pool.
+
+    ``k_hist``/``v_hist``/``slot_hist`` hold every cached token that precedes
+    the step (for a shared prefix: once). ``k_new``/``v_new``/``slot_new`` are
+    the step's own tokens, one per sequence. ``hist_rows[i]`` lists the rows
+    of ``k_hist`` that sequence i's blocks hold, in logical order.
+    """
+
+    cfg: DecodeConfig
+    seed: int
+    num_blocks: int
+    q: torch.Tensor  # [S, nq, d] bf16
+    k_new: torch.Tensor  # [S, nkv, d] bf16
+    v_new: torch.Tensor
+    slot_new: torch.Tensor  # [S] int32
+    k_hist: torch.Tensor  # [H, nkv, d] bf16
+    v_hist: torch.Tensor
+    slot_hist: torch.Tensor  # [H] int32
+    block_tables: torch.Tensor  # [S, max_blocks] int32, -1 padded
+    context_lens: torch.Tensor  # [S] int32
+    hist_rows: list = field(default_factory=list)  # per seq: 1-D int64 tensor (CPU)
+    k_scale: torch.Tensor | None = None  # [nkv] fp32 (FP8 cache only)
+    v_scale: torch.Tensor | None = None
+
+    @property
+    def is_fp8(self) -> bool:
+        return self.cfg.cache_dtype == CACHE_FP8
+
+    def kv_tokens(self) -> int:
+        return int(self.context_lens.sum().item())
+
+
+def _randn_bf16(shape, gen: torch.Generator, device) -> torch.Tensor:
+    """N(0,1) fp32 draws rounded to bf16 (round-to-nearest-even), chunked."""
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    chunk = 1 << 26
+    for i in range(0, flat.numel(), chunk):
+        n = min(chunk, flat.numel() - i)
+        flat[i : i + n] = torch.randn(n, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+def _structure(cfg: DecodeConfig, seed: int):
+    """Context lengths and physical block ids (device independent, CPU)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    S, bs = cfg.num_seqs, cfg.block_size
+    draws = torch.randint(cfg.ctx_lo, cfg.ctx_hi + 1, (S,), generator=g, dtype=torch.int64)
+    ctx = draws + cfg.prefix_tokens
+    if cfg.prefix_tokens % bs:
+        raise ValueError("a shared prefix must fill whole blocks")
+    shared = cfg.prefix_tokens // bs
+    own = [-(-int(c) // bs) - shared for c in ctx]
+    in_use = shared + sum(own)
+    nblk = cfg.pool_blocks if cfg.pool_blocks is not None else in_use + -(-in_use // 10)
+    if nblk < in_use:
+        raise ValueError(f"pool of {nblk} blocks cannot hold {in_use}")
+    perm = torch.randperm(nblk, generator=g, dtype=torch.int64)
+    tables = torch.full((S, cfg.max_blocks_per_seq), -1, dtype=torch.int64)
+    tables[:, :shared] = perm[:shared]
+    nxt = shared
+    for i in range(S):
+        tables[i, shared : shared + own[i]] = perm[nxt : nxt + own[i]]
+        nxt += own[i]
+    return ctx, tables, nblk
+
+
+def generate(cfg: DecodeConfig, seed: int = 0, device: str | torch.device = "cpu") -> Workload:
+    """Draw one decode step's inputs for ``cfg``.
+
+    Lengths and block ids come from a CPU generator seeded with ``seed`` and
+    are the same on every device. Q/K/V come from a generator on ``device``
+    seeded with ``seed + 1`` (torch's CPU and CUDA generators give different
+    streams, so data drawn on different devices differ; each is reproducible).
+    """
+    device = torch.device(device)
+    ctx, tables, nblk = _structure(cfg, seed)
+    S, nkv, d, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    P = cfg.prefix_tokens
+
+    # Row lists: the shared prefix once, then each sequence's own cached tokens
+    # (every position below its last one).
+    hist_rows = []
+    own_start = []
+    n = P
+    for i in range(S):
+        own = max(int(ctx[i]) - 1 - P, 0)
+        own_start.append(n)
+        n += own
+    H = n
+    pos = torch.empty(H, dtype=torch.int64)
+    seq_of = torch.empty(H, dtype=torch.int64)
+    pos[:P] = torch.arange(P)
+    seq_of[:P] = 0  # prefix rows use any sequence's table (all share it)
+    for i in range(S):
+        own = max(int(ctx[i]) - 1 - P, 0)
+        s0 = own_start[i]
+        pos[s0 : s0 + own] = torch.arange(P, P + own)
+        seq_of[s0 : s0 + own] = i
+        # The shared blocks always hold the whole prefix.
+        rows = torch.cat([torch.arange(P), torch.arange(s0, s0 + own)])
+        hist_rows.append(rows)
+    slot_hist = tables[seq_of, pos // bs] * bs + pos % bs
+
+    last = ctx - 1
+    slot_new = tables[torch.arange(S), last // bs] * bs + last % bs
+    # The step's token at a position inside the shared prefix is already cached.
+    slot_new = torch.where(last < P, torch.full_like(slot_new, -1), slot_new)
+
+    gd = torch.Generator(device=device).manual_seed(seed + 1)
+    q = _randn_bf16((S, cfg.num_q_heads, d), gd, device)
+    k_hist = _randn_bf16((H, nkv, d), gd, device)
+    v_hist = _randn_bf16((H, nkv, d), gd, device)
+    k_new = _randn_bf16((S, nkv, d), gd, device)
+    v_new = _randn_bf16((S, nkv, d), gd, device)
+
+    wl = Workload(
+        cfg=cfg,
+        seed=seed,
+        num_blocks=nblk,
+        q=q,
+        k_new=k_new,
+        v_new=v_new,
+        slot_new=slot_new.to(torch.int32).to(device),
+        k_hist=k_hist,
+        v_hist=v_hist,
+        slot_hist=slot_hist.to(torch.int32).to(device),
+        block_tables=tables.to(torch.int32).to(device),
+        context_lens=ctx.to(torch.int32).to(device),
+        hist_rows=hist_rows,
+    )
+    if cfg.cache_dtype == CACHE_FP8:
+        # One fp32 scale per KV head: the head's absolute maximum over every
+        # token of the step, divided by the largest E4M3 magnitude (448).
+        written = (slot_new >= 0).to(device)
+        kmax = k_hist.abs().amax(dim=(0, 2)) if H else torch.zeros(nkv, dtype=torch.bfloat16, device=device)
+        vmax = v_hist.abs().amax(dim=(0, 2)) if H else torch.zeros(nkv, dtype=torch.bfloat16, device=device)
+        if bool(written.any()):
+            kmax = torch.maximum(kmax, k_new[written].abs().amax(dim=(0, 2)))
+            vmax = torch.maximum(vmax, v_new[written].abs().amax(dim=(0, 2)))
+        # An all-zero head would give scale 0; any positive scale then encodes it exactly.
+        one = torch.ones_like(kmax)
+        kmax = torch.where(kmax > 0, kmax, one)
+        vmax = torch.where(vmax > 0, vmax, one)
+        wl.k_scale = kmax.float() / 448.0
+        wl.v_scale = vmax.float() / 448.0
+    elif cfg.cache_dtype != CACHE_BF16:
+        raise ValueError(cfg.cache_dtype)
+    return wl
+
+
+def subset_for_seqs(wl: Workload, seq_ids) -> dict:
+    """The rows one needs to rebuild the pool blocks of ``seq_ids`` only.
+
+    Returns host tensors: the history rows (and their slots) that live in
+    those sequences' blocks, plus the sequences' step inputs. Used to check a
+    sample of a full-size step on the CPU.
+    """
+    ids = torch.as_tensor(list(seq_ids), dtype=torch.int64)
+    rows = torch.unique(torch.cat([wl.hist_rows[int(i)] for i in ids]))
+    dev_rows = rows.to(wl.k_hist.device)
+    dev_ids = ids.to(wl.q.device)
+    return dict(
+        seq_ids=ids,
+        k_hist=wl.k_hist[dev_rows].cpu(),
+        v_hist=wl.v_hist[dev_rows].cpu(),
+        slot_hist=wl.slot_hist[dev_rows].cpu(),
+        q=wl.q[dev_ids].cpu(),
+        k_new=wl.k_new[dev_ids].cpu(),
+        v_new=wl.v_new[dev_ids].cpu(),
+        slot_new=wl.slot_new[dev_ids].cpu(),
+        block_tables=wl.block_tables[dev_ids].cpu(),
+        context_lens=wl.context_lens[dev_ids].cpu(),
+    )
+
+
+def logical_kv(wl: Workload, i: int):
+    """Sequence i's K and V rows ``[ctx, nkv, d]`` in logical token order.
+
+    Taken from the drawn rows themselves (not from any pool), so a check built
+    on it is independent of the pool layout, the block tables and the slots.
+    """
+    cfg = wl.cfg
+    P = cfg.prefix_tokens
+    ctx = int(wl.context_lens[i])
+    rows = wl.hist_rows[i].to(wl.k_hist.device)
+    k = wl.k_hist[rows]
+    v = wl.v_hist[rows]
+    if ctx > P:  # the step's own token is the last one
+        k = torch.cat([k, wl.k_new[i : i + 1]])
+        v = torch.cat([v, wl.v_new[i : i + 1]])
+    return k[:ctx], v[:ctx]

@@ -1,0 +1,368 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Each ``pin_*`` function takes a loaded oracle library and raises
+AssertionError when the oracle disagrees with:
+
+* brute-force attention over the sequence's tokens laid out contiguously,
+  taken straight from the drawn rows (no pool, no block table) and evaluated
+  with scipy's softmax and numpy einsum (a library special case);
+* the invariants the pages' block-table definition implies: any relabelling
+  of physical blocks, or a shared prefix copied into private blocks, changes
+  nothing ("DeepSeek复刻vLLM反超原版", section "vLLM：大模型推理的加速引擎与挑战":
+  logical blocks map to physical blocks through a block table, and KV blocks
+  can be shared within and across requests);
+* closed forms: one token returns its V row; identical keys return the mean
+  of V; a dominating key returns its own V row (pins token order and the
+  block / offset split at every block boundary);
+* the OCP E4M3 format points (tests/golden/e4m3_ocp_points.txt) and torch's
+  own float8_e4m3fn cast (a library routine) for the FP8 codec.
+
+The same functions run against deliberately broken copies of the oracle
+(tests/test_oracle_mutants.py) to show that each plausible mistake trips at
+least one of them.
+"""
+
+from __future__ import annotations
+
+import copy
+import os
+
+import numpy as np
+import scipy.special
+import torch
+
+import oracle as O
+from paged_kv_cache_482_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+TOL = 1e-12
+
+
+def cfg(**kw) -> W.DecodeConfig:
+    base = dict(name="pin", num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=16, block_size=4, ctx_lo=1,
+                ctx_hi=23)
+    base.update(kw)
+    return W.DecodeConfig(**base)
+
+
+def dequant(x_bf16: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
+    """bf16 rows [t, nkv, d] -> fp64 values of their E4M3 codes times scale (torch's cast)."""
+    y = x_bf16.float() / scale.float()[None, :, None]
+    codes = y.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return codes.double() * scale.double()[None, :, None]
+
+
+def brute_force(wl: W.Workload, i: int) -> np.ndarray:
+    """Contiguous softmax attention for sequence i from its logical K/V rows."""
+    c = wl.cfg
+    K, V = W.logical_kv(wl, i)
+    if wl.is_fp8:
+        K, V = dequant(K, wl.k_scale), dequant(V, wl.v_scale)
+    K = np.repeat(K.double().numpy(), c.group, axis=1)  # [ctx, nq, d]
+    V = np.repeat(V.double().numpy(), c.group, axis=1)
+    q = wl.q[i].double().numpy()  # [nq, d]
+    scale = np.float64(np.float32(c.softmax_scale))
+    s = np.einsum("hd,thd->ht", q, K) * scale
+    p = scipy.special.softmax(s, axis=1)
+    return np.einsum("ht,thd->hd", p, V)
+
+
+def _assert_close(a, b, tol=TOL, what=""):
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert np.all(np.isfinite(a)), f"{what}: non-finite oracle output"
+    assert err <= tol, f"{what}: max abs diff {err:.3e} > {tol:.1e}"
+
+
+def _run(wl, lib):
+    out, kp, vp, st = O.run_workload(wl, lib=lib)
+    assert st == O.ORC_OK, f"oracle status {st}"
+    return out, kp, vp
+
+
+# ----------------------------------------------------------------- attention
+
+
+def pin_bruteforce_bf16(lib):
+    for c, seed in [
+        (cfg(), 1),
+        (cfg(num_seqs=2, num_q_heads=8, num_kv_heads=1, head_dim=8, block_size=8, ctx_lo=1, ctx_hi=40), 2),
+        (cfg(num_seqs=2, num_q_heads=3, num_kv_heads=3, head_dim=12, block_size=16, ctx_lo=15, ctx_hi=33), 3),
+        (cfg(num_seqs=3, block_size=4, prefix_tokens=8, ctx_lo=0, ctx_hi=6), 4),
+    ]:
+        wl = W.generate(c, seed)
+        out, _, _ = _run(wl, lib)
+        for i in range(c.num_seqs):
+            _assert_close(out[i], brute_force(wl, i), what=f"bf16 seq {i} {c}")
+
+
+def pin_bruteforce_fp8(lib):
+    for c, seed in [
+        (cfg(cache_dtype=W.CACHE_FP8), 5),
+        (cfg(cache_dtype=W.CACHE_FP8, num_q_heads=8, num_kv_heads=2, head_dim=8, ctx_lo=30, ctx_hi=50), 6),
+    ]:
+        wl = W.generate(c, seed)
+        out, _, _ = _run(wl, lib)
+        for i in range(c.num_seqs):
+            _assert_close(out[i], brute_force(wl, i), what=f"fp8 seq {i}")
+
+
+def _relabel(wl: W.Workload, perm: torch.Tensor) -> W.Workload:
+    """The same step with physical block b renamed perm[b] everywhere."""
+    bs = wl.cfg.block_size
+    w2 = copy.copy(wl)
+    bt = wl.block_tables.long()
+    w2.block_tables = torch.where(bt >= 0, perm[bt.clamp(min=0)], bt).to(torch.int32)
+
+    def slots(s):
+        s = s.long()
+        return torch.where(s >= 0, perm[(s // bs).clamp(min=0)] * bs + s % bs, s).to(torch.int32)
+
+    w2.slot_hist = slots(wl.slot_hist)
+    w2.slot_new = slots(wl.slot_new)
+    return w2
+
+
+def pin_permutation_invariance(lib):
+    for c in (cfg(ctx_lo=5, ctx_hi=30), cfg(cache_dtype=W.CACHE_FP8), cfg(prefix_tokens=8, ctx_lo=0, ctx_hi=9)):
+        wl = W.generate(c, 7)
+        out, _, _ = _run(wl, lib)
+        g = torch.Generator().manual_seed(11)
+        for _ in range(2):
+            perm = torch.randperm(wl.num_blocks, generator=g)
+            out2, _, _ = _run(_relabel(wl, perm), lib)
+            assert np.array_equal(out, out2), "block relabelling changed the result"
+
+
+def pin_prefix_shared_equals_duplicated(lib):
+    c = cfg(num_seqs=4, prefix_tokens=8, ctx_lo=0, ctx_hi=7)
+    wl = W.generate(c, 8)
+    out, _, _ = _run(wl, lib)
+    bs, P = c.block_size, c.prefix_tokens
+    nshared = P // bs
+    S = c.num_seqs
+    w2 = copy.copy(wl)
+    w2.num_blocks = wl.num_blocks + S * nshared
+    bt = wl.block_tables.clone()
+    k_rows, v_rows, s_rows = [wl.k_hist], [wl.v_hist], [wl.slot_hist]
+    for i in range(S):
+        first = wl.num_blocks + i * nshared
+        bt[i, :nshared] = torch.arange(first, first + nshared, dtype=torch.int32)
+        k_rows.append(wl.k_hist[:P])
+        v_rows.append(wl.v_hist[:P])
+        s_rows.append(torch.arange(first * bs, first * bs + P, dtype=torch.int32))
+    w2.block_tables = bt
+    w2.k_hist = torch.cat(k_rows)
+    w2.v_hist = torch.cat(v_rows)
+    w2.slot_hist = torch.cat(s_rows)
+    out2, _, _ = _run(w2, lib)
+    assert np.array_equal(out, out2), "shared prefix differs from private copies"
+
+
+def pin_single_token_returns_v(lib):
+    for fp8 in (False, True):
+        c = cfg(num_q_heads=6, num_kv_heads=3, ctx_lo=1, ctx_hi=1,
+                cache_dtype=W.CACHE_FP8 if fp8 else W.CACHE_BF16)
+        wl = W.generate(c, 9)
+        out, _, _ = _run(wl, lib)
+        for i in range(c.num_seqs):
+            _, V = W.logical_kv(wl, i)
+            Vd = dequant(V, wl.v_scale) if fp8 else V.double()
+            expect = np.repeat(Vd[0].numpy(), c.group, axis=0)  # [nq, d]
+            assert np.array_equal(out[i], expect), "context of one token must return its V row exactly"
+
+
+def pin_identical_keys_mean_of_v(lib):
+    c = cfg(ctx_lo=3, ctx_hi=29)
+    wl = W.generate(c, 10)
+    wl.k_hist[:] = wl.k_hist[0:1].clone()
+    wl.k_new[:] = wl.k_hist[0:1]
+    out, _, _ = _run(wl, lib)
+    for i in range(c.num_seqs):
+        _, V = W.logical_kv(wl, i)
+        mean = np.repeat(V.double().numpy().mean(axis=0), c.group, axis=0)
+        _assert_close(out[i], mean, what="identical keys")
+
+
+def _logical_slot_row(wl, i, p):
+    """(tensor, row) holding logical token p of sequence i in the drawn rows."""
+    ctx = int(wl.context_lens[i])
+    if p == ctx - 1 and int(wl.slot_new[i]) >= 0:
+        return "new", i
+    return "hist", int(wl.hist_rows[i][p])
+
+
+def pin_dominant_key_returns_its_v(lib):
+    c = cfg(num_seqs=2, num_q_heads=2, num_kv_heads=1, head_dim=16, block_size=4, ctx_lo=13, ctx_hi=13)
+    for p in (0, 3, 4, 5, 8, 11, 12):
+        wl = W.generate(c, 12)
+        wl.q[:] = 1.0
+        wl.k_hist.zero_()
+        wl.k_new.zero_()
+        for i in range(c.num_seqs):
+            src, row = _logical_slot_row(wl, i, p)
+            (wl.k_new if src == "new" else wl.k_hist)[row] = 32.0  # score 128 against 0 elsewhere
+        out, _, _ = _run(wl, lib)
+        for i in range(c.num_seqs):
+            _, V = W.logical_kv(wl, i)
+            expect = np.repeat(V[p].double().numpy(), c.group, axis=0)
+            _assert_close(out[i], expect, what=f"dominant key at {p}")
+
+
+# --------------------------------------------------------------------- store
+
+
+def pin_store_layout(lib):
+    nblk, nkv, bs, d = 3, 2, 4, 4
+    g = torch.Generator().manual_seed(13)
+    k = torch.randn(6, nkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(6, nkv, d, generator=g).to(torch.bfloat16)
+    slots = torch.tensor([0, 5, -1, 11, 6, 2], dtype=torch.int32)
+    kp = O.new_pool(nblk, nkv, bs, d, False, W.CANARY_BF16)
+    vp = O.new_pool(nblk, nkv, bs, d, False, W.CANARY_BF16)
+    assert O.store_kvcache(k, v, kp, vp, slots, nblk, bs, lib=lib) == O.ORC_OK
+    ek = np.full((nblk, nkv, bs, d), W.CANARY_BF16, np.uint16)
+    ev = ek.copy()
+    kb = k.view(torch.int16).numpy().view(np.uint16)
+    vb = v.view(torch.int16).numpy().view(np.uint16)
+    for t, s in enumerate(slots.tolist()):
+        if s >= 0:
+            blk, off = divmod(s, bs)
+            ek[blk, :, off, :] = kb[t]
+            ev[blk, :, off, :] = vb[t]
+    assert np.array_equal(kp, ek) and np.array_equal(vp, ev), "bf16 store layout"
+    # A slot beyond the pool is refused and writes nothing.
+    kp2, vp2 = kp.copy(), vp.copy()
+    st = O.store_kvcache(k[:1], v[:1], kp2, vp2, torch.tensor([nblk * bs], dtype=torch.int32), nblk, bs, lib=lib)
+    assert st == O.ORC_ERR_BOUNDS and np.array_equal(kp2, kp) and np.array_equal(vp2, vp)
+    # FP8: the code in each slot is torch's E4M3 cast of x / scale (fp32 division).
+    ks = torch.tensor([0.01, 0.003], dtype=torch.float32)
+    vs = torch.tensor([0.02, 0.5], dtype=torch.float32)
+    kq = O.new_pool(nblk, nkv, bs, d, True, W.CANARY_FP8)
+    vq = O.new_pool(nblk, nkv, bs, d, True, W.CANARY_FP8)
+    assert O.store_kvcache(k, v, kq, vq, slots, nblk, bs, ks, vs, lib=lib) == O.ORC_OK
+    ck = (k.float() / ks[None, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    cv = (v.float() / vs[None, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ek = np.full((nblk, nkv, bs, d), W.CANARY_FP8, np.uint8)
+    ev = ek.copy()
+    for t, s in enumerate(slots.tolist()):
+        if s >= 0:
+            blk, off = divmod(s, bs)
+            ek[blk, :, off, :] = ck[t]
+            ev[blk, :, off, :] = cv[t]
+    assert np.array_equal(kq, ek) and np.array_equal(vq, ev), "fp8 store layout / codes"
+
+
+# ---------------------------------------------------------------- FP8 codec
+
+
+def read_golden_points():
+    pts = []
+    with open(os.path.join(GOLDEN, "e4m3_ocp_points.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                code, val = line.split()[:2]
+                pts.append((int(code, 16), float(val)))
+    return pts
+
+
+def pin_e4m3_decode_table(lib):
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib_vals = codes.view(torch.float8_e4m3fn).double().numpy()
+    for c in range(256):
+        got = O.e4m3_to_double(c, lib=lib)
+        want = lib_vals[c]
+        if np.isnan(want):
+            assert np.isnan(got), f"code {c:#x} must be NaN"
+        else:
+            assert got == want and np.signbit(got) == np.signbit(want), f"code {c:#x}: {got} != {want}"
+    for c, val in read_golden_points():
+        got = O.e4m3_to_double(c, lib=lib)
+        if np.isnan(val):
+            assert np.isnan(got)
+        else:
+            assert got == val and np.signbit(got) == np.signbit(val), f"OCP point {c:#x}"
+        if not np.isnan(val):
+            assert O.e4m3_from_float(val, lib=lib) == c, f"OCP point {c:#x} must encode back to itself"
+
+
+def _torch_encode(x: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(x.astype(np.float32)).clamp(-448.0, 448.0)
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_e4m3_encode(lib):
+    # a dense grid through the whole range, past saturation, both signs
+    grid = np.arange(-470 * 1024, 470 * 1024 + 1, dtype=np.float64) / 1024.0
+    # every exact midpoint between neighbouring codes (ties go to the even code)
+    vals = torch.arange(0, 0x7F, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    mids = (vals[:-1] + vals[1:]) / 2.0
+    # the subnormal range in fine steps, and a spread of magnitudes
+    fine = np.arange(0, 4097, dtype=np.float64) * 2.0**-18
+    spread = np.float32(np.exp(np.linspace(-30, 8, 3001)))
+    x = np.concatenate([grid, mids, -mids, fine, -fine, spread, -spread]).astype(np.float32)
+    want = _torch_encode(x)
+    got = np.fromiter((O.e4m3_from_float(float(v), lib=lib) for v in x), dtype=np.uint8, count=x.size)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"{bad.size} encodings differ, first x={x[bad[0]]!r}: {got[bad[0]]:#x} vs {want[bad[0]]:#x}"
+    # ties: the even neighbour, checked directly
+    for j, m in enumerate(mids):
+        assert O.e4m3_from_float(float(m), lib=lib) == (j if j % 2 == 0 else j + 1), f"tie at {m}"
+    assert O.e4m3_from_float(1e9, lib=lib) == 0x7E and O.e4m3_from_float(-1e9, lib=lib) == 0xFE
+    assert O.e4m3_from_float(float("nan"), lib=lib) & 0x7F == 0x7F
+
+
+def pin_bf16_widening(lib):
+    bits = np.arange(0, 65536, 97, dtype=np.uint16)
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    for b, w in zip(bits, want):
+        got = O.bf16_to_double(int(b), lib=lib)
+        assert (np.isnan(got) and np.isnan(w)) or got == w, f"bf16 {b:#x}"
+
+
+# ------------------------------------------------------------------ errors
+
+
+def pin_bounds_errors(lib):
+    c = cfg(ctx_lo=5, ctx_hi=20)
+    wl = W.generate(c, 14)
+    out, kp, vp = _run(wl, lib)
+    bt = wl.block_tables.clone()
+    bt[1, 0] = wl.num_blocks  # outside the pool
+    out2, st = O.paged_attention_decode(wl.q, kp, vp, bt, wl.context_lens, c.num_kv_heads, c.block_size,
+                                        c.softmax_scale, lib=lib)
+    assert st == O.ORC_ERR_BOUNDS
+    assert np.all(out2[1] == 0) and np.array_equal(out2[0], out[0]) and np.array_equal(out2[2], out[2])
+    for bad_len in (0, c.max_blocks_per_seq * c.block_size + 1):
+        cl = wl.context_lens.clone()
+        cl[2] = bad_len
+        out3, st = O.paged_attention_decode(wl.q, kp, vp, wl.block_tables, cl, c.num_kv_heads, c.block_size,
+                                            c.softmax_scale, lib=lib)
+        assert st == O.ORC_ERR_BOUNDS and np.all(out3[2] == 0) and np.array_equal(out3[0], out[0])
+
+
+ALL_PINS = [
+    pin_bruteforce_bf16,
+    pin_bruteforce_fp8,
+    pin_permutation_invariance,
+    pin_prefix_shared_equals_duplicated,
+    pin_single_token_returns_v,
+    pin_identical_keys_mean_of_v,
+    pin_dominant_key_returns_its_v,
+    pin_store_layout,
+    pin_e4m3_decode_table,
+    pin_e4m3_encode,
+    pin_bf16_widening,
+    pin_bounds_errors,
+]
+
+
+def run_all(lib) -> list[str]:
+    """Names of the pins that fail (or crash) against ``lib``."""
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except Exception as e:  # noqa: BLE001 - any failure counts
+            failed.append(f"{pin.__name__}: {type(e).__name__}: {str(e)[:120]}")
+    return failed

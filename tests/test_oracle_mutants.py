@@ -1,0 +1,95 @@
+"""Plant plausible mistakes in copies of the oracle; each must fail a pin.
+
+Every mutant below is a one-line change to ``oracle/pkv_oracle.c`` of the
+kind a reader could miss: a dropped term, a wrong index or sign, swapped
+operands, a transposed layout, a wrong rounding tie. The copy is compiled and
+the whole pin suite runs against it in a child process (so a crash counts as
+caught). If a mutant survived, the pins would not be pinning that line.
+"""
+
+import json
+import os
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+import oracle as O
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(os.path.dirname(HERE), "oracle", "pkv_oracle.c")
+
+# (name, original text, mutated text, which occurrence (0-based) to change)
+MUTANTS = [
+    ("gqa interleaved", "int g = h / group;", "int g = h % num_kv_heads;", 0),
+    ("offset from division", "int off = t % block_size;", "int off = (t / block_size) % block_size;", 0),
+    ("block from offset", "int64_t blk = table[t / block_size];", "int64_t blk = table[t % block_size];", 0),
+    ("pv offset", "int off = t % block_size;", "int off = (t + 1) % block_size;", 1),
+    ("scale dropped", "score[t] = (double)scale * dot;", "score[t] = dot;", 0),
+    ("max not subtracted", "w[t] = exp(score[t] - m);", "w[t] = exp(score[t]);", 0),
+    ("not normalised", "acc[i] / z;", "acc[i];", 0),
+    ("last token dropped", "for (t = 0; t < ctx; ++t) {\n                w[t]",
+     "for (t = 0; t < ctx - 1; ++t) {\n                w[t]", 0),
+    ("v read from k", "cache_value(v_cache, idx, fp8, v_scale, g)", "cache_value(k_cache, idx, fp8, v_scale, g)", 0),
+    ("q head of kv head", "q + ((int64_t)s * num_q_heads + h) * head_dim", "q + ((int64_t)s * num_q_heads + g) * head_dim", 0),
+    ("layout transposed", "((blk * nkv + h) * bs + off)", "((blk * bs + off) * nkv + h)", 0),
+    ("slot zero skipped", "if (slot < 0)", "if (slot <= 0)", 0),
+    ("k and v swapped", "((uint16_t *)k_cache)[dst] = k[src];", "((uint16_t *)k_cache)[dst] = v[src];", 0),
+    ("fp8 scale unused on read", "* (double)scale[h];", ";", 0),
+    ("fp8 scale multiplies on store", "float ky = kx / k_scale[h];", "float ky = kx * k_scale[h];", 0),
+    ("fp8 ties away", "(d_hi == d_lo && (lo & 1))", "(d_hi == d_lo)", 0),
+    ("fp8 saturation drops sign", "return sign | 0x7E;", "return 0x7E;", 0),
+    ("fp8 subnormal exponent", "ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)", 0),
+    ("fp8 bias", "e - 7);", "e - 8);", 0),
+    ("bf16 widening", "(uint32_t)bits << 16;", "(uint32_t)bits << 15;", 0),
+    ("bounds check off by one", "ctx > max_blocks_per_seq * block_size", "ctx > max_blocks_per_seq * block_size + 1", 0),
+    ("block id check", "table[t / block_size] >= num_blocks", "table[t / block_size] > num_blocks", 0),
+]
+
+
+def _mutate(src: str, old: str, new: str, which: int) -> str:
+    pos = -1
+    for _ in range(which + 1):
+        pos = src.find(old, pos + 1)
+        assert pos >= 0, f"mutation site not found: {old!r}"
+    return src[:pos] + new + src[pos + len(old):]
+
+
+def _run_mutant(args):
+    name, old, new, which, tmp = args
+    src = open(SRC).read()
+    path = os.path.join(tmp, name.replace(" ", "_") + ".c")
+    with open(path, "w") as f:
+        f.write(_mutate(src, old, new, which))
+    lib = path[:-2] + ".so"
+    O.build(path, lib, force=True)
+    r = subprocess.run([sys.executable, os.path.join(HERE, "_oracle_pin_runner.py"), lib],
+                       capture_output=True, text=True, timeout=600)
+    if r.returncode != 0:
+        return name, [f"crashed (rc={r.returncode})"]
+    return name, json.loads(r.stdout.strip().splitlines()[-1])
+
+
+def test_mutation_sites_exist():
+    src = open(SRC).read()
+    for name, old, _, which in MUTANTS:
+        assert src.count(old) > which, name
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    lib = str(tmp_path / "clean.so")
+    O.build(SRC, lib, force=True)
+    r = subprocess.run([sys.executable, os.path.join(HERE, "_oracle_pin_runner.py"), lib],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert json.loads(r.stdout.strip().splitlines()[-1]) == []
+
+
+def test_every_mutant_is_caught():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            results = list(ex.map(_run_mutant, [(*m, tmp) for m in MUTANTS]))
+    survivors = [name for name, failed in results if not failed]
+    assert not survivors, f"mutants not caught by any pin: {survivors}"
