@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark one paged decode step (store_kvcache + paged_attention_decode).
+
+A step is one pass of the whole hot path over one batch: write each
+sequence's new K/V row into its slot, then attend every query head over its
+paged context (plus the split-K reduce when the plan splits). Inputs are
+seeded synthetic tensors of the Qwen3-8B-shaped decode layer by default
+(1024 sequences, lengths uniform in [100, 2048], 32 query / 8 KV heads,
+head_dim 128, block_size 256, bf16 cache), resident in HBM before timing.
+The KV pools (4.6 GB read per step) are far larger than L2, so no flush is
+needed between steps.
+
+Prints one JSON line (rank 0). ``--impl reference`` times the fp64 CPU
+oracle instead, on bounded samples of the same workload.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (weak
+scaling, no collective on the data path); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_482_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention tokens/sec and achieved HBM GB/s (% of B200 peak)"
+UNIT = "tokens/s"
+NOMINAL_HBM_GBS = 8000.0  # the "~8 TB/s" the target percentage refers to
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["paged_kv_cache_482_b200/csrc/decode.cuh", "paged_kv_cache_482_b200/csrc/decode.cu",
+                  "paged_kv_cache_482_b200/csrc/pkv_common.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="qwen3_8b", choices=sorted(W.CONFIGS))
+    ap.add_argument("--partition", type=int, default=0, help="0 auto, -1 never split, >0 tokens per partition")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU work of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+
+def workload_desc(cfg: W.DecodeConfig) -> str:
+    if cfg.prefix_tokens:
+        ctx = f"{cfg.prefix_tokens} shared + U[{cfg.ctx_lo},{cfg.ctx_hi}]"
+    else:
+        ctx = f"U[{cfg.ctx_lo},{cfg.ctx_hi}]"
+    return (f"{cfg.name} paged decode layer: {cfg.num_seqs} seqs, ctx {ctx}, {cfg.num_q_heads}q/{cfg.num_kv_heads}kv "
+            f"heads, head_dim {cfg.head_dim}, block_size {cfg.block_size}, {cfg.cache_dtype} cache")
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg_name: str, partition_tokens: int):
+    """dram read+write bytes per decode launch from a committed ncu capture, if
+    it was taken on the current kernel source and the same workload."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except Exception:  # noqa: BLE001
+        return None
+    if rec.get("kernel_hash") != kernel_hash() or rec.get("workload") != cfg_name:
+        return None
+    if rec.get("partition_tokens") != partition_tokens:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def algorithmic_bytes(wl: W.Workload) -> dict:
+    """Bytes one decode launch must move at minimum."""
+    c = wl.cfg
+    esize = 1 if wl.is_fp8 else 2
+    ctx = wl.context_lens.long().cpu()
+    kv = int(ctx.sum()) * c.num_kv_heads * c.head_dim * esize * 2
+    qo = 2 * c.num_seqs * c.num_q_heads * c.head_dim * 2
+    nb = int(((ctx + c.block_size - 1) // c.block_size).sum())
+    meta = 4 * nb + 4 * c.num_seqs
+    if c.prefix_tokens:
+        # shared prefix blocks are read once from HBM (they stay in L2)
+        shared_tok = c.prefix_tokens
+        own = int((ctx - c.prefix_tokens).sum())
+        unique_kv = (shared_tok + own) * c.num_kv_heads * c.head_dim * esize * 2
+    else:
+        unique_kv = kv
+    return dict(kv=kv, unique_kv=unique_kv, q_out=qo, meta=meta, total=kv + qo + meta,
+                unique_total=unique_kv + qo + meta)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_ids):
+        self.samples = []
+        self.proc = None
+        self.window = None
+        try:
+            cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits", "-lms",
+                   "200"]
+            if device_ids:
+                cmd += ["-i", ",".join(str(d) for d in device_ids)]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:  # noqa: BLE001
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.samples.append((time.time(), parts))
+
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc is not None and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:  # noqa: BLE001
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        inwin = [p for t, p in self.samples if t0 <= t <= t1 + 0.25]
+        used = inwin or [p for _, p in self.samples[-3:]]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        sm, smax, pw = [], [], []
+        for p in used:
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+                pw.append(float(p[3]))
+            except ValueError:
+                pass
+            for n, v in zip(names, p[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons), "samples": len(inwin),
+                "samples_note": "in the timed window" if inwin else "nearest samples (window shorter than 200 ms)"}
+
+
+def nvsmi_ids(local_rank: int):
+    try:
+        props = torch.cuda.get_device_properties(local_rank)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            s = str(uuid)
+            return ["GPU-" + s if not s.startswith("GPU-") else s]
+    except Exception:  # noqa: BLE001
+        pass
+    return [local_rank]
+
+
+# --------------------------------------------------------------- CPU oracle
+
+
+def _compact(sub: dict, bs: int):
+    """Renumber the blocks a sample uses to 0..n-1 (relabelling physical blocks
+    leaves attention unchanged), so the host pools hold only those blocks."""
+    bt = sub["block_tables"].long()
+    used = torch.unique(bt[bt >= 0])
+    remap = torch.full((int(used.max()) + 1,), -1, dtype=torch.long)
+    remap[used] = torch.arange(used.numel())
+    out = dict(sub)
+    out["block_tables"] = torch.where(bt >= 0, remap[bt.clamp(min=0)], bt).to(torch.int32)
+
+    def slots(s):
+        s = s.long()
+        return torch.where(s >= 0, remap[(s // bs).clamp(min=0)] * bs + s % bs, s).to(torch.int32)
+
+    out["slot_hist"] = slots(sub["slot_hist"])
+    out["slot_new"] = slots(sub["slot_new"])
+    return out, int(used.numel())
+
+
+def oracle_sample_runner(wl: W.Workload, ids, threads: int):
+    """Prepare host pools for a sample (untimed); return a function that runs
+    the sample's step (store the new tokens, attend) on the CPU oracle."""
+    import oracle as O
+
+    c = wl.cfg
+    sub, nblk = _compact(W.subset_for_seqs(wl, ids), c.block_size)
+    fill = W.CANARY_FP8 if wl.is_fp8 else W.CANARY_BF16
+    kp = O.new_pool(nblk, c.num_kv_heads, c.block_size, c.head_dim, wl.is_fp8, fill)
+    vp = O.new_pool(nblk, c.num_kv_heads, c.block_size, c.head_dim, wl.is_fp8, fill)
+    ks = wl.k_scale.cpu() if wl.k_scale is not None else None
+    vs = wl.v_scale.cpu() if wl.v_scale is not None else None
+    O.store_kvcache(sub["k_hist"], sub["v_hist"], kp, vp, sub["slot_hist"], nblk, c.block_size, ks, vs)
+
+    def step():
+        O.store_kvcache(sub["k_new"], sub["v_new"], kp, vp, sub["slot_new"], nblk, c.block_size, ks, vs)
+        out, st = O.paged_attention_decode(sub["q"], kp, vp, sub["block_tables"], sub["context_lens"],
+                                           c.num_kv_heads, c.block_size, c.softmax_scale, ks, vs,
+                                           num_threads=threads)
+        return st
+
+    return step
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl: W.Workload, target_s: float) -> dict:
+    """Tokens/s of the oracle on a bounded sample, sized to about target_s."""
+    threads = cpu_threads()
+    S = wl.cfg.num_seqs
+    order = torch.randperm(S, generator=torch.Generator().manual_seed(123)).tolist()
+    n = min(S, max(threads, 4))
+    probe = oracle_sample_runner(wl, order[:n], threads)
+    t0 = time.perf_counter()
+    probe()
+    dt = time.perf_counter() - t0
+    n2 = int(min(S, max(n, n * target_s / max(dt, 1e-6))))
+    run = oracle_sample_runner(wl, order[:n2], threads)
+    t0 = time.perf_counter()
+    st = run()
+    dt = time.perf_counter() - t0
+    toks = int(wl.context_lens.cpu()[order[:n2]].sum())
+    return {"value": n2 / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n2} of {S} sequences ({toks} context tokens) of the same step, fp64, {dt:.2f} s, "
+                      f"OpenMP over sequences; status {st}"}
+
+
+# --------------------------------------------------------------- reference
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = W.CONFIGS[args.config]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = W.generate(cfg, args.seed, device=dev)
+    threads = cpu_threads()
+    S = cfg.num_seqs
+    # size each step's sample so that warm-up + timed steps take about two minutes
+    order = torch.randperm(S, generator=torch.Generator().manual_seed(7)).tolist()
+    probe = oracle_sample_runner(wl, order[: max(4, threads)], threads)
+    t0 = time.perf_counter()
+    probe()
+    per_seq = (time.perf_counter() - t0) / max(4, threads)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(min(S, max(1, budget / max(per_seq, 1e-9))))
+    runs = [oracle_sample_runner(wl, order[(i * n) % S:(i * n) % S + n] or order[:n], threads)
+            for i in range(min(4, args.steps + args.warmup))]
+    for i in range(args.warmup):
+        runs[i % len(runs)]()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        runs[i % len(runs)]()
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "sample_seqs_per_step": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} of {S} sequences per step, fp64 oracle, OpenMP over sequences"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- ours
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    from paged_kv_cache_482_b200 import pagedkv as K
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    cfg = W.CONFIGS[args.config]
+    wl = W.generate(cfg, args.seed + rank, device="cuda")
+    c = cfg
+    shape = (wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)
+    if wl.is_fp8:
+        kp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device="cuda")
+        vp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device="cuda")
+    else:
+        kp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+        vp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    H = wl.k_hist.shape[0]
+    for i in range(0, H, 1 << 20):
+        j = min(H, i + (1 << 20))
+        K.store_kvcache(wl.k_hist[i:j], wl.v_hist[i:j], kp, vp, wl.slot_hist[i:j], wl.k_scale, wl.v_scale)
+    step = K.DecodeStep(kp, vp, c.num_seqs, c.num_q_heads, wl.block_tables.shape[1], c.softmax_scale,
+                        wl.k_scale, wl.v_scale, max_context_len=c.max_context, partition_request=args.partition)
+    inputs = (wl.q, wl.k_new, wl.v_new, wl.slot_new, wl.block_tables, wl.context_lens)
+    launches_per_step = 2 + (1 if step.plan["partition_tokens"] > 0 else 0)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        step.run(*inputs)
+    torch.cuda.synchronize()
+    if int(step.dev_err.item()) != 0:
+        raise RuntimeError(f"device error word {int(step.dev_err.item())} during warm-up")
+
+    sampler = ClockSampler(nvsmi_ids(local)) if local == 0 else None
+    if sampler:
+        sampler.wait_first()
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kst)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    e_start.record(stream)
+    for k in range(Kst):
+        ev[k][0].record(stream)
+        K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, step.dev_err)
+        ev[k][1].record(stream)
+        K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, out=step.out,
+                                 k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context,
+                                 partition_request=args.partition, workspace=step.workspace, dev_err=step.dev_err)
+        ev[k][2].record(stream)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    elapsed_ms = e_start.elapsed_time(e_end)
+    decode_ms = statistics.mean(ev[k][1].elapsed_time(ev[k][2]) for k in range(Kst))
+    store_ms = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(Kst))
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
+    if sampler:
+        sampler.stop()
+    if int(step.dev_err.item()) != 0:
+        raise RuntimeError(f"device error word {int(step.dev_err.item())} in the timed steps")
+
+    # end to end: pinned host inputs -> device -> step -> host output, every step
+    host_in = [t.cpu().pin_memory() for t in inputs]
+    host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    for _ in range(3):
+        step.run_host(*host_in, host_out)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        step.run_host(*host_in, host_out)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = x0.elapsed_time(x1)
+
+    t = torch.tensor([elapsed_ms, decode_ms, e2e_ms], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, decode_ms, e2e_ms = (float(x) for x in t.tolist())
+
+    if rank == 0:
+        ab = algorithmic_bytes(wl)
+        peak, peak_kind = measured_peak()
+        bytes_launch = ab["unique_total"] if c.prefix_tokens else ab["total"]
+        achieved = bytes_launch / (decode_ms * 1e-3) / 1e9
+        pt = step.plan["partition_tokens"]
+        traffic = recorded_traffic(c.name, pt)
+        value = world * c.num_seqs * Kst / (elapsed_ms * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": Kst, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / Kst, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if wl.is_fp8 else "bf16", "data": "synthetic",
+            "config": {
+                "workload": workload_desc(c), "num_seqs": c.num_seqs, "seq_len": "ctx " + (
+                    f"{c.prefix_tokens}+U[{c.ctx_lo},{c.ctx_hi}]" if c.prefix_tokens else f"U[{c.ctx_lo},{c.ctx_hi}]"),
+                "kv_tokens": wl.kv_tokens(), "seed": args.seed, "partition_tokens": pt,
+                "parallelism": f"replicas x{world} (independent batches, no collective)",
+                "l2": f"no flush: {ab['kv'] / 1e9:.2f} GB of KV read per step, far above the 126 MB L2",
+            },
+            "attention_us": decode_ms * 1e3,
+            "store_us": store_ms * 1e3,
+            "hbm_gbs": achieved,
+            "hbm_pct_of_8tbs": 100.0 * achieved / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "paged_decode_kernel" + (" + paged_decode_reduce_kernel" if pt > 0 else ""),
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                         "algorithmic_bytes_per_launch": bytes_launch,
+                         "bytes_note": ("unique bytes: shared prefix counted once" if c.prefix_tokens else
+                                        "KV rows of every context token + q + out + block-table entries")},
+            "e2e": {"value": world * c.num_seqs * args.e2e_steps / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+            "gpu_launches": launches_per_step * Kst,
+            "clocks": clocks,
+        }
+        if c.prefix_tokens:
+            line["logical_gbs"] = ab["total"] / (decode_ms * 1e-3) / 1e9
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

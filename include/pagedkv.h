@@ -1,0 +1,180 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: one decode step of attention over a
+ * paged KV cache, on B200 (sm_100a).
+ *
+ * The operation. The KV cache is cut into fixed-size blocks that live
+ * anywhere in a physical pool; a per-sequence block table maps the logical
+ * block j of a sequence to a physical block, and several sequences may map
+ * to the same physical blocks (a shared prefix). Pages: "DeepSeek复刻vLLM反超
+ * 原版：AI推理新标杆", section "vLLM：大模型推理的加速引擎与挑战" (block table
+ * from logical to physical blocks, KV sharing within and across requests);
+ * "nano-vllm：轻量级大模型推理引擎的技术探索与实践", section "PagedAttention 原理
+ * 回顾" (fixed-size blocks, non-contiguous allocation); "Nano-vLLM：轻量高效的
+ * 大模型推理框架", section 三.1 (the block manager hands each request its
+ * blocks). The decode attends one new query token per sequence over its
+ * cached tokens in logical order, out = softmax(scale * q K^T) V, which the
+ * pages describe as bound by KV-cache read bandwidth ("nano-vllm-lite：深入
+ * 理解LLM推理机制的教育级开源项目", section 核心技术改进 2); the optional FP8
+ * cache is from the same page, section 核心技术改进 3 "FP8 KV Cache量化".
+ *
+ * Conventions (readings where the pages are silent):
+ *  - Pool layout: k_cache and v_cache are [num_blocks][num_kv_heads]
+ *    [block_size][head_dim], row-major, element type bf16 or E4M3 (1 byte).
+ *    Slot s is block s / block_size, offset s % block_size.
+ *  - Grouped-query attention: query head h reads KV head
+ *    h / (num_q_heads / num_kv_heads).
+ *  - context_lens[i] counts the step's own token, which store_kvcache
+ *    writes before the decode on the same stream.
+ *  - FP8: code = E4M3(x / scale[h]) with one IEEE fp32 division, round to
+ *    nearest even, saturating at +-448; value = code * scale[h].
+ *
+ * Ownership and execution. The caller owns every buffer (device memory unless
+ * stated) and keeps it alive until the stream work finishes. The library
+ * allocates nothing and keeps no state between calls; calls are re-entrant.
+ * Every call is asynchronous on the given stream (a cudaStream_t passed as
+ * void*; NULL is the legacy default stream) and returns once the work is
+ * queued.
+ *
+ * Errors. Arguments the host can check are checked before anything is
+ * launched; a failed check returns the status and launches nothing. Faults
+ * only the device can see (a slot, block id or length outside the pool or
+ * the table) set bits in *dev_err (device memory, one int, OR-ed atomically;
+ * the caller zeroes it) and the affected rows are skipped or written as
+ * zeros; the kernels never trap. A bounded wait inside a kernel that gives
+ * up sets PKV_DEVERR_TIMEOUT. dev_err may be NULL, in which case those
+ * faults are still skipped but not reported.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size */
+    PKV_ERR_UNSUPPORTED = 2,   /* shape the kernels are not built for */
+    PKV_ERR_WORKSPACE = 3,     /* workspace missing or too small */
+    PKV_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+    PKV_ERR_DEVICE_BOUNDS = 5, /* pkv_read_device_error: bounds bit set */
+    PKV_ERR_DEVICE_TIMEOUT = 6 /* pkv_read_device_error: timeout bit set */
+} pkv_status;
+
+typedef enum {
+    PKV_CACHE_BF16 = 0,
+    PKV_CACHE_FP8_E4M3 = 1
+} pkv_cache_dtype;
+
+/* Bits of the device error word. */
+#define PKV_DEVERR_BOUNDS 0x1
+#define PKV_DEVERR_TIMEOUT 0x2
+
+/*
+ * store_kvcache: for each token t < num_tokens with slot_mapping[t] >= 0,
+ * write k[t] and v[t] (all KV heads) into that slot of k_cache / v_cache.
+ * slot_mapping[t] == -1 skips token t (e.g. a token already held by a shared
+ * prefix block).
+ *
+ *  k, v          [num_tokens][num_kv_heads][head_dim] bf16, contiguous
+ *  k_cache, ...  pools as above; bf16 (copy) or E4M3 (quantised)
+ *  slot_mapping  [num_tokens] int32
+ *  k_scale, ...  [num_kv_heads] fp32, FP8 only (NULL for bf16)
+ *
+ * Host checks: non-null pointers, 16-byte aligned k/v/caches, head_dim a
+ * multiple of 8, sizes >= 1 (num_tokens may be 0: nothing is launched).
+ * Device check: slot >= num_blocks * block_size sets PKV_DEVERR_BOUNDS and
+ * the token is not written.
+ */
+PKV_API int pkv_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache,
+                      const int32_t *slot_mapping, int num_tokens, int num_kv_heads,
+                      int head_dim, int block_size, int64_t num_blocks, int cache_dtype,
+                      const float *k_scale, const float *v_scale, int *dev_err, void *stream);
+
+/*
+ * Split-K plan of a decode call. A sequence's tokens are cut into partitions
+ * of partition_tokens logical tokens; each partition is one thread block per
+ * KV head, and a reduce kernel merges the partials (flash-decoding). When
+ * partition_tokens == 0 the whole context is one partition, no workspace is
+ * used and no reduce kernel runs.
+ */
+typedef struct {
+    int partition_tokens;   /* 0: no split */
+    int max_partitions;     /* partitions of the longest allowed context */
+    size_t workspace_bytes; /* device scratch the decode needs (0: none) */
+} pkv_decode_plan;
+
+/*
+ * pkv_plan_decode: the plan pkv_paged_attention_decode will use for these
+ * sizes. partition_request: 0 = choose automatically, -1 = never split,
+ * > 0 = split into partitions of that many tokens (rounded up to the tile
+ * size of the kernel). Returns PKV_ERR_UNSUPPORTED for shapes without a
+ * kernel (head_dim not 64 or 128; group size not 1, 2, 4 or 8).
+ */
+PKV_API int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int block_size, int max_context_len, int cache_dtype,
+                    int partition_request, pkv_decode_plan *plan);
+
+/*
+ * paged_attention_decode: for each sequence i < num_seqs and query head h,
+ *   out[i][h][:] = sum_t softmax_t(scale * q[i][h] . K_t) V_t
+ * over the context_lens[i] tokens t of sequence i, where the K/V row of
+ * logical token t is slot block_tables[i][t / block_size] * block_size +
+ * t % block_size of the pools (KV head h / group). Scores, softmax and the
+ * weighted sum accumulate in fp32; out is rounded to bf16.
+ *
+ *  q                  [num_seqs][num_q_heads][head_dim] bf16, contiguous
+ *  block_tables       [num_seqs][max_blocks_per_seq] int32
+ *  context_lens       [num_seqs] int32, each in [1, min(max_context_len,
+ *                     max_blocks_per_seq * block_size)]
+ *  max_context_len    host-known bound on context_lens (sizes split-K)
+ *  partition_request  as in pkv_plan_decode
+ *  workspace          device scratch of at least plan.workspace_bytes,
+ *                     256-byte aligned (may be NULL when that is 0);
+ *                     contents need not be initialised and are clobbered
+ *  out                [num_seqs][num_q_heads][head_dim] bf16
+ *
+ * Host checks: pointers non-null and 16-byte aligned (q, caches, out,
+ * workspace), block_size a power of two in [8, 1024], head_dim and group
+ * supported, max_context_len >= 1 and <= max_blocks_per_seq * block_size,
+ * workspace large enough (PKV_ERR_WORKSPACE otherwise). Device checks: a
+ * length outside [1, max_context_len] or a block id outside
+ * [0, num_blocks) sets PKV_DEVERR_BOUNDS and that sequence's KV-head rows of
+ * out are written as zeros.
+ */
+PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_tables, int max_blocks_per_seq,
+                               const int32_t *context_lens, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int64_t num_blocks, float scale, int cache_dtype,
+                               const float *k_scale, const float *v_scale,
+                               int max_context_len, int partition_request, void *workspace,
+                               size_t workspace_bytes, void *out, int *dev_err, void *stream);
+
+/* Human-readable name of a pkv_status value (static storage). */
+PKV_API const char *pkv_status_string(int status);
+
+/*
+ * pkv_read_device_error: synchronise the stream, read *dev_err and map it to
+ * a status (PKV_OK, PKV_ERR_DEVICE_BOUNDS, PKV_ERR_DEVICE_TIMEOUT; the
+ * timeout bit wins). Does not clear the word.
+ */
+PKV_API int pkv_read_device_error(const int *dev_err, void *stream);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+PKV_API int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

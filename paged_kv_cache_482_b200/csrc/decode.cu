@@ -1,0 +1,108 @@
+// decode.cu -- instantiations and launch of the paged decode kernels.
+//
+// Tile shape per cache type: a stage holds TILE tokens of K and of V, 16 KB
+// in total, four stages deep, four consumer warps. That keeps 48 KB or more
+// of loads in flight per block and lets two to three blocks share an SM.
+#include <atomic>
+
+#include "decode.cuh"
+
+namespace pkv {
+
+namespace {
+
+template <int D, bool FP8>
+struct TileOf {
+    static constexpr int kRowBytes = D * (FP8 ? 1 : 2);
+    static constexpr int kTile = 16384 / (2 * kRowBytes);  // 32 (bf16 d128) .. 128 (e4m3 d64)
+};
+
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = 4;
+
+template <int D, int G, bool FP8>
+cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
+    constexpr int TILE = TileOf<D, FP8>::kTile;
+    constexpr int MINB = (G <= 4) ? 3 : 2;
+    using T = DecodeTraits<D, G, FP8, TILE, kStages, kConsumerWarps>;
+    auto kern = paged_decode_kernel<D, G, FP8, TILE, kStages, kConsumerWarps, MINB>;
+
+    // The opt-in to more than 48 KB of dynamic shared memory is a property of
+    // the function on a device; set it once per device.
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    const long long blocks = (long long)p.num_seqs * p.num_kv_heads * p.num_partitions;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)blocks, T::kThreads, T::kSmemBytes, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.num_partitions <= 1) return e;
+    paged_decode_reduce_kernel<D><<<(unsigned)((long long)p.num_seqs * p.num_q_heads), D, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <int D, bool FP8>
+cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) {
+    switch (group) {
+        case 1: return launch_one<D, 1, FP8>(p, stream);
+        case 2: return launch_one<D, 2, FP8>(p, stream);
+        case 4: return launch_one<D, 4, FP8>(p, stream);
+        case 8: return launch_one<D, 8, FP8>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+int decode_tile_tokens(int head_dim, int group, bool fp8) {
+    if (group != 1 && group != 2 && group != 4 && group != 8) return 0;
+    if (head_dim == 128) return fp8 ? TileOf<128, true>::kTile : TileOf<128, false>::kTile;
+    if (head_dim == 64) return fp8 ? TileOf<64, true>::kTile : TileOf<64, false>::kTile;
+    return 0;
+}
+
+int decode_max_blocks_per_partition() { return kMaxIdsPerPartition; }
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
+    DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16 *>(a.q);
+    p.k_cache = static_cast<const uint8_t *>(a.k_cache);
+    p.v_cache = static_cast<const uint8_t *>(a.v_cache);
+    p.block_tables = a.block_tables;
+    p.max_blocks_per_seq = a.max_blocks_per_seq;
+    p.context_lens = a.context_lens;
+    p.num_seqs = a.num_seqs;
+    p.num_q_heads = a.num_q_heads;
+    p.num_kv_heads = a.num_kv_heads;
+    p.block_size = a.block_size;
+    int lg = 0;
+    while ((1 << lg) < a.block_size) ++lg;
+    p.log2_block_size = lg;
+    p.num_blocks = a.num_blocks;
+    p.qk_scale_log2 = a.scale * 1.4426950408889634f;  // log2(e)
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    p.max_context_len = a.max_context_len;
+    p.partition_tokens = a.partition_tokens > 0 ? a.partition_tokens : a.max_context_len;
+    p.num_partitions = a.partition_tokens > 0 ? a.num_partitions : 1;
+    p.part_o = a.part_o;
+    p.part_ml = a.part_ml;
+    p.out = static_cast<__nv_bfloat16 *>(a.out);
+    p.dev_err = a.dev_err;
+    const int group = a.num_q_heads / a.num_kv_heads;
+    if (a.head_dim == 128)
+        return a.fp8 ? launch_group<128, true>(group, p, stream) : launch_group<128, false>(group, p, stream);
+    if (a.head_dim == 64)
+        return a.fp8 ? launch_group<64, true>(group, p, stream) : launch_group<64, false>(group, p, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pkv

@@ -1,0 +1,50 @@
+// pkv_launch.h -- internal launchers behind the C ABI (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pkv {
+
+cudaError_t launch_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache,
+                                 const int32_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                 int block_size, int64_t num_blocks, bool fp8, const float *k_scale,
+                                 const float *v_scale, int *dev_err, int num_sms, cudaStream_t stream);
+
+// Everything the decode kernels need, resolved by the host layer.
+struct DecodeArgs {
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_tables;
+    int max_blocks_per_seq;
+    const int32_t *context_lens;
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int head_dim;
+    int block_size;
+    int64_t num_blocks;
+    float scale;
+    bool fp8;
+    const float *k_scale;
+    const float *v_scale;
+    int max_context_len;
+    int partition_tokens;  // 0: one partition per sequence
+    int num_partitions;    // grid partitions per (sequence, KV head)
+    float *part_o;         // [num_seqs][num_q_heads][num_partitions][head_dim]
+    float *part_ml;        // [num_seqs][num_q_heads][num_partitions][2]
+    void *out;
+    int *dev_err;
+};
+
+// Tile (tokens per pipeline stage) of the decode kernel chosen for a shape;
+// split-K partitions are whole multiples of it. 0 when unsupported.
+int decode_tile_tokens(int head_dim, int group, bool fp8);
+// Largest number of physical blocks one partition may span.
+int decode_max_blocks_per_partition();
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+}  // namespace pkv

@@ -1,0 +1,239 @@
+"""Python binding of libpagedkv.so (ctypes).
+
+Argument marshalling only: tensors become device pointers, shapes become
+sizes, the current torch CUDA stream becomes the ``stream`` argument. Every
+step of the computation runs in the library's CUDA kernels. There is no CPU
+path: if ``libpagedkv.so`` is missing or cannot load, ``lib()`` raises.
+
+The functions mirror ``include/pagedkv.h``:
+
+* ``store_kvcache`` -- ``pkv_store_kvcache``
+* ``plan_decode`` -- ``pkv_plan_decode``
+* ``paged_attention_decode`` -- ``pkv_paged_attention_decode``
+* ``read_device_error`` -- ``pkv_read_device_error``
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
+
+PKV_OK = 0
+PKV_ERR_INVALID_ARG = 1
+PKV_ERR_UNSUPPORTED = 2
+PKV_ERR_WORKSPACE = 3
+PKV_ERR_CUDA = 4
+PKV_ERR_DEVICE_BOUNDS = 5
+PKV_ERR_DEVICE_TIMEOUT = 6
+
+PKV_CACHE_BF16 = 0
+PKV_CACHE_FP8_E4M3 = 1
+
+EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_paged_attention_decode", "pkv_status_string",
+            "pkv_read_device_error", "pkv_version")
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("partition_tokens", ctypes.c_int), ("max_partitions", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib(path: str = LIB_PATH):
+    """The loaded library; raises if it is not built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m paged_kv_cache_482_b200.build` "
+                               "(there is no CPU fallback)")
+        L = ctypes.CDLL(path)
+        c = ctypes
+        vp, i32, i64, f32, sz = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
+        L.pkv_store_kvcache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp, vp, vp]
+        L.pkv_store_kvcache.restype = i32
+        L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
+        L.pkv_plan_decode.restype = i32
+        L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i64, f32, i32, vp,
+                                                 vp, i32, i32, vp, sz, vp, vp, vp]
+        L.pkv_paged_attention_decode.restype = i32
+        L.pkv_status_string.argtypes = [i32]
+        L.pkv_status_string.restype = c.c_char_p
+        L.pkv_read_device_error.argtypes = [vp, vp]
+        L.pkv_read_device_error.restype = i32
+        L.pkv_version.argtypes = []
+        L.pkv_version.restype = i32
+        _lib = L
+        return L
+
+
+def status_string(status: int) -> str:
+    return lib().pkv_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _cache_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PKV_CACHE_BF16
+    if t.dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
+        return PKV_CACHE_FP8_E4M3
+    raise TypeError(f"KV pool dtype {t.dtype}: expected bfloat16 or an 8-bit E4M3 container")
+
+
+def _check(status: int, where: str):
+    if status != PKV_OK:
+        raise PagedKVError(status, where)
+
+
+def store_kvcache(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None, dev_err=None, stream=None):
+    """Write k/v ``[N, nkv, d]`` bf16 rows into pool slots ``slot_mapping`` (-1 skips)."""
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("k and v must be bfloat16")
+    if not (k.is_contiguous() and v.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous()):
+        raise ValueError("k, v and the pools must be contiguous")
+    if slot_mapping.dtype != torch.int32:
+        raise TypeError("slot_mapping must be int32")
+    N, nkv, d = k.shape
+    nblk, nkv2, bs, d2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or nkv2 != nkv or d2 != d or slot_mapping.numel() != N:
+        raise ValueError("shape mismatch between k/v, pools and slot_mapping")
+    st = lib().pkv_store_kvcache(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), N, nkv, d, bs,
+                                 nblk, _cache_dtype(k_cache), _ptr(k_scale), _ptr(v_scale), _ptr(dev_err),
+                                 _stream(stream))
+    _check(st, "pkv_store_kvcache")
+
+
+def plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, fp8=False,
+                partition_request=0) -> dict:
+    plan = _Plan()
+    st = lib().pkv_plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                               PKV_CACHE_FP8_E4M3 if fp8 else PKV_CACHE_BF16, partition_request,
+                               ctypes.byref(plan))
+    _check(st, "pkv_plan_decode")
+    return dict(partition_tokens=plan.partition_tokens, max_partitions=plan.max_partitions,
+                workspace_bytes=plan.workspace_bytes)
+
+
+def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out=None, k_scale=None,
+                           v_scale=None, max_context_len=None, partition_request=0, workspace=None, dev_err=None,
+                           stream=None):
+    """One decode step of paged attention; returns ``out`` ``[S, nq, d]`` bf16.
+
+    ``max_context_len`` defaults to the block-table capacity (no device
+    sync). A workspace is allocated with torch when the plan needs one and
+    none is given.
+    """
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise TypeError("q must be contiguous bfloat16")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if not block_tables.is_contiguous():
+        raise ValueError("block_tables must be contiguous")
+    S, nq, d = q.shape
+    nblk, nkv, bs, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("shape mismatch")
+    maxb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = maxb * bs
+    fp8 = _cache_dtype(k_cache) == PKV_CACHE_FP8_E4M3
+    if out is None:
+        out = torch.empty_like(q)
+    plan = plan_decode(S, nq, nkv, d, bs, max_context_len, fp8, partition_request)
+    if plan["workspace_bytes"] and workspace is None:
+        workspace = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().pkv_paged_attention_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), maxb,
+                                          _ptr(context_lens), S, nq, nkv, d, bs, nblk, float(scale),
+                                          PKV_CACHE_FP8_E4M3 if fp8 else PKV_CACHE_BF16, _ptr(k_scale),
+                                          _ptr(v_scale), int(max_context_len), int(partition_request),
+                                          _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_err), _stream(stream))
+    _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def read_device_error(dev_err, stream=None) -> int:
+    """Synchronise the stream and map the device error word to a status."""
+    return lib().pkv_read_device_error(_ptr(dev_err), _stream(stream))
+
+
+def version() -> int:
+    return lib().pkv_version()
+
+
+class DecodeStep:
+    """A decode step bound to resident pools: store the step's K/V, then attend.
+
+    Holds the plan and workspace for a fixed shape, so repeated steps launch
+    only the library's kernels. ``run_host`` takes the step's inputs from host
+    (pinned) memory, copies them to the device, runs the step and copies the
+    output back: the end-to-end form of the call.
+    """
+
+    def __init__(self, k_cache, v_cache, num_seqs, num_q_heads, max_blocks_per_seq, scale, k_scale=None,
+                 v_scale=None, max_context_len=None, partition_request=0, device=None):
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.k_scale, self.v_scale = k_scale, v_scale
+        nblk, nkv, bs, d = k_cache.shape
+        self.shape = (num_seqs, num_q_heads, nkv, d, bs)
+        self.max_blocks = max_blocks_per_seq
+        self.max_context_len = max_context_len or max_blocks_per_seq * bs
+        self.scale = scale
+        self.partition_request = partition_request
+        dev = device or k_cache.device
+        self.plan = plan_decode(num_seqs, num_q_heads, nkv, d, bs, self.max_context_len,
+                                _cache_dtype(k_cache) == PKV_CACHE_FP8_E4M3, partition_request)
+        self.workspace = (torch.empty(self.plan["workspace_bytes"], dtype=torch.uint8, device=dev)
+                          if self.plan["workspace_bytes"] else None)
+        self.out = torch.empty((num_seqs, num_q_heads, d), dtype=torch.bfloat16, device=dev)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._dev_inputs = None
+
+    def run(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, stream=None):
+        """Device inputs -> device output (no host traffic, no sync)."""
+        store_kvcache(k_new, v_new, self.k_cache, self.v_cache, slot_mapping, self.k_scale, self.v_scale,
+                      self.dev_err, stream)
+        return paged_attention_decode(q, self.k_cache, self.v_cache, block_tables, context_lens, self.scale,
+                                      out=self.out, k_scale=self.k_scale, v_scale=self.v_scale,
+                                      max_context_len=self.max_context_len,
+                                      partition_request=self.partition_request, workspace=self.workspace,
+                                      dev_err=self.dev_err, stream=stream)
+
+    def run_host(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, out_host, stream=None):
+        """Host (pinned) inputs -> host output: H2D copies, the step, D2H copy."""
+        if self._dev_inputs is None:
+            dev = self.k_cache.device
+            self._dev_inputs = [torch.empty_like(t, device=dev) for t in
+                                (q, k_new, v_new, slot_mapping, block_tables, context_lens)]
+        dq, dk, dv, ds, dbt, dcl = self._dev_inputs
+        for d_, h_ in zip(self._dev_inputs, (q, k_new, v_new, slot_mapping, block_tables, context_lens)):
+            d_.copy_(h_, non_blocking=True)
+        o = self.run(dq, dk, dv, ds, dbt, dcl, stream)
+        out_host.copy_(o, non_blocking=True)
+        return out_host

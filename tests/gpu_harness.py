@@ -1,0 +1,127 @@
+"""Run a seeded workload through the CUDA library and compare with the oracle.
+
+Both sides start from the same drawn rows: the GPU fills device pools with
+``store_kvcache`` and decodes with ``paged_attention_decode``; the oracle fills
+host pools with its own store and attends in fp64. Pools are compared byte for
+byte, outputs within the stated tolerance.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+from paged_kv_cache_482_b200 import pagedkv as K
+from paged_kv_cache_482_b200 import workloads as W
+
+# bf16 cache: max |g - r| <= 2e-2 and max |g - r| / max |r| <= 1e-2.
+# E4M3 cache: max |g - r| <= 5e-2 (attention over the dequantised cache).
+BF16_ABS, BF16_NORM_REL, FP8_ABS = 2e-2, 1e-2, 5e-2
+
+
+def device_pools(wl: W.Workload, device="cuda"):
+    c = wl.cfg
+    shape = (wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)
+    if wl.is_fp8:
+        kp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device=device)
+        vp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device=device)
+    else:
+        kp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device=device).view(torch.bfloat16)
+        vp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device=device).view(torch.bfloat16)
+    return kp, vp
+
+
+def to_device(wl: W.Workload, device="cuda") -> W.Workload:
+    import copy
+
+    w2 = copy.copy(wl)
+    for f in ("q", "k_new", "v_new", "slot_new", "k_hist", "v_hist", "slot_hist", "block_tables", "context_lens",
+              "k_scale", "v_scale"):
+        t = getattr(wl, f)
+        if t is not None:
+            setattr(w2, f, t.to(device).contiguous())
+    return w2
+
+
+def fill_history(wl: W.Workload, kp, vp, dev_err=None, chunk=1 << 20):
+    """Write every cached token of the workload into the device pools."""
+    H = wl.k_hist.shape[0]
+    for i in range(0, H, chunk):
+        j = min(H, i + chunk)
+        K.store_kvcache(wl.k_hist[i:j], wl.v_hist[i:j], kp, vp, wl.slot_hist[i:j], wl.k_scale, wl.v_scale, dev_err)
+
+
+def run_gpu(wl: W.Workload, partition_request=0, device="cuda", pools=None):
+    """(out, k_pool, v_pool, device status) after history + step store and decode."""
+    kp, vp = pools if pools is not None else device_pools(wl, device)
+    dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+    if pools is None:
+        fill_history(wl, kp, vp, dev_err)
+    K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, dev_err)
+    out = K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, wl.cfg.softmax_scale,
+                                   k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=wl.cfg.max_context,
+                                   partition_request=partition_request, dev_err=dev_err)
+    st = K.read_device_error(dev_err)
+    return out, kp, vp, st
+
+
+def pool_bytes(p: torch.Tensor) -> np.ndarray:
+    t = p.detach()
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
+    return t.cpu().numpy().view(np.uint16 if t.dtype == torch.int16 else np.uint8)
+
+
+def compare(out_gpu: torch.Tensor, ref: np.ndarray, fp8: bool, what=""):
+    g = out_gpu.float().cpu().double().numpy()
+    assert np.all(np.isfinite(g)), f"{what}: non-finite GPU output"
+    err = np.abs(g - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    scale = float(np.abs(ref).max()) if ref.size else 1.0
+    if fp8:
+        assert max_abs <= FP8_ABS, f"{what}: max abs {max_abs:.3e} > {FP8_ABS}"
+    else:
+        assert max_abs <= BF16_ABS, f"{what}: max abs {max_abs:.3e} > {BF16_ABS}"
+        assert max_abs <= BF16_NORM_REL * scale, f"{what}: normwise rel {max_abs / scale:.3e} > {BF16_NORM_REL}"
+    return max_abs
+
+
+def check_workload(wl_cpu: W.Workload, partition_request=0, threads=8, seq_ids=None):
+    """Full check of a workload drawn on the CPU: pools bit-exact, output in tolerance."""
+    wl = to_device(wl_cpu)
+    out, kp, vp, st = run_gpu(wl, partition_request)
+    assert st == K.PKV_OK, f"device status {st}"
+    ref, rkp, rvp, rst = O.run_workload(wl_cpu, num_threads=threads, seq_ids=seq_ids)
+    assert rst == O.ORC_OK
+    if seq_ids is None:
+        assert np.array_equal(pool_bytes(kp), rkp), "K pool differs from the oracle's"
+        assert np.array_equal(pool_bytes(vp), rvp), "V pool differs from the oracle's"
+        return compare(out, ref, wl.is_fp8, wl.cfg.name), out
+    return compare(out[seq_ids], ref, wl.is_fp8, wl.cfg.name), out
+
+
+def check_sampled(wl: W.Workload, seq_ids, partition_request=0, threads=8):
+    """Full-size GPU step; the oracle rebuilds and checks only ``seq_ids``."""
+    out, kp, vp, st = run_gpu(wl, partition_request)
+    assert st == K.PKV_OK, f"device status {st}"
+    ids = [int(i) for i in seq_ids]
+    ref, rkp, rvp, rst = O.run_workload(wl, num_threads=threads, seq_ids=ids)
+    assert rst == O.ORC_OK
+    blocks = torch.unique(wl.block_tables[ids].flatten())
+    blocks = blocks[blocks >= 0]
+    bl = blocks.cpu().numpy()
+    assert np.array_equal(pool_bytes(kp[blocks.long()]), rkp[bl]), "sampled K blocks differ from the oracle's"
+    assert np.array_equal(pool_bytes(vp[blocks.long()]), rvp[bl]), "sampled V blocks differ from the oracle's"
+    assert bool(torch.isfinite(out.float()).all()), "non-finite output somewhere in the full step"
+    return compare(out[torch.tensor(ids, device=out.device)], ref, wl.is_fp8, wl.cfg.name), out
+
+
+def sample_ids(wl: W.Workload, n: int, seed: int = 0):
+    """Longest, shortest and a seeded spread of other sequences."""
+    cl = wl.context_lens.cpu()
+    S = cl.numel()
+    g = torch.Generator().manual_seed(seed)
+    ids = {int(cl.argmax()), int(cl.argmin()), 0, S - 1}
+    ids |= set(torch.randperm(S, generator=g)[: max(0, n - len(ids))].tolist())
+    return sorted(ids)

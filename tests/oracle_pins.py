@@ -333,12 +333,19 @@ def pin_bounds_errors(lib):
                                         c.softmax_scale, lib=lib)
     assert st == O.ORC_ERR_BOUNDS
     assert np.all(out2[1] == 0) and np.array_equal(out2[0], out[0]) and np.array_equal(out2[2], out[2])
+    # a middle row, so that a length check that lets one extra token through
+    # reads the next row's (valid) entry instead of memory past the table
+    # Row 1 gets a full row of valid ids, so only the length check can refuse
+    # a length one past the table.
+    full = wl.block_tables.clone()
+    full[1, :] = full[1, 0]
     for bad_len in (0, c.max_blocks_per_seq * c.block_size + 1):
         cl = wl.context_lens.clone()
-        cl[2] = bad_len
-        out3, st = O.paged_attention_decode(wl.q, kp, vp, wl.block_tables, cl, c.num_kv_heads, c.block_size,
+        cl[1] = bad_len
+        out3, st = O.paged_attention_decode(wl.q, kp, vp, full, cl, c.num_kv_heads, c.block_size,
                                             c.softmax_scale, lib=lib)
-        assert st == O.ORC_ERR_BOUNDS and np.all(out3[2] == 0) and np.array_equal(out3[0], out[0])
+        assert st == O.ORC_ERR_BOUNDS and np.all(out3[1] == 0)
+        assert np.array_equal(out3[0], out[0]) and np.array_equal(out3[2], out[2])
 
 
 ALL_PINS = [

@@ -1,0 +1,135 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every symbol the
+header declares, and refuses bad arguments before launching anything."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def K():
+    from paged_kv_cache_482_b200 import build as B
+
+    B.build()
+    from paged_kv_cache_482_b200 import pagedkv
+
+    pagedkv.lib()
+    return pagedkv
+
+
+def declared_symbols():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names |= set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(pkv_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported(K):
+    names = declared_symbols()
+    assert {"pkv_store_kvcache", "pkv_paged_attention_decode", "pkv_plan_decode"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", K.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(pkv_\w+)", out))
+    assert names <= exported, f"missing: {names - exported}"
+    assert exported <= names, f"exported but not declared: {exported - names}"
+    for n in names:
+        getattr(K.lib(), n)
+
+
+def test_version_and_status_strings(K):
+    assert K.version() == 0x000100
+    for s in range(7):
+        assert K.status_string(s) and K.status_string(s) != "unknown status"
+    assert K.status_string(99) == "unknown status"
+
+
+def _decode(L, **kw):
+    a = dict(q=0x10000, kc=0x20000, vc=0x30000, bt=0x40000, maxb=8, cl=0x50000, S=4, nq=32, nkv=8, d=128, bs=256,
+             nblk=100, scale=0.088, dt=0, ks=None, vs=None, maxctx=2048, part=0, ws=None, wsb=0, out=0x60000,
+             err=None, stream=None)
+    a.update(kw)
+    return L.pkv_paged_attention_decode(a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cl"], a["S"], a["nq"],
+                                        a["nkv"], a["d"], a["bs"], a["nblk"], a["scale"], a["dt"], a["ks"], a["vs"],
+                                        a["maxctx"], a["part"], a["ws"], a["wsb"], a["out"], a["err"], a["stream"])
+
+
+def test_decode_host_checks(K):
+    L = K.lib()
+    assert _decode(L, q=None) == K.PKV_ERR_INVALID_ARG
+    assert _decode(L, q=0x10008) == K.PKV_ERR_INVALID_ARG  # misaligned
+    assert _decode(L, d=96) == K.PKV_ERR_UNSUPPORTED
+    assert _decode(L, nq=24, nkv=8) == K.PKV_ERR_UNSUPPORTED  # group 3
+    assert _decode(L, nq=30, nkv=8) == K.PKV_ERR_INVALID_ARG
+    assert _decode(L, bs=100) == K.PKV_ERR_INVALID_ARG
+    assert _decode(L, bs=4) == K.PKV_ERR_INVALID_ARG
+    assert _decode(L, maxctx=4096) == K.PKV_ERR_INVALID_ARG  # beyond the table
+    assert _decode(L, dt=1) == K.PKV_ERR_INVALID_ARG  # FP8 without scales
+    assert _decode(L, scale=float("nan")) == K.PKV_ERR_INVALID_ARG
+    assert _decode(L, part=256) == K.PKV_ERR_WORKSPACE  # split needs a workspace
+    assert _decode(L, part=256, ws=0x70000, wsb=16) == K.PKV_ERR_WORKSPACE
+    assert _decode(L, S=0) == K.PKV_OK  # nothing to do, nothing launched
+
+
+def test_store_host_checks(K):
+    L = K.lib()
+    ok = dict(k=0x10000, v=0x20000, kc=0x30000, vc=0x40000, sm=0x50000, N=4, nkv=8, d=128, bs=16, nblk=10, dt=0,
+              ks=None, vs=None)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.pkv_store_kvcache(a["k"], a["v"], a["kc"], a["vc"], a["sm"], a["N"], a["nkv"], a["d"], a["bs"],
+                                   a["nblk"], a["dt"], a["ks"], a["vs"], None, None)
+
+    assert call(k=None) == K.PKV_ERR_INVALID_ARG
+    assert call(kc=0x30004) == K.PKV_ERR_INVALID_ARG
+    assert call(d=12) == K.PKV_ERR_INVALID_ARG
+    assert call(dt=1) == K.PKV_ERR_INVALID_ARG
+    assert call(dt=7) == K.PKV_ERR_INVALID_ARG
+    assert call(N=0) == K.PKV_OK
+
+
+@pytest.mark.parametrize("name,split,ws", [
+    ("tiny", False, False), ("qwen3_0.6b", False, False), ("qwen3_8b", False, False),
+    ("prefix_shared", False, False), ("long_fp8", True, True)])
+def test_plans_of_the_workloads(K, name, split, ws):
+    from paged_kv_cache_482_b200 import workloads as W
+
+    c = W.CONFIGS[name]
+    p = K.plan_decode(c.num_seqs, c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size, c.max_context,
+                      c.cache_dtype == W.CACHE_FP8)
+    if name == "tiny":
+        return  # latency-bound; either plan is valid
+    assert (p["partition_tokens"] > 0) == split, p
+    assert (p["workspace_bytes"] > 0) == ws
+    if split:
+        assert p["max_partitions"] == -(-c.max_context // p["partition_tokens"])
+        rows = c.num_seqs * c.num_q_heads * p["max_partitions"]
+        assert p["workspace_bytes"] >= rows * (c.head_dim + 2) * 4
+
+
+def test_plan_requests(K):
+    p = K.plan_decode(4, 32, 8, 128, 16, 32768, True, 1000)
+    assert p["partition_tokens"] % 64 == 0 and p["partition_tokens"] >= 1000
+    p = K.plan_decode(4, 32, 8, 128, 256, 2048, False, -1)
+    assert p["partition_tokens"] == 0 and p["workspace_bytes"] == 0
+    with pytest.raises(K.PagedKVError):
+        K.plan_decode(4, 32, 8, 128, 16, 32768, True, -1)  # one partition cannot span 2048 blocks
+
+
+def test_binding_refuses_to_run_without_library(tmp_path):
+    from paged_kv_cache_482_b200 import pagedkv
+
+    with pytest.raises(RuntimeError):
+        pagedkv._lib_saved = pagedkv._lib
+        try:
+            pagedkv._lib = None
+            pagedkv.lib(str(tmp_path / "missing.so"))
+        finally:
+            pagedkv._lib = pagedkv._lib_saved
