@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--config", default="qwen3_8b", choices=sorted(W.CONFIGS))
     ap.add_argument("--partition", type=int, default=0, help="0 auto, -1 never split, >0 tokens per partition")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--num-seqs", type=int, default=0, help="override the workload's sequence count")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -199,6 +200,26 @@ def nvsmi_ids(local_rank: int):
     return [local_rank]
 
 
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (identity alone)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(world: int, seqs_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank decodes its own batch each step (weak
+    scaling); the job takes as long as its slowest rank."""
+    return world * seqs_per_rank * steps / (max_ms * 1e-3)
+
+
 # --------------------------------------------------------------- CPU oracle
 
 
@@ -277,10 +298,11 @@ def cpu_baseline(wl: W.Workload, target_s: float) -> dict:
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return 0
+    if rank_env()[1] != 0:
+        return 0  # the CPU oracle runs once, on rank 0
     cfg = W.CONFIGS[args.config]
+    if args.num_seqs:
+        cfg = cfg.with_(num_seqs=args.num_seqs, name=f"{cfg.name}[{args.num_seqs} seqs]")
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wl = W.generate(cfg, args.seed, device=dev)
     threads = cpu_threads()
@@ -325,9 +347,7 @@ def main():
 
     from paged_kv_cache_482_b200 import pagedkv as K
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -342,6 +362,8 @@ def main():
             dist.barrier()
 
     cfg = W.CONFIGS[args.config]
+    if args.num_seqs:
+        cfg = cfg.with_(num_seqs=args.num_seqs, name=f"{cfg.name}[{args.num_seqs} seqs]")
     wl = W.generate(cfg, args.seed + rank, device="cuda")
     c = cfg
     shape = (wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)
@@ -419,10 +441,7 @@ def main():
     barrier()
     e2e_ms = x0.elapsed_time(x1)
 
-    t = torch.tensor([elapsed_ms, decode_ms, e2e_ms], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, decode_ms, e2e_ms = (float(x) for x in t.tolist())
+    elapsed_ms, decode_ms, e2e_ms = max_over_ranks([elapsed_ms, decode_ms, e2e_ms], dist, device="cuda")
 
     if rank == 0:
         ab = algorithmic_bytes(wl)
@@ -431,7 +450,7 @@ def main():
         achieved = bytes_launch / (decode_ms * 1e-3) / 1e9
         pt = step.plan["partition_tokens"]
         traffic = recorded_traffic(c.name, pt)
-        value = world * c.num_seqs * Kst / (elapsed_ms * 1e-3)
+        value = job_throughput(world, c.num_seqs, Kst, elapsed_ms)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": Kst, "warmup": args.warmup,
             "ms_per_step": elapsed_ms / Kst, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -454,7 +473,7 @@ def main():
                          "algorithmic_bytes_per_launch": bytes_launch,
                          "bytes_note": ("unique bytes: shared prefix counted once" if c.prefix_tokens else
                                         "KV rows of every context token + q + out + block-table entries")},
-            "e2e": {"value": world * c.num_seqs * args.e2e_steps / (e2e_ms * 1e-3), "unit": UNIT,
+            "e2e": {"value": job_throughput(world, c.num_seqs, args.e2e_steps, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
             "gpu_launches": launches_per_step * Kst,
             "clocks": clocks,

@@ -51,11 +51,11 @@ def stale(lib: str = LIB) -> bool:
     return any(os.path.getmtime(d) > t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=(), lib: str = LIB) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=(), lib: str = LIB, build_dir: str = BUILD) -> str:
     """Compile and link; returns the library path."""
     if not force and not stale(lib):
         return lib
-    os.makedirs(BUILD, exist_ok=True)
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     inc = ["-I", INCLUDE, "-I", CSRC]
     flags = NVCC_FLAGS + list(extra_flags)
@@ -63,7 +63,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=(), lib: str =
         flags = flags + ["-Xptxas", "-v"]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         cmd = [cc, *ARCH, *flags, *inc, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:

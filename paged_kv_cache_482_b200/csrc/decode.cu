@@ -1,8 +1,8 @@
 // decode.cu -- instantiations and launch of the paged decode kernels.
 //
-// Tile shape per cache type: a stage holds TILE tokens of K and of V, 16 KB
-// in total, four stages deep, four consumer warps. That keeps 48 KB or more
-// of loads in flight per block and lets two to three blocks share an SM.
+// Tile shape: four warps, each taking up to four 32-lane steps of a tile;
+// stages hold K and V of one tile and the ring is about 48 KB deep, so that
+// four blocks share an SM with well over 100 KB of loads in flight.
 #include <atomic>
 
 #include "decode.cuh"
@@ -11,21 +11,15 @@ namespace pkv {
 
 namespace {
 
-template <int D, bool FP8>
-struct TileOf {
-    static constexpr int kRowBytes = D * (FP8 ? 1 : 2);
-    static constexpr int kTile = 16384 / (2 * kRowBytes);  // 32 (bf16 d128) .. 128 (e4m3 d64)
-};
-
-constexpr int kStages = 4;
-constexpr int kConsumerWarps = 4;
-
 template <int D, int G, bool FP8>
 cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
-    constexpr int TILE = TileOf<D, FP8>::kTile;
-    constexpr int MINB = (G <= 4) ? 3 : 2;
-    using T = DecodeTraits<D, G, FP8, TILE, kStages, kConsumerWarps>;
-    auto kern = paged_decode_kernel<D, G, FP8, TILE, kStages, kConsumerWarps, MINB>;
+    using T = DecodeTraits<D, G, FP8>;
+#ifdef PKV_DECODE_MIN_BLOCKS
+    constexpr int MINB = PKV_DECODE_MIN_BLOCKS;
+#else
+    constexpr int MINB = (G <= 4) ? 4 : 2;  // 4 x 128 threads at 128 registers fill the register file
+#endif
+    auto kern = paged_decode_kernel<D, G, FP8, MINB>;
 
     // The opt-in to more than 48 KB of dynamic shared memory is a property of
     // the function on a device; set it once per device.
@@ -50,6 +44,17 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
 }
 
 template <int D, bool FP8>
+int tile_of(int group) {
+    switch (group) {
+        case 1: return DecodeTraits<D, 1, FP8>::kTile;
+        case 2: return DecodeTraits<D, 2, FP8>::kTile;
+        case 4: return DecodeTraits<D, 4, FP8>::kTile;
+        case 8: return DecodeTraits<D, 8, FP8>::kTile;
+        default: return 0;
+    }
+}
+
+template <int D, bool FP8>
 cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) {
     switch (group) {
         case 1: return launch_one<D, 1, FP8>(p, stream);
@@ -63,9 +68,8 @@ cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) 
 }  // namespace
 
 int decode_tile_tokens(int head_dim, int group, bool fp8) {
-    if (group != 1 && group != 2 && group != 4 && group != 8) return 0;
-    if (head_dim == 128) return fp8 ? TileOf<128, true>::kTile : TileOf<128, false>::kTile;
-    if (head_dim == 64) return fp8 ? TileOf<64, true>::kTile : TileOf<64, false>::kTile;
+    if (head_dim == 128) return fp8 ? tile_of<128, true>(group) : tile_of<128, false>(group);
+    if (head_dim == 64) return fp8 ? tile_of<64, true>(group) : tile_of<64, false>(group);
     return 0;
 }
 

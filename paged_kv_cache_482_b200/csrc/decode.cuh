@@ -9,19 +9,26 @@
 // attention is computed flash-style, without materialising the score row
 // ("Nano-vLLM：轻量高效的大模型推理框架", section 三.3 注意力层).
 //
-// Block structure: NCW consumer warps + 1 producer warp.
-//  * Producer (one lane): walks the partition in tiles of TILE logical
+// Block structure: 4 consumer warps + 1 producer warp.
+//  * Producer (one lane): walks the partition in tiles of kTile logical
 //    tokens. A tile is cut at block boundaries into runs that are contiguous
 //    in the HND pool; each run of K and of V is one bulk copy (non-tensor TMA,
-//    cp.async.bulk) into a STAGES-deep ring in shared memory, completing on
+//    cp.async.bulk) into a kStages-deep ring in shared memory, completing on
 //    the stage's "full" mbarrier. Only valid tokens are copied.
-//  * Consumers: warp w owns rows [w*R, (w+1)*R) of every tile. A token row is
-//    spread over LPT = head_dim/8 lanes, 8 elements each (16-byte loads for
-//    bf16, 8-byte for E4M3), so a warp handles 32/LPT tokens per step. Per
-//    tile: all scores of the warp's rows (8 fp32 FMAs per head per lane, then
-//    a butterfly shuffle sum over the LPT lanes), the warp's running max per
-//    head, rescale, then P*V into fp32 accumulators. Scores are kept in base
-//    2: q is pre-multiplied by scale*log2(e) (and by the K scale for E4M3).
+//  * Consumers: warp w owns rows [w*kRows, (w+1)*kRows) of every tile. A row
+//    is spread over kLPT = head_dim/8 lanes ("chunk" = 8 elements each:
+//    16-byte loads for bf16, 8-byte for E4M3), so a warp covers kTPS rows per
+//    step and kSteps steps per tile.
+//      QK: each lane forms its chunk's partial dot for every (step, head)
+//      with packed f32x2 FMAs; a reduce-scatter butterfly over the kLPT
+//      lanes of a row then leaves each lane holding the full score of one
+//      (step, head), so the exponentials, the running max and the running
+//      sum are computed once per score, not once per lane.
+//      Softmax: per head, tile max over the warp's rows, rescale factor
+//      alpha, p = 2^(s - m); scores are base 2 because q is pre-multiplied
+//      by scale*log2(e) (and by the K scale for E4M3). p and alpha go through
+//      a few bytes of shared memory to the lanes that own the V chunks.
+//      PV: fp32 accumulators, packed f32x2 FMAs.
 //  * Epilogue: merge the warps' (max, sum, accumulators) in shared memory and
 //    write bf16 output, or, for split-K, the normalised fp32 partial with its
 //    (max, sum) for the reduce kernel.
@@ -65,32 +72,55 @@ struct DecodeParams {
 
 constexpr int kMaxIdsPerPartition = 256;
 
-template <int D, int G, bool FP8, int TILE, int STAGES, int NCW>
+// Tuning constants (compile-time; the defaults are the measured choice).
+#ifndef PKV_DECODE_CONSUMER_WARPS
+#define PKV_DECODE_CONSUMER_WARPS 4
+#endif
+#ifndef PKV_DECODE_MAX_STEPS
+#define PKV_DECODE_MAX_STEPS 4
+#endif
+#ifndef PKV_DECODE_RING_BYTES
+#define PKV_DECODE_RING_BYTES 49152
+#endif
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+constexpr int cclamp(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+
+template <int D, int G, bool FP8>
 struct DecodeTraits {
+    static constexpr int kNCW = PKV_DECODE_CONSUMER_WARPS;
     static constexpr int kESize = FP8 ? 1 : 2;
     static constexpr int kRowBytes = D * kESize;
-    static constexpr int kEPL = 8;               // elements per lane of a row
-    static constexpr int kLPT = D / kEPL;        // lanes per token row
-    static constexpr int kTPS = 32 / kLPT;       // tokens per warp step
-    static constexpr int kRows = TILE / NCW;     // rows per warp per tile
-    static constexpr int kSteps = kRows / kTPS;  // steps per warp per tile
-    static constexpr int kTileBytes = TILE * kRowBytes;
-    static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kThreads = (NCW + 1) * 32;
-    // shared memory layout (bytes)
-    static constexpr int kOffBars = STAGES * kStageBytes;
-    static constexpr int kOffIds = kOffBars + 2 * STAGES * 8;
-    static constexpr int kOffMerge = kOffIds + kMaxIdsPerPartition * 4;
-    static constexpr int kMergeFloats = NCW * G * D + 2 * NCW * G + NCW * G;
-    static constexpr int kSmemBytes = kOffMerge + kMergeFloats * 4;
-    static_assert(D % (kEPL * 1) == 0 && (32 % kLPT) == 0, "row mapping");
-    static_assert(kRows % kTPS == 0 && kSteps >= 1, "tile must split evenly over warps and steps");
-    static_assert(kStageBytes % 128 == 0, "stage alignment");
+    static constexpr int kLPT = D / 8;                    // lanes per row
+    static constexpr int kTPS = 32 / kLPT;                // rows per warp step
+    static constexpr int kSteps = cmin(PKV_DECODE_MAX_STEPS, kLPT / G);  // steps per tile
+    static constexpr int kNV = kSteps * G;                // scores per lane group (<= kLPT)
+    static constexpr int kShiftV = ilog2(kLPT) - ilog2(kNV);
+    static constexpr int kRows = kSteps * kTPS;           // rows per warp per tile
+    static constexpr int kTile = kRows * kNCW;            // tokens per tile
+    static constexpr int kTileBytes = kTile * kRowBytes;  // one tile of K (or of V)
+    static constexpr int kStages = cclamp(PKV_DECODE_RING_BYTES / (2 * kTileBytes), 2, 8);
+    static constexpr int kThreads = kNCW * 32;
+    static constexpr int kPBufFloats = 2 * kRows * G;     // per warp: p[2 tiles][row][head]
+    // shared memory layout (bytes); the merge area reuses the rings
+    static constexpr int kRingBytes = kStages * kTileBytes;  // one ring (K or V)
+    static constexpr int kOffV = kRingBytes;
+    static constexpr int kOffBars = 2 * kRingBytes;          // full_k[S], full_v[S]
+    static constexpr int kOffCnt = kOffBars + 2 * kStages * 8;  // done_k[S], done_v[S], issued_k, issued_v
+    static constexpr int kOffIds = kOffCnt + (2 * kStages + 2) * 4;
+    static constexpr int kOffPBuf = (kOffIds + kMaxIdsPerPartition * 4 + 15) / 16 * 16;
+    static constexpr int kSmemBytes = kOffPBuf + kNCW * kPBufFloats * 4;
+    static constexpr int kMergeFloats = kNCW * G * D + 3 * kNCW * G;
+    static_assert((32 % kLPT) == 0 && kLPT >= 2, "row mapping");
+    static_assert(kSteps >= 1 && kNV <= kLPT, "one score per lane after the reduction");
+    static_assert(kTileBytes % 128 == 0, "stage alignment");
+    static_assert(kMergeFloats * 4 <= 2 * kRingBytes, "merge area must fit in the rings");
 };
 
-// 8 elements of a cached row (bf16: 16 bytes, E4M3: 8 bytes) -> fp32.
+// 8 cached elements (bf16: 16 bytes, E4M3: 8 bytes) -> 8 floats (exact).
 template <bool FP8>
-__device__ __forceinline__ void load_row8(const uint8_t *p, float (&x)[8]) {
+__device__ __forceinline__ void load8(const uint8_t *p, float (&x)[8]) {
     if constexpr (FP8) {
         const uint2 w = *reinterpret_cast<const uint2 *>(p);
         const float2 a = e4m3x2_to_float2((uint16_t)(w.x & 0xffffu));
@@ -106,17 +136,44 @@ __device__ __forceinline__ void load_row8(const uint8_t *p, float (&x)[8]) {
     }
 }
 
-template <int D, int G, bool FP8, int TILE, int STAGES, int NCW, int MIN_BLOCKS>
-__global__ void __launch_bounds__((NCW + 1) * 32, MIN_BLOCKS) paged_decode_kernel(const DecodeParams p) {
-    using T = DecodeTraits<D, G, FP8, TILE, STAGES, NCW>;
+// Reduce-scatter of N partial sums over the lanes that differ in bits
+// O, O/2, ..., 1 of the lane index. Each lane holds its N values in a
+// lane-specific order -- position i holds logical value i ^ v_lane, where
+// v_lane is the lane's own bits O.. taken as a number -- so that in every
+// round the half a lane keeps is its lower half and the half it sends is its
+// upper half: no selects. After the scatter rounds x[0] is the full sum of
+// value v_lane; rounds past one value are plain butterflies.
+template <int N, int O>
+struct ReduceScatter {
+    static __device__ __forceinline__ void run(float *x) {
+        if constexpr (O >= 1) {
+            if constexpr (N > 1) {
+#pragma unroll
+                for (int i = 0; i < N / 2; ++i) x[i] += __shfl_xor_sync(0xffffffffu, x[i + N / 2], O);
+                ReduceScatter<N / 2, O / 2>::run(x);
+            } else {
+                x[0] += __shfl_xor_sync(0xffffffffu, x[0], O);
+                ReduceScatter<1, O / 2>::run(x);
+            }
+        }
+    }
+};
+
+template <int D, int G, bool FP8, int MIN_BLOCKS>
+__global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
+    paged_decode_kernel(const DecodeParams p) {
+    using T = DecodeTraits<D, G, FP8>;
+    constexpr int NCW = T::kNCW;
+    constexpr int TILE = T::kTile;
+    constexpr int STAGES = T::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + T::kOffBars);
-    uint64_t *empty_bar = full_bar + STAGES;
+    uint64_t *full_k = reinterpret_cast<uint64_t *>(smem + T::kOffBars);
+    uint64_t *full_v = full_k + STAGES;
+    int *done_k = reinterpret_cast<int *>(smem + T::kOffCnt);  // per stage: warps done, cumulative
+    int *done_v = done_k + STAGES;
+    int *issued_k = done_v + STAGES;  // tiles issued so far
+    int *issued_v = issued_k + 1;
     int32_t *ids = reinterpret_cast<int32_t *>(smem + T::kOffIds);
-    float *merge_acc = reinterpret_cast<float *>(smem + T::kOffMerge);  // [NCW][G][D]
-    float *merge_m = merge_acc + NCW * G * D;                             // [NCW][G]
-    float *merge_l = merge_m + NCW * G;                                   // [NCW][G]
-    float *merge_w = merge_l + NCW * G;                                   // [NCW][G]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -138,7 +195,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, MIN_BLOCKS) paged_decode_kerne
     if (!bad_len && start >= end) return;  // partition past this sequence's end
     if (bad_len && part != 0) return;
 
-    // Stage this partition's block ids (checked) and set up the barriers.
+    // Stage this partition's block ids (checked), zero the rings (rows past
+    // the end of a partial tile are then finite, so they can take part in
+    // the arithmetic with weight 0), set up the barriers.
     const int first_blk = start >> p.log2_block_size;
     const int n_blk = bad_len ? 0 : ((end - 1) >> p.log2_block_size) - first_blk + 1;
     int bad = bad_len || n_blk > kMaxIdsPerPartition;
@@ -148,10 +207,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, MIN_BLOCKS) paged_decode_kerne
         ids[i] = id;
         bad |= (id < 0 || (long long)id >= p.num_blocks);
     }
+    for (int i = tid; i < 2 * T::kRingBytes / 16; i += T::kThreads)
+        reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], NCW);
+            mbar_init(&full_k[s], 1);
+            mbar_init(&full_v[s], 1);
+            done_k[s] = 0;
+            done_v[s] = 0;
         }
         fence_barrier_init();
     }
@@ -175,180 +238,260 @@ __global__ void __launch_bounds__((NCW + 1) * 32, MIN_BLOCKS) paged_decode_kerne
     const long long head_stride = (long long)p.block_size * T::kRowBytes;  // bytes of one (block, head) run
     const long long blk_stride = head_stride * p.num_kv_heads;
 
-    if (warp == NCW) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int s = j % STAGES;
-                if (j >= STAGES && !mbar_wait(&empty_bar[s], ((j / STAGES) - 1) & 1)) {
-                    set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
-                    break;
-                }
-                const int a0 = start + j * TILE;
-                const int a1 = min(a0 + TILE, end);
-                uint8_t *ks = smem + s * T::kStageBytes;
-                uint8_t *vs = ks + T::kTileBytes;
-                mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(2 * (a1 - a0) * T::kRowBytes));
-                for (int a = a0; a < a1;) {
-                    const int lb = a >> p.log2_block_size;
-                    const int off = a & (p.block_size - 1);
-                    const int n = min(p.block_size - off, a1 - a);
-                    const long long phys = ids[lb - first_blk];
-                    const long long src = phys * blk_stride + kvh * head_stride + (long long)off * T::kRowBytes;
-                    const int dst = (a - a0) * T::kRowBytes;
-                    bulk_g2s(ks + dst, p.k_cache + src, (uint32_t)(n * T::kRowBytes), &full_bar[s]);
-                    bulk_g2s(vs + dst, p.v_cache + src, (uint32_t)(n * T::kRowBytes), &full_bar[s]);
-                    a += n;
-                }
-                issued = j + 1;
-            }
-            // Wait for every copy still in flight before this block may exit.
-            for (int j = max(0, issued - STAGES); j < issued; ++j)
-                if (!mbar_wait(&full_bar[j % STAGES], (j / STAGES) & 1)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+    // Issue the K (or V) half of tile j into its stage: the block-table runs
+    // that make up logical tokens [start + j*TILE, ...), one bulk copy each.
+    auto issue = [&](int j, bool is_v) {
+        const int s = j % STAGES;
+        const int a0 = start + j * TILE;
+        const int a1 = min(a0 + TILE, end);
+        uint8_t *dst0 = smem + (is_v ? T::kOffV : 0) + s * T::kTileBytes;
+        const uint8_t *src0 = is_v ? p.v_cache : p.k_cache;
+        uint64_t *bar = is_v ? &full_v[s] : &full_k[s];
+        mbar_arrive_expect_tx(bar, (uint32_t)((a1 - a0) * T::kRowBytes));
+        for (int a = a0; a < a1;) {
+            const int lb = a >> p.log2_block_size;
+            const int off = a & (p.block_size - 1);
+            const int n = min(p.block_size - off, a1 - a);
+            const long long phys = ids[lb - first_blk];
+            const long long src = phys * blk_stride + kvh * head_stride + (long long)off * T::kRowBytes;
+            bulk_g2s(dst0 + (a - a0) * T::kRowBytes, src0 + src, (uint32_t)(n * T::kRowBytes), bar);
+            a += n;
         }
-        return;
+    };
+    // Count a warp as done with the K (or V) half of tile j; the last warp
+    // refills that stage with tile j + STAGES.
+    // Callers __syncwarp() first, so every lane's reads of the stage are done.
+    auto release = [&](int j, bool is_v) {
+        if (lane == 0) {
+            __threadfence_block();
+            const int s = j % STAGES;
+            int *cnt = is_v ? &done_v[s] : &done_k[s];
+            const int prev = atomicAdd(cnt, 1);
+            if (prev == (j / STAGES) * NCW + NCW - 1 && j + STAGES < n_tiles) {
+                fence_proxy_async_smem();
+                issue(j + STAGES, is_v);
+                atomicMax(is_v ? issued_v : issued_k, j + STAGES + 1);
+            }
+        }
+    };
+    if (tid == 0) {
+        fence_proxy_async_smem();  // the zeroed rings, before the copies overwrite them
+        const int first = min(STAGES, n_tiles);
+        for (int j = 0; j < first; ++j) {
+            issue(j, false);
+            issue(j, true);
+        }
+        *issued_k = first;
+        *issued_v = first;
     }
 
-    // ---------------------------------------------------------------- consumers
-    const int sub = lane / T::kLPT;   // token within a step
-    const int chunk = lane % T::kLPT;  // 8-element chunk of the row
+    // ------------------------------------------------------------ per lane
+    constexpr int LPT = T::kLPT;
+    constexpr int TPS = T::kTPS;
+    constexpr int STEPS = T::kSteps;
+    constexpr int ROWS = T::kRows;
+    constexpr int LOG2G = ilog2(G);
+    constexpr int HEAD_BITS_END = T::kShiftV + LOG2G;  // lane bits below this: duplicate or head
+    const int sub = lane / LPT;    // row within a step
+    const int chunk = lane % LPT;  // 8-element chunk of the row
+    // The score this lane holds after the reduction: (my_st, my_h), row my_row.
+    const int my_v = chunk >> T::kShiftV;
+    const int my_h = my_v & (G - 1);
+    const int my_st = my_v >> LOG2G;
+    const int my_row = my_st * TPS + sub;
+    const bool canon = (chunk & ((1 << T::kShiftV) - 1)) == 0;  // first of its duplicates
+    float *pbuf = reinterpret_cast<float *>(smem + T::kOffPBuf) + warp * T::kPBufFloats;  // [2][ROWS][G]
 
+    // q in this lane's slot order: slot hs holds head hs ^ my_h (see ReduceScatter).
     float qf[G][8];
     {
         float qs = p.qk_scale_log2;
         if constexpr (FP8) qs *= __ldg(p.k_scale + kvh);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int hs = 0; hs < G; ++hs) {
+            const int h = hs ^ my_h;
             const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p.q + ((long long)seq * p.num_q_heads + qh0 + h) * D +
                                                                   chunk * 8));
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                qf[h][2 * i] = bf16lo(ww[i]) * qs;
-                qf[h][2 * i + 1] = bf16hi(ww[i]) * qs;
+                qf[hs][2 * i] = bf16lo(ww[i]) * qs;
+                qf[hs][2 * i + 1] = bf16hi(ww[i]) * qs;
             }
         }
     }
 
     float acc[G][8];
-    float m[G], l[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        m[h] = -CUDART_INF_F;
-        l[h] = 0.f;
+    for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[h][i] = 0.f;
-    }
+    float m = -CUDART_INF_F;  // running max of head my_h
+    float l = 0.f;            // running sum of this lane's rows of head my_h
 
-    const int row0 = warp * T::kRows;
-    for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % STAGES;
-        if (!mbar_wait(&full_bar[s], (j / STAGES) & 1)) {
-            set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
-            break;
-        }
-        const int n_valid = min(TILE, end - (start + j * TILE));
-        const int cnt = min(T::kRows, n_valid - row0);  // this warp's valid rows (warp-uniform)
-        if (cnt > 0) {
-            const uint8_t *ks = smem + s * T::kStageBytes + row0 * T::kRowBytes + chunk * 8 * T::kESize;
-            const uint8_t *vs = ks + T::kTileBytes;
-            float sc[T::kSteps][G];
-            float tmax[G];
+    const int row0 = warp * ROWS;
+    const int lane_off = row0 * T::kRowBytes + chunk * 8 * T::kESize;
+
+    // QK of tile j: this lane's partial dots in its (step, head) order.
+    auto qk = [&](int j, float (&sc)[T::kNV]) {
+        const uint8_t *ks = smem + (j % STAGES) * T::kTileBytes + lane_off;
 #pragma unroll
-            for (int h = 0; h < G; ++h) tmax[h] = -CUDART_INF_F;
+        for (int ps = 0; ps < STEPS; ++ps) {
+            float kf[8];
+            load8<FP8>(ks + ((ps ^ my_st) * TPS + sub) * T::kRowBytes, kf);
 #pragma unroll
-            for (int st = 0; st < T::kSteps; ++st) {
-                const int r = st * T::kTPS + sub;
-                if (st * T::kTPS < cnt) {
-                    const bool valid = r < cnt;
-                    float kf[8];
-                    if (valid) {
-                        load_row8<FP8>(ks + r * T::kRowBytes, kf);
-                    } else {
+            for (int hs = 0; hs < G; ++hs) {
+                float a = qf[hs][0] * kf[0];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) kf[i] = 0.f;
-                    }
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        float d = 0.f;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) d = fmaf(qf[h][i], kf[i], d);
-#pragma unroll
-                        for (int o = T::kLPT / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-                        sc[st][h] = valid ? d : -CUDART_INF_F;
-                        tmax[h] = fmaxf(tmax[h], sc[st][h]);
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < G; ++h) sc[st][h] = -CUDART_INF_F;
-                }
+                for (int i = 1; i < 8; ++i) a = fmaf(qf[hs][i], kf[i], a);
+                sc[ps * G + hs] = a;
             }
-            // warp-wide max per head, then rescale the running state
+        }
+    };
+    // Scores of tile j -> p (to this warp's p buffer) and the rescale factor
+    // of head my_h; returns whether any head of the warp changed its max.
+    auto softmax = [&](int j, float (&sc)[T::kNV], float &alpha) {
+        ReduceScatter<T::kNV, LPT / 2>::run(sc);
+        const int n_valid = min(TILE, end - (start + j * TILE));
+        const float sv = my_row < n_valid - row0 ? sc[0] : -CUDART_INF_F;
+        float tmax = sv;
+#pragma unroll
+        for (int o = 1 << HEAD_BITS_END; o < 32; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+        const float m_new = fmaxf(m, tmax);
+        const float mref = m_new == -CUDART_INF_F ? 0.f : m_new;  // no row seen yet: keep everything at 0
+        alpha = exp2f(m - mref);
+        const float pr = exp2f(sv - mref);
+        l = fmaf(l, alpha, pr);
+        m = m_new;
+        if (canon) pbuf[(j & 1) * ROWS * G + my_row * G + my_h] = pr;
+    };
+    // P * V of tile j into the accumulators (rows past the end have p = 0).
+    auto pv = [&](int j) {
+        const uint8_t *vs = smem + T::kOffV + (j % STAGES) * T::kTileBytes + lane_off;
+        const float *pb = pbuf + (j & 1) * ROWS * G;
+#pragma unroll
+        for (int st = 0; st < STEPS; ++st) {
+            const int r = st * TPS + sub;
+            float vf[8];
+            load8<FP8>(vs + r * T::kRowBytes, vf);
+            float pr[G];
+            if constexpr (G % 4 == 0) {
+#pragma unroll
+                for (int h = 0; h < G; h += 4) {
+                    const float4 t = *reinterpret_cast<const float4 *>(pb + r * G + h);
+                    pr[h] = t.x; pr[h + 1] = t.y; pr[h + 2] = t.z; pr[h + 3] = t.w;
+                }
+            } else if constexpr (G == 2) {
+                const float2 t = *reinterpret_cast<const float2 *>(pb + r * G);
+                pr[0] = t.x; pr[1] = t.y;
+            } else {
+                pr[0] = pb[r];
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[h][i] = fmaf(pr[h], vf[i], acc[h][i]);
+        }
+    };
+    // acc[h] *= alpha of head h (held by the lanes with my_h == h), only when
+    // some head's max moved.
+    auto rescale = [&](float alpha) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
             for (int h = 0; h < G; ++h) {
+                const float a = __shfl_sync(0xffffffffu, alpha, h << T::kShiftV);  // lane: chunk = h, step 0, row 0
 #pragma unroll
-                for (int o = T::kLPT; o < 32; o <<= 1) tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], o));
-                const float m_new = fmaxf(m[h], tmax[h]);
-                const float alpha = exp2f(m[h] - m_new);
-                m[h] = m_new;
-                l[h] *= alpha;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[h][i] *= alpha;
-            }
-            // P * V
-#pragma unroll
-            for (int st = 0; st < T::kSteps; ++st) {
-                const int r = st * T::kTPS + sub;
-                if (st * T::kTPS < cnt) {
-                    if (r < cnt) {
-                        float vf[8];
-                        load_row8<FP8>(vs + r * T::kRowBytes, vf);
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float pr = exp2f(sc[st][h] - m[h]);
-                            l[h] += pr;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) acc[h][i] = fmaf(pr, vf[i], acc[h][i]);
-                        }
-                    }
-                }
+                for (int i = 0; i < 8; ++i) acc[h][i] *= a;
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[s]);
+    };
+
+    // Software pipeline: iteration j runs QK of tile j, then the shuffle /
+    // exponential chain of tile j interleaved with P * V of tile j - 1.
+    bool ok = true;
+    if (n_tiles > 0) {
+        float sc[T::kNV];
+        float alpha;
+        if (!mbar_wait(&full_k[0], 0)) ok = false;
+        if (ok) {
+            qk(0, sc);
+            __syncwarp();
+            release(0, false);
+            softmax(0, sc, alpha);  // acc is still zero: nothing to rescale
+            __syncwarp();
+        }
+        for (int j = 1; ok && j < n_tiles; ++j) {
+            if (!mbar_wait(&full_k[j % STAGES], (j / STAGES) & 1) ||
+                !mbar_wait(&full_v[(j - 1) % STAGES], ((j - 1) / STAGES) & 1)) {
+                ok = false;
+                break;
+            }
+            qk(j, sc);
+            softmax(j, sc, alpha);
+            pv(j - 1);
+            __syncwarp();
+            release(j, false);
+            release(j - 1, true);
+            rescale(alpha);
+        }
+        if (ok && mbar_wait(&full_v[(n_tiles - 1) % STAGES], ((n_tiles - 1) / STAGES) & 1)) {
+            pv(n_tiles - 1);
+            __syncwarp();
+            release(n_tiles - 1, true);
+        } else {
+            ok = false;
+        }
     }
+    if (!ok) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
 
     // ------------------------------------------------------------- epilogue
-    // Sum over the token groups of the warp (lanes with the same chunk).
+    // l: sum over the lanes holding the same head (step and row bits).
 #pragma unroll
-    for (int o = T::kLPT; o < 32; o <<= 1) {
+    for (int o = 1 << HEAD_BITS_END; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    // accumulators: sum over the rows of a step (lanes with the same chunk).
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
+    for (int o = LPT; o < 32; o <<= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h)
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[h][i] += __shfl_xor_sync(0xffffffffu, acc[h][i], o);
-        }
     }
+    // Every warp is past the loop: no stage is read any more. Wait for any
+    // copy still in flight (only after a timeout), then reuse the rings.
+    __syncthreads();
+    if (tid == 0) {
+        const int ik = *issued_k, iv = *issued_v;
+        for (int j = max(0, ik - STAGES); j < ik; ++j)
+            if (!mbar_wait(&full_k[j % STAGES], (j / STAGES) & 1)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+        for (int j = max(0, iv - STAGES); j < iv; ++j)
+            if (!mbar_wait(&full_v[j % STAGES], (j / STAGES) & 1)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+    }
+    __syncthreads();
+    float *merge_acc = reinterpret_cast<float *>(smem);  // [NCW][G][D]
+    float *merge_m = merge_acc + NCW * G * D;            // [NCW][G]
+    float *merge_l = merge_m + NCW * G;                  // [NCW][G]
+    float *merge_w = merge_l + NCW * G;                  // [NCW][G]
     if (sub == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) merge_acc[(warp * G + h) * D + chunk * 8 + i] = acc[h][i];
-            if (chunk == 0) {
-                merge_m[warp * G + h] = m[h];
-                merge_l[warp * G + h] = l[h];
-            }
+            for (int i = 0; i < 8; i += 4)
+                *reinterpret_cast<float4 *>(merge_acc + (warp * G + h) * D + chunk * 8 + i) =
+                    make_float4(acc[h][i], acc[h][i + 1], acc[h][i + 2], acc[h][i + 3]);
+        if (canon && my_st == 0) {
+            merge_m[warp * G + my_h] = m;
+            merge_l[warp * G + my_h] = l;
         }
     }
-    named_sync(1, NCW * 32);
+    __syncthreads();
     if (tid < G) {
         const int h = tid;
         float M = -CUDART_INF_F;
         for (int w = 0; w < NCW; ++w) M = fmaxf(M, merge_m[w * G + h]);
         float L = 0.f;
         for (int w = 0; w < NCW; ++w) {
-            const float e = exp2f(merge_m[w * G + h] - M);  // 0 for a warp that saw no token
+            // 0 for a warp that saw no token (its m is -inf, its l and acc 0)
+            const float e = merge_m[w * G + h] == -CUDART_INF_F ? 0.f : exp2f(merge_m[w * G + h] - M);
             merge_w[w * G + h] = e;
             L += merge_l[w * G + h] * e;
         }
@@ -361,8 +504,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, MIN_BLOCKS) paged_decode_kerne
             ml[1] = L;
         }
     }
-    named_sync(1, NCW * 32);
-    for (int idx = tid; idx < G * D; idx += NCW * 32) {
+    __syncthreads();
+    for (int idx = tid; idx < G * D; idx += T::kThreads) {
         const int h = idx / D;
         float o = 0.f;
 #pragma unroll

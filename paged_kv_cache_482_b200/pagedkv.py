@@ -57,29 +57,33 @@ def lib(path: str = LIB_PATH):
     """The loaded library; raises if it is not built."""
     global _lib
     with _lock:
-        if _lib is not None:
-            return _lib
-        if not os.path.exists(path):
-            raise RuntimeError(f"{path} is missing: build it with `python -m paged_kv_cache_482_b200.build` "
-                               "(there is no CPU fallback)")
-        L = ctypes.CDLL(path)
-        c = ctypes
-        vp, i32, i64, f32, sz = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
-        L.pkv_store_kvcache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp, vp, vp]
-        L.pkv_store_kvcache.restype = i32
-        L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
-        L.pkv_plan_decode.restype = i32
-        L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i64, f32, i32, vp,
-                                                 vp, i32, i32, vp, sz, vp, vp, vp]
-        L.pkv_paged_attention_decode.restype = i32
-        L.pkv_status_string.argtypes = [i32]
-        L.pkv_status_string.restype = c.c_char_p
-        L.pkv_read_device_error.argtypes = [vp, vp]
-        L.pkv_read_device_error.restype = i32
-        L.pkv_version.argtypes = []
-        L.pkv_version.restype = i32
-        _lib = L
-        return L
+        if _lib is None:
+            _lib = load_library(path)
+        return _lib
+
+
+def load_library(path: str):
+    """Load and declare a libpagedkv.so at ``path`` (not cached)."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m paged_kv_cache_482_b200.build` "
+                           "(there is no CPU fallback)")
+    L = ctypes.CDLL(path)
+    c = ctypes
+    vp, i32, i64, f32, sz = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
+    L.pkv_store_kvcache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp, vp, vp]
+    L.pkv_store_kvcache.restype = i32
+    L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
+    L.pkv_plan_decode.restype = i32
+    L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i64, f32, i32, vp,
+                                             vp, i32, i32, vp, sz, vp, vp, vp]
+    L.pkv_paged_attention_decode.restype = i32
+    L.pkv_status_string.argtypes = [i32]
+    L.pkv_status_string.restype = c.c_char_p
+    L.pkv_read_device_error.argtypes = [vp, vp]
+    L.pkv_read_device_error.restype = i32
+    L.pkv_version.argtypes = []
+    L.pkv_version.restype = i32
+    return L
 
 
 def status_string(status: int) -> str:
