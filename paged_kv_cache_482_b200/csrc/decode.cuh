@@ -240,8 +240,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
 
     // Issue the K (or V) half of tile j into its stage: the block-table runs
     // that make up logical tokens [start + j*TILE, ...), one bulk copy each.
-    auto issue = [&](int j, bool is_v) {
-        const int s = j % STAGES;
+    auto issue = [&](int j, int s, bool is_v) {  // s == j % STAGES
         const int a0 = start + j * TILE;
         const int a1 = min(a0 + TILE, end);
         uint8_t *dst0 = smem + (is_v ? T::kOffV : 0) + s * T::kTileBytes;
@@ -260,16 +259,17 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     };
     // Count a warp as done with the K (or V) half of tile j; the last warp
     // refills that stage with tile j + STAGES.
-    // Callers __syncwarp() first, so every lane's reads of the stage are done.
-    auto release = [&](int j, bool is_v) {
+    // Warp done with the K (or V) half of tile j, which sits in stage s in
+    // round r (j = r * STAGES + s). Callers __syncwarp() first, so every
+    // lane's reads of the stage are done.
+    auto release = [&](int j, int s, int r, bool is_v) {
         if (lane == 0) {
             __threadfence_block();
-            const int s = j % STAGES;
             int *cnt = is_v ? &done_v[s] : &done_k[s];
             const int prev = atomicAdd(cnt, 1);
-            if (prev == (j / STAGES) * NCW + NCW - 1 && j + STAGES < n_tiles) {
+            if (prev == r * NCW + NCW - 1 && j + STAGES < n_tiles) {
                 fence_proxy_async_smem();
-                issue(j + STAGES, is_v);
+                issue(j + STAGES, s, is_v);
                 atomicMax(is_v ? issued_v : issued_k, j + STAGES + 1);
             }
         }
@@ -278,8 +278,8 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         fence_proxy_async_smem();  // the zeroed rings, before the copies overwrite them
         const int first = min(STAGES, n_tiles);
         for (int j = 0; j < first; ++j) {
-            issue(j, false);
-            issue(j, true);
+            issue(j, j, false);
+            issue(j, j, true);
         }
         *issued_k = first;
         *issued_v = first;
@@ -302,23 +302,28 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     const bool canon = (chunk & ((1 << T::kShiftV) - 1)) == 0;  // first of its duplicates
     float *pbuf = reinterpret_cast<float *>(smem + T::kOffPBuf) + warp * T::kPBufFloats;  // [2][ROWS][G]
 
-    // q in this lane's slot order: slot hs holds head hs ^ my_h (see ReduceScatter).
-    float qf[G][8];
-    {
-        float qs = p.qk_scale_log2;
-        if constexpr (FP8) qs *= __ldg(p.k_scale + kvh);
+    // q in this lane's slot order: slot hs holds head hs ^ my_h (see
+    // ReduceScatter). bf16 cache: q stays packed bf16 and QK uses the
+    // bf16 x bf16 -> fp32 FMA (exact products, fp32 sums); the scale is applied
+    // to the reduced score. E4M3 cache: q in fp32, pre-multiplied by the scale
+    // and the K scale.
+    uint32_t qw[G][4];
+    float qf[FP8 ? G : 1][8];
 #pragma unroll
-        for (int hs = 0; hs < G; ++hs) {
-            const int h = hs ^ my_h;
-            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p.q + ((long long)seq * p.num_q_heads + qh0 + h) * D +
-                                                                  chunk * 8));
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int hs = 0; hs < G; ++hs) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(
+            p.q + ((long long)seq * p.num_q_heads + qh0 + (hs ^ my_h)) * D + chunk * 8));
+        qw[hs][0] = w.x; qw[hs][1] = w.y; qw[hs][2] = w.z; qw[hs][3] = w.w;
+    }
+    if constexpr (FP8) {
+        const float qs = p.qk_scale_log2 * __ldg(p.k_scale + kvh);
+#pragma unroll
+        for (int hs = 0; hs < G; ++hs)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                qf[hs][2 * i] = bf16lo(ww[i]) * qs;
-                qf[hs][2 * i + 1] = bf16hi(ww[i]) * qs;
+                qf[hs][2 * i] = bf16lo(qw[hs][i]) * qs;
+                qf[hs][2 * i + 1] = bf16hi(qw[hs][i]) * qs;
             }
-        }
     }
 
     float acc[G][8];
@@ -332,19 +337,32 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     const int row0 = warp * ROWS;
     const int lane_off = row0 * T::kRowBytes + chunk * 8 * T::kESize;
 
-    // QK of tile j: this lane's partial dots in its (step, head) order.
-    auto qk = [&](int j, float (&sc)[T::kNV]) {
-        const uint8_t *ks = smem + (j % STAGES) * T::kTileBytes + lane_off;
+    // QK of the tile in K stage sk: this lane's partial dots in its (step, head) order.
+    auto qk = [&](int sk, float (&sc)[T::kNV]) {
+        const uint8_t *ks = smem + sk * T::kTileBytes + lane_off;
 #pragma unroll
         for (int ps = 0; ps < STEPS; ++ps) {
-            float kf[8];
-            load8<FP8>(ks + ((ps ^ my_st) * TPS + sub) * T::kRowBytes, kf);
+            const uint8_t *row = ks + ((ps ^ my_st) * TPS + sub) * T::kRowBytes;
+            if constexpr (FP8) {
+                float kf[8];
+                load8<FP8>(row, kf);
 #pragma unroll
-            for (int hs = 0; hs < G; ++hs) {
-                float a = qf[hs][0] * kf[0];
+                for (int hs = 0; hs < G; ++hs) {
+                    float a = qf[hs][0] * kf[0];
 #pragma unroll
-                for (int i = 1; i < 8; ++i) a = fmaf(qf[hs][i], kf[i], a);
-                sc[ps * G + hs] = a;
+                    for (int i = 1; i < 8; ++i) a = fmaf(qf[hs][i], kf[i], a);
+                    sc[ps * G + hs] = a;
+                }
+            } else {
+                const uint4 kw4 = *reinterpret_cast<const uint4 *>(row);
+                const uint32_t kw[4] = {kw4.x, kw4.y, kw4.z, kw4.w};
+#pragma unroll
+                for (int hs = 0; hs < G; ++hs) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) a = fma_bf16x2_acc(qw[hs][i], kw[i], a);
+                    sc[ps * G + hs] = a;
+                }
             }
         }
     };
@@ -352,6 +370,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     // of head my_h; returns whether any head of the warp changed its max.
     auto softmax = [&](int j, float (&sc)[T::kNV], float &alpha) {
         ReduceScatter<T::kNV, LPT / 2>::run(sc);
+        if constexpr (!FP8) sc[0] *= p.qk_scale_log2;
         const int n_valid = min(TILE, end - (start + j * TILE));
         const float sv = my_row < n_valid - row0 ? sc[0] : -CUDART_INF_F;
         float tmax = sv;
@@ -359,16 +378,17 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         for (int o = 1 << HEAD_BITS_END; o < 32; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
         const float m_new = fmaxf(m, tmax);
         const float mref = m_new == -CUDART_INF_F ? 0.f : m_new;  // no row seen yet: keep everything at 0
-        alpha = exp2f(m - mref);
-        const float pr = exp2f(sv - mref);
+        alpha = fast_exp2(m - mref);
+        const float pr = fast_exp2(sv - mref);
         l = fmaf(l, alpha, pr);
         m = m_new;
         if (canon) pbuf[(j & 1) * ROWS * G + my_row * G + my_h] = pr;
     };
-    // P * V of tile j into the accumulators (rows past the end have p = 0).
-    auto pv = [&](int j) {
-        const uint8_t *vs = smem + T::kOffV + (j % STAGES) * T::kTileBytes + lane_off;
-        const float *pb = pbuf + (j & 1) * ROWS * G;
+    // P * V of the tile in V stage sv (p buffer half pj) into the
+    // accumulators; rows past the end have p = 0.
+    auto pv = [&](int sv, int pj) {
+        const uint8_t *vs = smem + T::kOffV + sv * T::kTileBytes + lane_off;
+        const float *pb = pbuf + pj * ROWS * G;
 #pragma unroll
         for (int st = 0; st < STEPS; ++st) {
             const int r = st * TPS + sub;
@@ -408,36 +428,40 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
 
     // Software pipeline: iteration j runs QK of tile j, then the shuffle /
     // exponential chain of tile j interleaved with P * V of tile j - 1.
+    // (sk, rk) and (sv, rv): stage and round of K tile j and V tile j - 1.
     bool ok = true;
-    if (n_tiles > 0) {
+    {
         float sc[T::kNV];
         float alpha;
+        int sk = 0, rk = 0, sv = 0, rv = 0;
         if (!mbar_wait(&full_k[0], 0)) ok = false;
         if (ok) {
             qk(0, sc);
             __syncwarp();
-            release(0, false);
+            release(0, 0, 0, false);
             softmax(0, sc, alpha);  // acc is still zero: nothing to rescale
             __syncwarp();
+            if (++sk == STAGES) { sk = 0; ++rk; }
         }
         for (int j = 1; ok && j < n_tiles; ++j) {
-            if (!mbar_wait(&full_k[j % STAGES], (j / STAGES) & 1) ||
-                !mbar_wait(&full_v[(j - 1) % STAGES], ((j - 1) / STAGES) & 1)) {
+            if (!mbar_wait(&full_k[sk], rk & 1) || !mbar_wait(&full_v[sv], rv & 1)) {
                 ok = false;
                 break;
             }
-            qk(j, sc);
+            qk(sk, sc);
             softmax(j, sc, alpha);
-            pv(j - 1);
+            pv(sv, (j - 1) & 1);
             __syncwarp();
-            release(j, false);
-            release(j - 1, true);
+            release(j, sk, rk, false);
+            release(j - 1, sv, rv, true);
             rescale(alpha);
+            if (++sk == STAGES) { sk = 0; ++rk; }
+            if (++sv == STAGES) { sv = 0; ++rv; }
         }
-        if (ok && mbar_wait(&full_v[(n_tiles - 1) % STAGES], ((n_tiles - 1) / STAGES) & 1)) {
-            pv(n_tiles - 1);
+        if (ok && mbar_wait(&full_v[sv], rv & 1)) {
+            pv(sv, (n_tiles - 1) & 1);
             __syncwarp();
-            release(n_tiles - 1, true);
+            release(n_tiles - 1, sv, rv, true);
         } else {
             ok = false;
         }

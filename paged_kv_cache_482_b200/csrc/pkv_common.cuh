@@ -103,6 +103,26 @@ __device__ __forceinline__ void named_sync(int id, int count) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// acc + lo(a)*lo(b) + hi(a)*hi(b) for bf16 pairs a, b packed in 32-bit
+// words: bf16 x bf16 products are exact in fp32, the sums are fp32 (one
+// rounding per FMA), so no unpacking to fp32 is needed.
+__device__ __forceinline__ float fma_bf16x2_acc(uint32_t a, uint32_t b, float acc) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(a), "r"(b));
+    return acc;
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, which only drops weights that are negligible
+// against the running maximum's weight of 1).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Two E4M3 codes (low byte first) -> two floats (exact), through the
 // hardware e4m3x2 -> f16x2 conversion.
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
