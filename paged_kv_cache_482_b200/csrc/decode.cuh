@@ -9,33 +9,42 @@
 // attention is computed flash-style, without materialising the score row
 // ("Nano-vLLM：轻量高效的大模型推理框架", section 三.3 注意力层).
 //
-// Block structure: 4 consumer warps + 1 producer warp.
-//  * Producer (one lane): walks the partition in tiles of kTile logical
-//    tokens. A tile is cut at block boundaries into runs that are contiguous
-//    in the HND pool; each run of K and of V is one bulk copy (non-tensor TMA,
-//    cp.async.bulk) into a kStages-deep ring in shared memory, completing on
-//    the stage's "full" mbarrier. Only valid tokens are copied.
-//  * Consumers: warp w owns rows [w*kRows, (w+1)*kRows) of every tile. A row
-//    is spread over kLPT = head_dim/8 lanes ("chunk" = 8 elements each:
-//    16-byte loads for bf16, 8-byte for E4M3), so a warp covers kTPS rows per
+// Block structure: 4 warps, each running its own pipeline over its own rows.
+//  * Tiles: a partition is walked in tiles of kTile logical tokens; warp w
+//    owns rows [w*kRows, (w+1)*kRows) of every tile. Lane 0 of the warp cuts
+//    its rows at block boundaries into runs that are contiguous in the HND
+//    pool and bulk-copies each run of K and of V (non-tensor TMA,
+//    cp.async.bulk, no multicast) into the warp's slice of a kStages-deep K
+//    ring and V ring in shared memory, completing on the warp's own "full"
+//    mbarriers. Only valid tokens are copied; the rings are zeroed once so
+//    that rows past the end of a partial tile are finite and can take part
+//    in the arithmetic with weight 0. When the warp is done with a stage it
+//    refills it itself: no producer warp, no cross-warp counters.
+//  * Lanes: a row is spread over kLPT = head_dim/8 lanes (8 elements each:
+//    16-byte loads for bf16, 8-byte for E4M3); a warp covers kTPS rows per
 //    step and kSteps steps per tile.
-//      QK: each lane forms its chunk's partial dot for every (step, head)
-//      with packed f32x2 FMAs; a reduce-scatter butterfly over the kLPT
-//      lanes of a row then leaves each lane holding the full score of one
-//      (step, head), so the exponentials, the running max and the running
-//      sum are computed once per score, not once per lane.
-//      Softmax: per head, tile max over the warp's rows, rescale factor
-//      alpha, p = 2^(s - m); scores are base 2 because q is pre-multiplied
-//      by scale*log2(e) (and by the K scale for E4M3). p and alpha go through
-//      a few bytes of shared memory to the lanes that own the V chunks.
-//      PV: fp32 accumulators, packed f32x2 FMAs.
-//  * Epilogue: merge the warps' (max, sum, accumulators) in shared memory and
-//    write bf16 output, or, for split-K, the normalised fp32 partial with its
-//    (max, sum) for the reduce kernel.
+//  * QK: each lane forms its chunk's partial dot for every (step, head) --
+//    bf16 x bf16 -> fp32 FMAs on the packed cache for bf16, fp32 FMAs after
+//    an exact E4M3 -> fp32 conversion for FP8. A reduce-scatter butterfly
+//    over the kLPT lanes of a row then leaves each lane with the full score
+//    of one (step, head); each lane holds its values in a lane-permuted order
+//    so that no round needs a select.
+//  * Softmax: base 2 (q, or the score, is multiplied by scale*log2(e), and
+//    by the K scale for E4M3); per head, the tile max over the warp's rows,
+//    rescale factor alpha and p = 2^(s - m); p goes through a few bytes of
+//    shared memory to the lanes that own the V chunks. The accumulators are
+//    rescaled only when some head's max moved.
+//  * Software pipeline: iteration j runs QK of tile j, then the shuffle /
+//    exponential chain of tile j interleaved with P * V of tile j - 1 in one
+//    branch-free block, so the chain's latency hides behind FMAs.
+//  * P * V: fp32 accumulators; packed f32x2 FMAs with (p, p) pairs for bf16.
+//  * Epilogue: merge the warps' (max, sum, accumulators) in shared memory
+//    (reusing the rings) and write bf16 output, or, for split-K, the
+//    normalised fp32 partial with its (max, sum) for the reduce kernel.
 //
 // Every wait is bounded (PKV_DEVERR_TIMEOUT), every block id and length is
-// checked before a byte is copied (PKV_DEVERR_BOUNDS), and the producer
-// waits for its own copies in flight before the block exits.
+// checked before a byte is copied (PKV_DEVERR_BOUNDS), and each warp waits
+// for its own copies in flight before the block exits.
 #pragma once
 
 #include <math_constants.h>
@@ -102,13 +111,16 @@ struct DecodeTraits {
     static constexpr int kTileBytes = kTile * kRowBytes;  // one tile of K (or of V)
     static constexpr int kStages = cclamp(PKV_DECODE_RING_BYTES / (2 * kTileBytes), 2, 8);
     static constexpr int kThreads = kNCW * 32;
-    static constexpr int kPBufFloats = 2 * kRows * G;     // per warp: p[2 tiles][row][head]
+    // per warp, two tiles of p[row][head]; bf16 cache: stored as (p, p) pairs
+    // so that P * V runs on packed f32x2 FMAs without rearranging registers
+    static constexpr int kPSlot = FP8 ? 1 : 2;
+    static constexpr int kPBufFloats = 2 * kRows * G * kPSlot;
     // shared memory layout (bytes); the merge area reuses the rings
     static constexpr int kRingBytes = kStages * kTileBytes;  // one ring (K or V)
     static constexpr int kOffV = kRingBytes;
-    static constexpr int kOffBars = 2 * kRingBytes;          // full_k[S], full_v[S]
-    static constexpr int kOffCnt = kOffBars + 2 * kStages * 8;  // done_k[S], done_v[S], issued_k, issued_v
-    static constexpr int kOffIds = kOffCnt + (2 * kStages + 2) * 4;
+    static constexpr int kOffBars = 2 * kRingBytes;          // full_k[NCW][S], full_v[NCW][S]
+    static constexpr int kOffCnt = kOffBars + 2 * kNCW * kStages * 8;  // issued K, V tiles per warp
+    static constexpr int kOffIds = kOffCnt + 2 * kNCW * 4;
     static constexpr int kOffPBuf = (kOffIds + kMaxIdsPerPartition * 4 + 15) / 16 * 16;
     static constexpr int kSmemBytes = kOffPBuf + kNCW * kPBufFloats * 4;
     static constexpr int kMergeFloats = kNCW * G * D + 3 * kNCW * G;
@@ -167,12 +179,6 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     constexpr int TILE = T::kTile;
     constexpr int STAGES = T::kStages;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *full_k = reinterpret_cast<uint64_t *>(smem + T::kOffBars);
-    uint64_t *full_v = full_k + STAGES;
-    int *done_k = reinterpret_cast<int *>(smem + T::kOffCnt);  // per stage: warps done, cumulative
-    int *done_v = done_k + STAGES;
-    int *issued_k = done_v + STAGES;  // tiles issued so far
-    int *issued_v = issued_k + 1;
     int32_t *ids = reinterpret_cast<int32_t *>(smem + T::kOffIds);
 
     const int tid = threadIdx.x;
@@ -209,12 +215,16 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     }
     for (int i = tid; i < 2 * T::kRingBytes / 16; i += T::kThreads)
         reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (tid == 0) {
+    fence_proxy_async_smem();  // the zeros, before bulk copies overwrite them
+    // Each warp runs its own pipeline over its own rows of every tile: its
+    // barriers, its slice of each stage, its own refills.
+    uint64_t *full_k = reinterpret_cast<uint64_t *>(smem + T::kOffBars) + warp * STAGES;
+    uint64_t *full_v = full_k + NCW * STAGES;
+    int *issued = reinterpret_cast<int *>(smem + T::kOffCnt) + 2 * warp;  // K, V tiles this warp issued
+    if (lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_k[s], 1);
             mbar_init(&full_v[s], 1);
-            done_k[s] = 0;
-            done_v[s] = 0;
         }
         fence_barrier_init();
     }
@@ -238,15 +248,17 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     const long long head_stride = (long long)p.block_size * T::kRowBytes;  // bytes of one (block, head) run
     const long long blk_stride = head_stride * p.num_kv_heads;
 
-    // Issue the K (or V) half of tile j into its stage: the block-table runs
-    // that make up logical tokens [start + j*TILE, ...), one bulk copy each.
-    auto issue = [&](int j, int s, bool is_v) {  // s == j % STAGES
-        const int a0 = start + j * TILE;
-        const int a1 = min(a0 + TILE, end);
-        uint8_t *dst0 = smem + (is_v ? T::kOffV : 0) + s * T::kTileBytes;
+    // Issue this warp's rows of the K (or V) half of tile j into stage s:
+    // logical tokens [start + j*TILE + warp*ROWS, ...), split at block
+    // boundaries into contiguous runs of the HND pool, one bulk copy each.
+    constexpr int ROWS_W = T::kRows;
+    auto issue = [&](int j, int s, bool is_v) {
+        const int a0 = start + j * TILE + warp * ROWS_W;
+        const int a1 = min(a0 + ROWS_W, end);
+        uint8_t *dst0 = smem + (is_v ? T::kOffV : 0) + s * T::kTileBytes + warp * ROWS_W * T::kRowBytes;
         const uint8_t *src0 = is_v ? p.v_cache : p.k_cache;
         uint64_t *bar = is_v ? &full_v[s] : &full_k[s];
-        mbar_arrive_expect_tx(bar, (uint32_t)((a1 - a0) * T::kRowBytes));
+        mbar_arrive_expect_tx(bar, (uint32_t)(max(a1 - a0, 0) * T::kRowBytes));
         for (int a = a0; a < a1;) {
             const int lb = a >> p.log2_block_size;
             const int off = a & (p.block_size - 1);
@@ -257,32 +269,24 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
             a += n;
         }
     };
-    // Count a warp as done with the K (or V) half of tile j; the last warp
-    // refills that stage with tile j + STAGES.
-    // Warp done with the K (or V) half of tile j, which sits in stage s in
-    // round r (j = r * STAGES + s). Callers __syncwarp() first, so every
+    // This warp is done with the K (or V) half of tile j (in stage s): refill
+    // the stage with tile j + STAGES. Callers __syncwarp() first, so every
     // lane's reads of the stage are done.
-    auto release = [&](int j, int s, int r, bool is_v) {
-        if (lane == 0) {
-            __threadfence_block();
-            int *cnt = is_v ? &done_v[s] : &done_k[s];
-            const int prev = atomicAdd(cnt, 1);
-            if (prev == r * NCW + NCW - 1 && j + STAGES < n_tiles) {
-                fence_proxy_async_smem();
-                issue(j + STAGES, s, is_v);
-                atomicMax(is_v ? issued_v : issued_k, j + STAGES + 1);
-            }
+    auto release = [&](int j, int s, bool is_v) {
+        if (lane == 0 && j + STAGES < n_tiles) {
+            fence_proxy_async_smem();
+            issue(j + STAGES, s, is_v);
+            issued[is_v ? 1 : 0] = j + STAGES + 1;
         }
     };
-    if (tid == 0) {
-        fence_proxy_async_smem();  // the zeroed rings, before the copies overwrite them
+    if (lane == 0) {
         const int first = min(STAGES, n_tiles);
         for (int j = 0; j < first; ++j) {
             issue(j, j, false);
             issue(j, j, true);
         }
-        *issued_k = first;
-        *issued_v = first;
+        issued[0] = first;
+        issued[1] = first;
     }
 
     // ------------------------------------------------------------ per lane
@@ -382,35 +386,57 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         const float pr = fast_exp2(sv - mref);
         l = fmaf(l, alpha, pr);
         m = m_new;
-        if (canon) pbuf[(j & 1) * ROWS * G + my_row * G + my_h] = pr;
+        if (canon) {
+            if constexpr (FP8)
+                pbuf[(j & 1) * ROWS * G + my_row * G + my_h] = pr;
+            else
+                reinterpret_cast<float2 *>(pbuf)[(j & 1) * ROWS * G + my_row * G + my_h] = make_float2(pr, pr);
+        }
     };
     // P * V of the tile in V stage sv (p buffer half pj) into the
     // accumulators; rows past the end have p = 0.
     auto pv = [&](int sv, int pj) {
         const uint8_t *vs = smem + T::kOffV + sv * T::kTileBytes + lane_off;
-        const float *pb = pbuf + pj * ROWS * G;
 #pragma unroll
         for (int st = 0; st < STEPS; ++st) {
             const int r = st * TPS + sub;
             float vf[8];
             load8<FP8>(vs + r * T::kRowBytes, vf);
-            float pr[G];
-            if constexpr (G % 4 == 0) {
+            if constexpr (FP8) {
+                // scalar FMAs (measured faster here: the E4M3 path is conversion-bound)
+                const float *pb = pbuf + pj * ROWS * G;
+                float pr[G];
+                if constexpr (G % 4 == 0) {
 #pragma unroll
-                for (int h = 0; h < G; h += 4) {
-                    const float4 t = *reinterpret_cast<const float4 *>(pb + r * G + h);
-                    pr[h] = t.x; pr[h + 1] = t.y; pr[h + 2] = t.z; pr[h + 3] = t.w;
+                    for (int h = 0; h < G; h += 4) {
+                        const float4 t = *reinterpret_cast<const float4 *>(pb + r * G + h);
+                        pr[h] = t.x; pr[h + 1] = t.y; pr[h + 2] = t.z; pr[h + 3] = t.w;
+                    }
+                } else if constexpr (G == 2) {
+                    const float2 t = *reinterpret_cast<const float2 *>(pb + r * G);
+                    pr[0] = t.x; pr[1] = t.y;
+                } else {
+                    pr[0] = pb[r];
                 }
-            } else if constexpr (G == 2) {
-                const float2 t = *reinterpret_cast<const float2 *>(pb + r * G);
-                pr[0] = t.x; pr[1] = t.y;
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[h][i] = fmaf(pr[h], vf[i], acc[h][i]);
             } else {
-                pr[0] = pb[r];
+                // packed f32x2 FMAs: (p, p) x (v_2i, v_2i+1) + (acc_2i, acc_2i+1)
+                const float2 *pb = reinterpret_cast<const float2 *>(pbuf) + pj * ROWS * G;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float2 pp = pb[r * G + h];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 a = __ffma2_rn(pp, make_float2(vf[2 * i], vf[2 * i + 1]),
+                                                    make_float2(acc[h][2 * i], acc[h][2 * i + 1]));
+                        acc[h][2 * i] = a.x;
+                        acc[h][2 * i + 1] = a.y;
+                    }
+                }
             }
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[h][i] = fmaf(pr[h], vf[i], acc[h][i]);
         }
     };
     // acc[h] *= alpha of head h (held by the lanes with my_h == h), only when
@@ -438,7 +464,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         if (ok) {
             qk(0, sc);
             __syncwarp();
-            release(0, 0, 0, false);
+            release(0, 0, false);
             softmax(0, sc, alpha);  // acc is still zero: nothing to rescale
             __syncwarp();
             if (++sk == STAGES) { sk = 0; ++rk; }
@@ -452,8 +478,8 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
             softmax(j, sc, alpha);
             pv(sv, (j - 1) & 1);
             __syncwarp();
-            release(j, sk, rk, false);
-            release(j - 1, sv, rv, true);
+            release(j, sk, false);
+            release(j - 1, sv, true);
             rescale(alpha);
             if (++sk == STAGES) { sk = 0; ++rk; }
             if (++sv == STAGES) { sv = 0; ++rv; }
@@ -461,7 +487,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         if (ok && mbar_wait(&full_v[sv], rv & 1)) {
             pv(sv, (n_tiles - 1) & 1);
             __syncwarp();
-            release(n_tiles - 1, sv, rv, true);
+            release(n_tiles - 1, sv, true);
         } else {
             ok = false;
         }
@@ -482,13 +508,12 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     }
     // Every warp is past the loop: no stage is read any more. Wait for any
     // copy still in flight (only after a timeout), then reuse the rings.
-    __syncthreads();
-    if (tid == 0) {
-        const int ik = *issued_k, iv = *issued_v;
-        for (int j = max(0, ik - STAGES); j < ik; ++j)
-            if (!mbar_wait(&full_k[j % STAGES], (j / STAGES) & 1)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
-        for (int j = max(0, iv - STAGES); j < iv; ++j)
-            if (!mbar_wait(&full_v[j % STAGES], (j / STAGES) & 1)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+    if (lane == 0) {  // copies of this warp still in flight (only after a timeout)
+        for (int h = 0; h < 2; ++h) {
+            uint64_t *bars = h ? full_v : full_k;
+            for (int j = max(0, issued[h] - STAGES); j < issued[h]; ++j)
+                if (!mbar_wait(&bars[j % STAGES], (j / STAGES) & 1)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+        }
     }
     __syncthreads();
     float *merge_acc = reinterpret_cast<float *>(smem);  // [NCW][G][D]
