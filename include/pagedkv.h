@@ -160,6 +160,36 @@ PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const
                                int max_context_len, int partition_request, void *workspace,
                                size_t workspace_bytes, void *out, int *dev_err, void *stream);
 
+/*
+ * pkv_paged_attention_decode_static_scratch: pkv_paged_attention_decode for
+ * callers that cannot allocate device memory -- for example an engine that
+ * reserves all device memory for its KV pool at start-up and forbids later
+ * allocations, or a plugin that cannot reach its host framework's device
+ * allocator through a C ABI. (The pages have no counterpart: it only changes
+ * where the split-K scratch lives.)
+ *
+ * Same arguments and result as pkv_paged_attention_decode, without
+ * workspace / workspace_bytes: the split-K partials go to a library-owned
+ * device array of PKV_STATIC_SCRATCH_BYTES (32 MiB), which every GPU that
+ * loads the library holds until the process exits. Nothing is allocated:
+ * no cudaMalloc, cudaFree or allocating library routine is called.
+ *
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. A plan that needs more scratch than the array
+ * holds returns PKV_ERR_WORKSPACE and launches nothing. All calls share the
+ * one array and it keeps the last call's contents (the kernels need no
+ * zeroed scratch): calls that overlap on the GPU -- on different streams, or
+ * from different threads -- race on it and must be serialised by the caller.
+ */
+#define PKV_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+PKV_API int pkv_paged_attention_decode_static_scratch(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+    int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+    int cache_dtype, const float *k_scale, const float *v_scale, int max_context_len,
+    int partition_request, void *out, int *dev_err, void *stream);
+
 /* Human-readable name of a pkv_status value (static storage). */
 PKV_API const char *pkv_status_string(int status);
 

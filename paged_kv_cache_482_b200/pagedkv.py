@@ -35,7 +35,7 @@ PKV_CACHE_BF16 = 0
 PKV_CACHE_FP8_E4M3 = 1
 
 EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_paged_attention_decode", "pkv_status_string",
-            "pkv_read_device_error", "pkv_version")
+            "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch")
 
 
 class PagedKVError(RuntimeError):
@@ -83,6 +83,10 @@ def load_library(path: str):
     L.pkv_read_device_error.restype = i32
     L.pkv_version.argtypes = []
     L.pkv_version.restype = i32
+    if hasattr(L, "pkv_paged_attention_decode_static_scratch"):
+        L.pkv_paged_attention_decode_static_scratch.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
+                                                                i64, f32, i32, vp, vp, i32, i32, vp, vp, vp]
+        L.pkv_paged_attention_decode_static_scratch.restype = i32
     return L
 
 
@@ -180,6 +184,44 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
                                           _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_err), _stream(stream))
     _check(st, "pkv_paged_attention_decode")
     return out
+
+
+def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, context_lens, scale, out=None,
+                                          k_scale=None, v_scale=None, max_context_len=None, partition_request=0,
+                                          dev_err=None, stream=None):
+    """``paged_attention_decode`` for callers that cannot allocate device memory.
+
+    The split-K scratch comes from a fixed array inside the library
+    (``STATIC_SCRATCH_BYTES`` per GPU, held until exit) instead of a
+    workspace; nothing is allocated by the library. Pass ``out`` to avoid the
+    one allocation this wrapper would otherwise make for the result. Calls
+    that overlap on the GPU share the array and must be serialised; the first
+    call on a device should come before any stream capture.
+    """
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise TypeError("q must be contiguous bfloat16")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or not block_tables.is_contiguous():
+        raise TypeError("block_tables and context_lens must be contiguous int32")
+    S, nq, d = q.shape
+    nblk, nkv, bs, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("shape mismatch")
+    maxb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = maxb * bs
+    if out is None:
+        out = torch.empty_like(q)
+    dt = _cache_dtype(k_cache)
+    st = lib().pkv_paged_attention_decode_static_scratch(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                                         maxb, _ptr(context_lens), S, nq, nkv, d, bs, nblk,
+                                                         float(scale), dt, _ptr(k_scale), _ptr(v_scale),
+                                                         int(max_context_len), int(partition_request), _ptr(out),
+                                                         _ptr(dev_err), _stream(stream))
+    _check(st, "pkv_paged_attention_decode_static_scratch")
+    return out
+
+
+STATIC_SCRATCH_BYTES = 32 << 20  # PKV_STATIC_SCRATCH_BYTES
 
 
 def read_device_error(dev_err, stream=None) -> int:
