@@ -251,42 +251,56 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     // Issue this warp's rows of the K (or V) half of tile j into stage s:
     // logical tokens [start + j*TILE + warp*ROWS, ...), split at block
     // boundaries into contiguous runs of the HND pool, one bulk copy each.
+    // The warp's rows start on a multiple of ROWS, so when a block holds at
+    // least ROWS tokens they are always one run.
     constexpr int ROWS_W = T::kRows;
+    const long long head_off = (long long)kvh * head_stride;
     auto issue = [&](int j, int s, bool is_v) {
         const int a0 = start + j * TILE + warp * ROWS_W;
         const int a1 = min(a0 + ROWS_W, end);
         uint8_t *dst0 = smem + (is_v ? T::kOffV : 0) + s * T::kTileBytes + warp * ROWS_W * T::kRowBytes;
-        const uint8_t *src0 = is_v ? p.v_cache : p.k_cache;
-        uint64_t *bar = is_v ? &full_v[s] : &full_k[s];
+        const uint8_t *src0 = (is_v ? p.v_cache : p.k_cache) + head_off;
+        uint64_t *bar = (is_v ? full_v : full_k) + s;
         mbar_arrive_expect_tx(bar, (uint32_t)(max(a1 - a0, 0) * T::kRowBytes));
-        for (int a = a0; a < a1;) {
-            const int lb = a >> p.log2_block_size;
-            const int off = a & (p.block_size - 1);
-            const int n = min(p.block_size - off, a1 - a);
-            const long long phys = ids[lb - first_blk];
-            const long long src = phys * blk_stride + kvh * head_stride + (long long)off * T::kRowBytes;
-            bulk_g2s(dst0 + (a - a0) * T::kRowBytes, src0 + src, (uint32_t)(n * T::kRowBytes), bar);
-            a += n;
+        if (p.block_size >= ROWS_W) {
+            if (a1 > a0) {
+                const long long phys = ids[(a0 >> p.log2_block_size) - first_blk];
+                const int off = a0 & (p.block_size - 1);
+                bulk_g2s(dst0, src0 + phys * blk_stride + (long long)off * T::kRowBytes,
+                         (uint32_t)((a1 - a0) * T::kRowBytes), bar);
+            }
+        } else {
+            for (int a = a0; a < a1;) {
+                const int lb = a >> p.log2_block_size;
+                const int off = a & (p.block_size - 1);
+                const int n = min(p.block_size - off, a1 - a);
+                const long long phys = ids[lb - first_blk];
+                bulk_g2s(dst0 + (a - a0) * T::kRowBytes, src0 + phys * blk_stride + (long long)off * T::kRowBytes,
+                         (uint32_t)(n * T::kRowBytes), bar);
+                a += n;
+            }
         }
     };
-    // This warp is done with the K (or V) half of tile j (in stage s): refill
-    // the stage with tile j + STAGES. Callers __syncwarp() first, so every
-    // lane's reads of the stage are done.
-    auto release = [&](int j, int s, bool is_v) {
-        if (lane == 0 && j + STAGES < n_tiles) {
-            fence_proxy_async_smem();
-            issue(j + STAGES, s, is_v);
-            issued[is_v ? 1 : 0] = j + STAGES + 1;
+    // This warp is done with the K half of tile jk (stage sk) and the V half
+    // of tile jv (stage sv): refill those stages with tiles jk + STAGES and
+    // jv + STAGES -- lane 0 the K stage, lane 1 the V stage, through one
+    // code path. A negative tile index means "nothing to release". Callers
+    // __syncwarp() first, so every lane's reads of the stages are done.
+    auto release = [&](int jk, int sk, int jv, int sv) {
+        if (lane < 2) {
+            const bool is_v = lane == 1;
+            const int j = is_v ? jv : jk;
+            if (j >= 0 && j + STAGES < n_tiles) {
+                fence_proxy_async_smem();
+                issue(j + STAGES, is_v ? sv : sk, is_v);
+                issued[lane] = j + STAGES + 1;
+            }
         }
     };
-    if (lane == 0) {
+    if (lane < 2) {  // lane 0 primes the K ring, lane 1 the V ring
         const int first = min(STAGES, n_tiles);
-        for (int j = 0; j < first; ++j) {
-            issue(j, j, false);
-            issue(j, j, true);
-        }
-        issued[0] = first;
-        issued[1] = first;
+        for (int j = 0; j < first; ++j) issue(j, j, lane == 1);
+        issued[lane] = first;
     }
 
     // ------------------------------------------------------------ per lane
@@ -464,7 +478,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         if (ok) {
             qk(0, sc);
             __syncwarp();
-            release(0, 0, false);
+            release(0, 0, -1, 0);
             softmax(0, sc, alpha);  // acc is still zero: nothing to rescale
             __syncwarp();
             if (++sk == STAGES) { sk = 0; ++rk; }
@@ -478,8 +492,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
             softmax(j, sc, alpha);
             pv(sv, (j - 1) & 1);
             __syncwarp();
-            release(j, sk, false);
-            release(j - 1, sv, true);
+            release(j, sk, j - 1, sv);
             rescale(alpha);
             if (++sk == STAGES) { sk = 0; ++rk; }
             if (++sv == STAGES) { sv = 0; ++rv; }
@@ -487,7 +500,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         if (ok && mbar_wait(&full_v[sv], rv & 1)) {
             pv(sv, (n_tiles - 1) & 1);
             __syncwarp();
-            release(n_tiles - 1, sv, true);
+            release(-1, 0, n_tiles - 1, sv);
         } else {
             ok = false;
         }
