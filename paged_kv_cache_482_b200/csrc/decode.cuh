@@ -23,21 +23,22 @@
 //  * Lanes: a row is spread over kLPT = head_dim/8 lanes (8 elements each:
 //    16-byte loads for bf16, 8-byte for E4M3); a warp covers kTPS rows per
 //    step and kSteps steps per tile.
-//  * QK: each lane forms its chunk's partial dot for every (step, head) --
-//    bf16 x bf16 -> fp32 FMAs on the packed cache for bf16, fp32 FMAs after
-//    an exact E4M3 -> fp32 conversion for FP8. A reduce-scatter butterfly
+//  * QK: each lane forms its chunk's partial dot for every (step, head) with
+//    mixed-precision FMAs (exact 16-bit products, fp32 sums): bf16 x bf16 on
+//    the packed cache, or f16 x f16 after the exact E4M3 -> f16x2 conversion
+//    with q in f16 (block-scaled by a power of two). A reduce-scatter butterfly
 //    over the kLPT lanes of a row then leaves each lane with the full score
 //    of one (step, head); each lane holds its values in a lane-permuted order
 //    so that no round needs a select.
-//  * Softmax: base 2 (q, or the score, is multiplied by scale*log2(e), and
-//    by the K scale for E4M3); per head, the tile max over the warp's rows,
+//  * Softmax: base 2 (the reduced score is multiplied by scale*log2(e), and
+//    for E4M3 by the K scale and q's power of two); per head, the tile max over the warp's rows,
 //    rescale factor alpha and p = 2^(s - m); p goes through a few bytes of
 //    shared memory to the lanes that own the V chunks. The accumulators are
 //    rescaled only when some head's max moved.
 //  * Software pipeline: iteration j runs QK of tile j, then the shuffle /
 //    exponential chain of tile j interleaved with P * V of tile j - 1 in one
 //    branch-free block, so the chain's latency hides behind FMAs.
-//  * P * V: fp32 accumulators; packed f32x2 FMAs with (p, p) pairs for bf16.
+//  * P * V: fp32 accumulators; packed f32x2 FMAs with (p, p) pairs.
 //  * Epilogue: merge the warps' (max, sum, accumulators) in shared memory
 //    (reusing the rings) and write bf16 output, or, for split-K, the
 //    normalised fp32 partial with its (max, sum) for the reduce kernel.
@@ -111,10 +112,9 @@ struct DecodeTraits {
     static constexpr int kTileBytes = kTile * kRowBytes;  // one tile of K (or of V)
     static constexpr int kStages = cclamp(PKV_DECODE_RING_BYTES / (2 * kTileBytes), 2, 8);
     static constexpr int kThreads = kNCW * 32;
-    // per warp, two tiles of p[row][head]; bf16 cache: stored as (p, p) pairs
-    // so that P * V runs on packed f32x2 FMAs without rearranging registers
-    static constexpr int kPSlot = FP8 ? 1 : 2;
-    static constexpr int kPBufFloats = 2 * kRows * G * kPSlot;
+    // per warp, two tiles of p[row][head], stored as (p, p) pairs so that
+    // P * V runs on packed f32x2 FMAs without rearranging registers
+    static constexpr int kPBufFloats = 2 * kRows * G * 2;
     // shared memory layout (bytes); the merge area reuses the rings
     static constexpr int kRingBytes = kStages * kTileBytes;  // one ring (K or V)
     static constexpr int kOffV = kRingBytes;
@@ -326,22 +326,40 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     // to the reduced score. E4M3 cache: q in fp32, pre-multiplied by the scale
     // and the K scale.
     uint32_t qw[G][4];
-    float qf[FP8 ? G : 1][8];
 #pragma unroll
     for (int hs = 0; hs < G; ++hs) {
         const uint4 w = __ldg(reinterpret_cast<const uint4 *>(
             p.q + ((long long)seq * p.num_q_heads + qh0 + (hs ^ my_h)) * D + chunk * 8));
         qw[hs][0] = w.x; qw[hs][1] = w.y; qw[hs][2] = w.z; qw[hs][3] = w.w;
     }
+    // Multiplier of the reduced score: scale*log2(e) (and, for E4M3, the K
+    // scale and the power of two below).
+    float score_scale = p.qk_scale_log2;
     if constexpr (FP8) {
-        const float qs = p.qk_scale_log2 * __ldg(p.k_scale + kvh);
+        // QK runs as f32 += f16 x f16 FMAs on the f16 pairs the E4M3 codes
+        // convert to exactly. q becomes f16 after a power-of-two rescale that
+        // puts this block's largest |q| just under 2^15, so every element keeps
+        // its bf16 value exactly (elements below 2^-29 of the largest one are
+        // rounded to f16's subnormal grid); the power of two is undone on the
+        // score.
+        float mx = 0.f;
+#pragma unroll
+        for (int hs = 0; hs < G; ++hs)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[hs][i])), fabsf(bf16hi(qw[hs][i]))));
+#pragma unroll
+        for (int o = 1; o < LPT; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int e = 0;
+        frexpf(mx, &e);  // mx < 2^e (e = 0 for mx = 0)
+        const int k = 15 - e;
 #pragma unroll
         for (int hs = 0; hs < G; ++hs)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                qf[hs][2 * i] = bf16lo(qw[hs][i]) * qs;
-                qf[hs][2 * i + 1] = bf16hi(qw[hs][i]) * qs;
+                const __half2 h = __floats2half2_rn(ldexpf(bf16lo(qw[hs][i]), k), ldexpf(bf16hi(qw[hs][i]), k));
+                qw[hs][i] = *reinterpret_cast<const uint32_t *>(&h);
             }
+        score_scale = ldexpf(p.qk_scale_log2 * __ldg(p.k_scale + kvh), -k);
     }
 
     float acc[G][8];
@@ -362,13 +380,16 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         for (int ps = 0; ps < STEPS; ++ps) {
             const uint8_t *row = ks + ((ps ^ my_st) * TPS + sub) * T::kRowBytes;
             if constexpr (FP8) {
-                float kf[8];
-                load8<FP8>(row, kf);
+                const uint2 w = *reinterpret_cast<const uint2 *>(row);
+                const uint32_t kw[4] = {e4m3x2_to_f16x2((uint16_t)(w.x & 0xffffu)),
+                                        e4m3x2_to_f16x2((uint16_t)(w.x >> 16)),
+                                        e4m3x2_to_f16x2((uint16_t)(w.y & 0xffffu)),
+                                        e4m3x2_to_f16x2((uint16_t)(w.y >> 16))};
 #pragma unroll
                 for (int hs = 0; hs < G; ++hs) {
-                    float a = qf[hs][0] * kf[0];
+                    float a = 0.f;
 #pragma unroll
-                    for (int i = 1; i < 8; ++i) a = fmaf(qf[hs][i], kf[i], a);
+                    for (int i = 0; i < 4; ++i) a = fma_f16x2_acc(qw[hs][i], kw[i], a);
                     sc[ps * G + hs] = a;
                 }
             } else {
@@ -388,7 +409,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     // of head my_h; returns whether any head of the warp changed its max.
     auto softmax = [&](int j, float (&sc)[T::kNV], float &alpha) {
         ReduceScatter<T::kNV, LPT / 2>::run(sc);
-        if constexpr (!FP8) sc[0] *= p.qk_scale_log2;
+        sc[0] *= score_scale;
         const int n_valid = min(TILE, end - (start + j * TILE));
         const float sv = my_row < n_valid - row0 ? sc[0] : -CUDART_INF_F;
         float tmax = sv;
@@ -400,12 +421,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         const float pr = fast_exp2(sv - mref);
         l = fmaf(l, alpha, pr);
         m = m_new;
-        if (canon) {
-            if constexpr (FP8)
-                pbuf[(j & 1) * ROWS * G + my_row * G + my_h] = pr;
-            else
-                reinterpret_cast<float2 *>(pbuf)[(j & 1) * ROWS * G + my_row * G + my_h] = make_float2(pr, pr);
-        }
+        if (canon) reinterpret_cast<float2 *>(pbuf)[(j & 1) * ROWS * G + my_row * G + my_h] = make_float2(pr, pr);
     };
     // P * V of the tile in V stage sv (p buffer half pj) into the
     // accumulators; rows past the end have p = 0.
@@ -416,39 +432,17 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
             const int r = st * TPS + sub;
             float vf[8];
             load8<FP8>(vs + r * T::kRowBytes, vf);
-            if constexpr (FP8) {
-                // scalar FMAs (measured faster here: the E4M3 path is conversion-bound)
-                const float *pb = pbuf + pj * ROWS * G;
-                float pr[G];
-                if constexpr (G % 4 == 0) {
+            // packed f32x2 FMAs: (p, p) x (v_2i, v_2i+1) + (acc_2i, acc_2i+1)
+            const float2 *pb = reinterpret_cast<const float2 *>(pbuf) + pj * ROWS * G;
 #pragma unroll
-                    for (int h = 0; h < G; h += 4) {
-                        const float4 t = *reinterpret_cast<const float4 *>(pb + r * G + h);
-                        pr[h] = t.x; pr[h + 1] = t.y; pr[h + 2] = t.z; pr[h + 3] = t.w;
-                    }
-                } else if constexpr (G == 2) {
-                    const float2 t = *reinterpret_cast<const float2 *>(pb + r * G);
-                    pr[0] = t.x; pr[1] = t.y;
-                } else {
-                    pr[0] = pb[r];
-                }
+            for (int h = 0; h < G; ++h) {
+                const float2 pp = pb[r * G + h];
 #pragma unroll
-                for (int h = 0; h < G; ++h)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[h][i] = fmaf(pr[h], vf[i], acc[h][i]);
-            } else {
-                // packed f32x2 FMAs: (p, p) x (v_2i, v_2i+1) + (acc_2i, acc_2i+1)
-                const float2 *pb = reinterpret_cast<const float2 *>(pbuf) + pj * ROWS * G;
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float2 pp = pb[r * G + h];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 a = __ffma2_rn(pp, make_float2(vf[2 * i], vf[2 * i + 1]),
-                                                    make_float2(acc[h][2 * i], acc[h][2 * i + 1]));
-                        acc[h][2 * i] = a.x;
-                        acc[h][2 * i + 1] = a.y;
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const float2 a = __ffma2_rn(pp, make_float2(vf[2 * i], vf[2 * i + 1]),
+                                                make_float2(acc[h][2 * i], acc[h][2 * i + 1]));
+                    acc[h][2 * i] = a.x;
+                    acc[h][2 * i + 1] = a.y;
                 }
             }
         }

@@ -114,6 +114,23 @@ __device__ __forceinline__ float fma_bf16x2_acc(uint32_t a, uint32_t b, float ac
     return acc;
 }
 
+// acc + lo(a)*lo(b) + hi(a)*hi(b) for f16 pairs (products exact in fp32).
+__device__ __forceinline__ float fma_f16x2_acc(uint32_t a, uint32_t b, float acc) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %0;\n\tfma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(a), "r"(b));
+    return acc;
+}
+
+// Two E4M3 codes (low byte first) -> an f16 pair (exact: every E4M3 value
+// is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+    return h2;
+}
+
 // 2^x with the hardware approximation (relative error about 2^-22; results
 // below 2^-126 flush to zero, which only drops weights that are negligible
 // against the running maximum's weight of 1).
