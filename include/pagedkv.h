@@ -136,6 +136,12 @@ PKV_API int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int
  *  block_tables       [num_seqs][max_blocks_per_seq] int32
  *  context_lens       [num_seqs] int32, each in [1, min(max_context_len,
  *                     max_blocks_per_seq * block_size)]
+ *  seq_order          optional [num_seqs] int32, a permutation of
+ *                     0..num_seqs-1: the order in which sequences are
+ *                     scheduled (NULL: 0, 1, 2, ...). Longest first shortens
+ *                     the tail of the grid; the result does not depend on
+ *                     it. An entry outside [0, num_seqs) sets
+ *                     PKV_DEVERR_BOUNDS and is skipped.
  *  max_context_len    host-known bound on context_lens (sizes split-K)
  *  partition_request  as in pkv_plan_decode
  *  workspace          device scratch of at least plan.workspace_bytes,
@@ -153,7 +159,8 @@ PKV_API int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int
  */
 PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v_cache,
                                const int32_t *block_tables, int max_blocks_per_seq,
-                               const int32_t *context_lens, int num_seqs, int num_q_heads,
+                               const int32_t *context_lens, const int32_t *seq_order,
+                               int num_seqs, int num_q_heads,
                                int num_kv_heads, int head_dim, int block_size,
                                int64_t num_blocks, float scale, int cache_dtype,
                                const float *k_scale, const float *v_scale,
@@ -185,7 +192,8 @@ PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const
 #define PKV_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 PKV_API int pkv_paged_attention_decode_static_scratch(
     const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-    int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_q_heads,
+    int max_blocks_per_seq, const int32_t *context_lens, const int32_t *seq_order,
+    int num_seqs, int num_q_heads,
     int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
     int cache_dtype, const float *k_scale, const float *v_scale, int max_context_len,
     int partition_request, void *out, int *dev_err, void *stream);

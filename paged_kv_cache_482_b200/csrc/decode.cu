@@ -83,6 +83,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.block_tables = a.block_tables;
     p.max_blocks_per_seq = a.max_blocks_per_seq;
     p.context_lens = a.context_lens;
+    p.seq_order = a.seq_order;
     p.num_seqs = a.num_seqs;
     p.num_q_heads = a.num_q_heads;
     p.num_kv_heads = a.num_kv_heads;

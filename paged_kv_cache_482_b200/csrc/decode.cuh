@@ -62,6 +62,7 @@ struct DecodeParams {
     const int32_t *block_tables;
     int max_blocks_per_seq;
     const int32_t *context_lens;
+    const int32_t *seq_order;  // may be null: natural order
     int num_seqs;
     int num_q_heads;
     int num_kv_heads;
@@ -189,7 +190,12 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     const int part = blockIdx.x % p.num_partitions;
     const int rest = blockIdx.x / p.num_partitions;
     const int kvh = rest % p.num_kv_heads;
-    const int seq = rest / p.num_kv_heads;
+    const int seq_slot = rest / p.num_kv_heads;
+    const int seq = p.seq_order ? __ldg(p.seq_order + seq_slot) : seq_slot;
+    if (seq < 0 || seq >= p.num_seqs) {  // not a permutation entry: nothing to write to
+        if (threadIdx.x == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+        return;
+    }
 
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;

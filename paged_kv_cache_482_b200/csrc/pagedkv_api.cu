@@ -138,7 +138,8 @@ int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 }
 
 int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-                               int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_q_heads,
+                               int max_blocks_per_seq, const int32_t *context_lens, const int32_t *seq_order,
+                               int num_seqs, int num_q_heads,
                                int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
                                int cache_dtype, const float *k_scale, const float *v_scale, int max_context_len,
                                int partition_request, void *workspace, size_t workspace_bytes, void *out,
@@ -167,6 +168,7 @@ int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v
     a.block_tables = block_tables;
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.context_lens = context_lens;
+    a.seq_order = seq_order;
     a.num_seqs = num_seqs;
     a.num_q_heads = num_q_heads;
     a.num_kv_heads = num_kv_heads;

@@ -58,7 +58,8 @@ extern "C" {
 
 int pkv_paged_attention_decode_static_scratch(const void *q, const void *k_cache, const void *v_cache,
                                               const int32_t *block_tables, int max_blocks_per_seq,
-                                              const int32_t *context_lens, int num_seqs, int num_q_heads,
+                                              const int32_t *context_lens, const int32_t *seq_order,
+                                              int num_seqs, int num_q_heads,
                                               int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
                                               float scale, int cache_dtype, const float *k_scale,
                                               const float *v_scale, int max_context_len, int partition_request,
@@ -71,7 +72,8 @@ int pkv_paged_attention_decode_static_scratch(const void *q, const void *k_cache
     void *scratch = nullptr;
     st = static_scratch(&scratch);
     if (st != PKV_OK) return st;
-    return pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+    return pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, seq_order,
+                                      num_seqs,
                                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                                       cache_dtype, k_scale, v_scale, max_context_len, partition_request, scratch,
                                       kStaticScratchBytes, out, dev_err, stream);

@@ -20,6 +20,7 @@ struct DecodeArgs {
     const int32_t *block_tables;
     int max_blocks_per_seq;
     const int32_t *context_lens;
+    const int32_t *seq_order;  // may be null
     int num_seqs;
     int num_q_heads;
     int num_kv_heads;

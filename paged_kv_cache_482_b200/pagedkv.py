@@ -74,8 +74,8 @@ def load_library(path: str):
     L.pkv_store_kvcache.restype = i32
     L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
     L.pkv_plan_decode.restype = i32
-    L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i64, f32, i32, vp,
-                                             vp, i32, i32, vp, sz, vp, vp, vp]
+    L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i64, f32, i32,
+                                             vp, vp, i32, i32, vp, sz, vp, vp, vp]
     L.pkv_paged_attention_decode.restype = i32
     L.pkv_status_string.argtypes = [i32]
     L.pkv_status_string.restype = c.c_char_p
@@ -84,8 +84,8 @@ def load_library(path: str):
     L.pkv_version.argtypes = []
     L.pkv_version.restype = i32
     if hasattr(L, "pkv_paged_attention_decode_static_scratch"):
-        L.pkv_paged_attention_decode_static_scratch.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
-                                                                i64, f32, i32, vp, vp, i32, i32, vp, vp, vp]
+        L.pkv_paged_attention_decode_static_scratch.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
+                                                                i32, i64, f32, i32, vp, vp, i32, i32, vp, vp, vp]
         L.pkv_paged_attention_decode_static_scratch.restype = i32
     return L
 
@@ -150,12 +150,14 @@ def plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_c
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out=None, k_scale=None,
                            v_scale=None, max_context_len=None, partition_request=0, workspace=None, dev_err=None,
-                           stream=None):
+                           stream=None, seq_order=None):
     """One decode step of paged attention; returns ``out`` ``[S, nq, d]`` bf16.
 
     ``max_context_len`` defaults to the block-table capacity (no device
     sync). A workspace is allocated with torch when the plan needs one and
-    none is given.
+    none is given. ``seq_order`` (optional int32 device permutation of the
+    sequences) sets the order in which they are scheduled; longest first
+    shortens the tail (see ``longest_first``).
     """
     if q.dtype != torch.bfloat16 or not q.is_contiguous():
         raise TypeError("q must be contiguous bfloat16")
@@ -177,8 +179,10 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     if plan["workspace_bytes"] and workspace is None:
         workspace = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if seq_order is not None and (seq_order.dtype != torch.int32 or seq_order.numel() != S):
+        raise ValueError("seq_order must be an int32 permutation of the sequences")
     st = lib().pkv_paged_attention_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), maxb,
-                                          _ptr(context_lens), S, nq, nkv, d, bs, nblk, float(scale),
+                                          _ptr(context_lens), _ptr(seq_order), S, nq, nkv, d, bs, nblk, float(scale),
                                           PKV_CACHE_FP8_E4M3 if fp8 else PKV_CACHE_BF16, _ptr(k_scale),
                                           _ptr(v_scale), int(max_context_len), int(partition_request),
                                           _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_err), _stream(stream))
@@ -188,7 +192,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
 
 def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, context_lens, scale, out=None,
                                           k_scale=None, v_scale=None, max_context_len=None, partition_request=0,
-                                          dev_err=None, stream=None):
+                                          dev_err=None, stream=None, seq_order=None):
     """``paged_attention_decode`` for callers that cannot allocate device memory.
 
     The split-K scratch comes from a fixed array inside the library
@@ -213,7 +217,8 @@ def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, con
         out = torch.empty_like(q)
     dt = _cache_dtype(k_cache)
     st = lib().pkv_paged_attention_decode_static_scratch(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-                                                         maxb, _ptr(context_lens), S, nq, nkv, d, bs, nblk,
+                                                         maxb, _ptr(context_lens), _ptr(seq_order), S, nq, nkv, d,
+                                                         bs, nblk,
                                                          float(scale), dt, _ptr(k_scale), _ptr(v_scale),
                                                          int(max_context_len), int(partition_request), _ptr(out),
                                                          _ptr(dev_err), _stream(stream))
@@ -222,6 +227,12 @@ def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, con
 
 
 STATIC_SCRATCH_BYTES = 32 << 20  # PKV_STATIC_SCRATCH_BYTES
+
+
+def longest_first(context_lens_host: torch.Tensor) -> torch.Tensor:
+    """Host helper: the order that schedules the longest sequences first
+    (stable, int32). Engines know their lengths on the host."""
+    return torch.argsort(context_lens_host.to(torch.int64), descending=True, stable=True).to(torch.int32)
 
 
 def read_device_error(dev_err, stream=None) -> int:
@@ -261,7 +272,7 @@ class DecodeStep:
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
         self._dev_inputs = None
 
-    def run(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, stream=None):
+    def run(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, stream=None, seq_order=None):
         """Device inputs -> device output (no host traffic, no sync)."""
         store_kvcache(k_new, v_new, self.k_cache, self.v_cache, slot_mapping, self.k_scale, self.v_scale,
                       self.dev_err, stream)
@@ -269,17 +280,19 @@ class DecodeStep:
                                       out=self.out, k_scale=self.k_scale, v_scale=self.v_scale,
                                       max_context_len=self.max_context_len,
                                       partition_request=self.partition_request, workspace=self.workspace,
-                                      dev_err=self.dev_err, stream=stream)
+                                      dev_err=self.dev_err, stream=stream, seq_order=seq_order)
 
     def run_host(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, out_host, stream=None):
-        """Host (pinned) inputs -> host output: H2D copies, the step, D2H copy."""
+        """Host (pinned) inputs -> host output: the longest-first order is
+        computed from the host lengths, then H2D copies, the step, D2H copy."""
+        order = longest_first(context_lens)
+        host = (q, k_new, v_new, slot_mapping, block_tables, context_lens, order)
         if self._dev_inputs is None:
             dev = self.k_cache.device
-            self._dev_inputs = [torch.empty_like(t, device=dev) for t in
-                                (q, k_new, v_new, slot_mapping, block_tables, context_lens)]
-        dq, dk, dv, ds, dbt, dcl = self._dev_inputs
-        for d_, h_ in zip(self._dev_inputs, (q, k_new, v_new, slot_mapping, block_tables, context_lens)):
+            self._dev_inputs = [torch.empty_like(t, device=dev) for t in host]
+        for d_, h_ in zip(self._dev_inputs, host):
             d_.copy_(h_, non_blocking=True)
-        o = self.run(dq, dk, dv, ds, dbt, dcl, stream)
+        dq, dk, dv, ds, dbt, dcl, dord = self._dev_inputs
+        o = self.run(dq, dk, dv, ds, dbt, dcl, stream, seq_order=dord)
         out_host.copy_(o, non_blocking=True)
         return out_host

@@ -54,7 +54,7 @@ def _decode(L, **kw):
              nblk=100, scale=0.088, dt=0, ks=None, vs=None, maxctx=2048, part=0, ws=None, wsb=0, out=0x60000,
              err=None, stream=None)
     a.update(kw)
-    return L.pkv_paged_attention_decode(a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cl"], a["S"], a["nq"],
+    return L.pkv_paged_attention_decode(a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cl"], None, a["S"], a["nq"],
                                         a["nkv"], a["d"], a["bs"], a["nblk"], a["scale"], a["dt"], a["ks"], a["vs"],
                                         a["maxctx"], a["part"], a["ws"], a["wsb"], a["out"], a["err"], a["stream"])
 

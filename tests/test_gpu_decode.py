@@ -198,3 +198,31 @@ def test_canary_never_reaches_output():
     wl = to_device(W.generate(c, 19))
     out, _, _, st = run_gpu(wl, partition_request=0)
     assert st == K.PKV_OK and bool(torch.isfinite(out.float()).all())
+
+
+def test_sequence_order_does_not_change_results():
+    """seq_order only changes the schedule: outputs are bit-identical."""
+    c = cfg(num_seqs=9, ctx_lo=1, ctx_hi=600, block_size=16)
+    wl = to_device(W.generate(c, 20))
+    kp, vp = device_pools(wl)
+    fill_history(wl, kp, vp)
+    K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new)
+    orders = [K.longest_first(wl.context_lens.cpu()).cuda(),
+              torch.randperm(c.num_seqs, generator=torch.Generator().manual_seed(3)).to(torch.int32).cuda()]
+    for split in (0, 64):
+        base = K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                        max_context_len=c.max_context, partition_request=split)
+        for o in orders:
+            err = torch.zeros(1, dtype=torch.int32, device="cuda")
+            out = K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                           max_context_len=c.max_context, partition_request=split, seq_order=o,
+                                           dev_err=err)
+            assert K.read_device_error(err) == K.PKV_OK
+            assert torch.equal(out.view(torch.int16), base.view(torch.int16))
+    # an entry outside the sequences is reported and skipped
+    bad = orders[0].clone()
+    bad[0] = c.num_seqs
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                             max_context_len=c.max_context, seq_order=bad, dev_err=err)
+    assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS

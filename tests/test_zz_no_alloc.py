@@ -69,7 +69,7 @@ def test_plan_beyond_the_array_is_refused_before_launch():
     S, nq, nkv, d, bs, max_ctx, part = 1024, 32, 8, 128, 16, 32768, 64
     p = K.plan_decode(S, nq, nkv, d, bs, max_ctx, False, part)
     assert p["workspace_bytes"] > K.STATIC_SCRATCH_BYTES
-    st = L.pkv_paged_attention_decode_static_scratch(0x10000, 0x20000, 0x30000, 0x40000, max_ctx // bs, 0x50000, S,
+    st = L.pkv_paged_attention_decode_static_scratch(0x10000, 0x20000, 0x30000, 0x40000, max_ctx // bs, 0x50000, None, S,
                                                      nq, nkv, d, bs, 100000, 0.088, 0, None, None, max_ctx, part,
                                                      0x60000, None, None)
     assert st == K.PKV_ERR_WORKSPACE
