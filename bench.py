@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--component", choices=["decode", "block_manager"], default="decode",
+                    help="block_manager: time the host block manager's per-step bookkeeping instead")
     return ap.parse_args()
 
 
@@ -340,8 +342,95 @@ def run_reference(args):
 # -------------------------------------------------------------------- ours
 
 
+def run_block_manager(args):
+    """Host time of the block manager on the workload's request mix.
+
+    Admission: every request of the workload is added with its prompt (the
+    shared prefix of ``prefix_tokens`` tokens, then its own tokens), hitting
+    the cached prefix blocks. A decode step: one token appended to every
+    sequence (the slot_mapping of store_kvcache) and the block tables and
+    context lengths of all of them (the decode inputs). Timed on the host
+    clock; the oracle's Python manager does the same on a bounded sample.
+    """
+    import numpy as np
+
+    from paged_kv_cache_482_b200.blocks import BlockManager
+
+    cfg = W.CONFIGS[args.config if args.config != "qwen3_8b" else "prefix_shared"]
+    if args.num_seqs:
+        cfg = cfg.with_(num_seqs=args.num_seqs)
+    rng = np.random.default_rng(args.seed)
+    S, bs = cfg.num_seqs, cfg.block_size
+    prefix = rng.integers(0, 150000, cfg.prefix_tokens).tolist()
+    lens = rng.integers(max(cfg.ctx_lo, 1), cfg.ctx_hi + 1, S)
+    prompts = [prefix + rng.integers(0, 150000, int(n)).tolist() for n in lens]
+    steps, warm = args.steps, args.warmup
+    max_len = max(len(p) for p in prompts) + steps + warm
+    num_blocks = S * (-(-max_len // bs)) + 16
+    ids = np.arange(S, dtype=np.int64)
+
+    def admit(m):
+        hits = 0
+        for i, p in enumerate(prompts):
+            st, cached = m.add_sequence(i, p)
+            assert st == 0
+            hits += cached
+        return hits
+
+    m = BlockManager(num_blocks, bs)
+    t0 = time.perf_counter()
+    hits = admit(m)
+    t_admit = time.perf_counter() - t0
+    tokens = rng.integers(0, 150000, (steps + warm, S)).astype(np.int32)
+    maxb = -(-max_len // bs)
+    tables = np.empty((S, maxb), np.int32)
+    lens_out = np.empty(S, np.int32)
+    slots = np.empty(S, np.int32)
+    for j in range(warm):
+        m.append_tokens(ids, tokens[j], out=slots)
+        m.block_tables(ids, maxb, tables, lens_out)
+    t0 = time.perf_counter()
+    for j in range(warm, warm + steps):
+        m.append_tokens(ids, tokens[j], out=slots)
+        m.block_tables(ids, maxb, tables, lens_out)
+    step_us = (time.perf_counter() - t0) / steps * 1e6
+    n_prompt = sum(len(p) for p in prompts)
+    line = {
+        "metric": "block manager host time per decode step (append + block tables)",
+        "value": round(step_us, 2), "unit": "us/step", "higher_is_better": False, "n_gpus": 0,
+        "steps": steps, "warmup": warm, "dtype": "int32", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {S} sequences, shared prefix {cfg.prefix_tokens} tokens + "
+                               f"[{cfg.ctx_lo}, {cfg.ctx_hi}] own tokens, block_size {bs}, pool {num_blocks} blocks"},
+        "admission": {"value": round(n_prompt / t_admit, 1), "unit": "prompt tokens/s",
+                      "cached_tokens": int(hits), "prompt_tokens": int(n_prompt)},
+    }
+    if not args.no_cpu_baseline:
+        sys.path.insert(0, ROOT)
+        from oracle.block_manager import BlockManagerOracle
+
+        o = BlockManagerOracle(num_blocks, bs)
+        t0 = time.perf_counter()
+        admit(o)
+        o_admit = time.perf_counter() - t0
+        n_o = max(1, min(steps, 20))
+        t0 = time.perf_counter()
+        for j in range(n_o):
+            for i in range(S):
+                o.append_token(i, int(tokens[j, i]))
+            for i in range(S):
+                o.block_table(i)
+        o_us = (time.perf_counter() - t0) / n_o * 1e6
+        line["cpu_baseline"] = {"value": round(o_us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+                                "sample": f"{n_o} steps of the same {S} sequences; admission of all prompts "
+                                          f"{n_prompt / o_admit:.0f} prompt tokens/s"}
+    m.close()
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.component == "block_manager":
+        return run_block_manager(args)
     if args.impl == "reference":
         return run_reference(args)
 

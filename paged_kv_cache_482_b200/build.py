@@ -1,8 +1,9 @@
 """Build libpagedkv.so in-tree with nvcc for sm_100a.
 
 ``python -m paged_kv_cache_482_b200.build`` (or ``build()``) compiles every
-``csrc/*.cu`` to an object in ``_build/`` (in parallel) and links the shared
-library next to this file. Rebuilds only when a source or header is newer
+``csrc/*.cu`` (kernels and their host layer) and ``csrc/*.cpp`` (host-only
+code: the block manager) to an object in ``_build/`` (in parallel) and links
+the shared library next to this file. Rebuilds only when a source or header is newer
 than the library. No fast-math: the FP8 store must round exactly as the
 conversion intrinsic specifies, and divisions must be IEEE.
 """
@@ -36,7 +37,7 @@ def nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():
@@ -63,7 +64,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=(), lib: str =
         flags = flags + ["-Xptxas", "-v"]
 
     def compile_one(src):
-        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src).replace(".", "_") + ".o")
         cmd = [cc, *ARCH, *flags, *inc, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
