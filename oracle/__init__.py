@@ -56,6 +56,11 @@ def _bind(lib):
         + [c.c_void_p] * 3 + [c.c_int]
     )
     lib.orc_paged_attention_decode.restype = c.c_int
+    lib.orc_paged_attention_prefill.argtypes = (
+        [c.c_void_p] * 4 + [c.c_int, c.c_void_p, c.c_void_p] + [c.c_int] * 6 + [c.c_int64, c.c_float, c.c_int]
+        + [c.c_void_p] * 3 + [c.c_int]
+    )
+    lib.orc_paged_attention_prefill.restype = c.c_int
     return lib
 
 
@@ -138,6 +143,33 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_
     return out, st
 
 
+def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, num_kv_heads, block_size,
+                            scale, k_scale=None, v_scale=None, num_threads=1, lib=None):
+    """fp64 causal attention of each sequence's chunk of query tokens over its
+    paged K/V (the chunk is the last ``c`` of its ``context_lens`` positions).
+
+    ``q`` is ``[total_q, nq, d]`` bf16, ``cu_q_lens`` ``[S + 1]``. Returns
+    ``(out [total_q, nq, d] float64, status)``.
+    """
+    lib = lib or load()
+    q = _np(q, np.uint16)
+    bt = _np(block_tables, np.int32)
+    cu = _np(cu_q_lens, np.int32)
+    cl = _np(context_lens, np.int32)
+    T, nq, d = q.shape
+    S = cl.shape[0]
+    assert cu.shape == (S + 1,)
+    fp8 = k_cache.dtype == np.uint8
+    ks = _np(k_scale, np.float32) if fp8 else None
+    vs = _np(v_scale, np.float32) if fp8 else None
+    out = np.zeros((T, nq, d), dtype=np.float64)
+    nblk = k_cache.shape[0]
+    st = lib.orc_paged_attention_prefill(_p(q), _p(k_cache), _p(v_cache), _p(bt), bt.shape[1], _p(cu), _p(cl), S,
+                                         T, nq, num_kv_heads, d, block_size, nblk, float(scale), int(fp8), _p(ks),
+                                         _p(vs), _p(out), int(num_threads))
+    return out, st
+
+
 def e4m3_from_float(y: float, lib=None) -> int:
     return (lib or load()).orc_e4m3_from_float(float(y))
 
@@ -177,4 +209,24 @@ def run_workload(wl, num_threads=1, seq_ids=None, lib=None):
     out, st3 = paged_attention_decode(sub["q"], kp, vp, sub["block_tables"], sub["context_lens"],
                                       cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, wl.k_scale,
                                       wl.v_scale, num_threads=num_threads, lib=lib)
+    return out, kp, vp, st1 | st2 | st3
+
+
+def run_prefill_workload(wl, num_threads=1, lib=None):
+    """Fill host pools from a prefill workload's history, store its chunk
+    tokens, then attend. Returns ``(out [T, nq, d], k_pool, v_pool, status)``."""
+    from paged_kv_cache_482_b200 import workloads as W
+
+    cfg = wl.cfg
+    fp8 = wl.is_fp8
+    fill = W.CANARY_FP8 if fp8 else W.CANARY_BF16
+    kp = new_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, cfg.head_dim, fp8, fill)
+    vp = new_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, cfg.head_dim, fp8, fill)
+    st1 = store_kvcache(wl.k_hist, wl.v_hist, kp, vp, wl.slot_hist, wl.num_blocks, cfg.block_size, wl.k_scale,
+                        wl.v_scale, lib=lib)
+    st2 = store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.num_blocks, cfg.block_size, wl.k_scale,
+                        wl.v_scale, lib=lib)
+    out, st3 = paged_attention_prefill(wl.q, kp, vp, wl.block_tables, wl.cu_q_lens, wl.context_lens,
+                                       cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, wl.k_scale, wl.v_scale,
+                                       num_threads=num_threads, lib=lib)
     return out, kp, vp, st1 | st2 | st3

@@ -1,5 +1,6 @@
 /*
- * pkv_oracle.c -- plain, slow, fp64 CPU oracle for one paged decode step.
+ * pkv_oracle.c -- plain, slow, fp64 CPU oracle for paged attention: one
+ * decode step, and a chunk of prefill tokens attending causally.
  *
  * TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's
  * CPU-baseline leg are the only callers. It shares no code, header, table or
@@ -31,6 +32,13 @@
  *    nearest E4M3 value, ties to the even code, magnitudes beyond 448 clamped
  *    to 448 (NaN stays NaN);
  *  - FP8 read: code value times the head's scale, both exact in fp64.
+ *  - Chunked prefill ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目",
+ *    section 核心技术改进 2 "Chunked Prefill": a long prompt's prefill is cut
+ *    into chunks that run interleaved with decode work): a chunk of c new
+ *    tokens of a sequence whose K/V are already stored occupies the last c of
+ *    its context_len positions, and each of them attends causally -- to
+ *    itself and every earlier token of its sequence. A decode step is the
+ *    case c = 1.
  *
  * Every function here is pinned by a CPU test (brute force against a
  * library softmax, invariants, closed forms, the OCP format points and a
@@ -251,6 +259,109 @@ int orc_paged_attention_decode(const uint16_t *q, const void *k_cache, const voi
             }
             for (i = 0; i < head_dim; ++i)
                 out_s[(int64_t)h * head_dim + i] = acc[i] / z;
+        }
+        free(score);
+        free(w);
+        free(acc);
+    }
+    return status;
+}
+
+/*
+ * paged_attention_prefill: sequence s has c_s = cu_q_lens[s + 1] -
+ * cu_q_lens[s] query tokens, rows cu_q_lens[s] .. cu_q_lens[s + 1] - 1 of q
+ * ([total_q][num_q_heads][head_dim] bf16), and context_lens[s] tokens in the
+ * cache including those c_s. Query token i of the chunk sits at position
+ * p = context_lens[s] - c_s + i and attends over positions 0 .. p:
+ * out = softmax(scale * q K[0..p]^T) V[0..p], in fp64, written to the same
+ * row of out. A sequence with c_s = 0 has no rows. A sequence whose chunk is
+ * longer than its context, whose context does not fit its table row, or
+ * whose table names a block outside the pool gets zero rows and the call
+ * reports ORC_ERR_BOUNDS. cu_q_lens must start at 0, never decrease, and end
+ * at total_q (else ORC_ERR_ARG).
+ */
+int orc_paged_attention_prefill(const uint16_t *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *cu_q_lens, const int32_t *context_lens, int num_seqs,
+                                int total_q, int num_q_heads, int num_kv_heads, int head_dim,
+                                int block_size, int64_t num_blocks, float scale, int fp8,
+                                const float *k_scale, const float *v_scale, double *out,
+                                int num_threads)
+{
+    int status = ORC_OK;
+    int group, s;
+    if (!q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens || !out ||
+        num_seqs < 0 || total_q < 0 || num_q_heads < 1 || num_kv_heads < 1 ||
+        num_q_heads % num_kv_heads || head_dim < 1 || block_size < 1 || num_blocks < 1 ||
+        max_blocks_per_seq < 1 || (fp8 && (!k_scale || !v_scale)))
+        return ORC_ERR_ARG;
+    if (cu_q_lens[0] != 0 || cu_q_lens[num_seqs] != total_q)
+        return ORC_ERR_ARG;
+    for (s = 0; s < num_seqs; ++s)
+        if (cu_q_lens[s + 1] < cu_q_lens[s])
+            return ORC_ERR_ARG;
+    group = num_q_heads / num_kv_heads;
+    if (num_threads < 1)
+        num_threads = 1;
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads) reduction(| : status)
+    for (s = 0; s < num_seqs; ++s) {
+        const int32_t *table = block_tables + (int64_t)s * max_blocks_per_seq;
+        int c = cu_q_lens[s + 1] - cu_q_lens[s];
+        int ctx = context_lens[s];
+        int bad, h, t, i, r;
+        double *score, *w, *acc;
+        if (c == 0)
+            continue;
+        bad = (ctx < c || ctx > max_blocks_per_seq * block_size);
+        for (t = 0; !bad && t < ctx; t += block_size)
+            bad = (table[t / block_size] < 0 || table[t / block_size] >= num_blocks);
+        if (bad) {
+            memset(out + (int64_t)cu_q_lens[s] * num_q_heads * head_dim, 0,
+                   sizeof(double) * (size_t)c * num_q_heads * head_dim);
+            status |= ORC_ERR_BOUNDS;
+            continue;
+        }
+        score = (double *)malloc(sizeof(double) * (size_t)ctx);
+        w = (double *)malloc(sizeof(double) * (size_t)ctx);
+        acc = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        for (r = 0; r < c; ++r) {
+            int64_t row = cu_q_lens[s] + r;
+            int p = ctx - c + r; /* this query token's position */
+            for (h = 0; h < num_q_heads; ++h) {
+                int g = h / group;
+                const uint16_t *q_h = q + (row * num_q_heads + h) * head_dim;
+                double *out_h = out + (row * num_q_heads + h) * head_dim;
+                double m = -INFINITY, z = 0.0;
+                for (t = 0; t <= p; ++t) {
+                    int64_t blk = table[t / block_size];
+                    int off = t % block_size;
+                    double dot = 0.0;
+                    for (i = 0; i < head_dim; ++i) {
+                        int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
+                        dot += orc_bf16_to_double(q_h[i]) * cache_value(k_cache, idx, fp8, k_scale, g);
+                    }
+                    score[t] = (double)scale * dot;
+                    if (score[t] > m)
+                        m = score[t];
+                }
+                for (t = 0; t <= p; ++t) {
+                    w[t] = exp(score[t] - m);
+                    z += w[t];
+                }
+                for (i = 0; i < head_dim; ++i)
+                    acc[i] = 0.0;
+                for (t = 0; t <= p; ++t) {
+                    int64_t blk = table[t / block_size];
+                    int off = t % block_size;
+                    for (i = 0; i < head_dim; ++i) {
+                        int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
+                        acc[i] += w[t] * cache_value(v_cache, idx, fp8, v_scale, g);
+                    }
+                }
+                for (i = 0; i < head_dim; ++i)
+                    out_h[i] = acc[i] / z;
+            }
         }
         free(score);
         free(w);

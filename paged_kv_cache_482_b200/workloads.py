@@ -292,3 +292,185 @@ def logical_kv(wl: Workload, i: int):
         k = torch.cat([k, wl.k_new[i : i + 1]])
         v = torch.cat([v, wl.v_new[i : i + 1]])
     return k[:ctx], v[:ctx]
+
+
+# ---------------------------------------------------------------- prefill
+#
+# Chunked prefill ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section
+# 核心技术改进 2 "Chunked Prefill"): a long prompt is prefilled in chunks that
+# are scheduled together with decode requests. A sequence's step brings a
+# chunk of c new tokens on top of the h tokens it already has in the cache;
+# its context is h + c and the chunk is the last c positions. A decode
+# request in the same batch is the case c = 1.
+
+
+@dataclass(frozen=True)
+class PrefillConfig:
+    """Shape of one chunked-prefill step: per sequence a cached history of
+    ``hist_lo..hist_hi`` tokens and a chunk of ``chunk_lo..chunk_hi`` new
+    tokens (uniform, inclusive). ``decode_seqs`` more sequences join the same
+    batch with one new token each (history ``decode_hist_lo..decode_hist_hi``)."""
+
+    name: str
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    hist_lo: int
+    hist_hi: int
+    chunk_lo: int
+    chunk_hi: int
+    cache_dtype: str = CACHE_BF16
+    decode_seqs: int = 0
+    decode_hist_lo: int = 0
+    decode_hist_hi: int = 0
+    pool_blocks: int | None = None
+    scale: float | None = None
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.head_dim)
+
+    @property
+    def total_seqs(self) -> int:
+        return self.num_seqs + self.decode_seqs
+
+    @property
+    def max_context(self) -> int:
+        return max(self.hist_hi + self.chunk_hi, self.decode_hist_hi + 1)
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return -(-self.max_context // self.block_size)
+
+    def with_(self, **kw) -> "PrefillConfig":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return PrefillConfig(**d)
+
+
+PREFILL_CONFIGS: dict[str, PrefillConfig] = {
+    c.name: c
+    for c in (
+        PrefillConfig("prefill_tiny", 3, 4, 2, 64, 16, 0, 40, 1, 70, pool_blocks=64, scale=1.0 / 8.0),
+        # Qwen3-8B-shaped layer, 16 prompts each advancing by a 512-token chunk
+        PrefillConfig("prefill_qwen3_8b", 16, 32, 8, 128, 256, 0, 3584, 512, 512),
+        # the same chunks scheduled together with 240 decode requests
+        PrefillConfig("prefill_mixed", 4, 32, 8, 128, 256, 0, 3584, 512, 512, decode_seqs=240,
+                      decode_hist_lo=100, decode_hist_hi=2047),
+        PrefillConfig("prefill_fp8", 8, 32, 8, 128, 16, 1024, 8192, 256, 1024, cache_dtype=CACHE_FP8),
+    )
+}
+
+
+@dataclass
+class PrefillWorkload:
+    """All inputs of one chunked-prefill step plus the history that fills the pool.
+
+    Rows of ``q``/``k_new``/``v_new``/``slot_new`` are the chunk tokens of all
+    sequences back to back (sequence i owns rows ``cu_q_lens[i]`` to
+    ``cu_q_lens[i+1] - 1``). ``k_hist``/``v_hist``/``slot_hist`` are the cached
+    tokens before the chunks; ``hist_rows[i]`` lists sequence i's history rows
+    in logical order.
+    """
+
+    cfg: PrefillConfig
+    seed: int
+    num_blocks: int
+    q: torch.Tensor  # [T, nq, d] bf16
+    k_new: torch.Tensor  # [T, nkv, d] bf16
+    v_new: torch.Tensor
+    slot_new: torch.Tensor  # [T] int32
+    k_hist: torch.Tensor  # [H, nkv, d] bf16
+    v_hist: torch.Tensor
+    slot_hist: torch.Tensor  # [H] int32
+    block_tables: torch.Tensor  # [S, max_blocks] int32, -1 padded
+    cu_q_lens: torch.Tensor  # [S + 1] int32
+    context_lens: torch.Tensor  # [S] int32
+    hist_rows: list = field(default_factory=list)
+    k_scale: torch.Tensor | None = None
+    v_scale: torch.Tensor | None = None
+
+    @property
+    def is_fp8(self) -> bool:
+        return self.cfg.cache_dtype == CACHE_FP8
+
+    @property
+    def total_q(self) -> int:
+        return int(self.q.shape[0])
+
+
+def generate_prefill(cfg: PrefillConfig, seed: int = 0, device: str | torch.device = "cpu") -> PrefillWorkload:
+    """Draw one chunked-prefill step's inputs for ``cfg`` (structure from a CPU
+    generator seeded with ``seed``, data from a ``device`` generator seeded
+    with ``seed + 1``, as in :func:`generate`)."""
+    device = torch.device(device)
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    S, bs, nkv, d = cfg.total_seqs, cfg.block_size, cfg.num_kv_heads, cfg.head_dim
+    P, D = cfg.num_seqs, cfg.decode_seqs
+    hist = torch.cat([torch.randint(cfg.hist_lo, cfg.hist_hi + 1, (P,), generator=g, dtype=torch.int64),
+                      torch.randint(cfg.decode_hist_lo, cfg.decode_hist_hi + 1, (D,), generator=g,
+                                    dtype=torch.int64)])
+    chunk = torch.cat([torch.randint(cfg.chunk_lo, cfg.chunk_hi + 1, (P,), generator=g, dtype=torch.int64),
+                       torch.ones(D, dtype=torch.int64)])
+    ctx = hist + chunk
+    nb = [-(-int(c) // bs) for c in ctx]
+    in_use = sum(nb)
+    nblk = cfg.pool_blocks if cfg.pool_blocks is not None else in_use + -(-in_use // 10)
+    if nblk < in_use:
+        raise ValueError(f"pool of {nblk} blocks cannot hold {in_use}")
+    perm = torch.randperm(nblk, generator=g, dtype=torch.int64)
+    tables = torch.full((S, cfg.max_blocks_per_seq), -1, dtype=torch.int64)
+    nxt = 0
+    for i in range(S):
+        tables[i, : nb[i]] = perm[nxt : nxt + nb[i]]
+        nxt += nb[i]
+    cu = torch.zeros(S + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(chunk, 0)
+    H = int(hist.sum())
+    hist_start = torch.zeros(S + 1, dtype=torch.int64)
+    hist_start[1:] = torch.cumsum(hist, 0)
+    seq_h = torch.repeat_interleave(torch.arange(S), hist)
+    pos_h = torch.arange(H) - hist_start[seq_h]
+    slot_hist = tables[seq_h, pos_h // bs] * bs + pos_h % bs
+    T = int(cu[-1])
+    seq_q = torch.repeat_interleave(torch.arange(S), chunk)
+    pos_q = hist[seq_q] + torch.arange(T) - cu[seq_q]
+    slot_new = tables[seq_q, pos_q // bs] * bs + pos_q % bs
+    hist_rows = [torch.arange(int(hist_start[i]), int(hist_start[i + 1])) for i in range(S)]
+
+    gd = torch.Generator(device=device).manual_seed(seed + 1)
+    q = _randn_bf16((T, cfg.num_q_heads, d), gd, device)
+    k_hist = _randn_bf16((H, nkv, d), gd, device)
+    v_hist = _randn_bf16((H, nkv, d), gd, device)
+    k_new = _randn_bf16((T, nkv, d), gd, device)
+    v_new = _randn_bf16((T, nkv, d), gd, device)
+    wl = PrefillWorkload(
+        cfg=cfg, seed=seed, num_blocks=nblk, q=q, k_new=k_new, v_new=v_new,
+        slot_new=slot_new.to(torch.int32).to(device), k_hist=k_hist, v_hist=v_hist,
+        slot_hist=slot_hist.to(torch.int32).to(device), block_tables=tables.to(torch.int32).to(device),
+        cu_q_lens=cu.to(torch.int32).to(device), context_lens=ctx.to(torch.int32).to(device), hist_rows=hist_rows,
+    )
+    if cfg.cache_dtype == CACHE_FP8:
+        # per KV head: absolute maximum over every stored token / 448
+        kmax = torch.cat([k_hist, k_new]).abs().amax(dim=(0, 2)).float()
+        vmax = torch.cat([v_hist, v_new]).abs().amax(dim=(0, 2)).float()
+        one = torch.ones_like(kmax)
+        wl.k_scale = torch.where(kmax > 0, kmax, one) / 448.0
+        wl.v_scale = torch.where(vmax > 0, vmax, one) / 448.0
+    elif cfg.cache_dtype != CACHE_BF16:
+        raise ValueError(cfg.cache_dtype)
+    return wl
+
+
+def prefill_logical_kv(wl: PrefillWorkload, i: int):
+    """Sequence i's K and V rows ``[ctx, nkv, d]`` in logical order, from the
+    drawn rows (history, then its chunk), not from any pool."""
+    rows = wl.hist_rows[i].to(wl.k_hist.device)
+    a, b = int(wl.cu_q_lens[i]), int(wl.cu_q_lens[i + 1])
+    return torch.cat([wl.k_hist[rows], wl.k_new[a:b]]), torch.cat([wl.v_hist[rows], wl.v_new[a:b]])

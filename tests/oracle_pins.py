@@ -348,7 +348,173 @@ def pin_bounds_errors(lib):
         assert np.array_equal(out3[0], out[0]) and np.array_equal(out3[2], out[2])
 
 
+# ------------------------------------------------------------------ prefill
+
+
+def pcfg(**kw) -> W.PrefillConfig:
+    base = dict(name="ppin", num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=16, block_size=4, hist_lo=0,
+                hist_hi=13, chunk_lo=1, chunk_hi=9)
+    base.update(kw)
+    return W.PrefillConfig(**base)
+
+
+def _run_prefill(wl, lib):
+    out, kp, vp, st = O.run_prefill_workload(wl, lib=lib)
+    assert st == O.ORC_OK, f"oracle status {st}"
+    return out, kp, vp
+
+
+def prefill_brute_force(wl: W.PrefillWorkload, i: int) -> np.ndarray:
+    """Causal softmax attention of sequence i's chunk from its logical K/V rows
+    (no pool): query token j of a chunk of c sits at position ctx - c + j."""
+    c = wl.cfg
+    K, V = W.prefill_logical_kv(wl, i)
+    if wl.is_fp8:
+        K, V = dequant(K, wl.k_scale), dequant(V, wl.v_scale)
+    K = np.repeat(K.double().numpy(), c.group, axis=1)  # [ctx, nq, d]
+    V = np.repeat(V.double().numpy(), c.group, axis=1)
+    a, b = int(wl.cu_q_lens[i]), int(wl.cu_q_lens[i + 1])
+    q = wl.q[a:b].double().numpy()  # [c, nq, d]
+    ctx, n = K.shape[0], b - a
+    scale = np.float64(np.float32(c.softmax_scale))
+    s = np.einsum("jhd,thd->hjt", q, K) * scale
+    pos = ctx - n + np.arange(n)
+    s = np.where(np.arange(ctx)[None, None, :] <= pos[None, :, None], s, -np.inf)
+    p = scipy.special.softmax(s, axis=2)
+    return np.einsum("hjt,thd->jhd", p, V)
+
+
+def pin_prefill_bruteforce(lib):
+    for c, seed in [
+        (pcfg(), 21),
+        (pcfg(num_q_heads=8, num_kv_heads=1, head_dim=8, block_size=8, hist_hi=30, chunk_lo=5, chunk_hi=20), 22),
+        (pcfg(num_q_heads=3, num_kv_heads=3, head_dim=12, block_size=16, hist_lo=15, hist_hi=33), 23),
+        (pcfg(cache_dtype=W.CACHE_FP8, chunk_hi=12), 24),
+        (pcfg(num_seqs=2, decode_seqs=3, decode_hist_lo=1, decode_hist_hi=20), 25),
+    ]:
+        wl = W.generate_prefill(c, seed)
+        out, _, _ = _run_prefill(wl, lib)
+        for i in range(c.total_seqs):
+            a, b = int(wl.cu_q_lens[i]), int(wl.cu_q_lens[i + 1])
+            _assert_close(out[a:b], prefill_brute_force(wl, i), what=f"prefill seq {i} {c}")
+
+
+def pin_prefill_one_token_is_decode(lib):
+    """A chunk of one token is a decode step: the decode oracle's result (the
+    decode function is pinned on its own above)."""
+    c = pcfg(num_seqs=0, decode_seqs=5, decode_hist_lo=0, decode_hist_hi=21)
+    for fp8 in (False, True):
+        wl = W.generate_prefill(c.with_(cache_dtype=W.CACHE_FP8 if fp8 else W.CACHE_BF16), 26)
+        out, kp, vp = _run_prefill(wl, lib)
+        dec, st = O.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.num_kv_heads,
+                                           c.block_size, c.softmax_scale, wl.k_scale, wl.v_scale, lib=lib)
+        assert st == O.ORC_OK
+        assert np.array_equal(out, dec), "a one-token chunk differs from decode"
+
+
+def pin_prefill_chunking_invariance(lib):
+    """A prompt prefilled as one chunk or as two consecutive chunks gives every
+    token the same output (each token's result depends on its prefix only)."""
+    c = pcfg(num_seqs=3, hist_lo=0, hist_hi=9, chunk_lo=6, chunk_hi=14)
+    wl = W.generate_prefill(c, 27)
+    out, kp, vp = _run_prefill(wl, lib)
+    cu, cl = wl.cu_q_lens.long(), wl.context_lens.long()
+    n = cu[1:] - cu[:-1]
+    first = n // 2  # first chunk: the leading half of each sequence's chunk
+    rows1 = torch.cat([torch.arange(int(cu[i]), int(cu[i] + first[i])) for i in range(c.total_seqs)])
+    rows2 = torch.cat([torch.arange(int(cu[i] + first[i]), int(cu[i + 1])) for i in range(c.total_seqs)])
+    cu1 = torch.cat([torch.zeros(1, dtype=torch.int64), torch.cumsum(first, 0)]).to(torch.int32)
+    cu2 = torch.cat([torch.zeros(1, dtype=torch.int64), torch.cumsum(n - first, 0)]).to(torch.int32)
+    o1, st1 = O.paged_attention_prefill(wl.q[rows1], kp, vp, wl.block_tables, cu1, (cl - (n - first)).to(torch.int32),
+                                        c.num_kv_heads, c.block_size, c.softmax_scale, lib=lib)
+    o2, st2 = O.paged_attention_prefill(wl.q[rows2], kp, vp, wl.block_tables, cu2, wl.context_lens,
+                                        c.num_kv_heads, c.block_size, c.softmax_scale, lib=lib)
+    assert st1 == O.ORC_OK and st2 == O.ORC_OK
+    assert np.array_equal(out[rows1.numpy()], o1) and np.array_equal(out[rows2.numpy()], o2), "chunking changed a result"
+
+
+def pin_prefill_causal_mask(lib):
+    """A key that dominates every score takes over exactly the queries at or
+    after its position and leaves the earlier ones unchanged."""
+    c = pcfg(num_seqs=2, num_q_heads=2, num_kv_heads=1, head_dim=16, block_size=4, hist_lo=3, hist_hi=3,
+             chunk_lo=9, chunk_hi=9)
+    for p in (3, 4, 7, 8, 11):  # positions inside the chunk (positions 3 .. 11)
+        wl = W.generate_prefill(c, 28)
+        wl.q[:] = 1.0
+        base, _, _ = _run_prefill(wl, lib)
+        for i in range(c.total_seqs):
+            a = int(wl.cu_q_lens[i])
+            wl.k_new[a + p - 3] = 32.0  # chunk row of position p
+        out, _, _ = _run_prefill(wl, lib)
+        for i in range(c.total_seqs):
+            a = int(wl.cu_q_lens[i])
+            _, V = W.prefill_logical_kv(wl, i)
+            for j in range(9):
+                pos = 3 + j
+                if pos < p:
+                    assert np.array_equal(out[a + j], base[a + j]), f"query {pos} saw the key at {p}"
+                else:
+                    expect = np.repeat(V[p].double().numpy()[None], c.group, axis=0)[:, 0]
+                    _assert_close(out[a + j], expect, what=f"query {pos}, dominant key {p}")
+
+
+def pin_prefill_relabel_invariance(lib):
+    c = pcfg(hist_hi=20)
+    wl = W.generate_prefill(c, 29)
+    out, _, _ = _run_prefill(wl, lib)
+    perm = torch.randperm(wl.num_blocks, generator=torch.Generator().manual_seed(3))
+    bs = c.block_size
+    w2 = copy.copy(wl)
+    bt = wl.block_tables.long()
+    w2.block_tables = torch.where(bt >= 0, perm[bt.clamp(min=0)], bt).to(torch.int32)
+    w2.slot_hist = (perm[wl.slot_hist.long() // bs] * bs + wl.slot_hist.long() % bs).to(torch.int32)
+    w2.slot_new = (perm[wl.slot_new.long() // bs] * bs + wl.slot_new.long() % bs).to(torch.int32)
+    out2, _, _ = _run_prefill(w2, lib)
+    assert np.array_equal(out, out2), "block relabelling changed the prefill result"
+
+
+def pin_prefill_errors(lib):
+    c = pcfg(hist_lo=4, hist_hi=12)
+    wl = W.generate_prefill(c, 30)
+    out, kp, vp = _run_prefill(wl, lib)
+    cu, T = wl.cu_q_lens, wl.total_q
+
+    def call(bt=None, cu_=None, cl=None):
+        return O.paged_attention_prefill(wl.q, kp, vp, wl.block_tables if bt is None else bt,
+                                         cu if cu_ is None else cu_, wl.context_lens if cl is None else cl,
+                                         c.num_kv_heads, c.block_size, c.softmax_scale, lib=lib)
+
+    rows1 = slice(int(cu[1]), int(cu[2]))
+    others = np.r_[0:int(cu[1]), int(cu[2]):T]
+    bt = wl.block_tables.clone()
+    bt[1, 0] = wl.num_blocks
+    o, st = call(bt=bt)
+    assert st == O.ORC_ERR_BOUNDS and np.all(o[rows1] == 0) and np.array_equal(o[others], out[others])
+    cl = wl.context_lens.clone()
+    cl[1] = int(cu[2] - cu[1]) - 1  # a chunk longer than its context
+    o, st = call(cl=cl)
+    assert st == O.ORC_ERR_BOUNDS and np.all(o[rows1] == 0) and np.array_equal(o[others], out[others])
+    full = wl.block_tables.clone()
+    full[1, :] = full[1, 0]
+    cl = wl.context_lens.clone()
+    cl[1] = c.max_blocks_per_seq * c.block_size + 1
+    o, st = call(bt=full, cl=cl)
+    assert st == O.ORC_ERR_BOUNDS and np.all(o[rows1] == 0)
+    bad = cu.clone()
+    bad[1] = int(cu[2]) + 1  # decreasing from entry 1 to entry 2
+    assert call(cu_=bad)[1] == O.ORC_ERR_ARG
+    bad = cu.clone()
+    bad[-1] -= 1  # does not end at total_q
+    assert call(cu_=bad)[1] == O.ORC_ERR_ARG
+
+
 ALL_PINS = [
+    pin_prefill_bruteforce,
+    pin_prefill_one_token_is_decode,
+    pin_prefill_chunking_invariance,
+    pin_prefill_causal_mask,
+    pin_prefill_relabel_invariance,
+    pin_prefill_errors,
     pin_bruteforce_bf16,
     pin_bruteforce_fp8,
     pin_permutation_invariance,

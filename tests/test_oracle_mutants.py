@@ -46,6 +46,20 @@ MUTANTS = [
     ("bf16 widening", "(uint32_t)bits << 16;", "(uint32_t)bits << 15;", 0),
     ("bounds check off by one", "ctx > max_blocks_per_seq * block_size", "ctx > max_blocks_per_seq * block_size + 1", 0),
     ("block id check", "table[t / block_size] >= num_blocks", "table[t / block_size] > num_blocks", 0),
+    # chunked prefill
+    ("prefill gqa interleaved", "int g = h / group;", "int g = h % num_kv_heads;", 1),
+    ("prefill sees one future token", "int p = ctx - c + r;", "int p = ctx - c + r + 1;", 0),
+    ("prefill ignores the history", "int p = ctx - c + r;", "int p = r;", 0),
+    ("prefill mask excludes itself", "for (t = 0; t <= p; ++t) {\n                    w[t]",
+     "for (t = 0; t < p; ++t) {\n                    w[t]", 0),
+    ("prefill q row without offset", "q + (row * num_q_heads + h) * head_dim", "q + ((int64_t)r * num_q_heads + h) * head_dim", 0),
+    ("prefill out row without offset", "out + (row * num_q_heads + h) * head_dim", "out + ((int64_t)r * num_q_heads + h) * head_dim", 0),
+    ("prefill chunk longer than context", "bad = (ctx < c || ctx > max_blocks_per_seq * block_size);",
+     "bad = (ctx > max_blocks_per_seq * block_size);", 0),
+    ("prefill decreasing offsets accepted", "if (cu_q_lens[s + 1] < cu_q_lens[s])", "if (0)", 0),
+    ("prefill max not subtracted", "w[t] = exp(score[t] - m);", "w[t] = exp(score[t]);", 1),
+    ("prefill not normalised", "acc[i] / z;", "acc[i];", 1),
+    ("prefill v read from k", "cache_value(v_cache, idx, fp8, v_scale, g)", "cache_value(k_cache, idx, fp8, v_scale, g)", 1),
 ]
 
 

@@ -84,3 +84,28 @@ def test_logical_kv_orders_rows():
         assert torch.equal(k[:8], wl.k_hist[:8])
         if n > 8:
             assert torch.equal(k[-1], wl.k_new[i])
+
+
+@pytest.mark.parametrize("name", ["prefill_tiny", "prefill_qwen3_8b", "prefill_mixed"])
+def test_prefill_bookkeeping(name):
+    c = W.PREFILL_CONFIGS[name]
+    wl = W.generate_prefill(c, 8) if name == "prefill_tiny" else None
+    if wl is None:  # full size: structure only, no K/V drawn on the CPU
+        wl = W.generate_prefill(c.with_(head_dim=8, num_q_heads=2, num_kv_heads=1), 8)
+    S, bs = c.total_seqs, c.block_size
+    cu, ctx = wl.cu_q_lens.long(), wl.context_lens.long()
+    n = cu[1:] - cu[:-1]
+    assert int(cu[0]) == 0 and int(cu[-1]) == wl.total_q and (n >= 1).all()
+    assert (n[: c.num_seqs] >= c.chunk_lo).all() and (n[: c.num_seqs] <= c.chunk_hi).all()
+    assert (n[c.num_seqs :] == 1).all()
+    written = torch.cat([wl.slot_hist, wl.slot_new]).tolist()
+    assert len(set(written)) == len(written) and min(written) >= 0 and max(written) < wl.num_blocks * bs
+    for i in range(S):
+        nb = -(-int(ctx[i]) // bs)
+        row = wl.block_tables[i].tolist()
+        assert all(b >= 0 for b in row[:nb]) and all(b == -1 for b in row[nb:])
+        h = int(ctx[i] - n[i])
+        assert len(wl.hist_rows[i]) == h
+        for p in range(int(ctx[i])):  # every logical position's slot follows the table
+            sl = int(wl.slot_hist[wl.hist_rows[i][p]]) if p < h else int(wl.slot_new[int(cu[i]) + p - h])
+            assert sl == row[p // bs] * bs + p % bs
