@@ -51,7 +51,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="qwen3_8b", choices=sorted(W.CONFIGS))
+    ap.add_argument("--config", default="qwen3_8b", choices=sorted(W.CONFIGS) + sorted(W.PREFILL_CONFIGS),
+                    help="a decode workload, or a chunked-prefill one (prefill_*)")
     ap.add_argument("--partition", type=int, default=0, help="0 auto, -1 never split, >0 tokens per partition")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--num-seqs", type=int, default=0, help="override the workload's sequence count")
@@ -427,10 +428,269 @@ def run_block_manager(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ prefill
+
+
+def prefill_desc(cfg: W.PrefillConfig) -> str:
+    mix = f" + {cfg.decode_seqs} decode requests" if cfg.decode_seqs else ""
+    return (f"{cfg.name} chunked-prefill layer: {cfg.num_seqs} seqs x chunk U[{cfg.chunk_lo},{cfg.chunk_hi}] after "
+            f"history U[{cfg.hist_lo},{cfg.hist_hi}]{mix}, {cfg.num_q_heads}q/{cfg.num_kv_heads}kv heads, head_dim "
+            f"{cfg.head_dim}, block_size {cfg.block_size}, {cfg.cache_dtype} cache")
+
+
+def prefill_flops(wl) -> int:
+    """Causal attention FLOPs of one prefill launch: every (query token, head)
+    row takes 2 d FLOPs per key for QK and 2 d per key for PV, over the
+    p + 1 keys at or before its position p."""
+    c = wl.cfg
+    cu, ctx = wl.cu_q_lens.cpu().long(), wl.context_lens.cpu().long()
+    n = cu[1:] - cu[:-1]
+    keys = int((n * (ctx - n) + n * (n + 1) // 2).sum())
+    return keys * c.num_q_heads * 4 * c.head_dim
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), float(d["bf16_tflops"]), "measured"
+    except Exception:  # noqa: BLE001
+        return 1400.0, 1590.0, "fallback"
+
+
+def prefill_oracle_sampler(wl, threads: int):
+    """Host pools of the whole step (untimed) and a function that runs the
+    oracle on the given (sequence, chunk row) pairs, each as a one-token
+    chunk at its position (its result depends on the tokens up to it only)."""
+    import oracle as O
+
+    c = wl.cfg
+    fill = W.CANARY_FP8 if wl.is_fp8 else W.CANARY_BF16
+    kp = O.new_pool(wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim, wl.is_fp8, fill)
+    vp = O.new_pool(wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim, wl.is_fp8, fill)
+    ks = wl.k_scale.cpu() if wl.k_scale is not None else None
+    vs = wl.v_scale.cpu() if wl.v_scale is not None else None
+    O.store_kvcache(wl.k_hist.cpu(), wl.v_hist.cpu(), kp, vp, wl.slot_hist.cpu(), wl.num_blocks, c.block_size, ks, vs)
+    O.store_kvcache(wl.k_new.cpu(), wl.v_new.cpu(), kp, vp, wl.slot_new.cpu(), wl.num_blocks, c.block_size, ks, vs)
+    q, bt = wl.q.cpu(), wl.block_tables.cpu()
+    cu, cl = wl.cu_q_lens.cpu().long(), wl.context_lens.cpu().long()
+
+    def run(pairs):
+        rows = torch.tensor([int(cu[s]) + j for s, j in pairs])
+        ctx = torch.tensor([int(cl[s] - (cu[s + 1] - cu[s]) + j + 1) for s, j in pairs], dtype=torch.int32)
+        seqs = torch.tensor([s for s, _ in pairs])
+        out, st = O.paged_attention_prefill(q[rows], kp, vp, bt[seqs], torch.arange(len(pairs) + 1, dtype=torch.int32),
+                                            ctx, c.num_kv_heads, c.block_size, c.softmax_scale, ks, vs,
+                                            num_threads=threads)
+        return st
+
+    return run
+
+
+def prefill_sample_pairs(wl, n, seed):
+    """n (sequence, chunk row) pairs drawn uniformly from the step's rows."""
+    cu = wl.cu_q_lens.cpu().long()
+    rows = torch.randperm(wl.total_q, generator=torch.Generator().manual_seed(seed))[:n]
+    seq = torch.searchsorted(cu, rows, right=True) - 1
+    return [(int(s), int(r - cu[s])) for s, r in zip(seq, rows)]
+
+
+def prefill_cpu_baseline(wl, target_s: float) -> dict:
+    threads = cpu_threads()
+    run = prefill_oracle_sampler(wl, threads)
+    n = max(threads, 8)
+    t0 = time.perf_counter()
+    run(prefill_sample_pairs(wl, n, 1))
+    dt = time.perf_counter() - t0
+    n2 = int(min(wl.total_q, max(n, n * target_s / max(dt, 1e-6))))
+    t0 = time.perf_counter()
+    st = run(prefill_sample_pairs(wl, n2, 2))
+    dt = time.perf_counter() - t0
+    return {"value": n2 / dt, "unit": "query tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n2} of {wl.total_q} query tokens of the same step, drawn uniformly, each as a one-token "
+                      f"chunk at its position; fp64, {dt:.2f} s, OpenMP over tokens; status {st}"}
+
+
+def run_prefill_reference(args):
+    if rank_env()[1] != 0:
+        return 0
+    cfg = W.PREFILL_CONFIGS[args.config]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = W.generate_prefill(cfg, args.seed, device=dev)
+    threads = cpu_threads()
+    run = prefill_oracle_sampler(wl, threads)
+    n0 = max(threads, 8)
+    t0 = time.perf_counter()
+    run(prefill_sample_pairs(wl, n0, 1))
+    per_row = (time.perf_counter() - t0) / n0
+    n = int(min(wl.total_q, max(1, 120.0 / max(1, args.steps + args.warmup) / max(per_row, 1e-9))))
+    for i in range(args.warmup):
+        run(prefill_sample_pairs(wl, n, 10 + i))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        run(prefill_sample_pairs(wl, n, 100 + i))
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    unit = "query tokens/s"
+    print(json.dumps({
+        "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": prefill_desc(cfg), "sample_rows_per_step": n},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} of {wl.total_q} query tokens per step, each as a one-token chunk"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+PREFILL_METRIC = "chunked-prefill paged attention query tokens/sec and achieved tensor TFLOP/s"
+
+
+def run_prefill(args):
+    from paged_kv_cache_482_b200 import pagedkv as K
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    cfg = W.PREFILL_CONFIGS[args.config]
+    wl = W.generate_prefill(cfg, args.seed + rank, device="cuda")
+    c = cfg
+    shape = (wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)
+    if wl.is_fp8:
+        kp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device="cuda")
+        vp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device="cuda")
+    else:
+        kp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+        vp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.store_kvcache(wl.k_hist, wl.v_hist, kp, vp, wl.slot_hist, wl.k_scale, wl.v_scale, err)
+    cu = wl.cu_q_lens.cpu().long()
+    mq = int((cu[1:] - cu[:-1]).max())
+    out = torch.empty_like(wl.q)
+
+    def step(q, k_new, v_new, slot_new, bt, cu_d, cl):
+        K.store_kvcache(k_new, v_new, kp, vp, slot_new, wl.k_scale, wl.v_scale, err)
+        K.paged_attention_prefill(q, kp, vp, bt, cu_d, cl, c.softmax_scale, mq, out=out, k_scale=wl.k_scale,
+                                  v_scale=wl.v_scale, dev_err=err)
+
+    inputs = (wl.q, wl.k_new, wl.v_new, wl.slot_new, wl.block_tables, wl.cu_q_lens, wl.context_lens)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        step(*inputs)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())} during warm-up")
+
+    sampler = ClockSampler(nvsmi_ids(local)) if local == 0 else None
+    if sampler:
+        sampler.wait_first()
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kst)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    e_start.record(stream)
+    for k in range(Kst):
+        ev[k][0].record(stream)
+        K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, err)
+        ev[k][1].record(stream)
+        K.paged_attention_prefill(wl.q, kp, vp, wl.block_tables, wl.cu_q_lens, wl.context_lens, c.softmax_scale, mq,
+                                  out=out, k_scale=wl.k_scale, v_scale=wl.v_scale, dev_err=err)
+        ev[k][2].record(stream)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    elapsed_ms = e_start.elapsed_time(e_end)
+    attn_ms = statistics.mean(ev[k][1].elapsed_time(ev[k][2]) for k in range(Kst))
+    store_ms = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(Kst))
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
+    if sampler:
+        sampler.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())} in the timed steps")
+
+    # end to end: pinned host inputs -> device -> store + prefill -> host output, every step
+    host_in = [t.cpu().pin_memory() for t in inputs]
+    dev_in = [torch.empty_like(t) for t in inputs]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        step(*dev_in)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = x0.elapsed_time(x1)
+    elapsed_ms, attn_ms, e2e_ms = max_over_ranks([elapsed_ms, attn_ms, e2e_ms], dist, device="cuda")
+
+    if rank == 0:
+        flops = prefill_flops(wl)
+        peak_sus, peak_burst, kind = measured_tensor_peak()
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        T = wl.total_q
+        line = {
+            "metric": PREFILL_METRIC, "value": world * T * Kst / (elapsed_ms * 1e-3), "unit": "query tokens/s",
+            "n_gpus": world, "steps": Kst, "warmup": args.warmup, "ms_per_step": elapsed_ms / Kst,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 x bf16 -> fp32 (tcgen05)" + (", e4m3 cache" if wl.is_fp8 else ""), "data": "synthetic",
+            "config": {"workload": prefill_desc(c), "query_tokens": T, "kv_tokens": int(wl.context_lens.sum()),
+                       "max_q_len": mq, "seed": args.seed,
+                       "parallelism": f"replicas x{world} (independent batches, no collective)",
+                       "l2": "no flush: each step's pools and queries exceed 126 MB of L2"},
+            "attention_us": attn_ms * 1e3, "store_us": store_ms * 1e3,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
+                         "frac": achieved / peak_sus, "traffic": None, "kernel": "paged_prefill_kernel",
+                         "peak_source": f"{kind} cuBLAS bf16 GEMM, sustained (bf16_tflops_sustained); "
+                                        f"burst {peak_burst}",
+                         "algorithmic_flops_per_launch": flops,
+                         "flops_note": "causal: 4 * head_dim FLOPs per (query row, head, key at or before it)"},
+            "e2e": {"value": world * T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "query tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+            "gpu_launches": 2 * Kst,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = prefill_cpu_baseline(wl, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.component == "block_manager":
         return run_block_manager(args)
+    if args.config in W.PREFILL_CONFIGS:
+        return run_prefill_reference(args) if args.impl == "reference" else run_prefill(args)
     if args.impl == "reference":
         return run_reference(args)
 

@@ -91,7 +91,8 @@ typedef enum {
  *  k_scale, ...  [num_kv_heads] fp32, FP8 only (NULL for bf16)
  *
  * Host checks: non-null pointers, 16-byte aligned k/v/caches, head_dim a
- * multiple of 8, sizes >= 1 (num_tokens may be 0: nothing is launched).
+ * multiple of 8, sizes >= 1 (num_tokens may be 0: nothing is launched and no
+ * pointer is looked at).
  * Device check: slot >= num_blocks * block_size sets PKV_DEVERR_BOUNDS and
  * the token is not written.
  */
@@ -197,6 +198,47 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
     int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
     int cache_dtype, const float *k_scale, const float *v_scale, int max_context_len,
     int partition_request, void *out, int *dev_err, void *stream);
+
+/*
+ * pkv_paged_attention_prefill: chunked prefill over the paged cache
+ * ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section 核心技术改进 2
+ * "Chunked Prefill": a long prompt's prefill runs in chunks scheduled
+ * together with decode requests). Sequence i brings a chunk of
+ * c_i = cu_q_lens[i + 1] - cu_q_lens[i] query tokens (rows cu_q_lens[i] ..
+ * cu_q_lens[i + 1] - 1 of q) whose K/V pkv_store_kvcache has already written
+ * as the last c_i of its context_lens[i] positions. Token j of the chunk sits
+ * at position p = context_lens[i] - c_i + j and attends causally:
+ *   out[row][h][:] = sum_{t <= p} softmax_t(scale * q[row][h] . K_t) V_t
+ * (KV head h / group). A chunk of one token is a decode step, so one call
+ * can serve a batch mixing prefill chunks and decode requests; c_i = 0 is
+ * allowed (no rows). QK^T and PV run on the tensor cores with bf16 operands
+ * and fp32 accumulation (the E4M3 cache is widened to bf16 exactly); the
+ * softmax weights are rounded to bf16 for PV and the normaliser sums those
+ * rounded weights; out is rounded to bf16.
+ *
+ *  q             [total_q][num_q_heads][head_dim] bf16, contiguous
+ *  block_tables  [num_seqs][max_blocks_per_seq] int32
+ *  cu_q_lens     [num_seqs + 1] int32: 0, then running sums of the c_i
+ *  context_lens  [num_seqs] int32, c_i <= context_lens[i] <=
+ *                max_blocks_per_seq * block_size
+ *  max_q_len     host-known bound on every c_i (sizes the grid)
+ *  out           [total_q][num_q_heads][head_dim] bf16
+ *
+ * Host checks: pointers non-null, q / caches / out 16-byte aligned,
+ * head_dim 64 or 128, group 1, 2, 4 or 8, block_size a power of two in
+ * [8, 1024], max_q_len >= 1 (when total_q > 0). Device checks: cu_q_lens not
+ * starting at or above 0, decreasing or past total_q, a chunk longer than
+ * its context or than max_q_len, a context beyond the table row, or a block
+ * id outside [0, num_blocks) set PKV_DEVERR_BOUNDS; the sequence's rows are
+ * written as zeros where they can be located. The library allocates nothing.
+ */
+PKV_API int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *v_cache,
+                                        const int32_t *block_tables, int max_blocks_per_seq,
+                                        const int32_t *cu_q_lens, const int32_t *context_lens, int num_seqs,
+                                        int total_q, int num_q_heads, int num_kv_heads, int head_dim,
+                                        int block_size, int64_t num_blocks, float scale, int cache_dtype,
+                                        const float *k_scale, const float *v_scale, int max_q_len, void *out,
+                                        int *dev_err, void *stream);
 
 /* Human-readable name of a pkv_status value (static storage). */
 PKV_API const char *pkv_status_string(int status);

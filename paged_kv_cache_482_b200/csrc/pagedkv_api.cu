@@ -120,10 +120,10 @@ int pkv_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache
         return PKV_ERR_INVALID_ARG;
     if (cache_dtype != PKV_CACHE_BF16 && cache_dtype != PKV_CACHE_FP8_E4M3) return PKV_ERR_INVALID_ARG;
     const bool fp8 = cache_dtype == PKV_CACHE_FP8_E4M3;
+    if (num_tokens == 0) return PKV_OK;  // no rows to read: k, v, slot_mapping may be NULL
     if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
     if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
-    if (num_tokens == 0) return PKV_OK;
     cudaError_t e = pkv::launch_store_kvcache(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
                                               head_dim, block_size, num_blocks, fp8, k_scale, v_scale, dev_err,
                                               num_sms(), static_cast<cudaStream_t>(stream));
@@ -193,6 +193,54 @@ int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v
     a.out = out;
     a.dev_err = dev_err;
     cudaError_t e = pkv::launch_decode(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_tables, int max_blocks_per_seq, const int32_t *cu_q_lens,
+                                const int32_t *context_lens, int num_seqs, int total_q, int num_q_heads,
+                                int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
+                                int cache_dtype, const float *k_scale, const float *v_scale, int max_q_len, void *out,
+                                int *dev_err, void *stream) {
+    if (num_seqs < 0 || total_q < 0 || num_q_heads < 1 || num_kv_heads < 1) return PKV_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (cache_dtype != PKV_CACHE_BF16 && cache_dtype != PKV_CACHE_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (!pow2(block_size) || block_size < 8 || block_size > 1024) return PKV_ERR_INVALID_ARG;
+    if (!pkv::prefill_supported(head_dim, num_q_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
+    const bool fp8 = cache_dtype == PKV_CACHE_FP8_E4M3;
+    if (!q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens || !out)
+        return PKV_ERR_INVALID_ARG;
+    if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+    if (max_blocks_per_seq < 1 || num_blocks < 1 || num_blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;  // NaN
+    if (num_seqs == 0 || total_q == 0) return PKV_OK;
+    if (max_q_len < 1) return PKV_ERR_INVALID_ARG;
+
+    pkv::PrefillArgs a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.cu_q_lens = cu_q_lens;
+    a.context_lens = context_lens;
+    a.num_seqs = num_seqs;
+    a.total_q = total_q;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_dim = head_dim;
+    a.block_size = block_size;
+    a.num_blocks = num_blocks;
+    a.scale = scale;
+    a.fp8 = fp8;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.max_q_len = max_q_len;
+    a.out = out;
+    a.dev_err = dev_err;
+    cudaError_t e = pkv::launch_prefill(a, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidConfiguration) return PKV_ERR_UNSUPPORTED;
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

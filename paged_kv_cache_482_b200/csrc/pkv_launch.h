@@ -48,4 +48,32 @@ int decode_max_blocks_per_partition();
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
+// Everything the chunked-prefill kernel needs, resolved by the host layer.
+struct PrefillArgs {
+    const void *q;  // [total_q][num_q_heads][head_dim] bf16
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_tables;
+    int max_blocks_per_seq;
+    const int32_t *cu_q_lens;     // [num_seqs + 1]
+    const int32_t *context_lens;  // [num_seqs]
+    int num_seqs;
+    int total_q;
+    int num_q_heads;
+    int num_kv_heads;
+    int head_dim;
+    int block_size;
+    int64_t num_blocks;
+    float scale;
+    bool fp8;
+    const float *k_scale;
+    const float *v_scale;
+    int max_q_len;
+    void *out;
+    int *dev_err;
+};
+
+bool prefill_supported(int head_dim, int group);
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream);
+
 }  // namespace pkv

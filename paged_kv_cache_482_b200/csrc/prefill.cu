@@ -1,0 +1,526 @@
+// prefill.cu -- chunked-prefill paged attention on the 5th-generation tensor
+// cores (sm_100a): tcgen05.mma with operands in shared memory and fp32
+// accumulators in tensor memory.
+//
+// The operation ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section
+// 核心技术改进 2 "Chunked Prefill"; the paged cache of "DeepSeek复刻vLLM反超原版",
+// section "vLLM：大模型推理的加速引擎与挑战"): sequence s brings a chunk of
+// c = cu_q_lens[s+1] - cu_q_lens[s] query tokens whose K/V are already in the
+// cache as the last c of its context_lens[s] positions; token i of the chunk
+// (position p = ctx - c + i) attends over positions 0..p. A decode request is
+// the case c = 1, so one launch serves a batch that mixes both.
+//
+// Work unit: one CTA per (sequence, KV head, 128 query rows). A row is a
+// (chunk token, query head of the group) pair: row r = token r / G, head
+// r % G, so the G heads that share a KV head share every K/V tile. The CTA
+// walks the sequence's KV in tiles of 128 logical tokens up to its last
+// row's position:
+//   1. K/V tiles are gathered through the block table with 16-byte cp.async
+//      copies (zero-filled past the causal end) into shared memory, double
+//      buffered, in the 128-byte-swizzled layout the tensor core reads;
+//   2. one thread issues S = Q K^T (M 128, N 128, K head_dim) into tensor
+//      memory;
+//   3. the four warps each read their 32 tensor-memory lanes (one row per
+//      thread), apply the causal mask, update the running max / sum in the
+//      exp2 domain and write P = exp2(s - m) as bf16 into shared memory;
+//   4. one thread issues O_tile = P V (M 128, N head_dim, K 128; V read
+//      MN-major straight from its row layout) into a second tensor-memory
+//      buffer, which the threads fold into fp32 register accumulators with
+//      the rescale factor.
+// The FP8 cache is dequantised to bf16 while it is staged (both MMA operands
+// are bf16); k_scale folds into the softmax scale and v_scale into the final
+// normalisation.
+//
+// Shared-memory operand layout (all four operands): [head_dim / 64 or
+// 128 / 64 column blocks][rows][128 bytes], the 16-byte chunk c of row r
+// stored at chunk c ^ (r % 8) -- the canonical 128-byte swizzle, so one
+// descriptor form serves Q, K and P (K-major) and V (MN-major).
+#include "pkv_common.cuh"
+#include "pkv_launch.h"
+
+namespace pkv {
+namespace {
+
+constexpr int kRows = 128;  // MMA M: query rows per CTA
+constexpr int kBN = 64;     // KV tokens per tile
+constexpr int kThreads = 128;
+constexpr uint32_t kTmemCols = 256;  // S: 64 columns, O: up to 128 columns (two CTAs fill an SM's 512)
+constexpr uint32_t kMinSmem = 100u * 1024u;  // at most two CTAs per SM, whatever head_dim
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Layout {
+    static constexpr int kHalves = D / 64;
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kQBytes = kHalves * kRows * 128;
+    static constexpr uint32_t kTileBytes = kHalves * kBN * 128;
+    static constexpr uint32_t kK0 = kQ + kQBytes;
+    static constexpr uint32_t kV0 = kK0 + kTileBytes;
+    static constexpr uint32_t kBufStride = 2 * kTileBytes;  // K1 = K0 + stride, V1 = V0 + stride
+    // P (kRows x kBN bf16) overwrites the K tile it was computed from when it
+    // fits (head_dim 128): S has consumed that tile by the time P is written.
+    // Otherwise P has a buffer of its own, free once the previous P V is done.
+    static constexpr uint32_t kPBytes = (kBN / 64) * kRows * 128;
+    static constexpr bool kPInK = kPBytes <= kTileBytes;
+    static constexpr uint32_t kP = kK0 + 2 * kBufStride;
+    static constexpr uint32_t kBar = kP + (kPInK ? 0 : kPBytes);  // 2 mbarriers, TMEM address
+    static constexpr uint32_t kBytes = kBar + 64;
+    static constexpr uint32_t kAlloc = (kBytes + 1024 > kMinSmem) ? kBytes + 1024 : kMinSmem;  // + base alignment
+};
+
+// ------------------------------------------------------------ tcgen05 PTX
+
+// Shared-memory matrix descriptor (sm_100 form): start address, leading and
+// stride byte offsets (all >> 4), descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, A
+// K-major, B K-major or MN-major, M x N.
+constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t holder_saddr, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder_saddr),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on *bar once every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 consecutive fp32 columns into this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared16(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Eight E4M3 codes -> eight bf16 values (exact: every E4M3 value is a bf16 value).
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 w) {
+    uint4 o;
+    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w.x & 0xFFFFu));
+    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w.x >> 16));
+    float2 c = e4m3x2_to_float2(static_cast<uint16_t>(w.y & 0xFFFFu));
+    float2 d = e4m3x2_to_float2(static_cast<uint16_t>(w.y >> 16));
+    o.x = pack_bf16(a.x, a.y);
+    o.y = pack_bf16(b.x, b.y);
+    o.z = pack_bf16(c.x, c.y);
+    o.w = pack_bf16(d.x, d.y);
+    return o;
+}
+
+// Byte offset of 16-byte chunk c16 of row r in a swizzled operand of `rows` rows.
+__device__ __forceinline__ uint32_t swz(int rows, int r, int c16) {
+    return static_cast<uint32_t>((c16 >> 3) * rows * 128 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));
+}
+
+// Stage KV tile j (logical tokens j*kBN ..) of KV head kh into one K/V buffer.
+// Tokens at or past kv_end are zero-filled; their scores are masked anyway
+// and zeros keep P V finite.
+template <int D, bool FP8>
+__device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const int32_t *table, int kh, int j, int kv_end,
+                                             uint32_t sk, uint32_t sv) {
+    constexpr int kChunks = D / 8;             // 16-byte chunks per bf16 row
+    constexpr int kTokPerPass = kThreads / kChunks;
+    const int c16 = threadIdx.x % kChunks;
+    const int t_first = threadIdx.x / kChunks;
+    const int bs = a.block_size;
+#pragma unroll 4
+    for (int t = t_first; t < kBN; t += kTokPerPass) {
+        const int pos = j * kBN + t;
+        const bool valid = pos < kv_end;
+        const int p = valid ? pos : 0;
+        const int64_t blk = table[p / bs];
+        const int64_t elem = ((blk * a.num_kv_heads + kh) * bs + (p % bs)) * D + c16 * 8;
+        const uint32_t off = swz(kBN, t, c16);
+        if constexpr (FP8) {
+            uint2 kw = make_uint2(0, 0), vw = make_uint2(0, 0);
+            if (valid) {
+                kw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(a.k_cache) + elem));
+                vw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(a.v_cache) + elem));
+            }
+            st_shared16(sk + off, e4m3x8_to_bf16x8(kw));
+            st_shared16(sv + off, e4m3x8_to_bf16x8(vw));
+        } else {
+            const __nv_bfloat16 *kc = static_cast<const __nv_bfloat16 *>(a.k_cache);
+            const __nv_bfloat16 *vc = static_cast<const __nv_bfloat16 *>(a.v_cache);
+            cp_async16(sk + off, kc + elem, valid ? 16u : 0u);
+            cp_async16(sv + off, vc + elem, valid ? 16u : 0u);
+        }
+    }
+}
+
+template <int D, int G, bool FP8>
+__global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs a, int tiles_per_seq) {
+    using L = Layout<D>;
+    constexpr int TQ = kRows / G;  // chunk tokens per CTA
+    constexpr uint32_t kIdescS = idesc_bf16(kRows, kBN, false);
+    constexpr uint32_t kIdescPV = idesc_bf16(kRows, D, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *sm = smem_raw + (base - raw);
+    uint64_t *bar_s = reinterpret_cast<uint64_t *>(sm + L::kBar);
+    uint64_t *bar_pv = bar_s + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bar_s + 2);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int s = blockIdx.x / tiles_per_seq;
+    const int tile = tiles_per_seq - 1 - (blockIdx.x % tiles_per_seq);  // longest causal range first
+    const int kh = blockIdx.y;
+    const int nq = a.num_q_heads;
+
+    // ------------------------------------------------ bounds and bookkeeping
+    const int q0 = a.cu_q_lens[s];
+    const int q1 = a.cu_q_lens[s + 1];
+    if (q0 < 0 || q1 < q0 || q1 > a.total_q) {
+        if (tid == 0 && tile == 0 && kh == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
+        return;  // no row of this sequence can be located safely
+    }
+    const int c = q1 - q0;
+    const int t0 = tile * TQ;
+    if (t0 >= c) return;
+    const int ctx = a.context_lens[s];
+    const int32_t *table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+    bool bad = ctx < c || static_cast<int64_t>(ctx) > static_cast<int64_t>(a.max_blocks_per_seq) * a.block_size ||
+               c > a.max_q_len;
+    if (!bad) {
+        const int nblk_seq = (ctx + a.block_size - 1) / a.block_size;
+        for (int i = tid; i < nblk_seq; i += kThreads) {
+            const int32_t b = table[i];
+            if (b < 0 || b >= a.num_blocks) bad = true;
+        }
+    }
+    const int row_tok = t0 + tid / G;  // this thread's row
+    const int row_head = kh * G + tid % G;
+    const bool row_live = row_tok < c;
+    __nv_bfloat16 *out_row =
+        static_cast<__nv_bfloat16 *>(a.out) + (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + row_head) * D;
+    if (__syncthreads_or(bad)) {
+        if (row_live) {
+            for (int i = 0; i < D; i += 8) *reinterpret_cast<uint4 *>(out_row + i) = make_uint4(0, 0, 0, 0);
+        }
+        if (tid == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
+        return;
+    }
+    const int last_tok = min(t0 + TQ, c) - 1;
+    const int p_first = ctx - c + t0;  // position of the CTA's first row
+    const int p_last = ctx - c + last_tok;
+    const int kv_end = p_last + 1;
+    const int n_tiles = (kv_end + kBN - 1) / kBN;
+    const int row_pos = row_live ? ctx - c + row_tok : p_last;
+
+    // ------------------------------------------------ setup: TMEM, barriers
+    if (warp == 0) tmem_alloc(smem_addr(tmem_holder), kTmemCols);
+    if (tid == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_pv, 1);
+        fence_barrier_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t tmem_s = tmem;        // S: columns 0..kBN - 1
+    const uint32_t tmem_o = tmem + 128;  // O: columns 128..128 + D - 1
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+
+    const uint32_t sq = base + L::kQ;
+
+    // Q rows (zero past the chunk) and KV tile 0
+    {
+        constexpr int kChunks = D / 8;
+        const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q);
+        for (int i = tid; i < kRows * kChunks; i += kThreads) {
+            const int r = i / kChunks, c16 = i % kChunks;
+            const int tok = t0 + r / G;
+            const bool valid = tok < c;
+            const int64_t elem = (static_cast<int64_t>(q0 + (valid ? tok : 0)) * nq + kh * G + r % G) * D + c16 * 8;
+            cp_async16(sq + swz(kRows, r, c16), qp + elem, valid ? 16u : 0u);
+        }
+    }
+    load_kv_tile<D, FP8>(a, table, kh, 0, kv_end, base + L::kK0, base + L::kV0);
+    cp_async_commit();
+
+    const float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool timed_out = false;
+    uint64_t *pending = nullptr;  // the barrier a timed-out wait was on
+    uint32_t pending_parity = 0;
+
+    for (int j = 0; j < n_tiles; ++j) {
+        const uint32_t buf = static_cast<uint32_t>(j & 1) * L::kBufStride;
+        const uint32_t sk = base + L::kK0 + buf;
+        const uint32_t sv = base + L::kV0 + buf;
+        const uint32_t sp = L::kPInK ? sk : base + L::kP;
+        cp_async_wait0();  // this tile's copies (and Q) have landed
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // S = Q K^T (queued behind P V of the previous tile)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRows * 128 + (kk & 3) * 32);
+                const uint32_t boff = static_cast<uint32_t>((kk >> 2) * kBN * 128 + (kk & 3) * 32);
+                mma_bf16(tmem_s, sw128_desc(sq + aoff, 16, 1024), sw128_desc(sk + boff, 16, 1024), kIdescS,
+                         kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_s);
+        }
+        const bool ok_s = mbar_wait(bar_s, static_cast<uint32_t>(j & 1));
+        if (__syncthreads_or(!ok_s)) {
+            timed_out = true;
+            pending = bar_s;
+            pending_parity = static_cast<uint32_t>(j & 1);
+            break;
+        }
+        tc_fence_after();
+
+        // this row's scores (exp2 domain, causal mask) and their maximum
+        const int kv0 = j * kBN;
+        const bool masked = kv0 + kBN - 1 > p_first;  // some row sees a future or absent token
+        float x[kBN];
+#pragma unroll
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+            float v[32];
+            tmem_ld32(tmem_s + lane_base + ch * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[ch * 32 + i] = v[i] * sl2;
+        }
+        if (masked) {
+#pragma unroll
+            for (int i = 0; i < kBN; ++i)
+                if (kv0 + i > row_pos) x[i] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, x[i]);
+
+        // P V of the previous tile has finished: P, O and the other buffer are free
+        if (j > 0) {
+            const bool ok_pv = mbar_wait(bar_pv, static_cast<uint32_t>((j - 1) & 1));
+            if (__syncthreads_or(!ok_pv)) {
+                timed_out = true;
+                pending = bar_pv;
+                pending_parity = static_cast<uint32_t>((j - 1) & 1);
+                break;
+            }
+            tc_fence_after();
+        }
+        if (j + 1 < n_tiles) {
+            const uint32_t nbuf = static_cast<uint32_t>((j + 1) & 1) * L::kBufStride;
+            load_kv_tile<D, FP8>(a, table, kh, j + 1, kv_end, base + L::kK0 + nbuf, base + L::kV0 + nbuf);
+        }
+        cp_async_commit();
+
+        // Lazy rescale: the reference maximum moves only when the tile's
+        // maximum exceeds it by more than 8 (weights stay below 2^8); the
+        // final O / l is the same for any reference.
+        if (j == 0) {
+            m_run = mx;  // O is written, not accumulated, by the first P V
+        } else {
+            const bool grow = mx > m_run + 8.0f;
+            if (__any_sync(0xffffffffu, grow)) {  // tcgen05.ld/st are warp-wide
+                const float alpha = grow ? fast_exp2(m_run - mx) : 1.0f;
+                if (grow) {
+                    m_run = mx;
+                    l_run *= alpha;
+                }
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    float v[32];
+                    tmem_ld32(tmem_o + lane_base + ch * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32(tmem_o + lane_base + ch * 32, v);
+                }
+            }
+        }
+
+        // P = exp2(s - m) as bf16 into shared memory; l sums the rounded weights
+        // (masked scores are -inf, so their weights are exactly 0)
+        float lsum = 0.0f;
+#pragma unroll
+        for (int c16 = 0; c16 < kBN / 8; ++c16) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const int i0 = c16 * 8 + 2 * h;
+                w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
+                lsum += bf16lo(w[h]) + bf16hi(w[h]);
+            }
+            st_shared16(sp + swz(kRows, tid, c16), make_uint4(w[0], w[1], w[2], w[3]));
+        }
+        l_run += lsum;
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // O += P V
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+                const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRows * 128 + (kk & 3) * 32);
+                mma_bf16(tmem_o, sw128_desc(sp + aoff, 16, 1024),
+                         sw128_desc(sv + static_cast<uint32_t>(kk * 16 * 128), kBN * 128, 1024), kIdescPV,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(bar_pv);
+        }
+    }
+
+    if (!timed_out) {
+        const bool ok = mbar_wait(bar_pv, static_cast<uint32_t>((n_tiles - 1) & 1));
+        if (__syncthreads_or(!ok)) {
+            timed_out = true;
+            pending = bar_pv;
+            pending_parity = static_cast<uint32_t>((n_tiles - 1) & 1);
+        }
+    }
+    cp_async_wait0();
+    if (timed_out) {
+        // one more bounded wait for the MMAs in flight before TMEM is freed
+        if (tid == 0) {
+            set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
+            mbar_wait(pending, pending_parity);
+        }
+    } else {
+        tc_fence_after();
+        const float inv = (FP8 ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            float v[32];
+            tmem_ld32(tmem_o + lane_base + ch * 32, v);  // warp-wide: every lane loads
+            if (row_live) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                    uint4 w = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv), pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
+                                         pack_bf16(v[i + 4] * inv, v[i + 5] * inv),
+                                         pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
+                    *reinterpret_cast<uint4 *>(out_row + ch * 32 + i) = w;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D, int G, bool FP8>
+cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
+    constexpr int TQ = kRows / G;
+    const int tiles = (a.max_q_len + TQ - 1) / TQ;
+    const long long nx = static_cast<long long>(a.num_seqs) * tiles;
+    if (nx > 0x7FFFFFFFLL || a.num_kv_heads > 65535) return cudaErrorInvalidConfiguration;
+    auto kern = paged_prefill_kernel<D, G, FP8>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Layout<D>::kAlloc));
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), kThreads, Layout<D>::kAlloc, stream>>>(a, tiles);
+    return cudaGetLastError();
+}
+
+template <int D, bool FP8>
+cudaError_t launch_d(const PrefillArgs &a, int g, cudaStream_t stream) {
+    switch (g) {
+        case 1: return launch_t<D, 1, FP8>(a, stream);
+        case 2: return launch_t<D, 2, FP8>(a, stream);
+        case 4: return launch_t<D, 4, FP8>(a, stream);
+        case 8: return launch_t<D, 8, FP8>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool prefill_supported(int head_dim, int group) {
+    return (head_dim == 64 || head_dim == 128) && (group == 1 || group == 2 || group == 4 || group == 8);
+}
+
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
+    const int g = a.num_q_heads / a.num_kv_heads;
+    if (a.head_dim == 128)
+        return a.fp8 ? launch_d<128, true>(a, g, stream) : launch_d<128, false>(a, g, stream);
+    return a.fp8 ? launch_d<64, true>(a, g, stream) : launch_d<64, false>(a, g, stream);
+}
+
+}  // namespace pkv

@@ -10,6 +10,7 @@ The functions mirror ``include/pagedkv.h``:
 * ``store_kvcache`` -- ``pkv_store_kvcache``
 * ``plan_decode`` -- ``pkv_plan_decode``
 * ``paged_attention_decode`` -- ``pkv_paged_attention_decode``
+* ``paged_attention_prefill`` -- ``pkv_paged_attention_prefill``
 * ``read_device_error`` -- ``pkv_read_device_error``
 """
 
@@ -35,7 +36,8 @@ PKV_CACHE_BF16 = 0
 PKV_CACHE_FP8_E4M3 = 1
 
 EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_paged_attention_decode", "pkv_status_string",
-            "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch")
+            "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
+            "pkv_paged_attention_prefill")
 
 
 class PagedKVError(RuntimeError):
@@ -83,6 +85,9 @@ def load_library(path: str):
     L.pkv_read_device_error.restype = i32
     L.pkv_version.argtypes = []
     L.pkv_version.restype = i32
+    L.pkv_paged_attention_prefill.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i64, f32,
+                                              i32, vp, vp, i32, vp, vp, vp]
+    L.pkv_paged_attention_prefill.restype = i32
     if hasattr(L, "pkv_paged_attention_decode_static_scratch"):
         L.pkv_paged_attention_decode_static_scratch.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
                                                                 i32, i64, f32, i32, vp, vp, i32, i32, vp, vp, vp]
@@ -227,6 +232,36 @@ def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, con
 
 
 STATIC_SCRATCH_BYTES = 32 << 20  # PKV_STATIC_SCRATCH_BYTES
+
+
+def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, scale, max_q_len,
+                            out=None, k_scale=None, v_scale=None, dev_err=None, stream=None):
+    """Chunked prefill: each sequence's chunk of query tokens (rows
+    ``cu_q_lens[i]`` .. ``cu_q_lens[i+1] - 1`` of ``q``, ``[total_q, nq, d]``
+    bf16) attends causally over its paged context; returns ``out`` like ``q``.
+    ``max_q_len`` is a host-known bound on every chunk length."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise TypeError("q must be contiguous bfloat16")
+    for t, n in ((block_tables, "block_tables"), (cu_q_lens, "cu_q_lens"), (context_lens, "context_lens")):
+        if t.dtype != torch.int32 or not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous int32")
+    if not (k_cache.is_contiguous() and v_cache.is_contiguous()):
+        raise ValueError("the pools must be contiguous")
+    T, nq, d = q.shape
+    nblk, nkv, bs, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("pool shape does not match q")
+    S = context_lens.shape[0]
+    if cu_q_lens.shape[0] != S + 1 or block_tables.shape[0] != S:
+        raise ValueError("cu_q_lens must have num_seqs + 1 entries and block_tables num_seqs rows")
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib().pkv_paged_attention_prefill(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(cu_q_lens),
+        _ptr(context_lens), S, T, nq, nkv, d, bs, nblk, float(scale), _cache_dtype(k_cache), _ptr(k_scale),
+        _ptr(v_scale), int(max_q_len), _ptr(out), _ptr(dev_err), _stream(stream))
+    _check(st, "pkv_paged_attention_prefill")
+    return out
 
 
 def longest_first(context_lens_host: torch.Tensor) -> torch.Tensor:

@@ -93,6 +93,7 @@ def test_store_host_checks(K):
     assert call(dt=1) == K.PKV_ERR_INVALID_ARG
     assert call(dt=7) == K.PKV_ERR_INVALID_ARG
     assert call(N=0) == K.PKV_OK
+    assert call(N=0, k=None, v=None, sm=None, kc=None, vc=None) == K.PKV_OK  # nothing to read or write
 
 
 @pytest.mark.parametrize("name,split,ws", [
