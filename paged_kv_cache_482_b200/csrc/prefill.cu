@@ -15,9 +15,12 @@
 // r % G, so the G heads that share a KV head share every K/V tile. The CTA
 // walks the sequence's KV in tiles of 128 logical tokens up to its last
 // row's position:
-//   1. K/V tiles are gathered through the block table with 16-byte cp.async
-//      copies (zero-filled past the causal end) into shared memory, double
-//      buffered, in the 128-byte-swizzled layout the tensor core reads;
+//   1. K/V tiles are gathered through the block table into shared memory,
+//      double buffered, in the 128-byte-swizzled layout the tensor core
+//      reads: for a bf16 cache one thread issues tensor-map (TMA) copies of
+//      whole block runs (a 2-D view of the pool, 64 columns x up to 64 rows
+//      per copy, no multicast) and the V rows past the causal end are zeroed
+//      on the last tile; an E4M3 cache is loaded and widened by the threads;
 //   2. one thread issues S = Q K^T (M 128, N 128, K head_dim) into tensor
 //      memory;
 //   3. the four warps each read their 32 tensor-memory lanes (one row per
@@ -35,6 +38,11 @@
 // 128 / 64 column blocks][rows][128 bytes], the 16-byte chunk c of row r
 // stored at chunk c ^ (r % 8) -- the canonical 128-byte swizzle, so one
 // descriptor form serves Q, K and P (K-major) and V (MN-major).
+#include <cuda.h>
+
+#include <cstring>
+#include <mutex>
+
 #include "pkv_common.cuh"
 #include "pkv_launch.h"
 
@@ -46,6 +54,14 @@ constexpr int kBN = 64;     // KV tokens per tile
 constexpr int kThreads = 128;
 constexpr uint32_t kTmemCols = 256;  // S: 64 columns, O: up to 128 columns (two CTAs fill an SM's 512)
 constexpr uint32_t kMinSmem = 100u * 1024u;  // at most two CTAs per SM, whatever head_dim
+constexpr int kTableCap = 2048;              // block ids staged in shared memory (more: read from global)
+
+// A sequence's block-table row: the first kTableCap ids from shared memory.
+struct BlockIds {
+    const int32_t *smem;
+    const int32_t *gmem;
+    __device__ __forceinline__ int operator[](int i) const { return i < kTableCap ? smem[i] : __ldg(gmem + i); }
+};
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -63,8 +79,9 @@ struct Layout {
     static constexpr uint32_t kPBytes = (kBN / 64) * kRows * 128;
     static constexpr bool kPInK = kPBytes <= kTileBytes;
     static constexpr uint32_t kP = kK0 + 2 * kBufStride;
-    static constexpr uint32_t kBar = kP + (kPInK ? 0 : kPBytes);  // 2 mbarriers, TMEM address
-    static constexpr uint32_t kBytes = kBar + 64;
+    static constexpr uint32_t kBar = kP + (kPInK ? 0 : kPBytes);  // 4 mbarriers, TMEM address
+    static constexpr uint32_t kTable = kBar + 64;                  // the sequence's first block ids
+    static constexpr uint32_t kBytes = kTable + kTableCap * 4;
     static constexpr uint32_t kAlloc = (kBytes + 1024 > kMinSmem) ? kBytes + 1024 : kMinSmem;  // + base alignment
 };
 
@@ -155,6 +172,15 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// 2-D tensor-map copy of one box into shared memory, completing on *bar.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void st_shared16(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -188,8 +214,8 @@ __device__ __forceinline__ uint32_t swz(int rows, int r, int c16) {
 // Tokens at or past kv_end are zero-filled; their scores are masked anyway
 // and zeros keep P V finite.
 template <int D, bool FP8>
-__device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const int32_t *table, int kh, int j, int kv_end,
-                                             uint32_t sk, uint32_t sv) {
+__device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const BlockIds &table, int kh, int j, int kv_end,
+                                             int log2_bs, uint32_t sk, uint32_t sv) {
     constexpr int kChunks = D / 8;             // 16-byte chunks per bf16 row
     constexpr int kTokPerPass = kThreads / kChunks;
     const int c16 = threadIdx.x % kChunks;
@@ -200,8 +226,8 @@ __device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const int32_t
         const int pos = j * kBN + t;
         const bool valid = pos < kv_end;
         const int p = valid ? pos : 0;
-        const int64_t blk = table[p / bs];
-        const int64_t elem = ((blk * a.num_kv_heads + kh) * bs + (p % bs)) * D + c16 * 8;
+        const int64_t blk = table[p >> log2_bs];
+        const int64_t elem = ((blk * a.num_kv_heads + kh) * bs + (p & (bs - 1))) * D + c16 * 8;
         const uint32_t off = swz(kBN, t, c16);
         if constexpr (FP8) {
             uint2 kw = make_uint2(0, 0), vw = make_uint2(0, 0);
@@ -220,8 +246,46 @@ __device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const int32_t
     }
 }
 
+// One thread: stage KV tile j of KV head kh (bf16 cache) with tensor-map
+// copies. The pool is viewed as rows (block * nkv + head) * bs + offset of
+// head_dim elements; a copy moves 64 columns (one 128-byte swizzle span) of
+// min(bs, kBN) consecutive rows of one block. Blocks wholly past kv_end are
+// not copied.
+template <int D>
+__device__ __forceinline__ void tma_kv_tile(const CUtensorMap *mk, const CUtensorMap *mv, const BlockIds &table, int nkv,
+                                            int kh, int bs, int log2_bs, int j, int kv_end, uint32_t sk, uint32_t sv,
+                                            uint64_t *bar) {
+    constexpr int kHalves = D / 64;
+    const int kv0 = j * kBN;
+    if (bs >= kBN) {
+        const int blk = table[kv0 >> log2_bs];
+        const int row = (blk * nkv + kh) * bs + (kv0 & (bs - 1));
+        mbar_arrive_expect_tx(bar, 2u * kHalves * kBN * 128u);
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
+            tma_load_2d(sk + h * kBN * 128, mk, h * 64, row, bar);
+            tma_load_2d(sv + h * kBN * 128, mv, h * 64, row, bar);
+        }
+    } else {
+        const int end = min(kv0 + kBN, kv_end);
+        const int nb = (end - kv0 + bs - 1) >> log2_bs;
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(2 * kHalves * nb * bs * 128));
+        for (int i = 0; i < nb; ++i) {
+            const int blk = table[(kv0 >> log2_bs) + i];
+            const int row = (blk * nkv + kh) * bs;
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) {
+                tma_load_2d(sk + h * kBN * 128 + i * bs * 128, mk, h * 64, row, bar);
+                tma_load_2d(sv + h * kBN * 128 + i * bs * 128, mv, h * 64, row, bar);
+            }
+        }
+    }
+}
+
 template <int D, int G, bool FP8>
-__global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs a, int tiles_per_seq) {
+__global__ void __launch_bounds__(kThreads, 2)
+    paged_prefill_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
+                         const __grid_constant__ CUtensorMap map_v) {
     using L = Layout<D>;
     constexpr int TQ = kRows / G;  // chunk tokens per CTA
     constexpr uint32_t kIdescS = idesc_bf16(kRows, kBN, false);
@@ -233,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
     uint8_t *sm = smem_raw + (base - raw);
     uint64_t *bar_s = reinterpret_cast<uint64_t *>(sm + L::kBar);
     uint64_t *bar_pv = bar_s + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bar_s + 2);
+    uint64_t *bar_kv = bar_s + 2;  // one per K/V buffer (TMA copies)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bar_s + 4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -253,16 +318,19 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
     const int t0 = tile * TQ;
     if (t0 >= c) return;
     const int ctx = a.context_lens[s];
-    const int32_t *table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+    const int32_t *table_g = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+    int32_t *table_s = reinterpret_cast<int32_t *>(sm + L::kTable);
     bool bad = ctx < c || static_cast<int64_t>(ctx) > static_cast<int64_t>(a.max_blocks_per_seq) * a.block_size ||
                c > a.max_q_len;
     if (!bad) {
-        const int nblk_seq = (ctx + a.block_size - 1) / a.block_size;
+        const int nblk_seq = (ctx + a.block_size - 1) >> log2_bs;
         for (int i = tid; i < nblk_seq; i += kThreads) {
-            const int32_t b = table[i];
+            const int32_t b = table_g[i];
             if (b < 0 || b >= a.num_blocks) bad = true;
+            if (i < kTableCap) table_s[i] = b;
         }
     }
+    const BlockIds table{table_s, table_g};
     const int row_tok = t0 + tid / G;  // this thread's row
     const int row_head = kh * G + tid % G;
     const bool row_live = row_tok < c;
@@ -287,6 +355,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
     if (tid == 0) {
         mbar_init(bar_s, 1);
         mbar_init(bar_pv, 1);
+        mbar_init(bar_kv, 1);
+        mbar_init(bar_kv + 1, 1);
         fence_barrier_init();
     }
     tc_fence_before();
@@ -296,10 +366,24 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
     const uint32_t tmem_s = tmem;        // S: columns 0..kBN - 1
     const uint32_t tmem_o = tmem + 128;  // O: columns 128..128 + D - 1
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-
     const uint32_t sq = base + L::kQ;
+    auto kbuf = [&](int j) { return base + L::kK0 + static_cast<uint32_t>(j & 1) * L::kBufStride; };
+    auto vbuf = [&](int j) { return base + L::kV0 + static_cast<uint32_t>(j & 1) * L::kBufStride; };
 
-    // Q rows (zero past the chunk) and KV tile 0
+    // S = Q K_j^T, issued by thread 0 once tile j's K is in shared memory
+    auto issue_s = [&](int j) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRows * 128 + (kk & 3) * 32);
+            const uint32_t boff = static_cast<uint32_t>((kk >> 2) * kBN * 128 + (kk & 3) * 32);
+            mma_bf16(tmem_s, sw128_desc(sq + aoff, 16, 1024), sw128_desc(kbuf(j) + boff, 16, 1024), kIdescS,
+                     kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s);
+    };
+
+    // Q rows (zero past the chunk) and the first KV tiles
     {
         constexpr int kChunks = D / 8;
         const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q);
@@ -311,36 +395,33 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
             cp_async16(sq + swz(kRows, r, c16), qp + elem, valid ? 16u : 0u);
         }
     }
-    load_kv_tile<D, FP8>(a, table, kh, 0, kv_end, base + L::kK0, base + L::kV0);
+    if constexpr (FP8) {
+        load_kv_tile<D, FP8>(a, table, kh, 0, kv_end, log2_bs, kbuf(0), vbuf(0));
+    } else if (tid == 0) {
+        tma_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, 0, kv_end, kbuf(0), vbuf(0),
+                       bar_kv);
+        if (n_tiles > 1)
+            tma_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, 1, kv_end, kbuf(1),
+                           vbuf(1), bar_kv + 1);
+    }
     cp_async_commit();
-
-    const float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
-    float m_run = -INFINITY, l_run = 0.0f;
+    cp_async_wait0();
+    fence_proxy_async_smem();
+    __syncthreads();
     bool timed_out = false;
     uint64_t *pending = nullptr;  // the barrier a timed-out wait was on
     uint32_t pending_parity = 0;
+    if (tid == 0) {
+        if (FP8 || mbar_wait(bar_kv, 0)) issue_s(0);
+    }
+
+    const float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
+    float m_run = -INFINITY, l_run = 0.0f;
 
     for (int j = 0; j < n_tiles; ++j) {
-        const uint32_t buf = static_cast<uint32_t>(j & 1) * L::kBufStride;
-        const uint32_t sk = base + L::kK0 + buf;
-        const uint32_t sv = base + L::kV0 + buf;
-        const uint32_t sp = L::kPInK ? sk : base + L::kP;
-        cp_async_wait0();  // this tile's copies (and Q) have landed
-        fence_proxy_async_smem();
-        __syncthreads();
+        const uint32_t sk = kbuf(j), sv = vbuf(j);
+        const uint32_t sp = L::kPInK ? sk : base + L::kP;  // P replaces this tile's K once S is computed
 
-        // S = Q K^T (queued behind P V of the previous tile)
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRows * 128 + (kk & 3) * 32);
-                const uint32_t boff = static_cast<uint32_t>((kk >> 2) * kBN * 128 + (kk & 3) * 32);
-                mma_bf16(tmem_s, sw128_desc(sq + aoff, 16, 1024), sw128_desc(sk + boff, 16, 1024), kIdescS,
-                         kk > 0 ? 1u : 0u);
-            }
-            mma_commit(bar_s);
-        }
         const bool ok_s = mbar_wait(bar_s, static_cast<uint32_t>(j & 1));
         if (__syncthreads_or(!ok_s)) {
             timed_out = true;
@@ -366,9 +447,13 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
             for (int i = 0; i < kBN; ++i)
                 if (kv0 + i > row_pos) x[i] = -INFINITY;
         }
-        float mx = x[0];
+        float m8[8];
 #pragma unroll
-        for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, x[i]);
+        for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+        for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 
         // P V of the previous tile has finished: P, O and the other buffer are free
         if (j > 0) {
@@ -382,10 +467,13 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
             tc_fence_after();
         }
         if (j + 1 < n_tiles) {
-            const uint32_t nbuf = static_cast<uint32_t>((j + 1) & 1) * L::kBufStride;
-            load_kv_tile<D, FP8>(a, table, kh, j + 1, kv_end, base + L::kK0 + nbuf, base + L::kV0 + nbuf);
+            if constexpr (FP8) {
+                load_kv_tile<D, FP8>(a, table, kh, j + 1, kv_end, log2_bs, kbuf(j + 1), vbuf(j + 1));
+            } else if (tid == 0 && j + 1 >= 2) {  // tiles 0 and 1 were issued up front
+                tma_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, j + 1, kv_end,
+                               kbuf(j + 1), vbuf(j + 1), bar_kv + ((j + 1) & 1));
+            }
         }
-        cp_async_commit();
 
         // Lazy rescale: the reference maximum moves only when the tile's
         // maximum exceeds it by more than 8 (weights stay below 2^8); the
@@ -413,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
 
         // P = exp2(s - m) as bf16 into shared memory; l sums the rounded weights
         // (masked scores are -inf, so their weights are exactly 0)
-        float lsum = 0.0f;
+        float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int c16 = 0; c16 < kBN / 8; ++c16) {
             uint32_t w[4];
@@ -421,16 +509,29 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
             for (int h = 0; h < 4; ++h) {
                 const int i0 = c16 * 8 + 2 * h;
                 w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
-                lsum += bf16lo(w[h]) + bf16hi(w[h]);
+                l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
             }
             st_shared16(sp + swz(kRows, tid, c16), make_uint4(w[0], w[1], w[2], w[3]));
         }
-        l_run += lsum;
+        l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+
+        if constexpr (!FP8) {
+            const int valid_rows = kv_end - kv0;
+            if (valid_rows < kBN && mbar_wait(bar_kv + (j & 1), static_cast<uint32_t>((j >> 1) & 1))) {
+                // rows past the causal end: zero V so that 0-weight x stale data stays 0
+                constexpr int kHalves = D / 64;
+                const int n16 = (kBN - valid_rows) * 8;  // 16-byte chunks per half
+                for (int i = tid; i < kHalves * n16; i += kThreads) {
+                    const int h = i / n16, r = valid_rows + (i % n16) / 8, cc = i % 8;
+                    st_shared16(sv + h * kBN * 128 + r * 128 + cc * 16, make_uint4(0, 0, 0, 0));
+                }
+            }
+        }
         tc_fence_before();
         fence_proxy_async_smem();
         __syncthreads();
 
-        // O += P V
+        // O += P V_j, then S_{j+1} right behind it on the tensor core
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -441,6 +542,10 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
                          (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(bar_pv);
+            if (j + 1 < n_tiles) {
+                if (FP8 || mbar_wait(bar_kv + ((j + 1) & 1), static_cast<uint32_t>(((j + 1) >> 1) & 1)))
+                    issue_s(j + 1);
+            }
         }
     }
 
@@ -485,17 +590,65 @@ __global__ void __launch_bounds__(kThreads, 2) paged_prefill_kernel(PrefillArgs 
     }
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// The pool as a 2-D bf16 tensor: rows of head_dim elements; boxes of 64
+// columns x min(block_size, kBN) rows, 128-byte swizzle.
+bool make_pool_map(CUtensorMap *map, const void *pool, const PrefillArgs &a) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.head_dim),
+                                static_cast<cuuint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.head_dim) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(a.block_size < kBN ? a.block_size : kBN)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int G, bool FP8>
 cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int TQ = kRows / G;
     const int tiles = (a.max_q_len + TQ - 1) / TQ;
     const long long nx = static_cast<long long>(a.num_seqs) * tiles;
     if (nx > 0x7FFFFFFFLL || a.num_kv_heads > 65535) return cudaErrorInvalidConfiguration;
+    int log2_bs = 0;
+    while ((1 << log2_bs) < a.block_size) ++log2_bs;
+    CUtensorMap mk, mv;
+    memset(&mk, 0, sizeof(mk));
+    memset(&mv, 0, sizeof(mv));
+    if (!FP8) {
+        // TMA row coordinates are int32
+        if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * a.block_size > 0x7FFFFFFFLL)
+            return cudaErrorInvalidConfiguration;
+        if (!make_pool_map(&mk, a.k_cache, a) || !make_pool_map(&mv, a.v_cache, a)) return cudaErrorInvalidValue;
+    }
     auto kern = paged_prefill_kernel<D, G, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(Layout<D>::kAlloc));
     if (e != cudaSuccess) return e;
-    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), kThreads, Layout<D>::kAlloc, stream>>>(a, tiles);
+    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), kThreads, Layout<D>::kAlloc, stream>>>(a, tiles, log2_bs,
+                                                                                                 mk, mv);
     return cudaGetLastError();
 }
 

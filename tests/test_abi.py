@@ -134,3 +134,30 @@ def test_binding_refuses_to_run_without_library(tmp_path):
             pagedkv.lib(str(tmp_path / "missing.so"))
         finally:
             pagedkv._lib = pagedkv._lib_saved
+
+
+def test_prefill_host_checks(K):
+    L = K.lib()
+    ok = dict(q=0x10000, kc=0x20000, vc=0x30000, bt=0x40000, maxb=8, cu=0x50000, cl=0x60000, S=4, T=100, nq=32,
+              nkv=8, d=128, bs=256, nblk=100, scale=0.088, dt=0, ks=None, vs=None, mq=64, out=0x70000)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.pkv_paged_attention_prefill(a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cu"], a["cl"], a["S"],
+                                             a["T"], a["nq"], a["nkv"], a["d"], a["bs"], a["nblk"], a["scale"],
+                                             a["dt"], a["ks"], a["vs"], a["mq"], a["out"], None, None)
+
+    assert call(q=None) == K.PKV_ERR_INVALID_ARG
+    assert call(cu=None) == K.PKV_ERR_INVALID_ARG
+    assert call(out=0x70008) == K.PKV_ERR_INVALID_ARG  # misaligned
+    assert call(d=96) == K.PKV_ERR_UNSUPPORTED
+    assert call(nq=24) == K.PKV_ERR_UNSUPPORTED  # group 3
+    assert call(nq=30) == K.PKV_ERR_INVALID_ARG
+    assert call(bs=100) == K.PKV_ERR_INVALID_ARG
+    assert call(dt=1) == K.PKV_ERR_INVALID_ARG  # FP8 without scales
+    assert call(dt=5) == K.PKV_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == K.PKV_ERR_INVALID_ARG
+    assert call(mq=0) == K.PKV_ERR_INVALID_ARG
+    assert call(nblk=2**31) == K.PKV_ERR_INVALID_ARG
+    assert call(S=0) == K.PKV_OK and call(T=0) == K.PKV_OK  # nothing to do, nothing launched
