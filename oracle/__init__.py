@@ -61,6 +61,11 @@ def _bind(lib):
         + [c.c_void_p] * 3 + [c.c_int]
     )
     lib.orc_paged_attention_prefill.restype = c.c_int
+    lib.orc_bf16_from_double.argtypes = [c.c_double]
+    lib.orc_bf16_from_double.restype = c.c_uint16
+    lib.orc_fused_add_rmsnorm.argtypes = [c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_int, c.c_double,
+                                          c.c_void_p, c.c_void_p, c.c_int]
+    lib.orc_fused_add_rmsnorm.restype = c.c_int
     return lib
 
 
@@ -230,3 +235,23 @@ def run_prefill_workload(wl, num_threads=1, lib=None):
                                        cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, wl.k_scale, wl.v_scale,
                                        num_threads=num_threads, lib=lib)
     return out, kp, vp, st1 | st2 | st3
+
+
+def bf16_from_double(v: float, lib=None) -> int:
+    return (lib or load()).orc_bf16_from_double(float(v))
+
+
+def fused_add_rmsnorm(x, residual, weight, eps, num_threads=1, lib=None):
+    """fp64 residual add + RMSNorm of rows ``x`` ``[T, H]`` (bf16).
+
+    Returns ``(out [T, H] float64, residual_out [T, H] bf16 bits or None, status)``.
+    """
+    lib = lib or load()
+    x = _np(x, np.uint16)
+    T, H = x.shape
+    r = _np(residual, np.uint16) if residual is not None else None
+    w = _np(weight, np.uint16)
+    out = np.zeros((T, H), dtype=np.float64)
+    rout = np.zeros((T, H), dtype=np.uint16) if r is not None else None
+    st = lib.orc_fused_add_rmsnorm(_p(x), _p(r), _p(w), T, H, float(eps), _p(out), _p(rout), int(num_threads))
+    return out, rout, st

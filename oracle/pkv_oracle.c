@@ -1,6 +1,7 @@
 /*
- * pkv_oracle.c -- plain, slow, fp64 CPU oracle for paged attention: one
- * decode step, and a chunk of prefill tokens attending causally.
+ * pkv_oracle.c -- plain, slow, fp64 CPU oracle for paged attention (one
+ * decode step, and a chunk of prefill tokens attending causally) and for the
+ * residual add + RMSNorm of the layer around it.
  *
  * TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's
  * CPU-baseline leg are the only callers. It shares no code, header, table or
@@ -32,6 +33,10 @@
  *    nearest E4M3 value, ties to the even code, magnitudes beyond 448 clamped
  *    to 448 (NaN stays NaN);
  *  - FP8 read: code value times the head's scale, both exact in fp64.
+ *  - Add + RMSNorm (same page, section 核心技术改进 1 "CUDA融合内核：Add+RMSNorm":
+ *    the residual add and the RMSNorm that follows it, fused): h = x + r,
+ *    the residual stream continues as h, and the normalised output is
+ *    w * h / sqrt(mean(h^2) + eps) over the hidden dimension.
  *  - Chunked prefill ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目",
  *    section 核心技术改进 2 "Chunked Prefill": a long prompt's prefill is cut
  *    into chunks that run interleaved with decode work): a chunk of c new
@@ -368,4 +373,73 @@ int orc_paged_attention_prefill(const uint16_t *q, const void *k_cache, const vo
         free(acc);
     }
     return status;
+}
+
+/*
+ * Nearest bf16 value of an fp64 number, ties to the even significand,
+ * overflow to infinity (IEEE round-to-nearest-even with 8 significant bits,
+ * exponent range of binary32); returns the bf16 bit pattern. NaN gives the
+ * quiet NaN 0x7FC0.
+ */
+uint16_t orc_bf16_from_double(double v)
+{
+    double a = fabs(v), quantum, q, fl, r;
+    int e;
+    uint16_t sign = (v < 0 || (v == 0 && signbit(v))) ? 0x8000 : 0;
+    union { float f; uint32_t u; } cv;
+    if (v != v)
+        return 0x7FC0;
+    if (a == 0.0)
+        return sign;
+    frexp(a, &e); /* a = m * 2^e, 0.5 <= m < 1 */
+    if (e - 1 < -126)
+        quantum = ldexp(1.0, -133); /* subnormal spacing */
+    else
+        quantum = ldexp(1.0, e - 8); /* 8 significant bits */
+    q = a / quantum;                 /* exact: a power-of-two scaling */
+    fl = floor(q);
+    r = q - fl;
+    if (r > 0.5 || (r == 0.5 && fmod(fl, 2.0) == 1.0))
+        fl += 1.0;
+    a = fl * quantum;
+    if (a > 3.3895313892515355e38) /* beyond the largest finite bf16 */
+        return sign | 0x7F80;
+    cv.f = (float)a; /* exact: a has at most 8 significant bits */
+    return sign | (uint16_t)(cv.u >> 16);
+}
+
+/*
+ * fused_add_rmsnorm: for each of the num_tokens rows of hidden elements,
+ * h = x + residual (x alone when residual is NULL), computed exactly in
+ * fp64; residual_out (if not NULL) receives h rounded to bf16; out receives
+ * weight * h / sqrt(mean(h^2) + eps) in fp64.
+ */
+int orc_fused_add_rmsnorm(const uint16_t *x, const uint16_t *residual, const uint16_t *weight, int num_tokens,
+                          int hidden, double eps, double *out, uint16_t *residual_out, int num_threads)
+{
+    int t;
+    if (!x || !weight || !out || num_tokens < 0 || hidden < 1 || !(eps >= 0))
+        return ORC_ERR_ARG;
+    if (num_threads < 1)
+        num_threads = 1;
+#pragma omp parallel for schedule(static) num_threads(num_threads)
+    for (t = 0; t < num_tokens; ++t) {
+        const int64_t row = (int64_t)t * hidden;
+        double ss = 0.0, inv;
+        int i;
+        for (i = 0; i < hidden; ++i) {
+            double h = orc_bf16_to_double(x[row + i]);
+            if (residual)
+                h += orc_bf16_to_double(residual[row + i]);
+            out[row + i] = h;
+            ss += h * h;
+        }
+        inv = 1.0 / sqrt(ss / hidden + eps);
+        for (i = 0; i < hidden; ++i) {
+            if (residual_out)
+                residual_out[row + i] = orc_bf16_from_double(out[row + i]);
+            out[row + i] = orc_bf16_to_double(weight[i]) * (out[row + i] * inv);
+        }
+    }
+    return ORC_OK;
 }

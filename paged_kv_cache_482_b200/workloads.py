@@ -474,3 +474,53 @@ def prefill_logical_kv(wl: PrefillWorkload, i: int):
     rows = wl.hist_rows[i].to(wl.k_hist.device)
     a, b = int(wl.cu_q_lens[i]), int(wl.cu_q_lens[i + 1])
     return torch.cat([wl.k_hist[rows], wl.k_new[a:b]]), torch.cat([wl.v_hist[rows], wl.v_new[a:b]])
+
+
+# ------------------------------------------------------------ add + RMSNorm
+#
+# The residual add and RMSNorm around the attention of a layer
+# ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section 核心技术改进 1
+# "CUDA融合内核：Add+RMSNorm"): rows of hidden states, their residual stream
+# and the norm weight.
+
+
+@dataclass(frozen=True)
+class NormConfig:
+    name: str
+    num_tokens: int
+    hidden: int
+    eps: float = 1e-6
+    residual: bool = True
+
+
+NORM_CONFIGS: dict[str, NormConfig] = {
+    c.name: c
+    for c in (
+        NormConfig("norm_tiny", 5, 64),
+        NormConfig("norm_qwen3_0.6b", 256, 1024),
+        # Qwen3-8B hidden size, one decode step of 1024 sequences
+        NormConfig("norm_qwen3_8b_decode", 1024, 4096),
+        # Qwen3-8B hidden size, a chunked-prefill step of 16 x 512 tokens (larger than L2 in total)
+        NormConfig("norm_qwen3_8b", 8192, 4096),
+    )
+}
+
+
+@dataclass
+class NormWorkload:
+    cfg: NormConfig
+    seed: int
+    x: torch.Tensor  # [T, H] bf16
+    residual: torch.Tensor | None  # [T, H] bf16
+    weight: torch.Tensor  # [H] bf16
+
+
+def generate_norm(cfg: NormConfig, seed: int = 0, device: str | torch.device = "cpu") -> NormWorkload:
+    """x and the residual are N(0, 1) rounded to bf16; the weight is
+    1 + 0.1 N(0, 1) rounded to bf16 (a trained norm weight stays near 1)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(seed + 1)
+    x = _randn_bf16((cfg.num_tokens, cfg.hidden), g, device)
+    r = _randn_bf16((cfg.num_tokens, cfg.hidden), g, device) if cfg.residual else None
+    w = (1.0 + 0.1 * torch.randn(cfg.hidden, generator=g, device=device)).to(torch.bfloat16)
+    return NormWorkload(cfg, seed, x, r, w)

@@ -508,7 +508,69 @@ def pin_prefill_errors(lib):
     assert call(cu_=bad)[1] == O.ORC_ERR_ARG
 
 
+# ----------------------------------------------------------- add + RMSNorm
+
+
+def pin_rmsnorm_library(lib):
+    """out against torch's rms_norm (a library routine) in fp64 on the exact
+    sum, for several widths, eps values and with / without a residual."""
+    for T, H, eps, res, seed in ((3, 64, 1e-6, True, 1), (4, 1000, 1e-5, True, 2), (2, 8, 0.5, False, 3),
+                                 (5, 4096, 1e-6, True, 4)):
+        wl = W.generate_norm(W.NormConfig("p", T, H, eps, res), seed)
+        out, _, st = O.fused_add_rmsnorm(wl.x, wl.residual, wl.weight, eps, lib=lib)
+        assert st == O.ORC_OK
+        h = wl.x.double() + (wl.residual.double() if res else 0)
+        want = torch.nn.functional.rms_norm(h, (H,), wl.weight.double(), eps).numpy()
+        rel = np.abs(out - want).max() / np.abs(want).max()
+        assert rel <= 1e-13, f"rms_norm T={T} H={H}: rel {rel:.2e}"
+
+
+def pin_rmsnorm_residual_is_rounded_sum(lib):
+    """residual_out is the bf16 (round to nearest even) of x + r: torch's own
+    bf16 cast of the fp64 sum; and the bf16 rounding itself on arbitrary
+    binary32 values against torch's cast."""
+    wl = W.generate_norm(W.NormConfig("p", 16, 256), 5)
+    wl.residual[0, :8] = torch.tensor([1.0, -1.0, 2.0 ** -130, 3.0e38, 65504.0, 0.0, -0.0, 1e-3]).to(torch.bfloat16)
+    wl.x[0, :8] = torch.tensor([2.0 ** -8, -(2.0 ** -8), 2.0 ** -131, 3.0e38, 1.0, -0.0, -0.0, 3.0]).to(torch.bfloat16)
+    _, rout, st = O.fused_add_rmsnorm(wl.x, wl.residual, wl.weight, 1e-6, lib=lib)
+    want = (wl.x.double() + wl.residual.double()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert st == O.ORC_OK and np.array_equal(rout, want), "residual_out is not bf16(x + r)"
+    g = torch.Generator().manual_seed(6)
+    bits = torch.randint(-(2 ** 31), 2 ** 31 - 1, (20000,), generator=g, dtype=torch.int64).to(torch.int32)
+    f = bits.view(torch.float32)
+    f = f[torch.isfinite(f)]
+    ties = (torch.randint(0, 2 ** 16, (2000,), generator=g).to(torch.int32) << 16 | 0x8000).view(torch.float32)
+    vals = torch.cat([f, ties[torch.isfinite(ties)]])
+    want = vals.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([O.bf16_from_double(float(v), lib=lib) for v in vals.tolist()], dtype=np.uint16)
+    assert np.array_equal(got, want), "bf16 rounding differs from torch's cast"
+
+
+def pin_rmsnorm_closed_forms(lib):
+    H = 32
+    w = torch.linspace(0.5, 1.5, H).to(torch.bfloat16)
+    for c in (0.75, -3.0, 1e-3):
+        x = torch.full((1, H), c).to(torch.bfloat16)
+        out, _, _ = O.fused_add_rmsnorm(x, None, w, 1e-6, lib=lib)
+        cb = float(x[0, 0])
+        want = w.double().numpy() * cb / np.sqrt(cb * cb + 1e-6)
+        _assert_close(out[0], want, tol=1e-14, what=f"constant row {c}")
+    z = torch.zeros((2, H), dtype=torch.bfloat16)
+    out, _, _ = O.fused_add_rmsnorm(z, z, w, 1e-6, lib=lib)
+    assert np.array_equal(out, np.zeros_like(out)), "a zero row normalises to zeros"
+    wl = W.generate_norm(W.NormConfig("p", 3, H, 0.0, False), 7)
+    o1, _, _ = O.fused_add_rmsnorm(wl.x, None, wl.weight, 0.0, lib=lib)
+    o2, _, _ = O.fused_add_rmsnorm((wl.x.float() * -4.0).to(torch.bfloat16), None, wl.weight, 0.0, lib=lib)
+    _assert_close(o1, -o2, tol=1e-14, what="eps 0: scaling the row by -4 flips the sign only")
+    r0 = torch.zeros_like(wl.x)
+    o3, _, _ = O.fused_add_rmsnorm(wl.x, r0, wl.weight, 0.0, lib=lib)
+    assert np.array_equal(o1, o3), "a zero residual is no residual"
+
+
 ALL_PINS = [
+    pin_rmsnorm_library,
+    pin_rmsnorm_residual_is_rounded_sum,
+    pin_rmsnorm_closed_forms,
     pin_prefill_bruteforce,
     pin_prefill_one_token_is_decode,
     pin_prefill_chunking_invariance,

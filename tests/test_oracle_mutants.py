@@ -60,6 +60,21 @@ MUTANTS = [
     ("prefill max not subtracted", "w[t] = exp(score[t] - m);", "w[t] = exp(score[t]);", 1),
     ("prefill not normalised", "acc[i] / z;", "acc[i];", 1),
     ("prefill v read from k", "cache_value(v_cache, idx, fp8, v_scale, g)", "cache_value(k_cache, idx, fp8, v_scale, g)", 1),
+    # add + RMSNorm
+    ("rmsnorm eps outside sqrt", "inv = 1.0 / sqrt(ss / hidden + eps);", "inv = 1.0 / (sqrt(ss / hidden) + eps);", 0),
+    ("rmsnorm sum not mean", "inv = 1.0 / sqrt(ss / hidden + eps);", "inv = 1.0 / sqrt(ss + eps);", 0),
+    ("rmsnorm n - 1", "inv = 1.0 / sqrt(ss / hidden + eps);", "inv = 1.0 / sqrt(ss / (hidden - 1) + eps);", 0),
+    ("rmsnorm residual not added", "h += orc_bf16_to_double(residual[row + i]);", "h += 0.0;", 0),
+    ("rmsnorm residual out is x", "residual_out[row + i] = orc_bf16_from_double(out[row + i]);",
+     "residual_out[row + i] = x[row + i];", 0),
+    ("rmsnorm weight unused", "out[row + i] = orc_bf16_to_double(weight[i]) * (out[row + i] * inv);",
+     "out[row + i] = out[row + i] * inv;", 0),
+    ("rmsnorm abs not square", "ss += h * h;", "ss += fabs(h);", 0),
+    ("bf16 rounding ties away", "(r == 0.5 && fmod(fl, 2.0) == 1.0)", "(r == 0.5)", 0),
+    ("bf16 subnormal spacing", "quantum = ldexp(1.0, -133);", "quantum = ldexp(1.0, -132);", 0),
+    ("bf16 overflow kept finite", "return sign | 0x7F80;", "return sign | 0x7F7F;", 0),
+    ("bf16 sign of zero", "uint16_t sign = (v < 0 || (v == 0 && signbit(v))) ? 0x8000 : 0;",
+     "uint16_t sign = (v < 0) ? 0x8000 : 0;", 0),
 ]
 
 
