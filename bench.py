@@ -51,8 +51,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="qwen3_8b", choices=sorted(W.CONFIGS) + sorted(W.PREFILL_CONFIGS),
-                    help="a decode workload, or a chunked-prefill one (prefill_*)")
+    ap.add_argument("--config", default="qwen3_8b",
+                    choices=sorted(W.CONFIGS) + sorted(W.PREFILL_CONFIGS) + sorted(W.NORM_CONFIGS),
+                    help="a decode workload, a chunked-prefill one (prefill_*) or an add + RMSNorm one (norm_*)")
     ap.add_argument("--partition", type=int, default=0, help="0 auto, -1 never split, >0 tokens per partition")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--num-seqs", type=int, default=0, help="override the workload's sequence count")
@@ -685,10 +686,187 @@ def run_prefill(args):
     return 0
 
 
+# ------------------------------------------------------------ add + RMSNorm
+
+NORM_METRIC = "fused residual add + RMSNorm rows/sec and achieved HBM GB/s"
+
+
+def norm_desc(cfg) -> str:
+    return (f"{cfg.name} residual add + RMSNorm: {cfg.num_tokens} rows x hidden {cfg.hidden}, eps {cfg.eps}, "
+            f"{'with' if cfg.residual else 'without'} residual, bf16")
+
+
+def norm_bytes(cfg) -> int:
+    """Bytes one launch must move: x read and out written, the residual read
+    and written back, the weight read once."""
+    per = (4 if cfg.residual else 2) * 2
+    return cfg.num_tokens * cfg.hidden * per + cfg.hidden * 2
+
+
+def norm_cpu_baseline(wl, target_s: float) -> dict:
+    import oracle as O
+
+    threads = cpu_threads()
+    c = wl.cfg
+    x, r, w = wl.x.cpu(), (wl.residual.cpu() if wl.residual is not None else None), wl.weight.cpu()
+    n = max(1, min(c.num_tokens, 64))
+    t0 = time.perf_counter()
+    O.fused_add_rmsnorm(x[:n], r[:n] if r is not None else None, w, c.eps, num_threads=threads)
+    dt = time.perf_counter() - t0
+    n2 = int(min(c.num_tokens, max(n, n * target_s / max(dt, 1e-6))))
+    t0 = time.perf_counter()
+    _, _, st = O.fused_add_rmsnorm(x[:n2], r[:n2] if r is not None else None, w, c.eps, num_threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": n2 / dt, "unit": "rows/s", "cores": threads, "kind": "oracle",
+            "sample": f"the first {n2} of {c.num_tokens} rows, fp64, {dt:.2f} s, OpenMP over rows; status {st}"}
+
+
+def run_norm_reference(args):
+    if rank_env()[1] != 0:
+        return 0
+    import oracle as O
+
+    cfg = W.NORM_CONFIGS[args.config]
+    wl = W.generate_norm(cfg, args.seed, device="cuda" if torch.cuda.is_available() else "cpu")
+    threads = cpu_threads()
+    x, r, w = wl.x.cpu(), (wl.residual.cpu() if wl.residual is not None else None), wl.weight.cpu()
+    n = cfg.num_tokens
+    for _ in range(args.warmup):
+        O.fused_add_rmsnorm(x, r, w, cfg.eps, num_threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.fused_add_rmsnorm(x, r, w, cfg.eps, num_threads=threads)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    print(json.dumps({
+        "impl": "reference", "metric": NORM_METRIC, "value": value, "unit": "rows/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": norm_desc(cfg)},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": threads, "kind": "oracle",
+                         "sample": f"all {n} rows per step, fp64, OpenMP over rows"},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def run_norm(args):
+    from paged_kv_cache_482_b200 import pagedkv as K
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    cfg = W.NORM_CONFIGS[args.config]
+    wl = W.generate_norm(cfg, args.seed + rank, device="cuda")
+    x, r, w = wl.x, wl.residual, wl.weight
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        K.fused_add_rmsnorm(x, r, w, cfg.eps, out=out)
+    torch.cuda.synchronize()
+    # inputs larger than L2 (checked) or L2 flushed between steps
+    moved = norm_bytes(cfg)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if moved < (256 << 20) else None
+    sampler = ClockSampler(nvsmi_ids(local)) if local == 0 else None
+    if sampler:
+        sampler.wait_first()
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kst)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for k in range(Kst):
+        if flush is not None:
+            flush.zero_()
+        ev[k][0].record(stream)
+        K.fused_add_rmsnorm(x, r, w, cfg.eps, out=out)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    times = [ev[k][0].elapsed_time(ev[k][1]) for k in range(Kst)]
+    total_ms = sum(times)
+    kern_ms = statistics.mean(times)
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
+    if sampler:
+        sampler.stop()
+
+    host_in = [t.cpu().pin_memory() for t in (x, r) if t is not None]
+    dev_in = [torch.empty_like(t) for t in (x, r) if t is not None]
+    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2 if r is not None else 1)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step():
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        K.fused_add_rmsnorm(dev_in[0], dev_in[1] if r is not None else None, w, cfg.eps, out=out)
+        host_out[0].copy_(out, non_blocking=True)
+        if r is not None:
+            host_out[1].copy_(dev_in[1], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = x0.elapsed_time(x1)
+    total_ms, kern_ms, e2e_ms = max_over_ranks([total_ms, kern_ms, e2e_ms], dist, device="cuda")
+    if rank == 0:
+        peak, kind = measured_peak()
+        achieved = moved / (kern_ms * 1e-3) / 1e9
+        T = cfg.num_tokens
+        line = {
+            "metric": NORM_METRIC, "value": world * T * Kst / (total_ms * 1e-3), "unit": "rows/s", "n_gpus": world,
+            "steps": Kst, "warmup": args.warmup, "ms_per_step": total_ms / Kst, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, fp32 arithmetic", "data": "synthetic",
+            "config": {"workload": norm_desc(cfg), "seed": args.seed,
+                       "parallelism": f"replicas x{world} (independent rows, no collective)",
+                       "l2": ("flushed between steps (256 MB write, untimed)" if flush is not None else
+                              f"no flush: {moved / 1e6:.0f} MB moved per step, above the 126 MB L2")},
+            "kernel_us": kern_ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "kernel": "fused_add_rmsnorm_kernel",
+                         "peak_source": f"{kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                         "algorithmic_bytes_per_launch": moved,
+                         "bytes_note": "x and residual read, residual and out written, weight read once"},
+            "e2e": {"value": world * T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "rows/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+            "gpu_launches": Kst,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = norm_cpu_baseline(wl, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.component == "block_manager":
         return run_block_manager(args)
+    if args.config in W.NORM_CONFIGS:
+        return run_norm_reference(args) if args.impl == "reference" else run_norm(args)
     if args.config in W.PREFILL_CONFIGS:
         return run_prefill_reference(args) if args.impl == "reference" else run_prefill(args)
     if args.impl == "reference":

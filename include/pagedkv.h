@@ -240,6 +240,29 @@ PKV_API int pkv_paged_attention_prefill(const void *q, const void *k_cache, cons
                                         const float *k_scale, const float *v_scale, int max_q_len, void *out,
                                         int *dev_err, void *stream);
 
+/*
+ * pkv_fused_add_rmsnorm: the residual add and RMSNorm around attention in
+ * one kernel ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section
+ * 核心技术改进 1 "CUDA融合内核：Add+RMSNorm"). For each row t < num_tokens:
+ *   h = x[t] + residual[t]            (fp32; residual[t] <- bf16(h), RNE)
+ *   out[t] = weight * h / sqrt(mean(h^2) + eps)   (fp32, rounded to bf16)
+ * With residual == NULL, h = x[t] and nothing else is written.
+ *
+ *  x, out     [num_tokens][hidden] bf16; out may be x (in place)
+ *  residual   [num_tokens][hidden] bf16, read and overwritten (or NULL)
+ *  weight     [hidden] bf16
+ *
+ * The sum of squares is accumulated in fp32, so rows with elements beyond
+ * about 1e19 in magnitude (far outside any activation range) overflow it.
+ *
+ * Host checks: non-null x / weight / out, 16-byte aligned pointers, hidden a
+ * multiple of 8 in [8, 16384] (above: PKV_ERR_UNSUPPORTED), num_tokens >= 0,
+ * eps >= 0 and finite. No
+ * device-side checks are needed (every index is derived from the sizes).
+ */
+PKV_API int pkv_fused_add_rmsnorm(const void *x, void *residual, const void *weight, void *out, int num_tokens,
+                                  int hidden, float eps, void *stream);
+
 /* Human-readable name of a pkv_status value (static storage). */
 PKV_API const char *pkv_status_string(int status);
 

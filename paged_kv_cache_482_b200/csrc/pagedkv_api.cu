@@ -244,6 +244,20 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+int pkv_fused_add_rmsnorm(const void *x, void *residual, const void *weight, void *out, int num_tokens, int hidden,
+                          float eps, void *stream) {
+    if (!x || !weight || !out || num_tokens < 0) return PKV_ERR_INVALID_ARG;
+    if (hidden < 8 || hidden % 8 != 0) return PKV_ERR_INVALID_ARG;
+    if (hidden > pkv::norm_max_hidden()) return PKV_ERR_UNSUPPORTED;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return PKV_ERR_INVALID_ARG;  // negative, NaN or infinite
+    if (!aligned16(x) || !aligned16(weight) || !aligned16(out) || (residual && !aligned16(residual)))
+        return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    pkv::NormArgs a{x, residual, weight, out, num_tokens, hidden, eps};
+    cudaError_t e = pkv::launch_fused_add_rmsnorm(a, num_sms(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 int pkv_read_device_error(const int *dev_err, void *stream) {
     if (!dev_err) return PKV_ERR_INVALID_ARG;
     int h = 0;

@@ -73,6 +73,19 @@ struct PrefillArgs {
     int *dev_err;
 };
 
+struct NormArgs {
+    const void *x;   // [num_tokens][hidden] bf16
+    void *residual;  // [num_tokens][hidden] bf16, in / out; may be null
+    const void *weight;
+    void *out;
+    int num_tokens;
+    int hidden;
+    float eps;
+};
+
+int norm_max_hidden();
+cudaError_t launch_fused_add_rmsnorm(const NormArgs &a, int num_sms, cudaStream_t stream);
+
 bool prefill_supported(int head_dim, int group);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream);
 

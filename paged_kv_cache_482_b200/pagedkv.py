@@ -11,6 +11,7 @@ The functions mirror ``include/pagedkv.h``:
 * ``plan_decode`` -- ``pkv_plan_decode``
 * ``paged_attention_decode`` -- ``pkv_paged_attention_decode``
 * ``paged_attention_prefill`` -- ``pkv_paged_attention_prefill``
+* ``fused_add_rmsnorm`` -- ``pkv_fused_add_rmsnorm``
 * ``read_device_error`` -- ``pkv_read_device_error``
 """
 
@@ -37,7 +38,7 @@ PKV_CACHE_FP8_E4M3 = 1
 
 EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_paged_attention_decode", "pkv_status_string",
             "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
-            "pkv_paged_attention_prefill")
+            "pkv_paged_attention_prefill", "pkv_fused_add_rmsnorm")
 
 
 class PagedKVError(RuntimeError):
@@ -88,6 +89,8 @@ def load_library(path: str):
     L.pkv_paged_attention_prefill.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i64, f32,
                                               i32, vp, vp, i32, vp, vp, vp]
     L.pkv_paged_attention_prefill.restype = i32
+    L.pkv_fused_add_rmsnorm.argtypes = [vp, vp, vp, vp, i32, i32, f32, vp]
+    L.pkv_fused_add_rmsnorm.restype = i32
     if hasattr(L, "pkv_paged_attention_decode_static_scratch"):
         L.pkv_paged_attention_decode_static_scratch.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
                                                                 i32, i64, f32, i32, vp, vp, i32, i32, vp, vp, vp]
@@ -261,6 +264,26 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, contex
         _ptr(context_lens), S, T, nq, nkv, d, bs, nblk, float(scale), _cache_dtype(k_cache), _ptr(k_scale),
         _ptr(v_scale), int(max_q_len), _ptr(out), _ptr(dev_err), _stream(stream))
     _check(st, "pkv_paged_attention_prefill")
+    return out
+
+
+def fused_add_rmsnorm(x, residual, weight, eps, out=None, stream=None):
+    """Residual add + RMSNorm over the last dimension of ``x`` ``[T, H]`` bf16:
+    ``residual`` (or None) is updated in place to bf16(x + residual) and the
+    normalised rows are returned (in ``out``; ``out=x`` works in place)."""
+    for t, n in ((x, "x"), (weight, "weight")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous bfloat16")
+    if residual is not None and (residual.dtype != torch.bfloat16 or not residual.is_contiguous()
+                                 or residual.shape != x.shape):
+        raise TypeError("residual must be contiguous bfloat16 shaped like x")
+    if x.dim() != 2 or weight.shape != (x.shape[1],):
+        raise ValueError("x must be [T, H] and weight [H]")
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib().pkv_fused_add_rmsnorm(_ptr(x), _ptr(residual), _ptr(weight), _ptr(out), x.shape[0], x.shape[1],
+                                     float(eps), _stream(stream))
+    _check(st, "pkv_fused_add_rmsnorm")
     return out
 
 

@@ -161,3 +161,25 @@ def test_prefill_host_checks(K):
     assert call(mq=0) == K.PKV_ERR_INVALID_ARG
     assert call(nblk=2**31) == K.PKV_ERR_INVALID_ARG
     assert call(S=0) == K.PKV_OK and call(T=0) == K.PKV_OK  # nothing to do, nothing launched
+
+
+def test_norm_host_checks(K):
+    L = K.lib()
+    ok = dict(x=0x10000, r=0x20000, w=0x30000, out=0x40000, T=4, H=4096, eps=1e-6)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.pkv_fused_add_rmsnorm(a["x"], a["r"], a["w"], a["out"], a["T"], a["H"], a["eps"], None)
+
+    assert call(x=None) == K.PKV_ERR_INVALID_ARG
+    assert call(w=None) == K.PKV_ERR_INVALID_ARG
+    assert call(r=0x20008) == K.PKV_ERR_INVALID_ARG  # misaligned
+    assert call(H=12) == K.PKV_ERR_INVALID_ARG  # not a multiple of 8
+    assert call(H=0) == K.PKV_ERR_INVALID_ARG
+    assert call(H=16384 + 8) == K.PKV_ERR_UNSUPPORTED
+    assert call(eps=-1.0) == K.PKV_ERR_INVALID_ARG
+    assert call(eps=float("nan")) == K.PKV_ERR_INVALID_ARG
+    assert call(eps=float("inf")) == K.PKV_ERR_INVALID_ARG
+    assert call(T=-1) == K.PKV_ERR_INVALID_ARG
+    assert call(T=0) == K.PKV_OK  # nothing launched
