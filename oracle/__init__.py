@@ -110,20 +110,38 @@ def new_pool(num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
     return np.full(shape, fill, dtype=np.uint8 if fp8 else np.uint16)
 
 
+def fp8_mode(k_cache, k_scale) -> int:
+    """0: bf16 pool; 1: E4M3 with a scale per KV head ([nkv]); 2: E4M3 with
+    a scale per token and KV head (scale pools [num_blocks, nkv, block_size])."""
+    if k_cache.dtype != np.uint8:
+        return 0
+    return 2 if k_scale is not None and np.ndim(k_scale) == 3 else 1
+
+
+def new_scale_pool(num_blocks: int, num_kv_heads: int, block_size: int):
+    """A per-token scale pool, NaN where no token was stored."""
+    return np.full((num_blocks, num_kv_heads, block_size), np.nan, dtype=np.float32)
+
+
 def store_kvcache(k, v, k_cache, v_cache, slot_mapping, num_blocks, block_size, k_scale=None, v_scale=None,
                   lib=None) -> int:
-    """Write rows of k/v ``[N, nkv, d]`` (bf16) into host pools, in place."""
+    """Write rows of k/v ``[N, nkv, d]`` (bf16) into host pools, in place.
+    With per-token scale pools (numpy, 3-D) the scales are written too."""
     lib = lib or load()
     k = _np(k, np.uint16)
     v = _np(v, np.uint16)
     sm = _np(slot_mapping, np.int32)
     N, nkv, d = k.shape
-    fp8 = k_cache.dtype == np.uint8
-    ks = _np(k_scale, np.float32) if fp8 else None
-    vs = _np(v_scale, np.float32) if fp8 else None
+    mode = fp8_mode(k_cache, k_scale)
+    if mode == 2:
+        assert k_scale.dtype == np.float32 and k_scale.flags.c_contiguous and v_scale.flags.c_contiguous
+        ks, vs = k_scale, v_scale  # written in place
+    else:
+        ks = _np(k_scale, np.float32) if mode else None
+        vs = _np(v_scale, np.float32) if mode else None
     assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
     return lib.orc_store_kvcache(_p(k), _p(v), _p(k_cache), _p(v_cache), _p(sm), N, nkv, d, block_size,
-                                 num_blocks, int(fp8), _p(ks), _p(vs))
+                                 num_blocks, mode, _p(ks), _p(vs))
 
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads, block_size,
@@ -137,7 +155,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, num_
     bt = _np(block_tables, np.int32)
     cl = _np(context_lens, np.int32)
     S, nq, d = q.shape
-    fp8 = k_cache.dtype == np.uint8
+    fp8 = fp8_mode(k_cache, k_scale)
     ks = _np(k_scale, np.float32) if fp8 else None
     vs = _np(v_scale, np.float32) if fp8 else None
     out = np.zeros((S, nq, d), dtype=np.float64)
@@ -164,7 +182,7 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, contex
     T, nq, d = q.shape
     S = cl.shape[0]
     assert cu.shape == (S + 1,)
-    fp8 = k_cache.dtype == np.uint8
+    fp8 = fp8_mode(k_cache, k_scale)
     ks = _np(k_scale, np.float32) if fp8 else None
     vs = _np(v_scale, np.float32) if fp8 else None
     out = np.zeros((T, nq, d), dtype=np.float64)
@@ -201,6 +219,10 @@ def run_workload(wl, num_threads=1, seq_ids=None, lib=None):
     fill = W.CANARY_FP8 if fp8 else W.CANARY_BF16
     kp = new_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, cfg.head_dim, fp8, fill)
     vp = new_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, cfg.head_dim, fp8, fill)
+    ks, vs = wl.k_scale, wl.v_scale
+    if wl.token_scales:
+        ks = new_scale_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size)
+        vs = new_scale_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size)
     if seq_ids is None:
         sub = dict(k_hist=wl.k_hist, v_hist=wl.v_hist, slot_hist=wl.slot_hist, q=wl.q, k_new=wl.k_new,
                    v_new=wl.v_new, slot_new=wl.slot_new, block_tables=wl.block_tables,
@@ -208,12 +230,14 @@ def run_workload(wl, num_threads=1, seq_ids=None, lib=None):
     else:
         sub = W.subset_for_seqs(wl, seq_ids)
     st1 = store_kvcache(sub["k_hist"], sub["v_hist"], kp, vp, sub["slot_hist"], wl.num_blocks, cfg.block_size,
-                        wl.k_scale, wl.v_scale, lib=lib)
+                        ks, vs, lib=lib)
     st2 = store_kvcache(sub["k_new"], sub["v_new"], kp, vp, sub["slot_new"], wl.num_blocks, cfg.block_size,
-                        wl.k_scale, wl.v_scale, lib=lib)
+                        ks, vs, lib=lib)
     out, st3 = paged_attention_decode(sub["q"], kp, vp, sub["block_tables"], sub["context_lens"],
-                                      cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, wl.k_scale,
-                                      wl.v_scale, num_threads=num_threads, lib=lib)
+                                      cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, ks, vs,
+                                      num_threads=num_threads, lib=lib)
+    if wl.token_scales:
+        return out, kp, vp, st1 | st2 | st3, ks, vs
     return out, kp, vp, st1 | st2 | st3
 
 
@@ -227,13 +251,17 @@ def run_prefill_workload(wl, num_threads=1, lib=None):
     fill = W.CANARY_FP8 if fp8 else W.CANARY_BF16
     kp = new_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, cfg.head_dim, fp8, fill)
     vp = new_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, cfg.head_dim, fp8, fill)
-    st1 = store_kvcache(wl.k_hist, wl.v_hist, kp, vp, wl.slot_hist, wl.num_blocks, cfg.block_size, wl.k_scale,
-                        wl.v_scale, lib=lib)
-    st2 = store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.num_blocks, cfg.block_size, wl.k_scale,
-                        wl.v_scale, lib=lib)
+    ks, vs = wl.k_scale, wl.v_scale
+    if wl.token_scales:
+        ks = new_scale_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size)
+        vs = new_scale_pool(wl.num_blocks, cfg.num_kv_heads, cfg.block_size)
+    st1 = store_kvcache(wl.k_hist, wl.v_hist, kp, vp, wl.slot_hist, wl.num_blocks, cfg.block_size, ks, vs, lib=lib)
+    st2 = store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.num_blocks, cfg.block_size, ks, vs, lib=lib)
     out, st3 = paged_attention_prefill(wl.q, kp, vp, wl.block_tables, wl.cu_q_lens, wl.context_lens,
-                                       cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, wl.k_scale, wl.v_scale,
+                                       cfg.num_kv_heads, cfg.block_size, cfg.softmax_scale, ks, vs,
                                        num_threads=num_threads, lib=lib)
+    if wl.token_scales:
+        return out, kp, vp, st1 | st2 | st3, ks, vs
     return out, kp, vp, st1 | st2 | st3
 
 

@@ -33,6 +33,15 @@
  *    nearest E4M3 value, ties to the even code, magnitudes beyond 448 clamped
  *    to 448 (NaN stays NaN);
  *  - FP8 read: code value times the head's scale, both exact in fp64.
+ *  - FP8 with one scale per (token, KV head) (the same page, section 3, does
+ *    not fix the scale granularity; this is the finer of its two readings):
+ *    the store takes the row's largest |x| (over head_dim), s = that / 448
+ *    as one binary32 division, raised to the smallest normal binary32 if it
+ *    falls below it (so an all-zero row has a positive scale), writes s to
+ *    the scale pool [num_blocks][num_kv_heads][block_size] at the token's
+ *    slot and encodes x / s as above; a read multiplies the code by the
+ *    token's own scale. fp8 == 2 selects this mode (fp8 == 1: one scale per
+ *    KV head).
  *  - Add + RMSNorm (same page, section 核心技术改进 1 "CUDA融合内核：Add+RMSNorm":
  *    the residual add and the RMSNorm that follows it, fused): h = x + r,
  *    the residual stream continues as h, and the normalised output is
@@ -51,6 +60,7 @@
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fopenmp -shared -fPIC.
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -132,13 +142,14 @@ static int64_t pool_index(int64_t blk, int h, int off, int i, int nkv, int bs, i
 /*
  * store_kvcache: write token t's K and V rows (all KV heads) into the pool
  * slot slot_mapping[t]; slot -1 is skipped. Pools hold bf16 bit patterns
- * (fp8 == 0) or E4M3 codes (fp8 != 0). A slot beyond the pool is not
+ * (fp8 == 0) or E4M3 codes (fp8 == 1: scales per KV head, read; fp8 == 2:
+ * scale pools per token and KV head, written). A slot beyond the pool is not
  * written and the call reports ORC_ERR_BOUNDS.
  */
 int orc_store_kvcache(const uint16_t *k, const uint16_t *v, void *k_cache, void *v_cache,
                       const int32_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
                       int head_dim, int block_size, int64_t num_blocks, int fp8,
-                      const float *k_scale, const float *v_scale)
+                      float *k_scale, float *v_scale)
 {
     int status = ORC_OK;
     int64_t t;
@@ -158,14 +169,36 @@ int orc_store_kvcache(const uint16_t *k, const uint16_t *v, void *k_cache, void 
         blk = slot / block_size;
         off = (int)(slot % block_size);
         for (h = 0; h < num_kv_heads; ++h) {
+            float ks = 0.0f, vs = 0.0f;
+            if (fp8 == 1) {
+                ks = k_scale[h];
+                vs = v_scale[h];
+            } else if (fp8 == 2) {
+                /* this row's own scales: largest magnitude / 448 */
+                int64_t sidx = ((int64_t)blk * num_kv_heads + h) * block_size + off;
+                float ka = 0.0f, va = 0.0f;
+                for (i = 0; i < head_dim; ++i) {
+                    int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim + i;
+                    ka = fmaxf(ka, fabsf((float)orc_bf16_to_double(k[src])));
+                    va = fmaxf(va, fabsf((float)orc_bf16_to_double(v[src])));
+                }
+                ks = ka / 448.0f;
+                vs = va / 448.0f;
+                if (ks < FLT_MIN)
+                    ks = FLT_MIN;
+                if (vs < FLT_MIN)
+                    vs = FLT_MIN;
+                k_scale[sidx] = ks;
+                v_scale[sidx] = vs;
+            }
             for (i = 0; i < head_dim; ++i) {
                 int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim + i;
                 int64_t dst = pool_index(blk, h, off, i, num_kv_heads, block_size, head_dim);
                 if (fp8) {
                     float kx = (float)orc_bf16_to_double(k[src]);
                     float vx = (float)orc_bf16_to_double(v[src]);
-                    float ky = kx / k_scale[h];
-                    float vy = vx / v_scale[h];
+                    float ky = kx / ks;
+                    float vy = vx / vs;
                     ((uint8_t *)k_cache)[dst] = orc_e4m3_from_float(ky);
                     ((uint8_t *)v_cache)[dst] = orc_e4m3_from_float(vy);
                 } else {
@@ -178,12 +211,22 @@ int orc_store_kvcache(const uint16_t *k, const uint16_t *v, void *k_cache, void 
     return status;
 }
 
-/* One cached element as an exact fp64 value (bf16 bits, or code * scale). */
-static double cache_value(const void *cache, int64_t idx, int fp8, const float *scale, int h)
+/* One cached element as an exact fp64 value (bf16 bits, or code * scale):
+ * element idx of the pool, KV head h, and sidx its token's index in the
+ * per-token scale pools (fp8 == 2). */
+static double cache_value(const void *cache, int64_t idx, int fp8, const float *scale, int h, int64_t sidx)
 {
-    if (fp8)
+    if (fp8 == 1)
         return orc_e4m3_to_double(((const uint8_t *)cache)[idx]) * (double)scale[h];
+    if (fp8 == 2)
+        return orc_e4m3_to_double(((const uint8_t *)cache)[idx]) * (double)scale[sidx];
     return orc_bf16_to_double(((const uint16_t *)cache)[idx]);
+}
+
+/* Index of (block, kv head, offset) in a per-token scale pool. */
+static int64_t scale_index(int64_t blk, int h, int off, int nkv, int bs)
+{
+    return (blk * nkv + h) * bs + off;
 }
 
 /*
@@ -241,7 +284,7 @@ int orc_paged_attention_decode(const uint16_t *q, const void *k_cache, const voi
                 double dot = 0.0;
                 for (i = 0; i < head_dim; ++i) {
                     int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
-                    dot += orc_bf16_to_double(q_h[i]) * cache_value(k_cache, idx, fp8, k_scale, g);
+                    dot += orc_bf16_to_double(q_h[i]) * cache_value(k_cache, idx, fp8, k_scale, g, scale_index(blk, g, off, num_kv_heads, block_size));
                 }
                 score[t] = (double)scale * dot;
                 if (score[t] > m)
@@ -259,7 +302,7 @@ int orc_paged_attention_decode(const uint16_t *q, const void *k_cache, const voi
                 int off = t % block_size;
                 for (i = 0; i < head_dim; ++i) {
                     int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
-                    acc[i] += w[t] * cache_value(v_cache, idx, fp8, v_scale, g);
+                    acc[i] += w[t] * cache_value(v_cache, idx, fp8, v_scale, g, scale_index(blk, g, off, num_kv_heads, block_size));
                 }
             }
             for (i = 0; i < head_dim; ++i)
@@ -344,7 +387,7 @@ int orc_paged_attention_prefill(const uint16_t *q, const void *k_cache, const vo
                     double dot = 0.0;
                     for (i = 0; i < head_dim; ++i) {
                         int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
-                        dot += orc_bf16_to_double(q_h[i]) * cache_value(k_cache, idx, fp8, k_scale, g);
+                        dot += orc_bf16_to_double(q_h[i]) * cache_value(k_cache, idx, fp8, k_scale, g, scale_index(blk, g, off, num_kv_heads, block_size));
                     }
                     score[t] = (double)scale * dot;
                     if (score[t] > m)
@@ -361,7 +404,7 @@ int orc_paged_attention_prefill(const uint16_t *q, const void *k_cache, const vo
                     int off = t % block_size;
                     for (i = 0; i < head_dim; ++i) {
                         int64_t idx = pool_index(blk, g, off, i, num_kv_heads, block_size, head_dim);
-                        acc[i] += w[t] * cache_value(v_cache, idx, fp8, v_scale, g);
+                        acc[i] += w[t] * cache_value(v_cache, idx, fp8, v_scale, g, scale_index(blk, g, off, num_kv_heads, block_size));
                     }
                 }
                 for (i = 0; i < head_dim; ++i)

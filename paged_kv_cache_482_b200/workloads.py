@@ -38,7 +38,8 @@ CANARY_BF16 = 0x7FC0
 CANARY_FP8 = 0x7F
 
 CACHE_BF16 = "bf16"
-CACHE_FP8 = "fp8_e4m3"
+CACHE_FP8 = "fp8_e4m3"  # one fp32 scale per KV head, drawn by the harness
+CACHE_FP8_TOKEN = "fp8_e4m3_token"  # one fp32 scale per (token, KV head), written by the store
 
 
 @dataclass(frozen=True)
@@ -94,6 +95,8 @@ CONFIGS: dict[str, DecodeConfig] = {
         DecodeConfig("qwen3_8b", 1024, 32, 8, 128, 256, 100, 2048),
         DecodeConfig("prefix_shared", 512, 32, 8, 128, 256, 0, 512, prefix_tokens=1024),
         DecodeConfig("long_fp8", 64, 32, 8, 128, 16, 16384, 32768, cache_dtype=CACHE_FP8),
+        # the same long-context step with one scale per (token, KV head)
+        DecodeConfig("long_fp8_token", 64, 32, 8, 128, 16, 16384, 32768, cache_dtype=CACHE_FP8_TOKEN),
     )
 }
 
@@ -126,7 +129,11 @@ class Workload:
 
     @property
     def is_fp8(self) -> bool:
-        return self.cfg.cache_dtype == CACHE_FP8
+        return self.cfg.cache_dtype in (CACHE_FP8, CACHE_FP8_TOKEN)
+
+    @property
+    def token_scales(self) -> bool:
+        return self.cfg.cache_dtype == CACHE_FP8_TOKEN
 
     def kv_tokens(self) -> int:
         return int(self.context_lens.sum().item())
@@ -246,9 +253,18 @@ def generate(cfg: DecodeConfig, seed: int = 0, device: str | torch.device = "cpu
         vmax = torch.where(vmax > 0, vmax, one)
         wl.k_scale = kmax.float() / 448.0
         wl.v_scale = vmax.float() / 448.0
-    elif cfg.cache_dtype != CACHE_BF16:
+    elif cfg.cache_dtype not in (CACHE_BF16, CACHE_FP8_TOKEN):
         raise ValueError(cfg.cache_dtype)
     return wl
+
+
+def scale_pools(num_blocks: int, num_kv_heads: int, block_size: int, device="cpu"):
+    """Per-token scale pools [num_blocks, num_kv_heads, block_size] fp32 for
+    the E4M3 cache with per-token scales, NaN where no token was stored (any
+    read of an unwritten scale poisons the output)."""
+    shape = (num_blocks, num_kv_heads, block_size)
+    return (torch.full(shape, float("nan"), dtype=torch.float32, device=device),
+            torch.full(shape, float("nan"), dtype=torch.float32, device=device))
 
 
 def subset_for_seqs(wl: Workload, seq_ids) -> dict:
@@ -364,6 +380,7 @@ PREFILL_CONFIGS: dict[str, PrefillConfig] = {
         PrefillConfig("prefill_mixed", 4, 32, 8, 128, 256, 0, 3584, 512, 512, decode_seqs=240,
                       decode_hist_lo=100, decode_hist_hi=2047),
         PrefillConfig("prefill_fp8", 8, 32, 8, 128, 16, 1024, 8192, 256, 1024, cache_dtype=CACHE_FP8),
+        PrefillConfig("prefill_fp8_token", 8, 32, 8, 128, 16, 1024, 8192, 256, 1024, cache_dtype=CACHE_FP8_TOKEN),
     )
 }
 
@@ -398,7 +415,11 @@ class PrefillWorkload:
 
     @property
     def is_fp8(self) -> bool:
-        return self.cfg.cache_dtype == CACHE_FP8
+        return self.cfg.cache_dtype in (CACHE_FP8, CACHE_FP8_TOKEN)
+
+    @property
+    def token_scales(self) -> bool:
+        return self.cfg.cache_dtype == CACHE_FP8_TOKEN
 
     @property
     def total_q(self) -> int:
@@ -463,7 +484,7 @@ def generate_prefill(cfg: PrefillConfig, seed: int = 0, device: str | torch.devi
         one = torch.ones_like(kmax)
         wl.k_scale = torch.where(kmax > 0, kmax, one) / 448.0
         wl.v_scale = torch.where(vmax > 0, vmax, one) / 448.0
-    elif cfg.cache_dtype != CACHE_BF16:
+    elif cfg.cache_dtype not in (CACHE_BF16, CACHE_FP8_TOKEN):
         raise ValueError(cfg.cache_dtype)
     return wl
 

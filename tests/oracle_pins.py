@@ -52,12 +52,37 @@ def dequant(x_bf16: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
     return codes.double() * scale.double()[None, :, None]
 
 
+def token_scale(x_bf16: torch.Tensor) -> torch.Tensor:
+    """The per-(token, head) scale of rows [t, nkv, d]: the row's largest
+    magnitude / 448 in binary32, at least the smallest normal binary32."""
+    s = x_bf16.float().abs().amax(dim=-1) / 448.0
+    return torch.clamp(s, min=torch.finfo(torch.float32).tiny)
+
+
+def token_codes(x_bf16: torch.Tensor) -> torch.Tensor:
+    """E4M3 codes of rows [t, nkv, d] under their own per-token scales (torch's cast)."""
+    y = x_bf16.float() / token_scale(x_bf16)[..., None]
+    return y.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+
+
+def dequant_token(x_bf16: torch.Tensor) -> torch.Tensor:
+    return token_codes(x_bf16).double() * token_scale(x_bf16).double()[..., None]
+
+
+def dequant_kv(wl, K, V):
+    """The values a cache holds for logical rows K, V of workload wl."""
+    if getattr(wl, "token_scales", False):
+        return dequant_token(K), dequant_token(V)
+    if wl.is_fp8:
+        return dequant(K, wl.k_scale), dequant(V, wl.v_scale)
+    return K, V
+
+
 def brute_force(wl: W.Workload, i: int) -> np.ndarray:
     """Contiguous softmax attention for sequence i from its logical K/V rows."""
     c = wl.cfg
     K, V = W.logical_kv(wl, i)
-    if wl.is_fp8:
-        K, V = dequant(K, wl.k_scale), dequant(V, wl.v_scale)
+    K, V = dequant_kv(wl, K, V)
     K = np.repeat(K.double().numpy(), c.group, axis=1)  # [ctx, nq, d]
     V = np.repeat(V.double().numpy(), c.group, axis=1)
     q = wl.q[i].double().numpy()  # [nq, d]
@@ -74,7 +99,7 @@ def _assert_close(a, b, tol=TOL, what=""):
 
 
 def _run(wl, lib):
-    out, kp, vp, st = O.run_workload(wl, lib=lib)
+    out, kp, vp, st = O.run_workload(wl, lib=lib)[:4]
     assert st == O.ORC_OK, f"oracle status {st}"
     return out, kp, vp
 
@@ -206,6 +231,43 @@ def pin_dominant_key_returns_its_v(lib):
             _, V = W.logical_kv(wl, i)
             expect = np.repeat(V[p].double().numpy(), c.group, axis=0)
             _assert_close(out[i], expect, what=f"dominant key at {p}")
+
+
+def pin_bruteforce_fp8_token_scales(lib):
+    for c, seed in [
+        (cfg(cache_dtype=W.CACHE_FP8_TOKEN), 15),
+        (cfg(cache_dtype=W.CACHE_FP8_TOKEN, num_q_heads=8, num_kv_heads=2, head_dim=8, ctx_lo=30, ctx_hi=50), 16),
+        (cfg(cache_dtype=W.CACHE_FP8_TOKEN, prefix_tokens=8, ctx_lo=0, ctx_hi=9), 17),
+    ]:
+        wl = W.generate(c, seed)
+        out, _, _ = _run(wl, lib)
+        for i in range(c.num_seqs):
+            _assert_close(out[i], brute_force(wl, i), what=f"fp8 per-token seq {i}")
+
+
+def pin_token_scale_store(lib):
+    """Codes and per-token scales at every stored slot equal torch's: the row
+    amax / 448 in binary32 (floored at the smallest normal) and the E4M3 cast
+    of x / s; an all-zero row gets the floor scale and zero codes; a row
+    spanning the full range keeps its largest element at code 448."""
+    c = cfg(cache_dtype=W.CACHE_FP8_TOKEN, num_seqs=2, ctx_lo=9, ctx_hi=14)
+    wl = W.generate(c, 18)
+    wl.k_hist[0] = 0.0  # an all-zero row (every head)
+    wl.v_hist[1, 0, :] = torch.linspace(-3.0, 1.0, c.head_dim).to(torch.bfloat16)
+    out, kp, vp, st, ks, vs = O.run_workload(wl, lib=lib)
+    assert st == O.ORC_OK and np.all(np.isfinite(out))
+    bs = c.block_size
+    slots = wl.slot_hist.long()
+    blk, off = slots // bs, slots % bs
+    for pool, sp, rows in ((kp, ks, wl.k_hist), (vp, vs, wl.v_hist)):
+        got_codes = pool[blk.numpy(), :, off.numpy(), :]  # [H, nkv, d]
+        want_codes = token_codes(rows).view(torch.uint8).numpy()
+        assert np.array_equal(got_codes, want_codes), "per-token E4M3 codes"
+        got_s = sp[blk.numpy(), :, off.numpy()]
+        assert np.array_equal(got_s, token_scale(rows).numpy()), "per-token scales"
+    assert np.all(ks[blk[0], :, off[0]] == np.float32(torch.finfo(torch.float32).tiny))
+    assert np.all(kp[blk[0], :, off[0]] == 0)
+    assert vp[blk[1], 0, off[1], 0] == 0xFE  # -448: the row's largest magnitude
 
 
 # --------------------------------------------------------------------- store
@@ -359,7 +421,7 @@ def pcfg(**kw) -> W.PrefillConfig:
 
 
 def _run_prefill(wl, lib):
-    out, kp, vp, st = O.run_prefill_workload(wl, lib=lib)
+    out, kp, vp, st = O.run_prefill_workload(wl, lib=lib)[:4]
     assert st == O.ORC_OK, f"oracle status {st}"
     return out, kp, vp
 
@@ -369,8 +431,7 @@ def prefill_brute_force(wl: W.PrefillWorkload, i: int) -> np.ndarray:
     (no pool): query token j of a chunk of c sits at position ctx - c + j."""
     c = wl.cfg
     K, V = W.prefill_logical_kv(wl, i)
-    if wl.is_fp8:
-        K, V = dequant(K, wl.k_scale), dequant(V, wl.v_scale)
+    K, V = dequant_kv(wl, K, V)
     K = np.repeat(K.double().numpy(), c.group, axis=1)  # [ctx, nq, d]
     V = np.repeat(V.double().numpy(), c.group, axis=1)
     a, b = int(wl.cu_q_lens[i]), int(wl.cu_q_lens[i + 1])
@@ -390,6 +451,7 @@ def pin_prefill_bruteforce(lib):
         (pcfg(num_q_heads=8, num_kv_heads=1, head_dim=8, block_size=8, hist_hi=30, chunk_lo=5, chunk_hi=20), 22),
         (pcfg(num_q_heads=3, num_kv_heads=3, head_dim=12, block_size=16, hist_lo=15, hist_hi=33), 23),
         (pcfg(cache_dtype=W.CACHE_FP8, chunk_hi=12), 24),
+        (pcfg(cache_dtype=W.CACHE_FP8_TOKEN, chunk_hi=12, hist_hi=30), 31),
         (pcfg(num_seqs=2, decode_seqs=3, decode_hist_lo=1, decode_hist_hi=20), 25),
     ]:
         wl = W.generate_prefill(c, seed)
@@ -579,6 +641,8 @@ ALL_PINS = [
     pin_prefill_errors,
     pin_bruteforce_bf16,
     pin_bruteforce_fp8,
+    pin_bruteforce_fp8_token_scales,
+    pin_token_scale_store,
     pin_permutation_invariance,
     pin_prefix_shared_equals_duplicated,
     pin_single_token_returns_v,

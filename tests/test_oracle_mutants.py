@@ -32,13 +32,13 @@ MUTANTS = [
     ("not normalised", "acc[i] / z;", "acc[i];", 0),
     ("last token dropped", "for (t = 0; t < ctx; ++t) {\n                w[t]",
      "for (t = 0; t < ctx - 1; ++t) {\n                w[t]", 0),
-    ("v read from k", "cache_value(v_cache, idx, fp8, v_scale, g)", "cache_value(k_cache, idx, fp8, v_scale, g)", 0),
+    ("v read from k", "cache_value(v_cache, idx, fp8, v_scale, g,", "cache_value(k_cache, idx, fp8, v_scale, g,", 0),
     ("q head of kv head", "q + ((int64_t)s * num_q_heads + h) * head_dim", "q + ((int64_t)s * num_q_heads + g) * head_dim", 0),
     ("layout transposed", "((blk * nkv + h) * bs + off)", "((blk * bs + off) * nkv + h)", 0),
     ("slot zero skipped", "if (slot < 0)", "if (slot <= 0)", 0),
     ("k and v swapped", "((uint16_t *)k_cache)[dst] = k[src];", "((uint16_t *)k_cache)[dst] = v[src];", 0),
     ("fp8 scale unused on read", "* (double)scale[h];", ";", 0),
-    ("fp8 scale multiplies on store", "float ky = kx / k_scale[h];", "float ky = kx * k_scale[h];", 0),
+    ("fp8 scale multiplies on store", "float ky = kx / ks;", "float ky = kx * ks;", 0),
     ("fp8 ties away", "(d_hi == d_lo && (lo & 1))", "(d_hi == d_lo)", 0),
     ("fp8 saturation drops sign", "return sign | 0x7E;", "return 0x7E;", 0),
     ("fp8 subnormal exponent", "ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)", 0),
@@ -59,7 +59,16 @@ MUTANTS = [
     ("prefill decreasing offsets accepted", "if (cu_q_lens[s + 1] < cu_q_lens[s])", "if (0)", 0),
     ("prefill max not subtracted", "w[t] = exp(score[t] - m);", "w[t] = exp(score[t]);", 1),
     ("prefill not normalised", "acc[i] / z;", "acc[i];", 1),
-    ("prefill v read from k", "cache_value(v_cache, idx, fp8, v_scale, g)", "cache_value(k_cache, idx, fp8, v_scale, g)", 1),
+    ("prefill v read from k", "cache_value(v_cache, idx, fp8, v_scale, g,", "cache_value(k_cache, idx, fp8, v_scale, g,", 1),
+    # E4M3 with per-token scales
+    ("token scale read per head", "        return orc_e4m3_to_double(((const uint8_t *)cache)[idx]) * (double)scale[sidx];",
+     "        return orc_e4m3_to_double(((const uint8_t *)cache)[idx]) * (double)scale[h];", 0),
+    ("token scale amax without abs", "ka = fmaxf(ka, fabsf((float)orc_bf16_to_double(k[src])));",
+     "ka = fmaxf(ka, (float)orc_bf16_to_double(k[src]));", 0),
+    ("token scale 240", "ks = ka / 448.0f;", "ks = ka / 240.0f;", 0),
+    ("token scale no floor", "if (ks < FLT_MIN)\n                    ks = FLT_MIN;", "if (0)\n                    ks = FLT_MIN;", 0),
+    ("token scale wrong slot", "return (blk * nkv + h) * bs + off;", "return (blk * nkv + h) * bs + (off + 1) % bs;", 0),
+    ("token scale v from k", "vs = va / 448.0f;", "vs = ka / 448.0f;", 0),
     # add + RMSNorm
     ("rmsnorm eps outside sqrt", "inv = 1.0 / sqrt(ss / hidden + eps);", "inv = 1.0 / (sqrt(ss / hidden) + eps);", 0),
     ("rmsnorm sum not mean", "inv = 1.0 / sqrt(ss / hidden + eps);", "inv = 1.0 / sqrt(ss + eps);", 0),
