@@ -113,7 +113,9 @@ def algorithmic_bytes(wl: W.Workload) -> dict:
     c = wl.cfg
     esize = 1 if wl.is_fp8 else 2
     ctx = wl.context_lens.long().cpu()
-    kv = int(ctx.sum()) * c.num_kv_heads * c.head_dim * esize * 2
+    # per-token E4M3 scales: 4 bytes for K and 4 for V per (token, KV head)
+    row = c.head_dim * esize + (4 if wl.token_scales else 0)
+    kv = int(ctx.sum()) * c.num_kv_heads * row * 2
     qo = 2 * c.num_seqs * c.num_q_heads * c.head_dim * 2
     nb = int(((ctx + c.block_size - 1) // c.block_size).sum())
     meta = 4 * nb + 4 * c.num_seqs
@@ -121,7 +123,7 @@ def algorithmic_bytes(wl: W.Workload) -> dict:
         # shared prefix blocks are read once from HBM (they stay in L2)
         shared_tok = c.prefix_tokens
         own = int((ctx - c.prefix_tokens).sum())
-        unique_kv = (shared_tok + own) * c.num_kv_heads * c.head_dim * esize * 2
+        unique_kv = (shared_tok + own) * c.num_kv_heads * row * 2
     else:
         unique_kv = kv
     return dict(kv=kv, unique_kv=unique_kv, q_out=qo, meta=meta, total=kv + qo + meta,
@@ -258,6 +260,9 @@ def oracle_sample_runner(wl: W.Workload, ids, threads: int):
     vp = O.new_pool(nblk, c.num_kv_heads, c.block_size, c.head_dim, wl.is_fp8, fill)
     ks = wl.k_scale.cpu() if wl.k_scale is not None else None
     vs = wl.v_scale.cpu() if wl.v_scale is not None else None
+    if wl.token_scales:
+        ks = O.new_scale_pool(nblk, c.num_kv_heads, c.block_size)
+        vs = O.new_scale_pool(nblk, c.num_kv_heads, c.block_size)
     O.store_kvcache(sub["k_hist"], sub["v_hist"], kp, vp, sub["slot_hist"], nblk, c.block_size, ks, vs)
 
     def step():
@@ -471,6 +476,9 @@ def prefill_oracle_sampler(wl, threads: int):
     vp = O.new_pool(wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim, wl.is_fp8, fill)
     ks = wl.k_scale.cpu() if wl.k_scale is not None else None
     vs = wl.v_scale.cpu() if wl.v_scale is not None else None
+    if wl.token_scales:
+        ks = O.new_scale_pool(wl.num_blocks, c.num_kv_heads, c.block_size)
+        vs = O.new_scale_pool(wl.num_blocks, c.num_kv_heads, c.block_size)
     O.store_kvcache(wl.k_hist.cpu(), wl.v_hist.cpu(), kp, vp, wl.slot_hist.cpu(), wl.num_blocks, c.block_size, ks, vs)
     O.store_kvcache(wl.k_new.cpu(), wl.v_new.cpu(), kp, vp, wl.slot_new.cpu(), wl.num_blocks, c.block_size, ks, vs)
     q, bt = wl.q.cpu(), wl.block_tables.cpu()
@@ -576,6 +584,8 @@ def run_prefill(args):
         kp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
         vp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if wl.token_scales:  # one scale per (token, KV head), written by the store
+        wl.k_scale, wl.v_scale = W.scale_pools(wl.num_blocks, c.num_kv_heads, c.block_size, device="cuda")
     K.store_kvcache(wl.k_hist, wl.v_hist, kp, vp, wl.slot_hist, wl.k_scale, wl.v_scale, err)
     cu = wl.cu_q_lens.cpu().long()
     mq = int((cu[1:] - cu[:-1]).max())
@@ -900,6 +910,8 @@ def main():
     else:
         kp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
         vp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    if wl.token_scales:  # one scale per (token, KV head), written by the store
+        wl.k_scale, wl.v_scale = W.scale_pools(wl.num_blocks, c.num_kv_heads, c.block_size, device="cuda")
     H = wl.k_hist.shape[0]
     for i in range(0, H, 1 << 20):
         j = min(H, i + (1 << 20))

@@ -27,6 +27,14 @@
  *    writes before the decode on the same stream.
  *  - FP8: code = E4M3(x / scale[h]) with one IEEE fp32 division, round to
  *    nearest even, saturating at +-448; value = code * scale[h].
+ *  - FP8 with per-token scales (PKV_CACHE_FP8_E4M3_TOKEN; the page leaves
+ *    the scale granularity open): k_scale / v_scale are scale pools
+ *    [num_blocks][num_kv_heads][block_size] fp32, one scale per cached
+ *    (token, KV head) row. store_kvcache computes s = max(amax / 448, the
+ *    smallest normal fp32) for each row it writes (amax: the row's largest
+ *    |x|; one IEEE division), writes s at the row's slot and the codes
+ *    E4M3(x / s); a read is code * s of its own row. The scale pools need no
+ *    initialisation: only written rows are read.
  *
  * Ownership and execution. The caller owns every buffer (device memory unless
  * stated) and keeps it alive until the stream work finishes. The library
@@ -72,7 +80,8 @@ typedef enum {
 
 typedef enum {
     PKV_CACHE_BF16 = 0,
-    PKV_CACHE_FP8_E4M3 = 1
+    PKV_CACHE_FP8_E4M3 = 1,      /* one fp32 scale per KV head: [num_kv_heads] */
+    PKV_CACHE_FP8_E4M3_TOKEN = 2 /* one fp32 scale per (token, KV head): scale pools */
 } pkv_cache_dtype;
 
 /* Bits of the device error word. */
@@ -88,7 +97,10 @@ typedef enum {
  *  k, v          [num_tokens][num_kv_heads][head_dim] bf16, contiguous
  *  k_cache, ...  pools as above; bf16 (copy) or E4M3 (quantised)
  *  slot_mapping  [num_tokens] int32
- *  k_scale, ...  [num_kv_heads] fp32, FP8 only (NULL for bf16)
+ *  k_scale, ...  FP8 only (NULL for bf16): [num_kv_heads] fp32, read; or, for
+ *                PKV_CACHE_FP8_E4M3_TOKEN, the scale pools, written at each
+ *                stored row's slot (head_dim / 8 must then be a power of two
+ *                up to 32, i.e. head_dim 8 .. 256)
  *
  * Host checks: non-null pointers, 16-byte aligned k/v/caches, head_dim a
  * multiple of 8, sizes >= 1 (num_tokens may be 0: nothing is launched and no
@@ -99,7 +111,7 @@ typedef enum {
 PKV_API int pkv_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache,
                       const int32_t *slot_mapping, int num_tokens, int num_kv_heads,
                       int head_dim, int block_size, int64_t num_blocks, int cache_dtype,
-                      const float *k_scale, const float *v_scale, int *dev_err, void *stream);
+                      float *k_scale, float *v_scale, int *dev_err, void *stream);
 
 /*
  * Split-K plan of a decode call. A sequence's tokens are cut into partitions

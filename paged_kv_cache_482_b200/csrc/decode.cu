@@ -11,7 +11,7 @@ namespace pkv {
 
 namespace {
 
-template <int D, int G, bool FP8>
+template <int D, int G, bool FP8, bool TS>
 cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
     using T = DecodeTraits<D, G, FP8>;
 #ifdef PKV_DECODE_MIN_BLOCKS
@@ -19,7 +19,7 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
 #else
     constexpr int MINB = (G <= 4) ? 4 : 2;  // 4 x 128 threads at 128 registers fill the register file
 #endif
-    auto kern = paged_decode_kernel<D, G, FP8, MINB>;
+    auto kern = paged_decode_kernel<D, G, FP8, MINB, TS>;
 
     // The opt-in to more than 48 KB of dynamic shared memory is a property of
     // the function on a device; set it once per device.
@@ -54,13 +54,13 @@ int tile_of(int group) {
     }
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool TS = false>
 cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_one<D, 1, FP8>(p, stream);
-        case 2: return launch_one<D, 2, FP8>(p, stream);
-        case 4: return launch_one<D, 4, FP8>(p, stream);
-        case 8: return launch_one<D, 8, FP8>(p, stream);
+        case 1: return launch_one<D, 1, FP8, TS>(p, stream);
+        case 2: return launch_one<D, 2, FP8, TS>(p, stream);
+        case 4: return launch_one<D, 4, FP8, TS>(p, stream);
+        case 8: return launch_one<D, 8, FP8, TS>(p, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -103,6 +103,11 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.out = static_cast<__nv_bfloat16 *>(a.out);
     p.dev_err = a.dev_err;
     const int group = a.num_q_heads / a.num_kv_heads;
+    if (a.fp8 && a.token_scales) {
+        if (a.head_dim == 128) return launch_group<128, true, true>(group, p, stream);
+        if (a.head_dim == 64) return launch_group<64, true, true>(group, p, stream);
+        return cudaErrorInvalidValue;
+    }
     if (a.head_dim == 128)
         return a.fp8 ? launch_group<128, true>(group, p, stream) : launch_group<128, false>(group, p, stream);
     if (a.head_dim == 64)

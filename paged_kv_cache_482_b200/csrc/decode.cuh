@@ -172,7 +172,10 @@ struct ReduceScatter {
     }
 };
 
-template <int D, int G, bool FP8, int MIN_BLOCKS>
+// TS: E4M3 cache with one scale per (token, KV head) in scale pools shaped
+// like the cache without head_dim (p.k_scale / p.v_scale); each lane loads
+// the scales of the row its score belongs to, one tile ahead of use.
+template <int D, int G, bool FP8, int MIN_BLOCKS, bool TS = false>
 __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     paged_decode_kernel(const DecodeParams p) {
     using T = DecodeTraits<D, G, FP8>;
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
                 const __half2 h = __floats2half2_rn(ldexpf(bf16lo(qw[hs][i]), k), ldexpf(bf16hi(qw[hs][i]), k));
                 qw[hs][i] = *reinterpret_cast<const uint32_t *>(&h);
             }
-        score_scale = ldexpf(p.qk_scale_log2 * __ldg(p.k_scale + kvh), -k);
+        score_scale = ldexpf(TS ? p.qk_scale_log2 : p.qk_scale_log2 * __ldg(p.k_scale + kvh), -k);
     }
 
     float acc[G][8];
@@ -411,11 +414,27 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
             }
         }
     };
+    // Per-token scales of this lane's row of tile j (TS only): K scale
+    // multiplies the score, V scale the weight that P * V uses (l sums the
+    // unscaled weights). Rows past the end get 0 (their weight is 0 anyway).
+    auto tok_scales = [&](int j, float &ks, float &vs) {
+        ks = 0.f;
+        vs = 0.f;
+        if constexpr (TS) {
+            const int a = start + j * TILE + row0 + my_row;
+            if (a < end) {
+                const long long phys = ids[(a >> p.log2_block_size) - first_blk];
+                const long long idx = (phys * p.num_kv_heads + kvh) * p.block_size + (a & (p.block_size - 1));
+                ks = __ldg(p.k_scale + idx);
+                vs = __ldg(p.v_scale + idx);
+            }
+        }
+    };
     // Scores of tile j -> p (to this warp's p buffer) and the rescale factor
     // of head my_h; returns whether any head of the warp changed its max.
-    auto softmax = [&](int j, float (&sc)[T::kNV], float &alpha) {
+    auto softmax = [&](int j, float (&sc)[T::kNV], float &alpha, float ks, float vs) {
         ReduceScatter<T::kNV, LPT / 2>::run(sc);
-        sc[0] *= score_scale;
+        sc[0] *= TS ? score_scale * ks : score_scale;
         const int n_valid = min(TILE, end - (start + j * TILE));
         const float sv = my_row < n_valid - row0 ? sc[0] : -CUDART_INF_F;
         float tmax = sv;
@@ -427,7 +446,8 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         const float pr = fast_exp2(sv - mref);
         l = fmaf(l, alpha, pr);
         m = m_new;
-        if (canon) reinterpret_cast<float2 *>(pbuf)[(j & 1) * ROWS * G + my_row * G + my_h] = make_float2(pr, pr);
+        const float pw = TS ? pr * vs : pr;
+        if (canon) reinterpret_cast<float2 *>(pbuf)[(j & 1) * ROWS * G + my_row * G + my_h] = make_float2(pw, pw);
     };
     // P * V of the tile in V stage sv (p buffer half pj) into the
     // accumulators; rows past the end have p = 0.
@@ -473,13 +493,15 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     {
         float sc[T::kNV];
         float alpha;
+        float ks, vs;  // this lane's row scales (TS) for the tile being scored
         int sk = 0, rk = 0, sv = 0, rv = 0;
         if (!mbar_wait(&full_k[0], 0)) ok = false;
         if (ok) {
+            tok_scales(0, ks, vs);
             qk(0, sc);
             __syncwarp();
             release(0, 0, -1, 0);
-            softmax(0, sc, alpha);  // acc is still zero: nothing to rescale
+            softmax(0, sc, alpha, ks, vs);  // acc is still zero: nothing to rescale
             __syncwarp();
             if (++sk == STAGES) { sk = 0; ++rk; }
         }
@@ -488,8 +510,9 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
                 ok = false;
                 break;
             }
+            tok_scales(j, ks, vs);
             qk(sk, sc);
-            softmax(j, sc, alpha);
+            softmax(j, sc, alpha, ks, vs);
             pv(sv, (j - 1) & 1);
             __syncwarp();
             release(j, sk, j - 1, sv);
@@ -558,7 +581,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
             L += merge_l[w * G + h] * e;
         }
         float post = 1.f / L;
-        if constexpr (FP8) post *= __ldg(p.v_scale + kvh);
+        if constexpr (FP8 && !TS) post *= __ldg(p.v_scale + kvh);
         for (int w = 0; w < NCW; ++w) merge_w[w * G + h] *= post;
         if (!single) {
             float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * 2;

@@ -17,6 +17,7 @@ constexpr int kMaxPartitions = 1024;        // the reduce kernel's limit
 constexpr int kMinAutoPartitionTokens = 1024;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_dtype(int d) { return d == PKV_CACHE_BF16 || d == PKV_CACHE_FP8_E4M3 || d == PKV_CACHE_FP8_E4M3_TOKEN; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 int num_sms() {
@@ -39,9 +40,9 @@ int check_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, i
                 int max_context_len, int cache_dtype) {
     if (num_seqs < 0 || num_q_heads < 1 || num_kv_heads < 1 || max_context_len < 1) return PKV_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (cache_dtype != PKV_CACHE_BF16 && cache_dtype != PKV_CACHE_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
     if (!pow2(block_size) || block_size < 8 || block_size > 1024) return PKV_ERR_INVALID_ARG;
-    if (pkv::decode_tile_tokens(head_dim, num_q_heads / num_kv_heads, cache_dtype == PKV_CACHE_FP8_E4M3) == 0)
+    if (pkv::decode_tile_tokens(head_dim, num_q_heads / num_kv_heads, cache_dtype != PKV_CACHE_BF16) == 0)
         return PKV_ERR_UNSUPPORTED;
     return PKV_OK;
 }
@@ -50,7 +51,7 @@ int make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int
               int cache_dtype, int request, pkv_decode_plan *plan) {
     int st = check_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, cache_dtype);
     if (st != PKV_OK) return st;
-    const bool fp8 = cache_dtype == PKV_CACHE_FP8_E4M3;
+    const bool fp8 = cache_dtype != PKV_CACHE_BF16;
     const int tile = pkv::decode_tile_tokens(head_dim, num_q_heads / num_kv_heads, fp8);
     // A partition may span at most this many blocks (ids staged on chip); a
     // partition of pt tokens spans at most pt / block_size + 1 blocks.
@@ -114,19 +115,22 @@ const char *pkv_status_string(int status) {
 
 int pkv_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache, const int32_t *slot_mapping,
                       int num_tokens, int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
-                      int cache_dtype, const float *k_scale, const float *v_scale, int *dev_err, void *stream) {
+                      int cache_dtype, float *k_scale, float *v_scale, int *dev_err, void *stream) {
     if (num_tokens < 0 || num_kv_heads < 1 || head_dim < 8 || head_dim % 8 != 0 || block_size < 1 ||
         num_blocks < 1)
         return PKV_ERR_INVALID_ARG;
-    if (cache_dtype != PKV_CACHE_BF16 && cache_dtype != PKV_CACHE_FP8_E4M3) return PKV_ERR_INVALID_ARG;
-    const bool fp8 = cache_dtype == PKV_CACHE_FP8_E4M3;
+    if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
+    // per-token scales: the lanes of one row reduce its amax together
+    if (cache_dtype == PKV_CACHE_FP8_E4M3_TOKEN && (!pow2(head_dim / 8) || head_dim > 256))
+        return PKV_ERR_UNSUPPORTED;
+    const bool fp8 = cache_dtype != PKV_CACHE_BF16;
     if (num_tokens == 0) return PKV_OK;  // no rows to read: k, v, slot_mapping may be NULL
     if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
     if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
     cudaError_t e = pkv::launch_store_kvcache(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
-                                              head_dim, block_size, num_blocks, fp8, k_scale, v_scale, dev_err,
-                                              num_sms(), static_cast<cudaStream_t>(stream));
+                                              head_dim, block_size, num_blocks, cache_dtype, k_scale, v_scale,
+                                              dev_err, num_sms(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -148,7 +152,7 @@ int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v
     int st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, cache_dtype,
                        partition_request, &plan);
     if (st != PKV_OK) return st;
-    const bool fp8 = cache_dtype == PKV_CACHE_FP8_E4M3;
+    const bool fp8 = cache_dtype != PKV_CACHE_BF16;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PKV_ERR_INVALID_ARG;
     if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
@@ -177,6 +181,7 @@ int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v
     a.num_blocks = num_blocks;
     a.scale = scale;
     a.fp8 = fp8;
+    a.token_scales = cache_dtype == PKV_CACHE_FP8_E4M3_TOKEN;
     a.k_scale = k_scale;
     a.v_scale = v_scale;
     a.max_context_len = max_context_len;
@@ -204,10 +209,10 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
                                 int *dev_err, void *stream) {
     if (num_seqs < 0 || total_q < 0 || num_q_heads < 1 || num_kv_heads < 1) return PKV_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (cache_dtype != PKV_CACHE_BF16 && cache_dtype != PKV_CACHE_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
     if (!pow2(block_size) || block_size < 8 || block_size > 1024) return PKV_ERR_INVALID_ARG;
     if (!pkv::prefill_supported(head_dim, num_q_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
-    const bool fp8 = cache_dtype == PKV_CACHE_FP8_E4M3;
+    const bool fp8 = cache_dtype != PKV_CACHE_BF16;
     if (!q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens || !out)
         return PKV_ERR_INVALID_ARG;
     if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
@@ -234,6 +239,7 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
     a.num_blocks = num_blocks;
     a.scale = scale;
     a.fp8 = fp8;
+    a.token_scales = cache_dtype == PKV_CACHE_FP8_E4M3_TOKEN;
     a.k_scale = k_scale;
     a.v_scale = v_scale;
     a.max_q_len = max_q_len;

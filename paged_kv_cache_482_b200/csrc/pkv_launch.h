@@ -9,8 +9,8 @@ namespace pkv {
 
 cudaError_t launch_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache,
                                  const int32_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
-                                 int block_size, int64_t num_blocks, bool fp8, const float *k_scale,
-                                 const float *v_scale, int *dev_err, int num_sms, cudaStream_t stream);
+                                 int block_size, int64_t num_blocks, int mode, float *k_scale, float *v_scale,
+                                 int *dev_err, int num_sms, cudaStream_t stream);
 
 // Everything the decode kernels need, resolved by the host layer.
 struct DecodeArgs {
@@ -29,6 +29,7 @@ struct DecodeArgs {
     int64_t num_blocks;
     float scale;
     bool fp8;
+    bool token_scales;  // E4M3 with scale pools [num_blocks][num_kv_heads][block_size]
     const float *k_scale;
     const float *v_scale;
     int max_context_len;
@@ -66,6 +67,7 @@ struct PrefillArgs {
     int64_t num_blocks;
     float scale;
     bool fp8;
+    bool token_scales;  // E4M3 with scale pools [num_blocks][num_kv_heads][block_size]
     const float *k_scale;
     const float *v_scale;
     int max_q_len;

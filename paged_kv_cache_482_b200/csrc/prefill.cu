@@ -30,9 +30,13 @@
 //      MN-major straight from its row layout) into a second tensor-memory
 //      buffer, which the threads fold into fp32 register accumulators with
 //      the rescale factor.
-// The FP8 cache is dequantised to bf16 while it is staged (both MMA operands
-// are bf16); k_scale folds into the softmax scale and v_scale into the final
-// normalisation.
+// The FP8 cache is widened to bf16 while it is staged (exact: every E4M3
+// value is a bf16 value; both MMA operands are bf16). With one scale per KV
+// head, k_scale folds into the softmax scale and v_scale into the final
+// normalisation; with one scale per token, the tile's 64 K and 64 V scales
+// are staged next to it and multiply S column by column and P column by
+// column (in fp32, before P is rounded to bf16; l then sums the unscaled
+// weights).
 //
 // Shared-memory operand layout (all four operands): [head_dim / 64 or
 // 128 / 64 column blocks][rows][128 bytes], the 16-byte chunk c of row r
@@ -81,7 +85,8 @@ struct Layout {
     static constexpr uint32_t kP = kK0 + 2 * kBufStride;
     static constexpr uint32_t kBar = kP + (kPInK ? 0 : kPBytes);  // 4 mbarriers, TMEM address
     static constexpr uint32_t kTable = kBar + 64;                  // the sequence's first block ids
-    static constexpr uint32_t kBytes = kTable + kTableCap * 4;
+    static constexpr uint32_t kScales = kTable + kTableCap * 4;    // per-token scales: [2 buffers][K, V][kBN]
+    static constexpr uint32_t kBytes = kScales + 2 * 2 * kBN * 4;
     static constexpr uint32_t kAlloc = (kBytes + 1024 > kMinSmem) ? kBytes + 1024 : kMinSmem;  // + base alignment
 };
 
@@ -213,9 +218,22 @@ __device__ __forceinline__ uint32_t swz(int rows, int r, int c16) {
 // Stage KV tile j (logical tokens j*kBN ..) of KV head kh into one K/V buffer.
 // Tokens at or past kv_end are zero-filled; their scores are masked anyway
 // and zeros keep P V finite.
-template <int D, bool FP8>
+template <int D, bool FP8, bool TS = false>
 __device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const BlockIds &table, int kh, int j, int kv_end,
-                                             int log2_bs, uint32_t sk, uint32_t sv) {
+                                             int log2_bs, uint32_t sk, uint32_t sv, float *scales = nullptr) {
+    if constexpr (TS) {
+        // K scales of the tile's tokens in scales[0..kBN), V scales in [kBN, 2 kBN); 0 past the end
+        const int t = threadIdx.x % kBN;
+        const bool is_v = threadIdx.x >= kBN;
+        const int pos = j * kBN + t;
+        float sc = 0.0f;
+        if (pos < kv_end) {
+            const int64_t blk = table[pos >> log2_bs];
+            const int64_t idx = (blk * a.num_kv_heads + kh) * a.block_size + (pos & (a.block_size - 1));
+            sc = __ldg((is_v ? a.v_scale : a.k_scale) + idx);
+        }
+        scales[threadIdx.x] = sc;
+    }
     constexpr int kChunks = D / 8;             // 16-byte chunks per bf16 row
     constexpr int kTokPerPass = kThreads / kChunks;
     const int c16 = threadIdx.x % kChunks;
@@ -282,7 +300,7 @@ __device__ __forceinline__ void tma_kv_tile(const CUtensorMap *mk, const CUtenso
     }
 }
 
-template <int D, int G, bool FP8>
+template <int D, int G, bool FP8, bool TS = false>
 __global__ void __launch_bounds__(kThreads, 2)
     paged_prefill_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
                          const __grid_constant__ CUtensorMap map_v) {
@@ -368,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t sq = base + L::kQ;
     auto kbuf = [&](int j) { return base + L::kK0 + static_cast<uint32_t>(j & 1) * L::kBufStride; };
+    auto sbuf = [&](int j) { return reinterpret_cast<float *>(sm + L::kScales) + (j & 1) * 2 * kBN; };
     auto vbuf = [&](int j) { return base + L::kV0 + static_cast<uint32_t>(j & 1) * L::kBufStride; };
 
     // S = Q K_j^T, issued by thread 0 once tile j's K is in shared memory
@@ -396,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
     if constexpr (FP8) {
-        load_kv_tile<D, FP8>(a, table, kh, 0, kv_end, log2_bs, kbuf(0), vbuf(0));
+        load_kv_tile<D, FP8, TS>(a, table, kh, 0, kv_end, log2_bs, kbuf(0), vbuf(0), sbuf(0));
     } else if (tid == 0) {
         tma_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, 0, kv_end, kbuf(0), vbuf(0),
                        bar_kv);
@@ -415,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (FP8 || mbar_wait(bar_kv, 0)) issue_s(0);
     }
 
-    const float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
+    const float sl2 = a.scale * kLog2e * ((FP8 && !TS) ? __ldg(a.k_scale + kh) : 1.0f);
     float m_run = -INFINITY, l_run = 0.0f;
 
     for (int j = 0; j < n_tiles; ++j) {
@@ -435,12 +454,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int kv0 = j * kBN;
         const bool masked = kv0 + kBN - 1 > p_first;  // some row sees a future or absent token
         float x[kBN];
+        const float *tsc = sbuf(j);  // this tile's per-token scales (TS)
 #pragma unroll
         for (int ch = 0; ch < kBN / 32; ++ch) {
             float v[32];
             tmem_ld32(tmem_s + lane_base + ch * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[ch * 32 + i] = v[i] * sl2;
+            for (int i = 0; i < 32; ++i) x[ch * 32 + i] = TS ? v[i] * (sl2 * tsc[ch * 32 + i]) : v[i] * sl2;
         }
         if (masked) {
 #pragma unroll
@@ -468,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (j + 1 < n_tiles) {
             if constexpr (FP8) {
-                load_kv_tile<D, FP8>(a, table, kh, j + 1, kv_end, log2_bs, kbuf(j + 1), vbuf(j + 1));
+                load_kv_tile<D, FP8, TS>(a, table, kh, j + 1, kv_end, log2_bs, kbuf(j + 1), vbuf(j + 1), sbuf(j + 1));
             } else if (tid == 0 && j + 1 >= 2) {  // tiles 0 and 1 were issued up front
                 tma_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, j + 1, kv_end,
                                kbuf(j + 1), vbuf(j + 1), bar_kv + ((j + 1) & 1));
@@ -508,8 +528,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 const int i0 = c16 * 8 + 2 * h;
-                w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
-                l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
+                if constexpr (TS) {
+                    const float p0 = fast_exp2(x[i0] - m_run), p1 = fast_exp2(x[i0 + 1] - m_run);
+                    w[h] = pack_bf16(p0 * tsc[kBN + i0], p1 * tsc[kBN + i0 + 1]);
+                    l4[h] += p0 + p1;
+                } else {
+                    w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
+                    l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
+                }
             }
             st_shared16(sp + swz(kRows, tid, c16), make_uint4(w[0], w[1], w[2], w[3]));
         }
@@ -566,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else {
         tc_fence_after();
-        const float inv = (FP8 ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
+        const float inv = ((FP8 && !TS) ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
             float v[32];
@@ -626,7 +652,7 @@ bool make_pool_map(CUtensorMap *map, const void *pool, const PrefillArgs &a) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int G, bool FP8>
+template <int D, int G, bool FP8, bool TS>
 cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int TQ = kRows / G;
     const int tiles = (a.max_q_len + TQ - 1) / TQ;
@@ -643,7 +669,7 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
             return cudaErrorInvalidConfiguration;
         if (!make_pool_map(&mk, a.k_cache, a) || !make_pool_map(&mv, a.v_cache, a)) return cudaErrorInvalidValue;
     }
-    auto kern = paged_prefill_kernel<D, G, FP8>;
+    auto kern = paged_prefill_kernel<D, G, FP8, TS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(Layout<D>::kAlloc));
     if (e != cudaSuccess) return e;
@@ -652,13 +678,13 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool TS = false>
 cudaError_t launch_d(const PrefillArgs &a, int g, cudaStream_t stream) {
     switch (g) {
-        case 1: return launch_t<D, 1, FP8>(a, stream);
-        case 2: return launch_t<D, 2, FP8>(a, stream);
-        case 4: return launch_t<D, 4, FP8>(a, stream);
-        case 8: return launch_t<D, 8, FP8>(a, stream);
+        case 1: return launch_t<D, 1, FP8, TS>(a, stream);
+        case 2: return launch_t<D, 2, FP8, TS>(a, stream);
+        case 4: return launch_t<D, 4, FP8, TS>(a, stream);
+        case 8: return launch_t<D, 8, FP8, TS>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -671,6 +697,8 @@ bool prefill_supported(int head_dim, int group) {
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
+    if (a.fp8 && a.token_scales)
+        return a.head_dim == 128 ? launch_d<128, true, true>(a, g, stream) : launch_d<64, true, true>(a, g, stream);
     if (a.head_dim == 128)
         return a.fp8 ? launch_d<128, true>(a, g, stream) : launch_d<128, false>(a, g, stream);
     return a.fp8 ? launch_d<64, true>(a, g, stream) : launch_d<64, false>(a, g, stream);

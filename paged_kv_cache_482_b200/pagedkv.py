@@ -34,7 +34,8 @@ PKV_ERR_DEVICE_BOUNDS = 5
 PKV_ERR_DEVICE_TIMEOUT = 6
 
 PKV_CACHE_BF16 = 0
-PKV_CACHE_FP8_E4M3 = 1
+PKV_CACHE_FP8_E4M3 = 1  # k_scale / v_scale: [num_kv_heads] fp32
+PKV_CACHE_FP8_E4M3_TOKEN = 2  # k_scale / v_scale: scale pools [num_blocks, num_kv_heads, block_size] fp32
 
 EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_paged_attention_decode", "pkv_status_string",
             "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
@@ -114,10 +115,16 @@ def _stream(stream):
     return ctypes.c_void_p(int(stream))
 
 
-def _cache_dtype(t: torch.Tensor) -> int:
+def _cache_dtype(t: torch.Tensor, k_scale=None) -> int:
+    """The pool's cache type; an E4M3 pool whose scales are 3-D scale pools
+    ([num_blocks, num_kv_heads, block_size]) has one scale per token."""
     if t.dtype == torch.bfloat16:
         return PKV_CACHE_BF16
     if t.dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
+        if k_scale is not None and k_scale.dim() == 3:
+            if k_scale.shape != t.shape[:3] or k_scale.dtype != torch.float32 or not k_scale.is_contiguous():
+                raise ValueError("per-token scale pools must be contiguous fp32 [num_blocks, num_kv_heads, block_size]")
+            return PKV_CACHE_FP8_E4M3_TOKEN
         return PKV_CACHE_FP8_E4M3
     raise TypeError(f"KV pool dtype {t.dtype}: expected bfloat16 or an 8-bit E4M3 container")
 
@@ -140,7 +147,7 @@ def store_kvcache(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=No
     if v.shape != k.shape or v_cache.shape != k_cache.shape or nkv2 != nkv or d2 != d or slot_mapping.numel() != N:
         raise ValueError("shape mismatch between k/v, pools and slot_mapping")
     st = lib().pkv_store_kvcache(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), N, nkv, d, bs,
-                                 nblk, _cache_dtype(k_cache), _ptr(k_scale), _ptr(v_scale), _ptr(dev_err),
+                                 nblk, _cache_dtype(k_cache, k_scale), _ptr(k_scale), _ptr(v_scale), _ptr(dev_err),
                                  _stream(stream))
     _check(st, "pkv_store_kvcache")
 
@@ -180,10 +187,10 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     maxb = block_tables.shape[1]
     if max_context_len is None:
         max_context_len = maxb * bs
-    fp8 = _cache_dtype(k_cache) == PKV_CACHE_FP8_E4M3
+    dt = _cache_dtype(k_cache, k_scale)
     if out is None:
         out = torch.empty_like(q)
-    plan = plan_decode(S, nq, nkv, d, bs, max_context_len, fp8, partition_request)
+    plan = plan_decode(S, nq, nkv, d, bs, max_context_len, dt != PKV_CACHE_BF16, partition_request)
     if plan["workspace_bytes"] and workspace is None:
         workspace = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -191,7 +198,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         raise ValueError("seq_order must be an int32 permutation of the sequences")
     st = lib().pkv_paged_attention_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), maxb,
                                           _ptr(context_lens), _ptr(seq_order), S, nq, nkv, d, bs, nblk, float(scale),
-                                          PKV_CACHE_FP8_E4M3 if fp8 else PKV_CACHE_BF16, _ptr(k_scale),
+                                          dt, _ptr(k_scale),
                                           _ptr(v_scale), int(max_context_len), int(partition_request),
                                           _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_err), _stream(stream))
     _check(st, "pkv_paged_attention_decode")
@@ -223,7 +230,7 @@ def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, con
         max_context_len = maxb * bs
     if out is None:
         out = torch.empty_like(q)
-    dt = _cache_dtype(k_cache)
+    dt = _cache_dtype(k_cache, k_scale)
     st = lib().pkv_paged_attention_decode_static_scratch(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                                          maxb, _ptr(context_lens), _ptr(seq_order), S, nq, nkv, d,
                                                          bs, nblk,
@@ -261,7 +268,7 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, contex
         out = torch.empty_like(q)
     st = lib().pkv_paged_attention_prefill(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(cu_q_lens),
-        _ptr(context_lens), S, T, nq, nkv, d, bs, nblk, float(scale), _cache_dtype(k_cache), _ptr(k_scale),
+        _ptr(context_lens), S, T, nq, nkv, d, bs, nblk, float(scale), _cache_dtype(k_cache, k_scale), _ptr(k_scale),
         _ptr(v_scale), int(max_q_len), _ptr(out), _ptr(dev_err), _stream(stream))
     _check(st, "pkv_paged_attention_prefill")
     return out
@@ -323,7 +330,7 @@ class DecodeStep:
         self.partition_request = partition_request
         dev = device or k_cache.device
         self.plan = plan_decode(num_seqs, num_q_heads, nkv, d, bs, self.max_context_len,
-                                _cache_dtype(k_cache) == PKV_CACHE_FP8_E4M3, partition_request)
+                                _cache_dtype(k_cache, k_scale) != PKV_CACHE_BF16, partition_request)
         self.workspace = (torch.empty(self.plan["workspace_bytes"], dtype=torch.uint8, device=dev)
                           if self.plan["workspace_bytes"] else None)
         self.out = torch.empty((num_seqs, num_q_heads, d), dtype=torch.bfloat16, device=dev)
