@@ -417,6 +417,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     // Per-token scales of this lane's row of tile j (TS only): K scale
     // multiplies the score, V scale the weight that P * V uses (l sums the
     // unscaled weights). Rows past the end get 0 (their weight is 0 anyway).
+    // The loop loads tile j + 1's scales while it works on tile j.
     auto tok_scales = [&](int j, float &ks, float &vs) {
         ks = 0.f;
         vs = 0.f;
@@ -493,11 +494,13 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     {
         float sc[T::kNV];
         float alpha;
-        float ks, vs;  // this lane's row scales (TS) for the tile being scored
+        float ks, vs;      // this lane's row scales (TS) for the tile being scored
+        float ks_n, vs_n;  // ... and for the next tile, loaded one tile ahead
         int sk = 0, rk = 0, sv = 0, rv = 0;
         if (!mbar_wait(&full_k[0], 0)) ok = false;
         if (ok) {
             tok_scales(0, ks, vs);
+            tok_scales(1, ks_n, vs_n);
             qk(0, sc);
             __syncwarp();
             release(0, 0, -1, 0);
@@ -510,7 +513,9 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
                 ok = false;
                 break;
             }
-            tok_scales(j, ks, vs);
+            ks = ks_n;
+            vs = vs_n;
+            tok_scales(j + 1, ks_n, vs_n);
             qk(sk, sc);
             softmax(j, sc, alpha, ks, vs);
             pv(sv, (j - 1) & 1);

@@ -245,6 +245,7 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
     a.max_q_len = max_q_len;
     a.out = out;
     a.dev_err = dev_err;
+    a.small_cut = 0;
     cudaError_t e = pkv::launch_prefill(a, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidConfiguration) return PKV_ERR_UNSUPPORTED;
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;

@@ -42,30 +42,19 @@
 // 128 / 64 column blocks][rows][128 bytes], the 16-byte chunk c of row r
 // stored at chunk c ^ (r % 8) -- the canonical 128-byte swizzle, so one
 // descriptor form serves Q, K and P (K-major) and V (MN-major).
-#include <cuda.h>
-
-#include <cstring>
-#include <mutex>
-
-#include "pkv_common.cuh"
-#include "pkv_launch.h"
+#include "tc_common.cuh"
 
 namespace pkv {
 namespace {
 
+using namespace tc;
+
 constexpr int kRows = 128;  // MMA M: query rows per CTA
 constexpr int kBN = 64;     // KV tokens per tile
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;          // two threads per row: each owns half of the tile's score columns
+constexpr int kHalfCols = kBN / 2;
 constexpr uint32_t kTmemCols = 256;  // S: 64 columns, O: up to 128 columns (two CTAs fill an SM's 512)
 constexpr uint32_t kMinSmem = 100u * 1024u;  // at most two CTAs per SM, whatever head_dim
-constexpr int kTableCap = 2048;              // block ids staged in shared memory (more: read from global)
-
-// A sequence's block-table row: the first kTableCap ids from shared memory.
-struct BlockIds {
-    const int32_t *smem;
-    const int32_t *gmem;
-    __device__ __forceinline__ int operator[](int i) const { return i < kTableCap ? smem[i] : __ldg(gmem + i); }
-};
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -86,134 +75,10 @@ struct Layout {
     static constexpr uint32_t kBar = kP + (kPInK ? 0 : kPBytes);  // 4 mbarriers, TMEM address
     static constexpr uint32_t kTable = kBar + 64;                  // the sequence's first block ids
     static constexpr uint32_t kScales = kTable + kTableCap * 4;    // per-token scales: [2 buffers][K, V][kBN]
-    static constexpr uint32_t kBytes = kScales + 2 * 2 * kBN * 4;
+    static constexpr uint32_t kRed = kScales + 2 * 2 * kBN * 4;     // row-max halves: [2 tiles][2 halves][kRows]
+    static constexpr uint32_t kBytes = kRed + 3 * 2 * kRows * 4;  // + the final l exchange [2][kRows]
     static constexpr uint32_t kAlloc = (kBytes + 1024 > kMinSmem) ? kBytes + 1024 : kMinSmem;  // + base alignment
 };
-
-// ------------------------------------------------------------ tcgen05 PTX
-
-// Shared-memory matrix descriptor (sm_100 form): start address, leading and
-// stride byte offsets (all >> 4), descriptor version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, A
-// K-major, B K-major or MN-major, M x N.
-constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-           (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t holder_saddr, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder_saddr),
-                 "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive on *bar once every tcgen05 operation this thread issued so far has completed.
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's tensor-memory lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 32 consecutive fp32 columns into this thread's tensor-memory lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-        : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// 16-byte asynchronous copy global -> shared; src_bytes 0 writes zeros.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// 2-D tensor-map copy of one box into shared memory, completing on *bar.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-            "r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void st_shared16(uint32_t addr, uint4 v) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// Eight E4M3 codes -> eight bf16 values (exact: every E4M3 value is a bf16 value).
-__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 w) {
-    uint4 o;
-    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w.x & 0xFFFFu));
-    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w.x >> 16));
-    float2 c = e4m3x2_to_float2(static_cast<uint16_t>(w.y & 0xFFFFu));
-    float2 d = e4m3x2_to_float2(static_cast<uint16_t>(w.y >> 16));
-    o.x = pack_bf16(a.x, a.y);
-    o.y = pack_bf16(b.x, b.y);
-    o.z = pack_bf16(c.x, c.y);
-    o.w = pack_bf16(d.x, d.y);
-    return o;
-}
-
-// Byte offset of 16-byte chunk c16 of row r in a swizzled operand of `rows` rows.
-__device__ __forceinline__ uint32_t swz(int rows, int r, int c16) {
-    return static_cast<uint32_t>((c16 >> 3) * rows * 128 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));
-}
 
 // Stage KV tile j (logical tokens j*kBN ..) of KV head kh into one K/V buffer.
 // Tokens at or past kv_end are zero-filled; their scores are masked anyway
@@ -223,16 +88,18 @@ __device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const BlockId
                                              int log2_bs, uint32_t sk, uint32_t sv, float *scales = nullptr) {
     if constexpr (TS) {
         // K scales of the tile's tokens in scales[0..kBN), V scales in [kBN, 2 kBN); 0 past the end
-        const int t = threadIdx.x % kBN;
-        const bool is_v = threadIdx.x >= kBN;
-        const int pos = j * kBN + t;
-        float sc = 0.0f;
-        if (pos < kv_end) {
-            const int64_t blk = table[pos >> log2_bs];
-            const int64_t idx = (blk * a.num_kv_heads + kh) * a.block_size + (pos & (a.block_size - 1));
-            sc = __ldg((is_v ? a.v_scale : a.k_scale) + idx);
+        if (threadIdx.x < 2 * kBN) {
+            const int t = threadIdx.x % kBN;
+            const bool is_v = threadIdx.x >= kBN;
+            const int pos = j * kBN + t;
+            float sc = 0.0f;
+            if (pos < kv_end) {
+                const int64_t blk = table[pos >> log2_bs];
+                const int64_t idx = (blk * a.num_kv_heads + kh) * a.block_size + (pos & (a.block_size - 1));
+                sc = __ldg((is_v ? a.v_scale : a.k_scale) + idx);
+            }
+            scales[threadIdx.x] = sc;
         }
-        scales[threadIdx.x] = sc;
     }
     constexpr int kChunks = D / 8;             // 16-byte chunks per bf16 row
     constexpr int kTokPerPass = kThreads / kChunks;
@@ -335,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int c = q1 - q0;
     const int t0 = tile * TQ;
     if (t0 >= c) return;
+    if (a.small_cut > 0 && c > a.small_cut) return;  // a longer chunk: the warp-specialised kernel's
     const int ctx = a.context_lens[s];
     const int32_t *table_g = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
     int32_t *table_s = reinterpret_cast<int32_t *>(sm + L::kTable);
@@ -349,14 +217,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
     const BlockIds table{table_s, table_g};
-    const int row_tok = t0 + tid / G;  // this thread's row
-    const int row_head = kh * G + tid % G;
+    // Two threads per row: warps w and w + 4 read the same tensor-memory lanes
+    // (32 (w % 4) ..), the first the low half of the score and output
+    // columns, the second the high half.
+    const int row = tid & (kRows - 1);
+    const int half = tid >> 7;
+    const int row_tok = t0 + row / G;  // this thread's row
+    const int row_head = kh * G + row % G;
     const bool row_live = row_tok < c;
-    __nv_bfloat16 *out_row =
-        static_cast<__nv_bfloat16 *>(a.out) + (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + row_head) * D;
+    __nv_bfloat16 *out_row = static_cast<__nv_bfloat16 *>(a.out) +
+                             (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + row_head) * D + half * (D / 2);
     if (__syncthreads_or(bad)) {
         if (row_live) {
-            for (int i = 0; i < D; i += 8) *reinterpret_cast<uint4 *>(out_row + i) = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < D / 2; i += 8) *reinterpret_cast<uint4 *>(out_row + i) = make_uint4(0, 0, 0, 0);
         }
         if (tid == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
         return;
@@ -383,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = *tmem_holder;
     const uint32_t tmem_s = tmem;        // S: columns 0..kBN - 1
     const uint32_t tmem_o = tmem + 128;  // O: columns 128..128 + D - 1
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float *red = reinterpret_cast<float *>(sm + L::kRed);  // [2][2][kRows]
     const uint32_t sq = base + L::kQ;
     auto kbuf = [&](int j) { return base + L::kK0 + static_cast<uint32_t>(j & 1) * L::kBufStride; };
     auto sbuf = [&](int j) { return reinterpret_cast<float *>(sm + L::kScales) + (j & 1) * 2 * kBN; };
@@ -441,39 +315,40 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t sk = kbuf(j), sv = vbuf(j);
         const uint32_t sp = L::kPInK ? sk : base + L::kP;  // P replaces this tile's K once S is computed
 
+        // this thread's half of the row's scores (exp2 domain, causal mask) and its maximum
         const bool ok_s = mbar_wait(bar_s, static_cast<uint32_t>(j & 1));
+        const int kv0 = j * kBN;
+        const int col0 = half * kHalfCols;  // first score column of this thread
+        const bool masked = kv0 + kBN - 1 > p_first;  // some row sees a future or absent token
+        const float *tsc = sbuf(j);  // this tile's per-token scales (TS)
+        float x[kHalfCols];
+        float mx = -INFINITY;
+        if (ok_s) {
+            tc_fence_after();
+            float v[32];
+            tmem_ld32(tmem_s + lane_base + col0, v);
+#pragma unroll
+            for (int i = 0; i < kHalfCols; ++i) x[i] = TS ? v[i] * (sl2 * tsc[col0 + i]) : v[i] * sl2;
+            if (masked) {
+#pragma unroll
+                for (int i = 0; i < kHalfCols; ++i)
+                    if (kv0 + col0 + i > row_pos) x[i] = -INFINITY;
+            }
+            float m8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+            for (int i = 8; i < kHalfCols; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+            mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            red[((j & 1) * 2 + half) * kRows + row] = mx;
+        }
         if (__syncthreads_or(!ok_s)) {
             timed_out = true;
             pending = bar_s;
             pending_parity = static_cast<uint32_t>(j & 1);
             break;
         }
-        tc_fence_after();
-
-        // this row's scores (exp2 domain, causal mask) and their maximum
-        const int kv0 = j * kBN;
-        const bool masked = kv0 + kBN - 1 > p_first;  // some row sees a future or absent token
-        float x[kBN];
-        const float *tsc = sbuf(j);  // this tile's per-token scales (TS)
-#pragma unroll
-        for (int ch = 0; ch < kBN / 32; ++ch) {
-            float v[32];
-            tmem_ld32(tmem_s + lane_base + ch * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[ch * 32 + i] = TS ? v[i] * (sl2 * tsc[ch * 32 + i]) : v[i] * sl2;
-        }
-        if (masked) {
-#pragma unroll
-            for (int i = 0; i < kBN; ++i)
-                if (kv0 + i > row_pos) x[i] = -INFINITY;
-        }
-        float m8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = x[k];
-#pragma unroll
-        for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        mx = fmaxf(mx, red[((j & 1) * 2 + (half ^ 1)) * kRows + row]);  // the row's maximum
 
         // P V of the previous tile has finished: P, O and the other buffer are free
         if (j > 0) {
@@ -509,12 +384,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     l_run *= alpha;
                 }
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < D / 64; ++ch) {  // this thread's half of the row's O columns
                     float v[32];
-                    tmem_ld32(tmem_o + lane_base + ch * 32, v);
+                    tmem_ld32(tmem_o + lane_base + half * (D / 2) + ch * 32, v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                    tmem_st32(tmem_o + lane_base + ch * 32, v);
+                    tmem_st32(tmem_o + lane_base + half * (D / 2) + ch * 32, v);
                 }
             }
         }
@@ -523,21 +398,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         // (masked scores are -inf, so their weights are exactly 0)
         float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int c16 = 0; c16 < kBN / 8; ++c16) {
+        for (int c = 0; c < kHalfCols / 8; ++c) {
             uint32_t w[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                const int i0 = c16 * 8 + 2 * h;
+                const int i0 = c * 8 + 2 * h;
                 if constexpr (TS) {
                     const float p0 = fast_exp2(x[i0] - m_run), p1 = fast_exp2(x[i0 + 1] - m_run);
-                    w[h] = pack_bf16(p0 * tsc[kBN + i0], p1 * tsc[kBN + i0 + 1]);
+                    w[h] = pack_bf16(p0 * tsc[kBN + col0 + i0], p1 * tsc[kBN + col0 + i0 + 1]);
                     l4[h] += p0 + p1;
                 } else {
                     w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
                     l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
                 }
             }
-            st_shared16(sp + swz(kRows, tid, c16), make_uint4(w[0], w[1], w[2], w[3]));
+            st_shared16(sp + swz(kRows, row, col0 / 8 + c), make_uint4(w[0], w[1], w[2], w[3]));
         }
         l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
 
@@ -592,11 +467,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else {
         tc_fence_after();
-        const float inv = ((FP8 && !TS) ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
+        // the row's normaliser: this thread's partial sum plus its partner's
+        float *lred = red + 2 * 2 * kRows;  // past the max exchange buffers ([2][kRows] floats)
+        lred[half * kRows + row] = l_run;
+        __syncthreads();
+        const float l_row = l_run + lred[(half ^ 1) * kRows + row];
+        const float inv = ((FP8 && !TS) ? __ldg(a.v_scale + kh) : 1.0f) / l_row;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 0; ch < D / 64; ++ch) {
             float v[32];
-            tmem_ld32(tmem_o + lane_base + ch * 32, v);  // warp-wide: every lane loads
+            tmem_ld32(tmem_o + lane_base + half * (D / 2) + ch * 32, v);  // warp-wide: every lane loads
             if (row_live) {
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) {
@@ -616,42 +496,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library).
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-// The pool as a 2-D bf16 tensor: rows of head_dim elements; boxes of 64
-// columns x min(block_size, kBN) rows, 128-byte swizzle.
-bool make_pool_map(CUtensorMap *map, const void *pool, const PrefillArgs &a) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.head_dim),
-                                static_cast<cuuint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.head_dim) * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(a.block_size < kBN ? a.block_size : kBN)};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int G, bool FP8, bool TS>
 cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int TQ = kRows / G;
@@ -667,7 +511,7 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t stream) {
         // TMA row coordinates are int32
         if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * a.block_size > 0x7FFFFFFFLL)
             return cudaErrorInvalidConfiguration;
-        if (!make_pool_map(&mk, a.k_cache, a) || !make_pool_map(&mv, a.v_cache, a)) return cudaErrorInvalidValue;
+        if (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)) return cudaErrorInvalidValue;
     }
     auto kern = paged_prefill_kernel<D, G, FP8, TS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -697,6 +541,20 @@ bool prefill_supported(int head_dim, int group) {
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
+    if (!a.fp8) {
+        // bf16 cache. Chunks of more than one query tile (128 / G tokens) go to
+        // the warp-specialised kernel (two tiles per CTA, one CTA per SM);
+        // shorter ones -- decode requests among them -- to the one-tile kernel,
+        // which fits two CTAs per SM. Each kernel skips the other's sequences.
+        PrefillArgs small = a;
+        small.small_cut = kRows / g;
+        small.max_q_len = a.max_q_len < small.small_cut ? a.max_q_len : small.small_cut;
+        cudaError_t e = a.head_dim == 128 ? launch_d<128, false>(small, g, stream) : launch_d<64, false>(small, g, stream);
+        if (e != cudaSuccess || a.max_q_len <= small.small_cut) return e;
+        PrefillArgs large = a;
+        large.small_cut = small.small_cut;
+        return launch_prefill_ws(large, stream);
+    }
     if (a.fp8 && a.token_scales)
         return a.head_dim == 128 ? launch_d<128, true, true>(a, g, stream) : launch_d<64, true, true>(a, g, stream);
     if (a.head_dim == 128)

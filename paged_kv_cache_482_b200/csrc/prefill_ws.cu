@@ -1,0 +1,489 @@
+// prefill_ws.cu -- chunked-prefill paged attention, bf16 cache, warp-
+// specialised on the 5th-generation tensor cores (sm_100a).
+//
+// Same operation as prefill.cu ("nano-vllm-lite：深入理解LLM推理机制的教育级开源
+// 项目", section 核心技术改进 2 "Chunked Prefill"; paged cache of "DeepSeek复刻
+// vLLM反超原版", section "vLLM：大模型推理的加速引擎与挑战"): token i of a chunk
+// of c new tokens (position p = ctx - c + i) attends over positions 0..p.
+//
+// One CTA per (sequence, KV head, two query tiles of 128 rows each; a row is
+// a (chunk token, query head of the group) pair), one CTA per SM. Warp roles:
+//   warps 0-3  softmax of query tile A (one row per thread);
+//   warps 4-7  softmax of query tile B;
+//   warp 8     producer: tensor-map copies of 64-token K/V tiles into a
+//              three-stage ring (and the zeroing of V rows past the causal
+//              end on the last tile);
+//   warp 9     tensor-memory allocation and the MMA issue:
+//                S_A(0), S_B(0), S_A(1), S_B(1), then per tile j
+//                PV_A(j), PV_B(j), S_A(j+2), S_B(j+2), ...
+//              so that the tensor core works on one tile while the other
+//              tile's softmax runs, both tiles share every K/V tile, and S
+//              of the tile after next is ready before the softmax needs it.
+// Tensor memory (512 columns): two S buffers per query tile (64 columns
+// each) and O_A, O_B (128 columns each).
+// Everything between roles goes through mbarriers (full / empty K/V stages,
+// S ready, P ready, O done); every wait is bounded (1 s) and reports
+// PKV_DEVERR_TIMEOUT. The softmax uses the same arithmetic as prefill.cu:
+// exp2 domain, lazy rescale of O in tensor memory (the reference maximum
+// moves only when a tile's maximum exceeds it by more than 8), P rounded to
+// bf16 and the normaliser summing the rounded weights.
+#include "tc_common.cuh"
+
+namespace pkv {
+namespace {
+
+using namespace tc;
+
+constexpr int kRowsT = 128;  // rows per query tile (MMA M)
+constexpr int kBN = 64;      // KV tokens per tile
+constexpr int kStages = 3;   // K/V ring depth
+constexpr int kSoftmaxThreads = 256;
+constexpr int kThreads = kSoftmaxThreads + 64;  // + producer warp + MMA warp
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct WsLayout {
+    static constexpr int kHalves = D / 64;
+    static constexpr uint32_t kQTile = kHalves * kRowsT * 128;  // one query tile
+    static constexpr uint32_t kKV = kHalves * kBN * 128;        // one K (or V) tile
+    static constexpr uint32_t kQ = 0;                           // Q_A, Q_B
+    static constexpr uint32_t kRing = kQ + 2 * kQTile;          // stage s: K at kRing + s * 2 kKV, V after it
+    static constexpr uint32_t kP = kRing + kStages * 2 * kKV;   // P_A, P_B
+    static constexpr uint32_t kPTile = (kBN / 64) * kRowsT * 128;
+    static constexpr uint32_t kBar = kP + 2 * kPTile;
+    static constexpr uint32_t kTable = kBar + 256;
+    static constexpr uint32_t kBytes = kTable + kTableCap * 4;
+    static constexpr uint32_t kAlloc = kBytes + 1024;
+};
+
+struct Bars {
+    uint64_t kv_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[2][2];  // [query tile][S buffer]
+    uint64_t p_full[2];
+    uint64_t o_done[2];     // P V of a tile done (one phase per tile)
+    uint64_t q_full;
+    uint64_t vtail;
+    uint64_t drained;
+    uint32_t tmem;
+};
+
+// Producer: stage KV tile j (logical tokens j * kBN ..) into ring stage (sk, sv).
+template <int D>
+__device__ __forceinline__ void ws_kv_tile(const CUtensorMap *mk, const CUtensorMap *mv, const BlockIds &table,
+                                           int nkv, int kh, int bs, int log2_bs, int j, int kv_end, uint32_t sk,
+                                           uint32_t sv, uint64_t *bar) {
+    constexpr int kHalves = D / 64;
+    const int kv0 = j * kBN;
+    if (bs >= kBN) {
+        const int row = (table[kv0 >> log2_bs] * nkv + kh) * bs + (kv0 & (bs - 1));
+        mbar_arrive_expect_tx(bar, 2u * kHalves * kBN * 128u);
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
+            tma_load_2d(sk + h * kBN * 128, mk, h * 64, row, bar);
+            tma_load_2d(sv + h * kBN * 128, mv, h * 64, row, bar);
+        }
+    } else {
+        const int end = min(kv0 + kBN, kv_end);
+        const int nb = (end - kv0 + bs - 1) >> log2_bs;
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(2 * kHalves * nb * bs * 128));
+        for (int i = 0; i < nb; ++i) {
+            const int row = (table[(kv0 >> log2_bs) + i] * nkv + kh) * bs;
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) {
+                tma_load_2d(sk + h * kBN * 128 + i * bs * 128, mk, h * 64, row, bar);
+                tma_load_2d(sv + h * kBN * 128 + i * bs * 128, mv, h * 64, row, bar);
+            }
+        }
+    }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    paged_prefill_ws_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
+                            const __grid_constant__ CUtensorMap map_v) {
+    using L = WsLayout<D>;
+    constexpr int TQ = kRowsT / G;  // chunk tokens per query tile
+    constexpr uint32_t kIdescS = idesc_bf16(kRowsT, kBN, false);
+    constexpr uint32_t kIdescPV = idesc_bf16(kRowsT, D, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *sm = smem_raw + (base - raw);
+    Bars *bars = reinterpret_cast<Bars *>(sm + L::kBar);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int s = blockIdx.x / tiles_per_seq;
+    const int tile = tiles_per_seq - 1 - (blockIdx.x % tiles_per_seq);  // longest causal range first
+    const int kh = blockIdx.y;
+    const int nq = a.num_q_heads;
+
+    // ------------------------------------------------ bounds and bookkeeping
+    const int q0 = a.cu_q_lens[s];
+    const int q1 = a.cu_q_lens[s + 1];
+    if (q0 < 0 || q1 < q0 || q1 > a.total_q) {
+        if (tid == 0 && tile == 0 && kh == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
+        return;
+    }
+    const int c = q1 - q0;
+    const int t0 = tile * 2 * TQ;  // first chunk token of query tile A
+    if (t0 >= c) return;
+    if (c <= a.small_cut) return;  // a short chunk: the one-tile kernel's
+    const int ctx = a.context_lens[s];
+    const int32_t *table_g = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+    int32_t *table_s = reinterpret_cast<int32_t *>(sm + L::kTable);
+    bool bad = ctx < c || static_cast<int64_t>(ctx) > static_cast<int64_t>(a.max_blocks_per_seq) * a.block_size ||
+               c > a.max_q_len;
+    if (!bad) {
+        const int nblk_seq = (ctx + a.block_size - 1) >> log2_bs;
+        for (int i = tid; i < nblk_seq; i += kThreads) {
+            const int32_t b = table_g[i];
+            if (b < 0 || b >= a.num_blocks) bad = true;
+            if (i < kTableCap) table_s[i] = b;
+        }
+    }
+    const BlockIds table{table_s, table_g};
+
+    // softmax threads: query tile X, row r of it
+    const int X = (warp >> 2) & 1;
+    const int row = tid & (kRowsT - 1);
+    const int row_tok = t0 + X * TQ + row / G;
+    const bool row_live = warp < 8 && row_tok < c;
+    __nv_bfloat16 *out_row = static_cast<__nv_bfloat16 *>(a.out) +
+                             (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + kh * G + row % G) * D;
+    if (__syncthreads_or(bad)) {
+        if (row_live)
+            for (int i = 0; i < D; i += 8) *reinterpret_cast<uint4 *>(out_row + i) = make_uint4(0, 0, 0, 0);
+        if (tid == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
+        return;
+    }
+    const int last_tok = min(t0 + 2 * TQ, c) - 1;
+    const int p_last = ctx - c + last_tok;
+    const int kv_end = p_last + 1;
+    const int n_tiles = (kv_end + kBN - 1) / kBN;
+
+    // ------------------------------------------------ setup
+    if (warp == kMmaWarp) tmem_alloc(smem_addr(&bars->tmem), kTmemCols);
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bars->kv_full[i], 1);
+            mbar_init(&bars->kv_empty[i], 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->s_full[x][0], 1);
+            mbar_init(&bars->s_full[x][1], 1);
+            mbar_init(&bars->p_full[x], kRowsT);
+            mbar_init(&bars->o_done[x], 1);
+        }
+        mbar_init(&bars->q_full, kSoftmaxThreads);
+        mbar_init(&bars->vtail, 1);
+        mbar_init(&bars->drained, 1);
+        fence_barrier_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem;
+    auto kbuf = [&](int j) { return base + L::kRing + static_cast<uint32_t>(j % kStages) * 2 * L::kKV; };
+    auto vbuf = [&](int j) { return kbuf(j) + L::kKV; };
+    const uint32_t sq0 = base + L::kQ;
+    const uint32_t sp0 = base + L::kP;
+
+    if (warp < 8) {
+        // ================================================ softmax, query tile X
+        const uint32_t sq = sq0 + X * L::kQTile;
+        const uint32_t sp = sp0 + X * L::kPTile;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tmem_s0 = tmem + X * 2 * kBN;  // S buffers of this query tile: tmem_s0 + b * kBN
+        const uint32_t tmem_o = tmem + 256 + X * 128;
+        {
+            constexpr int kChunks = D / 8;
+            const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q);
+            for (int i = row; i < kRowsT * kChunks; i += kRowsT) {
+                const int r = i / kChunks, c16 = i % kChunks;
+                const int tok = t0 + X * TQ + r / G;
+                const bool valid = tok < c;
+                const int64_t elem =
+                    (static_cast<int64_t>(q0 + (valid ? tok : 0)) * nq + kh * G + r % G) * D + c16 * 8;
+                cp_async16(sq + swz(kRowsT, r, c16), qp + elem, valid ? 16u : 0u);
+            }
+            cp_async_commit();
+            cp_async_wait0();
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->q_full);
+        }
+        const int p_first = ctx - c + t0 + X * TQ;  // position of this tile's first row
+        const int row_pos = row_live ? ctx - c + row_tok : p_last;
+        const float sl2 = a.scale * kLog2e;
+        float m_run = -INFINITY, l_run = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            // warp-uniform: the tensor-memory loads and stores below are warp-wide
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[X][j & 1], static_cast<uint32_t>((j >> 1) & 1)))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tmem_s = tmem_s0 + (j & 1) * kBN;
+            const int kv0 = j * kBN;
+            const bool masked = kv0 + kBN - 1 > p_first;
+            float x[kBN];
+#pragma unroll
+            for (int ch = 0; ch < kBN / 32; ++ch) {
+                float v[32];
+                tmem_ld32(tmem_s + lane_base + ch * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[ch * 32 + i] = v[i] * sl2;
+            }
+            if (masked) {
+#pragma unroll
+                for (int i = 0; i < kBN; ++i)
+                    if (kv0 + i > row_pos) x[i] = -INFINITY;
+            }
+            float m8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+            for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            // P V_X(j - 1) must be done before O_X is rescaled and the P buffer rewritten
+            if (j > 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], static_cast<uint32_t>((j - 1) & 1)))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (j == 0) {
+                m_run = mx;  // O is written, not accumulated, by the first P V
+            } else {
+                const bool grow = mx > m_run + 8.0f;
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float alpha = grow ? fast_exp2(m_run - mx) : 1.0f;
+                    if (grow) {
+                        m_run = mx;
+                        l_run *= alpha;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        float v[32];
+                        tmem_ld32(tmem_o + lane_base + ch * 32, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                        tmem_st32(tmem_o + lane_base + ch * 32, v);
+                    }
+                }
+            }
+            float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int c16 = 0; c16 < kBN / 8; ++c16) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int i0 = c16 * 8 + 2 * h;
+                    w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
+                    l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
+                }
+                st_shared16(sp + swz(kRowsT, row, c16), make_uint4(w[0], w[1], w[2], w[3]));
+            }
+            l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[X]);
+        }
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], static_cast<uint32_t>((n_tiles - 1) & 1)))) {
+            tc_fence_after();
+            const float inv = 1.0f / l_run;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                float v[32];
+                tmem_ld32(tmem_o + lane_base + ch * 32, v);
+                if (row_live) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 w = make_uint4(pack_bf16(v[i] * inv, v[i + 1] * inv),
+                                             pack_bf16(v[i + 2] * inv, v[i + 3] * inv),
+                                             pack_bf16(v[i + 4] * inv, v[i + 5] * inv),
+                                             pack_bf16(v[i + 6] * inv, v[i + 7] * inv));
+                        *reinterpret_cast<uint4 *>(out_row + ch * 32 + i) = w;
+                    }
+                }
+            }
+        } else {
+            if (row == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == kProducerWarp) {
+        // ================================================ producer
+        int issued = 0;
+        if (lane == 0) {
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j % kStages, use = j / kStages;
+                if (use > 0 && !mbar_wait(&bars->kv_empty[st], static_cast<uint32_t>((use - 1) & 1))) {
+                    set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
+                    break;
+                }
+                ws_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, j, kv_end, kbuf(j),
+                              vbuf(j), &bars->kv_full[st]);
+                issued = j + 1;
+            }
+        }
+        issued = __shfl_sync(0xffffffffu, issued, 0);
+        // V rows past the causal end on the last tile: zero them, so that a
+        // zero weight times stale pool data stays zero.
+        const int last = n_tiles - 1;
+        const int valid_rows = kv_end - last * kBN;
+        bool tail_ok = issued == n_tiles;
+        if (tail_ok && valid_rows < kBN) {
+            tail_ok = mbar_wait(&bars->kv_full[last % kStages], static_cast<uint32_t>((last / kStages) & 1));
+            if (tail_ok) {
+                constexpr int kHalves = D / 64;
+                const int n16 = (kBN - valid_rows) * 8;
+                for (int i = lane; i < kHalves * n16; i += 32) {
+                    const int h = i / n16, r = valid_rows + (i % n16) / 8, cc = i % 8;
+                    st_shared16(vbuf(last) + h * kBN * 128 + r * 128 + cc * 16, make_uint4(0, 0, 0, 0));
+                }
+                fence_proxy_async_smem();
+            }
+        }
+        __syncwarp();
+        if (lane == 0) {
+            if (tail_ok) mbar_arrive(&bars->vtail);
+            // copies still in flight (only after a timeout): wait for them before the CTA exits
+            for (int j = max(0, issued - kStages); j < issued; ++j)
+                mbar_wait(&bars->kv_full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
+        }
+        __syncwarp();
+    } else {
+        // ================================================ MMA issue
+        if (lane == 0) {
+            bool ok = mbar_wait(&bars->q_full, 0);
+            auto issue_s = [&](int x, int j) {  // S_x(j) into S buffer j & 1 of query tile x
+                const uint32_t sq = sq0 + x * L::kQTile, sk = kbuf(j);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRowsT * 128 + (kk & 3) * 32);
+                    const uint32_t boff = static_cast<uint32_t>((kk >> 2) * kBN * 128 + (kk & 3) * 32);
+                    mma_bf16(tmem + (x * 2 + (j & 1)) * kBN, sw128_desc(sq + aoff, 16, 1024),
+                             sw128_desc(sk + boff, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars->s_full[x][j & 1]);
+            };
+            auto issue_pv = [&](int x, int j) {
+                const uint32_t sp = sp0 + x * L::kPTile, sv = vbuf(j);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRowsT * 128 + (kk & 3) * 32);
+                    mma_bf16(tmem + 256 + x * 128, sw128_desc(sp + aoff, 16, 1024),
+                             sw128_desc(sv + static_cast<uint32_t>(kk * 16 * 128), kBN * 128, 1024), kIdescPV,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&bars->o_done[x]);
+            };
+            auto kv_ready = [&](int j) {
+                const bool r = mbar_wait(&bars->kv_full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
+                tc_fence_after();
+                return r;
+            };
+            // S of the first two tiles
+            for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {
+                ok = kv_ready(j);
+                if (ok) {
+                    issue_s(0, j);
+                    issue_s(1, j);
+                }
+            }
+            // Per tile j: P V of both query tiles as soon as their P is
+            // ready, release tile j's ring stage, then S of tile j + 2 (its
+            // copy has had a whole tile to land; the softmax needs it only
+            // two tiles later).
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                if (j == n_tiles - 1) ok = mbar_wait(&bars->vtail, 0);  // V rows past the end are zero
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (!mbar_wait(&bars->p_full[x], static_cast<uint32_t>(j & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv(x, j);  // P_x(j) was read from S buffer j & 1: free for S_x(j + 2)
+                }
+                if (!ok) break;
+                mma_commit(&bars->kv_empty[j % kStages]);  // tile j's K and V are consumed
+                if (j + 2 < n_tiles) {
+                    if (!kv_ready(j + 2)) {
+                        ok = false;
+                        break;
+                    }
+                    issue_s(0, j + 2);
+                    issue_s(1, j + 2);
+                }
+            }
+            if (!ok) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
+            // every MMA issued so far has finished before tensor memory is freed
+            mma_commit(&bars->drained);
+            mbar_wait(&bars->drained, 0);
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D, int G>
+cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
+    constexpr int TQ = kRowsT / G;
+    const int tiles = (a.max_q_len + 2 * TQ - 1) / (2 * TQ);
+    const long long nx = static_cast<long long>(a.num_seqs) * tiles;
+    if (nx > 0x7FFFFFFFLL || a.num_kv_heads > 65535) return cudaErrorInvalidConfiguration;
+    if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * a.block_size > 0x7FFFFFFFLL)
+        return cudaErrorInvalidConfiguration;  // tensor-map row coordinates are int32
+    int log2_bs = 0;
+    while ((1 << log2_bs) < a.block_size) ++log2_bs;
+    CUtensorMap mk, mv;
+    memset(&mk, 0, sizeof(mk));
+    memset(&mv, 0, sizeof(mv));
+    if (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)) return cudaErrorInvalidValue;
+    auto kern = paged_prefill_ws_kernel<D, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(WsLayout<D>::kAlloc));
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), kThreads, WsLayout<D>::kAlloc, stream>>>(a, tiles, log2_bs,
+                                                                                                   mk, mv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream) {
+    const int g = a.num_q_heads / a.num_kv_heads;
+    if (a.head_dim == 128) {
+        switch (g) {
+            case 1: return launch_ws<128, 1>(a, stream);
+            case 2: return launch_ws<128, 2>(a, stream);
+            case 4: return launch_ws<128, 4>(a, stream);
+            case 8: return launch_ws<128, 8>(a, stream);
+        }
+    } else if (a.head_dim == 64) {
+        switch (g) {
+            case 1: return launch_ws<64, 1>(a, stream);
+            case 2: return launch_ws<64, 2>(a, stream);
+            case 4: return launch_ws<64, 4>(a, stream);
+            case 8: return launch_ws<64, 8>(a, stream);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pkv
