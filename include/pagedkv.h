@@ -238,7 +238,7 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  *
  * Host checks: pointers non-null, q / caches / out 16-byte aligned,
  * head_dim 64 or 128, group 1, 2, 4 or 8, block_size a power of two in
- * [8, 1024], max_q_len >= 1 (when total_q > 0). Device checks: cu_q_lens not
+ * [8, 1024], scale positive and finite, max_q_len >= 1 (when total_q > 0). Device checks: cu_q_lens not
  * starting at or above 0, decreasing or past total_q, a chunk longer than
  * its context or than max_q_len, a context beyond the table row, or a block
  * id outside [0, num_blocks) set PKV_DEVERR_BOUNDS; the sequence's rows are

@@ -218,7 +218,7 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
     if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
     if (max_blocks_per_seq < 1 || num_blocks < 1 || num_blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
-    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;  // NaN
+    if (!(scale > 0.0f) || scale > 3.0e38f) return PKV_ERR_INVALID_ARG;  // positive and finite
     if (num_seqs == 0 || total_q == 0) return PKV_OK;
     if (max_q_len < 1) return PKV_ERR_INVALID_ARG;
 

@@ -187,8 +187,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const int s = blockIdx.x / tiles_per_seq;
-    const int tile = tiles_per_seq - 1 - (blockIdx.x % tiles_per_seq);  // longest causal range first
+    // query-tile-major over the sequences: the last (longest causal range)
+    // tiles of every sequence are scheduled first
+    const int s = blockIdx.x % a.num_seqs;
+    const int tile = tiles_per_seq - 1 - blockIdx.x / a.num_seqs;
     const int kh = blockIdx.y;
     const int nq = a.num_q_heads;
 

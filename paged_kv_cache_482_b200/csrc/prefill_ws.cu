@@ -119,8 +119,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int s = blockIdx.x / tiles_per_seq;
-    const int tile = tiles_per_seq - 1 - (blockIdx.x % tiles_per_seq);  // longest causal range first
+    // query-tile-major over the sequences: the last (longest causal range)
+    // tiles of every sequence are scheduled first
+    const int s = blockIdx.x % a.num_seqs;
+    const int tile = tiles_per_seq - 1 - blockIdx.x / a.num_seqs;
     const int kh = blockIdx.y;
     const int nq = a.num_q_heads;
 
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[32];
                 tmem_ld32(tmem_s + lane_base + ch * 32, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[ch * 32 + i] = v[i] * sl2;
+                for (int i = 0; i < 32; ++i) x[ch * 32 + i] = v[i];  // raw scores; sl2 > 0 is applied below
             }
             if (masked) {
 #pragma unroll
@@ -251,8 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 8; ++k) m8[k] = x[k];
 #pragma unroll
             for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            // the tile's maximum in the exp2 domain (the scale is positive)
+            const float mx = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             // P V_X(j - 1) must be done before O_X is rescaled and the P buffer rewritten
             if (j > 0) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], static_cast<uint32_t>((j - 1) & 1)))) {
@@ -288,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int i0 = c16 * 8 + 2 * h;
-                    w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
-                    l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
+                    w[h] = pack_bf16(fast_exp2(fmaf(x[i0], sl2, -m_run)), fast_exp2(fmaf(x[i0 + 1], sl2, -m_run)));
+                    l4[h] = fma_bf16x2_acc(w[h], 0x3F803F80u, l4[h]);  // + both rounded weights (x 1.0)
                 }
                 st_shared16(sp + swz(kRowsT, row, c16), make_uint4(w[0], w[1], w[2], w[3]));
             }

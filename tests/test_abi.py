@@ -158,6 +158,7 @@ def test_prefill_host_checks(K):
     assert call(dt=1) == K.PKV_ERR_INVALID_ARG  # FP8 without scales
     assert call(dt=5) == K.PKV_ERR_INVALID_ARG
     assert call(scale=float("nan")) == K.PKV_ERR_INVALID_ARG
+    assert call(scale=-0.1) == K.PKV_ERR_INVALID_ARG and call(scale=0.0) == K.PKV_ERR_INVALID_ARG
     assert call(mq=0) == K.PKV_ERR_INVALID_ARG
     assert call(nblk=2**31) == K.PKV_ERR_INVALID_ARG
     assert call(S=0) == K.PKV_OK and call(T=0) == K.PKV_OK  # nothing to do, nothing launched
