@@ -11,7 +11,7 @@
 //   warps 0-3  softmax of query tile A (one row per thread);
 //   warps 4-7  softmax of query tile B;
 //   warp 8     producer: tensor-map copies of 64-token K/V tiles into a
-//              three-stage ring (and the zeroing of V rows past the causal
+//              four-stage ring (and the zeroing of V rows past the causal
 //              end on the last tile);
 //   warp 9     tensor-memory allocation and the MMA issue:
 //                S_A(0), S_B(0), S_A(1), S_B(1), then per tile j
@@ -20,7 +20,12 @@
 //              tile's softmax runs, both tiles share every K/V tile, and S
 //              of the tile after next is ready before the softmax needs it.
 // Tensor memory (512 columns): two S buffers per query tile (64 columns
-// each) and O_A, O_B (128 columns each).
+// each) and O_A, O_B (128 columns each). P (bf16, two per 32-bit column)
+// is written over the first 32 columns of the S buffer it came from and P V
+// takes its A operand from tensor memory, so P never touches shared memory;
+// S of tile j + 2 reuses the buffer only after P V of tile j, issued before
+// it by the same thread. The softmax waits for P V of the previous tile only
+// when it has to rescale O.
 // Everything between roles goes through mbarriers (full / empty K/V stages,
 // S ready, P ready, O done); every wait is bounded (1 s) and reports
 // PKV_DEVERR_TIMEOUT. The softmax uses the same arithmetic as prefill.cu:
@@ -36,7 +41,7 @@ using namespace tc;
 
 constexpr int kRowsT = 128;  // rows per query tile (MMA M)
 constexpr int kBN = 64;      // KV tokens per tile
-constexpr int kStages = 3;   // K/V ring depth
+constexpr int kStages = 4;   // K/V ring depth
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 64;  // + producer warp + MMA warp
 constexpr int kProducerWarp = 8;
@@ -51,9 +56,7 @@ struct WsLayout {
     static constexpr uint32_t kKV = kHalves * kBN * 128;        // one K (or V) tile
     static constexpr uint32_t kQ = 0;                           // Q_A, Q_B
     static constexpr uint32_t kRing = kQ + 2 * kQTile;          // stage s: K at kRing + s * 2 kKV, V after it
-    static constexpr uint32_t kP = kRing + kStages * 2 * kKV;   // P_A, P_B
-    static constexpr uint32_t kPTile = (kBN / 64) * kRowsT * 128;
-    static constexpr uint32_t kBar = kP + 2 * kPTile;
+    static constexpr uint32_t kBar = kRing + kStages * 2 * kKV;
     static constexpr uint32_t kTable = kBar + 256;
     static constexpr uint32_t kBytes = kTable + kTableCap * 4;
     static constexpr uint32_t kAlloc = kBytes + 1024;
@@ -63,8 +66,8 @@ struct Bars {
     uint64_t kv_full[kStages];
     uint64_t kv_empty[kStages];
     uint64_t s_full[2][2];  // [query tile][S buffer]
-    uint64_t p_full[2];
-    uint64_t o_done[2];     // P V of a tile done (one phase per tile)
+    uint64_t p_full[2][2];  // [query tile][S buffer]: P of a tile written
+    uint64_t o_done[2][2];  // [query tile][S buffer]: P V of a tile done
     uint64_t q_full;
     uint64_t vtail;
     uint64_t drained;
@@ -180,8 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(&bars->s_full[x][0], 1);
             mbar_init(&bars->s_full[x][1], 1);
-            mbar_init(&bars->p_full[x], kRowsT);
-            mbar_init(&bars->o_done[x], 1);
+            mbar_init(&bars->p_full[x][0], kRowsT);
+            mbar_init(&bars->p_full[x][1], kRowsT);
+            mbar_init(&bars->o_done[x][0], 1);
+            mbar_init(&bars->o_done[x][1], 1);
         }
         mbar_init(&bars->q_full, kSoftmaxThreads);
         mbar_init(&bars->vtail, 1);
@@ -195,12 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto kbuf = [&](int j) { return base + L::kRing + static_cast<uint32_t>(j % kStages) * 2 * L::kKV; };
     auto vbuf = [&](int j) { return kbuf(j) + L::kKV; };
     const uint32_t sq0 = base + L::kQ;
-    const uint32_t sp0 = base + L::kP;
 
     if (warp < 8) {
         // ================================================ softmax, query tile X
         const uint32_t sq = sq0 + X * L::kQTile;
-        const uint32_t sp = sp0 + X * L::kPTile;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tmem_s0 = tmem + X * 2 * kBN;  // S buffers of this query tile: tmem_s0 + b * kBN
         const uint32_t tmem_o = tmem + 256 + X * 128;
@@ -235,14 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tmem_s = tmem_s0 + (j & 1) * kBN;
             const int kv0 = j * kBN;
             const bool masked = kv0 + kBN - 1 > p_first;
-            float x[kBN];
-#pragma unroll
-            for (int ch = 0; ch < kBN / 32; ++ch) {
-                float v[32];
-                tmem_ld32(tmem_s + lane_base + ch * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[ch * 32 + i] = v[i];  // raw scores; sl2 > 0 is applied below
-            }
+            float x[kBN];  // raw scores; the (positive) scale is applied below
+            static_assert(kBN == 64, "one 64-column tensor-memory load per tile");
+            tmem_ld64(tmem_s + lane_base, x);
             if (masked) {
 #pragma unroll
                 for (int i = 0; i < kBN; ++i)
@@ -256,19 +254,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the tile's maximum in the exp2 domain (the scale is positive)
             const float mx = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                          fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            // P V_X(j - 1) must be done before O_X is rescaled and the P buffer rewritten
-            if (j > 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], static_cast<uint32_t>((j - 1) & 1)))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-            }
             if (j == 0) {
                 m_run = mx;  // O is written, not accumulated, by the first P V
             } else {
                 const bool grow = mx > m_run + 8.0f;
                 if (__any_sync(0xffffffffu, grow)) {
+                    // O_X must hold P V of tile j - 1 before it is rescaled. (This
+                    // buffer's barrier can be at most one phase past the one
+                    // waited for: P V of tile j + 1 needs this tile's P first.)
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[X][(j - 1) & 1],
+                                                           static_cast<uint32_t>(((j - 1) >> 1) & 1)))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                     const float alpha = grow ? fast_exp2(m_run - mx) : 1.0f;
                     if (grow) {
                         m_run = mx;
@@ -284,24 +283,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            // P = exp2(s * scale - m) as bf16 pairs over the first 32 columns of
+            // this S buffer; l sums the rounded weights
             float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float pw[kBN / 2];
 #pragma unroll
-            for (int c16 = 0; c16 < kBN / 8; ++c16) {
-                uint32_t w[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int i0 = c16 * 8 + 2 * h;
-                    w[h] = pack_bf16(fast_exp2(fmaf(x[i0], sl2, -m_run)), fast_exp2(fmaf(x[i0 + 1], sl2, -m_run)));
-                    l4[h] = fma_bf16x2_acc(w[h], 0x3F803F80u, l4[h]);  // + both rounded weights (x 1.0)
-                }
-                st_shared16(sp + swz(kRowsT, row, c16), make_uint4(w[0], w[1], w[2], w[3]));
+            for (int i = 0; i < kBN / 2; ++i) {
+                const uint32_t w = pack_bf16(fast_exp2(fmaf(x[2 * i], sl2, -m_run)),
+                                             fast_exp2(fmaf(x[2 * i + 1], sl2, -m_run)));
+                l4[i & 3] = fma_bf16x2_acc(w, 0x3F803F80u, l4[i & 3]);  // + both rounded weights (x 1.0)
+                pw[i] = __uint_as_float(w);
             }
+            tmem_st32(tmem_s + lane_base, pw);
             l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full[X]);
+            // per S buffer: the softmax can be a tile ahead of the MMA issue
+            // (S of tile j + 2 needs P V of tile j), never two phases of one barrier
+            mbar_arrive(&bars->p_full[X][j & 1]);
         }
-        if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], static_cast<uint32_t>((n_tiles - 1) & 1)))) {
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X][(n_tiles - 1) & 1],
+                                                    static_cast<uint32_t>(((n_tiles - 1) >> 1) & 1)))) {
             tc_fence_after();
             const float inv = 1.0f / l_run;
 #pragma unroll
@@ -379,16 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(&bars->s_full[x][j & 1]);
             };
-            auto issue_pv = [&](int x, int j) {
-                const uint32_t sp = sp0 + x * L::kPTile, sv = vbuf(j);
+            auto issue_pv = [&](int x, int j) {  // A = P_x(j) in tensor memory: 8 columns per 16 tokens
+                const uint32_t tp = tmem + (x * 2 + (j & 1)) * kBN, sv = vbuf(j);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRowsT * 128 + (kk & 3) * 32);
-                    mma_bf16(tmem + 256 + x * 128, sw128_desc(sp + aoff, 16, 1024),
-                             sw128_desc(sv + static_cast<uint32_t>(kk * 16 * 128), kBN * 128, 1024), kIdescPV,
-                             (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&bars->o_done[x]);
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_bf16_ts(tmem + 256 + x * 128, tp + kk * 8,
+                                sw128_desc(sv + static_cast<uint32_t>(kk * 16 * 128), kBN * 128, 1024), kIdescPV,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars->o_done[x][j & 1]);
             };
             auto kv_ready = [&](int j) {
                 const bool r = mbar_wait(&bars->kv_full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
@@ -410,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < n_tiles; ++j) {
                 if (j == n_tiles - 1) ok = mbar_wait(&bars->vtail, 0);  // V rows past the end are zero
                 for (int x = 0; x < 2 && ok; ++x) {
-                    if (!mbar_wait(&bars->p_full[x], static_cast<uint32_t>(j & 1))) {
+                    if (!mbar_wait(&bars->p_full[x][j & 1], static_cast<uint32_t>((j >> 1) & 1))) {
                         ok = false;
                         break;
                     }
