@@ -677,14 +677,18 @@ def run_prefill(args):
                        "l2": "no flush: each step's pools and queries exceed 126 MB of L2"},
             "attention_us": attn_ms * 1e3, "store_us": store_ms * 1e3,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
-                         "frac": achieved / peak_sus, "traffic": None, "kernel": "paged_prefill_kernel",
+                         "frac": achieved / peak_sus, "traffic": None,
+                         "kernel": "paged_prefill_kernel" if wl.is_fp8 else "paged_prefill_ws_kernel (+ paged_prefill_kernel)",
                          "peak_source": f"{kind} cuBLAS bf16 GEMM, sustained (bf16_tflops_sustained); "
                                         f"burst {peak_burst}",
                          "algorithmic_flops_per_launch": flops,
                          "flops_note": "causal: 4 * head_dim FLOPs per (query row, head, key at or before it)"},
             "e2e": {"value": world * T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "query tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
-            "gpu_launches": 2 * Kst,
+            # per step: the store, and for a bf16 cache the one-tile kernel (short
+            # chunks) plus, when some chunk is longer than 128 / G tokens, the
+            # warp-specialised kernel; an E4M3 cache has one prefill kernel
+            "gpu_launches": (1 + (1 if wl.is_fp8 else (2 if mq > 128 // c.group else 1))) * Kst,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
