@@ -35,6 +35,14 @@
  *  - A sequence's blocks are released last block first, so the tail of a
  *    cached prefix is reused before its head.
  *
+ * Contract with the caller: a full block is shared from the moment it is
+ * registered (when add_sequence takes it for a prompt, or when append_token
+ * fills it), while its K/V is written by the caller's store_kvcache. A
+ * sequence that hits a block must therefore attend only after the K/V of
+ * that block has been stored (stream order does it within one step; with
+ * chunked prefill, admit requests that could hit a prompt's blocks after
+ * those blocks have been prefilled).
+ *
  * Ownership: the manager owns its state; every call is synchronous host code
  * and the manager is not thread-safe (one caller at a time). Errors are
  * returned as pkv_status values (pagedkv.h); a failed call changes nothing.
