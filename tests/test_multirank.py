@@ -40,9 +40,20 @@ def _worker(rank, world, port, q):
         tput = bench.job_throughput(w, 1024, 100, got[0])
 
         class A:
-            steps, warmup, gpus = 2, 1, world
+            steps, warmup, gpus, seed = 2, 1, world, 0
+            config = "tiny"
 
-        ref_rc = bench.run_reference(A) if rank != 0 else None  # non-zero ranks return at once
+        class AP(A):
+            config = "prefill_tiny"
+
+        class AN(A):
+            config = "norm_tiny"
+
+        # the oracle legs (decode, prefill, add + RMSNorm) run on rank 0 alone:
+        # every other rank returns at once
+        ref_rc = None
+        if rank != 0:
+            ref_rc = (bench.run_reference(A), bench.run_prefill_reference(AP), bench.run_norm_reference(AN))
         q.put((rank, w, r, lr, got, tput, ref_rc))
     finally:
         dist.destroy_process_group()
@@ -64,7 +75,7 @@ def test_two_gloo_ranks_take_the_max_and_count_all_sequences():
         assert (w, r, lr) == (2, rank, rank)
         assert got == [11.0, 5.0, 14.0]  # element-wise max over the two ranks
         assert tput == pytest.approx(2 * 1024 * 100 / 11.0e-3)
-    assert res[1][6] == 0  # rank 1 skips the oracle leg
+    assert res[1][6] == (0, 0, 0)  # rank 1 skips every oracle leg
 
 
 def test_single_process_is_the_identity():
