@@ -69,6 +69,10 @@ SMALL = [
                     decode_hist_hi=900),
     W.PrefillConfig("fp8_bs16", 2, 8, 2, 128, 16, 50, 400, 30, 200, cache_dtype=W.CACHE_FP8),
     W.PrefillConfig("fp8_g8_d64", 2, 8, 1, 64, 256, 0, 300, 1, 90, cache_dtype=W.CACHE_FP8),
+    # the smallest and largest block sizes the API accepts: 8-row copies, and
+    # one block spanning sixteen 64-token tiles
+    W.PrefillConfig("bs8_g4", 3, 32, 8, 128, 8, 0, 200, 40, 300),
+    W.PrefillConfig("bs1024_g2_d64", 2, 8, 4, 64, 1024, 500, 1500, 70, 400),
 ]
 
 

@@ -151,6 +151,7 @@ PREFILL = [
     W.PrefillConfig("ptok_g8_d64", 2, 8, 1, 64, 256, 0, 300, 1, 90, cache_dtype=W.CACHE_FP8_TOKEN),
     W.PrefillConfig("ptok_mixed", 2, 32, 8, 128, 256, 0, 600, 60, 200, cache_dtype=W.CACHE_FP8_TOKEN, decode_seqs=4,
                     decode_hist_lo=1, decode_hist_hi=700),
+    W.PrefillConfig("ptok_bs8", 2, 8, 2, 128, 8, 10, 150, 20, 90, cache_dtype=W.CACHE_FP8_TOKEN),
 ]
 
 
