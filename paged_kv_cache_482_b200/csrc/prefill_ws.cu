@@ -10,22 +10,28 @@
 // a (chunk token, query head of the group) pair), one CTA per SM. Warp roles:
 //   warps 0-3  softmax of query tile A (one row per thread);
 //   warps 4-7  softmax of query tile B;
-//   warp 8     producer: tensor-map copies of 64-token K/V tiles into a
-//              four-stage ring (and the zeroing of V rows past the causal
+//   warp 8     producer: tensor-map copies of 128-token K/V tiles into a
+//              two-stage ring (and the zeroing of V rows past the causal
 //              end on the last tile);
 //   warp 9     tensor-memory allocation and the MMA issue:
-//                S_A(0), S_B(0), S_A(1), S_B(1), then per tile j
-//                PV_A(j), PV_B(j), S_A(j+2), S_B(j+2), ...
-//              so that the tensor core works on one tile while the other
-//              tile's softmax runs, both tiles share every K/V tile, and S
-//              of the tile after next is ready before the softmax needs it.
-// Tensor memory (512 columns): two S buffers per query tile (64 columns
-// each) and O_A, O_B (128 columns each). P (bf16, two per 32-bit column)
-// is written over the first 32 columns of the S buffer it came from and P V
-// takes its A operand from tensor memory, so P never touches shared memory;
-// S of tile j + 2 reuses the buffer only after P V of tile j, issued before
-// it by the same thread. The softmax waits for P V of the previous tile only
-// when it has to rescale O.
+//                S_A(0), S_B(0), then per tile j
+//                PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ...
+//              so that the tensor core works on one query tile while the
+//              other tile's softmax runs, and both share every K/V tile.
+// The 128-token KV tile makes S an M = N = 128 MMA: per unit of work it
+// reads half as much shared memory for the Q operand as N = 64 does, which
+// is what paced the tensor pipe with 64-token tiles.
+// Tensor memory (512 columns): S_A, S_B (128 columns each) and O_A, O_B
+// (128 columns each). P (bf16, two per 32-bit column) is written over the
+// first 64 columns of the S it came from and P V takes its A operand from
+// tensor memory, so P never touches shared memory. S of tile j + 1 reuses
+// the columns of P of tile j: it is issued after P V of tile j by the same
+// thread, and MMAs from one thread run in issue order. The commit of S(j+1)
+// therefore also covers P V(j): a softmax thread that sees S(j+1) may
+// rescale O without waiting for anything else.
+// The softmax makes two passes over S in tensor memory (row maximum, then
+// exponentials), 64 columns at a time, to keep its registers below the
+// budget of one 320-thread CTA per SM.
 // Everything between roles goes through mbarriers (full / empty K/V stages,
 // S ready, P ready, O done); every wait is bounded (1 s) and reports
 // PKV_DEVERR_TIMEOUT. The softmax uses the same arithmetic as prefill.cu:
@@ -40,8 +46,8 @@ namespace {
 using namespace tc;
 
 constexpr int kRowsT = 128;  // rows per query tile (MMA M)
-constexpr int kBN = 64;      // KV tokens per tile
-constexpr int kStages = 4;   // K/V ring depth
+constexpr int kBN = 128;     // KV tokens per tile
+constexpr int kStages = 2;   // K/V ring depth
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 64;  // + producer warp + MMA warp
 constexpr int kProducerWarp = 8;
@@ -65,9 +71,9 @@ struct WsLayout {
 struct Bars {
     uint64_t kv_full[kStages];
     uint64_t kv_empty[kStages];
-    uint64_t s_full[2][2];  // [query tile][S buffer]
-    uint64_t p_full[2][2];  // [query tile][S buffer]: P of a tile written
-    uint64_t o_done[2][2];  // [query tile][S buffer]: P V of a tile done
+    uint64_t s_full[2];     // [query tile]
+    uint64_t p_full[2];     // [query tile]: P of a tile written
+    uint64_t o_done[2];     // [query tile]: P V of a tile done
     uint64_t q_full;
     uint64_t vtail;
     uint64_t drained;
@@ -181,12 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->kv_empty[i], 1);
         }
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&bars->s_full[x][0], 1);
-            mbar_init(&bars->s_full[x][1], 1);
-            mbar_init(&bars->p_full[x][0], kRowsT);
-            mbar_init(&bars->p_full[x][1], kRowsT);
-            mbar_init(&bars->o_done[x][0], 1);
-            mbar_init(&bars->o_done[x][1], 1);
+            mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->p_full[x], kRowsT);
+            mbar_init(&bars->o_done[x], 1);
         }
         mbar_init(&bars->q_full, kSoftmaxThreads);
         mbar_init(&bars->vtail, 1);
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================ softmax, query tile X
         const uint32_t sq = sq0 + X * L::kQTile;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tmem_s0 = tmem + X * 2 * kBN;  // S buffers of this query tile: tmem_s0 + b * kBN
+        const uint32_t tmem_s = tmem + X * kBN;  // S (and P over its first 64 columns)
         const uint32_t tmem_o = tmem + 256 + X * 128;
         {
             constexpr int kChunks = D / 8;
@@ -229,45 +232,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
-            // warp-uniform: the tensor-memory loads and stores below are warp-wide
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[X][j & 1], static_cast<uint32_t>((j >> 1) & 1)))) {
+            // S_X(j) done implies P V_X(j - 1) done (issued before it): O_X is stable
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[X], static_cast<uint32_t>(j & 1)))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t tmem_s = tmem_s0 + (j & 1) * kBN;
             const int kv0 = j * kBN;
             const bool masked = kv0 + kBN - 1 > p_first;
-            float x[kBN];  // raw scores; the (positive) scale is applied below
-            static_assert(kBN == 64, "one 64-column tensor-memory load per tile");
-            tmem_ld64(tmem_s + lane_base, x);
-            if (masked) {
+            // pass 1: the row maximum over two 64-column halves
+            float mraw = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < kBN; ++i)
-                    if (kv0 + i > row_pos) x[i] = -INFINITY;
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[64];
+                tmem_ld64(tmem_s + lane_base + hh * 64, x);
+                if (masked) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (kv0 + hh * 64 + i > row_pos) x[i] = -INFINITY;
+                }
+                float m8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+                for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+                mraw = fmaxf(mraw, fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))));
             }
-            float m8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = x[k];
-#pragma unroll
-            for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-            // the tile's maximum in the exp2 domain (the scale is positive)
-            const float mx = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            const float mx = sl2 * mraw;
             if (j == 0) {
-                m_run = mx;  // O is written, not accumulated, by the first P V
+                m_run = mx;
             } else {
                 const bool grow = mx > m_run + 8.0f;
                 if (__any_sync(0xffffffffu, grow)) {
-                    // O_X must hold P V of tile j - 1 before it is rescaled. (This
-                    // buffer's barrier can be at most one phase past the one
-                    // waited for: P V of tile j + 1 needs this tile's P first.)
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[X][(j - 1) & 1],
-                                                           static_cast<uint32_t>(((j - 1) >> 1) & 1)))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
                     const float alpha = grow ? fast_exp2(m_run - mx) : 1.0f;
                     if (grow) {
                         m_run = mx;
@@ -283,26 +280,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // P = exp2(s * scale - m) as bf16 pairs over the first 32 columns of
-            // this S buffer; l sums the rounded weights
+            // pass 2: P as bf16 pairs over columns 0..63 (half hh of the scores ->
+            // columns 32 hh .. 32 hh + 31, read before they are overwritten)
             float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            float pw[kBN / 2];
 #pragma unroll
-            for (int i = 0; i < kBN / 2; ++i) {
-                const uint32_t w = pack_bf16(fast_exp2(fmaf(x[2 * i], sl2, -m_run)),
-                                             fast_exp2(fmaf(x[2 * i + 1], sl2, -m_run)));
-                l4[i & 3] = fma_bf16x2_acc(w, 0x3F803F80u, l4[i & 3]);  // + both rounded weights (x 1.0)
-                pw[i] = __uint_as_float(w);
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[64];
+                tmem_ld64(tmem_s + lane_base + hh * 64, x);
+                if (masked) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (kv0 + hh * 64 + i > row_pos) x[i] = -INFINITY;
+                }
+                float pw[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t w = pack_bf16(fast_exp2(fmaf(x[2 * i], sl2, -m_run)),
+                                                 fast_exp2(fmaf(x[2 * i + 1], sl2, -m_run)));
+                    l4[i & 3] = fma_bf16x2_acc(w, 0x3F803F80u, l4[i & 3]);
+                    pw[i] = __uint_as_float(w);
+                }
+                tmem_st32(tmem_s + lane_base + hh * 32, pw);
             }
-            tmem_st32(tmem_s + lane_base, pw);
             l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             tc_fence_before();
-            // per S buffer: the softmax can be a tile ahead of the MMA issue
-            // (S of tile j + 2 needs P V of tile j), never two phases of one barrier
-            mbar_arrive(&bars->p_full[X][j & 1]);
+            mbar_arrive(&bars->p_full[X]);
         }
-        if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X][(n_tiles - 1) & 1],
-                                                    static_cast<uint32_t>(((n_tiles - 1) >> 1) & 1)))) {
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], 0))) {
             tc_fence_after();
             const float inv = 1.0f / l_run;
 #pragma unroll
@@ -369,62 +373,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================ MMA issue
         if (lane == 0) {
             bool ok = mbar_wait(&bars->q_full, 0);
-            auto issue_s = [&](int x, int j) {  // S_x(j) into S buffer j & 1 of query tile x
+            auto issue_s = [&](int x, int j) {
                 const uint32_t sq = sq0 + x * L::kQTile, sk = kbuf(j);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * kRowsT * 128 + (kk & 3) * 32);
                     const uint32_t boff = static_cast<uint32_t>((kk >> 2) * kBN * 128 + (kk & 3) * 32);
-                    mma_bf16(tmem + (x * 2 + (j & 1)) * kBN, sw128_desc(sq + aoff, 16, 1024),
-                             sw128_desc(sk + boff, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                    mma_bf16(tmem + x * kBN, sw128_desc(sq + aoff, 16, 1024), sw128_desc(sk + boff, 16, 1024),
+                             kIdescS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full[x][j & 1]);
+                mma_commit(&bars->s_full[x]);
             };
-            auto issue_pv = [&](int x, int j) {  // A = P_x(j) in tensor memory: 8 columns per 16 tokens
-                const uint32_t tp = tmem + (x * 2 + (j & 1)) * kBN, sv = vbuf(j);
+            auto issue_pv = [&](int x, int j, bool last) {  // A = P_x(j) over the first 64 columns of S_x
+                const uint32_t tp = tmem + x * kBN, sv = vbuf(j);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
                     mma_bf16_ts(tmem + 256 + x * 128, tp + kk * 8,
                                 sw128_desc(sv + static_cast<uint32_t>(kk * 16 * 128), kBN * 128, 1024), kIdescPV,
                                 (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&bars->o_done[x][j & 1]);
+                if (last) mma_commit(&bars->o_done[x]);
             };
             auto kv_ready = [&](int j) {
                 const bool r = mbar_wait(&bars->kv_full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
                 tc_fence_after();
                 return r;
             };
-            // S of the first two tiles
-            for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {
-                ok = kv_ready(j);
-                if (ok) {
-                    issue_s(0, j);
-                    issue_s(1, j);
-                }
+            ok = ok && kv_ready(0);
+            if (ok) {
+                issue_s(0, 0);
+                issue_s(1, 0);
             }
-            // Per tile j: P V of both query tiles as soon as their P is
-            // ready, release tile j's ring stage, then S of tile j + 2 (its
-            // copy has had a whole tile to land; the softmax needs it only
-            // two tiles later).
+            // per tile j: P V_A(j), S_A(j + 1), P V_B(j), S_B(j + 1); K/V of tile
+            // j + 1 is awaited only after P V_A(j) is on the tensor pipe
             for (int j = 0; ok && j < n_tiles; ++j) {
-                if (j == n_tiles - 1) ok = mbar_wait(&bars->vtail, 0);  // V rows past the end are zero
+                const bool more = j + 1 < n_tiles;
+                if (!more) ok = mbar_wait(&bars->vtail, 0);
                 for (int x = 0; x < 2 && ok; ++x) {
-                    if (!mbar_wait(&bars->p_full[x][j & 1], static_cast<uint32_t>((j >> 1) & 1))) {
+                    if (!mbar_wait(&bars->p_full[x], static_cast<uint32_t>(j & 1))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    issue_pv(x, j);  // P_x(j) was read from S buffer j & 1: free for S_x(j + 2)
-                }
-                if (!ok) break;
-                mma_commit(&bars->kv_empty[j % kStages]);  // tile j's K and V are consumed
-                if (j + 2 < n_tiles) {
-                    if (!kv_ready(j + 2)) {
-                        ok = false;
-                        break;
+                    issue_pv(x, j, !more);
+                    if (x == 1) mma_commit(&bars->kv_empty[j % kStages]);
+                    if (more) {
+                        if (x == 0 && !kv_ready(j + 1)) {
+                            ok = false;
+                            break;
+                        }
+                        issue_s(x, j + 1);  // after P V_x(j): S_x is free
                     }
-                    issue_s(0, j + 2);
-                    issue_s(1, j + 2);
                 }
             }
             if (!ok) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
