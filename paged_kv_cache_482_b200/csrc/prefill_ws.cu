@@ -49,9 +49,12 @@ constexpr int kRowsT = 128;  // rows per query tile (MMA M)
 constexpr int kBN = 128;     // KV tokens per tile
 constexpr int kStages = 2;   // K/V ring depth
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = kSoftmaxThreads + 64;  // + producer warp + MMA warp
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;  // bf16: tensor-map producer; E4M3: converter
 constexpr int kMmaWarp = 9;
+constexpr int kConvWarps = 3;     // E4M3 converters: warps 8, 10, 11
+// bf16: softmax + producer + MMA warps; E4M3: softmax + three converters + MMA
+template <bool FP8>
+constexpr int ws_threads() { return FP8 ? kSoftmaxThreads + 32 * (kConvWarps + 1) : kSoftmaxThreads + 64; }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -110,8 +113,8 @@ __device__ __forceinline__ void ws_kv_tile(const CUtensorMap *mk, const CUtensor
     }
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int G, bool FP8>
+__global__ void __launch_bounds__(ws_threads<FP8>(), 1)
     paged_prefill_ws_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
                             const __grid_constant__ CUtensorMap map_v) {
     using L = WsLayout<D>;
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                c > a.max_q_len;
     if (!bad) {
         const int nblk_seq = (ctx + a.block_size - 1) >> log2_bs;
-        for (int i = tid; i < nblk_seq; i += kThreads) {
+        for (int i = tid; i < nblk_seq; i += ws_threads<FP8>()) {
             const int32_t b = table_g[i];
             if (b < 0 || b >= a.num_blocks) bad = true;
             if (i < kTableCap) table_s[i] = b;
@@ -183,12 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) tmem_alloc(smem_addr(&bars->tmem), kTmemCols);
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bars->kv_full[i], 1);
+            mbar_init(&bars->kv_full[i], FP8 ? kConvWarps : 1);
             mbar_init(&bars->kv_empty[i], 1);
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&bars->s_full[x], 1);
-            mbar_init(&bars->p_full[x], kRowsT);
+            mbar_init(&bars->p_full[x], kRowsT / 32);  // one arrive per softmax warp
             mbar_init(&bars->o_done[x], 1);
         }
         mbar_init(&bars->q_full, kSoftmaxThreads);
@@ -228,7 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int p_first = ctx - c + t0 + X * TQ;  // position of this tile's first row
         const int row_pos = row_live ? ctx - c + row_tok : p_last;
-        const float sl2 = a.scale * kLog2e;
+        // E4M3 with one scale per KV head: k_scale folds into the softmax scale
+        const float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
@@ -240,75 +244,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int kv0 = j * kBN;
             const bool masked = kv0 + kBN - 1 > p_first;
-            // pass 1: the row maximum over two 64-column halves
-            float mraw = -INFINITY;
+            // the row's 128 scores (one statement: two loads and their wait)
+            float x[kBN];
+            tmem_ld128(tmem_s + lane_base, x);
+            if (masked) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float x[64];
-                tmem_ld64(tmem_s + lane_base + hh * 64, x);
-                if (masked) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (kv0 + hh * 64 + i > row_pos) x[i] = -INFINITY;
-                }
-                float m8[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) m8[k] = x[k];
-#pragma unroll
-                for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-                mraw = fmaxf(mraw, fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))));
+                for (int i = 0; i < kBN; ++i)
+                    if (kv0 + i > row_pos) x[i] = -INFINITY;
             }
-            const float mx = sl2 * mraw;
+            float m8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+            for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+            const float mx = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            float alpha = 1.0f;
+            bool rescale = false;
             if (j == 0) {
                 m_run = mx;
             } else {
                 const bool grow = mx > m_run + 8.0f;
-                if (__any_sync(0xffffffffu, grow)) {
-                    const float alpha = grow ? fast_exp2(m_run - mx) : 1.0f;
-                    if (grow) {
-                        m_run = mx;
-                        l_run *= alpha;
-                    }
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        float v[32];
-                        tmem_ld32(tmem_o + lane_base + ch * 32, v);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                        tmem_st32(tmem_o + lane_base + ch * 32, v);
-                    }
+                rescale = __any_sync(0xffffffffu, grow);
+                if (grow) {
+                    alpha = fast_exp2(m_run - mx);
+                    m_run = mx;
+                    l_run *= alpha;
                 }
             }
-            // pass 2: P as bf16 pairs over columns 0..63 (half hh of the scores ->
-            // columns 32 hh .. 32 hh + 31, read before they are overwritten)
+            // P as bf16 pairs over columns 0..63 of S: scores 64 hh .. 64 hh + 63
+            // go to columns 32 hh .. 32 hh + 31 (all scores are in registers)
+            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
             float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                float x[64];
-                tmem_ld64(tmem_s + lane_base + hh * 64, x);
-                if (masked) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (kv0 + hh * 64 + i > row_pos) x[i] = -INFINITY;
-                }
                 float pw[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const uint32_t w = pack_bf16(fast_exp2(fmaf(x[2 * i], sl2, -m_run)),
-                                                 fast_exp2(fmaf(x[2 * i + 1], sl2, -m_run)));
+                    const float2 t = __ffma2_rn(make_float2(x[hh * 64 + 2 * i], x[hh * 64 + 2 * i + 1]), sl2x2, nm2);
+                    const uint32_t w = pack_bf16(fast_exp2(t.x), fast_exp2(t.y));
                     l4[i & 3] = fma_bf16x2_acc(w, 0x3F803F80u, l4[i & 3]);
                     pw[i] = __uint_as_float(w);
                 }
-                tmem_st32(tmem_s + lane_base + hh * 32, pw);
+                tmem_st32_async(tmem_s + lane_base + hh * 32, pw);
             }
             l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            // O rescale once the scores are out of the registers; P V of this
+            // tile is issued only after the arrive below
+            if (rescale) {
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    float v[32];
+                    tmem_ld32(tmem_o + lane_base + ch * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32_async(tmem_o + lane_base + ch * 32, v);
+                }
+            }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->p_full[X]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full[X]);
         }
         if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], 0))) {
             tc_fence_after();
-            const float inv = 1.0f / l_run;
+            const float inv = (FP8 ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 float v[32];
@@ -328,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (row == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
         }
         __syncwarp();
-    } else if (warp == kProducerWarp) {
-        // ================================================ producer
+    } else if (!FP8 && warp == kProducerWarp) {
+        // ================================================ producer (bf16)
         int issued = 0;
         if (lane == 0) {
             for (int j = 0; j < n_tiles; ++j) {
@@ -369,6 +369,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_wait(&bars->kv_full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
         }
         __syncwarp();
+    } else if (FP8 && warp != kMmaWarp) {
+        // ================================================ E4M3 converters (warps 8, 10, 11)
+        // Each thread loads 16-code chunks of the tile's K and V rows, widens
+        // them exactly to bf16 and stores them into the swizzled stage the
+        // MMAs read; rows past the causal end are written as zeros. The next
+        // tile's loads are in flight while the thread waits for its stage.
+        constexpr int kCW = kConvWarps * 32;
+        constexpr int kCPR = D / 16;              // 16-code chunks per row
+        constexpr int kChunks = 2 * kBN * kCPR;   // K and V chunks of one tile
+        constexpr int kPer = (kChunks + kCW - 1) / kCW;
+        const int ct = (warp == kProducerWarp ? 0 : warp - kMmaWarp) * 32 + lane;
+        const uint8_t *kpool = static_cast<const uint8_t *>(a.k_cache);
+        const uint8_t *vpool = static_cast<const uint8_t *>(a.v_cache);
+        uint4 w[kPer];
+        auto load = [&](int j) {
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int idx = ct + u * kCW;
+                w[u] = make_uint4(0, 0, 0, 0);
+                if (idx < kChunks) {
+                    const bool isv = idx >= kBN * kCPR;
+                    const int rem = isv ? idx - kBN * kCPR : idx;
+                    const int t = j * kBN + rem / kCPR;
+                    if (t < kv_end) {
+                        const int64_t off =
+                            ((static_cast<int64_t>(table[t >> log2_bs]) * a.num_kv_heads + kh) * a.block_size +
+                             (t & (a.block_size - 1))) * D + (rem % kCPR) * 16;
+                        w[u] = __ldg(reinterpret_cast<const uint4 *>((isv ? vpool : kpool) + off));
+                    }
+                }
+            }
+        };
+        bool ok = true;
+        load(0);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j % kStages, use = j / kStages;
+            if (use > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[st], static_cast<uint32_t>((use - 1) & 1)))) {
+                ok = false;
+                break;
+            }
+            const uint32_t sk = kbuf(j), sv = vbuf(j);
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int idx = ct + u * kCW;
+                if (idx < kChunks) {
+                    const bool isv = idx >= kBN * kCPR;
+                    const int rem = isv ? idx - kBN * kCPR : idx;
+                    const int r = rem / kCPR, c16 = 2 * (rem % kCPR);
+                    const uint32_t dst = isv ? sv : sk;
+                    st_shared16(dst + swz(kBN, r, c16), e4m3x8_to_bf16x8(make_uint2(w[u].x, w[u].y)));
+                    st_shared16(dst + swz(kBN, r, c16 + 1), e4m3x8_to_bf16x8(make_uint2(w[u].z, w[u].w)));
+                }
+            }
+            fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->kv_full[st]);
+            if (j + 1 < n_tiles) load(j + 1);
+        }
+        if (!ok && lane == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
+        __syncwarp();
     } else {
         // ================================================ MMA issue
         if (lane == 0) {
@@ -407,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // j + 1 is awaited only after P V_A(j) is on the tensor pipe
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const bool more = j + 1 < n_tiles;
-                if (!more) ok = mbar_wait(&bars->vtail, 0);
+                if (!FP8 && !more) ok = mbar_wait(&bars->vtail, 0);  // E4M3: converters zero the tail
                 for (int x = 0; x < 2 && ok; ++x) {
                     if (!mbar_wait(&bars->p_full[x], static_cast<uint32_t>(j & 1))) {
                         ok = false;
@@ -441,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, int G>
+template <int D, int G, bool FP8>
 cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int TQ = kRowsT / G;
     const int tiles = (a.max_q_len + 2 * TQ - 1) / (2 * TQ);
@@ -454,35 +515,36 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     CUtensorMap mk, mv;
     memset(&mk, 0, sizeof(mk));
     memset(&mv, 0, sizeof(mv));
-    if (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)) return cudaErrorInvalidValue;
-    auto kern = paged_prefill_ws_kernel<D, G>;
+    // the E4M3 path loads the codes with plain loads: no tensor maps
+    if (!FP8 && (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)))
+        return cudaErrorInvalidValue;
+    auto kern = paged_prefill_ws_kernel<D, G, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(WsLayout<D>::kAlloc));
     if (e != cudaSuccess) return e;
-    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), kThreads, WsLayout<D>::kAlloc, stream>>>(a, tiles, log2_bs,
-                                                                                                   mk, mv);
+    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), ws_threads<FP8>(), WsLayout<D>::kAlloc, stream>>>(
+        a, tiles, log2_bs, mk, mv);
     return cudaGetLastError();
+}
+
+template <int D, bool FP8>
+cudaError_t launch_ws_g(const PrefillArgs &a, int g, cudaStream_t stream) {
+    switch (g) {
+        case 1: return launch_ws<D, 1, FP8>(a, stream);
+        case 2: return launch_ws<D, 2, FP8>(a, stream);
+        case 4: return launch_ws<D, 4, FP8>(a, stream);
+        case 8: return launch_ws<D, 8, FP8>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
-    if (a.head_dim == 128) {
-        switch (g) {
-            case 1: return launch_ws<128, 1>(a, stream);
-            case 2: return launch_ws<128, 2>(a, stream);
-            case 4: return launch_ws<128, 4>(a, stream);
-            case 8: return launch_ws<128, 8>(a, stream);
-        }
-    } else if (a.head_dim == 64) {
-        switch (g) {
-            case 1: return launch_ws<64, 1>(a, stream);
-            case 2: return launch_ws<64, 2>(a, stream);
-            case 4: return launch_ws<64, 4>(a, stream);
-            case 8: return launch_ws<64, 8>(a, stream);
-        }
-    }
+    if (a.token_scales) return cudaErrorInvalidValue;  // per-token scales: the one-tile kernel
+    if (a.head_dim == 128) return a.fp8 ? launch_ws_g<128, true>(a, g, stream) : launch_ws_g<128, false>(a, g, stream);
+    if (a.head_dim == 64) return a.fp8 ? launch_ws_g<64, true>(a, g, stream) : launch_ws_g<64, false>(a, g, stream);
     return cudaErrorInvalidValue;
 }
 

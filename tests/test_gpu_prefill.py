@@ -2,7 +2,7 @@
 
 Pools are filled with store_kvcache (history, then the chunk tokens) and the
 tcgen05 prefill kernel attends; the oracle does the same on the host. Small
-cases compare every row; the full-size Qwen3-8B-shaped step compares sampled
+cases compare every row; the full-size Qwen3-8B-shaped steps (bf16 and E4M3 caches) compare sampled
 rows, each recomputed by the oracle as a one-token chunk at its position
 (a query's result depends only on the tokens up to it).
 """
@@ -73,6 +73,14 @@ SMALL = [
     # one block spanning sixteen 64-token tiles
     W.PrefillConfig("bs8_g4", 3, 32, 8, 128, 8, 0, 200, 40, 300),
     W.PrefillConfig("bs1024_g2_d64", 2, 8, 4, 64, 1024, 500, 1500, 70, 400),
+    # E4M3 chunks longer than one query tile take the converter warps of the
+    # warp-specialised kernel: every group size, both head sizes, the block
+    # size extremes, and tails that end inside a 128-token tile
+    W.PrefillConfig("fp8_g1_bs8", 2, 4, 4, 128, 8, 0, 300, 100, 300, cache_dtype=W.CACHE_FP8),
+    W.PrefillConfig("fp8_g2_d64_bs1024", 2, 8, 4, 64, 1024, 500, 1500, 70, 400, cache_dtype=W.CACHE_FP8),
+    W.PrefillConfig("fp8_g4_d128_bs256", 3, 32, 8, 128, 256, 0, 600, 33, 520, cache_dtype=W.CACHE_FP8),
+    W.PrefillConfig("fp8_mixed", 2, 32, 8, 128, 16, 0, 700, 60, 200, decode_seqs=6, decode_hist_lo=1,
+                    decode_hist_hi=900, cache_dtype=W.CACHE_FP8),
 ]
 
 
@@ -146,8 +154,9 @@ def test_empty_chunks_and_loose_bound():
     compare(out, ref[keep.numpy()], False, "gaps")
 
 
-def test_full_size_sampled():
-    cfg = W.PREFILL_CONFIGS["prefill_qwen3_8b"]
+@pytest.mark.parametrize("name", ["prefill_qwen3_8b", "prefill_fp8"])
+def test_full_size_sampled(name):
+    cfg = W.PREFILL_CONFIGS[name]
     wl = W.generate_prefill(cfg, 0, device="cuda")
     out, kp, vp, st = run_gpu(wl)
     assert st == K.PKV_OK
@@ -166,11 +175,13 @@ def test_full_size_sampled():
     bt = torch.stack([wl.block_tables[s] for s, _ in rows]).cpu()
     ctx = torch.tensor([int(cl[s] - (cu[s + 1] - cu[s]) + j + 1) for s, j in rows], dtype=torch.int32)
     cu1 = torch.arange(len(rows) + 1, dtype=torch.int32)
+    ks = wl.k_scale.cpu() if wl.is_fp8 else None
+    vs = wl.v_scale.cpu() if wl.is_fp8 else None
     ref, rst = O.paged_attention_prefill(q_rows, kp_h, vp_h, bt, cu1, ctx, cfg.num_kv_heads, cfg.block_size,
-                                         cfg.softmax_scale, num_threads=8)
+                                         cfg.softmax_scale, k_scale=ks, v_scale=vs, num_threads=8)
     assert rst == O.ORC_OK
     got = torch.stack([out[int(cu[s]) + j] for s, j in rows])
-    compare(got, ref, False, "prefill_qwen3_8b sampled")
+    compare(got, ref, wl.is_fp8, f"{name} sampled")
 
 
 def test_device_bounds():
