@@ -119,8 +119,10 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                             const __grid_constant__ CUtensorMap map_v) {
     using L = WsLayout<D>;
     constexpr int TQ = kRowsT / G;  // chunk tokens per query tile
-    constexpr uint32_t kIdescS = idesc_bf16(kRowsT, kBN, false);
-    constexpr uint32_t kIdescPV = idesc_bf16(kRowsT, D, true);
+    // bf16 cache: bf16 operands. E4M3 cache: f16 operands (one conversion per
+    // two codes; Q is scaled into f16 range per row, see the staging below).
+    constexpr uint32_t kIdescS = FP8 ? idesc_f16(kRowsT, kBN, false) : idesc_bf16(kRowsT, kBN, false);
+    constexpr uint32_t kIdescPV = FP8 ? idesc_f16(kRowsT, D, true) : idesc_bf16(kRowsT, D, true);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -213,26 +215,61 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tmem_s = tmem + X * kBN;  // S (and P over its first 64 columns)
         const uint32_t tmem_o = tmem + 256 + X * 128;
+        // E4M3 with one scale per KV head: k_scale folds into the softmax scale
+        float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
         {
             constexpr int kChunks = D / 8;
             const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q);
-            for (int i = row; i < kRowsT * kChunks; i += kRowsT) {
-                const int r = i / kChunks, c16 = i % kChunks;
-                const int tok = t0 + X * TQ + r / G;
-                const bool valid = tok < c;
-                const int64_t elem =
-                    (static_cast<int64_t>(q0 + (valid ? tok : 0)) * nq + kh * G + r % G) * D + c16 * 8;
-                cp_async16(sq + swz(kRowsT, r, c16), qp + elem, valid ? 16u : 0u);
+            if constexpr (!FP8) {
+                for (int i = row; i < kRowsT * kChunks; i += kRowsT) {
+                    const int r = i / kChunks, c16 = i % kChunks;
+                    const int tok = t0 + X * TQ + r / G;
+                    const bool valid = tok < c;
+                    const int64_t elem =
+                        (static_cast<int64_t>(q0 + (valid ? tok : 0)) * nq + kh * G + r % G) * D + c16 * 8;
+                    cp_async16(sq + swz(kRowsT, r, c16), qp + elem, valid ? 16u : 0u);
+                }
+                cp_async_commit();
+                cp_async_wait0();
+            } else {
+                // This thread's own row, times 2^kq with kq chosen so that the row's
+                // largest |q| lies in [2^14, 2^15): exact in f16 (a bf16 value has 8
+                // significant bits) down to 2^-31 of the row maximum. 2^-kq folds
+                // into the row's softmax scale. kq >= -114 (|q| < 2^129, infinities
+                // included); it is capped at 60 so that 2^-kq times the softmax
+                // scale stays a normal float: rows so small that the cap binds
+                // have scores below 2^-45 times the key norms, whose softmax is
+                // uniform either way.
+                const uint4 *qrow = reinterpret_cast<const uint4 *>(
+                    qp + (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + kh * G + row % G) * D);
+                uint4 qv[kChunks];
+                float amax = 0.0f;
+#pragma unroll
+                for (int c16 = 0; c16 < kChunks; ++c16) {
+                    qv[c16] = row_live ? __ldg(qrow + c16) : make_uint4(0, 0, 0, 0);
+                    const uint32_t wds[4] = {qv[c16].x, qv[c16].y, qv[c16].z, qv[c16].w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        amax = fmaxf(amax, fmaxf(fabsf(bf16lo(wds[k])), fabsf(bf16hi(wds[k]))));
+                }
+                const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 126;  // amax < 2^e
+                const int kq = min(60, 15 - e);
+                const float qs = __int_as_float((kq + 127) << 23);
+                sl2 *= __int_as_float((127 - kq) << 23);
+#pragma unroll
+                for (int c16 = 0; c16 < kChunks; ++c16) {
+                    const uint32_t wds[4] = {qv[c16].x, qv[c16].y, qv[c16].z, qv[c16].w};
+                    uint32_t h[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) h[k] = pack_f16(bf16lo(wds[k]) * qs, bf16hi(wds[k]) * qs);
+                    st_shared16(sq + swz(kRowsT, row, c16), make_uint4(h[0], h[1], h[2], h[3]));
+                }
             }
-            cp_async_commit();
-            cp_async_wait0();
             fence_proxy_async_smem();
             mbar_arrive(&bars->q_full);
         }
         const int p_first = ctx - c + t0 + X * TQ;  // position of this tile's first row
         const int row_pos = row_live ? ctx - c + row_tok : p_last;
-        // E4M3 with one scale per KV head: k_scale folds into the softmax scale
-        const float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
@@ -282,8 +319,14 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float2 t = __ffma2_rn(make_float2(x[hh * 64 + 2 * i], x[hh * 64 + 2 * i + 1]), sl2x2, nm2);
-                    const uint32_t w = pack_bf16(fast_exp2(t.x), fast_exp2(t.y));
-                    l4[i & 3] = fma_bf16x2_acc(w, 0x3F803F80u, l4[i & 3]);
+                    uint32_t w;
+                    if constexpr (FP8) {  // P in f16 (the E4M3 path's operand type)
+                        w = pack_f16(fast_exp2(t.x), fast_exp2(t.y));
+                        l4[i & 3] = fma_f16x2_acc(w, 0x3C003C00u, l4[i & 3]);
+                    } else {
+                        w = pack_bf16(fast_exp2(t.x), fast_exp2(t.y));
+                        l4[i & 3] = fma_bf16x2_acc(w, 0x3F803F80u, l4[i & 3]);
+                    }
                     pw[i] = __uint_as_float(w);
                 }
                 tmem_st32_async(tmem_s + lane_base + hh * 32, pw);
@@ -372,37 +415,46 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
     } else if (FP8 && warp != kMmaWarp) {
         // ================================================ E4M3 converters (warps 8, 10, 11)
         // Each thread loads 16-code chunks of the tile's K and V rows, widens
-        // them exactly to bf16 and stores them into the swizzled stage the
+        // them exactly to f16 and stores them into the swizzled stage the
         // MMAs read; rows past the causal end are written as zeros. The next
         // tile's loads are in flight while the thread waits for its stage.
         constexpr int kCW = kConvWarps * 32;
-        constexpr int kCPR = D / 16;              // 16-code chunks per row
-        constexpr int kChunks = 2 * kBN * kCPR;   // K and V chunks of one tile
-        constexpr int kPer = (kChunks + kCW - 1) / kCW;
+        constexpr int kCPR = D / 16;                  // 16-code chunks per row
+        constexpr int kHalf = kBN * kCPR;             // chunks of one operand's tile
+        constexpr int kPer = (kHalf + kCW - 1) / kCW;  // per thread and operand
         const int ct = (warp == kProducerWarp ? 0 : warp - kMmaWarp) * 32 + lane;
-        const uint8_t *kpool = static_cast<const uint8_t *>(a.k_cache);
-        const uint8_t *vpool = static_cast<const uint8_t *>(a.v_cache);
-        uint4 w[kPer];
-        auto load = [&](int j) {
+        uint4 wk[kPer], wv[kPer];
+        auto load = [&](uint4 (&w)[kPer], const void *pool, int j) {
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int idx = ct + u * kCW;
+                const int t = j * kBN + idx / kCPR;
                 w[u] = make_uint4(0, 0, 0, 0);
-                if (idx < kChunks) {
-                    const bool isv = idx >= kBN * kCPR;
-                    const int rem = isv ? idx - kBN * kCPR : idx;
-                    const int t = j * kBN + rem / kCPR;
-                    if (t < kv_end) {
-                        const int64_t off =
-                            ((static_cast<int64_t>(table[t >> log2_bs]) * a.num_kv_heads + kh) * a.block_size +
-                             (t & (a.block_size - 1))) * D + (rem % kCPR) * 16;
-                        w[u] = __ldg(reinterpret_cast<const uint4 *>((isv ? vpool : kpool) + off));
-                    }
+                if (idx < kHalf && t < kv_end) {
+                    const int64_t off = ((static_cast<int64_t>(table[t >> log2_bs]) * a.num_kv_heads + kh) *
+                                             a.block_size + (t & (a.block_size - 1))) * D + (idx % kCPR) * 16;
+                    w[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(pool) + off));
                 }
             }
         };
+        auto store = [&](const uint4 (&w)[kPer], uint32_t dst) {
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int idx = ct + u * kCW;
+                if (idx < kHalf) {
+                    const int r = idx / kCPR, c16 = 2 * (idx % kCPR);
+                    const uint2 h0 = e4m3x4_to_f16x4(w[u].x), h1 = e4m3x4_to_f16x4(w[u].y);
+                    const uint2 h2 = e4m3x4_to_f16x4(w[u].z), h3 = e4m3x4_to_f16x4(w[u].w);
+                    st_shared16(dst + swz(kBN, r, c16), make_uint4(h0.x, h0.y, h1.x, h1.y));
+                    st_shared16(dst + swz(kBN, r, c16 + 1), make_uint4(h2.x, h2.y, h3.x, h3.y));
+                }
+            }
+            fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+            __syncwarp();
+        };
         bool ok = true;
-        load(0);
+        load(wk, a.k_cache, 0);
+        load(wv, a.v_cache, 0);
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages, use = j / kStages;
             if (use > 0 &&
@@ -410,23 +462,12 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                 ok = false;
                 break;
             }
-            const uint32_t sk = kbuf(j), sv = vbuf(j);
-#pragma unroll
-            for (int u = 0; u < kPer; ++u) {
-                const int idx = ct + u * kCW;
-                if (idx < kChunks) {
-                    const bool isv = idx >= kBN * kCPR;
-                    const int rem = isv ? idx - kBN * kCPR : idx;
-                    const int r = rem / kCPR, c16 = 2 * (rem % kCPR);
-                    const uint32_t dst = isv ? sv : sk;
-                    st_shared16(dst + swz(kBN, r, c16), e4m3x8_to_bf16x8(make_uint2(w[u].x, w[u].y)));
-                    st_shared16(dst + swz(kBN, r, c16 + 1), e4m3x8_to_bf16x8(make_uint2(w[u].z, w[u].w)));
-                }
-            }
-            fence_proxy_async_smem();  // the tensor core reads these through the async proxy
-            __syncwarp();
+            // K of tile j, then the next tile's K codes load while V is widened
+            store(wk, kbuf(j));
+            if (j + 1 < n_tiles) load(wk, a.k_cache, j + 1);
+            store(wv, vbuf(j));
             if (lane == 0) mbar_arrive(&bars->kv_full[st]);
-            if (j + 1 < n_tiles) load(j + 1);
+            if (j + 1 < n_tiles) load(wv, a.v_cache, j + 1);
         }
         if (!ok && lane == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
         __syncwarp();

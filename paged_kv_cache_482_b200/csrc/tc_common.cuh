@@ -45,6 +45,12 @@ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major) {
            (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// The same with f16 A and B (format code 0 in both operand fields).
+constexpr uint32_t idesc_f16(int m, int n, bool b_mn_major) {
+    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t holder_saddr, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder_saddr),
                  "r"(ncols)
@@ -211,6 +217,24 @@ __device__ __forceinline__ void st_shared16(uint32_t addr, uint4 v) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Two floats -> f16x2 (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Four E4M3 codes (lowest byte first) -> four f16 values, two per word, with
+// one hardware conversion per pair. Exact: every E4M3 value, NaN included, is
+// an f16 value.
+__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t w) {
+    uint2 r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(r.x), "=r"(r.y)
+        : "r"(w));
+    return r;
 }
 
 // Eight E4M3 codes -> eight bf16 values (exact: every E4M3 value is a bf16 value).
