@@ -556,6 +556,16 @@ def run_prefill_reference(args):
 PREFILL_METRIC = "chunked-prefill paged attention query tokens/sec and achieved tensor TFLOP/s"
 
 
+def prefill_dtype(wl):
+    """Operand types of the prefill kernels for this cache (the tensor cores accumulate in fp32)."""
+    if not wl.is_fp8:
+        return "bf16 x bf16 -> fp32 (tcgen05)"
+    if wl.token_scales:
+        return "e4m3 cache (per-token scales) widened to bf16; bf16 x bf16 -> fp32 (tcgen05)"
+    return ("e4m3 cache widened to f16, Q scaled per row into f16; f16 x f16 -> fp32 (tcgen05); "
+            "chunks of one query tile or less: bf16 operands")
+
+
 def run_prefill(args):
     from paged_kv_cache_482_b200 import pagedkv as K
 
@@ -670,7 +680,7 @@ def run_prefill(args):
             "metric": PREFILL_METRIC, "value": world * T * Kst / (elapsed_ms * 1e-3), "unit": "query tokens/s",
             "n_gpus": world, "steps": Kst, "warmup": args.warmup, "ms_per_step": elapsed_ms / Kst,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 x bf16 -> fp32 (tcgen05)" + (", e4m3 cache" if wl.is_fp8 else ""), "data": "synthetic",
+            "dtype": prefill_dtype(wl), "data": "synthetic",
             "config": {"workload": prefill_desc(c), "query_tokens": T, "kv_tokens": int(wl.context_lens.sum()),
                        "max_q_len": mq, "seed": args.seed,
                        "parallelism": f"replicas x{world} (independent batches, no collective)",
