@@ -73,7 +73,8 @@ struct PrefillArgs {
     int max_q_len;
     void *out;
     int *dev_err;
-    // routing between the two bf16 kernels (set by launch_prefill): 0 = none;
+    // routing between the one-tile and warp-specialised kernels (set by
+    // launch_prefill for bf16 and per-head E4M3 caches): 0 = none;
     // > 0: the one-tile kernel takes the sequences with chunks of at most
     // small_cut tokens, the warp-specialised kernel the others
     int small_cut;
@@ -94,6 +95,6 @@ cudaError_t launch_fused_add_rmsnorm(const NormArgs &a, int num_sms, cudaStream_
 
 bool prefill_supported(int head_dim, int group);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream);
-cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream);  // bf16 cache, warp-specialised
+cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream);  // warp-specialised: bf16, per-head E4M3
 
 }  // namespace pkv

@@ -10,33 +10,30 @@
 // (position p = ctx - c + i) attends over positions 0..p. A decode request is
 // the case c = 1, so one launch serves a batch that mixes both.
 //
-// Work unit: one CTA per (sequence, KV head, 128 query rows). A row is a
-// (chunk token, query head of the group) pair: row r = token r / G, head
-// r % G, so the G heads that share a KV head share every K/V tile. The CTA
-// walks the sequence's KV in tiles of 128 logical tokens up to its last
-// row's position:
+// Work unit: one CTA per (sequence, KV head, 128 query rows), 256 threads and
+// two CTAs per SM. A row is a (chunk token, query head of the group) pair:
+// row r = token r / G, head r % G, so the G heads that share a KV head share
+// every K/V tile. For bf16 and per-head E4M3 caches this kernel takes the
+// chunks of at most one query tile (128 / G tokens, decode requests among
+// them) and prefill_ws.cu the longer ones; per-token E4M3 caches take this
+// kernel for every chunk. The CTA walks the sequence's KV in 64-token tiles up
+// to its last row's position:
 //   1. K/V tiles are gathered through the block table into shared memory,
 //      double buffered, in the 128-byte-swizzled layout the tensor core
 //      reads: for a bf16 cache one thread issues tensor-map (TMA) copies of
 //      whole block runs (a 2-D view of the pool, 64 columns x up to 64 rows
 //      per copy, no multicast) and the V rows past the causal end are zeroed
 //      on the last tile; an E4M3 cache is loaded and widened by the threads;
-//   2. one thread issues S = Q K^T (M 128, N 128, K head_dim) into tensor
-//      memory;
-//   3. the four warps each read their 32 tensor-memory lanes (one row per
-//      thread), apply the causal mask, update the running max / sum in the
-//      exp2 domain and write P = exp2(s - m) as bf16 into shared memory;
-//   4. one thread issues O_tile = P V (M 128, N head_dim, K 128; V read
-//      MN-major straight from its row layout) into a second tensor-memory
-//      buffer, which the threads fold into fp32 register accumulators with
-//      the rescale factor.
-// The FP8 cache is widened to bf16 while it is staged (exact: every E4M3
-// value is a bf16 value; both MMA operands are bf16). With one scale per KV
-// head, k_scale folds into the softmax scale and v_scale into the final
-// normalisation; with one scale per token, the tile's 64 K and 64 V scales
-// are staged next to it and multiply S column by column and P column by
-// column (in fp32, before P is rounded to bf16; l then sums the unscaled
-// weights).
+//   2. one thread issues S = Q K^T (M 128, N 64, K head_dim) into tensor
+//      memory, queued right behind P V of the previous tile;
+//   3. two threads per row read half of the row's tensor-memory columns each,
+//      apply the causal mask, combine the row maximum through shared memory
+//      and write P = exp2(s - m) as bf16 over the K tile S has consumed (or
+//      into a buffer of its own for head_dim 64);
+//   4. one thread issues O += P V (M 128, N head_dim, K 64; V read MN-major
+//      straight from its row layout) into a second tensor-memory buffer. The
+//      reference maximum moves only when a tile's maximum exceeds it by more
+//      than 8 (log2 domain); then the row's O is rescaled in tensor memory.
 //
 // Shared-memory operand layout (all four operands): [head_dim / 64 or
 // 128 / 64 column blocks][rows][128 bytes], the 16-byte chunk c of row r

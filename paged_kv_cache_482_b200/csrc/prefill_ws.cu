@@ -1,5 +1,6 @@
-// prefill_ws.cu -- chunked-prefill paged attention, bf16 cache, warp-
-// specialised on the 5th-generation tensor cores (sm_100a).
+// prefill_ws.cu -- chunked-prefill paged attention (bf16 cache, or E4M3 with
+// one scale per KV head), warp-specialised on the 5th-generation tensor cores
+// (sm_100a).
 //
 // Same operation as prefill.cu ("nano-vllm-lite：深入理解LLM推理机制的教育级开源
 // 项目", section 核心技术改进 2 "Chunked Prefill"; paged cache of "DeepSeek复刻
@@ -10,9 +11,11 @@
 // a (chunk token, query head of the group) pair), one CTA per SM. Warp roles:
 //   warps 0-3  softmax of query tile A (one row per thread);
 //   warps 4-7  softmax of query tile B;
-//   warp 8     producer: tensor-map copies of 128-token K/V tiles into a
-//              two-stage ring (and the zeroing of V rows past the causal
-//              end on the last tile);
+//   warp 8     bf16: producer, tensor-map copies of 128-token K/V tiles into
+//              a two-stage ring (and the zeroing of V rows past the causal
+//              end on the last tile). E4M3: one of three converter warps
+//              (8, 10, 11) that load the codes, widen them to f16 and store
+//              them into the ring;
 //   warp 9     tensor-memory allocation and the MMA issue:
 //                S_A(0), S_B(0), then per tile j
 //                PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ...
@@ -22,22 +25,25 @@
 // reads half as much shared memory for the Q operand as N = 64 does, which
 // is what paced the tensor pipe with 64-token tiles.
 // Tensor memory (512 columns): S_A, S_B (128 columns each) and O_A, O_B
-// (128 columns each). P (bf16, two per 32-bit column) is written over the
-// first 64 columns of the S it came from and P V takes its A operand from
+// (128 columns each). P (two 16-bit values per 32-bit column) is written over
+// the first 64 columns of the S it came from and P V takes its A operand from
 // tensor memory, so P never touches shared memory. S of tile j + 1 reuses
 // the columns of P of tile j: it is issued after P V of tile j by the same
 // thread, and MMAs from one thread run in issue order. The commit of S(j+1)
 // therefore also covers P V(j): a softmax thread that sees S(j+1) may
 // rescale O without waiting for anything else.
-// The softmax makes two passes over S in tensor memory (row maximum, then
-// exponentials), 64 columns at a time, to keep its registers below the
-// budget of one 320-thread CTA per SM.
+// A softmax thread takes its row's 128 scores from tensor memory in one
+// statement (two loads and their wait), and rescales O only after P is out of
+// its registers (168 registers a thread: 320 or 384 threads, one CTA per SM).
+// Operand types: bf16 for a bf16 cache. For E4M3, f16: every E4M3 value is
+// an f16 value (one conversion per two codes), Q is scaled per row by a power
+// of two into f16 range (exact for bf16 input), and P is packed as f16.
 // Everything between roles goes through mbarriers (full / empty K/V stages,
 // S ready, P ready, O done); every wait is bounded (1 s) and reports
 // PKV_DEVERR_TIMEOUT. The softmax uses the same arithmetic as prefill.cu:
 // exp2 domain, lazy rescale of O in tensor memory (the reference maximum
 // moves only when a tile's maximum exceeds it by more than 8), P rounded to
-// bf16 and the normaliser summing the rounded weights.
+// the operand type and the normaliser summing the rounded weights.
 #include "tc_common.cuh"
 
 namespace pkv {
