@@ -561,7 +561,9 @@ def prefill_dtype(wl):
     if not wl.is_fp8:
         return "bf16 x bf16 -> fp32 (tcgen05)"
     if wl.token_scales:
-        return "e4m3 cache (per-token scales) widened to bf16; bf16 x bf16 -> fp32 (tcgen05)"
+        return ("e4m3 cache with per-token scales: S in f16 x f16 (K widened to f16, Q scaled per row), "
+                "P V in bf16 x bf16 (V widened to bf16, P times the V scales) -> fp32 (tcgen05); "
+                "chunks of one query tile or less: bf16 operands")
     return ("e4m3 cache widened to f16, Q scaled per row into f16; f16 x f16 -> fp32 (tcgen05); "
             "chunks of one query tile or less: bf16 operands")
 

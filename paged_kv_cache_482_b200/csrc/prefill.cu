@@ -540,18 +540,17 @@ bool prefill_supported(int head_dim, int group) {
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
-    if (a.fp8 && a.token_scales)  // E4M3 with one scale per token: the one-tile kernel
-        return a.head_dim == 128 ? launch_d<128, true, true>(a, g, stream) : launch_d<64, true, true>(a, g, stream);
-    // bf16, or E4M3 with one scale per KV head. Chunks of more than one query
-    // tile (128 / G tokens) go to the warp-specialised kernel (two tiles per
-    // CTA, one CTA per SM); shorter ones -- decode requests among them -- to
-    // the one-tile kernel, which fits two CTAs per SM. Each kernel skips the
-    // other's sequences.
+    // Chunks of more than one query tile (128 / G tokens) go to the
+    // warp-specialised kernel (two tiles per CTA, one CTA per SM); shorter
+    // ones -- decode requests among them -- to the one-tile kernel, which fits
+    // two CTAs per SM. Each kernel skips the other's sequences.
     PrefillArgs small = a;
     small.small_cut = kRows / g;
     small.max_q_len = a.max_q_len < small.small_cut ? a.max_q_len : small.small_cut;
     cudaError_t e;
-    if (a.head_dim == 128)
+    if (a.fp8 && a.token_scales)
+        e = a.head_dim == 128 ? launch_d<128, true, true>(small, g, stream) : launch_d<64, true, true>(small, g, stream);
+    else if (a.head_dim == 128)
         e = a.fp8 ? launch_d<128, true>(small, g, stream) : launch_d<128, false>(small, g, stream);
     else
         e = a.fp8 ? launch_d<64, true>(small, g, stream) : launch_d<64, false>(small, g, stream);

@@ -73,7 +73,8 @@ struct WsLayout {
     static constexpr uint32_t kRing = kQ + 2 * kQTile;          // stage s: K at kRing + s * 2 kKV, V after it
     static constexpr uint32_t kBar = kRing + kStages * 2 * kKV;
     static constexpr uint32_t kTable = kBar + 256;
-    static constexpr uint32_t kBytes = kTable + kTableCap * 4;
+    static constexpr uint32_t kScales = kTable + kTableCap * 4;  // per-token E4M3: [stage][K, V][kBN] fp32
+    static constexpr uint32_t kBytes = kScales + kStages * 2 * kBN * 4;
     static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 
@@ -119,16 +120,19 @@ __device__ __forceinline__ void ws_kv_tile(const CUtensorMap *mk, const CUtensor
     }
 }
 
-template <int D, int G, bool FP8>
+template <int D, int G, bool FP8, bool TS>
 __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
     paged_prefill_ws_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
                             const __grid_constant__ CUtensorMap map_v) {
     using L = WsLayout<D>;
     constexpr int TQ = kRowsT / G;  // chunk tokens per query tile
-    // bf16 cache: bf16 operands. E4M3 cache: f16 operands (one conversion per
-    // two codes; Q is scaled into f16 range per row, see the staging below).
+    // bf16 cache: bf16 operands. E4M3 cache: f16 operands for S (one conversion
+    // per two codes; Q is scaled into f16 range per row, see the staging below)
+    // and for P V with one scale per KV head. With one scale per token, P is
+    // multiplied by the V scales before it is rounded, which may leave f16
+    // range: P V then runs in bf16 (P and V both bf16).
     constexpr uint32_t kIdescS = FP8 ? idesc_f16(kRowsT, kBN, false) : idesc_bf16(kRowsT, kBN, false);
-    constexpr uint32_t kIdescPV = FP8 ? idesc_f16(kRowsT, D, true) : idesc_bf16(kRowsT, D, true);
+    constexpr uint32_t kIdescPV = (FP8 && !TS) ? idesc_f16(kRowsT, D, true) : idesc_bf16(kRowsT, D, true);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -222,7 +226,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
         const uint32_t tmem_s = tmem + X * kBN;  // S (and P over its first 64 columns)
         const uint32_t tmem_o = tmem + 256 + X * 128;
         // E4M3 with one scale per KV head: k_scale folds into the softmax scale
-        float sl2 = a.scale * kLog2e * (FP8 ? __ldg(a.k_scale + kh) : 1.0f);
+        float sl2 = a.scale * kLog2e * ((FP8 && !TS) ? __ldg(a.k_scale + kh) : 1.0f);
         {
             constexpr int kChunks = D / 8;
             const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q);
@@ -290,6 +294,26 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
             // the row's 128 scores (one statement: two loads and their wait)
             float x[kBN];
             tmem_ld128(tmem_s + lane_base, x);
+            const float *tsc = reinterpret_cast<const float *>(sm + L::kScales) + (j % kStages) * 2 * kBN;
+            if constexpr (TS) {
+                // the converters staged this tile's per-token scales with its codes:
+                // x = s * (sl2 * k_scale of the column). The stage is refilled only
+                // after both query tiles have released this tile, so this wait
+                // cannot see a later phase.
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[j % kStages],
+                                                       static_cast<uint32_t>((j / kStages) & 1)))) {
+                    ok = false;
+                    break;
+                }
+                const float2 sl2x2 = make_float2(sl2, sl2);
+#pragma unroll
+                for (int i = 0; i < kBN / 2; ++i) {
+                    const float2 k2 = *reinterpret_cast<const float2 *>(tsc + 2 * i);
+                    const float2 v2 = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), __fmul2_rn(sl2x2, k2));
+                    x[2 * i] = v2.x;
+                    x[2 * i + 1] = v2.y;
+                }
+            }
             if (masked) {
 #pragma unroll
                 for (int i = 0; i < kBN; ++i)
@@ -300,8 +324,8 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
             for (int k = 0; k < 8; ++k) m8[k] = x[k];
 #pragma unroll
             for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-            const float mx = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            const float mx = (TS ? 1.0f : sl2) * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             float alpha = 1.0f;
             bool rescale = false;
             if (j == 0) {
@@ -317,7 +341,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
             }
             // P as bf16 pairs over columns 0..63 of S: scores 64 hh .. 64 hh + 63
             // go to columns 32 hh .. 32 hh + 31 (all scores are in registers)
-            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
+            const float2 sl2x2 = make_float2(TS ? 1.0f : sl2, TS ? 1.0f : sl2), nm2 = make_float2(-m_run, -m_run);
             float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -326,7 +350,12 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                 for (int i = 0; i < 32; ++i) {
                     const float2 t = __ffma2_rn(make_float2(x[hh * 64 + 2 * i], x[hh * 64 + 2 * i + 1]), sl2x2, nm2);
                     uint32_t w;
-                    if constexpr (FP8) {  // P in f16 (the E4M3 path's operand type)
+                    if constexpr (TS) {  // P times the V scales of its columns, in bf16; l sums the unscaled weights
+                        const float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
+                        const float2 v2 = *reinterpret_cast<const float2 *>(tsc + kBN + hh * 64 + 2 * i);
+                        w = pack_bf16(p0 * v2.x, p1 * v2.y);
+                        l4[i & 3] += p0 + p1;
+                    } else if constexpr (FP8) {  // P in f16 (the E4M3 path's operand type)
                         w = pack_f16(fast_exp2(t.x), fast_exp2(t.y));
                         l4[i & 3] = fma_f16x2_acc(w, 0x3C003C00u, l4[i & 3]);
                     } else {
@@ -357,7 +386,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
         }
         if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], 0))) {
             tc_fence_after();
-            const float inv = (FP8 ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
+            const float inv = ((FP8 && !TS) ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 float v[32];
@@ -443,24 +472,53 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                 }
             }
         };
-        auto store = [&](const uint4 (&w)[kPer], uint32_t dst) {
+        auto store = [&](const uint4 (&w)[kPer], uint32_t dst, bool to_bf16) {
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int idx = ct + u * kCW;
                 if (idx < kHalf) {
                     const int r = idx / kCPR, c16 = 2 * (idx % kCPR);
-                    const uint2 h0 = e4m3x4_to_f16x4(w[u].x), h1 = e4m3x4_to_f16x4(w[u].y);
-                    const uint2 h2 = e4m3x4_to_f16x4(w[u].z), h3 = e4m3x4_to_f16x4(w[u].w);
-                    st_shared16(dst + swz(kBN, r, c16), make_uint4(h0.x, h0.y, h1.x, h1.y));
-                    st_shared16(dst + swz(kBN, r, c16 + 1), make_uint4(h2.x, h2.y, h3.x, h3.y));
+                    if (to_bf16) {
+                        st_shared16(dst + swz(kBN, r, c16), e4m3x8_to_bf16x8(make_uint2(w[u].x, w[u].y)));
+                        st_shared16(dst + swz(kBN, r, c16 + 1), e4m3x8_to_bf16x8(make_uint2(w[u].z, w[u].w)));
+                    } else {
+                        const uint2 h0 = e4m3x4_to_f16x4(w[u].x), h1 = e4m3x4_to_f16x4(w[u].y);
+                        const uint2 h2 = e4m3x4_to_f16x4(w[u].z), h3 = e4m3x4_to_f16x4(w[u].w);
+                        st_shared16(dst + swz(kBN, r, c16), make_uint4(h0.x, h0.y, h1.x, h1.y));
+                        st_shared16(dst + swz(kBN, r, c16 + 1), make_uint4(h2.x, h2.y, h3.x, h3.y));
+                    }
                 }
             }
             fence_proxy_async_smem();  // the tensor core reads these through the async proxy
             __syncwarp();
         };
+        // per-token scales of a tile (TS): K at [0, kBN), V at [kBN, 2 kBN), 0 past the end
+        constexpr int kSPer = (2 * kBN + kCW - 1) / kCW;
+        float sc[kSPer];
+        auto load_scales = [&](int j) {
+#pragma unroll
+            for (int u = 0; u < kSPer; ++u) {
+                const int i = ct + u * kCW;
+                const int t = j * kBN + (i % kBN);
+                sc[u] = 0.0f;
+                if (TS && i < 2 * kBN && t < kv_end)
+                    sc[u] = __ldg((i < kBN ? a.k_scale : a.v_scale) +
+                                  (static_cast<int64_t>(table[t >> log2_bs]) * a.num_kv_heads + kh) * a.block_size +
+                                  (t & (a.block_size - 1)));
+            }
+        };
+        auto store_scales = [&](int j) {
+            float *dst = reinterpret_cast<float *>(sm + L::kScales) + (j % kStages) * 2 * kBN;
+#pragma unroll
+            for (int u = 0; u < kSPer; ++u) {
+                const int i = ct + u * kCW;
+                if (i < 2 * kBN) dst[i] = sc[u];
+            }
+        };
         bool ok = true;
         load(wk, a.k_cache, 0);
         load(wv, a.v_cache, 0);
+        if (TS) load_scales(0);
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages, use = j / kStages;
             if (use > 0 &&
@@ -469,11 +527,16 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                 break;
             }
             // K of tile j, then the next tile's K codes load while V is widened
-            store(wk, kbuf(j));
+            // (to bf16 with per-token scales, where P V runs in bf16)
+            if (TS) store_scales(j);
+            store(wk, kbuf(j), false);
             if (j + 1 < n_tiles) load(wk, a.k_cache, j + 1);
-            store(wv, vbuf(j));
+            store(wv, vbuf(j), TS);
             if (lane == 0) mbar_arrive(&bars->kv_full[st]);
-            if (j + 1 < n_tiles) load(wv, a.v_cache, j + 1);
+            if (j + 1 < n_tiles) {
+                load(wv, a.v_cache, j + 1);
+                if (TS) load_scales(j + 1);
+            }
         }
         if (!ok && lane == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
         __syncwarp();
@@ -549,7 +612,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
     }
 }
 
-template <int D, int G, bool FP8>
+template <int D, int G, bool FP8, bool TS>
 cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int TQ = kRowsT / G;
     const int tiles = (a.max_q_len + 2 * TQ - 1) / (2 * TQ);
@@ -565,7 +628,7 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     // the E4M3 path loads the codes with plain loads: no tensor maps
     if (!FP8 && (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)))
         return cudaErrorInvalidValue;
-    auto kern = paged_prefill_ws_kernel<D, G, FP8>;
+    auto kern = paged_prefill_ws_kernel<D, G, FP8, TS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(WsLayout<D>::kAlloc));
     if (e != cudaSuccess) return e;
@@ -574,13 +637,13 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool TS>
 cudaError_t launch_ws_g(const PrefillArgs &a, int g, cudaStream_t stream) {
     switch (g) {
-        case 1: return launch_ws<D, 1, FP8>(a, stream);
-        case 2: return launch_ws<D, 2, FP8>(a, stream);
-        case 4: return launch_ws<D, 4, FP8>(a, stream);
-        case 8: return launch_ws<D, 8, FP8>(a, stream);
+        case 1: return launch_ws<D, 1, FP8, TS>(a, stream);
+        case 2: return launch_ws<D, 2, FP8, TS>(a, stream);
+        case 4: return launch_ws<D, 4, FP8, TS>(a, stream);
+        case 8: return launch_ws<D, 8, FP8, TS>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -589,9 +652,14 @@ cudaError_t launch_ws_g(const PrefillArgs &a, int g, cudaStream_t stream) {
 
 cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
-    if (a.token_scales) return cudaErrorInvalidValue;  // per-token scales: the one-tile kernel
-    if (a.head_dim == 128) return a.fp8 ? launch_ws_g<128, true>(a, g, stream) : launch_ws_g<128, false>(a, g, stream);
-    if (a.head_dim == 64) return a.fp8 ? launch_ws_g<64, true>(a, g, stream) : launch_ws_g<64, false>(a, g, stream);
+    if (a.head_dim == 128) {
+        if (!a.fp8) return launch_ws_g<128, false, false>(a, g, stream);
+        return a.token_scales ? launch_ws_g<128, true, true>(a, g, stream) : launch_ws_g<128, true, false>(a, g, stream);
+    }
+    if (a.head_dim == 64) {
+        if (!a.fp8) return launch_ws_g<64, false, false>(a, g, stream);
+        return a.token_scales ? launch_ws_g<64, true, true>(a, g, stream) : launch_ws_g<64, true, false>(a, g, stream);
+    }
     return cudaErrorInvalidValue;
 }
 

@@ -152,6 +152,10 @@ PREFILL = [
     W.PrefillConfig("ptok_mixed", 2, 32, 8, 128, 256, 0, 600, 60, 200, cache_dtype=W.CACHE_FP8_TOKEN, decode_seqs=4,
                     decode_hist_lo=1, decode_hist_hi=700),
     W.PrefillConfig("ptok_bs8", 2, 8, 2, 128, 8, 10, 150, 20, 90, cache_dtype=W.CACHE_FP8_TOKEN),
+    # chunks longer than one query tile take the warp-specialised kernel's
+    # per-token path: G 1 and 2, block sizes 1024 and 32
+    W.PrefillConfig("ptok_g1_bs1024", 2, 4, 4, 128, 1024, 0, 1500, 130, 400, cache_dtype=W.CACHE_FP8_TOKEN),
+    W.PrefillConfig("ptok_g2_d64_bs32", 2, 8, 4, 64, 32, 100, 600, 70, 300, cache_dtype=W.CACHE_FP8_TOKEN),
 ]
 
 
