@@ -74,7 +74,7 @@ struct PrefillArgs {
     void *out;
     int *dev_err;
     // routing between the one-tile and warp-specialised kernels (set by
-    // launch_prefill for bf16 and per-head E4M3 caches): 0 = none;
+    // launch_prefill): 0 = none;
     // > 0: the one-tile kernel takes the sequences with chunks of at most
     // small_cut tokens, the warp-specialised kernel the others
     int small_cut;
@@ -95,6 +95,6 @@ cudaError_t launch_fused_add_rmsnorm(const NormArgs &a, int num_sms, cudaStream_
 
 bool prefill_supported(int head_dim, int group);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream);
-cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream);  // warp-specialised: bf16, per-head E4M3
+cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream);  // warp-specialised, every cache type
 
 }  // namespace pkv

@@ -13,11 +13,10 @@
 // Work unit: one CTA per (sequence, KV head, 128 query rows), 256 threads and
 // two CTAs per SM. A row is a (chunk token, query head of the group) pair:
 // row r = token r / G, head r % G, so the G heads that share a KV head share
-// every K/V tile. For bf16 and per-head E4M3 caches this kernel takes the
-// chunks of at most one query tile (128 / G tokens, decode requests among
-// them) and prefill_ws.cu the longer ones; per-token E4M3 caches take this
-// kernel for every chunk. The CTA walks the sequence's KV in 64-token tiles up
-// to its last row's position:
+// every K/V tile. This kernel takes the chunks of at most one query tile
+// (128 / G tokens, decode requests among them) and prefill_ws.cu the longer
+// ones, for every cache type. The CTA walks the sequence's KV in 64-token
+// tiles up to its last row's position:
 //   1. K/V tiles are gathered through the block table into shared memory,
 //      double buffered, in the 128-byte-swizzled layout the tensor core
 //      reads: for a bf16 cache one thread issues tensor-map (TMA) copies of

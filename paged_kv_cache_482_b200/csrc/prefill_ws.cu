@@ -1,6 +1,6 @@
-// prefill_ws.cu -- chunked-prefill paged attention (bf16 cache, or E4M3 with
-// one scale per KV head), warp-specialised on the 5th-generation tensor cores
-// (sm_100a).
+// prefill_ws.cu -- chunked-prefill paged attention (bf16 or E4M3 cache, one
+// scale per KV head or per token), warp-specialised on the 5th-generation
+// tensor cores (sm_100a).
 //
 // Same operation as prefill.cu ("nano-vllm-lite：深入理解LLM推理机制的教育级开源
 // 项目", section 核心技术改进 2 "Chunked Prefill"; paged cache of "DeepSeek复刻
@@ -37,7 +37,11 @@
 // its registers (168 registers a thread: 320 or 384 threads, one CTA per SM).
 // Operand types: bf16 for a bf16 cache. For E4M3, f16: every E4M3 value is
 // an f16 value (one conversion per two codes), Q is scaled per row by a power
-// of two into f16 range (exact for bf16 input), and P is packed as f16.
+// of two into f16 range (exact for bf16 input), and P is packed as f16. With
+// per-token scales, the converters also stage the tile's K and V scales;
+// scores are scaled by column, P is multiplied by the V scales before it is
+// rounded, and P V runs in bf16 (V widened to bf16), since P times a V scale
+// may leave f16 range.
 // Everything between roles goes through mbarriers (full / empty K/V stages,
 // S ready, P ready, O done); every wait is bounded (1 s) and reports
 // PKV_DEVERR_TIMEOUT. The softmax uses the same arithmetic as prefill.cu:
