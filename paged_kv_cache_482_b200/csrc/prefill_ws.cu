@@ -83,8 +83,8 @@ struct WsLayout {
 };
 
 struct Bars {
-    uint64_t kv_full[kStages];
-    uint64_t kv_empty[kStages];
+    uint64_t kv_full[kStages];   // stage written (MMA warp; softmax too, for per-token scales)
+    uint64_t kv_empty[kStages];  // P V_B of the stage's tile done: the stage may be refilled
     uint64_t s_full[2];     // [query tile]
     uint64_t p_full[2];     // [query tile]: P of a tile written
     uint64_t o_done[2];     // [query tile]: P V of a tile done
@@ -343,8 +343,9 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                     l_run *= alpha;
                 }
             }
-            // P as bf16 pairs over columns 0..63 of S: scores 64 hh .. 64 hh + 63
-            // go to columns 32 hh .. 32 hh + 31 (all scores are in registers)
+            // P as 16-bit pairs (bf16, or f16 for E4M3 with per-head scales) over
+            // columns 0..63 of S: scores 64 hh .. 64 hh + 63 go to columns
+            // 32 hh .. 32 hh + 31 (all scores are in registers)
             const float2 sl2x2 = make_float2(TS ? 1.0f : sl2, TS ? 1.0f : sl2), nm2 = make_float2(-m_run, -m_run);
             float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
