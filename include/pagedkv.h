@@ -223,10 +223,16 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  *   out[row][h][:] = sum_{t <= p} softmax_t(scale * q[row][h] . K_t) V_t
  * (KV head h / group). A chunk of one token is a decode step, so one call
  * can serve a batch mixing prefill chunks and decode requests; c_i = 0 is
- * allowed (no rows). QK^T and PV run on the tensor cores with bf16 operands
- * and fp32 accumulation (the E4M3 cache is widened to bf16 exactly); the
- * softmax weights are rounded to bf16 for PV and the normaliser sums those
- * rounded weights; out is rounded to bf16.
+ * allowed (no rows). QK^T and PV run on the tensor cores with fp32
+ * accumulation. Operands: bf16 for a bf16 cache. For an E4M3 cache the codes
+ * are widened exactly: chunks of more than 128 / group tokens use f16 for QK^T
+ * (q scaled per row by a power of two into f16 range, exact for bf16 q) and,
+ * with one scale per KV head, f16 for PV too; with per-token scales PV runs in
+ * bf16; shorter chunks use bf16. The softmax weights are rounded to the PV
+ * operand type and the normaliser sums those rounded weights, except with
+ * per-token scales, where a weight is multiplied by its token's V scale
+ * before rounding and the normaliser sums the unscaled weights. out is
+ * rounded to bf16.
  *
  *  q             [total_q][num_q_heads][head_dim] bf16, contiguous
  *  block_tables  [num_seqs][max_blocks_per_seq] int32
