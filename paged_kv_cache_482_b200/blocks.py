@@ -56,7 +56,15 @@ def _i64(a):
 
 
 def _p(a):
-    return ctypes.c_void_p(a.ctypes.data) if a.size else None
+    """Address of a contiguous array's data (None when empty). A ctypes view of
+    the buffer is the cheapest route for a writable array (a third of the cost
+    of ``a.ctypes.data``, which read-only arrays still take)."""
+    if not a.size:
+        return None
+    try:
+        return ctypes.addressof(ctypes.c_char.from_buffer(a))
+    except (TypeError, ValueError):
+        return a.ctypes.data
 
 
 class BlockManager:

@@ -21,7 +21,6 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
-#include <unordered_map>
 #include <vector>
 
 #include "pagedkv_blocks.h"
@@ -61,8 +60,96 @@ Key chain_key(const Key &parent, const int32_t *tok, int n) {
 struct Seq {
     std::vector<int32_t> table;
     int64_t num_tokens = 0;
+    int32_t off = 0;        // num_tokens % block_size, kept so that appends divide nothing
     Key last_full = kRoot;  // key of the last full block (the next block's parent)
     uint32_t stamp = 0;     // repeated-id check in batch calls
+};
+
+// Live sequences by id: open addressing with linear probing and
+// backward-shift deletion over a power-of-two table, the records in a slab
+// whose slots are reused. A decode step looks every sequence up twice
+// (append, then the table row), so the lookup is a multiply, a mask and
+// usually one compare. Pointers into the slab stay valid until the next
+// insert.
+class SeqTable {
+  public:
+    Seq *find(int64_t id) {
+        if (count_ == 0) return nullptr;
+        for (uint64_t i = home(id);; i = (i + 1) & mask_) {
+            if (val_[i] < 0) return nullptr;
+            if (key_[i] == id) return &slab_[val_[i]];
+        }
+    }
+    const Seq *find(int64_t id) const { return const_cast<SeqTable *>(this)->find(id); }
+
+    // id must be absent. Throws std::bad_alloc before any change.
+    Seq *insert(int64_t id) {
+        if ((count_ + 1) * 2 > val_.size()) grow();
+        int32_t slot;
+        if (!free_.empty()) {
+            slot = free_.back();
+            free_.pop_back();
+        } else {
+            free_.reserve(slab_.size() + 1);  // so that erase never allocates
+            slab_.emplace_back();
+            slot = static_cast<int32_t>(slab_.size() - 1);
+        }
+        uint64_t i = home(id);
+        while (val_[i] >= 0) i = (i + 1) & mask_;
+        key_[i] = id;
+        val_[i] = slot;
+        ++count_;
+        return &slab_[slot];
+    }
+
+    // id must be present.
+    void erase(int64_t id) {
+        uint64_t i = home(id);
+        while (key_[i] != id || val_[i] < 0) i = (i + 1) & mask_;
+        slab_[val_[i]] = Seq{};
+        free_.push_back(val_[i]);
+        val_[i] = -1;
+        --count_;
+        // pull later entries of the probe run back over the hole when their
+        // home is at or before it
+        for (uint64_t j = (i + 1) & mask_; val_[j] >= 0; j = (j + 1) & mask_) {
+            if (((j - home(key_[j])) & mask_) >= ((j - i) & mask_)) {
+                key_[i] = key_[j];
+                val_[i] = val_[j];
+                val_[j] = -1;
+                i = j;
+            }
+        }
+    }
+
+  private:
+    uint64_t home(int64_t id) const {
+        const uint64_t h = static_cast<uint64_t>(id) * 0x9E3779B97F4A7C15ull;
+        return (h ^ (h >> 29)) & mask_;
+    }
+    void grow() {
+        const size_t cap = val_.empty() ? 64 : 2 * val_.size();
+        std::vector<int64_t> key(cap);
+        std::vector<int32_t> val(cap, -1);
+        const uint64_t mask = cap - 1;
+        std::swap(key, key_);
+        std::swap(val, val_);
+        mask_ = mask;
+        for (size_t i = 0; i < val.size(); ++i) {
+            if (val[i] < 0) continue;
+            uint64_t k = home(key[i]);
+            while (val_[k] >= 0) k = (k + 1) & mask_;
+            key_[k] = key[i];
+            val_[k] = val[i];
+        }
+    }
+
+    std::vector<int64_t> key_;
+    std::vector<int32_t> val_;  // slab slot, -1 empty
+    uint64_t mask_ = 0;
+    size_t count_ = 0;
+    std::vector<Seq> slab_;
+    std::vector<int32_t> free_;
 };
 
 }  // namespace
@@ -84,7 +171,8 @@ struct pkv_block_manager {
     std::vector<int32_t> slot_of;  // block -> index in `table` (for deletion)
     std::vector<int32_t> table;    // open addressing: block id or -1
     uint64_t mask;
-    std::unordered_map<int64_t, Seq> seqs;
+    SeqTable seqs;
+    std::vector<Seq *> step;  // scratch of the batch calls
     uint32_t stamp = 0;
 
     pkv_block_manager(int64_t n, int b) : nb(n), bs(b) {
@@ -200,21 +288,23 @@ struct pkv_block_manager {
 
     // Appends one token to s (a free block must exist when one is needed).
     int32_t append(Seq &s, int32_t tok) {
-        const int64_t n = s.num_tokens;
-        if (n % bs == 0) {
+        const int off = s.off;
+        if (off == 0) {  // the sequence's blocks are all full: open one
             const int32_t b = take_free();
             ref[b] = 1;
             s.table.push_back(b);
         }
-        const int32_t b = s.table[n / bs];
-        const int off = static_cast<int>(n % bs);
+        const int32_t b = s.table.back();  // the block holding position num_tokens
         tokens[static_cast<size_t>(b) * bs + off] = tok;
         fill[b] = off + 1;
-        s.num_tokens = n + 1;
+        s.num_tokens += 1;
         if (off + 1 == bs) {
             const Key k = chain_key(s.last_full, &tokens[static_cast<size_t>(b) * bs], bs);
             insert(b, k, s.last_full);
             s.last_full = k;
+            s.off = 0;
+        } else {
+            s.off = off + 1;
         }
         return static_cast<int32_t>(static_cast<int64_t>(b) * bs + off);
     }
@@ -237,7 +327,7 @@ void pkv_bm_destroy(pkv_block_manager *bm) { delete bm; }
 int pkv_bm_add_sequence(pkv_block_manager *bm, int64_t seq_id, const int32_t *tokens, int num_tokens,
                         int *num_cached_tokens) {
     if (!bm || !tokens || !num_cached_tokens || num_tokens < 1) return PKV_ERR_INVALID_ARG;
-    if (bm->seqs.count(seq_id)) return PKV_ERR_INVALID_ARG;
+    if (bm->seqs.find(seq_id)) return PKV_ERR_INVALID_ARG;
     const int bs = bm->bs;
     const int64_t n_blocks = (static_cast<int64_t>(num_tokens) + bs - 1) / bs;
     if (n_blocks > bm->nb) return PKV_ERR_WORKSPACE;
@@ -260,9 +350,9 @@ int pkv_bm_add_sequence(pkv_block_manager *bm, int64_t seq_id, const int32_t *to
     if (bm->nfree - free_hits < need) return PKV_ERR_WORKSPACE;
     try {
         Seq s;
-        s.table.reserve(n_blocks + 1);
-        auto ins = bm->seqs.emplace(seq_id, std::move(s));
-        Seq &q = ins.first->second;
+        s.table.reserve(n_blocks + 1);  // appends below stay within it: nothing throws after the insert
+        Seq &q = *bm->seqs.insert(seq_id);
+        q = std::move(s);
         for (int32_t b : hits) {
             if (bm->ref[b] == 0) bm->q_remove(b);
             ++bm->ref[b];
@@ -280,10 +370,10 @@ int pkv_bm_add_sequence(pkv_block_manager *bm, int64_t seq_id, const int32_t *to
 
 int pkv_bm_append_token(pkv_block_manager *bm, int64_t seq_id, int32_t token, int64_t *slot) {
     if (!bm || !slot) return PKV_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-    Seq &s = it->second;
-    if (s.num_tokens % bm->bs == 0 && bm->nfree == 0) return PKV_ERR_WORKSPACE;
+    Seq *sp = bm->seqs.find(seq_id);
+    if (!sp) return PKV_ERR_INVALID_ARG;
+    Seq &s = *sp;
+    if (s.off == 0 && bm->nfree == 0) return PKV_ERR_WORKSPACE;
     if (s.num_tokens >= INT32_MAX) return PKV_ERR_INVALID_ARG;
     *slot = bm->append(s, token);
     return PKV_OK;
@@ -291,19 +381,19 @@ int pkv_bm_append_token(pkv_block_manager *bm, int64_t seq_id, int32_t token, in
 
 int pkv_bm_free_sequence(pkv_block_manager *bm, int64_t seq_id) {
     if (!bm) return PKV_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-    bm->release(it->second);
-    bm->seqs.erase(it);
+    Seq *sp = bm->seqs.find(seq_id);
+    if (!sp) return PKV_ERR_INVALID_ARG;
+    bm->release(*sp);
+    bm->seqs.erase(seq_id);
     return PKV_OK;
 }
 
 int pkv_bm_block_table(const pkv_block_manager *bm, int64_t seq_id, int32_t *row, int max_blocks,
                        int *num_tokens) {
     if (!bm || !num_tokens || max_blocks < 0 || (max_blocks > 0 && !row)) return PKV_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-    const Seq &s = it->second;
+    const Seq *sp = bm->seqs.find(seq_id);
+    if (!sp) return PKV_ERR_INVALID_ARG;
+    const Seq &s = *sp;
     const int n = static_cast<int>(s.table.size());
     *num_tokens = static_cast<int>(s.num_tokens);
     if (n > max_blocks) return PKV_ERR_INVALID_ARG;
@@ -314,9 +404,9 @@ int pkv_bm_block_table(const pkv_block_manager *bm, int64_t seq_id, int32_t *row
 
 int pkv_bm_slots(const pkv_block_manager *bm, int64_t seq_id, int start, int count, int32_t *slots) {
     if (!bm || start < 0 || count < 0 || (count > 0 && !slots)) return PKV_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-    const Seq &s = it->second;
+    const Seq *sp = bm->seqs.find(seq_id);
+    if (!sp) return PKV_ERR_INVALID_ARG;
+    const Seq &s = *sp;
     if (static_cast<int64_t>(start) + count > s.num_tokens) return PKV_ERR_INVALID_ARG;
     const int bs = bm->bs;
     for (int i = 0; i < count; ++i) {
@@ -339,7 +429,7 @@ int pkv_bm_append_tokens(pkv_block_manager *bm, const int64_t *seq_ids, const in
     if (!bm || n < 0 || (n > 0 && (!seq_ids || !tokens || !slots))) return PKV_ERR_INVALID_ARG;
     if (n == 0) return PKV_OK;
     // pass 1: every id live and distinct; count the blocks the step needs
-    std::vector<Seq *> ss;
+    std::vector<Seq *> &ss = bm->step;
     try {
         ss.resize(n);
     } catch (const std::bad_alloc &) {
@@ -349,14 +439,14 @@ int pkv_bm_append_tokens(pkv_block_manager *bm, const int64_t *seq_ids, const in
     int64_t need = 0;
     int bad = 0;
     for (int i = 0; i < n; ++i) {
-        auto it = bm->seqs.find(seq_ids[i]);
-        if (it == bm->seqs.end() || it->second.stamp == st || it->second.num_tokens >= INT32_MAX) {
+        Seq *q = bm->seqs.find(seq_ids[i]);
+        if (!q || q->stamp == st || q->num_tokens >= INT32_MAX) {
             bad = 1;
             break;
         }
-        it->second.stamp = st;
-        ss[i] = &it->second;
-        need += it->second.num_tokens % bm->bs == 0;
+        q->stamp = st;
+        ss[i] = q;
+        need += q->off == 0;
     }
     if (bad) return PKV_ERR_INVALID_ARG;
     if (need > bm->nfree) return PKV_ERR_WORKSPACE;
@@ -370,9 +460,9 @@ int pkv_bm_block_tables(const pkv_block_manager *bm, const int64_t *seq_ids, int
     if (!bm || n < 0 || max_blocks < 0) return PKV_ERR_INVALID_ARG;
     if (n > 0 && (!seq_ids || !block_tables || !context_lens)) return PKV_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
-        auto it = bm->seqs.find(seq_ids[i]);
-        if (it == bm->seqs.end()) return PKV_ERR_INVALID_ARG;
-        const Seq &s = it->second;
+        const Seq *sp = bm->seqs.find(seq_ids[i]);
+        if (!sp) return PKV_ERR_INVALID_ARG;
+        const Seq &s = *sp;
         const int nb = static_cast<int>(s.table.size());
         if (nb > max_blocks) return PKV_ERR_INVALID_ARG;
         int32_t *row = block_tables + static_cast<size_t>(i) * max_blocks;
