@@ -102,10 +102,14 @@ class SeqTable {
         return &slab_[slot];
     }
 
-    // id must be present.
+    // Removes id (nothing happens when it is absent).
     void erase(int64_t id) {
+        if (count_ == 0) return;
         uint64_t i = home(id);
-        while (key_[i] != id || val_[i] < 0) i = (i + 1) & mask_;
+        for (;; i = (i + 1) & mask_) {
+            if (val_[i] < 0) return;
+            if (key_[i] == id) break;
+        }
         slab_[val_[i]] = Seq{};
         free_.push_back(val_[i]);
         val_[i] = -1;
