@@ -265,11 +265,11 @@ def oracle_sample_runner(wl: W.Workload, ids, threads: int):
         vs = O.new_scale_pool(nblk, c.num_kv_heads, c.block_size)
     O.store_kvcache(sub["k_hist"], sub["v_hist"], kp, vp, sub["slot_hist"], nblk, c.block_size, ks, vs)
 
-    def step():
+    def step(num_threads=threads):
         O.store_kvcache(sub["k_new"], sub["v_new"], kp, vp, sub["slot_new"], nblk, c.block_size, ks, vs)
         out, st = O.paged_attention_decode(sub["q"], kp, vp, sub["block_tables"], sub["context_lens"],
                                            c.num_kv_heads, c.block_size, c.softmax_scale, ks, vs,
-                                           num_threads=threads)
+                                           num_threads=num_threads)
         return st
 
     return step
@@ -316,9 +316,17 @@ def cpu_baseline(wl: W.Workload, target_s: float) -> dict:
     st = run()
     dt = time.perf_counter() - t0
     toks = int(wl.context_lens.cpu()[order[:n2]].sum())
+    # the same oracle on one thread, over the first n2 / threads sequences of the sample
+    n1 = max(1, n2 // threads)
+    run1 = run if n1 == n2 else (probe if n1 == n else oracle_sample_runner(wl, order[:n1], 1))
+    t0 = time.perf_counter()
+    run1(1)
+    dt1 = time.perf_counter() - t0
     return {"value": n2 / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{n2} of {S} sequences ({toks} context tokens) of the same step, fp64, {dt:.2f} s, "
-                      f"OpenMP over sequences; status {st}"}
+                      f"OpenMP over sequences; status {st}",
+            "single_thread": {"value": n1 / dt1, "unit": UNIT, "cores": 1,
+                              "sample": f"the first {n1} of those sequences, {dt1:.2f} s"}}
 
 
 # --------------------------------------------------------------- reference
