@@ -60,12 +60,24 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--out", default="", help="also append the JSON line to this file")
     ap.add_argument("--component", choices=["decode", "block_manager"], default="decode",
                     help="block_manager: time the host block manager's per-step bookkeeping instead")
     return ap.parse_args()
 
 
 # ------------------------------------------------------------------ helpers
+
+
+def emit(line: dict, args) -> None:
+    """Print the one JSON line (and append it to --out when given)."""
+    text = json.dumps(line)
+    print(text, flush=True)
+    if getattr(args, "out", ""):
+        d = os.path.dirname(os.path.abspath(args.out))
+        os.makedirs(d, exist_ok=True)
+        with open(args.out, "a") as f:
+            f.write(text + "\n")
 
 
 def workload_desc(cfg: W.DecodeConfig) -> str:
@@ -194,6 +206,73 @@ class ClockSampler:
                 "samples_note": "in the timed window" if inwin else "nearest samples (window shorter than 200 ms)"}
 
 
+class NvmlSampler:
+    """SM clock, power and clock-event reasons read through NVML every 5 ms
+    (reads only), so that even a window of a few milliseconds holds samples.
+    Same summary() as ClockSampler; make_sampler falls back to nvidia-smi."""
+
+    PERIOD_S = 0.005
+
+    def __init__(self, device_id):
+        import pynvml as N
+
+        self.N = N
+        N.nvmlInit()
+        if isinstance(device_id, str):
+            self.h = N.nvmlDeviceGetHandleByUUID(device_id)
+        else:
+            self.h = N.nvmlDeviceGetHandleByIndex(int(device_id))
+        self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM))
+        self.bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                     "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                     "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                     "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+        self.samples = []
+        self.running = True
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+
+    def _poll(self):
+        N = self.N
+        while self.running:
+            try:
+                sm = float(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                pw = N.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.time(), sm, pw, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.005)
+
+    def stop(self):
+        self.running = False
+        self.thread.join(timeout=1.0)
+
+    def summary(self, t0, t1):
+        inwin = [x for x in self.samples if t0 <= x[0] <= t1]
+        used = inwin or self.samples[-3:]
+        reasons = sorted({n for _, _, _, rs in used for n, b in self.bits.items() if rs & b})
+        sm = [x[1] for x in used]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "power_w_max": max(x[2] for x in used) if used else None, "reasons": reasons,
+                "samples": len(inwin), "sampler": "NVML every 5 ms",
+                "samples_note": "in the timed window" if inwin else "nearest samples (no sample in the window)"}
+
+
+def make_sampler(local_rank: int):
+    """NVML sampler for this rank's GPU, else the nvidia-smi one."""
+    ids = nvsmi_ids(local_rank)
+    try:
+        return NvmlSampler(ids[0])
+    except Exception:  # noqa: BLE001
+        return ClockSampler(ids)
+
+
 def nvsmi_ids(local_rank: int):
     try:
         props = torch.cuda.get_device_properties(local_rank)
@@ -320,13 +399,15 @@ def cpu_baseline(wl: W.Workload, target_s: float) -> dict:
     n1 = max(1, n2 // threads)
     run1 = run if n1 == n2 else (probe if n1 == n else oracle_sample_runner(wl, order[:n1], 1))
     t0 = time.perf_counter()
-    run1(1)
+    st1 = run1(1)
     dt1 = time.perf_counter() - t0
+    if st != 0 or st1 != 0:
+        raise RuntimeError(f"the oracle returned status {st} (all cores) / {st1} (one thread) on its sample")
     return {"value": n2 / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{n2} of {S} sequences ({toks} context tokens) of the same step, fp64, {dt:.2f} s, "
                       f"OpenMP over sequences; status {st}",
             "single_thread": {"value": n1 / dt1, "unit": UNIT, "cores": 1,
-                              "sample": f"the first {n1} of those sequences, {dt1:.2f} s"}}
+                              "sample": f"the first {n1} of those sequences, {dt1:.2f} s; status {st1}"}}
 
 
 # --------------------------------------------------------------- reference
@@ -373,7 +454,7 @@ def run_reference(args):
                          "sample": f"{n} of {S} sequences per step, fp64 oracle, OpenMP over sequences"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(line, args)
     return 0
 
 
@@ -462,7 +543,7 @@ def run_block_manager(args):
                                 "sample": f"{n_o} steps of the same {S} sequences; admission of all prompts "
                                           f"{n_prompt / o_admit:.0f} prompt tokens/s"}
     m.close()
-    print(json.dumps(line), flush=True)
+    emit(line, args)
 
 
 # ------------------------------------------------------------------ prefill
@@ -572,7 +653,7 @@ def run_prefill_reference(args):
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
     unit = "query tokens/s"
-    print(json.dumps({
+    emit({
         "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -580,7 +661,7 @@ def run_prefill_reference(args):
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": f"{n} of {wl.total_q} query tokens per step, each as a one-token chunk"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }), flush=True)
+    }, args)
     return 0
 
 
@@ -647,7 +728,7 @@ def run_prefill(args):
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item())} during warm-up")
 
-    sampler = ClockSampler(nvsmi_ids(local)) if local == 0 else None
+    sampler = make_sampler(local) if local == 0 else None
     if sampler:
         sampler.wait_first()
     Kst = args.steps
@@ -736,7 +817,7 @@ def run_prefill(args):
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = prefill_cpu_baseline(wl, args.cpu_seconds)
-        print(json.dumps(line), flush=True)
+        emit(line, args)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -795,7 +876,7 @@ def run_norm_reference(args):
         O.fused_add_rmsnorm(x, r, w, cfg.eps, num_threads=threads)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
-    print(json.dumps({
+    emit({
         "impl": "reference", "metric": NORM_METRIC, "value": value, "unit": "rows/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -803,7 +884,7 @@ def run_norm_reference(args):
         "cpu_baseline": {"value": value, "unit": "rows/s", "cores": threads, "kind": "oracle",
                          "sample": f"all {n} rows per step, fp64, OpenMP over rows"},
         "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }), flush=True)
+    }, args)
     return 0
 
 
@@ -835,7 +916,7 @@ def run_norm(args):
     # inputs larger than L2 (checked) or L2 flushed between steps
     moved = norm_bytes(cfg)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if moved < (256 << 20) else None
-    sampler = ClockSampler(nvsmi_ids(local)) if local == 0 else None
+    sampler = make_sampler(local) if local == 0 else None
     if sampler:
         sampler.wait_first()
     Kst = args.steps
@@ -911,7 +992,7 @@ def run_norm(args):
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = norm_cpu_baseline(wl, args.cpu_seconds)
-        print(json.dumps(line), flush=True)
+        emit(line, args)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -977,7 +1058,7 @@ def main():
     if int(step.dev_err.item()) != 0:
         raise RuntimeError(f"device error word {int(step.dev_err.item())} during warm-up")
 
-    sampler = ClockSampler(nvsmi_ids(local)) if local == 0 else None
+    sampler = make_sampler(local) if local == 0 else None
     if sampler:
         sampler.wait_first()
     Kst = args.steps
@@ -1073,7 +1154,7 @@ def main():
             line["logical_gbs"] = ab["total"] / (decode_ms * 1e-3) / 1e9
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
-        print(json.dumps(line), flush=True)
+        emit(line, args)
 
     if dist is not None:
         dist.barrier()

@@ -138,6 +138,23 @@ PKV_API int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int
                     int partition_request, pkv_decode_plan *plan);
 
 /*
+ * pkv_decode_workspace_bytes: device scratch that is always enough for
+ * pkv_paged_attention_decode with partition_request = 0 (automatic split-K)
+ * on num_seqs sequences of num_q_heads query heads of head_dim, with
+ * contexts of at most max_context_len tokens -- whatever the KV head count,
+ * block size and cache type. The problem statement gives only these four
+ * sizes ("DeepSeek复刻vLLM反超原版：AI推理新标杆", section "vLLM：大模型推理的加速
+ * 引擎与挑战": one query token per sequence against its block table), so the
+ * value is a bound over the plans the other arguments can select: an
+ * automatic plan never cuts partitions shorter than 1024 tokens, so it uses
+ * at most ceil(max_context_len / 1024) partitions of (head_dim + 2) floats per
+ * (sequence, query head). Returns 0 when no automatic plan can split
+ * (max_context_len <= 1024) and for sizes below 1. pkv_plan_decode gives the
+ * exact figure for one shape (and for explicit partition requests).
+ */
+PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len);
+
+/*
  * paged_attention_decode: for each sequence i < num_seqs and query head h,
  *   out[i][h][:] = sum_t softmax_t(scale * q[i][h] . K_t) V_t
  * over the context_lens[i] tokens t of sequence i, where the K/V row of
@@ -154,7 +171,10 @@ PKV_API int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int
  *                     scheduled (NULL: 0, 1, 2, ...). Longest first shortens
  *                     the tail of the grid; the result does not depend on
  *                     it. An entry outside [0, num_seqs) sets
- *                     PKV_DEVERR_BOUNDS and is skipped.
+ *                     PKV_DEVERR_BOUNDS and is skipped; the out rows of a
+ *                     sequence that no valid entry names are then left
+ *                     unwritten (the split-K merge follows the same
+ *                     order, so it never reads partials of another call).
  *  max_context_len    host-known bound on context_lens (sizes split-K)
  *  partition_request  as in pkv_plan_decode
  *  workspace          device scratch of at least plan.workspace_bytes,

@@ -62,7 +62,7 @@ struct Seq {
     int64_t num_tokens = 0;
     int32_t off = 0;        // num_tokens % block_size, kept so that appends divide nothing
     Key last_full = kRoot;  // key of the last full block (the next block's parent)
-    uint32_t stamp = 0;     // repeated-id check in batch calls
+    uint64_t stamp = 0;     // repeated-id check in batch calls (64 bits: never wraps)
 };
 
 // Live sequences by id: open addressing with linear probing and
@@ -177,7 +177,7 @@ struct pkv_block_manager {
     uint64_t mask;
     SeqTable seqs;
     std::vector<Seq *> step;  // scratch of the batch calls
-    uint32_t stamp = 0;
+    uint64_t stamp = 0;       // batch-call counter; records start at 0, calls at 1
 
     pkv_block_manager(int64_t n, int b) : nb(n), bs(b) {
         tokens.assign(static_cast<size_t>(n) * b, 0);
@@ -439,7 +439,7 @@ int pkv_bm_append_tokens(pkv_block_manager *bm, const int64_t *seq_ids, const in
     } catch (const std::bad_alloc &) {
         return PKV_ERR_WORKSPACE;
     }
-    const uint32_t st = ++bm->stamp;
+    const uint64_t st = ++bm->stamp;
     int64_t need = 0;
     int bad = 0;
     for (int i = 0; i < n; ++i) {

@@ -609,11 +609,16 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
 }
 
 // Merge the split-K partials of one (sequence, query head): weights
-// l_p * 2^(m_p - M) over the sequence's partitions, fixed order.
+// l_p * 2^(m_p - M) over the sequence's partitions, fixed order. The grid
+// visits sequences through seq_order like the decode grid, so it merges only
+// partials this call's decode blocks wrote; a sequence that no valid entry
+// names is left alone by both.
 template <int D>
 __global__ void __launch_bounds__(D) paged_decode_reduce_kernel(const DecodeParams p) {
     const int qh = blockIdx.x % p.num_q_heads;
-    const int seq = blockIdx.x / p.num_q_heads;
+    const int seq_slot = blockIdx.x / p.num_q_heads;
+    const int seq = p.seq_order ? __ldg(p.seq_order + seq_slot) : seq_slot;
+    if (seq < 0 || seq >= p.num_seqs) return;  // the decode grid reported it
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
     if (ctx < 1 || ctx > p.max_context_len || ctx > table_cap) return;  // decode wrote zeros

@@ -74,6 +74,9 @@ int make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int
             if (t < kMinAutoPartitionTokens) t = kMinAutoPartitionTokens;
             t = (long long)round_up((size_t)t, (size_t)tile);
             if (t > max_pt) t = max_pt;
+            // pkv_decode_workspace_bytes relies on automatic partitions never
+            // being shorter than kMinAutoPartitionTokens
+            if (t < kMinAutoPartitionTokens) return PKV_ERR_UNSUPPORTED;
             if (t < max_context_len) pt = t;
         }
     } else {
@@ -139,6 +142,17 @@ int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     if (!plan) return PKV_ERR_INVALID_ARG;
     return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, cache_dtype,
                      partition_request, plan);
+}
+
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len) {
+    if (num_seqs < 1 || num_q_heads < 1 || head_dim < 1 || max_context_len < 1) return 0;
+    // An automatic plan never cuts partitions shorter than
+    // kMinAutoPartitionTokens (and the longest partition cap is above it for
+    // every supported block size), so it has at most this many partitions.
+    const long long np = ((long long)max_context_len + kMinAutoPartitionTokens - 1) / kMinAutoPartitionTokens;
+    if (np <= 1) return 0;
+    const size_t rows = (size_t)num_seqs * num_q_heads * (size_t)np;
+    return round_up(rows * head_dim * sizeof(float), 256) + round_up(rows * 2 * sizeof(float), 256);
 }
 
 int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,

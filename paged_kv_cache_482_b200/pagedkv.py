@@ -9,6 +9,7 @@ The functions mirror ``include/pagedkv.h``:
 
 * ``store_kvcache`` -- ``pkv_store_kvcache``
 * ``plan_decode`` -- ``pkv_plan_decode``
+* ``decode_workspace_bytes`` -- ``pkv_decode_workspace_bytes``
 * ``paged_attention_decode`` -- ``pkv_paged_attention_decode``
 * ``paged_attention_prefill`` -- ``pkv_paged_attention_prefill``
 * ``fused_add_rmsnorm`` -- ``pkv_fused_add_rmsnorm``
@@ -37,7 +38,7 @@ PKV_CACHE_BF16 = 0
 PKV_CACHE_FP8_E4M3 = 1  # k_scale / v_scale: [num_kv_heads] fp32
 PKV_CACHE_FP8_E4M3_TOKEN = 2  # k_scale / v_scale: scale pools [num_blocks, num_kv_heads, block_size] fp32
 
-EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_paged_attention_decode", "pkv_status_string",
+EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_decode_workspace_bytes", "pkv_paged_attention_decode", "pkv_status_string",
             "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
             "pkv_paged_attention_prefill", "pkv_fused_add_rmsnorm")
 
@@ -78,6 +79,8 @@ def load_library(path: str):
     L.pkv_store_kvcache.restype = i32
     L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
     L.pkv_plan_decode.restype = i32
+    L.pkv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.pkv_decode_workspace_bytes.restype = sz
     L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i64, f32, i32,
                                              vp, vp, i32, i32, vp, sz, vp, vp, vp]
     L.pkv_paged_attention_decode.restype = i32
@@ -161,6 +164,11 @@ def plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_c
     _check(st, "pkv_plan_decode")
     return dict(partition_tokens=plan.partition_tokens, max_partitions=plan.max_partitions,
                 workspace_bytes=plan.workspace_bytes)
+
+
+def decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len) -> int:
+    """Scratch bytes that suffice for any automatic split-K plan of these sizes."""
+    return int(lib().pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))
 
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out=None, k_scale=None,

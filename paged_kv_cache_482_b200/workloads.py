@@ -150,12 +150,18 @@ def _randn_bf16(shape, gen: torch.Generator, device) -> torch.Tensor:
     return out
 
 
-def _structure(cfg: DecodeConfig, seed: int):
-    """Context lengths and physical block ids (device independent, CPU)."""
+def _structure(cfg: DecodeConfig, seed: int, ctx_override=None):
+    """Context lengths and physical block ids (device independent, CPU).
+    ``ctx_override`` ({sequence: context length}) replaces drawn lengths, e.g.
+    to put some sequences exactly on split-K partition edges."""
     g = torch.Generator(device="cpu").manual_seed(seed)
     S, bs = cfg.num_seqs, cfg.block_size
     draws = torch.randint(cfg.ctx_lo, cfg.ctx_hi + 1, (S,), generator=g, dtype=torch.int64)
     ctx = draws + cfg.prefix_tokens
+    for i, n in (ctx_override or {}).items():
+        if not (max(1, cfg.prefix_tokens) <= int(n) <= cfg.max_context):
+            raise ValueError(f"context length {n} outside [{max(1, cfg.prefix_tokens)}, {cfg.max_context}]")
+        ctx[int(i)] = int(n)
     if cfg.prefix_tokens % bs:
         raise ValueError("a shared prefix must fill whole blocks")
     shared = cfg.prefix_tokens // bs
@@ -174,16 +180,17 @@ def _structure(cfg: DecodeConfig, seed: int):
     return ctx, tables, nblk
 
 
-def generate(cfg: DecodeConfig, seed: int = 0, device: str | torch.device = "cpu") -> Workload:
+def generate(cfg: DecodeConfig, seed: int = 0, device: str | torch.device = "cpu", ctx_override=None) -> Workload:
     """Draw one decode step's inputs for ``cfg``.
 
     Lengths and block ids come from a CPU generator seeded with ``seed`` and
-    are the same on every device. Q/K/V come from a generator on ``device``
-    seeded with ``seed + 1`` (torch's CPU and CUDA generators give different
-    streams, so data drawn on different devices differ; each is reproducible).
+    are the same on every device (``ctx_override`` replaces chosen lengths).
+    Q/K/V come from a generator on ``device`` seeded with ``seed + 1``
+    (torch's CPU and CUDA generators give different streams, so data drawn on
+    different devices differ; each is reproducible).
     """
     device = torch.device(device)
-    ctx, tables, nblk = _structure(cfg, seed)
+    ctx, tables, nblk = _structure(cfg, seed, ctx_override)
     S, nkv, d, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
     P = cfg.prefix_tokens
 

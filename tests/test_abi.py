@@ -124,6 +124,52 @@ def test_plan_requests(K):
         K.plan_decode(4, 32, 8, 128, 16, 32768, True, -1)  # one partition cannot span 2048 blocks
 
 
+@pytest.mark.parametrize("name", ["tiny", "qwen3_0.6b", "qwen3_8b", "prefix_shared", "long_fp8"])
+def test_workspace_bound_covers_every_automatic_plan(K, name):
+    """pkv_decode_workspace_bytes(num_seqs, nq, d, max_context_len) is enough
+    for the automatic plan of every KV head count, block size and cache type
+    those four sizes allow, and is 0 exactly when no such plan can split."""
+    from paged_kv_cache_482_b200 import workloads as W
+
+    c = W.CONFIGS[name]
+    bound = K.decode_workspace_bytes(c.num_seqs, c.num_q_heads, c.head_dim, c.max_context)
+    L = K.lib()
+    worst = 0
+    for g in (1, 2, 4, 8):
+        if c.num_q_heads % g:
+            continue
+        for bs in (8, 16, 32, 64, 128, 256, 512, 1024):
+            for dt in (K.PKV_CACHE_BF16, K.PKV_CACHE_FP8_E4M3, K.PKV_CACHE_FP8_E4M3_TOKEN):
+                plan = K._Plan()
+                st = L.pkv_plan_decode(c.num_seqs, c.num_q_heads, c.num_q_heads // g, c.head_dim, bs,
+                                       c.max_context, dt, 0, ctypes.byref(plan))
+                assert st == K.PKV_OK
+                assert plan.workspace_bytes <= bound, (g, bs, dt)
+                worst = max(worst, plan.workspace_bytes)
+    assert (bound == 0) == (c.max_context <= 1024)
+    if name == "long_fp8":
+        assert worst > 0  # the bound is exercised by a real split
+
+
+def test_workspace_bound_sweep(K):
+    import random
+
+    rng = random.Random(3)
+    L = K.lib()
+    for _ in range(400):
+        S, nq, d, ctx = rng.randint(1, 600), rng.choice([8, 16, 32, 64]), rng.choice([64, 128]), rng.randint(1, 70000)
+        bound = K.decode_workspace_bytes(S, nq, d, ctx)
+        g = rng.choice([1, 2, 4, 8])
+        bs = rng.choice([8, 16, 256, 1024])
+        plan = K._Plan()
+        st = L.pkv_plan_decode(S, nq, nq // g, d, bs, ctx, rng.choice([0, 1, 2]), 0, ctypes.byref(plan))
+        if st == K.PKV_OK:
+            assert plan.workspace_bytes <= bound, (S, nq, d, ctx, g, bs)
+    assert K.decode_workspace_bytes(0, 32, 128, 4096) == 0
+    assert K.decode_workspace_bytes(4, 32, 128, 1024) == 0
+    assert K.decode_workspace_bytes(4, 32, 128, 1025) > 0
+
+
 def test_binding_refuses_to_run_without_library(tmp_path):
     from paged_kv_cache_482_b200 import pagedkv
 

@@ -67,3 +67,71 @@ def test_churn_matches_a_dict():
     for k in keys:
         assert m.free_sequence(int(k)) == K.PKV_OK
     assert m.num_free() == nb
+
+
+def _home(sid: int, mask: int) -> int:
+    """Home slot of an id in the manager's live-sequence table (a multiply by
+    the 64-bit golden ratio, an xor-shift, a mask), restated here only to pick
+    ids that collide on purpose."""
+    h = (sid * 0x9E3779B97F4A7C15) & (2**64 - 1)
+    return (h ^ (h >> 29)) & mask
+
+
+def _ids_with_home(slot: int, n: int, mask: int = 63, start: int = 1):
+    out, x = [], start
+    while len(out) < n:
+        if _home(x, mask) == slot:
+            out.append(x)
+        x += 1
+    return out
+
+
+def test_probe_runs_that_wrap_and_erase_from_their_middle():
+    """With at most 32 live sequences the table has 64 slots. Ids whose home
+    slots are 60, 62, 63, 0 and 1 build one long probe run that wraps past the
+    end of the table; erasing from its middle must shift the right entries
+    back (backward-shift deletion) so that every remaining id is still found,
+    and an erased id is gone."""
+    groups = [_ids_with_home(60, 10), _ids_with_home(62, 4), _ids_with_home(63, 3), _ids_with_home(0, 4),
+              _ids_with_home(1, 3)]
+    ids = [i for g in groups for i in g]
+    assert len(set(ids)) == len(ids) <= 32
+    rng = np.random.default_rng(11)
+    m = BlockManager(512, 4)
+    live = {}
+
+    def check_all():
+        for sid in ids:
+            if sid in live:
+                table, n = m.block_table(sid)
+                assert n == live[sid]
+            else:
+                try:
+                    m.block_table(sid)
+                    raise AssertionError(f"erased id {sid} still found")
+                except K.PagedKVError:
+                    pass
+
+    # interleaved inserts: the run starting at 60 wraps and absorbs the others
+    order = [g[i] for i in range(10) for g in groups if i < len(g)]
+    for k, sid in enumerate(order):
+        st, _ = m.add_sequence(sid, np.array([k % 3] * (1 + k % 5)))
+        assert st == K.PKV_OK
+        live[sid] = 1 + k % 5
+        check_all()
+    # erase from the middle of the run, then churn
+    for sid in (groups[0][4], groups[3][1], groups[0][0], groups[2][1], groups[1][3]):
+        assert m.free_sequence(sid) == K.PKV_OK
+        live.pop(sid)
+        check_all()
+    for step in range(3000):
+        sid = ids[int(rng.integers(0, len(ids)))]
+        if sid in live:
+            assert m.free_sequence(sid) == K.PKV_OK
+            live.pop(sid)
+        else:
+            n = int(rng.integers(1, 6))
+            st, _ = m.add_sequence(sid, rng.integers(0, 3, n))
+            assert st == K.PKV_OK
+            live[sid] = n
+        check_all()

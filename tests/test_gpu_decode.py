@@ -219,10 +219,26 @@ def test_sequence_order_does_not_change_results():
                                            dev_err=err)
             assert K.read_device_error(err) == K.PKV_OK
             assert torch.equal(out.view(torch.int16), base.view(torch.int16))
-    # an entry outside the sequences is reported and skipped
+    # an entry outside the sequences is reported and skipped: the sequence it
+    # displaced keeps its old out rows (split or not, after a call that left
+    # that sequence's partials in the workspace), every other row is exact
     bad = orders[0].clone()
+    skipped = int(bad[0])
     bad[0] = c.num_seqs
-    err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
-                             max_context_len=c.max_context, seq_order=bad, dev_err=err)
-    assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS
+    for split in (0, 64):
+        base = K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                        max_context_len=c.max_context, partition_request=split)
+        plan = K.plan_decode(c.num_seqs, c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size, c.max_context,
+                             False, split)
+        ws = torch.empty(max(plan["workspace_bytes"], 256), dtype=torch.uint8, device="cuda")
+        K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                 max_context_len=c.max_context, partition_request=split, workspace=ws)
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = torch.full_like(wl.q, 7.0)
+        K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, out=out,
+                                 max_context_len=c.max_context, partition_request=split, workspace=ws,
+                                 seq_order=bad, dev_err=err)
+        assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS
+        assert bool((out[skipped].float() == 7.0).all())
+        keep = [i for i in range(c.num_seqs) if i != skipped]
+        assert torch.equal(out[keep].view(torch.int16), base[keep].view(torch.int16))

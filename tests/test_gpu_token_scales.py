@@ -93,10 +93,17 @@ def test_zero_and_outlier_rows():
 
 
 def test_long_fp8_token_sampled():
-    wl = W.generate(W.CONFIGS["long_fp8_token"], 0, device="cuda")
+    """The full-size split-K step with per-token scales; 16+ sequences checked,
+    among them lengths on partition edges (k * P, k * P + 1, k * P - 1)."""
+    from test_gpu_configs import edge_lengths
+
+    cfg = W.CONFIGS["long_fp8_token"]
+    override, pt = edge_lengths(cfg)
+    wl = W.generate(cfg, 0, device="cuda", ctx_override=override)
     out, (kp, vp, ks, vs), st = run_decode(wl)
     assert st == K.PKV_OK and bool(torch.isfinite(out.float()).all())
-    ids = sample_ids(wl, 5)
+    ids = sorted(set(sample_ids(wl, 10)) | set(override))
+    assert len(ids) >= 16
     ref, rkp, rvp, rst, rks, rvs = O.run_workload(wl, num_threads=THREADS, seq_ids=ids)
     assert rst == O.ORC_OK
     blocks = torch.unique(wl.block_tables[ids].flatten())

@@ -16,9 +16,6 @@ import torch
 from paged_kv_cache_482_b200 import pagedkv as K
 from paged_kv_cache_482_b200 import workloads as W
 
-BF16_ABS, FP8_ABS = 2e-2, 5e-2
-
-
 def _setup(cfg, seed):
     wl = W.generate(cfg, seed)
     dev = {f: getattr(wl, f).cuda().contiguous() if getattr(wl, f) is not None else None
@@ -35,6 +32,28 @@ def _setup(cfg, seed):
     return wl, dev, kp, vp
 
 
+def _padded_tables(bt, width):
+    """Block tables widened to `width` columns with -1 (unused entries)."""
+    if bt.shape[1] >= width:
+        return bt
+    pad = torch.full((bt.shape[0], width - bt.shape[1]), -1, dtype=bt.dtype, device=bt.device)
+    return torch.cat([bt, pad], dim=1).contiguous()
+
+
+def _both(d, kp, vp, cfg, part, max_ctx, width, fp8):
+    """(static-scratch result, workspace result) on the same inputs and plan."""
+    bt = _padded_tables(d["block_tables"], width)
+    ref = K.paged_attention_decode(d["q"], kp, vp, bt, d["context_lens"], cfg.softmax_scale, k_scale=d["k_scale"],
+                                   v_scale=d["v_scale"], max_context_len=max_ctx, partition_request=part)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full_like(d["q"], float("nan"))
+    K.paged_attention_decode_static_scratch(d["q"], kp, vp, bt, d["context_lens"], cfg.softmax_scale, out=out,
+                                            k_scale=d["k_scale"], v_scale=d["v_scale"], max_context_len=max_ctx,
+                                            partition_request=part, dev_err=err)
+    assert K.read_device_error(err) == K.PKV_OK
+    return out, ref
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("cfg,part", [
     (W.DecodeConfig("na_bf16", 6, 16, 4, 128, 16, 200, 1500), 256),
@@ -42,24 +61,27 @@ def _setup(cfg, seed):
     (W.DecodeConfig("na_bf16_d64", 4, 4, 2, 64, 32, 1, 900), 128),
 ])
 def test_static_scratch_matches_workspace_entry_point_twice(cfg, part):
-    wl, d, kp, vp = _setup(cfg, 5)
-    plan = K.plan_decode(cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size,
-                         cfg.max_context, wl.is_fp8, part)
+    """Two calls in a row on different batches: the second batch has shorter
+    contexts, so it has fewer partitions per sequence than the first and the
+    array still holds first-call partials that would be wrong if read. Both
+    results must be bit-identical to the workspace entry point on the same
+    inputs and plan (the same kernels run on the same data)."""
+    wl_a, da, kpa, vpa = _setup(cfg, 5)
+    short = cfg.with_(name=cfg.name + "_short", ctx_lo=1, ctx_hi=max(2, cfg.ctx_hi // 3))
+    wl_b, db, kpb, vpb = _setup(short, 6)
+    max_ctx = cfg.max_context
+    width = da["block_tables"].shape[1]
+    plan = K.plan_decode(cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size, max_ctx,
+                         wl_a.is_fp8, part)
     assert plan["workspace_bytes"] > 0, "the case must exercise the split-K scratch"
-    ref = K.paged_attention_decode(d["q"], kp, vp, d["block_tables"], d["context_lens"], cfg.softmax_scale,
-                                   k_scale=d["k_scale"], v_scale=d["v_scale"], max_context_len=cfg.max_context,
-                                   partition_request=part)
-    tol = FP8_ABS if wl.is_fp8 else BF16_ABS
-    for _ in range(2):  # the second call finds the first call's partials in the array
-        err = torch.zeros(1, dtype=torch.int32, device="cuda")
-        out = torch.full_like(d["q"], float("nan"))
-        K.paged_attention_decode_static_scratch(d["q"], kp, vp, d["block_tables"], d["context_lens"],
-                                                cfg.softmax_scale, out=out, k_scale=d["k_scale"],
-                                                v_scale=d["v_scale"], max_context_len=cfg.max_context,
-                                                partition_request=part, dev_err=err)
-        assert K.read_device_error(err) == K.PKV_OK
+    pt = plan["partition_tokens"]
+    parts_a = (-(-da["context_lens"].long() // pt)).max().item()
+    parts_b = (-(-db["context_lens"].long() // pt)).max().item()
+    assert parts_b < parts_a, "the second call must leave stale first-call partials behind"
+    for d, kp, vp, wl in ((da, kpa, vpa, wl_a), (db, kpb, vpb, wl_b)):
+        out, ref = _both(d, kp, vp, cfg, part, max_ctx, width, wl.is_fp8)
         assert bool(torch.isfinite(out.float()).all())
-        assert float((out.float() - ref.float()).abs().max()) <= tol
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
 
 
 def test_plan_beyond_the_array_is_refused_before_launch():
