@@ -4,8 +4,10 @@
 // stages hold K and V of one tile and the ring is about 48 KB deep, so that
 // four blocks share an SM with well over 100 KB of loads in flight.
 #include <atomic>
+#include <cstring>
 
 #include "decode.cuh"
+#include "decode_mma.cuh"
 
 namespace pkv {
 
@@ -43,6 +45,66 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// E4M3 cache, head_dim 128: the warp-MMA kernel (decode_mma.cuh).
+template <int G, bool TS>
+cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
+    using T = MmaTraits<G>;
+#ifdef PKV_MMA_MIN_BLOCKS
+    constexpr int MINB = PKV_MMA_MIN_BLOCKS;
+#else
+    constexpr int MINB = 3;
+#endif
+    auto kern = paged_decode_mma_kernel<G, MINB, TS>;
+    static std::atomic<unsigned long long> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kAlloc);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    const long long blocks = (long long)p.num_seqs * p.num_kv_heads * p.num_partitions;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    // tensor-map row coordinates are int32
+    const long long rows = p.num_blocks * p.num_kv_heads * p.block_size;
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const int box_rows = p.block_size < 16 ? p.block_size : 16;
+    CUtensorMap mk, mv;
+    std::memset(&mk, 0, sizeof(mk));
+    std::memset(&mv, 0, sizeof(mv));
+    if (!make_e4m3_pool_map(&mk, p.k_cache, rows, box_rows) || !make_e4m3_pool_map(&mv, p.v_cache, rows, box_rows))
+        return cudaErrorInvalidValue;
+    kern<<<(unsigned)blocks, T::kThreads, T::kAlloc, stream>>>(p, mk, mv, box_rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.num_partitions <= 1) return e;
+    paged_decode_reduce_kernel<128><<<(unsigned)((long long)p.num_seqs * p.num_q_heads), 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool TS>
+cudaError_t launch_mma(int group, const DecodeParams &p, cudaStream_t stream) {
+    switch (group) {
+        case 1: return launch_mma_one<1, TS>(p, stream);
+        case 2: return launch_mma_one<2, TS>(p, stream);
+        case 4: return launch_mma_one<4, TS>(p, stream);
+        case 8: return launch_mma_one<8, TS>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+int mma_tile_of(int group) {
+    switch (group) {
+        case 1: return MmaTraits<1>::kTile;
+        case 2: return MmaTraits<2>::kTile;
+        case 4: return MmaTraits<4>::kTile;
+        case 8: return MmaTraits<8>::kTile;
+        default: return 0;
+    }
+}
+
 template <int D, bool FP8>
 int tile_of(int group) {
     switch (group) {
@@ -68,7 +130,7 @@ cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) 
 }  // namespace
 
 int decode_tile_tokens(int head_dim, int group, bool fp8) {
-    if (head_dim == 128) return fp8 ? tile_of<128, true>(group) : tile_of<128, false>(group);
+    if (head_dim == 128) return fp8 ? mma_tile_of(group) : tile_of<128, false>(group);
     if (head_dim == 64) return fp8 ? tile_of<64, true>(group) : tile_of<64, false>(group);
     return 0;
 }
@@ -103,6 +165,8 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.out = static_cast<__nv_bfloat16 *>(a.out);
     p.dev_err = a.dev_err;
     const int group = a.num_q_heads / a.num_kv_heads;
+    if (a.fp8 && a.head_dim == 128) return a.token_scales ? launch_mma<true>(group, p, stream)
+                                                          : launch_mma<false>(group, p, stream);
     if (a.fp8 && a.token_scales) {
         if (a.head_dim == 128) return launch_group<128, true, true>(group, p, stream);
         if (a.head_dim == 64) return launch_group<64, true, true>(group, p, stream);

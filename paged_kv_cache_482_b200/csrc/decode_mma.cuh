@@ -1,0 +1,559 @@
+// decode_mma.cuh -- paged decode attention over an E4M3 cache (head_dim 128)
+// with the products on the warp-level tensor-core MMA (sm_100a).
+//
+// Why: with one byte per cached element, the CUDA-core decode is bound by
+// instruction issue, not by HBM -- every (token, KV head) costs 2 * G * 128
+// multiply-adds plus the E4M3 widening against only 256 bytes of K and V.
+// The G query heads of a KV head against a tile of tokens are small matrix
+// products, [tokens x d] x [d x G] for the scores and [d x tokens] x [tokens
+// x G] for P V, so this kernel hands them to mma.sync m16n8k16 (f16 operands,
+// fp32 accumulation): every E4M3 code widens exactly to f16 (one conversion
+// per pair, straight into an operand register), q is scaled by a power of
+// two into f16 (exact for bf16 q), and the MMA forms the exact products and
+// accumulates them in fp32. What remains on the CUDA cores is the widening,
+// the softmax and the bookkeeping. The problem is the pages' decode
+// ("DeepSeek复刻vLLM反超原版", section "vLLM：大模型推理的加速引擎与挑战":
+// block tables into a shared pool; "nano-vllm-lite", section 核心技术改进 3:
+// the FP8 KV cache and its 2x smaller reads).
+//
+// Block structure: one thread block of kNW warps per (sequence, KV head,
+// partition); every K/V byte of the partition is read from HBM once. Each
+// warp owns kWT consecutive tokens of every kTile-token tile and runs its own
+// pipeline: lane 0 copies its rows of K and V with tensor-map copies
+// (cp.async.bulk.tensor, 16-row boxes of 128 bytes, 128-byte swizzle, no
+// multicast) into a kStages-deep ring, completing on the warp's own
+// mbarriers, and refills a stage once the warp is done with it.
+//
+// Per 16-token group (fragment layouts of m16n8k16; g = lane / 4, t = lane % 4):
+//  * Scores, S^T[16 tokens x 8 heads] = K[16 x 128] . Q^T[128 x 8]: A = K rows
+//    g and g + 8, B = q of head g (zero for g >= G). The contraction order of
+//    the 128 dims is free, so k-step i takes dims 32t + 4i .. 32t + 4i + 3 of
+//    each lane's rows: a lane reads 32 contiguous codes of two rows, and one
+//    conversion per code pair gives an operand register. The swizzle makes
+//    these reads free of bank conflicts.
+//  * Softmax in base 2 over the warp's tile (scores times scale * log2 e,
+//    the K scale and q's power of two), with a lazy reference maximum: it
+//    moves only when the tile maximum exceeds it by more than 8, so weights
+//    stay <= 2^8 (f16 range) and the accumulators are rescaled rarely.
+//  * The weights, packed to f16, are transposed in registers
+//    (movmatrix.trans) into the B operand of P V.
+//  * P V, O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] . P^T[16 x 8]: m-tile
+//    j covers dims 16g + 2j (row g) and 16g + 2j + 1 (row g + 8), so a lane
+//    reads 16 contiguous codes of 4 rows; byte permutes pair two tokens' codes
+//    at one dim before the conversion.
+//  * Rows past the end of the context (inside the last copied box) are
+//    excluded: their scores become -inf and their V codes zero.
+//  * Per-token scales (TS): the K and V scale runs are bulk-copied with the
+//    boxes; a score is multiplied by its token's K scale; a weight by its V
+//    scale times 2^-E before it is rounded to f16, where E tracks the largest
+//    V scale seen so far (a rise of E rescales the accumulators exactly, like
+//    a rise of the maximum), and l sums the unscaled weights.
+//  * Epilogue as in the CUDA-core kernel: the warps' (max, sum, accumulators)
+//    merge in shared memory, then bf16 output or a normalised split-K partial.
+//
+// Every wait is bounded (PKV_DEVERR_TIMEOUT), every block id and length is
+// checked before a byte is copied (PKV_DEVERR_BOUNDS), and each warp waits
+// for its own copies in flight before the block exits.
+#pragma once
+
+#include <cuda.h>
+
+#include "decode.cuh"
+#include "tc_common.cuh"
+
+namespace pkv {
+
+#ifndef PKV_MMA_WARPS
+#define PKV_MMA_WARPS 4
+#endif
+#ifndef PKV_MMA_WARP_TOKENS
+#define PKV_MMA_WARP_TOKENS 32
+#endif
+#ifndef PKV_MMA_STAGES
+#define PKV_MMA_STAGES 2
+#endif
+
+template <int G>
+struct MmaTraits {
+    static constexpr int kD = 128;
+    static constexpr int kNW = PKV_MMA_WARPS;
+    static constexpr int kWT = PKV_MMA_WARP_TOKENS;  // tokens per warp per tile
+    static constexpr int kNGW = kWT / 16;            // 16-token groups per warp per tile
+    static constexpr int kTile = kNW * kWT;
+    static constexpr int kStages = PKV_MMA_STAGES;
+    static constexpr int kGroupBytes = 16 * 128;  // 16 rows of 128 codes
+    static constexpr int kSliceBytes = kWT * 128;  // a warp's K (or V) rows of one tile
+    // [stage][warp][K slice | V slice], 1024-byte aligned (the swizzle atom)
+    static constexpr int kStageBytes = kNW * 2 * kSliceBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kOffScales = kRingBytes;  // [stage][warp][K | V][kWT] fp32 (per-token scales)
+    static constexpr int kScaleBytes = kStages * kNW * 2 * kWT * 4;
+    static constexpr int kOffBars = kOffScales + kScaleBytes;  // full_k[NW][S], full_v[NW][S]
+    static constexpr int kOffCnt = kOffBars + 2 * kNW * kStages * 8;
+    static constexpr int kOffIds = kOffCnt + kNW * 4;
+    static constexpr int kSmemBytes = kOffIds + kMaxIdsPerPartition * 4;
+    static constexpr int kAlloc = kSmemBytes + 1024;  // + base alignment
+    static constexpr int kThreads = kNW * 32;
+    static constexpr int kMergeFloats = kNW * G * kD + 3 * kNW * G;
+    static_assert(kWT % 16 == 0 && kNGW >= 1, "whole 16-token groups");
+    static_assert(kMergeFloats * 4 <= kRingBytes, "merge area must fit in the ring");
+    static_assert(G >= 1 && G <= 8, "one n8 column per query head");
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float lds32f(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// D += A . B, m16n8k16, f16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8 x 8 matrix of 16-bit elements held one word per lane
+// (lane g*4 + t holds row g, columns 2t and 2t + 1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+template <int G, int MIN_BLOCKS, bool TS>
+__global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
+    paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
+                            const __grid_constant__ CUtensorMap map_v, int box_rows) {
+    using T = MmaTraits<G>;
+    constexpr int D = T::kD;
+    constexpr int NW = T::kNW;
+    constexpr int WT = T::kWT;
+    constexpr int NGW = T::kNGW;
+    constexpr int TILE = T::kTile;
+    constexpr int STAGES = T::kStages;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    const uint32_t sbase = smem_addr(smem);
+    int32_t *ids = reinterpret_cast<int32_t *>(smem + T::kOffIds);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int g = lane >> 2;  // fragment row group
+    const int t = lane & 3;   // thread in group
+
+    const int part = blockIdx.x % p.num_partitions;
+    const int rest = blockIdx.x / p.num_partitions;
+    const int kvh = rest % p.num_kv_heads;
+    const int seq_slot = rest / p.num_kv_heads;
+    const int seq = p.seq_order ? __ldg(p.seq_order + seq_slot) : seq_slot;
+    if (seq < 0 || seq >= p.num_seqs) {
+        if (tid == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+        return;
+    }
+    const int ctx = __ldg(p.context_lens + seq);
+    const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
+    const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
+    const int start = part * p.partition_tokens;
+    const int end = bad_len ? start : min(start + p.partition_tokens, ctx);
+    const int n_parts_seq = bad_len ? 1 : (ctx + p.partition_tokens - 1) / p.partition_tokens;
+    const bool single = n_parts_seq == 1;
+    if (!bad_len && start >= end) return;
+    if (bad_len && part != 0) return;
+
+    const int first_blk = start >> p.log2_block_size;
+    const int n_blk = bad_len ? 0 : ((end - 1) >> p.log2_block_size) - first_blk + 1;
+    int bad = bad_len || n_blk > kMaxIdsPerPartition;
+    const int32_t *table = p.block_tables + (long long)seq * p.max_blocks_per_seq + first_blk;
+    for (int i = tid; i < n_blk && i < kMaxIdsPerPartition; i += T::kThreads) {
+        const int32_t id = __ldg(table + i);
+        ids[i] = id;
+        bad |= (id < 0 || (long long)id >= p.num_blocks);
+    }
+    uint64_t *full_k = reinterpret_cast<uint64_t *>(smem + T::kOffBars) + warp * STAGES;
+    uint64_t *full_v = full_k + NW * STAGES;
+    int *issued = reinterpret_cast<int *>(smem + T::kOffCnt) + warp;  // tiles this warp issued
+    if (lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_k[s], 1);
+            mbar_init(&full_v[s], 1);
+        }
+        fence_barrier_init();
+    }
+    bad = __syncthreads_or(bad);
+    const int qh0 = kvh * G;
+    if (bad) {
+        if (tid == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+        if (single || bad_len) {
+            for (int i = tid; i < G * D; i += T::kThreads)
+                p.out[((long long)seq * p.num_q_heads + qh0) * D + i] = __float2bfloat16_rn(0.f);
+        } else if (tid < G) {
+            float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + tid) * p.num_partitions + part) * 2;
+            ml[0] = -CUDART_INF_F;
+            ml[1] = 0.f;
+        }
+        return;
+    }
+
+    const int n_tiles = (end - start + TILE - 1) / TILE;
+    const int bs_mask = p.block_size - 1;
+    const int lbs = p.log2_block_size;
+    // This warp's rows of tile j: logical tokens [start + j*TILE + warp*WT, ...).
+    auto warp_tok0 = [&](int j) { return start + j * TILE + warp * WT; };
+    // Issue this warp's K and V boxes (and, TS, scale runs) of tile j into
+    // stage s. Only boxes holding at least one valid token are copied; a box
+    // never leaves its (block, KV head) run, since box_rows divides 16 and
+    // the block size, and groups start on multiples of 16.
+    auto issue = [&](int j, int s) {
+        const int a0 = warp_tok0(j);
+        const int nv = min(end - a0, WT);
+        uint32_t bytes = 0;
+        for (int a = 0; a < nv; a += box_rows) bytes += box_rows * 128 + (TS ? box_rows * 4 : 0);
+        mbar_arrive_expect_tx(&full_k[s], bytes);
+        mbar_arrive_expect_tx(&full_v[s], bytes);
+        const uint32_t sk = sbase + s * T::kStageBytes + warp * 2 * T::kSliceBytes;
+        const uint32_t sv = sk + T::kSliceBytes;
+        for (int a = 0; a < nv; a += box_rows) {
+            const int tok = a0 + a;
+            const long long phys = ids[(tok >> lbs) - first_blk];
+            const long long row = (phys * p.num_kv_heads + kvh) * p.block_size + (tok & bs_mask);
+            tc::tma_load_2d(sk + a * 128, &map_k, 0, (int)row, &full_k[s]);
+            tc::tma_load_2d(sv + a * 128, &map_v, 0, (int)row, &full_v[s]);
+            if constexpr (TS) {
+                uint8_t *sc = smem + T::kOffScales + ((s * NW + warp) * 2) * WT * 4;
+                bulk_g2s(sc + a * 4, p.k_scale + row, box_rows * 4, &full_k[s]);
+                bulk_g2s(sc + WT * 4 + a * 4, p.v_scale + row, box_rows * 4, &full_v[s]);
+            }
+        }
+    };
+    if (lane == 0) {
+        int n = 0;
+        for (int j = 0; j < min(STAGES, n_tiles) && warp_tok0(j) < end; ++j, ++n) issue(j, j);
+        *issued = n;
+    }
+    __syncwarp();
+
+    // q of head qh0 + g, dims 32t .. 32t + 31, as f16 pairs in k-step order:
+    // qf[i][0] = dims 32t + 4i, +1; qf[i][1] = dims 32t + 4i + 2, +3 (zero
+    // for g >= G). Scaled by 2^k so that the largest |q| of the KV head's
+    // group lies in [2^14, 2^15): exact for bf16 q down to 2^-29 of it.
+    uint32_t qf[8][2];
+    float score_scale;
+    {
+        uint32_t qw[16];
+        if (g < G) {
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(p.q + ((long long)seq * p.num_q_heads + qh0 + g) * D + 32 * t);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 w = __ldg(src + i);
+                qw[4 * i] = w.x;
+                qw[4 * i + 1] = w.y;
+                qw[4 * i + 2] = w.z;
+                qw[4 * i + 3] = w.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) qw[i] = 0u;
+        }
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int e = 0;
+        frexpf(mx, &e);  // mx < 2^e
+        const int k = 15 - e;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            qf[i][0] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i]), k), ldexpf(bf16hi(qw[2 * i]), k));
+            qf[i][1] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i + 1]), k), ldexpf(bf16hi(qw[2 * i + 1]), k));
+        }
+        score_scale = ldexpf(TS ? p.qk_scale_log2 : p.qk_scale_log2 * __ldg(p.k_scale + kvh), -k);
+    }
+
+    float o[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[j][i] = 0.f;
+    float m_ref[2] = {-CUDART_INF_F, -CUDART_INF_F};  // heads 2t, 2t + 1 (base-2 units)
+    float l[2] = {0.f, 0.f};
+    int vexp = -100000;  // TS: weights are scaled by 2^-vexp before rounding
+
+    // Swizzled row r, 16-byte chunk c of a 16-row group at byte address base.
+    auto sw = [](uint32_t base, int r, int c) { return base + r * 128 + (((c ^ r) & 7) << 4); };
+
+    bool ok = true;
+    int s = 0, rnd = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+        const int a0 = warp_tok0(j);
+        const int nv = min(end - a0, WT);  // valid tokens of this warp in tile j
+        if (nv <= 0) break;                // only in the last tile
+        if (!mbar_wait(&full_k[s], rnd & 1)) {
+            ok = false;
+            break;
+        }
+        const uint32_t sk = sbase + s * T::kStageBytes + warp * 2 * T::kSliceBytes;
+        const uint32_t sv = sk + T::kSliceBytes;
+        const uint32_t ssc = smem_addr(smem + T::kOffScales) + ((s * NW + warp) * 2) * WT * 4;
+
+        // ---- scores of the warp's groups (x: base-2 units)
+        float x[NGW][4];
+#pragma unroll
+        for (int gi = 0; gi < NGW; ++gi) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            if (gi * 16 < nv) {
+                const uint32_t kg = sk + gi * T::kGroupBytes;
+                const uint4 k0 = lds128(sw(kg, g, 2 * t));
+                const uint4 k1 = lds128(sw(kg, g, 2 * t + 1));
+                const uint4 k2 = lds128(sw(kg, g + 8, 2 * t));
+                const uint4 k3 = lds128(sw(kg, g + 8, 2 * t + 1));
+                const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint2 a = tc::e4m3x4_to_f16x4(wg[i]);  // row g: dims +0,+1 | +2,+3
+                    const uint2 b = tc::e4m3x4_to_f16x4(wh[i]);  // row g + 8
+                    mma_f16_16816(c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
+                }
+            }
+            float ks0 = score_scale, ks1 = score_scale;
+            if constexpr (TS) {
+                ks0 *= lds32f(ssc + (gi * 16 + g) * 4);
+                ks1 *= lds32f(ssc + (gi * 16 + g + 8) * 4);
+            }
+            // c: (token g, head 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1)
+            const bool v0 = gi * 16 + g < nv, v1 = gi * 16 + g + 8 < nv;
+            x[gi][0] = v0 ? c[0] * ks0 : -CUDART_INF_F;
+            x[gi][1] = v0 ? c[1] * ks0 : -CUDART_INF_F;
+            x[gi][2] = v1 ? c[2] * ks1 : -CUDART_INF_F;
+            x[gi][3] = v1 ? c[3] * ks1 : -CUDART_INF_F;
+        }
+        // ---- tile maximum per head, lazy reference maximum
+        float mx[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            mx[h] = fmaxf(x[0][h], x[0][2 + h]);
+#pragma unroll
+            for (int gi = 1; gi < NGW; ++gi) mx[h] = fmaxf(mx[h], fmaxf(x[gi][h], x[gi][2 + h]));
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+        }
+        const bool move = mx[0] > m_ref[0] + 8.f || mx[1] > m_ref[1] + 8.f;
+        float alpha[2] = {1.f, 1.f};
+        bool rescale = __any_sync(0xffffffffu, move);
+        if (rescale) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float mn = fmaxf(m_ref[h], mx[h]);
+                alpha[h] = m_ref[h] == -CUDART_INF_F ? 0.f : fast_exp2(m_ref[h] - mn);
+                m_ref[h] = mn;
+            }
+        }
+        const float mr0 = m_ref[0] == -CUDART_INF_F ? 0.f : m_ref[0];
+        const float mr1 = m_ref[1] == -CUDART_INF_F ? 0.f : m_ref[1];
+        l[0] *= alpha[0];
+        l[1] *= alpha[1];
+        float pw[NGW][4];
+#pragma unroll
+        for (int gi = 0; gi < NGW; ++gi) {
+            pw[gi][0] = fast_exp2(x[gi][0] - mr0);
+            pw[gi][1] = fast_exp2(x[gi][1] - mr1);
+            pw[gi][2] = fast_exp2(x[gi][2] - mr0);
+            pw[gi][3] = fast_exp2(x[gi][3] - mr1);
+            l[0] += pw[gi][0] + pw[gi][2];
+            l[1] += pw[gi][1] + pw[gi][3];
+        }
+
+        if (!mbar_wait(&full_v[s], rnd & 1)) {
+            ok = false;
+            break;
+        }
+        if constexpr (TS) {
+            // V scales of the thread's tokens (rows g, g + 8 of each group; 0
+            // past the end). A tile maximum at or above 2^vexp raises vexp and
+            // rescales the accumulators by 2^-rise (exact), so that the
+            // weights times 2^-vexp stay below 2^9 in f16.
+            float vsc[NGW][2];
+            float vm = 0.f;
+#pragma unroll
+            for (int gi = 0; gi < NGW; ++gi) {
+                const bool v0 = gi * 16 + g < nv, v1 = gi * 16 + g + 8 < nv;
+                vsc[gi][0] = v0 ? lds32f(ssc + WT * 4 + (gi * 16 + g) * 4) : 0.f;
+                vsc[gi][1] = v1 ? lds32f(ssc + WT * 4 + (gi * 16 + g + 8) * 4) : 0.f;
+                vm = fmaxf(vm, fmaxf(vsc[gi][0], vsc[gi][1]));
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+            int ev = 0;
+            frexpf(vm, &ev);  // vm < 2^ev; the same in every lane
+            if (ev > vexp) {
+                const float f = ldexpf(1.f, vexp - ev);  // 0 for the first rise
+                alpha[0] *= f;
+                alpha[1] *= f;
+                rescale = true;
+                vexp = ev;
+            }
+            const float vinv = ldexpf(1.f, -vexp);
+#pragma unroll
+            for (int gi = 0; gi < NGW; ++gi) {
+                const float f0 = vsc[gi][0] * vinv, f1 = vsc[gi][1] * vinv;
+                pw[gi][0] *= f0;
+                pw[gi][1] *= f0;
+                pw[gi][2] *= f1;
+                pw[gi][3] *= f1;
+            }
+        }
+        if (rescale) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                o[jj][0] *= alpha[0];
+                o[jj][1] *= alpha[1];
+                o[jj][2] *= alpha[0];
+                o[jj][3] *= alpha[1];
+            }
+        }
+        // ---- P V
+#pragma unroll
+        for (int gi = 0; gi < NGW; ++gi) {
+            if (gi * 16 >= nv) continue;
+            const uint32_t b0 = movmatrix_trans(tc::pack_f16(pw[gi][0], pw[gi][1]));  // tokens 2t, 2t+1 of head g
+            const uint32_t b1 = movmatrix_trans(tc::pack_f16(pw[gi][2], pw[gi][3]));  // tokens 2t+8, 2t+9
+            const uint32_t vg = sv + gi * T::kGroupBytes;
+            uint4 r0 = lds128(sw(vg, 2 * t, g));
+            uint4 r1 = lds128(sw(vg, 2 * t + 1, g));
+            uint4 r2 = lds128(sw(vg, 2 * t + 8, g));
+            uint4 r3 = lds128(sw(vg, 2 * t + 9, g));
+            if (gi * 16 + 16 > nv) {  // rows past the end: zero codes (stale slots may hold NaN)
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                if (gi * 16 + 2 * t >= nv) r0 = z;
+                if (gi * 16 + 2 * t + 1 >= nv) r1 = z;
+                if (gi * 16 + 2 * t + 8 >= nv) r2 = z;
+                if (gi * 16 + 2 * t + 9 >= nv) r3 = z;
+            }
+            const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+            const uint32_t w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                // dims 16g + 4qd .. +3 of tokens (2t, 2t+1) and (2t+8, 2t+9)
+                const uint2 x0 = tc::e4m3x4_to_f16x4(__byte_perm(w0[qd], w1[qd], 0x5140));
+                const uint2 x1 = tc::e4m3x4_to_f16x4(__byte_perm(w0[qd], w1[qd], 0x7362));
+                const uint2 y0 = tc::e4m3x4_to_f16x4(__byte_perm(w2[qd], w3[qd], 0x5140));
+                const uint2 y1 = tc::e4m3x4_to_f16x4(__byte_perm(w2[qd], w3[qd], 0x7362));
+                mma_f16_16816(o[2 * qd], x0.x, x0.y, y0.x, y0.y, b0, b1);
+                mma_f16_16816(o[2 * qd + 1], x1.x, x1.y, y1.x, y1.y, b0, b1);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) {
+            const int jn = j + STAGES;
+            if (jn < n_tiles && warp_tok0(jn) < end) {
+                fence_proxy_async_smem();
+                issue(jn, s);
+                *issued = jn + 1;
+            }
+        }
+        if (++s == STAGES) {
+            s = 0;
+            ++rnd;
+        }
+    }
+    if (!ok) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+    (void)rnd;
+
+    // ------------------------------------------------------------- epilogue
+    // l: sum over the lanes of the same heads (the g bits).
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+    if (lane == 0) {  // copies of this warp still in flight (only after a timeout)
+        const int n_iss = *issued;
+        for (int jj = max(0, n_iss - STAGES); jj < n_iss; ++jj) {
+            const int ss = jj % STAGES;
+            const uint32_t par = (jj / STAGES) & 1;
+            if (!mbar_wait(&full_k[ss], par) || !mbar_wait(&full_v[ss], par)) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+        }
+    }
+    __syncthreads();
+    float *merge_acc = reinterpret_cast<float *>(smem);  // [NW][G][D]
+    float *merge_m = merge_acc + NW * G * D;            // [NW][G]
+    float *merge_l = merge_m + NW * G;                  // [NW][G]
+    float *merge_w = merge_l + NW * G;                  // [NW][G]
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int head = 2 * t + h;
+        if (head < G) {
+            const float sc = TS ? ldexpf(1.f, vexp) : 1.f;  // TS: undo the 2^-vexp of the weights
+            float *dst = merge_acc + (warp * G + head) * D + 16 * g;
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2)
+                *reinterpret_cast<float4 *>(dst + 2 * jj) =
+                    make_float4(o[jj][h] * sc, o[jj][2 + h] * sc, o[jj + 1][h] * sc, o[jj + 1][2 + h] * sc);
+            if (g == 0) {
+                merge_m[warp * G + head] = m_ref[h];
+                merge_l[warp * G + head] = l[h];
+            }
+        }
+    }
+    __syncthreads();
+    if (tid < G) {
+        const int h = tid;
+        float M = -CUDART_INF_F;
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, merge_m[w * G + h]);
+        float L = 0.f;
+        for (int w = 0; w < NW; ++w) {
+            const float e = merge_m[w * G + h] == -CUDART_INF_F ? 0.f : exp2f(merge_m[w * G + h] - M);
+            merge_w[w * G + h] = e;
+            L += merge_l[w * G + h] * e;
+        }
+        float post = 1.f / L;
+        if constexpr (!TS) post *= __ldg(p.v_scale + kvh);
+        for (int w = 0; w < NW; ++w) merge_w[w * G + h] *= post;
+        if (!single) {
+            float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * 2;
+            ml[0] = M;
+            ml[1] = L;
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < G * D; idx += T::kThreads) {
+        const int h = idx / D;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) acc = fmaf(merge_acc[(w * G + h) * D + (idx % D)], merge_w[w * G + h], acc);
+        if (single) {
+            p.out[((long long)seq * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(acc);
+        } else {
+            p.part_o[(((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * D + (idx % D)] = acc;
+        }
+    }
+}
+
+// The E4M3 pool as a 2-D tensor of 128-byte rows (one (block, KV head, slot)
+// row each); boxes of 128 bytes x box_rows rows, 128-byte swizzle.
+inline bool make_e4m3_pool_map(CUtensorMap *map, const void *pool, long long rows, int box_rows) {
+    tc::EncodeTiledFn fn = tc::encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(pool), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace pkv

@@ -53,6 +53,20 @@ def test_lengths_at_block_and_tile_boundaries(bs):
         check_workload(wl, partition_request=split)
 
 
+@pytest.mark.parametrize("bs", [8, 16, 32, 256])
+def test_fp8_lengths_at_group_and_tile_boundaries(bs):
+    """E4M3 cache, head_dim 128 (the warp-MMA kernel): lengths around its
+    16-token groups, 32-token warp slices and 128-token tiles, whole and
+    split into 128-token partitions."""
+    lens = sorted({1, 2, 15, 16, 17, 31, 32, 33, 47, 63, 64, 65, 95, 96, 97, 127, 128, 129, 255, 256, 257,
+                   bs - 1, bs, bs + 1} - {0})
+    c = cfg(num_seqs=len(lens), num_q_heads=8, num_kv_heads=2, block_size=bs, ctx_lo=1, ctx_hi=max(lens),
+            cache_dtype=W.CACHE_FP8)
+    wl = _with_lengths(c, W.generate(c, 12), lens)
+    for split in (-1, 128):
+        check_workload(wl, partition_request=split)
+
+
 def _with_lengths(c, wl, lens):
     """A workload of the same pool with given lengths (rows re-drawn)."""
     g = torch.Generator().manual_seed(99)

@@ -92,6 +92,28 @@ def test_zero_and_outlier_rows():
     compare(out, ref, True, "edge rows")
 
 
+@pytest.mark.parametrize("rising", [True, False])
+def test_v_scales_spanning_many_powers_of_two(rising):
+    """V rows whose magnitudes (and so per-token scales) change by 2^17 along
+    each sequence: rising, every few tiles brings a larger V scale (the
+    kernel rescales its accumulators); falling, later weights times their V
+    scale are tiny against the first ones."""
+    cfg = W.DecodeConfig("tok_range", 4, 32, 8, 128, 16, 600, 1400, cache_dtype=W.CACHE_FP8_TOKEN)
+    wl = W.generate(cfg, 4)
+    rows = torch.zeros(wl.k_hist.shape[0], dtype=torch.float32)
+    for r in wl.hist_rows:
+        n = len(r)
+        k = torch.linspace(-16, 1, n) if rising else torch.linspace(1, -16, n)
+        rows[r] = torch.exp2(torch.floor(k))
+    wl.v_hist = (wl.v_hist.float() * rows[:, None, None]).to(torch.bfloat16)
+    out, (kp, vp, ks, vs), st = run_decode(wl)
+    assert st == K.PKV_OK
+    ref, rkp, rvp, rst, rks, rvs = O.run_workload(wl, num_threads=THREADS)
+    assert rst == O.ORC_OK
+    assert np.array_equal(scale_bits(vs), scale_bits(rvs))
+    compare(out, ref, True, "v scale range")
+
+
 def test_long_fp8_token_sampled():
     """The full-size split-K step with per-token scales; 16+ sequences checked,
     among them lengths on partition edges (k * P, k * P + 1, k * P - 1)."""
