@@ -114,6 +114,43 @@ PKV_API int pkv_store_kvcache(const void *k, const void *v, void *k_cache, void 
                       float *k_scale, float *v_scale, int *dev_err, void *stream);
 
 /*
+ * store_kvcache_rope: the rotary position embedding of q and k fused with
+ * store_kvcache. The FP8 cache of "nano-vllm-lite：深入理解LLM推理机制的教育级开
+ * 源项目" (section 核心技术改进 3) holds rotated keys, so the rotation that
+ * precedes the write is done in the same pass. The rotation is the RoFormer
+ * paper's (Su et al., 2021): pair i of a row at position m = positions[t]
+ * turns by the angle whose cosine and sine are cos_sin[m][i] and
+ * cos_sin[m][head_dim/2 + i]; the caller builds the table once
+ * (theta_i = base^(-2i/head_dim) in the paper). For every element pair, in
+ * binary32 with one rounding per step and then bf16 round-to-nearest-even:
+ *   x' = fma(-y, sin, x * cos),  y' = fma(x, sin, y * cos)
+ * Pairs are (i, i + head_dim/2) for rope_style 0 and (2i, 2i + 1) for
+ * rope_style 1. The result is exactly store_kvcache of the rotated k (bf16)
+ * and of v, and q_out = the rotated q.
+ *
+ *  q, q_out      [num_tokens][num_q_heads][head_dim] bf16, or both NULL (keys
+ *                only); q_out may be q (in place)
+ *  k, v          [num_tokens][num_kv_heads][head_dim] bf16
+ *  positions     [num_tokens] int32, each in [0, max_position)
+ *  cos_sin       [max_position][head_dim] fp32 (cos of the head_dim/2 angles,
+ *                then their sin), 16-byte aligned
+ *  other arguments as pkv_store_kvcache
+ *
+ * Host checks: as pkv_store_kvcache, plus head_dim a multiple of 16 with
+ * head_dim / 16 a power of two (16 .. 512), rope_style 0 or 1, q and q_out
+ * both given or both NULL, max_position >= 1. Device checks: a position
+ * outside [0, max_position) sets PKV_DEVERR_BOUNDS and nothing of that token
+ * is written (neither q_out nor the cache); slots as in pkv_store_kvcache
+ * (slot -1 skips the cache write but q is still rotated).
+ */
+PKV_API int pkv_store_kvcache_rope(const void *q, void *q_out, const void *k, const void *v, void *k_cache,
+                                   void *v_cache, const int32_t *slot_mapping, const int32_t *positions,
+                                   const float *cos_sin, int max_position, int rope_style, int num_tokens,
+                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                   int64_t num_blocks, int cache_dtype, float *k_scale, float *v_scale,
+                                   int *dev_err, void *stream);
+
+/*
  * Split-K plan of a decode call. A sequence's tokens are cut into partitions
  * of partition_tokens logical tokens; each partition is one thread block per
  * KV head, and a reduce kernel merges the partials (flash-decoding). When

@@ -66,6 +66,12 @@ def _bind(lib):
     lib.orc_fused_add_rmsnorm.argtypes = [c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_int, c.c_double,
                                           c.c_void_p, c.c_void_p, c.c_int]
     lib.orc_fused_add_rmsnorm.restype = c.c_int
+    lib.orc_rope.argtypes = [c.c_void_p] * 3 + [c.c_int64, c.c_int, c.c_int, c.c_void_p, c.c_int64, c.c_int]
+    lib.orc_rope.restype = c.c_int
+    lib.orc_store_kvcache_rope.argtypes = ([c.c_void_p] * 8 + [c.c_int64, c.c_int, c.c_int, c.c_int, c.c_int,
+                                                                c.c_int64, c.c_int, c.c_void_p, c.c_void_p,
+                                                                c.c_void_p, c.c_int64, c.c_int])
+    lib.orc_store_kvcache_rope.restype = c.c_int
     return lib
 
 
@@ -191,6 +197,48 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, contex
                                          T, nq, num_kv_heads, d, block_size, nblk, float(scale), int(fp8), _p(ks),
                                          _p(vs), _p(out), int(num_threads))
     return out, st
+
+
+def rope(x, positions, cos_sin, style=0, lib=None):
+    """bf16 rows ``[N, heads, d]`` rotated at ``positions`` with the binary32
+    table ``cos_sin [max_position, d]`` (cos of the d/2 angles, then sin).
+    Returns ``(out uint16 [N, heads, d], status)``; rows with an out-of-range
+    position stay zero."""
+    lib = lib or load()
+    x = _np(x, np.uint16)
+    pos = _np(positions, np.int32)
+    cs = _np(cos_sin, np.float32)
+    N, H, d = x.shape
+    out = np.zeros_like(x)
+    st = lib.orc_rope(_p(x), _p(out), _p(pos), N, H, d, _p(cs), cs.shape[0], int(style))
+    return out, st
+
+
+def store_kvcache_rope(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin, num_blocks, block_size,
+                       k_scale=None, v_scale=None, style=0, lib=None):
+    """orc_rope of q and k, then orc_store_kvcache of the rotated k and of v
+    into the host pools (in place). ``q`` may be None. Returns
+    ``(q_out uint16 or None, status)``."""
+    lib = lib or load()
+    k = _np(k, np.uint16)
+    v = _np(v, np.uint16)
+    sm = _np(slot_mapping, np.int32)
+    pos = _np(positions, np.int32)
+    cs = _np(cos_sin, np.float32)
+    N, nkv, d = k.shape
+    mode = fp8_mode(k_cache, k_scale)
+    if mode == 2:
+        ks, vs = k_scale, v_scale
+    else:
+        ks = _np(k_scale, np.float32) if mode else None
+        vs = _np(v_scale, np.float32) if mode else None
+    qn = _np(q, np.uint16) if q is not None else None
+    q_out = np.zeros_like(qn) if qn is not None else None
+    nq = qn.shape[1] if qn is not None else 0
+    st = lib.orc_store_kvcache_rope(_p(qn), _p(q_out), _p(k), _p(v), _p(k_cache), _p(v_cache), _p(sm), _p(pos), N,
+                                    nq, nkv, d, block_size, num_blocks, mode, _p(ks), _p(vs), _p(cs), cs.shape[0],
+                                    int(style))
+    return q_out, st
 
 
 def e4m3_from_float(y: float, lib=None) -> int:

@@ -46,6 +46,10 @@
  *    the residual add and the RMSNorm that follows it, fused): h = x + r,
  *    the residual stream continues as h, and the normalised output is
  *    w * h / sqrt(mean(h^2) + eps) over the hidden dimension.
+ *  - Rotary position embedding of q and k before the store (orc_rope,
+ *    orc_store_kvcache_rope; readings next to them): the rotation of the
+ *    RoFormer paper, from a caller-built cos/sin table, in binary32 with a
+ *    fixed operation order because its result is rounded to bf16.
  *  - Chunked prefill ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目",
  *    section 核心技术改进 2 "Chunked Prefill": a long prompt's prefill is cut
  *    into chunks that run interleaved with decode work): a chunk of c new
@@ -485,4 +489,126 @@ int orc_fused_add_rmsnorm(const uint16_t *x, const uint16_t *residual, const uin
         }
     }
     return ORC_OK;
+}
+
+/*
+ * Rotary position embedding (Su, Lu, Pan, Murtadha, Wen, Liu, "RoFormer:
+ * Enhanced Transformer with Rotary Position Embedding", 2021): a head vector
+ * of head_dim elements is cut into head_dim / 2 coordinate pairs, and pair i
+ * of a token at position m is rotated by the angle m * theta_i,
+ *     (x, y) -> (x cos - y sin, x sin + y cos).
+ * The pages name the FP8 cache that the rotated keys are stored into
+ * ("nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section 核心技术改进 3)
+ * but give no formula for the rotation; these readings are taken:
+ *  - the angles come from a table the caller builds once, cos_sin[m] =
+ *    cos(m theta_0 .. m theta_{d/2-1}) then sin(...), binary32, for
+ *    positions 0 .. max_position - 1 (theta_i = base^(-2i/d) in the paper);
+ *  - pair i is (i, i + d/2) for style 0 (the halves of the vector) and
+ *    (2i, 2i + 1) for style 1 (neighbours, as the paper writes it);
+ *  - the rotated value is rounded to bf16 (the cache and q are bf16), so the
+ *    arithmetic that decides the bf16 bits is fixed, in binary32, one
+ *    rounding per step: x' = fma(-y, sin, x * cos), y' = fma(x, sin, y * cos)
+ *    (fmaf is correctly rounded), then round to nearest even.
+ * A position outside [0, max_position) leaves the row unwritten and the call
+ * reports ORC_ERR_BOUNDS.
+ */
+static void pair_index(int i, int head_dim, int style, int *a, int *b)
+{
+    if (style == 1) {
+        *a = 2 * i;
+        *b = 2 * i + 1;
+    } else {
+        *a = i;
+        *b = i + head_dim / 2;
+    }
+}
+
+int orc_rope(const uint16_t *x, uint16_t *out, const int32_t *positions, int64_t num_tokens, int num_heads,
+             int head_dim, const float *cos_sin, int64_t max_position, int style)
+{
+    int status = ORC_OK;
+    int64_t t;
+    if (!x || !out || !positions || !cos_sin || num_tokens < 0 || num_heads < 1 || head_dim < 2 ||
+        head_dim % 2 != 0 || max_position < 1 || (style != 0 && style != 1))
+        return ORC_ERR_ARG;
+    for (t = 0; t < num_tokens; ++t) {
+        int64_t m = positions[t];
+        int h, i;
+        if (m < 0 || m >= max_position) {
+            status = ORC_ERR_BOUNDS;
+            continue;
+        }
+        for (h = 0; h < num_heads; ++h) {
+            const uint16_t *row = x + (t * num_heads + h) * (int64_t)head_dim;
+            uint16_t *dst = out + (t * num_heads + h) * (int64_t)head_dim;
+            for (i = 0; i < head_dim / 2; ++i) {
+                int a, b;
+                float xa, xb, c, s, ya, yb;
+                pair_index(i, head_dim, style, &a, &b);
+                xa = (float)orc_bf16_to_double(row[a]);
+                xb = (float)orc_bf16_to_double(row[b]);
+                c = cos_sin[m * head_dim + i];
+                s = cos_sin[m * head_dim + head_dim / 2 + i];
+                ya = fmaf(-xb, s, xa * c);
+                yb = fmaf(xa, s, xb * c);
+                dst[a] = orc_bf16_from_double((double)ya);
+                dst[b] = orc_bf16_from_double((double)yb);
+            }
+        }
+    }
+    return status;
+}
+
+/*
+ * store_kvcache_rope: q (if given) and k rotated at each token's position,
+ * then k (rotated) and v (as is) stored exactly as orc_store_kvcache does --
+ * the composition of the two steps, fused on the GPU. A token whose position
+ * is out of range is neither rotated nor stored (ORC_ERR_BOUNDS).
+ */
+int orc_store_kvcache_rope(const uint16_t *q, uint16_t *q_out, const uint16_t *k, const uint16_t *v,
+                           void *k_cache, void *v_cache, const int32_t *slot_mapping, const int32_t *positions,
+                           int64_t num_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int64_t num_blocks, int fp8, float *k_scale, float *v_scale, const float *cos_sin,
+                           int64_t max_position, int style)
+{
+    int status = ORC_OK, st;
+    int64_t t;
+    uint16_t *k_rot;
+    int32_t *slots;
+    if (!k || !v || !slot_mapping || !positions || num_tokens < 0 || (q && !q_out) || (q && num_q_heads < 1))
+        return ORC_ERR_ARG;
+    if (num_tokens == 0)
+        return ORC_OK;
+    k_rot = (uint16_t *)calloc((size_t)num_tokens * num_kv_heads * head_dim, sizeof(uint16_t));
+    slots = (int32_t *)malloc((size_t)num_tokens * sizeof(int32_t));
+    if (!k_rot || !slots) {
+        free(k_rot);
+        free(slots);
+        return ORC_ERR_ARG;
+    }
+    if (q) {
+        st = orc_rope(q, q_out, positions, num_tokens, num_q_heads, head_dim, cos_sin, max_position, style);
+        if (st == ORC_ERR_ARG) {
+            free(k_rot);
+            free(slots);
+            return st;
+        }
+    }
+    st = orc_rope(k, k_rot, positions, num_tokens, num_kv_heads, head_dim, cos_sin, max_position, style);
+    if (st == ORC_ERR_ARG) {
+        free(k_rot);
+        free(slots);
+        return st;
+    }
+    for (t = 0; t < num_tokens; ++t) {
+        int bad = positions[t] < 0 || positions[t] >= max_position;
+        if (bad)
+            status = ORC_ERR_BOUNDS;
+        slots[t] = bad ? -1 : slot_mapping[t];
+    }
+    st = orc_store_kvcache(k_rot, v, k_cache, v_cache, slots, num_tokens, num_kv_heads, head_dim, block_size,
+                           num_blocks, fp8, k_scale, v_scale);
+    free(k_rot);
+    free(slots);
+    return st != ORC_OK ? st : status;
 }

@@ -137,6 +137,34 @@ int pkv_store_kvcache(const void *k, const void *v, void *k_cache, void *v_cache
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+int pkv_store_kvcache_rope(const void *q, void *q_out, const void *k, const void *v, void *k_cache, void *v_cache,
+                           const int32_t *slot_mapping, const int32_t *positions, const float *cos_sin,
+                           int max_position, int rope_style, int num_tokens, int num_q_heads, int num_kv_heads,
+                           int head_dim, int block_size, int64_t num_blocks, int cache_dtype, float *k_scale,
+                           float *v_scale, int *dev_err, void *stream) {
+    if (num_tokens < 0 || num_kv_heads < 1 || head_dim < 16 || head_dim % 16 != 0 || block_size < 1 ||
+        num_blocks < 1 || max_position < 1 || (rope_style != 0 && rope_style != 1))
+        return PKV_ERR_INVALID_ARG;
+    if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
+    // a row spans head_dim / 16 adjacent lanes (a power of two up to 32)
+    if (!pow2(head_dim / 16) || head_dim > 512) return PKV_ERR_UNSUPPORTED;
+    if ((q == nullptr) != (q_out == nullptr)) return PKV_ERR_INVALID_ARG;
+    if (q && num_q_heads < 1) return PKV_ERR_INVALID_ARG;
+    const bool fp8 = cache_dtype != PKV_CACHE_BF16;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping || !positions || !cos_sin) return PKV_ERR_INVALID_ARG;
+    if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(cos_sin) ||
+        (q && (!aligned16(q) || !aligned16(q_out))))
+        return PKV_ERR_INVALID_ARG;
+    cudaError_t e = pkv::launch_store_kvcache_rope(q, q_out, k, v, k_cache, v_cache, slot_mapping, positions,
+                                                   cos_sin, max_position, rope_style, num_tokens, num_q_heads,
+                                                   num_kv_heads, head_dim, block_size, num_blocks, cache_dtype,
+                                                   k_scale, v_scale, dev_err, num_sms(),
+                                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 int pkv_plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                     int max_context_len, int cache_dtype, int partition_request, pkv_decode_plan *plan) {
     if (!plan) return PKV_ERR_INVALID_ARG;

@@ -12,6 +12,13 @@ cudaError_t launch_store_kvcache(const void *k, const void *v, void *k_cache, vo
                                  int block_size, int64_t num_blocks, int mode, float *k_scale, float *v_scale,
                                  int *dev_err, int num_sms, cudaStream_t stream);
 
+cudaError_t launch_store_kvcache_rope(const void *q, void *q_out, const void *k, const void *v, void *k_cache,
+                                      void *v_cache, const int32_t *slot_mapping, const int32_t *positions,
+                                      const float *cos_sin, int max_position, int style, int num_tokens,
+                                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                      int64_t num_blocks, int mode, float *k_scale, float *v_scale, int *dev_err,
+                                      int num_sms, cudaStream_t stream);
+
 // Everything the decode kernels need, resolved by the host layer.
 struct DecodeArgs {
     const void *q;

@@ -8,6 +8,7 @@ path: if ``libpagedkv.so`` is missing or cannot load, ``lib()`` raises.
 The functions mirror ``include/pagedkv.h``:
 
 * ``store_kvcache`` -- ``pkv_store_kvcache``
+* ``store_kvcache_rope`` -- ``pkv_store_kvcache_rope``
 * ``plan_decode`` -- ``pkv_plan_decode``
 * ``decode_workspace_bytes`` -- ``pkv_decode_workspace_bytes``
 * ``paged_attention_decode`` -- ``pkv_paged_attention_decode``
@@ -38,7 +39,7 @@ PKV_CACHE_BF16 = 0
 PKV_CACHE_FP8_E4M3 = 1  # k_scale / v_scale: [num_kv_heads] fp32
 PKV_CACHE_FP8_E4M3_TOKEN = 2  # k_scale / v_scale: scale pools [num_blocks, num_kv_heads, block_size] fp32
 
-EXPORTED = ("pkv_store_kvcache", "pkv_plan_decode", "pkv_decode_workspace_bytes", "pkv_paged_attention_decode", "pkv_status_string",
+EXPORTED = ("pkv_store_kvcache", "pkv_store_kvcache_rope", "pkv_plan_decode", "pkv_decode_workspace_bytes", "pkv_paged_attention_decode", "pkv_status_string",
             "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
             "pkv_paged_attention_prefill", "pkv_fused_add_rmsnorm")
 
@@ -77,6 +78,8 @@ def load_library(path: str):
     vp, i32, i64, f32, sz = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
     L.pkv_store_kvcache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, vp, vp, vp, vp]
     L.pkv_store_kvcache.restype = i32
+    L.pkv_store_kvcache_rope.argtypes = [vp] * 9 + [i32] * 7 + [i64, i32, vp, vp, vp, vp]
+    L.pkv_store_kvcache_rope.restype = i32
     L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
     L.pkv_plan_decode.restype = i32
     L.pkv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
@@ -153,6 +156,41 @@ def store_kvcache(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=No
                                  nblk, _cache_dtype(k_cache, k_scale), _ptr(k_scale), _ptr(v_scale), _ptr(dev_err),
                                  _stream(stream))
     _check(st, "pkv_store_kvcache")
+
+
+def store_kvcache_rope(k, v, k_cache, v_cache, slot_mapping, positions, cos_sin, q=None, q_out=None, style=0,
+                       k_scale=None, v_scale=None, dev_err=None, stream=None):
+    """Rotate k (and q into ``q_out``) at ``positions`` with the fp32 table
+    ``cos_sin [max_position, d]``, then store the rotated k and v like
+    ``store_kvcache``. Returns ``q_out`` (allocated when q is given without it)."""
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("k and v must be bfloat16")
+    if slot_mapping.dtype != torch.int32 or positions.dtype != torch.int32:
+        raise TypeError("slot_mapping and positions must be int32")
+    if cos_sin.dtype != torch.float32 or cos_sin.dim() != 2 or not cos_sin.is_contiguous():
+        raise TypeError("cos_sin must be a contiguous fp32 [max_position, head_dim] table")
+    for t in (k, v, k_cache, v_cache):
+        if not t.is_contiguous():
+            raise ValueError("k, v and the pools must be contiguous")
+    N, nkv, d = k.shape
+    nblk, nkv2, bs, d2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or nkv2 != nkv or d2 != d:
+        raise ValueError("shape mismatch between k/v and the pools")
+    if slot_mapping.numel() != N or positions.numel() != N or cos_sin.shape[1] != d:
+        raise ValueError("slot_mapping / positions / cos_sin do not match k")
+    nq = 0
+    if q is not None:
+        if q.dtype != torch.bfloat16 or not q.is_contiguous() or q.shape[0] != N or q.shape[2] != d:
+            raise ValueError("q must be contiguous bf16 [N, nq, head_dim]")
+        nq = q.shape[1]
+        if q_out is None:
+            q_out = torch.empty_like(q)
+    st = lib().pkv_store_kvcache_rope(_ptr(q), _ptr(q_out), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(slot_mapping), _ptr(positions), _ptr(cos_sin), cos_sin.shape[0], style, N,
+                                      nq, nkv, d, bs, nblk, _cache_dtype(k_cache, k_scale), _ptr(k_scale),
+                                      _ptr(v_scale), _ptr(dev_err), _stream(stream))
+    _check(st, "pkv_store_kvcache_rope")
+    return q_out
 
 
 def plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, fp8=False,

@@ -552,3 +552,112 @@ def generate_norm(cfg: NormConfig, seed: int = 0, device: str | torch.device = "
     r = _randn_bf16((cfg.num_tokens, cfg.hidden), g, device) if cfg.residual else None
     w = (1.0 + 0.1 * torch.randn(cfg.hidden, generator=g, device=device)).to(torch.bfloat16)
     return NormWorkload(cfg, seed, x, r, w)
+
+
+# ------------------------------------------------- rotary embedding + store
+#
+# The rotary position embedding of q and k that precedes the cache write
+# (the FP8 cache of "nano-vllm-lite：深入理解LLM推理机制的教育级开源项目", section
+# 核心技术改进 3, stores the rotated keys). The rotation itself is the RoFormer
+# paper's (Su et al., 2021); an engine builds its cos/sin table once.
+
+ROPE_HALF = 0  # pairs (i, i + d/2)
+ROPE_INTERLEAVED = 1  # pairs (2i, 2i + 1)
+
+
+def rope_cache(max_position: int, head_dim: int, base: float = 1_000_000.0, device="cpu") -> torch.Tensor:
+    """The table a rotary embedding reads: row m holds cos(m theta_i) for
+    i < head_dim / 2, then sin(m theta_i), theta_i = base^(-2i / head_dim),
+    evaluated in fp64 and stored as fp32 ``[max_position, head_dim]``."""
+    i = torch.arange(head_dim // 2, dtype=torch.float64)
+    theta = base ** (-2.0 * i / head_dim)
+    ang = torch.arange(max_position, dtype=torch.float64)[:, None] * theta[None, :]
+    return torch.cat([torch.cos(ang), torch.sin(ang)], dim=1).to(torch.float32).contiguous().to(device)
+
+
+@dataclass(frozen=True)
+class RopeConfig:
+    """One step of rotary embedding + store: num_tokens new tokens (one per
+    sequence at decode, or the tokens of prefill chunks) at positions below
+    max_position, written into distinct slots of a pool."""
+
+    name: str
+    num_tokens: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    max_position: int
+    style: int = ROPE_HALF
+    cache_dtype: str = CACHE_BF16
+    base: float = 1_000_000.0
+    pool_blocks: int | None = None  # None: enough for every token, plus 10 %
+
+    @property
+    def is_fp8(self) -> bool:
+        return self.cache_dtype in (CACHE_FP8, CACHE_FP8_TOKEN)
+
+    @property
+    def token_scales(self) -> bool:
+        return self.cache_dtype == CACHE_FP8_TOKEN
+
+    def with_(self, **kw) -> "RopeConfig":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return RopeConfig(**d)
+
+
+ROPE_CONFIGS: dict[str, RopeConfig] = {
+    c.name: c
+    for c in (
+        RopeConfig("rope_tiny", 4, 2, 1, 64, 16, 300),
+        # one decode step of the Qwen3-8B-shaped layer: 1024 sequences at positions below 2048
+        RopeConfig("rope_qwen3_8b", 1024, 32, 8, 128, 256, 2048),
+        RopeConfig("rope_qwen3_8b_fp8", 1024, 32, 8, 128, 256, 2048, cache_dtype=CACHE_FP8_TOKEN),
+        # a chunked-prefill step of 16 x 512 tokens (inputs and cache writes above L2 in total)
+        RopeConfig("rope_prefill_qwen3_8b", 8192, 32, 8, 128, 256, 32768),
+        RopeConfig("rope_prefill_qwen3_8b_fp8", 8192, 32, 8, 128, 256, 32768, cache_dtype=CACHE_FP8_TOKEN),
+    )
+}
+
+
+@dataclass
+class RopeWorkload:
+    cfg: RopeConfig
+    seed: int
+    num_blocks: int
+    q: torch.Tensor  # [N, nq, d] bf16
+    k: torch.Tensor  # [N, nkv, d] bf16
+    v: torch.Tensor
+    positions: torch.Tensor  # [N] int32
+    slot_mapping: torch.Tensor  # [N] int32, distinct slots
+    cos_sin: torch.Tensor  # [max_position, d] fp32
+    k_scale: torch.Tensor | None = None  # [nkv] fp32 (one scale per KV head)
+    v_scale: torch.Tensor | None = None
+
+
+def generate_rope(cfg: RopeConfig, seed: int = 0, device: str | torch.device = "cpu") -> RopeWorkload:
+    """Positions uniform in [0, max_position); slots distinct, from a seeded
+    permutation of the pool; q/k/v N(0, 1) rounded to bf16."""
+    device = torch.device(device)
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    N, bs = cfg.num_tokens, cfg.block_size
+    need = -(-N // bs)
+    nblk = cfg.pool_blocks if cfg.pool_blocks is not None else need + -(-need // 10) + 1
+    positions = torch.randint(0, cfg.max_position, (N,), generator=g, dtype=torch.int64)
+    slots = torch.randperm(nblk * bs, generator=g)[:N]
+    gd = torch.Generator(device=device).manual_seed(seed + 1)
+    q = _randn_bf16((N, cfg.num_q_heads, cfg.head_dim), gd, device)
+    k = _randn_bf16((N, cfg.num_kv_heads, cfg.head_dim), gd, device)
+    v = _randn_bf16((N, cfg.num_kv_heads, cfg.head_dim), gd, device)
+    wl = RopeWorkload(cfg, seed, nblk, q, k, v, positions.to(torch.int32).to(device),
+                      slots.to(torch.int32).to(device), rope_cache(cfg.max_position, cfg.head_dim, cfg.base, device))
+    if cfg.cache_dtype == CACHE_FP8:
+        # one scale per KV head over the rows as drawn: rotation keeps each
+        # pair's norm, so |rotated| <= sqrt(2) * amax; the scale leaves room
+        one = torch.ones(cfg.num_kv_heads, dtype=torch.float32, device=device)
+        km = k.float().abs().amax(dim=(0, 2)) if N else one
+        vm = v.float().abs().amax(dim=(0, 2)) if N else one
+        wl.k_scale = torch.where(km > 0, km, one) * 1.5 / 448.0
+        wl.v_scale = torch.where(vm > 0, vm, one) / 448.0
+    return wl

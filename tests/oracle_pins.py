@@ -629,7 +629,171 @@ def pin_rmsnorm_closed_forms(lib):
     assert np.array_equal(o1, o3), "a zero residual is no residual"
 
 
+# ------------------------------------------------ rotary embedding + store
+# The rotation of the RoFormer paper (Su et al., 2021): pair i of a token at
+# position m turns by m * theta_i, theta_i = base^(-2i/d). The references
+# below recompute the angles from that definition in fp64, independently of
+# the fp32 table the oracle reads.
+
+
+def _rope_pairs(d, style):
+    i = np.arange(d // 2)
+    return (2 * i, 2 * i + 1) if style == W.ROPE_INTERLEAVED else (i, i + d // 2)
+
+
+def rope_fp64(x_bf16, positions, d, base, style):
+    """fp64 rotation of bf16 rows [N, H, d] from the definition."""
+    x = x_bf16.float().double().numpy()
+    m = positions.long().numpy().astype(np.float64)[:, None, None]
+    i = np.arange(d // 2, dtype=np.float64)
+    ang = m * base ** (-2.0 * i / d)[None, None, :]
+    a, b = _rope_pairs(d, style)
+    out = np.empty_like(x)
+    out[..., a] = x[..., a] * np.cos(ang) - x[..., b] * np.sin(ang)
+    out[..., b] = x[..., a] * np.sin(ang) + x[..., b] * np.cos(ang)
+    return out
+
+
+def _bf16_bits_to_f64(u16):
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def rcfg(**kw) -> W.RopeConfig:
+    base = dict(name="rope", num_tokens=7, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16,
+                max_position=5000)
+    base.update(kw)
+    return W.RopeConfig(**base)
+
+
+def pin_rope_position_zero_is_identity(lib):
+    for style in (W.ROPE_HALF, W.ROPE_INTERLEAVED):
+        wl = W.generate_rope(rcfg(style=style), 31)
+        pos = torch.zeros_like(wl.positions)
+        out, st = O.rope(wl.k, pos, wl.cos_sin, style, lib=lib)
+        assert st == O.ORC_OK and np.array_equal(out, wl.k.view(torch.int16).numpy().view(np.uint16)), \
+            "position 0 must leave every element unchanged"
+
+
+def pin_rope_fp64_rotation(lib):
+    """Within one bf16 rounding (plus binary32 slack) of the fp64 rotation,
+    for both pairings, head sizes 64 and 128, positions up to 32767."""
+    for style in (W.ROPE_HALF, W.ROPE_INTERLEAVED):
+        for d, mp, base in ((64, 5000, 10000.0), (128, 32768, 1_000_000.0)):
+            wl = W.generate_rope(rcfg(style=style, head_dim=d, max_position=mp, base=base, num_tokens=40), 32)
+            out, st = O.rope(wl.q, wl.positions, wl.cos_sin, style, lib=lib)
+            assert st == O.ORC_OK
+            got = _bf16_bits_to_f64(out)
+            ref = rope_fp64(wl.q, wl.positions, d, base, style)
+            x = wl.q.float().double().numpy()
+            a, b = _rope_pairs(d, style)
+            pair = np.abs(x[..., a]) + np.abs(x[..., b])  # binary32 slack scales with the pair's size
+            slack_full = np.empty_like(x)
+            slack_full[..., a] = pair
+            slack_full[..., b] = pair
+            err = np.abs(got - ref)
+            assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -18 * slack_full + 1e-30), \
+                f"style {style} d {d}: max err {err.max():.3e}"
+
+
+def pin_rope_styles_are_a_permutation(lib):
+    """The two pairings are the same rotation on permuted coordinates: moving
+    element i + d/2 next to element i turns the half pairing into the
+    neighbour pairing, bit for bit."""
+    d = 128
+    wl = W.generate_rope(rcfg(head_dim=d, num_tokens=20), 33)
+    perm = np.empty(d, dtype=np.int64)
+    perm[0::2] = np.arange(d // 2)
+    perm[1::2] = np.arange(d // 2) + d // 2
+    half, st1 = O.rope(wl.k, wl.positions, wl.cos_sin, W.ROPE_HALF, lib=lib)
+    inter, st2 = O.rope(wl.k[..., torch.from_numpy(perm)].contiguous(), wl.positions, wl.cos_sin,
+                        W.ROPE_INTERLEAVED, lib=lib)
+    assert st1 == st2 == O.ORC_OK
+    assert np.array_equal(half[..., perm], inter), "pairings differ by more than a permutation"
+
+
+def pin_rope_relative_positions(lib):
+    """<R_m q, R_n k> depends only on n - m: it equals <q, R_{n-m} k>
+    evaluated in fp64 from the definition (within bf16 rounding)."""
+    d, base = 128, 10000.0
+    for style in (W.ROPE_HALF, W.ROPE_INTERLEAVED):
+        wl = W.generate_rope(rcfg(head_dim=d, base=base, style=style, num_tokens=24, num_q_heads=2,
+                                  num_kv_heads=2), 34)
+        pos_q = wl.positions
+        pos_k = torch.flip(wl.positions, [0])
+        rq, st1 = O.rope(wl.q, pos_q, wl.cos_sin, style, lib=lib)
+        rk, st2 = O.rope(wl.k, pos_k, wl.cos_sin, style, lib=lib)
+        assert st1 == st2 == O.ORC_OK
+        dots = (_bf16_bits_to_f64(rq) * _bf16_bits_to_f64(rk)).sum(-1)
+        rel = rope_fp64(wl.k, pos_k - pos_q, d, base, style)  # R_{n-m} k (negative angles allowed)
+        ref = (wl.q.float().double().numpy() * rel).sum(-1)
+        nq = np.linalg.norm(wl.q.float().double().numpy(), axis=-1)
+        nk = np.linalg.norm(wl.k.float().double().numpy(), axis=-1)
+        assert np.all(np.abs(dots - ref) <= 2.0 ** -7 * nq * nk), np.abs(dots - ref).max()
+
+
+def pin_rope_bounds(lib):
+    wl = W.generate_rope(rcfg(max_position=100), 35)
+    pos = wl.positions.clone() % 100
+    pos[1] = -1
+    pos[3] = 100
+    out, st = O.rope(wl.k, pos, wl.cos_sin[:100], W.ROPE_HALF, lib=lib)
+    assert st == O.ORC_ERR_BOUNDS
+    assert not out[1].any() and not out[3].any(), "rows with a bad position must stay unwritten"
+    good, st2 = O.rope(wl.k[[0, 2]], pos[[0, 2]], wl.cos_sin[:100], W.ROPE_HALF, lib=lib)
+    assert st2 == O.ORC_OK and np.array_equal(out[[0, 2]], good)
+
+
+def pin_store_rope_is_rope_then_store(lib):
+    """The fused call equals rope of q and k followed by the plain store, for
+    every cache type; a bad position stores nothing, slot -1 is skipped."""
+    for dt in (W.CACHE_BF16, W.CACHE_FP8, W.CACHE_FP8_TOKEN):
+        wl = W.generate_rope(rcfg(cache_dtype=dt, num_tokens=9, max_position=64), 36)
+        pos = wl.positions.clone()
+        pos[2] = 64  # out of range
+        slots = wl.slot_mapping.clone()
+        slots[4] = -1
+        nb, bs, nkv, d = wl.num_blocks, wl.cfg.block_size, wl.cfg.num_kv_heads, wl.cfg.head_dim
+        fp8 = dt != W.CACHE_BF16
+        fill = W.CANARY_FP8 if fp8 else W.CANARY_BF16
+        pools = [O.new_pool(nb, nkv, bs, d, fp8, fill) for _ in range(4)]
+        if dt == W.CACHE_FP8_TOKEN:
+            sc = [O.new_scale_pool(nb, nkv, bs) for _ in range(4)]
+        else:
+            sc = [wl.k_scale, wl.v_scale, wl.k_scale, wl.v_scale]
+        q_out, st = O.store_kvcache_rope(wl.q, wl.k, wl.v, pools[0], pools[1], slots, pos, wl.cos_sin, nb, bs,
+                                         sc[0], sc[1], lib=lib)
+        assert st == O.ORC_ERR_BOUNDS
+        rq, _ = O.rope(wl.q, pos, wl.cos_sin, lib=lib)
+        rk, _ = O.rope(wl.k, pos, wl.cos_sin, lib=lib)
+        slots2 = slots.clone()
+        slots2[2] = -1
+        st2 = O.store_kvcache(torch.from_numpy(rk.view(np.int16)).view(torch.bfloat16), wl.v, pools[2], pools[3],
+                              slots2, nb, bs, sc[2], sc[3], lib=lib)
+        assert st2 == O.ORC_OK
+        assert np.array_equal(q_out, rq)
+        assert np.array_equal(pools[0], pools[2]) and np.array_equal(pools[1], pools[3]), dt
+        if dt == W.CACHE_FP8_TOKEN:
+            assert np.array_equal(sc[0], sc[2], equal_nan=True) and np.array_equal(sc[1], sc[3], equal_nan=True)
+
+
+def pin_rope_table(lib):
+    """The workload's table is the definition's cos and sin in binary32."""
+    cs = W.rope_cache(300, 64, 10000.0).double().numpy()
+    i = np.arange(32)
+    for m in (0, 1, 7, 299):
+        ang = m * 10000.0 ** (-2.0 * i / 64)
+        assert np.all(np.abs(cs[m, :32] - np.cos(ang)) <= 2.0 ** -24)
+        assert np.all(np.abs(cs[m, 32:] - np.sin(ang)) <= 2.0 ** -24)
+
+
 ALL_PINS = [
+    pin_rope_position_zero_is_identity,
+    pin_rope_fp64_rotation,
+    pin_rope_styles_are_a_permutation,
+    pin_rope_relative_positions,
+    pin_rope_bounds,
+    pin_store_rope_is_rope_then_store,
+    pin_rope_table,
     pin_rmsnorm_library,
     pin_rmsnorm_residual_is_rounded_sum,
     pin_rmsnorm_closed_forms,

@@ -23,6 +23,15 @@ SRC = os.path.join(os.path.dirname(HERE), "oracle", "pkv_oracle.c")
 
 # (name, original text, mutated text, which occurrence (0-based) to change)
 MUTANTS = [
+    ("rope sin sign", "ya = fmaf(-xb, s, xa * c);", "ya = fmaf(xb, s, xa * c);", 0),
+    ("rope partner", "*b = i + head_dim / 2;", "*b = head_dim - 1 - i;", 0),
+    ("rope cos for sin", "s = cos_sin[m * head_dim + head_dim / 2 + i];", "s = cos_sin[m * head_dim + i];", 0),
+    ("rope angle index", "c = cos_sin[m * head_dim + i];", "c = cos_sin[m * head_dim + head_dim / 2 - 1 - i];", 0),
+    ("rope position off by one", "int64_t m = positions[t];", "int64_t m = positions[t] > 0 ? positions[t] - 1 : 0;",
+     0),
+    ("rope pairings swapped", "if (style == 1) {", "if (style == 0) {", 0),
+    ("rope store unrotated k", "st = orc_store_kvcache(k_rot, v,", "st = orc_store_kvcache(k, v,", 0),
+    ("rope bad position stored", "slots[t] = bad ? -1 : slot_mapping[t];", "slots[t] = slot_mapping[t];", 0),
     ("gqa interleaved", "int g = h / group;", "int g = h % num_kv_heads;", 0),
     ("offset from division", "int off = t % block_size;", "int off = (t / block_size) % block_size;", 0),
     ("block from offset", "int64_t blk = table[t / block_size];", "int64_t blk = table[t % block_size];", 0),
