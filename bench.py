@@ -52,8 +52,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="qwen3_8b",
-                    choices=sorted(W.CONFIGS) + sorted(W.PREFILL_CONFIGS) + sorted(W.NORM_CONFIGS),
-                    help="a decode workload, a chunked-prefill one (prefill_*) or an add + RMSNorm one (norm_*)")
+                    choices=sorted(W.CONFIGS) + sorted(W.PREFILL_CONFIGS) + sorted(W.NORM_CONFIGS) +
+                    sorted(W.ROPE_CONFIGS),
+                    help="a decode workload, a chunked-prefill one (prefill_*), an add + RMSNorm one (norm_*) or a "
+                         "fused RoPE + store one (rope_*)")
     ap.add_argument("--partition", type=int, default=0, help="0 auto, -1 never split, >0 tokens per partition")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--num-seqs", type=int, default=0, help="override the workload's sequence count")
@@ -999,8 +1001,221 @@ def run_norm(args):
     return 0
 
 
+# ------------------------------------------------- rotary embedding + store
+
+ROPE_METRIC = "fused RoPE + store_kvcache tokens/sec and achieved HBM GB/s"
+
+
+def rope_desc(cfg) -> str:
+    style = "half pairs (i, i+d/2)" if cfg.style == W.ROPE_HALF else "neighbour pairs (2i, 2i+1)"
+    return (f"{cfg.name}: {cfg.num_tokens} tokens at positions < {cfg.max_position}, {cfg.num_q_heads}q/"
+            f"{cfg.num_kv_heads}kv heads, head_dim {cfg.head_dim}, block_size {cfg.block_size}, {cfg.cache_dtype} "
+            f"cache, {style}")
+
+
+def rope_bytes(cfg) -> int:
+    """Bytes one launch must move: q in and out, k and v in, the two cache
+    rows out (plus per-token scales), each token's table row, positions and
+    slots."""
+    N, nq, nkv, d = cfg.num_tokens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim
+    es = 1 if cfg.is_fp8 else 2
+    return (N * nq * d * 2 * 2 + N * nkv * d * 2 * 2 + N * nkv * d * es * 2 + (N * nkv * 8 if cfg.token_scales else 0)
+            + N * d * 4 + N * 8)
+
+
+def _rope_pools(wl, device="cuda"):
+    c = wl.cfg
+    shape = (wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)
+    if c.is_fp8:
+        kp = torch.full(shape, W.CANARY_FP8, dtype=torch.uint8, device=device)
+    else:
+        kp = torch.full(shape, W.CANARY_BF16, dtype=torch.int16, device=device).view(torch.bfloat16)
+    vp = kp.clone()
+    if c.token_scales:
+        ks, vs = W.scale_pools(wl.num_blocks, c.num_kv_heads, c.block_size, device=device)
+    else:
+        ks, vs = wl.k_scale, wl.v_scale
+    return kp, vp, ks, vs
+
+
+def rope_cpu_baseline(wl, target_s: float) -> dict:
+    import oracle as O
+
+    threads = cpu_threads()
+    c = wl.cfg
+    q, k, v, pos, sl, cs = (t.cpu() for t in (wl.q, wl.k, wl.v, wl.positions, wl.slot_mapping, wl.cos_sin))
+    ks, vs = wl.k_scale, wl.v_scale
+    hk = O.new_pool(wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim, c.is_fp8, 0)
+    hv = O.new_pool(wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim, c.is_fp8, 0)
+    if c.token_scales:
+        ks = O.new_scale_pool(wl.num_blocks, c.num_kv_heads, c.block_size)
+        vs = O.new_scale_pool(wl.num_blocks, c.num_kv_heads, c.block_size)
+    elif ks is not None:
+        ks, vs = ks.cpu(), vs.cpu()
+
+    def run(n):
+        return O.store_kvcache_rope(q[:n], k[:n], v[:n], hk, hv, sl[:n], pos[:n], cs, wl.num_blocks, c.block_size,
+                                    ks, vs, style=c.style)[1]
+
+    n = max(1, min(c.num_tokens, 64))
+    t0 = time.perf_counter()
+    run(n)
+    dt = time.perf_counter() - t0
+    n2 = int(min(c.num_tokens, max(n, n * target_s / max(dt, 1e-6))))
+    t0 = time.perf_counter()
+    st = run(n2)
+    dt = time.perf_counter() - t0
+    if st != 0:
+        raise RuntimeError(f"the oracle returned status {st} on its sample")
+    return {"value": n2 / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"the first {n2} of {c.num_tokens} tokens, binary32 rotation + store, {dt:.2f} s, "
+                      f"one thread; status {st}"}
+
+
+def run_rope_reference(args):
+    if rank_env()[1] != 0:
+        return 0
+    cfg = W.ROPE_CONFIGS[args.config]
+    wl = W.generate_rope(cfg, args.seed)
+    per_step = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    vals = [rope_cpu_baseline(wl, per_step)["value"] for _ in range(args.warmup + args.steps)][args.warmup:]
+    value = statistics.mean(vals)
+    emit({
+        "impl": "reference", "metric": ROPE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": cfg.num_tokens / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": rope_desc(cfg)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "a bounded prefix of the step's tokens per step, one thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }, args)
+    return 0
+
+
+def run_rope(args):
+    from paged_kv_cache_482_b200 import pagedkv as K
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    cfg = W.ROPE_CONFIGS[args.config]
+    wl = W.generate_rope(cfg, args.seed + rank, device="cuda")
+    kp, vp, ks, vs = _rope_pools(wl)
+    q_out = torch.empty_like(wl.q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(q, k, v, pos, sl):
+        K.store_kvcache_rope(k, v, kp, vp, sl, pos, wl.cos_sin, q=q, q_out=q_out, style=cfg.style, k_scale=ks,
+                             v_scale=vs, dev_err=err)
+
+    args_dev = (wl.q, wl.k, wl.v, wl.positions, wl.slot_mapping)
+    for _ in range(max(3, args.warmup)):
+        step(*args_dev)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())} during warm-up")
+    moved = rope_bytes(cfg)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if moved < (256 << 20) else None
+    stream = torch.cuda.current_stream()
+    sampler = make_sampler(local) if local == 0 else None
+    if sampler:
+        sampler.wait_first()
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kst)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for kk in range(Kst):
+        if flush is not None:
+            flush.zero_()
+        ev[kk][0].record(stream)
+        step(*args_dev)
+        ev[kk][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    times = [ev[kk][0].elapsed_time(ev[kk][1]) for kk in range(Kst)]
+    total_ms, kern_ms = sum(times), statistics.mean(times)
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
+    if sampler:
+        sampler.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())} in the timed steps")
+
+    host_in = [t.cpu().pin_memory() for t in args_dev]
+    dev_in = [torch.empty_like(t) for t in args_dev]
+    host_out = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        step(*dev_in)
+        host_out.copy_(q_out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = x0.elapsed_time(x1)
+    total_ms, kern_ms, e2e_ms = max_over_ranks([total_ms, kern_ms, e2e_ms], dist, device="cuda")
+    if rank == 0:
+        peak, kind = measured_peak()
+        achieved = moved / (kern_ms * 1e-3) / 1e9
+        N = cfg.num_tokens
+        line = {
+            "metric": ROPE_METRIC, "value": world * N * Kst / (total_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": Kst, "warmup": args.warmup, "ms_per_step": total_ms / Kst, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("bf16 in, binary32 rotation, " + ("e4m3" if cfg.is_fp8 else "bf16") + " cache"),
+            "data": "synthetic",
+            "config": {"workload": rope_desc(cfg), "seed": args.seed,
+                       "parallelism": f"replicas x{world} (independent tokens, no collective)",
+                       "l2": ("flushed between steps (256 MB write, untimed)" if flush is not None else
+                              f"no flush: {moved / 1e6:.0f} MB moved per step, above the 126 MB L2")},
+            "kernel_us": kern_ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "kernel": "store_kvcache_rope_kernel",
+                         "peak_source": f"{kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                         "algorithmic_bytes_per_launch": moved,
+                         "bytes_note": "q in/out, k and v in, cache rows (and scales) out, table rows, positions, slots"},
+            "e2e": {"value": world * N * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+            "gpu_launches": Kst,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = rope_cpu_baseline(wl, args.cpu_seconds)
+        emit(line, args)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
+    if args.config in W.ROPE_CONFIGS:
+        return run_rope_reference(args) if args.impl == "reference" else run_rope(args)
     if args.component == "block_manager":
         return run_block_manager(args)
     if args.config in W.NORM_CONFIGS:
