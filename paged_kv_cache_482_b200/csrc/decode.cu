@@ -45,16 +45,20 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-// E4M3 cache, head_dim 128: the warp-MMA kernel (decode_mma.cuh).
-template <int G, bool TS>
+// head_dim 128: the warp-MMA kernel (decode_mma.cuh) for E4M3 and, unless
+// built with PKV_DECODE_BF16_MMA=0, for bf16.
+#ifndef PKV_DECODE_BF16_MMA
+#define PKV_DECODE_BF16_MMA 1
+#endif
+template <int G, bool BF, bool TS>
 cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
-    using T = MmaTraits<G>;
+    using T = MmaTraits<G, BF>;
 #ifdef PKV_MMA_MIN_BLOCKS
     constexpr int MINB = PKV_MMA_MIN_BLOCKS;
 #else
     constexpr int MINB = 3;
 #endif
-    auto kern = paged_decode_mma_kernel<G, MINB, TS>;
+    auto kern = paged_decode_mma_kernel<G, BF, MINB, TS>;
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -75,8 +79,11 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
     CUtensorMap mk, mv;
     std::memset(&mk, 0, sizeof(mk));
     std::memset(&mv, 0, sizeof(mv));
-    if (!make_e4m3_pool_map(&mk, p.k_cache, rows, box_rows) || !make_e4m3_pool_map(&mv, p.v_cache, rows, box_rows))
-        return cudaErrorInvalidValue;
+    const bool mapped = BF ? make_bf16_pool_map(&mk, p.k_cache, rows, box_rows) &&
+                                 make_bf16_pool_map(&mv, p.v_cache, rows, box_rows)
+                           : make_e4m3_pool_map(&mk, p.k_cache, rows, box_rows) &&
+                                 make_e4m3_pool_map(&mv, p.v_cache, rows, box_rows);
+    if (!mapped) return cudaErrorInvalidValue;
     kern<<<(unsigned)blocks, T::kThreads, T::kAlloc, stream>>>(p, mk, mv, box_rows);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.num_partitions <= 1) return e;
@@ -84,23 +91,24 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <bool TS>
+template <bool BF, bool TS>
 cudaError_t launch_mma(int group, const DecodeParams &p, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_mma_one<1, TS>(p, stream);
-        case 2: return launch_mma_one<2, TS>(p, stream);
-        case 4: return launch_mma_one<4, TS>(p, stream);
-        case 8: return launch_mma_one<8, TS>(p, stream);
+        case 1: return launch_mma_one<1, BF, TS>(p, stream);
+        case 2: return launch_mma_one<2, BF, TS>(p, stream);
+        case 4: return launch_mma_one<4, BF, TS>(p, stream);
+        case 8: return launch_mma_one<8, BF, TS>(p, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
+template <bool BF>
 int mma_tile_of(int group) {
     switch (group) {
-        case 1: return MmaTraits<1>::kTile;
-        case 2: return MmaTraits<2>::kTile;
-        case 4: return MmaTraits<4>::kTile;
-        case 8: return MmaTraits<8>::kTile;
+        case 1: return MmaTraits<1, BF>::kTile;
+        case 2: return MmaTraits<2, BF>::kTile;
+        case 4: return MmaTraits<4, BF>::kTile;
+        case 8: return MmaTraits<8, BF>::kTile;
         default: return 0;
     }
 }
@@ -130,7 +138,9 @@ cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) 
 }  // namespace
 
 int decode_tile_tokens(int head_dim, int group, bool fp8) {
-    if (head_dim == 128) return fp8 ? mma_tile_of(group) : tile_of<128, false>(group);
+    if (head_dim == 128)
+        return fp8 ? mma_tile_of<false>(group) : (PKV_DECODE_BF16_MMA ? mma_tile_of<true>(group)
+                                                                       : tile_of<128, false>(group));
     if (head_dim == 64) return fp8 ? tile_of<64, true>(group) : tile_of<64, false>(group);
     return 0;
 }
@@ -165,8 +175,9 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.out = static_cast<__nv_bfloat16 *>(a.out);
     p.dev_err = a.dev_err;
     const int group = a.num_q_heads / a.num_kv_heads;
-    if (a.fp8 && a.head_dim == 128) return a.token_scales ? launch_mma<true>(group, p, stream)
-                                                          : launch_mma<false>(group, p, stream);
+    if (a.fp8 && a.head_dim == 128) return a.token_scales ? launch_mma<false, true>(group, p, stream)
+                                                          : launch_mma<false, false>(group, p, stream);
+    if (PKV_DECODE_BF16_MMA && !a.fp8 && a.head_dim == 128) return launch_mma<true, false>(group, p, stream);
     if (a.fp8 && a.token_scales) {
         if (a.head_dim == 128) return launch_group<128, true, true>(group, p, stream);
         if (a.head_dim == 64) return launch_group<64, true, true>(group, p, stream);

@@ -1,6 +1,9 @@
 // decode_mma.cuh -- paged decode attention over an E4M3 cache (head_dim 128)
 // with the products on the warp-level tensor-core MMA (sm_100a).
 //
+// Two cache types share the kernel (template flag BF): E4M3 (one byte per
+// element) and bf16.
+//
 // Why: with one byte per cached element, the CUDA-core decode is bound by
 // instruction issue, not by HBM -- every (token, KV head) costs 2 * G * 128
 // multiply-adds plus the E4M3 widening against only 256 bytes of K and V.
@@ -11,7 +14,12 @@
 // per pair, straight into an operand register), q is scaled by a power of
 // two into f16 (exact for bf16 q), and the MMA forms the exact products and
 // accumulates them in fp32. What remains on the CUDA cores is the widening,
-// the softmax and the bookkeeping. The problem is the pages' decode
+// the softmax and the bookkeeping. A bf16 cache feeds the MMA directly (bf16
+// operands, no widening); its weights go in as a bf16 pair hi + lo (two MMAs)
+// so that they keep about 16 significant bits. With bf16 the CUDA-core kernel
+// already streams HBM near its peak, but its instruction stream is what
+// limits it when the K/V come from L2 (blocks shared by many sequences), and
+// it draws the power that caps the clock. The problem is the pages' decode
 // ("DeepSeek复刻vLLM反超原版", section "vLLM：大模型推理的加速引擎与挑战":
 // block tables into a shared pool; "nano-vllm-lite", section 核心技术改进 3:
 // the FP8 KV cache and its 2x smaller reads).
@@ -20,27 +28,31 @@
 // partition); every K/V byte of the partition is read from HBM once. Each
 // warp owns kWT consecutive tokens of every kTile-token tile and runs its own
 // pipeline: lane 0 copies its rows of K and V with tensor-map copies
-// (cp.async.bulk.tensor, 16-row boxes of 128 bytes, 128-byte swizzle, no
+// (cp.async.bulk.tensor, 16-row boxes of 128 bytes -- one per row for E4M3,
+// the two 64-element halves of a row for bf16 -- 128-byte swizzle, no
 // multicast) into a kStages-deep ring, completing on the warp's own
 // mbarriers, and refills a stage once the warp is done with it.
 //
 // Per 16-token group (fragment layouts of m16n8k16; g = lane / 4, t = lane % 4):
 //  * Scores, S^T[16 tokens x 8 heads] = K[16 x 128] . Q^T[128 x 8]: A = K rows
 //    g and g + 8, B = q of head g (zero for g >= G). The contraction order of
-//    the 128 dims is free, so k-step i takes dims 32t + 4i .. 32t + 4i + 3 of
-//    each lane's rows: a lane reads 32 contiguous codes of two rows, and one
-//    conversion per code pair gives an operand register. The swizzle makes
-//    these reads free of bank conflicts.
+//    the 128 dims is free, so a lane's k-steps cover 32 dims of its two rows
+//    that sit in two adjacent 16-byte chunks of each 128-byte half row:
+//    E4M3, dims 32t .. 32t + 31 (one conversion per code pair gives an
+//    operand register); bf16, dims 16t .. 16t + 15 and 64 + 16t .. + 15 (the
+//    words are the operand registers). The swizzle makes these reads free of
+//    bank conflicts.
 //  * Softmax in base 2 over the warp's tile (scores times scale * log2 e,
 //    the K scale and q's power of two), with a lazy reference maximum: it
 //    moves only when the tile maximum exceeds it by more than 8, so weights
 //    stay <= 2^8 (f16 range) and the accumulators are rescaled rarely.
 //  * The weights, packed to f16, are transposed in registers
 //    (movmatrix.trans) into the B operand of P V.
-//  * P V, O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] . P^T[16 x 8]: m-tile
-//    j covers dims 16g + 2j (row g) and 16g + 2j + 1 (row g + 8), so a lane
-//    reads 16 contiguous codes of 4 rows; byte permutes pair two tokens' codes
-//    at one dim before the conversion.
+//  * P V, O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] . P^T[16 x 8]: an
+//    m-tile covers dims e (row g) and e + 1 (row g + 8), with e = 16g + 2j
+//    (E4M3) or 64h + 8g + 2q (bf16, m-tile 4h + q), so a lane reads the
+//    16-byte chunk g of 4 rows (of each half, bf16); byte permutes pair two
+//    tokens' elements at one dim (before the conversion, for E4M3).
 //  * Rows past the end of the context (inside the last copied box) are
 //    excluded: their scores become -inf and their V codes zero.
 //  * Per-token scales (TS): the K and V scale runs are bulk-copied with the
@@ -73,16 +85,26 @@ namespace pkv {
 #define PKV_MMA_STAGES 2
 #endif
 
-template <int G>
+#ifndef PKV_MMA_WARP_TOKENS_BF16
+#define PKV_MMA_WARP_TOKENS_BF16 16
+#endif
+#ifndef PKV_MMA_STAGES_BF16
+#define PKV_MMA_STAGES_BF16 2
+#endif
+
+template <int G, bool BF = false>
 struct MmaTraits {
     static constexpr int kD = 128;
     static constexpr int kNW = PKV_MMA_WARPS;
-    static constexpr int kWT = PKV_MMA_WARP_TOKENS;  // tokens per warp per tile
+    static constexpr int kWT = BF ? PKV_MMA_WARP_TOKENS_BF16 : PKV_MMA_WARP_TOKENS;  // tokens per warp per tile
     static constexpr int kNGW = kWT / 16;            // 16-token groups per warp per tile
     static constexpr int kTile = kNW * kWT;
-    static constexpr int kStages = PKV_MMA_STAGES;
-    static constexpr int kGroupBytes = 16 * 128;  // 16 rows of 128 codes
-    static constexpr int kSliceBytes = kWT * 128;  // a warp's K (or V) rows of one tile
+    static constexpr int kStages = BF ? PKV_MMA_STAGES_BF16 : PKV_MMA_STAGES;
+    static constexpr int kRowBytes = BF ? 256 : 128;
+    static constexpr int kHalves = BF ? 2 : 1;  // 128-byte boxes per row
+    // a 16-row group: [half][16 rows][128 bytes]
+    static constexpr int kGroupBytes = 16 * kRowBytes;
+    static constexpr int kSliceBytes = kWT * kRowBytes;  // a warp's K (or V) rows of one tile
     // [stage][warp][K slice | V slice], 1024-byte aligned (the swizzle atom)
     static constexpr int kStageBytes = kNW * 2 * kSliceBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
@@ -122,6 +144,25 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D += A . B, m16n8k16, bf16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool BF>
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    if constexpr (BF)
+        mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
+    else
+        mma_f16_16816(d, a0, a1, a2, a3, b0, b1);
+}
+
 // Transpose of an 8 x 8 matrix of 16-bit elements held one word per lane
 // (lane g*4 + t holds row g, columns 2t and 2t + 1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -130,11 +171,12 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     return y;
 }
 
-template <int G, int MIN_BLOCKS, bool TS>
-__global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
+template <int G, bool BF, int MIN_BLOCKS, bool TS>
+__global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
                             const __grid_constant__ CUtensorMap map_v, int box_rows) {
-    using T = MmaTraits<G>;
+    static_assert(!(BF && TS), "per-token scales exist only for E4M3");
+    using T = MmaTraits<G, BF>;
     constexpr int D = T::kD;
     constexpr int NW = T::kNW;
     constexpr int WT = T::kWT;
@@ -219,7 +261,7 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
         const int a0 = warp_tok0(j);
         const int nv = min(end - a0, WT);
         uint32_t bytes = 0;
-        for (int a = 0; a < nv; a += box_rows) bytes += box_rows * 128 + (TS ? box_rows * 4 : 0);
+        for (int a = 0; a < nv; a += box_rows) bytes += box_rows * T::kRowBytes + (TS ? box_rows * 4 : 0);
         mbar_arrive_expect_tx(&full_k[s], bytes);
         mbar_arrive_expect_tx(&full_v[s], bytes);
         const uint32_t sk = sbase + s * T::kStageBytes + warp * 2 * T::kSliceBytes;
@@ -228,8 +270,13 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
             const int tok = a0 + a;
             const long long phys = ids[(tok >> lbs) - first_blk];
             const long long row = (phys * p.num_kv_heads + kvh) * p.block_size + (tok & bs_mask);
-            tc::tma_load_2d(sk + a * 128, &map_k, 0, (int)row, &full_k[s]);
-            tc::tma_load_2d(sv + a * 128, &map_v, 0, (int)row, &full_v[s]);
+            // group a / 16, rows a % 16 .. of each 128-byte half
+            const uint32_t dst = (a >> 4) * T::kGroupBytes + (a & 15) * 128;
+#pragma unroll
+            for (int hh = 0; hh < T::kHalves; ++hh) {
+                tc::tma_load_2d(sk + dst + hh * 2048, &map_k, hh * 64, (int)row, &full_k[s]);
+                tc::tma_load_2d(sv + dst + hh * 2048, &map_v, hh * 64, (int)row, &full_v[s]);
+            }
             if constexpr (TS) {
                 uint8_t *sc = smem + T::kOffScales + ((s * NW + warp) * 2) * WT * 4;
                 bulk_g2s(sc + a * 4, p.k_scale + row, box_rows * 4, &full_k[s]);
@@ -248,16 +295,19 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
     // qf[i][0] = dims 32t + 4i, +1; qf[i][1] = dims 32t + 4i + 2, +3 (zero
     // for g >= G). Scaled by 2^k so that the largest |q| of the KV head's
     // group lies in [2^14, 2^15): exact for bf16 q down to 2^-29 of it.
+    // bf16: q stays bf16 (exact), k-step i takes dims 16t + 4i .. + 3 (i < 4)
+    // and 64 + 16t + 4(i - 4) .. + 3 (i >= 4), the words of two 16-byte chunks
+    // of each half.
     uint32_t qf[8][2];
     float score_scale;
     {
         uint32_t qw[16];
         if (g < G) {
-            const uint4 *src =
-                reinterpret_cast<const uint4 *>(p.q + ((long long)seq * p.num_q_heads + qh0 + g) * D + 32 * t);
+            const __nv_bfloat16 *qrow = p.q + ((long long)seq * p.num_q_heads + qh0 + g) * D;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint4 w = __ldg(src + i);
+                const int e0 = BF ? (i >> 1) * 64 + 16 * t + (i & 1) * 8 : 32 * t + 8 * i;
+                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qrow + e0));
                 qw[4 * i] = w.x;
                 qw[4 * i + 1] = w.y;
                 qw[4 * i + 2] = w.z;
@@ -267,6 +317,14 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
 #pragma unroll
             for (int i = 0; i < 16; ++i) qw[i] = 0u;
         }
+      if constexpr (BF) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            qf[i][0] = qw[2 * i];
+            qf[i][1] = qw[2 * i + 1];
+        }
+        score_scale = p.qk_scale_log2;
+      } else {
         float mx = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
@@ -281,6 +339,7 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
             qf[i][1] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i + 1]), k), ldexpf(bf16hi(qw[2 * i + 1]), k));
         }
         score_scale = ldexpf(TS ? p.qk_scale_log2 : p.qk_scale_log2 * __ldg(p.k_scale + kvh), -k);
+      }
     }
 
     float o[8][4];
@@ -316,17 +375,33 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
             float c[4] = {0.f, 0.f, 0.f, 0.f};
             if (gi * 16 < nv) {
                 const uint32_t kg = sk + gi * T::kGroupBytes;
-                const uint4 k0 = lds128(sw(kg, g, 2 * t));
-                const uint4 k1 = lds128(sw(kg, g, 2 * t + 1));
-                const uint4 k2 = lds128(sw(kg, g + 8, 2 * t));
-                const uint4 k3 = lds128(sw(kg, g + 8, 2 * t + 1));
-                const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
+                if constexpr (BF) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint2 a = tc::e4m3x4_to_f16x4(wg[i]);  // row g: dims +0,+1 | +2,+3
-                    const uint2 b = tc::e4m3x4_to_f16x4(wh[i]);  // row g + 8
-                    mma_f16_16816(c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint4 k0 = lds128(sw(kg + hh * 2048, g, 2 * t));
+                        const uint4 k1 = lds128(sw(kg + hh * 2048, g, 2 * t + 1));
+                        const uint4 k2 = lds128(sw(kg + hh * 2048, g + 8, 2 * t));
+                        const uint4 k3 = lds128(sw(kg + hh * 2048, g + 8, 2 * t + 1));
+                        const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                        const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            mma_bf16_16816(c, wg[2 * i], wh[2 * i], wg[2 * i + 1], wh[2 * i + 1], qf[4 * hh + i][0],
+                                           qf[4 * hh + i][1]);
+                    }
+                } else {
+                    const uint4 k0 = lds128(sw(kg, g, 2 * t));
+                    const uint4 k1 = lds128(sw(kg, g, 2 * t + 1));
+                    const uint4 k2 = lds128(sw(kg, g + 8, 2 * t));
+                    const uint4 k3 = lds128(sw(kg, g + 8, 2 * t + 1));
+                    const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint2 a = tc::e4m3x4_to_f16x4(wg[i]);  // row g: dims +0,+1 | +2,+3
+                        const uint2 b = tc::e4m3x4_to_f16x4(wh[i]);  // row g + 8
+                        mma_f16_16816(c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
+                    }
                 }
             }
             float ks0 = score_scale, ks1 = score_scale;
@@ -429,9 +504,46 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
 #pragma unroll
         for (int gi = 0; gi < NGW; ++gi) {
             if (gi * 16 >= nv) continue;
+            const uint32_t vg = sv + gi * T::kGroupBytes;
+            if constexpr (BF) {
+                // weights as bf16 hi + lo: p - hi is exact in fp32 and lo keeps
+                // the next 8 bits
+                const uint32_t h01 = tc::pack_bf16(pw[gi][0], pw[gi][1]), h23 = tc::pack_bf16(pw[gi][2], pw[gi][3]);
+                const uint32_t l01 = tc::pack_bf16(pw[gi][0] - bf16lo(h01), pw[gi][1] - bf16hi(h01));
+                const uint32_t l23 = tc::pack_bf16(pw[gi][2] - bf16lo(h23), pw[gi][3] - bf16hi(h23));
+                const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+                const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t vh = vg + hh * 2048;
+                    uint4 r0 = lds128(sw(vh, 2 * t, g));
+                    uint4 r1 = lds128(sw(vh, 2 * t + 1, g));
+                    uint4 r2 = lds128(sw(vh, 2 * t + 8, g));
+                    uint4 r3 = lds128(sw(vh, 2 * t + 9, g));
+                    if (gi * 16 + 16 > nv) {  // rows past the end: zero (stale slots may hold NaN)
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                        if (gi * 16 + 2 * t >= nv) r0 = z;
+                        if (gi * 16 + 2 * t + 1 >= nv) r1 = z;
+                        if (gi * 16 + 2 * t + 8 >= nv) r2 = z;
+                        if (gi * 16 + 2 * t + 9 >= nv) r3 = z;
+                    }
+                    const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+                    const uint32_t w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
+#pragma unroll
+                    for (int qd = 0; qd < 4; ++qd) {
+                        // dims 64hh + 8g + 2qd, + 1 of tokens (2t, 2t+1) and (2t+8, 2t+9)
+                        const uint32_t a0 = __byte_perm(w0[qd], w1[qd], 0x5410);
+                        const uint32_t a1 = __byte_perm(w0[qd], w1[qd], 0x7632);
+                        const uint32_t a2 = __byte_perm(w2[qd], w3[qd], 0x5410);
+                        const uint32_t a3 = __byte_perm(w2[qd], w3[qd], 0x7632);
+                        mma_bf16_16816(o[4 * hh + qd], a0, a1, a2, a3, bh0, bh1);
+                        mma_bf16_16816(o[4 * hh + qd], a0, a1, a2, a3, bl0, bl1);
+                    }
+                }
+                continue;
+            }
             const uint32_t b0 = movmatrix_trans(tc::pack_f16(pw[gi][0], pw[gi][1]));  // tokens 2t, 2t+1 of head g
             const uint32_t b1 = movmatrix_trans(tc::pack_f16(pw[gi][2], pw[gi][3]));  // tokens 2t+8, 2t+9
-            const uint32_t vg = sv + gi * T::kGroupBytes;
             uint4 r0 = lds128(sw(vg, 2 * t, g));
             uint4 r1 = lds128(sw(vg, 2 * t + 1, g));
             uint4 r2 = lds128(sw(vg, 2 * t + 8, g));
@@ -497,11 +609,14 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
         const int head = 2 * t + h;
         if (head < G) {
             const float sc = TS ? ldexpf(1.f, vexp) : 1.f;  // TS: undo the 2^-vexp of the weights
-            float *dst = merge_acc + (warp * G + head) * D + 16 * g;
+            float *dst = merge_acc + (warp * G + head) * D;
 #pragma unroll
-            for (int jj = 0; jj < 8; jj += 2)
-                *reinterpret_cast<float4 *>(dst + 2 * jj) =
+            for (int jj = 0; jj < 8; jj += 2) {
+                // m-tiles jj, jj + 1 hold dims e, e + 1, e + 2, e + 3
+                const int e = BF ? (jj >> 2) * 64 + 8 * g + 2 * (jj & 3) : 16 * g + 2 * jj;
+                *reinterpret_cast<float4 *>(dst + e) =
                     make_float4(o[jj][h] * sc, o[jj][2 + h] * sc, o[jj + 1][h] * sc, o[jj + 1][2 + h] * sc);
+            }
             if (g == 0) {
                 merge_m[warp * G + head] = m_ref[h];
                 merge_l[warp * G + head] = l[h];
@@ -520,7 +635,7 @@ __global__ void __launch_bounds__(MmaTraits<G>::kThreads, MIN_BLOCKS)
             L += merge_l[w * G + h] * e;
         }
         float post = 1.f / L;
-        if constexpr (!TS) post *= __ldg(p.v_scale + kvh);
+        if constexpr (!TS && !BF) post *= __ldg(p.v_scale + kvh);
         for (int w = 0; w < NW; ++w) merge_w[w * G + h] *= post;
         if (!single) {
             float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * 2;
@@ -552,6 +667,20 @@ inline bool make_e4m3_pool_map(CUtensorMap *map, const void *pool, long long row
     const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(pool), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The bf16 pool as a 2-D tensor of 128-element rows; boxes of 64 elements
+// (128 bytes) x box_rows rows, 128-byte swizzle (a row takes two boxes).
+inline bool make_bf16_pool_map(CUtensorMap *map, const void *pool, long long rows, int box_rows) {
+    tc::EncodeTiledFn fn = tc::encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
