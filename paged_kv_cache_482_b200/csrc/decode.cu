@@ -174,6 +174,8 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.part_ml = a.part_ml;
     p.out = static_cast<__nv_bfloat16 *>(a.out);
     p.dev_err = a.dev_err;
+    p.cu_q_lens = a.cu_q_lens;
+    p.total_q = a.total_q;
     const int group = a.num_q_heads / a.num_kv_heads;
     if (a.fp8 && a.head_dim == 128) return a.token_scales ? launch_mma<false, true>(group, p, stream)
                                                           : launch_mma<false, false>(group, p, stream);

@@ -79,8 +79,15 @@ struct DecodeParams {
     float *part_ml;
     __nv_bfloat16 *out;
     int *dev_err;
+    // Rows of a chunked-prefill call routed here: when set, sequence i is
+    // served only if its chunk is one token (cu_q_lens[i + 1] - cu_q_lens[i]
+    // == 1), and its q and out row is cu_q_lens[i] (of total_q rows).
+    const int32_t *cu_q_lens;
+    int total_q;
 };
 
+// Block ids of a partition staged in shared memory; ids beyond are read
+// from the table row in global memory (every id is checked up front).
 constexpr int kMaxIdsPerPartition = 256;
 
 // Tuning constants (compile-time; the defaults are the measured choice).
@@ -200,6 +207,12 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         return;
     }
 
+    long long row = seq;  // q / out row
+    if (p.cu_q_lens) {
+        const int q0 = __ldg(p.cu_q_lens + seq), q1 = __ldg(p.cu_q_lens + seq + 1);
+        if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 != 1) return;  // the prefill kernels' sequence
+        row = q0;
+    }
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
     const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
@@ -210,18 +223,19 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
     if (!bad_len && start >= end) return;  // partition past this sequence's end
     if (bad_len && part != 0) return;
 
-    // Stage this partition's block ids (checked), zero the rings (rows past
-    // the end of a partial tile are then finite, so they can take part in
-    // the arithmetic with weight 0), set up the barriers.
+    // Check every block id of this partition and stage the first ones, zero
+    // the rings (rows past the end of a partial tile are then finite, so they
+    // can take part in the arithmetic with weight 0), set up the barriers.
     const int first_blk = start >> p.log2_block_size;
     const int n_blk = bad_len ? 0 : ((end - 1) >> p.log2_block_size) - first_blk + 1;
-    int bad = bad_len || n_blk > kMaxIdsPerPartition;
+    int bad = bad_len;
     const int32_t *table = p.block_tables + (long long)seq * p.max_blocks_per_seq + first_blk;
-    for (int i = tid; i < n_blk && i < kMaxIdsPerPartition; i += T::kThreads) {
+    for (int i = tid; i < n_blk; i += T::kThreads) {
         const int32_t id = __ldg(table + i);
-        ids[i] = id;
+        if (i < kMaxIdsPerPartition) ids[i] = id;
         bad |= (id < 0 || (long long)id >= p.num_blocks);
     }
+    auto blk_id = [&](int i) -> long long { return i < kMaxIdsPerPartition ? ids[i] : __ldg(table + i); };
     for (int i = tid; i < 2 * T::kRingBytes / 16; i += T::kThreads)
         reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();  // the zeros, before bulk copies overwrite them
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         if (tid == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
         if (single || bad_len) {
             for (int i = tid; i < G * D; i += T::kThreads)
-                p.out[((long long)seq * p.num_q_heads + qh0) * D + i] = __float2bfloat16_rn(0.f);
+                p.out[(row * p.num_q_heads + qh0) * D + i] = __float2bfloat16_rn(0.f);
         } else if (tid < G) {
             float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + tid) * p.num_partitions + part) * 2;
             ml[0] = -CUDART_INF_F;
@@ -273,7 +287,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         mbar_arrive_expect_tx(bar, (uint32_t)(max(a1 - a0, 0) * T::kRowBytes));
         if (p.block_size >= ROWS_W) {
             if (a1 > a0) {
-                const long long phys = ids[(a0 >> p.log2_block_size) - first_blk];
+                const long long phys = blk_id((a0 >> p.log2_block_size) - first_blk);
                 const int off = a0 & (p.block_size - 1);
                 bulk_g2s(dst0, src0 + phys * blk_stride + (long long)off * T::kRowBytes,
                          (uint32_t)((a1 - a0) * T::kRowBytes), bar);
@@ -283,7 +297,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
                 const int lb = a >> p.log2_block_size;
                 const int off = a & (p.block_size - 1);
                 const int n = min(p.block_size - off, a1 - a);
-                const long long phys = ids[lb - first_blk];
+                const long long phys = blk_id(lb - first_blk);
                 bulk_g2s(dst0 + (a - a0) * T::kRowBytes, src0 + phys * blk_stride + (long long)off * T::kRowBytes,
                          (uint32_t)(n * T::kRowBytes), bar);
                 a += n;
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
 #pragma unroll
     for (int hs = 0; hs < G; ++hs) {
         const uint4 w = __ldg(reinterpret_cast<const uint4 *>(
-            p.q + ((long long)seq * p.num_q_heads + qh0 + (hs ^ my_h)) * D + chunk * 8));
+            p.q + (row * p.num_q_heads + qh0 + (hs ^ my_h)) * D + chunk * 8));
         qw[hs][0] = w.x; qw[hs][1] = w.y; qw[hs][2] = w.z; qw[hs][3] = w.w;
     }
     // Multiplier of the reduced score: scale*log2(e) (and, for E4M3, the K
@@ -424,7 +438,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
         if constexpr (TS) {
             const int a = start + j * TILE + row0 + my_row;
             if (a < end) {
-                const long long phys = ids[(a >> p.log2_block_size) - first_blk];
+                const long long phys = blk_id((a >> p.log2_block_size) - first_blk);
                 const long long idx = (phys * p.num_kv_heads + kvh) * p.block_size + (a & (p.block_size - 1));
                 ks = __ldg(p.k_scale + idx);
                 vs = __ldg(p.v_scale + idx);
@@ -601,7 +615,7 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
 #pragma unroll
         for (int w = 0; w < NCW; ++w) o = fmaf(merge_acc[(w * G + h) * D + (idx % D)], merge_w[w * G + h], o);
         if (single) {
-            p.out[((long long)seq * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(o);
+            p.out[(row * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(o);
         } else {
             p.part_o[(((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * D + (idx % D)] = o;
         }

@@ -204,6 +204,12 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
         if (tid == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
         return;
     }
+    long long row = seq;  // q / out row
+    if (p.cu_q_lens) {
+        const int q0 = __ldg(p.cu_q_lens + seq), q1 = __ldg(p.cu_q_lens + seq + 1);
+        if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 != 1) return;  // the prefill kernels' sequence
+        row = q0;
+    }
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
     const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
@@ -214,13 +220,14 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     if (!bad_len && start >= end) return;
     if (bad_len && part != 0) return;
 
+    // every block id of the partition is checked; the first ones are staged
     const int first_blk = start >> p.log2_block_size;
     const int n_blk = bad_len ? 0 : ((end - 1) >> p.log2_block_size) - first_blk + 1;
-    int bad = bad_len || n_blk > kMaxIdsPerPartition;
+    int bad = bad_len;
     const int32_t *table = p.block_tables + (long long)seq * p.max_blocks_per_seq + first_blk;
-    for (int i = tid; i < n_blk && i < kMaxIdsPerPartition; i += T::kThreads) {
+    for (int i = tid; i < n_blk; i += T::kThreads) {
         const int32_t id = __ldg(table + i);
-        ids[i] = id;
+        if (i < kMaxIdsPerPartition) ids[i] = id;
         bad |= (id < 0 || (long long)id >= p.num_blocks);
     }
     uint64_t *full_k = reinterpret_cast<uint64_t *>(smem + T::kOffBars) + warp * STAGES;
@@ -239,7 +246,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
         if (tid == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
         if (single || bad_len) {
             for (int i = tid; i < G * D; i += T::kThreads)
-                p.out[((long long)seq * p.num_q_heads + qh0) * D + i] = __float2bfloat16_rn(0.f);
+                p.out[(row * p.num_q_heads + qh0) * D + i] = __float2bfloat16_rn(0.f);
         } else if (tid < G) {
             float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + tid) * p.num_partitions + part) * 2;
             ml[0] = -CUDART_INF_F;
@@ -268,7 +275,8 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
         const uint32_t sv = sk + T::kSliceBytes;
         for (int a = 0; a < nv; a += box_rows) {
             const int tok = a0 + a;
-            const long long phys = ids[(tok >> lbs) - first_blk];
+            const int bi = (tok >> lbs) - first_blk;
+            const long long phys = bi < kMaxIdsPerPartition ? ids[bi] : __ldg(table + bi);
             const long long row = (phys * p.num_kv_heads + kvh) * p.block_size + (tok & bs_mask);
             // group a / 16, rows a % 16 .. of each 128-byte half
             const uint32_t dst = (a >> 4) * T::kGroupBytes + (a & 15) * 128;
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     {
         uint32_t qw[16];
         if (g < G) {
-            const __nv_bfloat16 *qrow = p.q + ((long long)seq * p.num_q_heads + qh0 + g) * D;
+            const __nv_bfloat16 *qrow = p.q + (row * p.num_q_heads + qh0 + g) * D;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int e0 = BF ? (i >> 1) * 64 + 16 * t + (i & 1) * 8 : 32 * t + 8 * i;
@@ -650,7 +658,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
 #pragma unroll
         for (int w = 0; w < NW; ++w) acc = fmaf(merge_acc[(w * G + h) * D + (idx % D)], merge_w[w * G + h], acc);
         if (single) {
-            p.out[((long long)seq * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(acc);
+            p.out[(row * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(acc);
         } else {
             p.part_o[(((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * D + (idx % D)] = acc;
         }

@@ -59,10 +59,10 @@ int make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int
     const long long max_pt = max_pt_ids / tile * tile;
     long long pt = 0;  // 0: no split
     if (request == -1) {
-        if ((long long)max_context_len > max_pt_ids) return PKV_ERR_UNSUPPORTED;
+        // one partition per sequence, of any length (block ids beyond the
+        // staged ones are read from the table)
     } else if (request > 0) {
         pt = round_up((size_t)request, (size_t)tile);
-        if (pt > max_pt) return PKV_ERR_UNSUPPORTED;
         if (pt >= max_context_len) pt = 0;
     } else if (request == 0) {
         const long long units = (long long)num_seqs * num_kv_heads;

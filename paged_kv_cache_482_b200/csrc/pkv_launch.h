@@ -46,6 +46,11 @@ struct DecodeArgs {
     float *part_ml;        // [num_seqs][num_q_heads][num_partitions][2]
     void *out;
     int *dev_err;
+    // one-token chunks of a chunked-prefill call (null for a decode call):
+    // sequence i is served only if cu_q_lens[i + 1] - cu_q_lens[i] == 1, and
+    // its q / out row is cu_q_lens[i]
+    const int32_t *cu_q_lens = nullptr;
+    int total_q = 0;
 };
 
 // Tile (tokens per pipeline stage) of the decode kernel chosen for a shape;
@@ -85,6 +90,9 @@ struct PrefillArgs {
     // > 0: the one-tile kernel takes the sequences with chunks of at most
     // small_cut tokens, the warp-specialised kernel the others
     int small_cut;
+    // the one-tile kernel skips chunks shorter than this (one-token chunks
+    // go to the decode kernel when it is 2)
+    int small_min = 0;
 };
 
 struct NormArgs {

@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int t0 = tile * TQ;
     if (t0 >= c) return;
     if (a.small_cut > 0 && c > a.small_cut) return;  // a longer chunk: the warp-specialised kernel's
+    if (c < a.small_min) return;                     // a one-token chunk: the decode kernel's
     const int ctx = a.context_lens[s];
     const int32_t *table_g = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
     int32_t *table_s = reinterpret_cast<int32_t *>(sm + L::kTable);
@@ -539,14 +540,46 @@ bool prefill_supported(int head_dim, int group) {
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
-    // Chunks of more than one query tile (128 / G tokens) go to the
-    // warp-specialised kernel (two tiles per CTA, one CTA per SM); shorter
-    // ones -- decode requests among them -- to the one-tile kernel, which fits
-    // two CTAs per SM. Each kernel skips the other's sequences.
+    // One-token chunks (decode requests in the batch) go to the decode
+    // kernel, which streams their K/V at HBM speed instead of filling 1 / 128
+    // of an MMA tile; chunks of more than one query tile (128 / G tokens) go
+    // to the warp-specialised kernel (two tiles per CTA, one CTA per SM);
+    // the rest to the one-tile kernel, which fits two CTAs per SM. Each
+    // kernel skips the others' sequences.
+    DecodeArgs d;
+    d.q = a.q;
+    d.k_cache = a.k_cache;
+    d.v_cache = a.v_cache;
+    d.block_tables = a.block_tables;
+    d.max_blocks_per_seq = a.max_blocks_per_seq;
+    d.context_lens = a.context_lens;
+    d.seq_order = nullptr;
+    d.num_seqs = a.num_seqs;
+    d.num_q_heads = a.num_q_heads;
+    d.num_kv_heads = a.num_kv_heads;
+    d.head_dim = a.head_dim;
+    d.block_size = a.block_size;
+    d.num_blocks = a.num_blocks;
+    d.scale = a.scale;
+    d.fp8 = a.fp8;
+    d.token_scales = a.token_scales;
+    d.k_scale = a.k_scale;
+    d.v_scale = a.v_scale;
+    d.max_context_len = a.max_blocks_per_seq * a.block_size;  // the table's capacity
+    d.partition_tokens = 0;                                   // no split: nothing to allocate
+    d.num_partitions = 1;
+    d.part_o = nullptr;
+    d.part_ml = nullptr;
+    d.out = a.out;
+    d.dev_err = a.dev_err;
+    d.cu_q_lens = a.cu_q_lens;
+    d.total_q = a.total_q;
+    cudaError_t e = launch_decode(d, stream);
+    if (e != cudaSuccess || a.max_q_len <= 1) return e;
     PrefillArgs small = a;
     small.small_cut = kRows / g;
+    small.small_min = 2;
     small.max_q_len = a.max_q_len < small.small_cut ? a.max_q_len : small.small_cut;
-    cudaError_t e;
     if (a.fp8 && a.token_scales)
         e = a.head_dim == 128 ? launch_d<128, true, true>(small, g, stream) : launch_d<64, true, true>(small, g, stream);
     else if (a.head_dim == 128)

@@ -67,6 +67,25 @@ def test_fp8_lengths_at_group_and_tile_boundaries(bs):
         check_workload(wl, partition_request=split)
 
 
+@pytest.mark.parametrize("d,dt", [(64, W.CACHE_BF16), (128, W.CACHE_BF16), (128, W.CACHE_FP8),
+                                  (128, W.CACHE_FP8_TOKEN)])
+def test_unsplit_partition_beyond_the_staged_block_ids(d, dt):
+    """No split on contexts of up to 500 blocks of 8 tokens: the block ids
+    past the 256 staged in shared memory come from the table row."""
+    c = cfg(num_seqs=3, num_q_heads=8, num_kv_heads=2, head_dim=d, block_size=8, ctx_lo=2100, ctx_hi=4000,
+            cache_dtype=dt)
+    wl = W.generate(c, 17)
+    if dt == W.CACHE_FP8_TOKEN:
+        from test_gpu_token_scales import run_decode
+
+        out, _, st = run_decode(wl, partition=-1)
+        ref, _, _, rst, _, _ = O.run_workload(wl, num_threads=8)
+        assert st == K.PKV_OK and rst == O.ORC_OK
+        compare(out, ref, True, "unsplit, per-token scales")
+    else:
+        check_workload(wl, partition_request=-1)
+
+
 def _with_lengths(c, wl, lens):
     """A workload of the same pool with given lengths (rows re-drawn)."""
     g = torch.Generator().manual_seed(99)
