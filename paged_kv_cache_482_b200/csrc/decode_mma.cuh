@@ -358,6 +358,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     float m_ref[2] = {-CUDART_INF_F, -CUDART_INF_F};  // heads 2t, 2t + 1 (base-2 units)
     float l[2] = {0.f, 0.f};
     int vexp = -100000;  // TS: weights are scaled by 2^-vexp before rounding
+    float vinv = 0.f;    // 2^-vexp
 
     // Swizzled row r, 16-byte chunk c of a 16-row group at byte address base.
     auto sw = [](uint32_t base, int r, int c) { return base + r * 128 + (((c ^ r) & 7) << 4); };
@@ -480,16 +481,17 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
             }
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-            int ev = 0;
-            frexpf(vm, &ev);  // vm < 2^ev; the same in every lane
+            // vm < 2^ev (vm >= the smallest normal: scales are floored there,
+            // and the tile has a valid token); the same in every lane
+            const int ev = (int)(__float_as_uint(vm) >> 23) - 126;
             if (ev > vexp) {
                 const float f = ldexpf(1.f, vexp - ev);  // 0 for the first rise
                 alpha[0] *= f;
                 alpha[1] *= f;
                 rescale = true;
                 vexp = ev;
+                vinv = ldexpf(1.f, -vexp);
             }
-            const float vinv = ldexpf(1.f, -vexp);
 #pragma unroll
             for (int gi = 0; gi < NGW; ++gi) {
                 const float f0 = vsc[gi][0] * vinv, f1 = vsc[gi][1] * vinv;
