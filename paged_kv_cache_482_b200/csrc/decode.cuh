@@ -84,7 +84,44 @@ struct DecodeParams {
     // == 1), and its q and out row is cu_q_lens[i] (of total_q rows).
     const int32_t *cu_q_lens;
     int total_q;
+    // Shared-prefix (cascade) mode, when cu_group_seqs is set: sequences
+    // cu_group_seqs[j] .. cu_group_seqs[j + 1] - 1 form group j, whose first
+    // group_prefix[j] tokens are the same cached blocks for every member. The
+    // prefix kernel writes each member's prefix partial to slot 0; the decode
+    // kernel attends the rest of each sequence, partition p to slot p + 1.
+    const int32_t *cu_group_seqs;
+    const int32_t *group_prefix;
+    int num_groups;
+    int max_group_seqs;  // host bound: sizes the prefix kernel's grid
+    int grid_partitions;  // partitions per (sequence, KV head) in the decode grid
 };
+
+// Group of sequence seq in shared-prefix mode (largest j with
+// cu_group_seqs[j] <= seq; -1 when seq precedes group 0).
+__device__ __forceinline__ int group_of(const DecodeParams &p, int seq) {
+    int lo = 0, hi = p.num_groups - 1, ans = -1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.cu_group_seqs + mid) <= seq) {
+            ans = mid;
+            lo = mid + 1;
+        } else {
+            hi = mid - 1;
+        }
+    }
+    return ans;
+}
+
+// Prefix length of sequence seq in shared-prefix mode, or -1 when it is not
+// usable (negative, not a whole number of blocks, past the context, or the
+// sequence in no group).
+__device__ __forceinline__ int prefix_of(const DecodeParams &p, int seq, int ctx) {
+    const int j = group_of(p, seq);
+    if (j < 0 || seq >= __ldg(p.cu_group_seqs + j + 1)) return -1;
+    const int P = __ldg(p.group_prefix + j);
+    if (P < 0 || P > ctx || (P & (p.block_size - 1)) != 0) return -1;
+    return P;
+}
 
 // Block ids of a partition staged in shared memory; ids beyond are read
 // from the table row in global memory (every id is checked up front).
@@ -635,16 +672,27 @@ __global__ void __launch_bounds__(D) paged_decode_reduce_kernel(const DecodePara
     if (seq < 0 || seq >= p.num_seqs) return;  // the decode grid reported it
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
-    if (ctx < 1 || ctx > p.max_context_len || ctx > table_cap) return;  // decode wrote zeros
-    const int n = (ctx + p.partition_tokens - 1) / p.partition_tokens;
-    if (n <= 1) return;  // decode wrote the output itself
-    const long long base = ((long long)seq * p.num_q_heads + qh) * p.num_partitions;
+    const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
+    // partial slots first .. first + n - 1 of this sequence
+    int first = 0, n = 0, bad0 = 0;
+    if (p.cu_group_seqs) {  // slot 0: the shared prefix (when there is one), then the suffix partitions
+        const int P = bad_len ? -1 : prefix_of(p, seq, ctx);
+        bad0 = P < 0;
+        const int n_suf = P >= 0 ? (ctx - P + p.partition_tokens - 1) / p.partition_tokens : 0;
+        first = P == 0 ? 1 : 0;
+        n = (P != 0) + n_suf;
+    } else {
+        if (bad_len) return;  // decode wrote zeros
+        n = (ctx + p.partition_tokens - 1) / p.partition_tokens;
+        if (n <= 1) return;  // decode wrote the output itself
+    }
+    const long long base = ((long long)seq * p.num_q_heads + qh) * p.num_partitions + first;
     __shared__ float w_s[1024];
     __shared__ int bad_s;
     if (threadIdx.x == 0) {
         float M = -CUDART_INF_F;
-        int bad = 0;
-        for (int i = 0; i < n; ++i) {
+        int bad = bad0 || bad_len;
+        for (int i = 0; i < n && !bad; ++i) {
             const float li = p.part_ml[(base + i) * 2 + 1];
             bad |= !(li > 0.f);
             M = fmaxf(M, p.part_ml[(base + i) * 2]);

@@ -171,6 +171,171 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     return y;
 }
 
+// Swizzled row r, 16-byte chunk c of a 16-row group at byte address base.
+__device__ __forceinline__ uint32_t swz16(uint32_t base, int r, int c) {
+    return base + r * 128 + (((c ^ r) & 7) << 4);
+}
+
+// q fragments of the row this lane's column g reads (qrow; null: a column
+// with no query, zeros), for k-steps in the order of the K reads below:
+// qf[i][0] = dims d_i, d_i + 1, qf[i][1] = dims d_i + 2, d_i + 3, with d_i =
+// 32t + 4i (E4M3) or 64(i / 4) + 16t + 4(i % 4) (bf16). E4M3: q becomes f16
+// after a power-of-two rescale that puts the warp's largest |q| in
+// [2^14, 2^15) (exact for bf16 q down to 2^-29 of it); bf16: q as is.
+// Returns the multiplier of a raw score into base-2 units (score_scale_log2
+// times the undoing power of two). Every lane of the warp must call it.
+template <bool BF>
+__device__ __forceinline__ float load_q_frags(const __nv_bfloat16 *qrow, int t, float score_scale_log2,
+                                              uint32_t (&qf)[8][2]) {
+    uint32_t qw[16];
+    if (qrow) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e0 = BF ? (i >> 1) * 64 + 16 * t + (i & 1) * 8 : 32 * t + 8 * i;
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qrow + e0));
+            qw[4 * i] = w.x;
+            qw[4 * i + 1] = w.y;
+            qw[4 * i + 2] = w.z;
+            qw[4 * i + 3] = w.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) qw[i] = 0u;
+    }
+    if constexpr (BF) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            qf[i][0] = qw[2 * i];
+            qf[i][1] = qw[2 * i + 1];
+        }
+        return score_scale_log2;
+    } else {
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int e = 0;
+        frexpf(mx, &e);  // mx < 2^e
+        const int k = 15 - e;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            qf[i][0] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i]), k), ldexpf(bf16hi(qw[2 * i]), k));
+            qf[i][1] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i + 1]), k), ldexpf(bf16hi(qw[2 * i + 1]), k));
+        }
+        return ldexpf(score_scale_log2, -k);
+    }
+}
+
+// Raw scores of one 16-token group: c = S^T fragment (tokens g, g + 8 x
+// columns 2t, 2t + 1), accumulated onto c.
+template <bool BF>
+__device__ __forceinline__ void qk_group(uint32_t kg, int g, int t, const uint32_t (&qf)[8][2], float (&c)[4]) {
+    if constexpr (BF) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint4 k0 = lds128(swz16(kg + hh * 2048, g, 2 * t));
+            const uint4 k1 = lds128(swz16(kg + hh * 2048, g, 2 * t + 1));
+            const uint4 k2 = lds128(swz16(kg + hh * 2048, g + 8, 2 * t));
+            const uint4 k3 = lds128(swz16(kg + hh * 2048, g + 8, 2 * t + 1));
+            const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                mma_bf16_16816(c, wg[2 * i], wh[2 * i], wg[2 * i + 1], wh[2 * i + 1], qf[4 * hh + i][0],
+                               qf[4 * hh + i][1]);
+        }
+    } else {
+        const uint4 k0 = lds128(swz16(kg, g, 2 * t));
+        const uint4 k1 = lds128(swz16(kg, g, 2 * t + 1));
+        const uint4 k2 = lds128(swz16(kg, g + 8, 2 * t));
+        const uint4 k3 = lds128(swz16(kg, g + 8, 2 * t + 1));
+        const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+        const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint2 a = tc::e4m3x4_to_f16x4(wg[i]);  // row g: dims +0,+1 | +2,+3
+            const uint2 b = tc::e4m3x4_to_f16x4(wh[i]);  // row g + 8
+            mma_f16_16816(c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
+        }
+    }
+}
+
+// o += P V of one 16-token group. pw: the weights of tokens g, g + 8 x
+// columns 2t, 2t + 1 (already times 2^-vexp and the V scale for per-token
+// scales). Rows at or past n_valid (of 16) read as zero: stale slots of a
+// partial box may hold NaN.
+template <bool BF>
+__device__ __forceinline__ void pv_group(uint32_t vg, int g, int t, const float (&pw)[4], int n_valid,
+                                         float (&o)[8][4]) {
+    uint4 r[2][4];
+#pragma unroll
+    for (int hh = 0; hh < (BF ? 2 : 1); ++hh) {
+        const uint32_t vh = vg + hh * 2048;
+        r[hh][0] = lds128(swz16(vh, 2 * t, g));
+        r[hh][1] = lds128(swz16(vh, 2 * t + 1, g));
+        r[hh][2] = lds128(swz16(vh, 2 * t + 8, g));
+        r[hh][3] = lds128(swz16(vh, 2 * t + 9, g));
+        if (n_valid < 16) {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            if (2 * t >= n_valid) r[hh][0] = z;
+            if (2 * t + 1 >= n_valid) r[hh][1] = z;
+            if (2 * t + 8 >= n_valid) r[hh][2] = z;
+            if (2 * t + 9 >= n_valid) r[hh][3] = z;
+        }
+    }
+    if constexpr (BF) {
+        // weights as bf16 hi + lo: p - hi is exact in fp32 and lo keeps the
+        // next 8 bits
+        const uint32_t h01 = tc::pack_bf16(pw[0], pw[1]), h23 = tc::pack_bf16(pw[2], pw[3]);
+        const uint32_t l01 = tc::pack_bf16(pw[0] - bf16lo(h01), pw[1] - bf16hi(h01));
+        const uint32_t l23 = tc::pack_bf16(pw[2] - bf16lo(h23), pw[3] - bf16hi(h23));
+        const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+        const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t w0[4] = {r[hh][0].x, r[hh][0].y, r[hh][0].z, r[hh][0].w};
+            const uint32_t w1[4] = {r[hh][1].x, r[hh][1].y, r[hh][1].z, r[hh][1].w};
+            const uint32_t w2[4] = {r[hh][2].x, r[hh][2].y, r[hh][2].z, r[hh][2].w};
+            const uint32_t w3[4] = {r[hh][3].x, r[hh][3].y, r[hh][3].z, r[hh][3].w};
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                // dims 64hh + 8g + 2qd, + 1 of tokens (2t, 2t+1) and (2t+8, 2t+9)
+                const uint32_t a0 = __byte_perm(w0[qd], w1[qd], 0x5410);
+                const uint32_t a1 = __byte_perm(w0[qd], w1[qd], 0x7632);
+                const uint32_t a2 = __byte_perm(w2[qd], w3[qd], 0x5410);
+                const uint32_t a3 = __byte_perm(w2[qd], w3[qd], 0x7632);
+                mma_bf16_16816(o[4 * hh + qd], a0, a1, a2, a3, bh0, bh1);
+                mma_bf16_16816(o[4 * hh + qd], a0, a1, a2, a3, bl0, bl1);
+            }
+        }
+    } else {
+        const uint32_t b0 = movmatrix_trans(tc::pack_f16(pw[0], pw[1]));  // tokens 2t, 2t+1 of column g
+        const uint32_t b1 = movmatrix_trans(tc::pack_f16(pw[2], pw[3]));  // tokens 2t+8, 2t+9
+        const uint32_t w0[4] = {r[0][0].x, r[0][0].y, r[0][0].z, r[0][0].w};
+        const uint32_t w1[4] = {r[0][1].x, r[0][1].y, r[0][1].z, r[0][1].w};
+        const uint32_t w2[4] = {r[0][2].x, r[0][2].y, r[0][2].z, r[0][2].w};
+        const uint32_t w3[4] = {r[0][3].x, r[0][3].y, r[0][3].z, r[0][3].w};
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+            // dims 16g + 4qd .. +3 of tokens (2t, 2t+1) and (2t+8, 2t+9)
+            const uint2 x0 = tc::e4m3x4_to_f16x4(__byte_perm(w0[qd], w1[qd], 0x5140));
+            const uint2 x1 = tc::e4m3x4_to_f16x4(__byte_perm(w0[qd], w1[qd], 0x7362));
+            const uint2 y0 = tc::e4m3x4_to_f16x4(__byte_perm(w2[qd], w3[qd], 0x5140));
+            const uint2 y1 = tc::e4m3x4_to_f16x4(__byte_perm(w2[qd], w3[qd], 0x7362));
+            mma_f16_16816(o[2 * qd], x0.x, x0.y, y0.x, y0.y, b0, b1);
+            mma_f16_16816(o[2 * qd + 1], x1.x, x1.y, y1.x, y1.y, b0, b1);
+        }
+    }
+}
+
+// Dim held by accumulator o[j][0..1] (o[j][2..3]: the next dim) of row
+// group g: 16g + 2j (E4M3) or 64(j / 4) + 8g + 2(j % 4) (bf16).
+template <bool BF>
+__device__ __forceinline__ int acc_dim(int j, int g) {
+    return BF ? (j >> 2) * 64 + 8 * g + 2 * (j & 3) : 16 * g + 2 * j;
+}
+
 template <int G, bool BF, int MIN_BLOCKS, bool TS>
 __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
@@ -195,8 +360,8 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     const int g = lane >> 2;  // fragment row group
     const int t = lane & 3;   // thread in group
 
-    const int part = blockIdx.x % p.num_partitions;
-    const int rest = blockIdx.x / p.num_partitions;
+    const int part = blockIdx.x % p.grid_partitions;
+    const int rest = blockIdx.x / p.grid_partitions;
     const int kvh = rest % p.num_kv_heads;
     const int seq_slot = rest / p.num_kv_heads;
     const int seq = p.seq_order ? __ldg(p.seq_order + seq_slot) : seq_slot;
@@ -213,10 +378,22 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
     const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
-    const int start = part * p.partition_tokens;
+    // Shared-prefix mode: this kernel attends tokens [P, ctx) of the sequence
+    // (its group's shared prefix is the prefix kernel's) and always writes a
+    // partial, to slot part + 1.
+    int P = 0;
+    if (p.cu_group_seqs && !bad_len) {
+        P = prefix_of(p, seq, ctx);
+        if (P < 0) {  // the merge writes zeros for this sequence
+            if (tid == 0 && part == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+            return;
+        }
+    }
+    const int pslot = part + (p.cu_group_seqs ? 1 : 0);
+    const int start = P + part * p.partition_tokens;
     const int end = bad_len ? start : min(start + p.partition_tokens, ctx);
-    const int n_parts_seq = bad_len ? 1 : (ctx + p.partition_tokens - 1) / p.partition_tokens;
-    const bool single = n_parts_seq == 1;
+    const int n_parts_seq = bad_len ? 1 : (ctx - P + p.partition_tokens - 1) / p.partition_tokens;
+    const bool single = n_parts_seq == 1 && !p.cu_group_seqs;
     if (!bad_len && start >= end) return;
     if (bad_len && part != 0) return;
 
@@ -248,7 +425,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
             for (int i = tid; i < G * D; i += T::kThreads)
                 p.out[(row * p.num_q_heads + qh0) * D + i] = __float2bfloat16_rn(0.f);
         } else if (tid < G) {
-            float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + tid) * p.num_partitions + part) * 2;
+            float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + tid) * p.num_partitions + pslot) * 2;
             ml[0] = -CUDART_INF_F;
             ml[1] = 0.f;
         }
@@ -303,52 +480,10 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     // qf[i][0] = dims 32t + 4i, +1; qf[i][1] = dims 32t + 4i + 2, +3 (zero
     // for g >= G). Scaled by 2^k so that the largest |q| of the KV head's
     // group lies in [2^14, 2^15): exact for bf16 q down to 2^-29 of it.
-    // bf16: q stays bf16 (exact), k-step i takes dims 16t + 4i .. + 3 (i < 4)
-    // and 64 + 16t + 4(i - 4) .. + 3 (i >= 4), the words of two 16-byte chunks
-    // of each half.
     uint32_t qf[8][2];
-    float score_scale;
-    {
-        uint32_t qw[16];
-        if (g < G) {
-            const __nv_bfloat16 *qrow = p.q + (row * p.num_q_heads + qh0 + g) * D;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e0 = BF ? (i >> 1) * 64 + 16 * t + (i & 1) * 8 : 32 * t + 8 * i;
-                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qrow + e0));
-                qw[4 * i] = w.x;
-                qw[4 * i + 1] = w.y;
-                qw[4 * i + 2] = w.z;
-                qw[4 * i + 3] = w.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) qw[i] = 0u;
-        }
-      if constexpr (BF) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            qf[i][0] = qw[2 * i];
-            qf[i][1] = qw[2 * i + 1];
-        }
-        score_scale = p.qk_scale_log2;
-      } else {
-        float mx = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        int e = 0;
-        frexpf(mx, &e);  // mx < 2^e
-        const int k = 15 - e;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            qf[i][0] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i]), k), ldexpf(bf16hi(qw[2 * i]), k));
-            qf[i][1] = tc::pack_f16(ldexpf(bf16lo(qw[2 * i + 1]), k), ldexpf(bf16hi(qw[2 * i + 1]), k));
-        }
-        score_scale = ldexpf(TS ? p.qk_scale_log2 : p.qk_scale_log2 * __ldg(p.k_scale + kvh), -k);
-      }
-    }
+    const float score_scale = load_q_frags<BF>(
+        g < G ? p.q + (row * p.num_q_heads + qh0 + g) * D : nullptr, t,
+        (BF || TS) ? p.qk_scale_log2 : p.qk_scale_log2 * __ldg(p.k_scale + kvh), qf);
 
     float o[8][4];
 #pragma unroll
@@ -359,9 +494,6 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
     float l[2] = {0.f, 0.f};
     int vexp = -100000;  // TS: weights are scaled by 2^-vexp before rounding
     float vinv = 0.f;    // 2^-vexp
-
-    // Swizzled row r, 16-byte chunk c of a 16-row group at byte address base.
-    auto sw = [](uint32_t base, int r, int c) { return base + r * 128 + (((c ^ r) & 7) << 4); };
 
     bool ok = true;
     int s = 0, rnd = 0;
@@ -382,37 +514,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
 #pragma unroll
         for (int gi = 0; gi < NGW; ++gi) {
             float c[4] = {0.f, 0.f, 0.f, 0.f};
-            if (gi * 16 < nv) {
-                const uint32_t kg = sk + gi * T::kGroupBytes;
-                if constexpr (BF) {
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const uint4 k0 = lds128(sw(kg + hh * 2048, g, 2 * t));
-                        const uint4 k1 = lds128(sw(kg + hh * 2048, g, 2 * t + 1));
-                        const uint4 k2 = lds128(sw(kg + hh * 2048, g + 8, 2 * t));
-                        const uint4 k3 = lds128(sw(kg + hh * 2048, g + 8, 2 * t + 1));
-                        const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                        const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            mma_bf16_16816(c, wg[2 * i], wh[2 * i], wg[2 * i + 1], wh[2 * i + 1], qf[4 * hh + i][0],
-                                           qf[4 * hh + i][1]);
-                    }
-                } else {
-                    const uint4 k0 = lds128(sw(kg, g, 2 * t));
-                    const uint4 k1 = lds128(sw(kg, g, 2 * t + 1));
-                    const uint4 k2 = lds128(sw(kg, g + 8, 2 * t));
-                    const uint4 k3 = lds128(sw(kg, g + 8, 2 * t + 1));
-                    const uint32_t wg[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                    const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint2 a = tc::e4m3x4_to_f16x4(wg[i]);  // row g: dims +0,+1 | +2,+3
-                        const uint2 b = tc::e4m3x4_to_f16x4(wh[i]);  // row g + 8
-                        mma_f16_16816(c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
-                    }
-                }
-            }
+            if (gi * 16 < nv) qk_group<BF>(sk + gi * T::kGroupBytes, g, t, qf, c);
             float ks0 = score_scale, ks1 = score_scale;
             if constexpr (TS) {
                 ks0 *= lds32f(ssc + (gi * 16 + g) * 4);
@@ -513,70 +615,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
         // ---- P V
 #pragma unroll
         for (int gi = 0; gi < NGW; ++gi) {
-            if (gi * 16 >= nv) continue;
-            const uint32_t vg = sv + gi * T::kGroupBytes;
-            if constexpr (BF) {
-                // weights as bf16 hi + lo: p - hi is exact in fp32 and lo keeps
-                // the next 8 bits
-                const uint32_t h01 = tc::pack_bf16(pw[gi][0], pw[gi][1]), h23 = tc::pack_bf16(pw[gi][2], pw[gi][3]);
-                const uint32_t l01 = tc::pack_bf16(pw[gi][0] - bf16lo(h01), pw[gi][1] - bf16hi(h01));
-                const uint32_t l23 = tc::pack_bf16(pw[gi][2] - bf16lo(h23), pw[gi][3] - bf16hi(h23));
-                const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
-                const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint32_t vh = vg + hh * 2048;
-                    uint4 r0 = lds128(sw(vh, 2 * t, g));
-                    uint4 r1 = lds128(sw(vh, 2 * t + 1, g));
-                    uint4 r2 = lds128(sw(vh, 2 * t + 8, g));
-                    uint4 r3 = lds128(sw(vh, 2 * t + 9, g));
-                    if (gi * 16 + 16 > nv) {  // rows past the end: zero (stale slots may hold NaN)
-                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                        if (gi * 16 + 2 * t >= nv) r0 = z;
-                        if (gi * 16 + 2 * t + 1 >= nv) r1 = z;
-                        if (gi * 16 + 2 * t + 8 >= nv) r2 = z;
-                        if (gi * 16 + 2 * t + 9 >= nv) r3 = z;
-                    }
-                    const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
-                    const uint32_t w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
-#pragma unroll
-                    for (int qd = 0; qd < 4; ++qd) {
-                        // dims 64hh + 8g + 2qd, + 1 of tokens (2t, 2t+1) and (2t+8, 2t+9)
-                        const uint32_t a0 = __byte_perm(w0[qd], w1[qd], 0x5410);
-                        const uint32_t a1 = __byte_perm(w0[qd], w1[qd], 0x7632);
-                        const uint32_t a2 = __byte_perm(w2[qd], w3[qd], 0x5410);
-                        const uint32_t a3 = __byte_perm(w2[qd], w3[qd], 0x7632);
-                        mma_bf16_16816(o[4 * hh + qd], a0, a1, a2, a3, bh0, bh1);
-                        mma_bf16_16816(o[4 * hh + qd], a0, a1, a2, a3, bl0, bl1);
-                    }
-                }
-                continue;
-            }
-            const uint32_t b0 = movmatrix_trans(tc::pack_f16(pw[gi][0], pw[gi][1]));  // tokens 2t, 2t+1 of head g
-            const uint32_t b1 = movmatrix_trans(tc::pack_f16(pw[gi][2], pw[gi][3]));  // tokens 2t+8, 2t+9
-            uint4 r0 = lds128(sw(vg, 2 * t, g));
-            uint4 r1 = lds128(sw(vg, 2 * t + 1, g));
-            uint4 r2 = lds128(sw(vg, 2 * t + 8, g));
-            uint4 r3 = lds128(sw(vg, 2 * t + 9, g));
-            if (gi * 16 + 16 > nv) {  // rows past the end: zero codes (stale slots may hold NaN)
-                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                if (gi * 16 + 2 * t >= nv) r0 = z;
-                if (gi * 16 + 2 * t + 1 >= nv) r1 = z;
-                if (gi * 16 + 2 * t + 8 >= nv) r2 = z;
-                if (gi * 16 + 2 * t + 9 >= nv) r3 = z;
-            }
-            const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
-            const uint32_t w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-                // dims 16g + 4qd .. +3 of tokens (2t, 2t+1) and (2t+8, 2t+9)
-                const uint2 x0 = tc::e4m3x4_to_f16x4(__byte_perm(w0[qd], w1[qd], 0x5140));
-                const uint2 x1 = tc::e4m3x4_to_f16x4(__byte_perm(w0[qd], w1[qd], 0x7362));
-                const uint2 y0 = tc::e4m3x4_to_f16x4(__byte_perm(w2[qd], w3[qd], 0x5140));
-                const uint2 y1 = tc::e4m3x4_to_f16x4(__byte_perm(w2[qd], w3[qd], 0x7362));
-                mma_f16_16816(o[2 * qd], x0.x, x0.y, y0.x, y0.y, b0, b1);
-                mma_f16_16816(o[2 * qd + 1], x1.x, x1.y, y1.x, y1.y, b0, b1);
-            }
+            if (gi * 16 < nv) pv_group<BF>(sv + gi * T::kGroupBytes, g, t, pw[gi], nv - gi * 16, o);
         }
         __syncwarp();
         if (lane == 0) {
@@ -623,7 +662,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
 #pragma unroll
             for (int jj = 0; jj < 8; jj += 2) {
                 // m-tiles jj, jj + 1 hold dims e, e + 1, e + 2, e + 3
-                const int e = BF ? (jj >> 2) * 64 + 8 * g + 2 * (jj & 3) : 16 * g + 2 * jj;
+                const int e = acc_dim<BF>(jj, g);
                 *reinterpret_cast<float4 *>(dst + e) =
                     make_float4(o[jj][h] * sc, o[jj][2 + h] * sc, o[jj + 1][h] * sc, o[jj + 1][2 + h] * sc);
             }
@@ -648,7 +687,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
         if constexpr (!TS && !BF) post *= __ldg(p.v_scale + kvh);
         for (int w = 0; w < NW; ++w) merge_w[w * G + h] *= post;
         if (!single) {
-            float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * 2;
+            float *ml = p.part_ml + (((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + pslot) * 2;
             ml[0] = M;
             ml[1] = L;
         }
@@ -662,7 +701,7 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
         if (single) {
             p.out[(row * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(acc);
         } else {
-            p.part_o[(((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + part) * D + (idx % D)] = acc;
+            p.part_o[(((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + pslot) * D + (idx % D)] = acc;
         }
     }
 }
