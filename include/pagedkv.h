@@ -238,6 +238,53 @@ PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const
                                size_t workspace_bytes, void *out, int *dev_err, void *stream);
 
 /*
+ * pkv_paged_attention_decode_shared_prefix: the same decode for a batch
+ * whose sequences share cached prefixes, computed as a cascade. Blocks that
+ * several requests share (prefix caching: "Nano-vLLM：轻量高效的大模型推理框架",
+ * section 三.2(1) 前缀缓存; sharing within and across requests:
+ * "DeepSeek复刻vLLM反超原版：AI推理新标杆", section "vLLM：大模型推理的加速引擎
+ * 与挑战") are then read and multiplied once per group of members instead of
+ * once per sequence: a prefix kernel attends each group's shared tokens for
+ * up to 32 query rows at a time, the decode kernel attends each sequence's
+ * own tokens, and the split-K merge combines the two (out is the same
+ * attention as pkv_paged_attention_decode, to rounding).
+ *
+ *  cu_group_seqs        [num_groups + 1] int32, device: group j is
+ *                       sequences cu_group_seqs[j] .. cu_group_seqs[j+1] - 1
+ *                       (consecutive in the batch; the groups cover it in
+ *                       order, single sequences are groups of one)
+ *  group_prefix_tokens  [num_groups] int32, device: P_j, the number of
+ *                       leading tokens every member of group j shares: a
+ *                       multiple of block_size, at most each member's
+ *                       context length, and the members' block-table
+ *                       entries 0 .. P_j / block_size - 1 are the same
+ *                       physical blocks (0: nothing shared)
+ *  max_group_seqs       host-known bound on the group sizes (sizes the grid)
+ *  workspace            at least pkv_plan_decode_shared_prefix's
+ *                       workspace_bytes (the prefix partial is one more
+ *                       split-K slot per (sequence, query head)), 256-byte
+ *                       aligned
+ *  other arguments as pkv_paged_attention_decode (no seq_order)
+ *
+ * Device checks: a P_j that is not a multiple of block_size or exceeds a
+ * member's context, a member whose shared block ids differ from the first
+ * member's, or groups that do not lie inside the batch set
+ * PKV_DEVERR_BOUNDS and the affected sequences' out rows are written as
+ * zeros (where they can be located). head_dim 64, or num_groups == 0,
+ * run the ordinary decode (same result).
+ */
+PKV_API int pkv_plan_decode_shared_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                          int block_size, int max_context_len, int cache_dtype,
+                                          int partition_request, pkv_decode_plan *plan);
+PKV_API int pkv_paged_attention_decode_shared_prefix(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+    const int32_t *context_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int64_t num_blocks, float scale, int cache_dtype, const float *k_scale, const float *v_scale,
+    int max_context_len, const int32_t *cu_group_seqs, const int32_t *group_prefix_tokens, int num_groups,
+    int max_group_seqs, int partition_request, void *workspace, size_t workspace_bytes, void *out, int *dev_err,
+    void *stream);
+
+/*
  * pkv_paged_attention_decode_static_scratch: pkv_paged_attention_decode for
  * callers that cannot allocate device memory -- for example an engine that
  * reserves all device memory for its KV pool at start-up and forbids later

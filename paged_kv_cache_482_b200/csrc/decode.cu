@@ -69,7 +69,7 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    const long long blocks = (long long)p.num_seqs * p.num_kv_heads * p.num_partitions;
+    const long long blocks = (long long)p.num_seqs * p.num_kv_heads * p.grid_partitions;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // tensor-map row coordinates are int32
@@ -84,9 +84,29 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
                            : make_e4m3_pool_map(&mk, p.k_cache, rows, box_rows) &&
                                  make_e4m3_pool_map(&mv, p.v_cache, rows, box_rows);
     if (!mapped) return cudaErrorInvalidValue;
+    if (p.cu_group_seqs) {  // the shared prefixes first: slot 0 of every member
+        using PT = PrefixTraits<BF>;
+        auto pk = paged_prefix_mma_kernel<G, BF, TS>;
+        static std::atomic<unsigned long long> configured_prefix{0};
+        if (!(configured_prefix.load(std::memory_order_acquire) & bit)) {
+            e = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, PT::kAlloc);
+            if (e != cudaSuccess) return e;
+            configured_prefix.fetch_or(bit, std::memory_order_acq_rel);
+        }
+        const int per_block = PT::kNW * (8 / G);
+        const long long chunks = ((long long)p.max_group_seqs + per_block - 1) / per_block;
+        const long long gx = chunks * p.num_groups;
+        if (gx > 0x7fffffffLL || p.num_kv_heads > 65535) return cudaErrorInvalidConfiguration;
+        if (gx > 0) {
+            pk<<<dim3((unsigned)gx, (unsigned)p.num_kv_heads), PT::kThreads, PT::kAlloc, stream>>>(p, mk, mv, box_rows,
+                                                                                                  (int)chunks);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+    }
     kern<<<(unsigned)blocks, T::kThreads, T::kAlloc, stream>>>(p, mk, mv, box_rows);
     e = cudaGetLastError();
-    if (e != cudaSuccess || p.num_partitions <= 1) return e;
+    if (e != cudaSuccess || (p.num_partitions <= 1 && !p.cu_group_seqs)) return e;
     paged_decode_reduce_kernel<128><<<(unsigned)((long long)p.num_seqs * p.num_q_heads), 128, 0, stream>>>(p);
     return cudaGetLastError();
 }
@@ -170,12 +190,21 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.max_context_len = a.max_context_len;
     p.partition_tokens = a.partition_tokens > 0 ? a.partition_tokens : a.max_context_len;
     p.num_partitions = a.partition_tokens > 0 ? a.num_partitions : 1;
+    if (a.cu_group_seqs) {  // slot 0 holds the shared prefix; the grid covers the suffix partitions
+        if (a.head_dim != 128) return cudaErrorInvalidValue;
+        p.num_partitions = a.num_partitions;
+    }
     p.part_o = a.part_o;
     p.part_ml = a.part_ml;
     p.out = static_cast<__nv_bfloat16 *>(a.out);
     p.dev_err = a.dev_err;
     p.cu_q_lens = a.cu_q_lens;
     p.total_q = a.total_q;
+    p.cu_group_seqs = a.cu_group_seqs;
+    p.group_prefix = a.group_prefix;
+    p.num_groups = a.num_groups;
+    p.max_group_seqs = a.max_group_seqs;
+    p.grid_partitions = a.cu_group_seqs ? p.num_partitions - 1 : p.num_partitions;
     const int group = a.num_q_heads / a.num_kv_heads;
     if (a.fp8 && a.head_dim == 128) return a.token_scales ? launch_mma<false, true>(group, p, stream)
                                                           : launch_mma<false, false>(group, p, stream);

@@ -329,6 +329,103 @@ __device__ __forceinline__ void pv_group(uint32_t vg, int g, int t, const float 
     }
 }
 
+// Softmax of one tile of NG groups in base 2 for the lane's columns 2t, 2t + 1:
+// x holds the scaled scores (-inf past the end). The reference maximum moves
+// only when the tile maximum exceeds it by more than 8 (so weights stay below
+// 2^8); alpha receives the factor the accumulators must take (1 when nothing
+// moved, in every lane when the return value is false), l is rescaled and
+// takes the new weights pw.
+template <int NG>
+__device__ __forceinline__ bool tile_softmax(const float (&x)[NG][4], float (&m_ref)[2], float (&l)[2],
+                                             float (&alpha)[2], float (&pw)[NG][4]) {
+    float mx[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(x[0][h], x[0][2 + h]);
+#pragma unroll
+        for (int gi = 1; gi < NG; ++gi) mx[h] = fmaxf(mx[h], fmaxf(x[gi][h], x[gi][2 + h]));
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+    }
+    const bool move = mx[0] > m_ref[0] + 8.f || mx[1] > m_ref[1] + 8.f;
+    alpha[0] = alpha[1] = 1.f;
+    const bool rescale = __any_sync(0xffffffffu, move);
+    if (rescale) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float mn = fmaxf(m_ref[h], mx[h]);
+            alpha[h] = m_ref[h] == -CUDART_INF_F ? 0.f : fast_exp2(m_ref[h] - mn);
+            m_ref[h] = mn;
+        }
+    }
+    const float mr0 = m_ref[0] == -CUDART_INF_F ? 0.f : m_ref[0];
+    const float mr1 = m_ref[1] == -CUDART_INF_F ? 0.f : m_ref[1];
+    l[0] *= alpha[0];
+    l[1] *= alpha[1];
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+        pw[gi][0] = fast_exp2(x[gi][0] - mr0);
+        pw[gi][1] = fast_exp2(x[gi][1] - mr1);
+        pw[gi][2] = fast_exp2(x[gi][2] - mr0);
+        pw[gi][3] = fast_exp2(x[gi][3] - mr1);
+        l[0] += pw[gi][0] + pw[gi][2];
+        l[1] += pw[gi][1] + pw[gi][3];
+    }
+    return rescale;
+}
+
+// Per-token V scales (E4M3 with scale pools): the scales of the lane's rows
+// g, g + 8 of each group sit at vs_addr + 4 * row (0 past nv). A tile maximum
+// at or above 2^vexp raises vexp and folds the exact factor 2^-rise into
+// alpha, so that the weights times 2^-vexp stay below 2^9 in f16; the weights
+// are multiplied by their token's scale times 2^-vexp.
+template <int NG>
+__device__ __forceinline__ bool tile_vscale(uint32_t vs_addr, int nv, int g, int &vexp, float &vinv,
+                                            float (&alpha)[2], float (&pw)[NG][4]) {
+    float vsc[NG][2];
+    float vm = 0.f;
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+        const bool v0 = gi * 16 + g < nv, v1 = gi * 16 + g + 8 < nv;
+        vsc[gi][0] = v0 ? lds32f(vs_addr + (gi * 16 + g) * 4) : 0.f;
+        vsc[gi][1] = v1 ? lds32f(vs_addr + (gi * 16 + g + 8) * 4) : 0.f;
+        vm = fmaxf(vm, fmaxf(vsc[gi][0], vsc[gi][1]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+    // vm < 2^ev (vm >= the smallest normal: scales are floored there, and the
+    // tile has a valid token); the same in every lane
+    const int ev = (int)(__float_as_uint(vm) >> 23) - 126;
+    bool rise = false;
+    if (ev > vexp) {
+        const float f = ldexpf(1.f, vexp - ev);  // 0 for the first rise
+        alpha[0] *= f;
+        alpha[1] *= f;
+        rise = true;
+        vexp = ev;
+        vinv = ldexpf(1.f, -vexp);
+    }
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+        const float f0 = vsc[gi][0] * vinv, f1 = vsc[gi][1] * vinv;
+        pw[gi][0] *= f0;
+        pw[gi][1] *= f0;
+        pw[gi][2] *= f1;
+        pw[gi][3] *= f1;
+    }
+    return rise;
+}
+
+__device__ __forceinline__ void rescale_acc(float (&o)[8][4], const float (&alpha)[2]) {
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+        o[jj][0] *= alpha[0];
+        o[jj][1] *= alpha[1];
+        o[jj][2] *= alpha[0];
+        o[jj][3] *= alpha[1];
+    }
+}
+
 // Dim held by accumulator o[j][0..1] (o[j][2..3]: the next dim) of row
 // group g: 16g + 2j (E4M3) or 64(j / 4) + 8g + 2(j % 4) (bf16).
 template <bool BF>
@@ -527,91 +624,14 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
             x[gi][2] = v1 ? c[2] * ks1 : -CUDART_INF_F;
             x[gi][3] = v1 ? c[3] * ks1 : -CUDART_INF_F;
         }
-        // ---- tile maximum per head, lazy reference maximum
-        float mx[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            mx[h] = fmaxf(x[0][h], x[0][2 + h]);
-#pragma unroll
-            for (int gi = 1; gi < NGW; ++gi) mx[h] = fmaxf(mx[h], fmaxf(x[gi][h], x[gi][2 + h]));
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
-        }
-        const bool move = mx[0] > m_ref[0] + 8.f || mx[1] > m_ref[1] + 8.f;
-        float alpha[2] = {1.f, 1.f};
-        bool rescale = __any_sync(0xffffffffu, move);
-        if (rescale) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float mn = fmaxf(m_ref[h], mx[h]);
-                alpha[h] = m_ref[h] == -CUDART_INF_F ? 0.f : fast_exp2(m_ref[h] - mn);
-                m_ref[h] = mn;
-            }
-        }
-        const float mr0 = m_ref[0] == -CUDART_INF_F ? 0.f : m_ref[0];
-        const float mr1 = m_ref[1] == -CUDART_INF_F ? 0.f : m_ref[1];
-        l[0] *= alpha[0];
-        l[1] *= alpha[1];
-        float pw[NGW][4];
-#pragma unroll
-        for (int gi = 0; gi < NGW; ++gi) {
-            pw[gi][0] = fast_exp2(x[gi][0] - mr0);
-            pw[gi][1] = fast_exp2(x[gi][1] - mr1);
-            pw[gi][2] = fast_exp2(x[gi][2] - mr0);
-            pw[gi][3] = fast_exp2(x[gi][3] - mr1);
-            l[0] += pw[gi][0] + pw[gi][2];
-            l[1] += pw[gi][1] + pw[gi][3];
-        }
-
+        float alpha[2], pw[NGW][4];
+        bool rescale = tile_softmax<NGW>(x, m_ref, l, alpha, pw);
         if (!mbar_wait(&full_v[s], rnd & 1)) {
             ok = false;
             break;
         }
-        if constexpr (TS) {
-            // V scales of the thread's tokens (rows g, g + 8 of each group; 0
-            // past the end). A tile maximum at or above 2^vexp raises vexp and
-            // rescales the accumulators by 2^-rise (exact), so that the
-            // weights times 2^-vexp stay below 2^9 in f16.
-            float vsc[NGW][2];
-            float vm = 0.f;
-#pragma unroll
-            for (int gi = 0; gi < NGW; ++gi) {
-                const bool v0 = gi * 16 + g < nv, v1 = gi * 16 + g + 8 < nv;
-                vsc[gi][0] = v0 ? lds32f(ssc + WT * 4 + (gi * 16 + g) * 4) : 0.f;
-                vsc[gi][1] = v1 ? lds32f(ssc + WT * 4 + (gi * 16 + g + 8) * 4) : 0.f;
-                vm = fmaxf(vm, fmaxf(vsc[gi][0], vsc[gi][1]));
-            }
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-            // vm < 2^ev (vm >= the smallest normal: scales are floored there,
-            // and the tile has a valid token); the same in every lane
-            const int ev = (int)(__float_as_uint(vm) >> 23) - 126;
-            if (ev > vexp) {
-                const float f = ldexpf(1.f, vexp - ev);  // 0 for the first rise
-                alpha[0] *= f;
-                alpha[1] *= f;
-                rescale = true;
-                vexp = ev;
-                vinv = ldexpf(1.f, -vexp);
-            }
-#pragma unroll
-            for (int gi = 0; gi < NGW; ++gi) {
-                const float f0 = vsc[gi][0] * vinv, f1 = vsc[gi][1] * vinv;
-                pw[gi][0] *= f0;
-                pw[gi][1] *= f0;
-                pw[gi][2] *= f1;
-                pw[gi][3] *= f1;
-            }
-        }
-        if (rescale) {
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                o[jj][0] *= alpha[0];
-                o[jj][1] *= alpha[1];
-                o[jj][2] *= alpha[0];
-                o[jj][3] *= alpha[1];
-            }
-        }
+        if constexpr (TS) rescale |= tile_vscale<NGW>(ssc + WT * 4, nv, g, vexp, vinv, alpha, pw);
+        if (rescale) rescale_acc(o, alpha);
         // ---- P V
 #pragma unroll
         for (int gi = 0; gi < NGW; ++gi) {
@@ -702,6 +722,276 @@ __global__ void __launch_bounds__(MmaTraits<G, BF>::kThreads, MIN_BLOCKS)
             p.out[(row * p.num_q_heads + qh0) * D + idx] = __float2bfloat16_rn(acc);
         } else {
             p.part_o[(((long long)seq * p.num_q_heads + qh0 + h) * p.num_partitions + pslot) * D + (idx % D)] = acc;
+        }
+    }
+}
+
+// ------------------------------------------------------- shared prefixes
+//
+// Shared-prefix (cascade) decode, the prefix half. Sequences that share
+// their first P cached tokens (the same physical blocks: prefix caching,
+// "Nano-vLLM：轻量高效的大模型推理框架", section 三.2(1) 前缀缓存; sharing across
+// requests, "DeepSeek复刻vLLM反超原版", section "vLLM：大模型推理的加速引擎与挑战")
+// attend those tokens here once per group of member sequences instead of
+// once each: a thread block takes up to 4 * (8 / G) members of one group and
+// one KV head; a producer warp copies the prefix tile by tile (the same
+// tensor-map boxes as the decode kernel) into a ring that every consumer
+// warp reads; consumer warp w computes the 8 columns (member, head) of its
+// 8 / G members with the decode kernel's per-group MMA code, so each K/V
+// fragment read from shared memory serves 8 query rows and each tile read
+// from L2 or HBM serves all the block's members. Each member gets its
+// prefix partial (normalised O, max, sum) in split-K slot 0; the decode
+// kernel writes the suffix partials and the merge combines them.
+//
+// Checks (PKV_DEVERR_BOUNDS; the member's partial gets sum 0, which makes the
+// merge write zeros): P a whole number of blocks within the table, the
+// leader's block ids inside the pool, every member's context at least P and
+// every member's first P / block_size block ids equal to the leader's.
+
+template <bool BF>
+struct PrefixTraits {
+    static constexpr int kNW = 4;  // consumer warps; warp kNW issues the copies
+    static constexpr int kThreads = (kNW + 1) * 32;
+    static constexpr int kRowBytes = BF ? 256 : 128;
+    static constexpr int kHalves = BF ? 2 : 1;
+    static constexpr int kGroupBytes = 16 * kRowBytes;
+    static constexpr int kNG = BF ? 2 : 4;  // 16-token groups per stage
+    static constexpr int kTT = 16 * kNG;    // tokens per stage
+    static constexpr int kStages = 4;
+    static constexpr int kHalfBytes = kNG * kGroupBytes;  // K (or V) of one stage
+    static constexpr int kStageBytes = 2 * kHalfBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kOffScales = kRingBytes;  // [stage][K | V][kTT] fp32
+    static constexpr int kOffBars = kOffScales + kStages * 2 * kTT * 4;  // full_k[S], full_v[S], empty[S]
+    static constexpr int kOffFlags = kOffBars + 3 * kStages * 8;
+    static constexpr int kOffIds = kOffFlags + 16;
+    static constexpr int kSmemBytes = kOffIds + kMaxIdsPerPartition * 4;
+    static constexpr int kAlloc = kSmemBytes + 1024;
+};
+
+template <int G, bool BF, bool TS>
+__global__ void __launch_bounds__(PrefixTraits<BF>::kThreads, 1)
+    paged_prefix_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
+                            const __grid_constant__ CUtensorMap map_v, int box_rows, int max_chunks) {
+    static_assert(!(BF && TS), "per-token scales exist only for E4M3");
+    using T = PrefixTraits<BF>;
+    constexpr int D = 128;
+    constexpr int NW = T::kNW;
+    constexpr int NG = T::kNG;
+    constexpr int TT = T::kTT;
+    constexpr int STAGES = T::kStages;
+    constexpr int SPW = 8 / G;        // member sequences per consumer warp
+    constexpr int MC = NW * SPW;      // member sequences per block
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
+    uint8_t *smem = smem_raw + pad;
+    const uint32_t sbase = smem_addr(smem);
+    int32_t *ids = reinterpret_cast<int32_t *>(smem + T::kOffIds);
+    unsigned *bad_mask = reinterpret_cast<unsigned *>(smem + T::kOffFlags);
+    uint64_t *full_k = reinterpret_cast<uint64_t *>(smem + T::kOffBars);
+    uint64_t *full_v = full_k + STAGES;
+    uint64_t *empty = full_v + STAGES;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int g = lane >> 2;
+    const int t = lane & 3;
+    const int grp = blockIdx.x / max_chunks;
+    const int chunk = blockIdx.x % max_chunks;
+    const int kvh = blockIdx.y;
+    if (grp >= p.num_groups) return;
+    const int m0 = __ldg(p.cu_group_seqs + grp), m1 = __ldg(p.cu_group_seqs + grp + 1);
+    if (m0 < 0 || m1 < m0 || m1 > p.num_seqs) {  // members cannot be located safely
+        if (tid == 0 && chunk == 0 && kvh == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+        return;
+    }
+    const int first = m0 + chunk * MC;
+    if (first >= m1) return;
+    const int last = min(first + MC, m1);
+    const int P = __ldg(p.group_prefix + grp);
+    if (P == 0) return;  // nothing shared: the decode kernel attends every token
+
+    const int lbs = p.log2_block_size;
+    const int bs_mask = p.block_size - 1;
+    const int table_cap = p.max_blocks_per_seq << lbs;
+    const bool p_ok = P > 0 && (P & bs_mask) == 0 && P <= table_cap;
+    const int n_blk = p_ok ? P >> lbs : 0;
+    const int32_t *lead = p.block_tables + (long long)m0 * p.max_blocks_per_seq;
+    if (tid == 0) *bad_mask = 0u;
+    __syncthreads();
+    int bad_all = !p_ok;
+    for (int i = tid; i < n_blk; i += T::kThreads) {
+        const int32_t id = __ldg(lead + i);
+        if (i < kMaxIdsPerPartition) ids[i] = id;
+        bad_all |= (id < 0 || (long long)id >= p.num_blocks);
+    }
+    for (int mi = 0; mi < last - first; ++mi) {
+        const int m = first + mi;
+        const int32_t *row = p.block_tables + (long long)m * p.max_blocks_per_seq;
+        int bad_m = 0;
+        if (tid == 0) {
+            const int c = __ldg(p.context_lens + m);
+            bad_m = c < P || c > p.max_context_len || c > table_cap;
+        }
+        for (int i = tid; i < n_blk; i += T::kThreads) bad_m |= __ldg(row + i) != __ldg(lead + i);
+        if (bad_m) atomicOr(bad_mask, 1u << mi);
+    }
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_k[s], 1);
+            mbar_init(&full_v[s], 1);
+            mbar_init(&empty[s], NW);
+        }
+        fence_barrier_init();
+    }
+    bad_all = __syncthreads_or(bad_all);
+    const unsigned bmask = *bad_mask;
+    const int qh0 = kvh * G;
+    if (bad_all || bmask) {
+        if (tid == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+    }
+    if (bad_all) {  // every member's prefix partial: sum 0 (the merge writes zeros)
+        for (int i = tid; i < (last - first) * G; i += T::kThreads) {
+            float *ml = p.part_ml + (((long long)(first + i / G) * p.num_q_heads + qh0 + i % G) * p.num_partitions) * 2;
+            ml[0] = -CUDART_INF_F;
+            ml[1] = 0.f;
+        }
+        return;
+    }
+
+    const int n_tiles = (P + TT - 1) / TT;
+    if (warp == NW) {  // ------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % STAGES;
+                if (j >= STAGES && !mbar_wait(&empty[s], ((j / STAGES) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int a0 = j * TT;
+                const int nv = min(P - a0, TT);
+                uint32_t bytes = 0;
+                for (int a = 0; a < nv; a += box_rows) bytes += box_rows * T::kRowBytes + (TS ? box_rows * 4 : 0);
+                mbar_arrive_expect_tx(&full_k[s], bytes);
+                mbar_arrive_expect_tx(&full_v[s], bytes);
+                const uint32_t sk = sbase + s * T::kStageBytes;
+                const uint32_t sv = sk + T::kHalfBytes;
+                for (int a = 0; a < nv; a += box_rows) {
+                    const int tok = a0 + a;
+                    const int bi = tok >> lbs;
+                    const long long phys = bi < kMaxIdsPerPartition ? ids[bi] : __ldg(lead + bi);
+                    const long long row = (phys * p.num_kv_heads + kvh) * p.block_size + (tok & bs_mask);
+                    const uint32_t dst = (a >> 4) * T::kGroupBytes + (a & 15) * 128;
+#pragma unroll
+                    for (int hh = 0; hh < T::kHalves; ++hh) {
+                        tc::tma_load_2d(sk + dst + hh * 2048, &map_k, hh * 64, (int)row, &full_k[s]);
+                        tc::tma_load_2d(sv + dst + hh * 2048, &map_v, hh * 64, (int)row, &full_v[s]);
+                    }
+                    if constexpr (TS) {
+                        uint8_t *sc = smem + T::kOffScales + s * 2 * TT * 4;
+                        bulk_g2s(sc + a * 4, p.k_scale + row, box_rows * 4, &full_k[s]);
+                        bulk_g2s(sc + TT * 4 + a * 4, p.v_scale + row, box_rows * 4, &full_v[s]);
+                    }
+                }
+                issued = j + 1;
+            }
+            if (!ok) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+            // copies still in flight (only when the consumers gave up)
+            for (int jj = max(0, issued - STAGES); jj < issued; ++jj) {
+                const uint32_t par = (jj / STAGES) & 1;
+                if (!mbar_wait(&full_k[jj % STAGES], par) || !mbar_wait(&full_v[jj % STAGES], par))
+                    set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+            }
+        }
+        return;  // no block-wide barrier follows
+    }
+
+    // ------------------------------------------------------------ consumers
+    // column g of warp w: member first + w * SPW + g / G, head qh0 + g % G
+    const int my_member = first + warp * SPW + g / G;
+    uint32_t qf[8][2];
+    const float score_scale = load_q_frags<BF>(
+        my_member < last ? p.q + ((long long)my_member * p.num_q_heads + qh0 + g % G) * D : nullptr, t,
+        (BF || TS) ? p.qk_scale_log2 : p.qk_scale_log2 * __ldg(p.k_scale + kvh), qf);
+    float o[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[j][i] = 0.f;
+    float m_ref[2] = {-CUDART_INF_F, -CUDART_INF_F};
+    float l[2] = {0.f, 0.f};
+    int vexp = -100000;
+    float vinv = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % STAGES;
+        const uint32_t par = (j / STAGES) & 1;
+        const int nv = min(P - j * TT, TT);
+        if (!mbar_wait(&full_k[s], par)) {
+            ok = false;
+            break;
+        }
+        const uint32_t sk = sbase + s * T::kStageBytes;
+        const uint32_t sv = sk + T::kHalfBytes;
+        const uint32_t ssc = smem_addr(smem + T::kOffScales) + s * 2 * TT * 4;
+        float x[NG][4];
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            if (gi * 16 < nv) qk_group<BF>(sk + gi * T::kGroupBytes, g, t, qf, c);
+            float ks0 = score_scale, ks1 = score_scale;
+            if constexpr (TS) {
+                ks0 *= lds32f(ssc + (gi * 16 + g) * 4);
+                ks1 *= lds32f(ssc + (gi * 16 + g + 8) * 4);
+            }
+            const bool v0 = gi * 16 + g < nv, v1 = gi * 16 + g + 8 < nv;
+            x[gi][0] = v0 ? c[0] * ks0 : -CUDART_INF_F;
+            x[gi][1] = v0 ? c[1] * ks0 : -CUDART_INF_F;
+            x[gi][2] = v1 ? c[2] * ks1 : -CUDART_INF_F;
+            x[gi][3] = v1 ? c[3] * ks1 : -CUDART_INF_F;
+        }
+        float alpha[2], pw[NG][4];
+        bool rescale = tile_softmax<NG>(x, m_ref, l, alpha, pw);
+        if (!mbar_wait(&full_v[s], par)) {
+            ok = false;
+            break;
+        }
+        if constexpr (TS) rescale |= tile_vscale<NG>(ssc + TT * 4, nv, g, vexp, vinv, alpha, pw);
+        if (rescale) rescale_acc(o, alpha);
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi)
+            if (gi * 16 < nv) pv_group<BF>(sv + gi * T::kGroupBytes, g, t, pw[gi], nv - gi * 16, o);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (!ok) set_error(p.dev_err, PKV_DEVERR_TIMEOUT);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+    // each lane writes its two columns' dims of the slot-0 partial
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int col = 2 * t + h;
+        const int member = first + warp * SPW + col / G;
+        if (member >= last) continue;
+        const bool bad_m = ((bmask >> (member - first)) & 1u) || !ok;
+        const long long slot = ((long long)member * p.num_q_heads + qh0 + col % G) * p.num_partitions;
+        float inv = bad_m ? 0.f : 1.f / l[h];
+        if constexpr (TS) inv *= ldexpf(1.f, vexp);  // undo the 2^-vexp of the weights
+        if constexpr (!TS && !BF) inv *= __ldg(p.v_scale + kvh);
+        float *dst = p.part_o + slot * D;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const int e = acc_dim<BF>(jj, g);
+            *reinterpret_cast<float2 *>(dst + e) = make_float2(o[jj][h] * inv, o[jj][2 + h] * inv);
+        }
+        if (g == 0) {
+            p.part_ml[slot * 2] = bad_m ? -CUDART_INF_F : m_ref[h];
+            p.part_ml[slot * 2 + 1] = bad_m ? 0.f : l[h];
         }
     }
 }

@@ -183,6 +183,104 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, i
     return round_up(rows * head_dim * sizeof(float), 256) + round_up(rows * 2 * sizeof(float), 256);
 }
 
+namespace {
+
+// Plan of the shared-prefix decode: the suffix partitions of the ordinary
+// plan (one, of max_context_len tokens, when it does not split) plus slot 0.
+int make_shared_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_context_len, int cache_dtype, int request, pkv_decode_plan *plan) {
+    int st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, cache_dtype,
+                       request, plan);
+    if (st != PKV_OK) return st;
+    if (head_dim != 128) return PKV_OK;  // served by the ordinary decode (same result)
+    const int np_suffix = plan->partition_tokens > 0 ? plan->max_partitions : 1;
+    if (np_suffix + 1 > kMaxPartitions) return PKV_ERR_UNSUPPORTED;
+    if (plan->partition_tokens == 0) plan->partition_tokens = max_context_len;
+    plan->max_partitions = np_suffix + 1;
+    const size_t rows = (size_t)num_seqs * num_q_heads * plan->max_partitions;
+    plan->workspace_bytes = round_up(rows * head_dim * sizeof(float), 256) + round_up(rows * 2 * sizeof(float), 256);
+    return PKV_OK;
+}
+
+}  // namespace
+
+int pkv_plan_decode_shared_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int max_context_len, int cache_dtype, int partition_request,
+                                  pkv_decode_plan *plan) {
+    if (!plan) return PKV_ERR_INVALID_ARG;
+    return make_shared_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, cache_dtype,
+                            partition_request, plan);
+}
+
+int pkv_paged_attention_decode_shared_prefix(const void *q, const void *k_cache, const void *v_cache,
+                                             const int32_t *block_tables, int max_blocks_per_seq,
+                                             const int32_t *context_lens, int num_seqs, int num_q_heads,
+                                             int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                                             float scale, int cache_dtype, const float *k_scale,
+                                             const float *v_scale, int max_context_len,
+                                             const int32_t *cu_group_seqs, const int32_t *group_prefix_tokens,
+                                             int num_groups, int max_group_seqs, int partition_request,
+                                             void *workspace, size_t workspace_bytes, void *out, int *dev_err,
+                                             void *stream) {
+    if (num_groups < 0 || (num_groups > 0 && (!cu_group_seqs || !group_prefix_tokens || max_group_seqs < 1)))
+        return PKV_ERR_INVALID_ARG;
+    if (num_groups == 0 || head_dim != 128)  // nothing declared shared, or no prefix kernel for this head size
+        return pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                          nullptr, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                          num_blocks, scale, cache_dtype, k_scale, v_scale, max_context_len,
+                                          partition_request, workspace, workspace_bytes, out, dev_err, stream);
+    pkv_decode_plan plan;
+    int st = make_shared_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                              cache_dtype, partition_request, &plan);
+    if (st != PKV_OK) return st;
+    const bool fp8 = cache_dtype != PKV_CACHE_BF16;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PKV_ERR_INVALID_ARG;
+    if (fp8 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+    if (max_blocks_per_seq < 1 || num_blocks < 1 || num_blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size) return PKV_ERR_INVALID_ARG;
+    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return PKV_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+
+    pkv::DecodeArgs a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.context_lens = context_lens;
+    a.seq_order = nullptr;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_dim = head_dim;
+    a.block_size = block_size;
+    a.num_blocks = num_blocks;
+    a.scale = scale;
+    a.fp8 = fp8;
+    a.token_scales = cache_dtype == PKV_CACHE_FP8_E4M3_TOKEN;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.max_context_len = max_context_len;
+    a.partition_tokens = plan.partition_tokens;
+    a.num_partitions = plan.max_partitions;
+    const size_t rows = (size_t)num_seqs * num_q_heads * plan.max_partitions;
+    a.part_o = static_cast<float *>(workspace);
+    a.part_ml =
+        reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(rows * head_dim * sizeof(float), 256));
+    a.out = out;
+    a.dev_err = dev_err;
+    a.cu_group_seqs = cu_group_seqs;
+    a.group_prefix = group_prefix_tokens;
+    a.num_groups = num_groups;
+    a.max_group_seqs = max_group_seqs;
+    cudaError_t e = pkv::launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidConfiguration) return PKV_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                                int max_blocks_per_seq, const int32_t *context_lens, const int32_t *seq_order,
                                int num_seqs, int num_q_heads,

@@ -51,6 +51,13 @@ struct DecodeArgs {
     // its q / out row is cu_q_lens[i]
     const int32_t *cu_q_lens = nullptr;
     int total_q = 0;
+    // shared-prefix (cascade) mode (null: off): groups of sequences
+    // cu_group_seqs[j] .. cu_group_seqs[j + 1] - 1 share their first
+    // group_prefix[j] tokens; num_partitions then counts the prefix slot too
+    const int32_t *cu_group_seqs = nullptr;
+    const int32_t *group_prefix = nullptr;
+    int num_groups = 0;
+    int max_group_seqs = 0;
 };
 
 // Tile (tokens per pipeline stage) of the decode kernel chosen for a shape;

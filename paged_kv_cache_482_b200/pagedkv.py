@@ -12,6 +12,8 @@ The functions mirror ``include/pagedkv.h``:
 * ``plan_decode`` -- ``pkv_plan_decode``
 * ``decode_workspace_bytes`` -- ``pkv_decode_workspace_bytes``
 * ``paged_attention_decode`` -- ``pkv_paged_attention_decode``
+* ``plan_decode_shared_prefix`` / ``paged_attention_decode_shared_prefix`` --
+  ``pkv_plan_decode_shared_prefix`` / ``pkv_paged_attention_decode_shared_prefix``
 * ``paged_attention_prefill`` -- ``pkv_paged_attention_prefill``
 * ``fused_add_rmsnorm`` -- ``pkv_fused_add_rmsnorm``
 * ``read_device_error`` -- ``pkv_read_device_error``
@@ -39,7 +41,8 @@ PKV_CACHE_BF16 = 0
 PKV_CACHE_FP8_E4M3 = 1  # k_scale / v_scale: [num_kv_heads] fp32
 PKV_CACHE_FP8_E4M3_TOKEN = 2  # k_scale / v_scale: scale pools [num_blocks, num_kv_heads, block_size] fp32
 
-EXPORTED = ("pkv_store_kvcache", "pkv_store_kvcache_rope", "pkv_plan_decode", "pkv_decode_workspace_bytes", "pkv_paged_attention_decode", "pkv_status_string",
+EXPORTED = ("pkv_store_kvcache", "pkv_store_kvcache_rope", "pkv_plan_decode", "pkv_decode_workspace_bytes", "pkv_plan_decode_shared_prefix",
+            "pkv_paged_attention_decode_shared_prefix", "pkv_paged_attention_decode", "pkv_status_string",
             "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
             "pkv_paged_attention_prefill", "pkv_fused_add_rmsnorm")
 
@@ -82,6 +85,12 @@ def load_library(path: str):
     L.pkv_store_kvcache_rope.restype = i32
     L.pkv_plan_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
     L.pkv_plan_decode.restype = i32
+    L.pkv_plan_decode_shared_prefix.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
+    L.pkv_plan_decode_shared_prefix.restype = i32
+    L.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i64,
+                                                           f32, i32, vp, vp, i32, vp, vp, i32, i32, i32, vp, sz, vp,
+                                                           vp, vp]
+    L.pkv_paged_attention_decode_shared_prefix.restype = i32
     L.pkv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.pkv_decode_workspace_bytes.restype = sz
     L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i64, f32, i32,
@@ -202,6 +211,54 @@ def plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_c
     _check(st, "pkv_plan_decode")
     return dict(partition_tokens=plan.partition_tokens, max_partitions=plan.max_partitions,
                 workspace_bytes=plan.workspace_bytes)
+
+
+def plan_decode_shared_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                              cache_dtype=PKV_CACHE_BF16, partition_request=0) -> dict:
+    plan = _Plan()
+    st = lib().pkv_plan_decode_shared_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                             max_context_len, int(cache_dtype), partition_request,
+                                             ctypes.byref(plan))
+    _check(st, "pkv_plan_decode_shared_prefix")
+    return dict(partition_tokens=plan.partition_tokens, max_partitions=plan.max_partitions,
+                workspace_bytes=plan.workspace_bytes)
+
+
+def paged_attention_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale, cu_group_seqs,
+                                         group_prefix_tokens, max_group_seqs, out=None, k_scale=None, v_scale=None,
+                                         max_context_len=None, partition_request=0, workspace=None, dev_err=None,
+                                         stream=None):
+    """Decode of a batch whose consecutive groups of sequences share cached
+    prefixes (int32 device tensors ``cu_group_seqs [G+1]`` and
+    ``group_prefix_tokens [G]``); same result as ``paged_attention_decode``."""
+    S, nq, d = q.shape
+    nblk, nkv, bs, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("q and the pools disagree")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if cu_group_seqs.dtype != torch.int32 or group_prefix_tokens.dtype != torch.int32:
+        raise TypeError("cu_group_seqs and group_prefix_tokens must be int32")
+    G = group_prefix_tokens.numel()
+    if cu_group_seqs.numel() != G + 1:
+        raise ValueError("cu_group_seqs must have one more entry than group_prefix_tokens")
+    maxb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = maxb * bs
+    dt = _cache_dtype(k_cache, k_scale)
+    plan = plan_decode_shared_prefix(S, nq, nkv, d, bs, max_context_len, dt, partition_request)
+    if out is None:
+        out = torch.empty_like(q)
+    if plan["workspace_bytes"] and workspace is None:
+        workspace = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().pkv_paged_attention_decode_shared_prefix(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), maxb, _ptr(context_lens), S, nq, nkv, d, bs, nblk,
+        float(scale), dt, _ptr(k_scale), _ptr(v_scale), int(max_context_len), _ptr(cu_group_seqs),
+        _ptr(group_prefix_tokens), G, int(max_group_seqs), int(partition_request), _ptr(workspace), ws_bytes,
+        _ptr(out), _ptr(dev_err), _stream(stream))
+    _check(st, "pkv_paged_attention_decode_shared_prefix")
+    return out
 
 
 def decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len) -> int:

@@ -126,6 +126,10 @@ class Workload:
     hist_rows: list = field(default_factory=list)  # per seq: 1-D int64 tensor (CPU)
     k_scale: torch.Tensor | None = None  # [nkv] fp32 (FP8 cache only)
     v_scale: torch.Tensor | None = None
+    # sequences group_bounds[j] .. group_bounds[j + 1] - 1 share their first
+    # group_prefix[j] tokens (the same physical blocks)
+    group_bounds: list | None = None
+    group_prefix: list | None = None
 
     @property
     def is_fp8(self) -> bool:
@@ -244,6 +248,8 @@ def generate(cfg: DecodeConfig, seed: int = 0, device: str | torch.device = "cpu
         block_tables=tables.to(torch.int32).to(device),
         context_lens=ctx.to(torch.int32).to(device),
         hist_rows=hist_rows,
+        group_bounds=[0, S],
+        group_prefix=[P],
     )
     if cfg.cache_dtype == CACHE_FP8:
         # One fp32 scale per KV head: the head's absolute maximum over every
@@ -262,6 +268,53 @@ def generate(cfg: DecodeConfig, seed: int = 0, device: str | torch.device = "cpu
         wl.v_scale = vmax.float() / 448.0
     elif cfg.cache_dtype not in (CACHE_BF16, CACHE_FP8_TOKEN):
         raise ValueError(cfg.cache_dtype)
+    return wl
+
+
+def merge(parts: list[Workload], name: str = "merged") -> Workload:
+    """One batch made of several workloads of the same heads, head size, block
+    size and cache type: their pools side by side (block ids and slots
+    offset), their sequences one after the other. Each part's sequences stay
+    a group with the part's shared prefix (``group_bounds``). One scale per
+    KV head becomes the largest of the parts' (inputs both sides read)."""
+    c0 = parts[0].cfg
+    for w in parts:
+        c = w.cfg
+        if (c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size, c.cache_dtype) != \
+                (c0.num_q_heads, c0.num_kv_heads, c0.head_dim, c0.block_size, c0.cache_dtype):
+            raise ValueError("parts must share heads, head size, block size and cache type")
+    bs = c0.block_size
+    width = max(w.block_tables.shape[1] for w in parts)
+    tables, slots_h, slots_n, hist_rows = [], [], [], []
+    blk_off, row_off = 0, 0
+    for w in parts:
+        bt = w.block_tables.cpu().long()
+        bt = torch.where(bt >= 0, bt + blk_off, bt)
+        pad = torch.full((bt.shape[0], width - bt.shape[1]), -1, dtype=torch.long)
+        tables.append(torch.cat([bt, pad], dim=1))
+        sh, sn = w.slot_hist.cpu().long(), w.slot_new.cpu().long()
+        slots_h.append(torch.where(sh >= 0, sh + blk_off * bs, sh))
+        slots_n.append(torch.where(sn >= 0, sn + blk_off * bs, sn))
+        hist_rows += [r + row_off for r in w.hist_rows]
+        blk_off += w.num_blocks
+        row_off += w.k_hist.shape[0]
+    ctx = torch.cat([w.context_lens.cpu() for w in parts])
+    dev = parts[0].q.device
+    cfg = c0.with_(name=name, num_seqs=int(ctx.numel()), ctx_lo=1, ctx_hi=int(ctx.max()), prefix_tokens=0,
+                   pool_blocks=blk_off)
+    wl = Workload(cfg=cfg, seed=parts[0].seed, num_blocks=blk_off,
+                  q=torch.cat([w.q for w in parts]), k_new=torch.cat([w.k_new for w in parts]),
+                  v_new=torch.cat([w.v_new for w in parts]), slot_new=torch.cat(slots_n).to(torch.int32).to(dev),
+                  k_hist=torch.cat([w.k_hist for w in parts]), v_hist=torch.cat([w.v_hist for w in parts]),
+                  slot_hist=torch.cat(slots_h).to(torch.int32).to(dev),
+                  block_tables=torch.cat(tables).to(torch.int32).to(dev), context_lens=ctx.to(torch.int32).to(dev),
+                  hist_rows=hist_rows)
+    if c0.cache_dtype == CACHE_FP8:
+        wl.k_scale = torch.stack([w.k_scale for w in parts]).amax(0)
+        wl.v_scale = torch.stack([w.v_scale for w in parts]).amax(0)
+    sizes = [w.cfg.num_seqs for w in parts]
+    wl.group_bounds = [0] + list(torch.tensor(sizes).cumsum(0).tolist())
+    wl.group_prefix = [w.cfg.prefix_tokens for w in parts]
     return wl
 
 
