@@ -40,7 +40,8 @@ METRIC = "paged decode attention tokens/sec and achieved HBM GB/s (% of B200 pea
 UNIT = "tokens/s"
 NOMINAL_HBM_GBS = 8000.0  # the "~8 TB/s" the target percentage refers to
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["paged_kv_cache_482_b200/csrc/decode.cuh", "paged_kv_cache_482_b200/csrc/decode.cu",
+KERNEL_SOURCES = ["paged_kv_cache_482_b200/csrc/decode.cuh", "paged_kv_cache_482_b200/csrc/decode_mma.cuh",
+                  "paged_kv_cache_482_b200/csrc/decode.cu",
                   "paged_kv_cache_482_b200/csrc/pkv_common.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 
@@ -63,6 +64,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out", default="", help="also append the JSON line to this file")
+    ap.add_argument("--no-shared-prefix", action="store_true",
+                    help="attend a shared-prefix batch with the ordinary decode call instead of the cascade")
     ap.add_argument("--component", choices=["decode", "block_manager"], default="decode",
                     help="block_manager: time the host block manager's per-step bookkeeping instead")
     return ap.parse_args()
@@ -1259,10 +1262,16 @@ def main():
     for i in range(0, H, 1 << 20):
         j = min(H, i + (1 << 20))
         K.store_kvcache(wl.k_hist[i:j], wl.v_hist[i:j], kp, vp, wl.slot_hist[i:j], wl.k_scale, wl.v_scale)
+    # a batch whose sequences share a cached prefix goes through the shared-prefix (cascade) call, as an
+    # engine with a prefix cache would issue it (the groups come from the block manager's hits)
+    shared = bool(c.prefix_tokens) and not args.no_shared_prefix
+    groups = (wl.group_bounds, wl.group_prefix, c.num_seqs) if shared else None
     step = K.DecodeStep(kp, vp, c.num_seqs, c.num_q_heads, wl.block_tables.shape[1], c.softmax_scale,
-                        wl.k_scale, wl.v_scale, max_context_len=c.max_context, partition_request=args.partition)
+                        wl.k_scale, wl.v_scale, max_context_len=c.max_context, partition_request=args.partition,
+                        groups=groups)
     inputs = (wl.q, wl.k_new, wl.v_new, wl.slot_new, wl.block_tables, wl.context_lens)
-    launches_per_step = 2 + (1 if step.plan["partition_tokens"] > 0 else 0)
+    # store + decode (+ reduce when split); shared prefix: store + prefix + decode + merge
+    launches_per_step = 4 if shared else 2 + (1 if step.plan["partition_tokens"] > 0 else 0)
     # The scheduler knows the lengths on the host: visit the longest sequences first.
     order = K.longest_first(wl.context_lens.cpu()).cuda()
 
@@ -1288,10 +1297,17 @@ def main():
         ev[k][0].record(stream)
         K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, step.dev_err)
         ev[k][1].record(stream)
-        K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, out=step.out,
-                                 k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context,
-                                 partition_request=args.partition, workspace=step.workspace, dev_err=step.dev_err,
-                                 seq_order=order)
+        if shared:
+            K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                                   step.groups[0], step.groups[1], step.groups[2], out=step.out,
+                                                   k_scale=wl.k_scale, v_scale=wl.v_scale,
+                                                   max_context_len=c.max_context, partition_request=args.partition,
+                                                   workspace=step.workspace, dev_err=step.dev_err)
+        else:
+            K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, out=step.out,
+                                     k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context,
+                                     partition_request=args.partition, workspace=step.workspace,
+                                     dev_err=step.dev_err, seq_order=order)
         ev[k][2].record(stream)
     e_end.record(stream)
     torch.cuda.synchronize()
@@ -1311,6 +1327,8 @@ def main():
     host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
     # inputs plus the longest-first order that run_host computes and uploads each step
     h2d = sum(t.numel() * t.element_size() for t in host_in) + 4 * c.num_seqs
+    if shared:  # the groups' bounds and prefix lengths
+        h2d += 4 * (2 * len(wl.group_prefix) + 1)
     d2h = host_out.numel() * host_out.element_size()
     for _ in range(3):
         step.run_host(*host_in, host_out)
@@ -1345,7 +1363,8 @@ def main():
                 "workload": workload_desc(c), "num_seqs": c.num_seqs, "seq_len": "ctx " + (
                     f"{c.prefix_tokens}+U[{c.ctx_lo},{c.ctx_hi}]" if c.prefix_tokens else f"U[{c.ctx_lo},{c.ctx_hi}]"),
                 "kv_tokens": wl.kv_tokens(), "seed": args.seed, "partition_tokens": pt,
-                "schedule": "longest sequence first (order from host lengths)",
+                "schedule": ("shared-prefix cascade: each group's prefix once per block of members, then the "
+                             "suffixes" if shared else "longest sequence first (order from host lengths)"),
                 "parallelism": f"replicas x{world} (independent batches, no collective)",
                 "l2": f"no flush: {ab['kv'] / 1e9:.2f} GB of KV read per step, far above the 126 MB L2",
             },
@@ -1355,7 +1374,9 @@ def main():
             "hbm_pct_of_8tbs": 100.0 * achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "paged_decode_kernel" + (" + paged_decode_reduce_kernel" if pt > 0 else ""),
+                         "kernel": (("paged_prefix_mma_kernel + " if shared else "") +
+                                    ("paged_decode_mma_kernel" if c.head_dim == 128 else "paged_decode_kernel") +
+                                    (" + paged_decode_reduce_kernel" if pt > 0 or shared else "")),
                          "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                          "algorithmic_bytes_per_launch": bytes_launch,
                          "bytes_note": ("unique bytes: shared prefix counted once" if c.prefix_tokens else

@@ -422,7 +422,10 @@ class DecodeStep:
     """
 
     def __init__(self, k_cache, v_cache, num_seqs, num_q_heads, max_blocks_per_seq, scale, k_scale=None,
-                 v_scale=None, max_context_len=None, partition_request=0, device=None):
+                 v_scale=None, max_context_len=None, partition_request=0, device=None, groups=None):
+        """``groups`` = (cu_group_seqs, group_prefix_tokens, max_group_seqs):
+        consecutive sequences that share cached prefixes, attended through
+        ``paged_attention_decode_shared_prefix``."""
         self.k_cache, self.v_cache = k_cache, v_cache
         self.k_scale, self.v_scale = k_scale, v_scale
         nblk, nkv, bs, d = k_cache.shape
@@ -432,8 +435,20 @@ class DecodeStep:
         self.scale = scale
         self.partition_request = partition_request
         dev = device or k_cache.device
-        self.plan = plan_decode(num_seqs, num_q_heads, nkv, d, bs, self.max_context_len,
-                                _cache_dtype(k_cache, k_scale) != PKV_CACHE_BF16, partition_request)
+        self.groups = None
+        if groups is not None:
+            cu, pre, mg = groups
+            host_cu = torch.as_tensor(cu, dtype=torch.int32).cpu()
+            host_pre = torch.as_tensor(pre, dtype=torch.int32).cpu()
+            if torch.cuda.is_available():
+                host_cu, host_pre = host_cu.pin_memory(), host_pre.pin_memory()
+            self._host_groups = (host_cu, host_pre)
+            self.groups = (host_cu.to(dev), host_pre.to(dev), int(mg))
+            self.plan = plan_decode_shared_prefix(num_seqs, num_q_heads, nkv, d, bs, self.max_context_len,
+                                                  _cache_dtype(k_cache, k_scale), partition_request)
+        else:
+            self.plan = plan_decode(num_seqs, num_q_heads, nkv, d, bs, self.max_context_len,
+                                    _cache_dtype(k_cache, k_scale) != PKV_CACHE_BF16, partition_request)
         self.workspace = (torch.empty(self.plan["workspace_bytes"], dtype=torch.uint8, device=dev)
                           if self.plan["workspace_bytes"] else None)
         self.out = torch.empty((num_seqs, num_q_heads, d), dtype=torch.bfloat16, device=dev)
@@ -444,6 +459,13 @@ class DecodeStep:
         """Device inputs -> device output (no host traffic, no sync)."""
         store_kvcache(k_new, v_new, self.k_cache, self.v_cache, slot_mapping, self.k_scale, self.v_scale,
                       self.dev_err, stream)
+        if self.groups is not None:
+            cu, pre, mg = self.groups
+            return paged_attention_decode_shared_prefix(
+                q, self.k_cache, self.v_cache, block_tables, context_lens, self.scale, cu, pre, mg, out=self.out,
+                k_scale=self.k_scale, v_scale=self.v_scale, max_context_len=self.max_context_len,
+                partition_request=self.partition_request, workspace=self.workspace, dev_err=self.dev_err,
+                stream=stream)
         return paged_attention_decode(q, self.k_cache, self.v_cache, block_tables, context_lens, self.scale,
                                       out=self.out, k_scale=self.k_scale, v_scale=self.v_scale,
                                       max_context_len=self.max_context_len,
@@ -461,6 +483,9 @@ class DecodeStep:
         for d_, h_ in zip(self._dev_inputs, host):
             d_.copy_(h_, non_blocking=True)
         dq, dk, dv, ds, dbt, dcl, dord = self._dev_inputs
+        if self.groups is not None:  # the step's groups come from the host too
+            self.groups[0].copy_(self._host_groups[0], non_blocking=True)
+            self.groups[1].copy_(self._host_groups[1], non_blocking=True)
         o = self.run(dq, dk, dv, ds, dbt, dcl, stream, seq_order=dord)
         out_host.copy_(o, non_blocking=True)
         return out_host

@@ -124,7 +124,7 @@ def test_bad_groups_zero_only_their_rows():
     wl.block_tables = bt
     cu, pre, mg = groups_of(wl)
     pre_bad = pre.clone()
-    pre_bad[0] = 48  # not a multiple of 16 (block size): the whole first group
+    pre_bad[0] = 40  # not a multiple of 16 (the block size): the whole first group
     out, st = run_shared(wl, kp, vp, cu=cu, pre=pre_bad)
     assert st == K.PKV_ERR_DEVICE_BOUNDS
     zero = list(range(wl.group_bounds[0], wl.group_bounds[1])) + [victim]
