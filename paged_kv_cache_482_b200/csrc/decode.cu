@@ -1,4 +1,6 @@
-// decode.cu -- instantiations and launch of the paged decode kernels.
+// decode.cu -- instantiations and launch of the paged decode kernels: the
+// warp-MMA kernels (decode_mma.cuh) at head_dim 128, the CUDA-core kernel
+// (decode.cuh) at head_dim 64.
 //
 // Tile shape: four warps, each taking up to four 32-lane steps of a tile;
 // stages hold K and V of one tile and the ring is about 48 KB deep, so that
@@ -45,11 +47,7 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-// head_dim 128: the warp-MMA kernel (decode_mma.cuh) for E4M3 and, unless
-// built with PKV_DECODE_BF16_MMA=0, for bf16.
-#ifndef PKV_DECODE_BF16_MMA
-#define PKV_DECODE_BF16_MMA 1
-#endif
+// head_dim 128: the warp-MMA kernel (decode_mma.cuh), every cache type.
 template <int G, bool BF, bool TS>
 cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
     using T = MmaTraits<G, BF>;
@@ -158,9 +156,7 @@ cudaError_t launch_group(int group, const DecodeParams &p, cudaStream_t stream) 
 }  // namespace
 
 int decode_tile_tokens(int head_dim, int group, bool fp8) {
-    if (head_dim == 128)
-        return fp8 ? mma_tile_of<false>(group) : (PKV_DECODE_BF16_MMA ? mma_tile_of<true>(group)
-                                                                       : tile_of<128, false>(group));
+    if (head_dim == 128) return fp8 ? mma_tile_of<false>(group) : mma_tile_of<true>(group);
     if (head_dim == 64) return fp8 ? tile_of<64, true>(group) : tile_of<64, false>(group);
     return 0;
 }
@@ -206,18 +202,14 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.max_group_seqs = a.max_group_seqs;
     p.grid_partitions = a.cu_group_seqs ? p.num_partitions - 1 : p.num_partitions;
     const int group = a.num_q_heads / a.num_kv_heads;
-    if (a.fp8 && a.head_dim == 128) return a.token_scales ? launch_mma<false, true>(group, p, stream)
-                                                          : launch_mma<false, false>(group, p, stream);
-    if (PKV_DECODE_BF16_MMA && !a.fp8 && a.head_dim == 128) return launch_mma<true, false>(group, p, stream);
-    if (a.fp8 && a.token_scales) {
-        if (a.head_dim == 128) return launch_group<128, true, true>(group, p, stream);
-        if (a.head_dim == 64) return launch_group<64, true, true>(group, p, stream);
-        return cudaErrorInvalidValue;
+    if (a.head_dim == 128) {
+        if (!a.fp8) return launch_mma<true, false>(group, p, stream);
+        return a.token_scales ? launch_mma<false, true>(group, p, stream) : launch_mma<false, false>(group, p, stream);
     }
-    if (a.head_dim == 128)
-        return a.fp8 ? launch_group<128, true>(group, p, stream) : launch_group<128, false>(group, p, stream);
-    if (a.head_dim == 64)
+    if (a.head_dim == 64) {  // the CUDA-core kernel (decode.cuh)
+        if (a.fp8 && a.token_scales) return launch_group<64, true, true>(group, p, stream);
         return a.fp8 ? launch_group<64, true>(group, p, stream) : launch_group<64, false>(group, p, stream);
+    }
     return cudaErrorInvalidValue;
 }
 

@@ -1,4 +1,6 @@
-// decode.cuh -- paged decode attention kernels (sm_100a, CUDA cores).
+// decode.cuh -- paged decode attention on the CUDA cores (sm_100a): the
+// kernel for head_dim 64 (head_dim 128 runs on the warp-level MMA,
+// decode_mma.cuh), the split-K merge both use, and the parameters they share.
 //
 // One thread block per (sequence, KV head, partition). It serves all G query
 // heads that share the KV head, so every K/V byte of the partition is read

@@ -688,6 +688,10 @@ class RopeWorkload:
     k_scale: torch.Tensor | None = None  # [nkv] fp32 (one scale per KV head)
     v_scale: torch.Tensor | None = None
 
+    @property
+    def is_fp8(self) -> bool:
+        return self.cfg.is_fp8
+
 
 def generate_rope(cfg: RopeConfig, seed: int = 0, device: str | torch.device = "cpu") -> RopeWorkload:
     """Positions uniform in [0, max_position); slots distinct, from a seeded
