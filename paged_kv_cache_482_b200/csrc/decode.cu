@@ -15,6 +15,10 @@ namespace pkv {
 
 namespace {
 
+unsigned reduce_blocks(const DecodeParams &p) {
+    return (unsigned)(((long long)p.num_seqs * p.num_q_heads + kReduceWarps - 1) / kReduceWarps);
+}
+
 template <int D, int G, bool FP8, bool TS>
 cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
     using T = DecodeTraits<D, G, FP8>;
@@ -43,7 +47,7 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
     kern<<<(unsigned)blocks, T::kThreads, T::kSmemBytes, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.num_partitions <= 1) return e;
-    paged_decode_reduce_kernel<D><<<(unsigned)((long long)p.num_seqs * p.num_q_heads), D, 0, stream>>>(p);
+    paged_decode_reduce_kernel<D><<<reduce_blocks(p), 32 * kReduceWarps, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -105,7 +109,7 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
     kern<<<(unsigned)blocks, T::kThreads, T::kAlloc, stream>>>(p, mk, mv, box_rows);
     e = cudaGetLastError();
     if (e != cudaSuccess || (p.num_partitions <= 1 && !p.cu_group_seqs)) return e;
-    paged_decode_reduce_kernel<128><<<(unsigned)((long long)p.num_seqs * p.num_q_heads), 128, 0, stream>>>(p);
+    paged_decode_reduce_kernel<128><<<reduce_blocks(p), 32 * kReduceWarps, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -662,24 +662,34 @@ __global__ void __launch_bounds__(DecodeTraits<D, G, FP8>::kThreads, MIN_BLOCKS)
 }
 
 // Merge the split-K partials of one (sequence, query head): weights
-// l_p * 2^(m_p - M) over the sequence's partitions, fixed order. The grid
-// visits sequences through seq_order like the decode grid, so it merges only
+// l_p * 2^(m_p - M) over the sequence's partitions, in partition order. One
+// warp per (sequence, query head), four per block: the lanes load the
+// partitions' (max, sum) pairs together and reduce them with shuffles, then
+// each lane accumulates D / 32 dims over the partitions. The grid visits
+// sequences through seq_order like the decode grid, so it merges only
 // partials this call's decode blocks wrote; a sequence that no valid entry
 // names is left alone by both.
+constexpr int kReduceWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(D) paged_decode_reduce_kernel(const DecodeParams p) {
-    const int qh = blockIdx.x % p.num_q_heads;
-    const int seq_slot = blockIdx.x / p.num_q_heads;
+__global__ void __launch_bounds__(32 * kReduceWarps) paged_decode_reduce_kernel(const DecodeParams p) {
+    constexpr int DPL = D / 32;  // dims per lane
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
+    if (row >= (long long)p.num_seqs * p.num_q_heads) return;
+    const int qh = (int)(row % p.num_q_heads);
+    const int seq_slot = (int)(row / p.num_q_heads);
     const int seq = p.seq_order ? __ldg(p.seq_order + seq_slot) : seq_slot;
     if (seq < 0 || seq >= p.num_seqs) return;  // the decode grid reported it
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
     const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
     // partial slots first .. first + n - 1 of this sequence
-    int first = 0, n = 0, bad0 = 0;
+    int first = 0, n = 0;
+    bool bad = false;
     if (p.cu_group_seqs) {  // slot 0: the shared prefix (when there is one), then the suffix partitions
         const int P = bad_len ? -1 : prefix_of(p, seq, ctx);
-        bad0 = P < 0;
+        bad = P < 0;
         const int n_suf = P >= 0 ? (ctx - P + p.partition_tokens - 1) / p.partition_tokens : 0;
         first = P == 0 ? 1 : 0;
         n = (P != 0) + n_suf;
@@ -689,31 +699,48 @@ __global__ void __launch_bounds__(D) paged_decode_reduce_kernel(const DecodePara
         if (n <= 1) return;  // decode wrote the output itself
     }
     const long long base = ((long long)seq * p.num_q_heads + qh) * p.num_partitions + first;
-    __shared__ float w_s[1024];
-    __shared__ int bad_s;
-    if (threadIdx.x == 0) {
-        float M = -CUDART_INF_F;
-        int bad = bad0 || bad_len;
-        for (int i = 0; i < n && !bad; ++i) {
-            const float li = p.part_ml[(base + i) * 2 + 1];
-            bad |= !(li > 0.f);
-            M = fmaxf(M, p.part_ml[(base + i) * 2]);
-        }
-        float L = 0.f;
-        for (int i = 0; i < n && !bad; ++i) {
-            const float e = p.part_ml[(base + i) * 2 + 1] * exp2f(p.part_ml[(base + i) * 2] - M);
-            w_s[i] = e;
-            L += e;
-        }
-        const float inv = bad ? 0.f : 1.f / L;
-        for (int i = 0; i < n && !bad; ++i) w_s[i] *= inv;
-        bad_s = bad;
+    // maximum over the partitions, and whether any is empty (sum 0: a bad block)
+    float M = -CUDART_INF_F;
+    bool empty = false;
+    for (int i = lane; i < n && !bad; i += 32) {
+        const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (base + i) * 2);
+        M = fmaxf(M, ml.x);
+        empty |= !(ml.y > 0.f);
     }
-    __syncthreads();
-    float o = 0.f;
-    if (!bad_s)
-        for (int i = 0; i < n; ++i) o = fmaf(p.part_o[(base + i) * D + threadIdx.x], w_s[i], o);
-    p.out[((long long)seq * p.num_q_heads + qh) * D + threadIdx.x] = __float2bfloat16_rn(o);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    bad = __any_sync(0xffffffffu, bad || empty);
+    float acc[DPL];
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+    if (!bad) {
+        float L = 0.f;
+        for (int i = lane; i < n; i += 32) {
+            const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (base + i) * 2);
+            L += ml.y * exp2f(ml.x - M);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float inv = 1.f / L;
+        for (int i = 0; i < n; ++i) {
+            const float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + (base + i) * 2);
+            const float w = ml.y * exp2f(ml.x - M) * inv;
+            const float *po = p.part_o + (base + i) * D + lane * DPL;
+            if constexpr (DPL == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(po);
+                acc[0] = fmaf(v.x, w, acc[0]);
+                acc[1] = fmaf(v.y, w, acc[1]);
+                acc[2] = fmaf(v.z, w, acc[2]);
+                acc[3] = fmaf(v.w, w, acc[3]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < DPL; ++k) acc[k] = fmaf(po[k], w, acc[k]);
+            }
+        }
+    }
+    __nv_bfloat16 *dst = p.out + ((long long)seq * p.num_q_heads + qh) * D + lane * DPL;
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) dst[k] = __float2bfloat16_rn(acc[k]);
 }
 
 }  // namespace pkv

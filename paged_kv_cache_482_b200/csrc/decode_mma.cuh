@@ -228,9 +228,11 @@ __device__ __forceinline__ float load_q_frags(const __nv_bfloat16 *qrow, int t, 
 }
 
 // Raw scores of one 16-token group: c = S^T fragment (tokens g, g + 8 x
-// columns 2t, 2t + 1), accumulated onto c.
+// columns 2t, 2t + 1). Two accumulators take alternate k-steps (two
+// independent MMA chains) and are added at the end.
 template <bool BF>
 __device__ __forceinline__ void qk_group(uint32_t kg, int g, int t, const uint32_t (&qf)[8][2], float (&c)[4]) {
+    float c2[4] = {0.f, 0.f, 0.f, 0.f};
     if constexpr (BF) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -242,8 +244,8 @@ __device__ __forceinline__ void qk_group(uint32_t kg, int g, int t, const uint32
             const uint32_t wh[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                mma_bf16_16816(c, wg[2 * i], wh[2 * i], wg[2 * i + 1], wh[2 * i + 1], qf[4 * hh + i][0],
-                               qf[4 * hh + i][1]);
+                mma_bf16_16816((i & 1) ? c2 : c, wg[2 * i], wh[2 * i], wg[2 * i + 1], wh[2 * i + 1],
+                               qf[4 * hh + i][0], qf[4 * hh + i][1]);
         }
     } else {
         const uint4 k0 = lds128(swz16(kg, g, 2 * t));
@@ -256,9 +258,11 @@ __device__ __forceinline__ void qk_group(uint32_t kg, int g, int t, const uint32
         for (int i = 0; i < 8; ++i) {
             const uint2 a = tc::e4m3x4_to_f16x4(wg[i]);  // row g: dims +0,+1 | +2,+3
             const uint2 b = tc::e4m3x4_to_f16x4(wh[i]);  // row g + 8
-            mma_f16_16816(c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
+            mma_f16_16816((i & 1) ? c2 : c, a.x, b.x, a.y, b.y, qf[i][0], qf[i][1]);
         }
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) c[k] += c2[k];
 }
 
 // o += P V of one 16-token group. pw: the weights of tokens g, g + 8 x
@@ -755,9 +759,9 @@ struct PrefixTraits {
     static constexpr int kRowBytes = BF ? 256 : 128;
     static constexpr int kHalves = BF ? 2 : 1;
     static constexpr int kGroupBytes = 16 * kRowBytes;
-    static constexpr int kNG = BF ? 2 : 4;  // 16-token groups per stage
-    static constexpr int kTT = 16 * kNG;    // tokens per stage
-    static constexpr int kStages = 4;
+    static constexpr int kNG = 4;        // 16-token groups per stage
+    static constexpr int kTT = 16 * kNG;  // tokens per stage
+    static constexpr int kStages = BF ? 3 : 4;
     static constexpr int kHalfBytes = kNG * kGroupBytes;  // K (or V) of one stage
     static constexpr int kStageBytes = 2 * kHalfBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
@@ -770,7 +774,7 @@ struct PrefixTraits {
 };
 
 template <int G, bool BF, bool TS>
-__global__ void __launch_bounds__(PrefixTraits<BF>::kThreads, 1)
+__global__ void __launch_bounds__(PrefixTraits<BF>::kThreads, 2)
     paged_prefix_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
                             const __grid_constant__ CUtensorMap map_v, int box_rows, int max_chunks) {
     static_assert(!(BF && TS), "per-token scales exist only for E4M3");

@@ -129,10 +129,9 @@ __global__ void __launch_bounds__(256) store_kvcache_kernel(StoreParams p) {
 // contract). The rotated k is then stored exactly as store_kvcache stores a
 // bf16 row; v is stored as is; q is written rotated to q_out.
 //
-// One thread handles 8 pairs (the same 8 of every row) of up to kRopeRows
-// rows of one token -- rows are the q heads, then the KV heads -- so a row
-// takes d/16 adjacent lanes: it loads its 2 x 32 bytes of the token's table
-// row once, then per row two 16-byte loads and stores per tensor.
+// One thread handles 8 pairs of one (token, row) -- rows are the q heads,
+// then the KV heads -- so a row takes d/16 adjacent lanes: two 16-byte loads
+// and stores per tensor, and 2 x 32 bytes of the table.
 
 struct RopeParams {
     const uint4 *q;  // may be null
@@ -195,23 +194,20 @@ __device__ __forceinline__ void interleave(const uint4 &x, const uint4 &y, uint4
                    __byte_perm(x.w, y.w, 0x7632));
 }
 
-constexpr int kRopeRows = 8;  // rows per thread
-
 template <int MODE, int STYLE>
 __global__ void __launch_bounds__(256) store_kvcache_rope_kernel(RopeParams p) {
     const long long stride = (long long)gridDim.x * blockDim.x;
     const int L = p.lanes_per_row;
     const int rows = p.num_q_heads + p.num_kv_heads;
-    const int row_groups = (rows + kRopeRows - 1) / kRopeRows;
     const int cpr = p.head_dim / 8;  // 16-byte chunks per row
     for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < p.total_units; u += stride) {
         const int c = (int)(u % L);
-        const long long gi = u / L;
-        const int rg = (int)(gi % row_groups);
-        const long long token = gi / row_groups;
+        const long long rowi = u / L;
+        const int r = (int)(rowi % rows);
+        const long long token = rowi / rows;
         const int m = p.positions[token];
         if (m < 0 || m >= p.max_position) {
-            if (c == 0 && rg == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+            if (c == 0 && r == 0) set_error(p.dev_err, PKV_DEVERR_BOUNDS);
             continue;
         }
         // chunk indices of the two halves this lane handles
@@ -223,80 +219,76 @@ __global__ void __launch_bounds__(256) store_kvcache_rope_kernel(RopeParams p) {
         const float4 c0 = __ldg(cs), c1 = __ldg(cs + 1), s0 = __ldg(sn), s1 = __ldg(sn + 1);
         const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-        const int r_end = min(rows, (rg + 1) * kRopeRows);
-#pragma unroll 2
-        for (int r = rg * kRopeRows; r < r_end; ++r) {
-            if (r < p.num_q_heads) {
-                const long long base = (token * p.num_q_heads + r) * cpr;
-                uint4 a = __ldg(p.q + base + ca), b = __ldg(p.q + base + cb);
-                if constexpr (STYLE == 1) {
-                    uint4 x, y;
-                    deinterleave(a, b, x, y);
-                    rotate8(x, y, cv, sv);
-                    interleave(x, y, a, b);
-                } else {
-                    rotate8(a, b, cv, sv);
-                }
-                p.q_out[base + ca] = a;
-                p.q_out[base + cb] = b;
-                continue;
-            }
-            const int head = r - p.num_q_heads;
-            const long long slot = p.slots[token];
-            if (slot < 0) continue;
-            if (slot >= p.pool_slots) {
-                set_error(p.dev_err, PKV_DEVERR_BOUNDS);
-                continue;
-            }
-            const long long base = (token * p.num_kv_heads + head) * cpr;
-            uint4 ka = __ldg(p.k + base + ca), kb = __ldg(p.k + base + cb);
-            const uint4 va = __ldg(p.v + base + ca), vb = __ldg(p.v + base + cb);
+        if (r < p.num_q_heads) {
+            const long long base = (token * p.num_q_heads + r) * cpr;
+            uint4 a = __ldg(p.q + base + ca), b = __ldg(p.q + base + cb);
             if constexpr (STYLE == 1) {
                 uint4 x, y;
-                deinterleave(ka, kb, x, y);
+                deinterleave(a, b, x, y);
                 rotate8(x, y, cv, sv);
-                interleave(x, y, ka, kb);
+                interleave(x, y, a, b);
             } else {
-                rotate8(ka, kb, cv, sv);
+                rotate8(a, b, cv, sv);
             }
-            const long long blk = slot / p.block_size;
-            const long long off = slot - blk * p.block_size;
-            const long long row = (blk * p.num_kv_heads + head) * p.block_size + off;  // pool row
-            const long long ea = row * p.head_dim + ca * 8LL, eb = row * p.head_dim + cb * 8LL;  // element offsets
-            if constexpr (MODE == 0) {
-                __nv_bfloat16 *kc = static_cast<__nv_bfloat16 *>(p.k_cache), *vc = static_cast<__nv_bfloat16 *>(p.v_cache);
-                *reinterpret_cast<uint4 *>(kc + ea) = ka;
-                *reinterpret_cast<uint4 *>(kc + eb) = kb;
-                *reinterpret_cast<uint4 *>(vc + ea) = va;
-                *reinterpret_cast<uint4 *>(vc + eb) = vb;
-            } else {
-                float ks, vs;
-                if constexpr (MODE == 2) {
-                    // the row's L lanes are adjacent (L divides 32 and the stride)
-                    const int lane = threadIdx.x & 31;
-                    const unsigned group = (L == 32 ? 0xffffffffu : ((1u << L) - 1u)) << (lane & ~(L - 1));
-                    float km = fmaxf(amax8(ka), amax8(kb)), vm = fmaxf(amax8(va), amax8(vb));
-                    for (int o = L >> 1; o > 0; o >>= 1) {
-                        km = fmaxf(km, __shfl_xor_sync(group, km, o, L));
-                        vm = fmaxf(vm, __shfl_xor_sync(group, vm, o, L));
-                    }
-                    ks = token_scale(km);
-                    vs = token_scale(vm);
-                    if (c == 0) {
-                        p.k_scale[row] = ks;
-                        p.v_scale[row] = vs;
-                    }
-                } else {
-                    ks = __ldg(p.k_scale + head);
-                    vs = __ldg(p.v_scale + head);
+            p.q_out[base + ca] = a;
+            p.q_out[base + cb] = b;
+            continue;
+        }
+        const int head = r - p.num_q_heads;
+        const long long slot = p.slots[token];
+        if (slot < 0) continue;
+        if (slot >= p.pool_slots) {
+            set_error(p.dev_err, PKV_DEVERR_BOUNDS);
+            continue;
+        }
+        const long long base = (token * p.num_kv_heads + head) * cpr;
+        uint4 ka = __ldg(p.k + base + ca), kb = __ldg(p.k + base + cb);
+        const uint4 va = __ldg(p.v + base + ca), vb = __ldg(p.v + base + cb);
+        if constexpr (STYLE == 1) {
+            uint4 x, y;
+            deinterleave(ka, kb, x, y);
+            rotate8(x, y, cv, sv);
+            interleave(x, y, ka, kb);
+        } else {
+            rotate8(ka, kb, cv, sv);
+        }
+        const long long blk = slot / p.block_size;
+        const long long off = slot - blk * p.block_size;
+        const long long row = (blk * p.num_kv_heads + head) * p.block_size + off;  // pool row
+        const long long ea = row * p.head_dim + ca * 8LL, eb = row * p.head_dim + cb * 8LL;  // element offsets
+        if constexpr (MODE == 0) {
+            __nv_bfloat16 *kc = static_cast<__nv_bfloat16 *>(p.k_cache), *vc = static_cast<__nv_bfloat16 *>(p.v_cache);
+            *reinterpret_cast<uint4 *>(kc + ea) = ka;
+            *reinterpret_cast<uint4 *>(kc + eb) = kb;
+            *reinterpret_cast<uint4 *>(vc + ea) = va;
+            *reinterpret_cast<uint4 *>(vc + eb) = vb;
+        } else {
+            float ks, vs;
+            if constexpr (MODE == 2) {
+                // the row's L lanes are adjacent (L divides 32 and the stride)
+                const int lane = threadIdx.x & 31;
+                const unsigned group = (L == 32 ? 0xffffffffu : ((1u << L) - 1u)) << (lane & ~(L - 1));
+                float km = fmaxf(amax8(ka), amax8(kb)), vm = fmaxf(amax8(va), amax8(vb));
+                for (int o = L >> 1; o > 0; o >>= 1) {
+                    km = fmaxf(km, __shfl_xor_sync(group, km, o, L));
+                    vm = fmaxf(vm, __shfl_xor_sync(group, vm, o, L));
                 }
-                uint8_t *kc = static_cast<uint8_t *>(p.k_cache), *vc = static_cast<uint8_t *>(p.v_cache);
-                *reinterpret_cast<uint2 *>(kc + ea) = quantise8(ka, ks);
-                *reinterpret_cast<uint2 *>(kc + eb) = quantise8(kb, ks);
-                *reinterpret_cast<uint2 *>(vc + ea) = quantise8(va, vs);
-                *reinterpret_cast<uint2 *>(vc + eb) = quantise8(vb, vs);
+                ks = token_scale(km);
+                vs = token_scale(vm);
+                if (c == 0) {
+                    p.k_scale[row] = ks;
+                    p.v_scale[row] = vs;
+                }
+            } else {
+                ks = __ldg(p.k_scale + head);
+                vs = __ldg(p.v_scale + head);
             }
-        }  // rows of the group
+            uint8_t *kc = static_cast<uint8_t *>(p.k_cache), *vc = static_cast<uint8_t *>(p.v_cache);
+            *reinterpret_cast<uint2 *>(kc + ea) = quantise8(ka, ks);
+            *reinterpret_cast<uint2 *>(kc + eb) = quantise8(kb, ks);
+            *reinterpret_cast<uint2 *>(vc + ea) = quantise8(va, vs);
+            *reinterpret_cast<uint2 *>(vc + eb) = quantise8(vb, vs);
+        }
     }
 }
 
@@ -336,8 +328,7 @@ cudaError_t launch_store_kvcache_rope(const void *q, void *q_out, const void *k,
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.dev_err = dev_err;
-    p.total_units = (long long)num_tokens * ((p.num_q_heads + num_kv_heads + kRopeRows - 1) / kRopeRows) *
-                    p.lanes_per_row;
+    p.total_units = (long long)num_tokens * (p.num_q_heads + num_kv_heads) * p.lanes_per_row;
     long long blocks = (p.total_units + 255) / 256;
     const long long cap = (long long)num_sms * 16;
     if (blocks > cap) blocks = cap;
