@@ -38,10 +38,15 @@
  *
  * Ownership and execution. The caller owns every buffer (device memory unless
  * stated) and keeps it alive until the stream work finishes. The library
- * allocates nothing and keeps no state between calls; calls are re-entrant.
- * Every call is asynchronous on the given stream (a cudaStream_t passed as
- * void*; NULL is the legacy default stream) and returns once the work is
- * queued.
+ * allocates no device memory. Its only state across calls is looked up or
+ * created once per device and kept for the process: the static scratch's
+ * device address (pkv_paged_attention_decode_static_scratch) and one
+ * low-priority stream for the one-token chunks of a mixed prefill batch
+ * (pkv_paged_attention_prefill). Calls are re-entrant. Every call is
+ * asynchronous on the given stream (a cudaStream_t passed as void*; NULL is
+ * the legacy default stream) and returns once the work is queued; work the
+ * library puts on its own stream is joined back into the given stream with
+ * events before the call returns, so the call stays stream-ordered.
  *
  * Errors. Arguments the host can check are checked before anything is
  * launched; a failed check returns the status and launches nothing. Faults
@@ -353,6 +358,12 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  * its context or than max_q_len, a context beyond the table row, or a block
  * id outside [0, num_blocks) set PKV_DEVERR_BOUNDS; the sequence's rows are
  * written as zeros where they can be located. The library allocates nothing.
+ *
+ * Routing: one-token chunks run in the decode kernel; when the batch also
+ * has longer chunks (max_q_len > 1), they run on the library's low-priority
+ * stream of this device, beside the chunk kernels on the given stream
+ * (forked from and joined back into it with events), so that their blocks
+ * use the SMs the long chunks' few blocks leave idle.
  */
 PKV_API int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *v_cache,
                                         const int32_t *block_tables, int max_blocks_per_seq,

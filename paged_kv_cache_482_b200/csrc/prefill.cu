@@ -38,6 +38,8 @@
 // 128 / 64 column blocks][rows][128 bytes], the 16-byte chunk c of row r
 // stored at chunk c ^ (r % 8) -- the canonical 128-byte swizzle, so one
 // descriptor form serves Q, K and P (K-major) and V (MN-major).
+#include <atomic>
+
 #include "tc_common.cuh"
 
 namespace pkv {
@@ -538,6 +540,59 @@ bool prefill_supported(int head_dim, int group) {
     return (head_dim == 64 || head_dim == 128) && (group == 1 || group == 2 || group == 4 || group == 8);
 }
 
+namespace {
+
+// The chunk kernels of a batch: the one-tile kernel for chunks of 2 ..
+// 128 / G tokens, the warp-specialised kernel for longer ones.
+cudaError_t launch_chunks(const PrefillArgs &a, int g, cudaStream_t stream) {
+    PrefillArgs small = a;
+    small.small_cut = kRows / g;
+    small.small_min = 2;
+    small.max_q_len = a.max_q_len < small.small_cut ? a.max_q_len : small.small_cut;
+    cudaError_t e = cudaSuccess;
+    if (a.max_q_len > small.small_cut) {  // the long chunks first: their few blocks should start first
+        PrefillArgs large = a;
+        large.small_cut = small.small_cut;
+        e = launch_prefill_ws(large, stream);
+        if (e != cudaSuccess) return e;
+    }
+    if (a.fp8 && a.token_scales)
+        return a.head_dim == 128 ? launch_d<128, true, true>(small, g, stream)
+                                 : launch_d<64, true, true>(small, g, stream);
+    if (a.head_dim == 128) return a.fp8 ? launch_d<128, true>(small, g, stream) : launch_d<128, false>(small, g, stream);
+    return a.fp8 ? launch_d<64, true>(small, g, stream) : launch_d<64, false>(small, g, stream);
+}
+
+// A low-priority stream per device, created on first use and kept for the
+// process: the one-token chunks of a mixed batch run on it, beside the chunk
+// kernels, so that their blocks fill the SMs the few long-chunk blocks leave
+// idle; the caller's stream waits for it before anything queued later.
+cudaStream_t side_stream() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<cudaStream_t> streams[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    cudaStream_t s = streams[dev].load(std::memory_order_acquire);
+    if (s) return s;
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&s, cudaStreamNonBlocking, least) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    cudaStream_t expected = nullptr;
+    if (!streams[dev].compare_exchange_strong(expected, s, std::memory_order_acq_rel)) {
+        cudaStreamDestroy(s);  // another thread made one first
+        return expected;
+    }
+    return s;
+}
+
+}  // namespace
+
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
     // One-token chunks (decode requests in the batch) go to the decode
@@ -574,22 +629,27 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     d.dev_err = a.dev_err;
     d.cu_q_lens = a.cu_q_lens;
     d.total_q = a.total_q;
-    cudaError_t e = launch_decode(d, stream);
-    if (e != cudaSuccess || a.max_q_len <= 1) return e;
-    PrefillArgs small = a;
-    small.small_cut = kRows / g;
-    small.small_min = 2;
-    small.max_q_len = a.max_q_len < small.small_cut ? a.max_q_len : small.small_cut;
-    if (a.fp8 && a.token_scales)
-        e = a.head_dim == 128 ? launch_d<128, true, true>(small, g, stream) : launch_d<64, true, true>(small, g, stream);
-    else if (a.head_dim == 128)
-        e = a.fp8 ? launch_d<128, true>(small, g, stream) : launch_d<128, false>(small, g, stream);
-    else
-        e = a.fp8 ? launch_d<64, true>(small, g, stream) : launch_d<64, false>(small, g, stream);
-    if (e != cudaSuccess || a.max_q_len <= small.small_cut) return e;
-    PrefillArgs large = a;
-    large.small_cut = small.small_cut;
-    return launch_prefill_ws(large, stream);
+    if (a.max_q_len <= 1) return launch_decode(d, stream);  // decode requests only
+    cudaStream_t side = side_stream();
+    cudaEvent_t fork = nullptr, join = nullptr;
+    if (!side || cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();  // no side stream: everything on the caller's stream
+        if (fork) cudaEventDestroy(fork);
+        cudaError_t e = launch_decode(d, stream);
+        return e != cudaSuccess ? e : launch_chunks(a, g, stream);
+    }
+    cudaError_t e = cudaEventRecord(fork, stream);
+    if (e == cudaSuccess) e = launch_chunks(a, g, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+    if (e == cudaSuccess) e = launch_decode(d, side);
+    // join even after a failure, so that nothing later on the caller's stream
+    // overtakes work already queued on the side stream
+    cudaError_t e2 = cudaEventRecord(join, side);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(stream, join, 0);
+    cudaEventDestroy(fork);  // released once the waits are resolved
+    cudaEventDestroy(join);
+    return e != cudaSuccess ? e : e2;
 }
 
 }  // namespace pkv
