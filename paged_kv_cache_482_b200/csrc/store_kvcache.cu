@@ -330,10 +330,7 @@ cudaError_t launch_store_kvcache_rope(const void *q, void *q_out, const void *k,
     p.dev_err = dev_err;
     p.total_units = (long long)num_tokens * (p.num_q_heads + num_kv_heads) * p.lanes_per_row;
     long long blocks = (p.total_units + 255) / 256;
-#ifndef PKV_ROPE_BLOCKS_PER_SM
-#define PKV_ROPE_BLOCKS_PER_SM 16
-#endif
-    const long long cap = (long long)num_sms * PKV_ROPE_BLOCKS_PER_SM;
+    const long long cap = (long long)num_sms * 16;  // grid-stride beyond 16 blocks per SM (an uncapped grid measured slower)
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (mode == 2)

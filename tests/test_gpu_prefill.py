@@ -213,3 +213,40 @@ def test_device_bounds():
     K.paged_attention_prefill(wl.q, kp, vp, wl.block_tables, bad_cu, wl.context_lens, cfg.softmax_scale,
                               max_q_len(wl), dev_err=err)
     assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS
+
+
+@pytest.mark.parametrize("dt", [W.CACHE_BF16, W.CACHE_FP8_TOKEN])
+def test_mixed_batch_is_ordered_on_the_callers_stream(dt):
+    """A mixed batch runs its one-token chunks on the library's side stream.
+    Work queued on the caller's (non-default) stream right after the call,
+    with no synchronisation in between, must see every output row: a copy
+    taken that way equals the oracle's result, and a second call that
+    overwrites the output on the same stream is not overtaken either."""
+    cfg = W.PrefillConfig("ordered", 3, 32, 8, 128, 16, 100, 1500, 200, 400, cache_dtype=dt, decode_seqs=64,
+                          decode_hist_lo=500, decode_hist_hi=3000)
+    wl_cpu = W.generate_prefill(cfg, 3)
+    wl = to_device(wl_cpu)
+    kp, vp = device_pools(wl)
+    if wl.token_scales:
+        wl.k_scale, wl.v_scale = W.scale_pools(wl.num_blocks, cfg.num_kv_heads, cfg.block_size, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.store_kvcache(wl.k_hist, wl.v_hist, kp, vp, wl.slot_hist, wl.k_scale, wl.v_scale, err)
+    K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, err)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = torch.full_like(wl.q, float("nan"))
+        K.paged_attention_prefill(wl.q, kp, vp, wl.block_tables, wl.cu_q_lens, wl.context_lens, cfg.softmax_scale,
+                                  max_q_len(wl), k_scale=wl.k_scale, v_scale=wl.v_scale, out=out, dev_err=err)
+        first = out.clone()  # queued right behind the call on s
+        out.fill_(float("nan"))
+        K.paged_attention_prefill(wl.q, kp, vp, wl.block_tables, wl.cu_q_lens, wl.context_lens, cfg.softmax_scale,
+                                  max_q_len(wl), k_scale=wl.k_scale, v_scale=wl.v_scale, out=out, dev_err=err)
+        second = out.clone()
+    s.synchronize()
+    assert K.read_device_error(err) == K.PKV_OK
+    assert bool(torch.isfinite(first.float()).all()) and torch.equal(first.view(torch.int16), second.view(torch.int16))
+    if dt == W.CACHE_BF16:
+        ref, _, _, rst = O.run_prefill_workload(wl_cpu, num_threads=8)
+        assert rst == O.ORC_OK
+        compare(first, ref, False, "mixed batch on a side stream")
