@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out", default="", help="also append the JSON line to this file")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step's kernels from Python instead of replaying CUDA graphs of the step")
     ap.add_argument("--no-shared-prefix", action="store_true",
                     help="attend a shared-prefix batch with the ordinary decode call instead of the cascade")
     ap.add_argument("--component", choices=["decode", "block_manager"], default="decode",
@@ -1292,11 +1294,10 @@ def main():
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    e_start.record(stream)
-    for k in range(Kst):
-        ev[k][0].record(stream)
+    def store():
         K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, step.dev_err)
-        ev[k][1].record(stream)
+
+    def decode():
         if shared:
             K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
                                                    step.groups[0], step.groups[1], step.groups[2], out=step.out,
@@ -1308,6 +1309,16 @@ def main():
                                      k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context,
                                      partition_request=args.partition, workspace=step.workspace,
                                      dev_err=step.dev_err, seq_order=order)
+
+    if not args.no_graph:  # each half of the step recorded once as a CUDA graph, replayed every step
+        store, decode = K.graphed(store), K.graphed(decode)
+        torch.cuda.synchronize()
+    e_start.record(stream)
+    for k in range(Kst):
+        ev[k][0].record(stream)
+        store()
+        ev[k][1].record(stream)
+        decode()
         ev[k][2].record(stream)
     e_end.record(stream)
     torch.cuda.synchronize()
@@ -1365,6 +1376,7 @@ def main():
                 "kv_tokens": wl.kv_tokens(), "seed": args.seed, "partition_tokens": pt,
                 "schedule": ("shared-prefix cascade: each group's prefix once per block of members, then the "
                              "suffixes" if shared else "longest sequence first (order from host lengths)"),
+                "launch": "Python calls" if args.no_graph else "CUDA graphs of the store and of the decode, replayed",
                 "parallelism": f"replicas x{world} (independent batches, no collective)",
                 "l2": f"no flush: {ab['kv'] / 1e9:.2f} GB of KV read per step, far above the 126 MB L2",
             },

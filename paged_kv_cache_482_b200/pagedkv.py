@@ -412,6 +412,27 @@ def version() -> int:
     return lib().pkv_version()
 
 
+def graphed(fn):
+    """Record ``fn()`` (library calls on fixed device tensors) once as a CUDA
+    graph and return a function that replays it on the current stream. ``fn``
+    runs once first, outside the capture, so that one-time set-up (kernel
+    attributes, the library's side stream) is done before recording."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+
+    def replay():
+        g.replay()
+
+    replay.graph = g
+    return replay
+
+
 class DecodeStep:
     """A decode step bound to resident pools: store the step's K/V, then attend.
 
