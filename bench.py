@@ -1343,6 +1343,7 @@ def main():
     d2h = host_out.numel() * host_out.element_size()
     for _ in range(3):
         step.run_host(*host_in, host_out)
+    step.flush(stream)  # the timed copies start after x0
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -1351,6 +1352,7 @@ def main():
     x0.record(stream)
     for _ in range(args.e2e_steps):
         step.run_host(*host_in, host_out)
+    step.flush(stream)  # x1 after the last output copy
     x1.record(stream)
     torch.cuda.synchronize()
     barrier()

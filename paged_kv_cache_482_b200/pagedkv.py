@@ -494,19 +494,75 @@ class DecodeStep:
                                       dev_err=self.dev_err, stream=stream, seq_order=seq_order)
 
     def run_host(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, out_host, stream=None):
-        """Host (pinned) inputs -> host output: the longest-first order is
-        computed from the host lengths, then H2D copies, the step, D2H copy."""
-        order = longest_first(context_lens)
-        host = (q, k_new, v_new, slot_mapping, block_tables, context_lens, order)
+        """One step from host (pinned) inputs to a host output: the end-to-end
+        form of the call. The longest-first order is computed from the host
+        lengths; the inputs are copied in on a copy stream into one of two sets
+        of device buffers, the step runs on ``stream`` (default: the current
+        stream), and the output is copied out on a second copy stream from one
+        of two device outputs. So the copies of one step overlap the kernels of
+        the steps around it, and nothing waits on the host unless it runs two
+        steps ahead of the GPU. Returns once queued; ``flush(stream)`` makes
+        ``stream`` wait for every queued output copy."""
+        cs = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream()
+        dev = self.k_cache.device
         if self._dev_inputs is None:
-            dev = self.k_cache.device
-            self._dev_inputs = [torch.empty_like(t, device=dev) for t in host]
-        for d_, h_ in zip(self._dev_inputs, host):
-            d_.copy_(h_, non_blocking=True)
-        dq, dk, dv, ds, dbt, dcl, dord = self._dev_inputs
-        if self.groups is not None:  # the step's groups come from the host too
-            self.groups[0].copy_(self._host_groups[0], non_blocking=True)
-            self.groups[1].copy_(self._host_groups[1], non_blocking=True)
-        o = self.run(dq, dk, dv, ds, dbt, dcl, stream, seq_order=dord)
-        out_host.copy_(o, non_blocking=True)
+            self._h2d, self._d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+            self._dev_inputs, self._outs, self._order_host = [], [], []
+            for _ in range(2):
+                self._dev_inputs.append([torch.empty(t.shape, dtype=t.dtype, device=dev)
+                                         for t in (q, k_new, v_new, slot_mapping, block_tables, context_lens)] +
+                                        [torch.empty(context_lens.shape, dtype=torch.int32, device=dev)])
+                self._outs.append(torch.empty_like(self.out))
+                self._order_host.append(torch.empty(context_lens.shape, dtype=torch.int32).pin_memory())
+            self._ev = {k: [None, None] for k in ("in_ready", "in_free", "out_free")}
+            self._flip = 0
+            self._primed = False
+        if not self._primed:  # the first copies start after what is already queued on cs
+            start = torch.cuda.Event()
+            start.record(cs)
+            self._h2d.wait_event(start)
+            self._primed = True
+        i = self._flip
+        self._flip ^= 1
+        ev = self._ev
+        if ev["in_ready"][i] is not None:
+            ev["in_ready"][i].synchronize()  # the pinned order buffer of two steps ago has been copied
+        self._order_host[i].copy_(longest_first(context_lens))
+        bufs = self._dev_inputs[i]
+        if ev["in_free"][i] is not None:
+            self._h2d.wait_event(ev["in_free"][i])  # the step two back is done reading set i
+        with torch.cuda.stream(self._h2d):
+            for d_, h_ in zip(bufs, (q, k_new, v_new, slot_mapping, block_tables, context_lens, self._order_host[i])):
+                d_.copy_(h_, non_blocking=True)
+            if self.groups is not None:  # the step's groups come from the host too
+                self.groups[0].copy_(self._host_groups[0], non_blocking=True)
+                self.groups[1].copy_(self._host_groups[1], non_blocking=True)
+        ev["in_ready"][i] = torch.cuda.Event()
+        ev["in_ready"][i].record(self._h2d)
+        cs.wait_event(ev["in_ready"][i])
+        if ev["out_free"][i] is not None:
+            cs.wait_event(ev["out_free"][i])  # the output copy of two steps ago is done with output i
+        dq, dk, dv, ds, dbt, dcl, dord = bufs
+        keep = self.out
+        self.out = self._outs[i]
+        try:
+            o = self.run(dq, dk, dv, ds, dbt, dcl, cs, seq_order=dord)
+        finally:
+            self.out = keep
+        ev["in_free"][i] = torch.cuda.Event()
+        ev["in_free"][i].record(cs)
+        self._d2h.wait_event(ev["in_free"][i])
+        with torch.cuda.stream(self._d2h):
+            out_host.copy_(o, non_blocking=True)
+        ev["out_free"][i] = torch.cuda.Event()
+        ev["out_free"][i].record(self._d2h)
         return out_host
+
+    def flush(self, stream=None):
+        """Make ``stream`` (default: current) wait for every output copy that
+        ``run_host`` queued; the next ``run_host`` starts a new pipeline."""
+        cs = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream()
+        if self._dev_inputs is not None:
+            cs.wait_stream(self._d2h)
+            cs.wait_stream(self._h2d)
+            self._primed = False
