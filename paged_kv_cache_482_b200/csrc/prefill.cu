@@ -542,20 +542,21 @@ bool prefill_supported(int head_dim, int group) {
 
 namespace {
 
-// The chunk kernels of a batch: the one-tile kernel for chunks of 2 ..
-// 128 / G tokens, the warp-specialised kernel for longer ones.
-cudaError_t launch_chunks(const PrefillArgs &a, int g, cudaStream_t stream) {
+// The warp-specialised kernel for the chunks longer than one query tile
+// (128 / G tokens); nothing when there are none.
+cudaError_t launch_long_chunks(const PrefillArgs &a, int g, cudaStream_t stream) {
+    if (a.max_q_len <= kRows / g) return cudaSuccess;
+    PrefillArgs large = a;
+    large.small_cut = kRows / g;
+    return launch_prefill_ws(large, stream);
+}
+
+// The one-tile kernel for chunks of 2 .. 128 / G tokens.
+cudaError_t launch_short_chunks(const PrefillArgs &a, int g, cudaStream_t stream) {
     PrefillArgs small = a;
     small.small_cut = kRows / g;
     small.small_min = 2;
     small.max_q_len = a.max_q_len < small.small_cut ? a.max_q_len : small.small_cut;
-    cudaError_t e = cudaSuccess;
-    if (a.max_q_len > small.small_cut) {  // the long chunks first: their few blocks should start first
-        PrefillArgs large = a;
-        large.small_cut = small.small_cut;
-        e = launch_prefill_ws(large, stream);
-        if (e != cudaSuccess) return e;
-    }
     if (a.fp8 && a.token_scales)
         return a.head_dim == 128 ? launch_d<128, true, true>(small, g, stream)
                                  : launch_d<64, true, true>(small, g, stream);
@@ -564,9 +565,10 @@ cudaError_t launch_chunks(const PrefillArgs &a, int g, cudaStream_t stream) {
 }
 
 // A low-priority stream per device, created on first use and kept for the
-// process: the one-token chunks of a mixed batch run on it, beside the chunk
-// kernels, so that their blocks fill the SMs the few long-chunk blocks leave
-// idle; the caller's stream waits for it before anything queued later.
+// process: the one-token and short chunks of a mixed batch run on it, beside
+// the long-chunk kernel, so that their many small blocks fill the SMs the few
+// long-chunk blocks leave idle; the caller's stream waits for it before
+// anything queued later.
 cudaStream_t side_stream() {
     constexpr int kMaxDevices = 64;
     static std::atomic<cudaStream_t> streams[kMaxDevices];
@@ -636,13 +638,15 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
         cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
         cudaGetLastError();  // no side stream: everything on the caller's stream
         if (fork) cudaEventDestroy(fork);
-        cudaError_t e = launch_decode(d, stream);
-        return e != cudaSuccess ? e : launch_chunks(a, g, stream);
+        cudaError_t e = launch_long_chunks(a, g, stream);
+        if (e == cudaSuccess) e = launch_decode(d, stream);
+        return e != cudaSuccess ? e : launch_short_chunks(a, g, stream);
     }
     cudaError_t e = cudaEventRecord(fork, stream);
-    if (e == cudaSuccess) e = launch_chunks(a, g, stream);
+    if (e == cudaSuccess) e = launch_long_chunks(a, g, stream);  // first: its few blocks start first
     if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
     if (e == cudaSuccess) e = launch_decode(d, side);
+    if (e == cudaSuccess) e = launch_short_chunks(a, g, side);
     // join even after a failure, so that nothing later on the caller's stream
     // overtakes work already queued on the side stream
     cudaError_t e2 = cudaEventRecord(join, side);

@@ -233,3 +233,60 @@ def test_norm_host_checks(K):
     assert call(eps=float("inf")) == K.PKV_ERR_INVALID_ARG
     assert call(T=-1) == K.PKV_ERR_INVALID_ARG
     assert call(T=0) == K.PKV_OK  # nothing launched
+
+
+def test_rope_store_host_checks(K):
+    L = K.lib()
+    ok = dict(q=0x10000, qo=0x11000, k=0x20000, v=0x30000, kc=0x40000, vc=0x50000, sm=0x60000, pos=0x70000,
+              cs=0x80000, mp=4096, style=0, N=4, nq=32, nkv=8, d=128, bs=16, nblk=10, dt=0, ks=None, vs=None)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.pkv_store_kvcache_rope(a["q"], a["qo"], a["k"], a["v"], a["kc"], a["vc"], a["sm"], a["pos"],
+                                        a["cs"], a["mp"], a["style"], a["N"], a["nq"], a["nkv"], a["d"], a["bs"],
+                                        a["nblk"], a["dt"], a["ks"], a["vs"], None, None)
+
+    assert call(d=24) == K.PKV_ERR_INVALID_ARG          # not a multiple of 16
+    assert call(d=48) == K.PKV_ERR_UNSUPPORTED          # 3 lanes per row
+    assert call(style=2) == K.PKV_ERR_INVALID_ARG
+    assert call(qo=None) == K.PKV_ERR_INVALID_ARG        # q without q_out
+    assert call(mp=0) == K.PKV_ERR_INVALID_ARG
+    assert call(cs=0x80008) == K.PKV_ERR_INVALID_ARG     # table not 16-byte aligned
+    assert call(dt=1) == K.PKV_ERR_INVALID_ARG           # E4M3 without scales
+    assert call(pos=None) == K.PKV_ERR_INVALID_ARG
+    assert call(N=0) == K.PKV_OK
+    assert call(N=0, q=None, qo=None, k=None, v=None, pos=None, cs=None, sm=None) == K.PKV_OK
+
+
+def test_shared_prefix_plan_and_host_checks(K):
+    L = K.lib()
+    for dt in (K.PKV_CACHE_BF16, K.PKV_CACHE_FP8_E4M3, K.PKV_CACHE_FP8_E4M3_TOKEN):
+        for part in (0, 256, -1):
+            plain = K.plan_decode(512, 32, 8, 128, 256, 1536, dt != K.PKV_CACHE_BF16, part)
+            shared = K.plan_decode_shared_prefix(512, 32, 8, 128, 256, 1536, dt, part)
+            np_suffix = plain["max_partitions"] if plain["partition_tokens"] else 1
+            assert shared["max_partitions"] == np_suffix + 1  # slot 0 holds the shared prefix
+            assert shared["workspace_bytes"] >= 512 * 32 * shared["max_partitions"] * 130 * 4
+            assert shared["partition_tokens"] == (plain["partition_tokens"] or 1536)
+    # head_dim 64 has no prefix kernel: the plan is the ordinary one
+    assert K.plan_decode_shared_prefix(8, 8, 2, 64, 16, 900) == K.plan_decode(8, 8, 2, 64, 16, 900)
+
+    def call(**kw):
+        a = dict(q=0x10000, kc=0x20000, vc=0x30000, bt=0x40000, maxb=8, cl=0x50000, S=4, nq=32, nkv=8, d=128,
+                 bs=256, nblk=100, scale=0.088, dt=0, ks=None, vs=None, maxctx=2048, cu=0x60000, pre=0x61000,
+                 ng=2, mg=3, part=0, ws=None, wsb=0, out=0x70000)
+        a.update(kw)
+        return L.pkv_paged_attention_decode_shared_prefix(
+            a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cl"], a["S"], a["nq"], a["nkv"], a["d"], a["bs"],
+            a["nblk"], a["scale"], a["dt"], a["ks"], a["vs"], a["maxctx"], a["cu"], a["pre"], a["ng"], a["mg"],
+            a["part"], a["ws"], a["wsb"], a["out"], None, None)
+
+    assert call(ng=-1) == K.PKV_ERR_INVALID_ARG
+    assert call(cu=None) == K.PKV_ERR_INVALID_ARG
+    assert call(mg=0) == K.PKV_ERR_INVALID_ARG
+    assert call(ws=None) == K.PKV_ERR_WORKSPACE           # the prefix slot always needs scratch
+    assert call(ws=0x90000, wsb=64) == K.PKV_ERR_WORKSPACE
+    assert call(ws=0x90010, wsb=1 << 30) == K.PKV_ERR_INVALID_ARG  # not 256-byte aligned
+    assert call(q=0x10008, ws=0x90000, wsb=1 << 30) == K.PKV_ERR_INVALID_ARG
+    assert call(S=0, ws=0x90000, wsb=1 << 30) == K.PKV_OK

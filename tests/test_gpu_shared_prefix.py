@@ -80,7 +80,7 @@ def mixed_groups(dt, g=4, bs=16, seed=0):
     return W.merge(parts)
 
 
-CASES = [(dt, g) for dt in (W.CACHE_BF16, W.CACHE_FP8, W.CACHE_FP8_TOKEN) for g in (1, 4, 8)]
+CASES = [(dt, g) for dt in (W.CACHE_BF16, W.CACHE_FP8, W.CACHE_FP8_TOKEN) for g in (1, 4, 8)] + [(W.CACHE_BF16, 2)]
 
 
 @pytest.mark.parametrize("dt,g", CASES, ids=[f"{dt}-g{g}" for dt, g in CASES])
