@@ -361,10 +361,10 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  *
  * Routing: one-token chunks run in the decode kernel, chunks of up to 128 / G
  * tokens in a one-tile kernel, longer ones in a warp-specialised kernel.
- * When the batch has chunks longer than one token (max_q_len > 1), the first
- * two run on the library's low-priority stream of this device, beside the
- * long-chunk kernel on the given stream (forked from and joined back into it
- * with events), so that their many small blocks use the SMs the long
+ * When the batch has chunks longer than one token (max_q_len > 1), the
+ * one-token chunks run on the library's low-priority stream of this device,
+ * beside the chunk kernels on the given stream (forked from and joined back
+ * into it with events), so that their many small blocks use the SMs the long
  * chunks' few blocks leave idle.
  */
 PKV_API int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *v_cache,
