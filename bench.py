@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--out", default="", help="also append the JSON line to this file")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step's kernels from Python instead of replaying CUDA graphs of the step")
+    ap.add_argument("--no-staging", action="store_true",
+                    help="E4M3 prefill: widen the codes in every CTA instead of once into a workspace")
     ap.add_argument("--no-shared-prefix", action="store_true",
                     help="attend a shared-prefix batch with the ordinary decode call instead of the cascade")
     ap.add_argument("--component", choices=["decode", "block_manager"], default="decode",
@@ -740,11 +742,19 @@ def run_prefill(args):
     cu = wl.cu_q_lens.cpu().long()
     mq = int((cu[1:] - cu[:-1]).max())
     out = torch.empty_like(wl.q)
+    # E4M3: the widening workspace (allocated once, like a serving engine would)
+    ws = None
+    if wl.is_fp8 and not args.no_staging:
+        nbytes = K.prefill_workspace_bytes(wl.block_tables.shape[0], c.num_kv_heads, c.head_dim,
+                                           wl.block_tables.shape[1], c.block_size,
+                                           K.PKV_CACHE_FP8_E4M3_TOKEN if wl.token_scales else K.PKV_CACHE_FP8_E4M3)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda") if nbytes else None
+    long_chunks = mq > 128 // c.group
 
     def step(q, k_new, v_new, slot_new, bt, cu_d, cl):
         K.store_kvcache(k_new, v_new, kp, vp, slot_new, wl.k_scale, wl.v_scale, err)
         K.paged_attention_prefill(q, kp, vp, bt, cu_d, cl, c.softmax_scale, mq, out=out, k_scale=wl.k_scale,
-                                  v_scale=wl.v_scale, dev_err=err)
+                                  v_scale=wl.v_scale, dev_err=err, workspace=ws)
 
     inputs = (wl.q, wl.k_new, wl.v_new, wl.slot_new, wl.block_tables, wl.cu_q_lens, wl.context_lens)
     stream = torch.cuda.current_stream()
@@ -769,7 +779,7 @@ def run_prefill(args):
         K.store_kvcache(wl.k_new, wl.v_new, kp, vp, wl.slot_new, wl.k_scale, wl.v_scale, err)
         ev[k][1].record(stream)
         K.paged_attention_prefill(wl.q, kp, vp, wl.block_tables, wl.cu_q_lens, wl.context_lens, c.softmax_scale, mq,
-                                  out=out, k_scale=wl.k_scale, v_scale=wl.v_scale, dev_err=err)
+                                  out=out, k_scale=wl.k_scale, v_scale=wl.v_scale, dev_err=err, workspace=ws)
         ev[k][2].record(stream)
     e_end.record(stream)
     torch.cuda.synchronize()
@@ -823,22 +833,27 @@ def run_prefill(args):
             "dtype": prefill_dtype(wl), "data": "synthetic",
             "config": {"workload": prefill_desc(c), "query_tokens": T, "kv_tokens": int(wl.context_lens.sum()),
                        "max_q_len": mq, "seed": args.seed,
+                       "e4m3_widening": (None if not wl.is_fp8 else
+                                         "once per call into a workspace" if ws is not None else "in every CTA"),
                        "parallelism": f"replicas x{world} (independent batches, no collective)",
                        "l2": "no flush: each step's pools and queries exceed 126 MB of L2"},
             "attention_us": attn_ms * 1e3, "store_us": store_ms * 1e3,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                          "frac": achieved / peak_sus, "traffic": None,
-                         "kernel": "paged_prefill_kernel" if wl.is_fp8 else "paged_prefill_ws_kernel (+ paged_prefill_kernel)",
+                         "kernel": ("paged_prefill_ws_kernel (+ widen_kv_kernel, paged_prefill_kernel, decode)"
+                                    if ws is not None and long_chunks else
+                                    "paged_prefill_ws_kernel (+ paged_prefill_kernel, decode)"),
                          "peak_source": f"{kind} cuBLAS bf16 GEMM, sustained (bf16_tflops_sustained); "
                                         f"burst {peak_burst}",
                          "algorithmic_flops_per_launch": flops,
                          "flops_note": "causal: 4 * head_dim FLOPs per (query row, head, key at or before it)"},
             "e2e": {"value": world * T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "query tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
-            # per step: the store, and for a bf16 cache the one-tile kernel (short
-            # chunks) plus, when some chunk is longer than 128 / G tokens, the
-            # warp-specialised kernel; an E4M3 cache has one prefill kernel
-            "gpu_launches": (1 + (1 if wl.is_fp8 else (2 if mq > 128 // c.group else 1))) * Kst,
+            # per step: the store, the one-tile kernel (short chunks), the decode
+            # kernel (one-token chunks) and, when some chunk is longer than
+            # 128 / G tokens, the warp-specialised kernel (after the widening
+            # kernel when an E4M3 workspace is given)
+            "gpu_launches": (2 if mq <= 1 else 3 + (1 + (1 if ws is not None else 0) if long_chunks else 0)) * Kst,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:

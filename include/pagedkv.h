@@ -349,6 +349,19 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  *  context_lens  [num_seqs] int32, c_i <= context_lens[i] <=
  *                max_blocks_per_seq * block_size
  *  max_q_len     host-known bound on every c_i (sizes the grid)
+ *  workspace     optional, E4M3 cache only (ignored for bf16; may be NULL):
+ *                at least pkv_prefill_workspace_bytes(...) bytes, 16-byte
+ *                aligned, owned by the caller, contents not kept between
+ *                calls. With it, the codes of the sequences whose chunks are
+ *                longer than 128 / G tokens are widened once per call into
+ *                dense 16-bit rows there (K f16; V f16, or bf16 with
+ *                per-token scales; the per-token scales as fp32 rows; zeros
+ *                past the context), and the warp-specialised kernel copies
+ *                its tiles from there instead of widening the codes in every
+ *                CTA: the same operand values, so the same result for finite
+ *                cache contents. NULL: the CTAs widen the codes themselves.
+ *                A non-NULL workspace smaller than a nonzero bound returns
+ *                PKV_ERR_WORKSPACE and launches nothing.
  *  out           [total_q][num_q_heads][head_dim] bf16
  *
  * Host checks: pointers non-null, q / caches / out 16-byte aligned,
@@ -372,8 +385,21 @@ PKV_API int pkv_paged_attention_prefill(const void *q, const void *k_cache, cons
                                         const int32_t *cu_q_lens, const int32_t *context_lens, int num_seqs,
                                         int total_q, int num_q_heads, int num_kv_heads, int head_dim,
                                         int block_size, int64_t num_blocks, float scale, int cache_dtype,
-                                        const float *k_scale, const float *v_scale, int max_q_len, void *out,
-                                        int *dev_err, void *stream);
+                                        const float *k_scale, const float *v_scale, int max_q_len,
+                                        void *workspace, size_t workspace_bytes, void *out, int *dev_err,
+                                        void *stream);
+
+/*
+ * pkv_prefill_workspace_bytes: size of the optional widening workspace of
+ * pkv_paged_attention_prefill for an E4M3 cache:
+ *   num_seqs * num_kv_heads * R * (4 * head_dim + (per-token scales ? 8 : 0))
+ * with R = max_blocks_per_seq * block_size rounded up to a multiple of 128
+ * (the table's capacity: one run of R staging rows per sequence and KV
+ * head). 0 for a bf16 cache, for arguments below 1, and when the staging
+ * would have 2^31 rows or more (the call then widens in its CTAs).
+ */
+PKV_API size_t pkv_prefill_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                                           int block_size, int cache_dtype);
 
 /*
  * pkv_fused_add_rmsnorm: the residual add and RMSNorm around attention in

@@ -341,12 +341,19 @@ int pkv_paged_attention_decode(const void *q, const void *k_cache, const void *v
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+size_t pkv_prefill_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                                   int block_size, int cache_dtype) {
+    if (!valid_dtype(cache_dtype)) return 0;
+    return pkv::prefill_workspace_bytes(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
+                                        cache_dtype != PKV_CACHE_BF16, cache_dtype == PKV_CACHE_FP8_E4M3_TOKEN);
+}
+
 int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *v_cache,
                                 const int32_t *block_tables, int max_blocks_per_seq, const int32_t *cu_q_lens,
                                 const int32_t *context_lens, int num_seqs, int total_q, int num_q_heads,
                                 int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, float scale,
-                                int cache_dtype, const float *k_scale, const float *v_scale, int max_q_len, void *out,
-                                int *dev_err, void *stream) {
+                                int cache_dtype, const float *k_scale, const float *v_scale, int max_q_len,
+                                void *workspace, size_t workspace_bytes, void *out, int *dev_err, void *stream) {
     if (num_seqs < 0 || total_q < 0 || num_q_heads < 1 || num_kv_heads < 1) return PKV_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
     if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
@@ -359,6 +366,14 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
     if (max_blocks_per_seq < 1 || num_blocks < 1 || num_blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || scale > 3.0e38f) return PKV_ERR_INVALID_ARG;  // positive and finite
+    if (workspace && !aligned16(workspace)) return PKV_ERR_INVALID_ARG;
+    // the widening workspace: used by an E4M3 cache when its bound is nonzero
+    size_t staging_need = 0;
+    if (workspace && fp8) {
+        staging_need = pkv_prefill_workspace_bytes(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
+                                                   cache_dtype);
+        if (staging_need && workspace_bytes < staging_need) return PKV_ERR_WORKSPACE;
+    }
     if (num_seqs == 0 || total_q == 0) return PKV_OK;
     if (max_q_len < 1) return PKV_ERR_INVALID_ARG;
 
@@ -386,6 +401,10 @@ int pkv_paged_attention_prefill(const void *q, const void *k_cache, const void *
     a.out = out;
     a.dev_err = dev_err;
     a.small_cut = 0;
+    if (staging_need) {
+        a.staging = workspace;
+        a.staging_stride = pkv::prefill_staging_stride(max_blocks_per_seq, block_size);
+    }
     cudaError_t e = pkv::launch_prefill(a, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidConfiguration) return PKV_ERR_UNSUPPORTED;
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;

@@ -100,7 +100,18 @@ struct PrefillArgs {
     // the one-tile kernel skips chunks shorter than this (one-token chunks
     // go to the decode kernel when it is 2)
     int small_min = 0;
+    // E4M3 only, may be null: the widening workspace (prefill_ws.cu, Staging)
+    // and its rows per (sequence, KV head), a multiple of 128
+    void *staging = nullptr;
+    int staging_stride = 0;
 };
+
+// Staging rows per (sequence, KV head) of the E4M3 prefill workspace (the
+// table capacity rounded up to 128) and the workspace's bytes; 0 when there
+// is no staging (bf16 cache, or more rows than int32 tensor-map coordinates).
+int prefill_staging_stride(int max_blocks_per_seq, int block_size);
+size_t prefill_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq, int block_size,
+                               bool fp8, bool token_scales);
 
 struct NormArgs {
     const void *x;   // [num_tokens][hidden] bf16

@@ -42,6 +42,14 @@
 // scores are scaled by column, P is multiplied by the V scales before it is
 // rounded, and P V runs in bf16 (V widened to bf16), since P times a V scale
 // may leave f16 range.
+// With a workspace (E4M3 only), a widening kernel first expands the codes of
+// the sequences with long chunks once into dense 16-bit rows (K f16; V f16,
+// or bf16 with per-token scales; the per-token scales as fp32 rows), one
+// run of rows per (sequence, KV head), zeros past the context; warp 8 is then
+// a tensor-map producer as for a bf16 cache (one copy per 64-column half of a
+// 128-token tile, plus two 512-byte copies of the tile's scales), and no CTA
+// widens anything. The operands the MMAs see are the same 16-bit values, so
+// the result is the same as with the converter warps.
 // Everything between roles goes through mbarriers (full / empty K/V stages,
 // S ready, P ready, O done); every wait is bounded (1 s) and reports
 // PKV_DEVERR_TIMEOUT. The softmax uses the same arithmetic as prefill.cu:
@@ -124,10 +132,117 @@ __device__ __forceinline__ void ws_kv_tile(const CUtensorMap *mk, const CUtensor
     }
 }
 
-template <int D, int G, bool FP8, bool TS>
-__global__ void __launch_bounds__(ws_threads<FP8>(), 1)
+// Dense staging of E4M3 K/V (workspace layout): rows of D 16-bit values,
+// row (s * num_kv_heads + kv head) * staging_stride + position; K rows, then V
+// rows, then (per-token scales) the K and V scales as fp32, one per row.
+struct Staging {
+    uint16_t *k;
+    uint16_t *v;
+    float *k_scale;
+    float *v_scale;
+};
+
+template <int D>
+__host__ __device__ __forceinline__ Staging staging_of(const PrefillArgs &a) {
+    const long long rows = static_cast<long long>(a.num_seqs) * a.num_kv_heads * a.staging_stride;
+    Staging st;
+    st.k = static_cast<uint16_t *>(a.staging);
+    st.v = st.k + rows * D;
+    st.k_scale = reinterpret_cast<float *>(st.v + rows * D);
+    st.v_scale = st.k_scale + rows;
+    return st;
+}
+
+// Widening of the E4M3 K/V codes into the staging rows, one unit = 128 rows
+// of one (sequence, KV head), for the sequences whose chunks the
+// warp-specialised kernel takes (longer than small_cut). Rows past the
+// context are written as zeros; units wholly past it are never read and are
+// skipped. Sequences the attention kernel will reject (bad cu_q_lens or
+// lengths) are skipped; a block id outside the pool gives zero rows (the
+// attention kernel reports it).
+template <int D, bool TS>
+__global__ void __launch_bounds__(256) widen_kv_kernel(PrefillArgs a, int log2_bs, long long units) {
+    constexpr int kCPR = D / 16;  // 16-code chunks per row
+    const int tiles = a.staging_stride / kBN;
+    const Staging st = staging_of<D>(a);
+    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+        const int tile = static_cast<int>(u % tiles);
+        const long long sk = u / tiles;  // s * num_kv_heads + kv head
+        const int kh = static_cast<int>(sk % a.num_kv_heads);
+        const int s = static_cast<int>(sk / a.num_kv_heads);
+        const int q0 = a.cu_q_lens[s], q1 = a.cu_q_lens[s + 1];
+        if (q0 < 0 || q1 < q0 || q1 > a.total_q) continue;
+        const int c = q1 - q0;
+        if (c <= a.small_cut || c > a.max_q_len) continue;
+        const int ctx = a.context_lens[s];
+        if (ctx < c || static_cast<long long>(ctx) > static_cast<long long>(a.max_blocks_per_seq) * a.block_size)
+            continue;
+        const int t0 = tile * kBN;
+        if (t0 >= ctx) continue;
+        const int32_t *table = a.block_tables + static_cast<long long>(s) * a.max_blocks_per_seq;
+        const long long drow0 = sk * a.staging_stride + t0;
+        for (int i = threadIdx.x; i < kBN * kCPR; i += blockDim.x) {
+            const int r = i / kCPR, cc = i % kCPR, t = t0 + r;
+            uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0, v0 = k0, v1 = k0;
+            if (t < ctx) {
+                const int b = __ldg(table + (t >> log2_bs));
+                if (b >= 0 && b < a.num_blocks) {
+                    const long long prow = (static_cast<long long>(b) * a.num_kv_heads + kh) * a.block_size +
+                                           (t & (a.block_size - 1));
+                    const uint4 kc = __ldg(reinterpret_cast<const uint4 *>(
+                        static_cast<const uint8_t *>(a.k_cache) + prow * D + cc * 16));
+                    const uint4 vc = __ldg(reinterpret_cast<const uint4 *>(
+                        static_cast<const uint8_t *>(a.v_cache) + prow * D + cc * 16));
+                    const uint2 h0 = e4m3x4_to_f16x4(kc.x), h1 = e4m3x4_to_f16x4(kc.y);
+                    const uint2 h2 = e4m3x4_to_f16x4(kc.z), h3 = e4m3x4_to_f16x4(kc.w);
+                    k0 = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    k1 = make_uint4(h2.x, h2.y, h3.x, h3.y);
+                    if constexpr (TS) {  // P V runs in bf16 with per-token scales
+                        v0 = e4m3x8_to_bf16x8(make_uint2(vc.x, vc.y));
+                        v1 = e4m3x8_to_bf16x8(make_uint2(vc.z, vc.w));
+                    } else {
+                        const uint2 g0 = e4m3x4_to_f16x4(vc.x), g1 = e4m3x4_to_f16x4(vc.y);
+                        const uint2 g2 = e4m3x4_to_f16x4(vc.z), g3 = e4m3x4_to_f16x4(vc.w);
+                        v0 = make_uint4(g0.x, g0.y, g1.x, g1.y);
+                        v1 = make_uint4(g2.x, g2.y, g3.x, g3.y);
+                    }
+                }
+            }
+            uint4 *kd = reinterpret_cast<uint4 *>(st.k + (drow0 + r) * D + cc * 16);
+            uint4 *vd = reinterpret_cast<uint4 *>(st.v + (drow0 + r) * D + cc * 16);
+            kd[0] = k0;
+            kd[1] = k1;
+            vd[0] = v0;
+            vd[1] = v1;
+        }
+        if constexpr (TS) {
+            for (int r = threadIdx.x; r < kBN; r += blockDim.x) {
+                const int t = t0 + r;
+                float ks = 0.0f, vs = 0.0f;
+                if (t < ctx) {
+                    const int b = __ldg(table + (t >> log2_bs));
+                    if (b >= 0 && b < a.num_blocks) {
+                        const long long prow = (static_cast<long long>(b) * a.num_kv_heads + kh) * a.block_size +
+                                               (t & (a.block_size - 1));
+                        ks = __ldg(a.k_scale + prow);
+                        vs = __ldg(a.v_scale + prow);
+                    }
+                }
+                st.k_scale[drow0 + r] = ks;
+                st.v_scale[drow0 + r] = vs;
+            }
+        }
+    }
+}
+
+// STG (E4M3 only): K/V tiles come from the staging rows by tensor-map copies
+// (map_k / map_v cover the staging instead of the pools); otherwise E4M3
+// codes are widened by the converter warps.
+template <int D, int G, bool FP8, bool TS, bool STG>
+__global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
     paged_prefill_ws_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
                             const __grid_constant__ CUtensorMap map_v) {
+    constexpr bool CONV = FP8 && !STG;  // converter warps widen the codes
     using L = WsLayout<D>;
     constexpr int TQ = kRowsT / G;  // chunk tokens per query tile
     // bf16 cache: bf16 operands. E4M3 cache: f16 operands for S (one conversion
@@ -172,7 +287,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                c > a.max_q_len;
     if (!bad) {
         const int nblk_seq = (ctx + a.block_size - 1) >> log2_bs;
-        for (int i = tid; i < nblk_seq; i += ws_threads<FP8>()) {
+        for (int i = tid; i < nblk_seq; i += ws_threads<CONV>()) {
             const int32_t b = table_g[i];
             if (b < 0 || b >= a.num_blocks) bad = true;
             if (i < kTableCap) table_s[i] = b;
@@ -202,7 +317,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
     if (warp == kMmaWarp) tmem_alloc(smem_addr(&bars->tmem), kTmemCols);
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bars->kv_full[i], FP8 ? kConvWarps : 1);
+            mbar_init(&bars->kv_full[i], CONV ? kConvWarps : 1);
             mbar_init(&bars->kv_empty[i], 1);
         }
         for (int x = 0; x < 2; ++x) {
@@ -411,28 +526,49 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
             if (row == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
         }
         __syncwarp();
-    } else if (!FP8 && warp == kProducerWarp) {
-        // ================================================ producer (bf16)
+    } else if (!CONV && warp == kProducerWarp) {
+        // ================================================ producer (bf16 pools, or E4M3 staging rows)
         int issued = 0;
         if (lane == 0) {
+            const int srow0 = (s * a.num_kv_heads + kh) * a.staging_stride;  // staging: int32 (host-checked)
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kStages, use = j / kStages;
                 if (use > 0 && !mbar_wait(&bars->kv_empty[st], static_cast<uint32_t>((use - 1) & 1))) {
                     set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
                     break;
                 }
-                ws_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, j, kv_end, kbuf(j),
-                              vbuf(j), &bars->kv_full[st]);
+                if constexpr (STG) {
+                    uint64_t *bar = &bars->kv_full[st];
+                    const int row = srow0 + j * kBN;
+                    mbar_arrive_expect_tx(bar, 2u * (D / 64) * kBN * 128u + (TS ? 2u * kBN * 4u : 0u));
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) {
+                        tma_load_2d(kbuf(j) + h * kBN * 128, &map_k, h * 64, row, bar);
+                        tma_load_2d(vbuf(j) + h * kBN * 128, &map_v, h * 64, row, bar);
+                    }
+                    if constexpr (TS) {
+                        const Staging sg = staging_of<D>(a);
+                        float *tsc = reinterpret_cast<float *>(sm + L::kScales) + st * 2 * kBN;
+                        bulk_g2s(tsc, sg.k_scale + row, kBN * 4, bar);
+                        bulk_g2s(tsc + kBN, sg.v_scale + row, kBN * 4, bar);
+                    }
+                } else {
+                    ws_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, j, kv_end,
+                                  kbuf(j), vbuf(j), &bars->kv_full[st]);
+                }
                 issued = j + 1;
             }
         }
         issued = __shfl_sync(0xffffffffu, issued, 0);
-        // V rows past the causal end on the last tile: zero them, so that a
-        // zero weight times stale pool data stays zero.
+        // V rows past the causal end on the last tile (bf16 pools): zero them,
+        // so that a zero weight times stale pool data stays zero. The staging
+        // rows past the context are zeros already, and the rows between the
+        // causal end and the context hold cached values (finite for finite
+        // data), so a zero weight gives zero there too.
         const int last = n_tiles - 1;
         const int valid_rows = kv_end - last * kBN;
         bool tail_ok = issued == n_tiles;
-        if (tail_ok && valid_rows < kBN) {
+        if (!STG && tail_ok && valid_rows < kBN) {
             tail_ok = mbar_wait(&bars->kv_full[last % kStages], static_cast<uint32_t>((last / kStages) & 1));
             if (tail_ok) {
                 constexpr int kHalves = D / 64;
@@ -452,7 +588,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
                 mbar_wait(&bars->kv_full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
         }
         __syncwarp();
-    } else if (FP8 && warp != kMmaWarp) {
+    } else if (CONV && warp != kMmaWarp) {
         // ================================================ E4M3 converters (warps 8, 10, 11)
         // Each thread loads 16-code chunks of the tile's K and V rows, widens
         // them exactly to f16 and stores them into the swizzled stage the
@@ -583,7 +719,7 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
             // j + 1 is awaited only after P V_A(j) is on the tensor pipe
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const bool more = j + 1 < n_tiles;
-                if (!FP8 && !more) ok = mbar_wait(&bars->vtail, 0);  // E4M3: converters zero the tail
+                if (!FP8 && !more) ok = mbar_wait(&bars->vtail, 0);  // E4M3: converters or staging zero the tail
                 for (int x = 0; x < 2 && ok; ++x) {
                     if (!mbar_wait(&bars->p_full[x], static_cast<uint32_t>(j & 1))) {
                         ok = false;
@@ -617,6 +753,20 @@ __global__ void __launch_bounds__(ws_threads<FP8>(), 1)
     }
 }
 
+// The staging rows as a 2-D tensor of 16-bit elements: boxes of 64 columns x
+// 128 rows, 128-byte swizzle (the layout the converters write).
+inline bool make_staging_map(CUtensorMap *map, const void *base, long long rows, int head_dim) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBN)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int G, bool FP8, bool TS>
 cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int TQ = kRowsT / G;
@@ -630,15 +780,38 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     CUtensorMap mk, mv;
     memset(&mk, 0, sizeof(mk));
     memset(&mv, 0, sizeof(mv));
-    // the E4M3 path loads the codes with plain loads: no tensor maps
+    const dim3 grid(static_cast<unsigned>(nx), a.num_kv_heads);
+    if (FP8 && a.staging) {
+        // widen once into the staging rows, then copy tiles from there
+        const long long rows = static_cast<long long>(a.num_seqs) * a.num_kv_heads * a.staging_stride;
+        if (rows > 0x7FFFFFFFLL || a.staging_stride % kBN != 0) return cudaErrorInvalidConfiguration;
+        const Staging st = staging_of<D>(a);
+        if (!make_staging_map(&mk, st.k, rows, D) || !make_staging_map(&mv, st.v, rows, D))
+            return cudaErrorInvalidValue;
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return cudaGetLastError();
+        const long long units = rows / kBN;
+        const long long wblocks = units < 16LL * sms ? units : 16LL * sms;
+        widen_kv_kernel<D, TS><<<static_cast<unsigned>(wblocks), 256, 0, stream>>>(a, log2_bs, units);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        auto kern = paged_prefill_ws_kernel<D, G, true, TS, true>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(WsLayout<D>::kAlloc));
+        if (e != cudaSuccess) return e;
+        kern<<<grid, ws_threads<false>(), WsLayout<D>::kAlloc, stream>>>(a, tiles, log2_bs, mk, mv);
+        return cudaGetLastError();
+    }
+    // the E4M3 path without staging loads the codes with plain loads: no tensor maps
     if (!FP8 && (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)))
         return cudaErrorInvalidValue;
-    auto kern = paged_prefill_ws_kernel<D, G, FP8, TS>;
+    auto kern = paged_prefill_ws_kernel<D, G, FP8, TS, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(WsLayout<D>::kAlloc));
     if (e != cudaSuccess) return e;
-    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), ws_threads<FP8>(), WsLayout<D>::kAlloc, stream>>>(
-        a, tiles, log2_bs, mk, mv);
+    kern<<<grid, ws_threads<FP8>(), WsLayout<D>::kAlloc, stream>>>(a, tiles, log2_bs, mk, mv);
     return cudaGetLastError();
 }
 
@@ -654,6 +827,22 @@ cudaError_t launch_ws_g(const PrefillArgs &a, int g, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int prefill_staging_stride(int max_blocks_per_seq, int block_size) {
+    const long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;
+    const long long stride = (cap + kBN - 1) / kBN * kBN;
+    return stride > 0x7FFFFFFFLL ? 0 : static_cast<int>(stride);
+}
+
+size_t prefill_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq, int block_size,
+                               bool fp8, bool token_scales) {
+    if (!fp8 || num_seqs < 1 || num_kv_heads < 1 || head_dim < 1 || max_blocks_per_seq < 1 || block_size < 1)
+        return 0;
+    const long long stride = prefill_staging_stride(max_blocks_per_seq, block_size);
+    const long long rows = static_cast<long long>(num_seqs) * num_kv_heads * stride;
+    if (stride == 0 || rows > 0x7FFFFFFFLL) return 0;
+    return static_cast<size_t>(rows) * (4u * static_cast<size_t>(head_dim) + (token_scales ? 8u : 0u));
+}
 
 cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;

@@ -15,6 +15,7 @@ The functions mirror ``include/pagedkv.h``:
 * ``plan_decode_shared_prefix`` / ``paged_attention_decode_shared_prefix`` --
   ``pkv_plan_decode_shared_prefix`` / ``pkv_paged_attention_decode_shared_prefix``
 * ``paged_attention_prefill`` -- ``pkv_paged_attention_prefill``
+* ``prefill_workspace_bytes`` -- ``pkv_prefill_workspace_bytes``
 * ``fused_add_rmsnorm`` -- ``pkv_fused_add_rmsnorm``
 * ``read_device_error`` -- ``pkv_read_device_error``
 """
@@ -41,10 +42,11 @@ PKV_CACHE_BF16 = 0
 PKV_CACHE_FP8_E4M3 = 1  # k_scale / v_scale: [num_kv_heads] fp32
 PKV_CACHE_FP8_E4M3_TOKEN = 2  # k_scale / v_scale: scale pools [num_blocks, num_kv_heads, block_size] fp32
 
-EXPORTED = ("pkv_store_kvcache", "pkv_store_kvcache_rope", "pkv_plan_decode", "pkv_decode_workspace_bytes", "pkv_plan_decode_shared_prefix",
-            "pkv_paged_attention_decode_shared_prefix", "pkv_paged_attention_decode", "pkv_status_string",
-            "pkv_read_device_error", "pkv_version", "pkv_paged_attention_decode_static_scratch",
-            "pkv_paged_attention_prefill", "pkv_fused_add_rmsnorm")
+EXPORTED = ("pkv_store_kvcache", "pkv_store_kvcache_rope", "pkv_plan_decode", "pkv_decode_workspace_bytes",
+            "pkv_plan_decode_shared_prefix", "pkv_paged_attention_decode_shared_prefix",
+            "pkv_paged_attention_decode", "pkv_status_string", "pkv_read_device_error", "pkv_version",
+            "pkv_paged_attention_decode_static_scratch", "pkv_paged_attention_prefill",
+            "pkv_prefill_workspace_bytes", "pkv_fused_add_rmsnorm")
 
 
 class PagedKVError(RuntimeError):
@@ -103,8 +105,10 @@ def load_library(path: str):
     L.pkv_version.argtypes = []
     L.pkv_version.restype = i32
     L.pkv_paged_attention_prefill.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i64, f32,
-                                              i32, vp, vp, i32, vp, vp, vp]
+                                              i32, vp, vp, i32, vp, sz, vp, vp, vp]
     L.pkv_paged_attention_prefill.restype = i32
+    L.pkv_prefill_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.pkv_prefill_workspace_bytes.restype = sz
     L.pkv_fused_add_rmsnorm.argtypes = [vp, vp, vp, vp, i32, i32, f32, vp]
     L.pkv_fused_add_rmsnorm.restype = i32
     if hasattr(L, "pkv_paged_attention_decode_static_scratch"):
@@ -347,12 +351,22 @@ def paged_attention_decode_static_scratch(q, k_cache, v_cache, block_tables, con
 STATIC_SCRATCH_BYTES = 32 << 20  # PKV_STATIC_SCRATCH_BYTES
 
 
+def prefill_workspace_bytes(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq, block_size, cache_dtype) -> int:
+    """Bytes of the optional E4M3 widening workspace of ``paged_attention_prefill``
+    (0 for a bf16 cache, or when the staging does not fit int32 rows)."""
+    return int(lib().pkv_prefill_workspace_bytes(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
+                                                 cache_dtype))
+
+
 def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, scale, max_q_len,
-                            out=None, k_scale=None, v_scale=None, dev_err=None, stream=None):
+                            out=None, k_scale=None, v_scale=None, dev_err=None, stream=None, workspace=None):
     """Chunked prefill: each sequence's chunk of query tokens (rows
     ``cu_q_lens[i]`` .. ``cu_q_lens[i+1] - 1`` of ``q``, ``[total_q, nq, d]``
     bf16) attends causally over its paged context; returns ``out`` like ``q``.
-    ``max_q_len`` is a host-known bound on every chunk length."""
+    ``max_q_len`` is a host-known bound on every chunk length. ``workspace``
+    (E4M3 cache, optional): a device buffer of at least
+    ``prefill_workspace_bytes(...)`` bytes into which the codes of the long
+    chunks' contexts are widened once per call (same result, fewer conversions)."""
     if q.dtype != torch.bfloat16 or not q.is_contiguous():
         raise TypeError("q must be contiguous bfloat16")
     for t, n in ((block_tables, "block_tables"), (cu_q_lens, "cu_q_lens"), (context_lens, "context_lens")):
@@ -369,10 +383,11 @@ def paged_attention_prefill(q, k_cache, v_cache, block_tables, cu_q_lens, contex
         raise ValueError("cu_q_lens must have num_seqs + 1 entries and block_tables num_seqs rows")
     if out is None:
         out = torch.empty_like(q)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = lib().pkv_paged_attention_prefill(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(cu_q_lens),
         _ptr(context_lens), S, T, nq, nkv, d, bs, nblk, float(scale), _cache_dtype(k_cache, k_scale), _ptr(k_scale),
-        _ptr(v_scale), int(max_q_len), _ptr(out), _ptr(dev_err), _stream(stream))
+        _ptr(v_scale), int(max_q_len), _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_err), _stream(stream))
     _check(st, "pkv_paged_attention_prefill")
     return out
 

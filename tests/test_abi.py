@@ -188,14 +188,16 @@ def test_binding_refuses_to_run_without_library(tmp_path):
 def test_prefill_host_checks(K):
     L = K.lib()
     ok = dict(q=0x10000, kc=0x20000, vc=0x30000, bt=0x40000, maxb=8, cu=0x50000, cl=0x60000, S=4, T=100, nq=32,
-              nkv=8, d=128, bs=256, nblk=100, scale=0.088, dt=0, ks=None, vs=None, mq=64, out=0x70000)
+              nkv=8, d=128, bs=256, nblk=100, scale=0.088, dt=0, ks=None, vs=None, mq=64, ws=None, wsb=0,
+              out=0x70000)
 
     def call(**kw):
         a = dict(ok)
         a.update(kw)
         return L.pkv_paged_attention_prefill(a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cu"], a["cl"], a["S"],
                                              a["T"], a["nq"], a["nkv"], a["d"], a["bs"], a["nblk"], a["scale"],
-                                             a["dt"], a["ks"], a["vs"], a["mq"], a["out"], None, None)
+                                             a["dt"], a["ks"], a["vs"], a["mq"], a["ws"], a["wsb"], a["out"], None,
+                                             None)
 
     assert call(q=None) == K.PKV_ERR_INVALID_ARG
     assert call(cu=None) == K.PKV_ERR_INVALID_ARG
@@ -211,6 +213,28 @@ def test_prefill_host_checks(K):
     assert call(mq=0) == K.PKV_ERR_INVALID_ARG
     assert call(nblk=2**31) == K.PKV_ERR_INVALID_ARG
     assert call(S=0) == K.PKV_OK and call(T=0) == K.PKV_OK  # nothing to do, nothing launched
+    # the E4M3 widening workspace: checked before anything is launched
+    fp8 = dict(dt=1, ks=0x80000, vs=0x90000)
+    assert call(ws=0xA0000, wsb=4096, **fp8) == K.PKV_ERR_WORKSPACE
+    assert call(ws=0xA0000, wsb=4096, dt=2, ks=0x80000, vs=0x90000) == K.PKV_ERR_WORKSPACE
+    assert call(ws=0xA0008, wsb=1 << 40, **fp8) == K.PKV_ERR_INVALID_ARG  # misaligned
+    assert call(ws=0xA0000, wsb=0, S=0, **fp8) == K.PKV_OK  # no sequences: no bound
+
+
+def test_prefill_workspace_bytes(K):
+    L = K.lib()
+    wb = K.prefill_workspace_bytes
+    # rows per (sequence, KV head): the table capacity rounded up to 128
+    assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_FP8_E4M3) == 4 * 8 * 2048 * (4 * 128)
+    assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_FP8_E4M3_TOKEN) == 4 * 8 * 2048 * (4 * 128 + 8)
+    assert wb(3, 2, 64, 3, 16, K.PKV_CACHE_FP8_E4M3) == 3 * 2 * 128 * (4 * 64)
+    assert wb(1, 1, 128, 9, 16, K.PKV_CACHE_FP8_E4M3) == 256 * 512  # 144 -> 256 rows
+    assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_BF16) == 0
+    assert wb(0, 8, 128, 8, 256, K.PKV_CACHE_FP8_E4M3) == 0 and wb(4, 8, 128, 0, 256, 1) == 0
+    assert wb(4, 8, 128, 8, 256, 7) == 0  # unknown cache type
+    # 2^20 sequences x 8 heads x 16384 rows: beyond int32 tensor-map rows
+    assert wb(1 << 20, 8, 128, 1024, 16, K.PKV_CACHE_FP8_E4M3) == 0
+    assert L.pkv_prefill_workspace_bytes(2, 2, 128, 1, 128, 1) == 2 * 2 * 128 * 512
 
 
 def test_norm_host_checks(K):
