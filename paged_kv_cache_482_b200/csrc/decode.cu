@@ -52,8 +52,12 @@ cudaError_t launch_one(const DecodeParams &p, cudaStream_t stream) {
 }
 
 // head_dim 128: the warp-MMA kernel (decode_mma.cuh), every cache type.
+// tc_prefix: the shared prefixes of a cascade are attended elsewhere (on the
+// tensor cores, launch_prefix_tc); otherwise the prefix kernel below does it.
+// merge: launch the split-K merge after the decode kernel (when one is
+// needed); false when the caller launches it (launch_merge) itself.
 template <int G, bool BF, bool TS>
-cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
+cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream, bool tc_prefix, bool merge) {
     using T = MmaTraits<G, BF>;
 #ifdef PKV_MMA_MIN_BLOCKS
     constexpr int MINB = PKV_MMA_MIN_BLOCKS;
@@ -86,7 +90,7 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
                            : make_e4m3_pool_map(&mk, p.k_cache, rows, box_rows) &&
                                  make_e4m3_pool_map(&mv, p.v_cache, rows, box_rows);
     if (!mapped) return cudaErrorInvalidValue;
-    if (p.cu_group_seqs) {  // the shared prefixes first: slot 0 of every member
+    if (p.cu_group_seqs && !tc_prefix) {  // the shared prefixes first: slot 0 of every member
         using PT = PrefixTraits<BF>;
         auto pk = paged_prefix_mma_kernel<G, BF, TS>;
         static std::atomic<unsigned long long> configured_prefix{0};
@@ -108,20 +112,59 @@ cudaError_t launch_mma_one(const DecodeParams &p, cudaStream_t stream) {
     }
     kern<<<(unsigned)blocks, T::kThreads, T::kAlloc, stream>>>(p, mk, mv, box_rows);
     e = cudaGetLastError();
-    if (e != cudaSuccess || (p.num_partitions <= 1 && !p.cu_group_seqs)) return e;
+    if (e != cudaSuccess || !merge || (p.num_partitions <= 1 && !p.cu_group_seqs)) return e;
+    paged_decode_reduce_kernel<128><<<reduce_blocks(p), 32 * kReduceWarps, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// The split-K merge of a head_dim-128 decode whose partials are all written.
+cudaError_t launch_merge(const DecodeParams &p, cudaStream_t stream) {
+    if (p.num_partitions <= 1 && !p.cu_group_seqs) return cudaSuccess;
     paged_decode_reduce_kernel<128><<<reduce_blocks(p), 32 * kReduceWarps, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
 template <bool BF, bool TS>
-cudaError_t launch_mma(int group, const DecodeParams &p, cudaStream_t stream) {
+cudaError_t launch_mma(int group, const DecodeParams &p, cudaStream_t stream, bool tc_prefix = false,
+                       bool merge = true) {
     switch (group) {
-        case 1: return launch_mma_one<1, BF, TS>(p, stream);
-        case 2: return launch_mma_one<2, BF, TS>(p, stream);
-        case 4: return launch_mma_one<4, BF, TS>(p, stream);
-        case 8: return launch_mma_one<8, BF, TS>(p, stream);
+        case 1: return launch_mma_one<1, BF, TS>(p, stream, tc_prefix, merge);
+        case 2: return launch_mma_one<2, BF, TS>(p, stream, tc_prefix, merge);
+        case 4: return launch_mma_one<4, BF, TS>(p, stream, tc_prefix, merge);
+        case 8: return launch_mma_one<8, BF, TS>(p, stream, tc_prefix, merge);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// bf16 cascade: the shared prefixes on the tensor cores, on the caller's
+// stream and launched first (one CTA per SM, on far fewer SMs than there are
+// at the sizes where prefixes are shared), beside the suffix decode on the
+// library's low-priority side stream, which fills the other SMs; the merge
+// runs on the caller's stream once both are done. Without a side stream,
+// everything in order on the caller's stream.
+cudaError_t launch_cascade_tc(int group, const DecodeArgs &a, const DecodeParams &p, cudaStream_t stream) {
+    cudaStream_t side = library_side_stream();
+    cudaEvent_t fork = nullptr, join = nullptr;
+    if (!side || cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        if (fork) cudaEventDestroy(fork);
+        const cudaError_t e = launch_prefix_tc(a, stream);
+        return e != cudaSuccess ? e : launch_mma<true, false>(group, p, stream, true);
+    }
+    cudaError_t e = cudaEventRecord(fork, stream);
+    if (e == cudaSuccess) e = launch_prefix_tc(a, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+    if (e == cudaSuccess) e = launch_mma<true, false>(group, p, side, true, false);
+    // join even after a failure, so that nothing later on the caller's stream
+    // overtakes work already queued on the side stream
+    cudaError_t e2 = cudaEventRecord(join, side);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(stream, join, 0);
+    cudaEventDestroy(fork);  // released once the waits are resolved
+    cudaEventDestroy(join);
+    if (e != cudaSuccess) return e;
+    if (e2 != cudaSuccess) return e2;
+    return launch_merge(p, stream);
 }
 
 template <bool BF>
@@ -207,7 +250,11 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.grid_partitions = a.cu_group_seqs ? p.num_partitions - 1 : p.num_partitions;
     const int group = a.num_q_heads / a.num_kv_heads;
     if (a.head_dim == 128) {
-        if (!a.fp8) return launch_mma<true, false>(group, p, stream);
+        if (!a.fp8) {
+            if (a.cu_group_seqs && prefix_tc_supported(a.head_dim, group, false))
+                return launch_cascade_tc(group, a, p, stream);  // bf16 cascade
+            return launch_mma<true, false>(group, p, stream);
+        }
         return a.token_scales ? launch_mma<false, true>(group, p, stream) : launch_mma<false, false>(group, p, stream);
     }
     if (a.head_dim == 64) {  // the CUDA-core kernel (decode.cuh)

@@ -104,7 +104,29 @@ struct PrefillArgs {
     // and its rows per (sequence, KV head), a multiple of 128
     void *staging = nullptr;
     int staging_stride = 0;
+    // shared-prefix mode of the warp-specialised kernel (launch_prefix_tc;
+    // null: off): the rows of group j are its members' queries (sequences
+    // cu_group_seqs[j] ..), the keys its group_prefix[j] shared tokens, and
+    // each row's result its split-K slot-0 partial in part_o / part_ml
+    const int32_t *cu_group_seqs = nullptr;
+    const int32_t *group_prefix = nullptr;
+    int num_groups = 0;
+    int max_context_len = 0;
+    float *part_o = nullptr;
+    float *part_ml = nullptr;
+    int num_partitions = 0;
 };
+
+// The shared prefixes of a cascade decode (DecodeArgs with cu_group_seqs)
+// on the tensor cores: every member's slot-0 partial. bf16 cache, head_dim
+// 128 (prefix_tc_supported); the decode kernel then attends the suffixes.
+bool prefix_tc_supported(int head_dim, int group, bool fp8);
+cudaError_t launch_prefix_tc(const DecodeArgs &d, cudaStream_t stream);
+
+// The library's low-priority stream of the current device (created on first
+// use, kept for the process; null if it cannot be made). Work put on it is
+// forked from and joined back into the caller's stream with events.
+cudaStream_t library_side_stream();
 
 // Staging rows per (sequence, KV head) of the E4M3 prefill workspace (the
 // table capacity rounded up to 128) and the workspace's bytes; 0 when there

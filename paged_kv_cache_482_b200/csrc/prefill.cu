@@ -564,13 +564,17 @@ cudaError_t launch_short_chunks(const PrefillArgs &a, int g, cudaStream_t stream
     return a.fp8 ? launch_d<64, true>(small, g, stream) : launch_d<64, false>(small, g, stream);
 }
 
+}  // namespace
+
 // A low-priority stream per device, created on first use and kept for the
-// process: the one-token chunks of a mixed batch run on it, beside the chunk
-// kernels, so that their blocks fill the SMs the few long-chunk blocks leave
-// idle; the caller's stream waits for it before anything queued later. (The
-// short chunks stay on the caller's stream: moved to the side stream they
-// competed with the long chunks for the SMs and the batch took 5 % longer.)
-cudaStream_t side_stream() {
+// process. The one-token chunks of a mixed prefill batch run on it, beside
+// the chunk kernels, so that their blocks fill the SMs the few long-chunk
+// blocks leave idle (the short chunks stay on the caller's stream: moved to
+// the side stream they competed with the long chunks for the SMs and the
+// batch took 5 % longer); so does the suffix decode of a bf16 cascade, beside
+// the shared-prefix kernel (decode.cu). The caller's stream waits for it
+// before anything queued later.
+cudaStream_t library_side_stream() {
     constexpr int kMaxDevices = 64;
     static std::atomic<cudaStream_t> streams[kMaxDevices];
     int dev = 0;
@@ -593,8 +597,6 @@ cudaStream_t side_stream() {
     }
     return s;
 }
-
-}  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     const int g = a.num_q_heads / a.num_kv_heads;
@@ -633,7 +635,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     d.cu_q_lens = a.cu_q_lens;
     d.total_q = a.total_q;
     if (a.max_q_len <= 1) return launch_decode(d, stream);  // decode requests only
-    cudaStream_t side = side_stream();
+    cudaStream_t side = library_side_stream();
     cudaEvent_t fork = nullptr, join = nullptr;
     if (!side || cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {

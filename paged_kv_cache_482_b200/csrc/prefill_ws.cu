@@ -238,7 +238,15 @@ __global__ void __launch_bounds__(256) widen_kv_kernel(PrefillArgs a, int log2_b
 // STG (E4M3 only): K/V tiles come from the staging rows by tensor-map copies
 // (map_k / map_v cover the staging instead of the pools); otherwise E4M3
 // codes are widened by the converter warps.
-template <int D, int G, bool FP8, bool TS, bool STG>
+// PFX (bf16 cache, shared-prefix decode): a unit is a group of sequences
+// that share their first group_prefix[s] cached tokens, its rows are
+// (member, query head) pairs (member i's query is q row cu_group_seqs[s] + i),
+// the keys are the shared tokens, read through the first member's table, with
+// no causal mask, and each row's result is its split-K slot-0 partial
+// (normalised O, maximum, sum) for the merge -- the product of the members'
+// queries with the shared keys is a dense contraction, run here on the
+// tensor cores instead of once per member.
+template <int D, int G, bool FP8, bool TS, bool STG, bool PFX>
 __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
     paged_prefill_ws_kernel(PrefillArgs a, int tiles_per_seq, int log2_bs, const __grid_constant__ CUtensorMap map_k,
                             const __grid_constant__ CUtensorMap map_v) {
@@ -262,29 +270,35 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    // query-tile-major over the sequences: the last (longest causal range)
-    // tiles of every sequence are scheduled first
-    const int s = blockIdx.x % a.num_seqs;
-    const int tile = tiles_per_seq - 1 - blockIdx.x / a.num_seqs;
+    // query-tile-major over the sequences (groups): the last (longest causal
+    // range) tiles of every sequence are scheduled first
+    const int units = PFX ? a.num_groups : a.num_seqs;
+    const int s = blockIdx.x % units;
+    const int tile = tiles_per_seq - 1 - blockIdx.x / units;
     const int kh = blockIdx.y;
     const int nq = a.num_q_heads;
 
     // ------------------------------------------------ bounds and bookkeeping
-    const int q0 = a.cu_q_lens[s];
-    const int q1 = a.cu_q_lens[s + 1];
-    if (q0 < 0 || q1 < q0 || q1 > a.total_q) {
+    // rows: the chunk's tokens, or (PFX) the group's members
+    const int q0 = PFX ? a.cu_group_seqs[s] : a.cu_q_lens[s];
+    const int q1 = PFX ? a.cu_group_seqs[s + 1] : a.cu_q_lens[s + 1];
+    if (q0 < 0 || q1 < q0 || q1 > (PFX ? a.num_seqs : a.total_q)) {
         if (tid == 0 && tile == 0 && kh == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
         return;
     }
     const int c = q1 - q0;
-    const int t0 = tile * 2 * TQ;  // first chunk token of query tile A
+    const int t0 = tile * 2 * TQ;  // first chunk token (member) of query tile A
     if (t0 >= c) return;
-    if (c <= a.small_cut) return;  // a short chunk: the one-tile kernel's
-    const int ctx = a.context_lens[s];
-    const int32_t *table_g = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+    if (!PFX && c <= a.small_cut) return;  // a short chunk: the one-tile kernel's
+    const int P = PFX ? a.group_prefix[s] : 0;
+    if (PFX && P == 0) return;  // nothing shared: the decode kernel attends every token
+    const long long cap = static_cast<long long>(a.max_blocks_per_seq) * a.block_size;
+    // keys 0 .. ctx - 1: the sequence's context, or the group's shared tokens
+    const int ctx = PFX ? P : a.context_lens[s];
+    const int32_t *table_g = a.block_tables + static_cast<int64_t>(PFX ? q0 : s) * a.max_blocks_per_seq;
     int32_t *table_s = reinterpret_cast<int32_t *>(sm + L::kTable);
-    bool bad = ctx < c || static_cast<int64_t>(ctx) > static_cast<int64_t>(a.max_blocks_per_seq) * a.block_size ||
-               c > a.max_q_len;
+    bool bad = PFX ? (P < 0 || (P & (a.block_size - 1)) != 0 || P > cap)
+                   : (ctx < c || static_cast<int64_t>(ctx) > cap || c > a.max_q_len);
     if (!bad) {
         const int nblk_seq = (ctx + a.block_size - 1) >> log2_bs;
         for (int i = tid; i < nblk_seq; i += ws_threads<CONV>()) {
@@ -294,22 +308,55 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
         }
     }
     const BlockIds table{table_s, table_g};
+    // PFX: a member whose context is shorter than the shared tokens, or whose
+    // table does not start with the first member's blocks, gets an empty
+    // partial (sum 0: the merge writes zeros) and PKV_DEVERR_BOUNDS; one flag
+    // per member of this unit, in the (unused) scale slots
+    uint8_t *mflag = sm + L::kScales;
+    if constexpr (PFX) {
+        const int nm = min(c - t0, 2 * TQ);
+        const int nblk = bad ? 0 : P >> log2_bs;
+        for (int m = warp; m < nm; m += ws_threads<CONV>() / 32) {
+            const int seq = q0 + t0 + m;
+            const int cm = __ldg(a.context_lens + seq);
+            bool bm = cm < P || cm > a.max_context_len || cm > cap;
+            const int32_t *mrow = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks_per_seq;
+            for (int i = lane; i < nblk; i += 32) bm |= __ldg(mrow + i) != __ldg(table_g + i);
+            bm = __any_sync(0xffffffffu, bm);
+            if (lane == 0) mflag[m] = bm ? 1 : 0;
+        }
+    }
 
     // softmax threads: query tile X, row r of it
     const int X = (warp >> 2) & 1;
     const int row = tid & (kRowsT - 1);
     const int row_tok = t0 + X * TQ + row / G;
     const bool row_live = warp < 8 && row_tok < c;
-    __nv_bfloat16 *out_row = static_cast<__nv_bfloat16 *>(a.out) +
-                             (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + kh * G + row % G) * D;
+    __nv_bfloat16 *out_row = PFX ? nullptr
+                                 : static_cast<__nv_bfloat16 *>(a.out) +
+                                       (static_cast<int64_t>(q0 + (row_live ? row_tok : 0)) * nq + kh * G + row % G) * D;
+    // PFX: this row's slot-0 partial
+    const long long pslot =
+        PFX ? (static_cast<long long>(q0 + (row_live ? row_tok : 0)) * nq + kh * G + row % G) * a.num_partitions : 0;
     if (__syncthreads_or(bad)) {
-        if (row_live)
-            for (int i = 0; i < D; i += 8) *reinterpret_cast<uint4 *>(out_row + i) = make_uint4(0, 0, 0, 0);
+        if (row_live) {
+            if constexpr (PFX) {
+                a.part_ml[pslot * 2] = -INFINITY;
+                a.part_ml[pslot * 2 + 1] = 0.0f;
+            } else {
+                for (int i = 0; i < D; i += 8) *reinterpret_cast<uint4 *>(out_row + i) = make_uint4(0, 0, 0, 0);
+            }
+        }
         if (tid == 0) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
         return;
     }
+    if constexpr (PFX) {
+        bool any = false;
+        for (int m = tid; m < min(c - t0, 2 * TQ); m += ws_threads<CONV>()) any |= mflag[m] != 0;
+        if (any) set_error(a.dev_err, PKV_DEVERR_BOUNDS);
+    }
     const int last_tok = min(t0 + 2 * TQ, c) - 1;
-    const int p_last = ctx - c + last_tok;
+    const int p_last = PFX ? P - 1 : ctx - c + last_tok;
     const int kv_end = p_last + 1;
     const int n_tiles = (kv_end + kBN - 1) / kBN;
 
@@ -397,8 +444,10 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
             fence_proxy_async_smem();
             mbar_arrive(&bars->q_full);
         }
-        const int p_first = ctx - c + t0 + X * TQ;  // position of this tile's first row
-        const int row_pos = row_live ? ctx - c + row_tok : p_last;
+        // position of this tile's first row, and of this row (PFX: every row
+        // sees all the shared tokens)
+        const int p_first = PFX ? P - 1 : ctx - c + t0 + X * TQ;
+        const int row_pos = PFX ? P - 1 : (row_live ? ctx - c + row_tok : p_last);
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
@@ -507,8 +556,28 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
         if (ok && __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], 0))) {
             tc_fence_after();
             const float inv = ((FP8 && !TS) ? __ldg(a.v_scale + kh) : 1.0f) / l_run;
+            if constexpr (PFX) {  // the slot-0 partial: O / l, then (maximum, sum)
+                const bool bm = row_live && mflag[row_tok - t0] != 0;
+                float *dst = a.part_o + pslot * D;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    float v[32];
+                    tmem_ld32(tmem_o + lane_base + ch * 32, v);
+                    if (row_live) {
+                        const float w = bm ? 0.0f : inv;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(dst + ch * 32 + i) =
+                                make_float4(v[i] * w, v[i + 1] * w, v[i + 2] * w, v[i + 3] * w);
+                    }
+                }
+                if (row_live) {
+                    a.part_ml[pslot * 2] = bm ? -INFINITY : m_run;
+                    a.part_ml[pslot * 2 + 1] = bm ? 0.0f : l_run;
+                }
+            }
+#pragma unroll
+            for (int ch = 0; ch < (PFX ? 0 : D / 32); ++ch) {
                 float v[32];
                 tmem_ld32(tmem_o + lane_base + ch * 32, v);
                 if (row_live) {
@@ -524,6 +593,10 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
             }
         } else {
             if (row == 0) set_error(a.dev_err, PKV_DEVERR_TIMEOUT);
+            if (PFX && row_live) {  // an empty partial: the merge writes zeros
+                a.part_ml[pslot * 2] = -INFINITY;
+                a.part_ml[pslot * 2 + 1] = 0.0f;
+            }
         }
         __syncwarp();
     } else if (!CONV && warp == kProducerWarp) {
@@ -797,7 +870,7 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
         widen_kv_kernel<D, TS><<<static_cast<unsigned>(wblocks), 256, 0, stream>>>(a, log2_bs, units);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        auto kern = paged_prefill_ws_kernel<D, G, true, TS, true>;
+        auto kern = paged_prefill_ws_kernel<D, G, true, TS, true, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(WsLayout<D>::kAlloc));
         if (e != cudaSuccess) return e;
@@ -807,7 +880,7 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
     // the E4M3 path without staging loads the codes with plain loads: no tensor maps
     if (!FP8 && (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)))
         return cudaErrorInvalidValue;
-    auto kern = paged_prefill_ws_kernel<D, G, FP8, TS, false>;
+    auto kern = paged_prefill_ws_kernel<D, G, FP8, TS, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(WsLayout<D>::kAlloc));
     if (e != cudaSuccess) return e;
@@ -827,6 +900,80 @@ cudaError_t launch_ws_g(const PrefillArgs &a, int g, cudaStream_t stream) {
 }
 
 }  // namespace
+
+namespace {
+
+template <int G>
+cudaError_t launch_prefix_g(const PrefillArgs &a, cudaStream_t stream) {
+    constexpr int TQ = kRowsT / G;
+    const int tiles = (a.max_q_len + 2 * TQ - 1) / (2 * TQ);
+    const long long nx = static_cast<long long>(a.num_groups) * tiles;
+    if (nx <= 0) return cudaSuccess;
+    if (nx > 0x7FFFFFFFLL || a.num_kv_heads > 65535) return cudaErrorInvalidConfiguration;
+    if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * a.block_size > 0x7FFFFFFFLL)
+        return cudaErrorInvalidConfiguration;  // tensor-map row coordinates are int32
+    int log2_bs = 0;
+    while ((1 << log2_bs) < a.block_size) ++log2_bs;
+    CUtensorMap mk, mv;
+    memset(&mk, 0, sizeof(mk));
+    memset(&mv, 0, sizeof(mv));
+    if (!make_pool_map(&mk, a.k_cache, a, kBN) || !make_pool_map(&mv, a.v_cache, a, kBN)) return cudaErrorInvalidValue;
+    auto kern = paged_prefill_ws_kernel<128, G, false, false, false, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(WsLayout<128>::kAlloc));
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(static_cast<unsigned>(nx), a.num_kv_heads), ws_threads<false>(), WsLayout<128>::kAlloc, stream>>>(
+        a, tiles, log2_bs, mk, mv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefix_tc_supported(int head_dim, int group, bool fp8) {
+    return head_dim == 128 && !fp8 && (group == 1 || group == 2 || group == 4 || group == 8);
+}
+
+cudaError_t launch_prefix_tc(const DecodeArgs &d, cudaStream_t stream) {
+    const int g = d.num_q_heads / d.num_kv_heads;
+    if (!d.cu_group_seqs || !prefix_tc_supported(d.head_dim, g, d.fp8)) return cudaErrorInvalidValue;
+    PrefillArgs a;
+    a.q = d.q;
+    a.k_cache = d.k_cache;
+    a.v_cache = d.v_cache;
+    a.block_tables = d.block_tables;
+    a.max_blocks_per_seq = d.max_blocks_per_seq;
+    a.cu_q_lens = nullptr;
+    a.context_lens = d.context_lens;
+    a.num_seqs = d.num_seqs;
+    a.total_q = d.num_seqs;
+    a.num_q_heads = d.num_q_heads;
+    a.num_kv_heads = d.num_kv_heads;
+    a.head_dim = d.head_dim;
+    a.block_size = d.block_size;
+    a.num_blocks = d.num_blocks;
+    a.scale = d.scale;
+    a.fp8 = false;
+    a.token_scales = false;
+    a.k_scale = nullptr;
+    a.v_scale = nullptr;
+    a.max_q_len = d.max_group_seqs;  // members per group: sizes the grid like a chunk length
+    a.out = nullptr;
+    a.dev_err = d.dev_err;
+    a.small_cut = 0;
+    a.cu_group_seqs = d.cu_group_seqs;
+    a.group_prefix = d.group_prefix;
+    a.num_groups = d.num_groups;
+    a.max_context_len = d.max_context_len;
+    a.part_o = d.part_o;
+    a.part_ml = d.part_ml;
+    a.num_partitions = d.num_partitions;
+    switch (g) {
+        case 1: return launch_prefix_g<1>(a, stream);
+        case 2: return launch_prefix_g<2>(a, stream);
+        case 4: return launch_prefix_g<4>(a, stream);
+        default: return launch_prefix_g<8>(a, stream);
+    }
+}
 
 int prefill_staging_stride(int max_blocks_per_seq, int block_size) {
     const long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;

@@ -26,6 +26,7 @@ import ctypes
 import os
 import threading
 
+import numpy as np
 import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
@@ -414,8 +415,13 @@ def fused_add_rmsnorm(x, residual, weight, eps, out=None, stream=None):
 
 def longest_first(context_lens_host: torch.Tensor) -> torch.Tensor:
     """Host helper: the order that schedules the longest sequences first
-    (stable, int32). Engines know their lengths on the host."""
-    return torch.argsort(context_lens_host.to(torch.int64), descending=True, stable=True).to(torch.int32)
+    (stable: equal lengths keep their order; int32). Engines know their
+    lengths on the host."""
+    return torch.from_numpy(_longest_first_np(context_lens_host.numpy()))
+
+
+def _longest_first_np(lens) -> np.ndarray:
+    return np.argsort(-lens.astype(np.int64), kind="stable").astype(np.int32)
 
 
 def read_device_error(dev_err, stream=None) -> int:
@@ -516,20 +522,29 @@ class DecodeStep:
         stream), and the output is copied out on a second copy stream from one
         of two device outputs. So the copies of one step overlap the kernels of
         the steps around it, and nothing waits on the host unless it runs two
-        steps ahead of the GPU. Returns once queued; ``flush(stream)`` makes
+        steps ahead of the GPU. The store and the attention on buffer set i are
+        recorded as a CUDA graph the first time set i is used (that first step
+        also runs them once eagerly; a repeated store writes the same values)
+        and replayed after that, so a step costs the host one graph launch
+        besides the copies. Returns once queued; ``flush(stream)`` makes
         ``stream`` wait for every queued output copy."""
         cs = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream()
         dev = self.k_cache.device
         if self._dev_inputs is None:
             self._h2d, self._d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-            self._dev_inputs, self._outs, self._order_host = [], [], []
+            self._dev_inputs, self._outs, self._order_host, self._graphs = [], [], [], [None, None]
             for _ in range(2):
                 self._dev_inputs.append([torch.empty(t.shape, dtype=t.dtype, device=dev)
                                          for t in (q, k_new, v_new, slot_mapping, block_tables, context_lens)] +
                                         [torch.empty(context_lens.shape, dtype=torch.int32, device=dev)])
                 self._outs.append(torch.empty_like(self.out))
                 self._order_host.append(torch.empty(context_lens.shape, dtype=torch.int32).pin_memory())
-            self._ev = {k: [None, None] for k in ("in_ready", "in_free", "out_free")}
+            # events reused step after step (re-recording one is safe once its
+            # earlier waits are queued); "used" marks a set's first round
+            self._ev_ready = [torch.cuda.Event(), torch.cuda.Event()]
+            self._ev_free = [torch.cuda.Event(), torch.cuda.Event()]
+            self._ev_out = [torch.cuda.Event(), torch.cuda.Event()]
+            self._used = [False, False]
             self._flip = 0
             self._primed = False
         if not self._primed:  # the first copies start after what is already queued on cs
@@ -539,38 +554,43 @@ class DecodeStep:
             self._primed = True
         i = self._flip
         self._flip ^= 1
-        ev = self._ev
-        if ev["in_ready"][i] is not None:
-            ev["in_ready"][i].synchronize()  # the pinned order buffer of two steps ago has been copied
-        self._order_host[i].copy_(longest_first(context_lens))
+        used = self._used[i]
+        if used:
+            self._ev_ready[i].synchronize()  # the pinned order buffer of two steps ago has been copied
+        self._order_host[i].numpy()[:] = _longest_first_np(context_lens.numpy())
         bufs = self._dev_inputs[i]
-        if ev["in_free"][i] is not None:
-            self._h2d.wait_event(ev["in_free"][i])  # the step two back is done reading set i
+        if used:
+            self._h2d.wait_event(self._ev_free[i])  # the step two back is done reading set i
         with torch.cuda.stream(self._h2d):
             for d_, h_ in zip(bufs, (q, k_new, v_new, slot_mapping, block_tables, context_lens, self._order_host[i])):
                 d_.copy_(h_, non_blocking=True)
             if self.groups is not None:  # the step's groups come from the host too
                 self.groups[0].copy_(self._host_groups[0], non_blocking=True)
                 self.groups[1].copy_(self._host_groups[1], non_blocking=True)
-        ev["in_ready"][i] = torch.cuda.Event()
-        ev["in_ready"][i].record(self._h2d)
-        cs.wait_event(ev["in_ready"][i])
-        if ev["out_free"][i] is not None:
-            cs.wait_event(ev["out_free"][i])  # the output copy of two steps ago is done with output i
-        dq, dk, dv, ds, dbt, dcl, dord = bufs
-        keep = self.out
-        self.out = self._outs[i]
-        try:
-            o = self.run(dq, dk, dv, ds, dbt, dcl, cs, seq_order=dord)
-        finally:
-            self.out = keep
-        ev["in_free"][i] = torch.cuda.Event()
-        ev["in_free"][i].record(cs)
-        self._d2h.wait_event(ev["in_free"][i])
+        self._ev_ready[i].record(self._h2d)
+        cs.wait_event(self._ev_ready[i])
+        if used:
+            cs.wait_event(self._ev_out[i])  # the output copy of two steps ago is done with output i
+        with torch.cuda.stream(cs):
+            if self._graphs[i] is None:
+                dq, dk, dv, ds, dbt, dcl, dord = bufs
+
+                def device_step(i=i):
+                    keep = self.out
+                    self.out = self._outs[i]
+                    try:
+                        self.run(dq, dk, dv, ds, dbt, dcl, seq_order=dord)
+                    finally:
+                        self.out = keep
+
+                self._graphs[i] = graphed(device_step)
+            self._graphs[i]()
+        self._ev_free[i].record(cs)
+        self._d2h.wait_event(self._ev_free[i])
         with torch.cuda.stream(self._d2h):
-            out_host.copy_(o, non_blocking=True)
-        ev["out_free"][i] = torch.cuda.Event()
-        ev["out_free"][i].record(self._d2h)
+            out_host.copy_(self._outs[i], non_blocking=True)
+        self._ev_out[i].record(self._d2h)
+        self._used[i] = True
         return out_host
 
     def flush(self, stream=None):

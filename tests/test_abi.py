@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -314,3 +315,18 @@ def test_shared_prefix_plan_and_host_checks(K):
     assert call(ws=0x90010, wsb=1 << 30) == K.PKV_ERR_INVALID_ARG  # not 256-byte aligned
     assert call(q=0x10008, ws=0x90000, wsb=1 << 30) == K.PKV_ERR_INVALID_ARG
     assert call(S=0, ws=0x90000, wsb=1 << 30) == K.PKV_OK
+
+
+def test_longest_first_is_a_stable_descending_order(K):
+    """The host order helper: lengths non-increasing along the order, equal
+    lengths in their original order, every sequence exactly once."""
+    g = torch.Generator().manual_seed(3)
+    for n in (1, 7, 512, 1025):
+        lens = torch.randint(0, 40, (n,), generator=g, dtype=torch.int32)  # many ties
+        order = K.longest_first(lens)
+        assert order.dtype == torch.int32 and sorted(order.tolist()) == list(range(n))
+        sl = lens[order.long()]
+        assert bool((sl[:-1] >= sl[1:]).all())
+        for a, b in zip(order[:-1].tolist(), order[1:].tolist()):
+            if lens[a] == lens[b]:
+                assert a < b

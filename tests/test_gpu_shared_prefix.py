@@ -142,3 +142,35 @@ def test_prefix_shared_full_size_sampled():
     ids = sorted(set(sample_ids(wl, 24)) | set((wl.slot_new < 0).nonzero().flatten().tolist()[:4]))
     ref = oracle_of(wl, seq_ids=ids)
     compare(out[torch.tensor(ids, device="cuda")], ref, False, "prefix_shared full size")
+
+
+@pytest.mark.parametrize("dt", [W.CACHE_BF16, W.CACHE_FP8])
+def test_cascade_is_ordered_on_the_callers_stream(dt):
+    """The bf16 cascade runs its suffix decode on the library's side stream,
+    beside the shared-prefix kernel on the caller's stream. Work queued on the
+    caller's (non-default) stream right after the call, with no
+    synchronisation in between, must see every output row, and a second call
+    that overwrites the output on the same stream must not be overtaken."""
+    wl_cpu = mixed_groups(dt, g=4, bs=16, seed=11)
+    wl = to_device(wl_cpu)
+    kp, vp = pools_for(wl)
+    cu, pre, mg = groups_of(wl)
+    c = wl.cfg
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = torch.full_like(wl.q, float("nan"))
+        kw = dict(out=out, k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context, dev_err=err)
+        K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, cu,
+                                               pre, mg, **kw)
+        first = out.clone()  # queued right behind the call on s
+        out.fill_(float("nan"))
+        K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, cu,
+                                               pre, mg, **kw)
+        second = out.clone()
+    s.synchronize()
+    assert K.read_device_error(err) == K.PKV_OK
+    assert bool(torch.isfinite(first.float()).all())
+    assert torch.equal(first.view(torch.int16), second.view(torch.int16))
+    compare(first, oracle_of(wl_cpu), dt != W.CACHE_BF16, f"cascade on a side stream ({dt})")
