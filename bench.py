@@ -295,6 +295,48 @@ def nvsmi_ids(local_rank: int):
 
 
 
+_HOST_AFFINITY = {"prev": None, "desc": "not bound"}
+
+
+def bind_host_to_gpu(local_rank: int) -> str:
+    """Restrict this process's host thread to the CPU cores that NVML reports
+    as local to its GPU, before any pinned host buffer is made. Pinned pages
+    then sit on the socket whose PCIe root the GPU hangs off, so host<->device
+    copies do not cross the inter-socket link; left unbound, the placement
+    follows whichever core the process starts on and the end-to-end numbers
+    vary from run to run. The oracle baselines get the full set back
+    (restore_host_affinity). Returns a description for the JSON line."""
+    try:
+        import pynvml as N
+
+        N.nvmlInit()
+        ident = nvsmi_ids(local_rank)[0]
+        h = N.nvmlDeviceGetHandleByUUID(ident) if isinstance(ident, str) else N.nvmlDeviceGetHandleByIndex(int(ident))
+        ncpu = os.cpu_count() or 1
+        words = N.nvmlDeviceGetCpuAffinity(h, (ncpu + 63) // 64)
+        local = {w * 64 + b for w, word in enumerate(words) for b in range(64) if (int(word) >> b) & 1}
+        prev = os.sched_getaffinity(0)
+        cores = local & prev
+        if not cores:
+            _HOST_AFFINITY["desc"] = "not bound (NVML gave no usable local cores)"
+        elif cores == prev:
+            _HOST_AFFINITY["desc"] = f"all {len(prev)} usable cores are local to the GPU (NVML)"
+        else:
+            os.sched_setaffinity(0, cores)
+            _HOST_AFFINITY["prev"] = prev
+            _HOST_AFFINITY["desc"] = f"bound to the {len(cores)} of {len(prev)} cores local to the GPU (NVML affinity)"
+    except Exception as e:  # noqa: BLE001
+        _HOST_AFFINITY["desc"] = f"not bound ({type(e).__name__})"
+    return _HOST_AFFINITY["desc"]
+
+
+def restore_host_affinity() -> None:
+    """Give the process its original cores back (before an oracle baseline)."""
+    if _HOST_AFFINITY["prev"] is not None:
+        os.sched_setaffinity(0, _HOST_AFFINITY["prev"])
+        _HOST_AFFINITY["prev"] = None
+
+
 class L2Flush:
     """Leaves L2 cold and clean between timed steps: a 256 MB write (the
     flush), then a 256 MB read of a second buffer, which writes the first
@@ -407,6 +449,7 @@ def probe_size(wl: W.Workload, order, threads: int, max_tokens: int = 32768) -> 
 def cpu_baseline(wl: W.Workload, target_s: float) -> dict:
     """Tokens/s of the oracle on a bounded sample: its preparation (untimed) and
     its step (timed) take about target_s together."""
+    restore_host_affinity()
     threads = cpu_threads()
     S = wl.cfg.num_seqs
     order = torch.randperm(S, generator=torch.Generator().manual_seed(123)).tolist()
@@ -645,6 +688,7 @@ def prefill_sample_pairs(wl, n, seed):
 
 
 def prefill_cpu_baseline(wl, target_s: float) -> dict:
+    restore_host_affinity()
     threads = cpu_threads()
     run = prefill_oracle_sampler(wl, threads)
     n = max(threads, 8)
@@ -713,6 +757,7 @@ def run_prefill(args):
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
+    host_cores = bind_host_to_gpu(local)
     dist = None
     if world > 1:
         import datetime
@@ -836,6 +881,7 @@ def run_prefill(args):
                        "e4m3_widening": (None if not wl.is_fp8 else
                                          "once per call into a workspace" if ws is not None else "in every CTA"),
                        "parallelism": f"replicas x{world} (independent batches, no collective)",
+                       "host_cores": host_cores,
                        "l2": "no flush: each step's pools and queries exceed 126 MB of L2"},
             "attention_us": attn_ms * 1e3, "store_us": store_ms * 1e3,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
@@ -883,6 +929,7 @@ def norm_bytes(cfg) -> int:
 
 
 def norm_cpu_baseline(wl, target_s: float) -> dict:
+    restore_host_affinity()
     import oracle as O
 
     threads = cpu_threads()
@@ -934,6 +981,7 @@ def run_norm(args):
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
+    host_cores = bind_host_to_gpu(local)
     dist = None
     if world > 1:
         import datetime
@@ -1018,6 +1066,7 @@ def run_norm(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, fp32 arithmetic", "data": "synthetic",
             "config": {"workload": norm_desc(cfg), "seed": args.seed,
                        "parallelism": f"replicas x{world} (independent rows, no collective)",
+                       "host_cores": host_cores,
                        "l2": (L2Flush.desc if flush is not None else
                               f"no flush: {moved / 1e6:.0f} MB moved per step, above the 126 MB L2")},
             "kernel_us": kern_ms * 1e3,
@@ -1078,6 +1127,7 @@ def _rope_pools(wl, device="cuda"):
 
 
 def rope_cpu_baseline(wl, target_s: float) -> dict:
+    restore_host_affinity()
     import oracle as O
 
     threads = cpu_threads()
@@ -1136,6 +1186,7 @@ def run_rope(args):
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
+    host_cores = bind_host_to_gpu(local)
     dist = None
     if world > 1:
         import datetime
@@ -1229,6 +1280,7 @@ def run_rope(args):
             "data": "synthetic",
             "config": {"workload": rope_desc(cfg), "seed": args.seed,
                        "parallelism": f"replicas x{world} (independent tokens, no collective)",
+                       "host_cores": host_cores,
                        "l2": (L2Flush.desc if flush is not None else
                               f"no flush: {moved / 1e6:.0f} MB moved per step, above the 126 MB L2")},
             "kernel_us": kern_ms * 1e3,
@@ -1268,6 +1320,7 @@ def main():
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
+    host_cores = bind_host_to_gpu(local)
     dist = None
     if world > 1:
         import datetime
@@ -1414,6 +1467,7 @@ def main():
                              "suffixes" if shared else "longest sequence first (order from host lengths)"),
                 "launch": "Python calls" if args.no_graph else "CUDA graphs of the store and of the decode, replayed",
                 "parallelism": f"replicas x{world} (independent batches, no collective)",
+                "host_cores": host_cores,
                 "l2": f"no flush: {ab['kv'] / 1e9:.2f} GB of KV read per step, far above the 126 MB L2",
             },
             "attention_us": decode_ms * 1e3,
