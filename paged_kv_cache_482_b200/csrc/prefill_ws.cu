@@ -160,8 +160,10 @@ __host__ __device__ __forceinline__ Staging staging_of(const PrefillArgs &a) {
 // skipped. Sequences the attention kernel will reject (bad cu_q_lens or
 // lengths) are skipped; a block id outside the pool gives zero rows (the
 // attention kernel reports it).
+constexpr int kWidenThreads = 256;
+
 template <int D, bool TS>
-__global__ void __launch_bounds__(256) widen_kv_kernel(PrefillArgs a, int log2_bs, long long units) {
+__global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(PrefillArgs a, int log2_bs, long long units) {
     constexpr int kCPR = D / 16;  // 16-code chunks per row
     const int tiles = a.staging_stride / kBN;
     const Staging st = staging_of<D>(a);
@@ -181,43 +183,65 @@ __global__ void __launch_bounds__(256) widen_kv_kernel(PrefillArgs a, int log2_b
         if (t0 >= ctx) continue;
         const int32_t *table = a.block_tables + static_cast<long long>(s) * a.max_blocks_per_seq;
         const long long drow0 = sk * a.staging_stride + t0;
-        for (int i = threadIdx.x; i < kBN * kCPR; i += blockDim.x) {
-            const int r = i / kCPR, cc = i % kCPR, t = t0 + r;
-            uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0, v0 = k0, v1 = k0;
+        // kIt chunks per thread: every block id, then every code load, then
+        // the conversions and stores, so that a thread's loads are in flight
+        // together
+        constexpr int kIt = kBN * kCPR / kWidenThreads;
+        int r[kIt];
+        long long prow[kIt];
+#pragma unroll
+        for (int u = 0; u < kIt; ++u) {
+            const int i = threadIdx.x + u * kWidenThreads;
+            r[u] = i / kCPR;
+            const int t = t0 + r[u];
+            prow[u] = -1;
             if (t < ctx) {
                 const int b = __ldg(table + (t >> log2_bs));
-                if (b >= 0 && b < a.num_blocks) {
-                    const long long prow = (static_cast<long long>(b) * a.num_kv_heads + kh) * a.block_size +
-                                           (t & (a.block_size - 1));
-                    const uint4 kc = __ldg(reinterpret_cast<const uint4 *>(
-                        static_cast<const uint8_t *>(a.k_cache) + prow * D + cc * 16));
-                    const uint4 vc = __ldg(reinterpret_cast<const uint4 *>(
-                        static_cast<const uint8_t *>(a.v_cache) + prow * D + cc * 16));
-                    const uint2 h0 = e4m3x4_to_f16x4(kc.x), h1 = e4m3x4_to_f16x4(kc.y);
-                    const uint2 h2 = e4m3x4_to_f16x4(kc.z), h3 = e4m3x4_to_f16x4(kc.w);
-                    k0 = make_uint4(h0.x, h0.y, h1.x, h1.y);
-                    k1 = make_uint4(h2.x, h2.y, h3.x, h3.y);
-                    if constexpr (TS) {  // P V runs in bf16 with per-token scales
-                        v0 = e4m3x8_to_bf16x8(make_uint2(vc.x, vc.y));
-                        v1 = e4m3x8_to_bf16x8(make_uint2(vc.z, vc.w));
-                    } else {
-                        const uint2 g0 = e4m3x4_to_f16x4(vc.x), g1 = e4m3x4_to_f16x4(vc.y);
-                        const uint2 g2 = e4m3x4_to_f16x4(vc.z), g3 = e4m3x4_to_f16x4(vc.w);
-                        v0 = make_uint4(g0.x, g0.y, g1.x, g1.y);
-                        v1 = make_uint4(g2.x, g2.y, g3.x, g3.y);
-                    }
+                if (b >= 0 && b < a.num_blocks)
+                    prow[u] = (static_cast<long long>(b) * a.num_kv_heads + kh) * a.block_size + (t & (a.block_size - 1));
+            }
+        }
+        const int cc = threadIdx.x % kCPR;  // the same 16-code column in every chunk of this thread
+        uint4 kc[kIt], vc[kIt];
+#pragma unroll
+        for (int u = 0; u < kIt; ++u) {
+            kc[u] = make_uint4(0, 0, 0, 0);
+            vc[u] = kc[u];
+            if (prow[u] >= 0) {
+                kc[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.k_cache) + prow[u] * D +
+                                                            cc * 16));
+                vc[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.v_cache) + prow[u] * D +
+                                                            cc * 16));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kIt; ++u) {
+            uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0, v0 = k0, v1 = k0;
+            if (prow[u] >= 0) {  // zeros past the context (and for a bad block id)
+                const uint2 h0 = e4m3x4_to_f16x4(kc[u].x), h1 = e4m3x4_to_f16x4(kc[u].y);
+                const uint2 h2 = e4m3x4_to_f16x4(kc[u].z), h3 = e4m3x4_to_f16x4(kc[u].w);
+                k0 = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                k1 = make_uint4(h2.x, h2.y, h3.x, h3.y);
+                if constexpr (TS) {  // P V runs in bf16 with per-token scales
+                    v0 = e4m3x8_to_bf16x8(make_uint2(vc[u].x, vc[u].y));
+                    v1 = e4m3x8_to_bf16x8(make_uint2(vc[u].z, vc[u].w));
+                } else {
+                    const uint2 g0 = e4m3x4_to_f16x4(vc[u].x), g1 = e4m3x4_to_f16x4(vc[u].y);
+                    const uint2 g2 = e4m3x4_to_f16x4(vc[u].z), g3 = e4m3x4_to_f16x4(vc[u].w);
+                    v0 = make_uint4(g0.x, g0.y, g1.x, g1.y);
+                    v1 = make_uint4(g2.x, g2.y, g3.x, g3.y);
                 }
             }
-            uint4 *kd = reinterpret_cast<uint4 *>(st.k + (drow0 + r) * D + cc * 16);
-            uint4 *vd = reinterpret_cast<uint4 *>(st.v + (drow0 + r) * D + cc * 16);
+            uint4 *kd = reinterpret_cast<uint4 *>(st.k + (drow0 + r[u]) * D + cc * 16);
+            uint4 *vd = reinterpret_cast<uint4 *>(st.v + (drow0 + r[u]) * D + cc * 16);
             kd[0] = k0;
             kd[1] = k1;
             vd[0] = v0;
             vd[1] = v1;
         }
         if constexpr (TS) {
-            for (int r = threadIdx.x; r < kBN; r += blockDim.x) {
-                const int t = t0 + r;
+            for (int rr = threadIdx.x; rr < kBN; rr += blockDim.x) {
+                const int t = t0 + rr;
                 float ks = 0.0f, vs = 0.0f;
                 if (t < ctx) {
                     const int b = __ldg(table + (t >> log2_bs));
@@ -228,8 +252,8 @@ __global__ void __launch_bounds__(256) widen_kv_kernel(PrefillArgs a, int log2_b
                         vs = __ldg(a.v_scale + prow);
                     }
                 }
-                st.k_scale[drow0 + r] = ks;
-                st.v_scale[drow0 + r] = vs;
+                st.k_scale[drow0 + rr] = ks;
+                st.v_scale[drow0 + rr] = vs;
             }
         }
     }
@@ -867,7 +891,7 @@ cudaError_t launch_ws(const PrefillArgs &a, cudaStream_t stream) {
             return cudaGetLastError();
         const long long units = rows / kBN;
         const long long wblocks = units < 16LL * sms ? units : 16LL * sms;
-        widen_kv_kernel<D, TS><<<static_cast<unsigned>(wblocks), 256, 0, stream>>>(a, log2_bs, units);
+        widen_kv_kernel<D, TS><<<static_cast<unsigned>(wblocks), kWidenThreads, 0, stream>>>(a, log2_bs, units);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         auto kern = paged_prefill_ws_kernel<D, G, true, TS, true, false>;
