@@ -638,6 +638,19 @@ def prefill_flops(wl) -> int:
     return keys * c.num_q_heads * 4 * c.head_dim
 
 
+def prefill_split(wl):
+    """(FLOPs of the chunks longer than one token, K/V bytes that the one-token
+    chunks -- decode requests, run in the decode kernel -- must read)."""
+    c = wl.cfg
+    cu, ctx = wl.cu_q_lens.cpu().long(), wl.context_lens.cpu().long()
+    n = cu[1:] - cu[:-1]
+    long_ = n > 1
+    keys = int((n * (ctx - n) + n * (n + 1) // 2)[long_].sum())
+    es = 1 if wl.is_fp8 else 2
+    row = 2 * c.head_dim * es + (8 if wl.token_scales else 0)
+    return keys * c.num_q_heads * 4 * c.head_dim, int(ctx[n == 1].sum()) * c.num_kv_heads * row
+
+
 def measured_tensor_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -902,6 +915,17 @@ def run_prefill(args):
             "gpu_launches": (2 if mq <= 1 else 3 + (1 + (1 if ws is not None else 0) if long_chunks else 0)) * Kst,
             "clocks": clocks,
         }
+        chunk_flops, decode_bytes = prefill_split(wl)
+        if decode_bytes:  # a mixed batch: tensor work and a K/V stream at once
+            hbm, _ = measured_peak()
+            t_tc, t_hbm = chunk_flops / (peak_sus * 1e12) * 1e6, decode_bytes / (hbm * 1e9) * 1e6
+            line["mixed_bound"] = {
+                "chunk_flops": chunk_flops, "decode_kv_bytes": decode_bytes,
+                "tensor_us": t_tc, "hbm_us": t_hbm, "lower_bound_us": max(t_tc, t_hbm),
+                "frac": max(t_tc, t_hbm) / (attn_ms * 1e3),
+                "note": "the roofline above counts FLOPs only; the one-token chunks are a K/V stream. Lower "
+                        "bound of the call: the larger of the chunks' FLOPs at the sustained tensor peak and "
+                        "the decode rows' K/V bytes at the measured copy bandwidth (perfect overlap)"}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = prefill_cpu_baseline(wl, args.cpu_seconds)
         emit(line, args)
