@@ -250,9 +250,12 @@ PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const
  * "DeepSeek复刻vLLM反超原版：AI推理新标杆", section "vLLM：大模型推理的加速引擎
  * 与挑战") are then read and multiplied once per group of members instead of
  * once per sequence: a prefix kernel attends each group's shared tokens for
- * up to 32 query rows at a time, the decode kernel attends each sequence's
- * own tokens, and the split-K merge combines the two (out is the same
- * attention as pkv_paged_attention_decode, to rounding).
+ * many query rows at a time (bf16: the tcgen05 kernel, 256 rows of (member,
+ * query head) per CTA, run beside the suffix decode on the library's side
+ * stream; E4M3: up to 32 rows per block on the warp-level MMA), the decode
+ * kernel attends each sequence's own tokens, and the split-K merge combines
+ * the two (out is the same attention as pkv_paged_attention_decode, to
+ * rounding).
  *
  *  cu_group_seqs        [num_groups + 1] int32, device: group j is
  *                       sequences cu_group_seqs[j] .. cu_group_seqs[j+1] - 1
@@ -269,7 +272,11 @@ PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const
  *                       workspace_bytes (the prefix partial is one more
  *                       split-K slot per (sequence, query head)), 256-byte
  *                       aligned
- *  other arguments as pkv_paged_attention_decode (no seq_order)
+ *  seq_order            optional (NULL: natural order), as for
+ *                       pkv_paged_attention_decode: the order in which the
+ *                       suffix decode and the merge visit the sequences
+ *                       (the groups keep their batch positions)
+ *  other arguments as pkv_paged_attention_decode
  *
  * Device checks: a P_j that is not a multiple of block_size or exceeds a
  * member's context, a member whose shared block ids differ from the first
@@ -283,7 +290,8 @@ PKV_API int pkv_plan_decode_shared_prefix(int num_seqs, int num_q_heads, int num
                                           int partition_request, pkv_decode_plan *plan);
 PKV_API int pkv_paged_attention_decode_shared_prefix(
     const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
-    const int32_t *context_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    const int32_t *context_lens, const int32_t *seq_order, int num_seqs, int num_q_heads, int num_kv_heads,
+    int head_dim, int block_size,
     int64_t num_blocks, float scale, int cache_dtype, const float *k_scale, const float *v_scale,
     int max_context_len, const int32_t *cu_group_seqs, const int32_t *group_prefix_tokens, int num_groups,
     int max_group_seqs, int partition_request, void *workspace, size_t workspace_bytes, void *out, int *dev_err,

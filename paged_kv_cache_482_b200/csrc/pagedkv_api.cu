@@ -214,8 +214,9 @@ int pkv_plan_decode_shared_prefix(int num_seqs, int num_q_heads, int num_kv_head
 
 int pkv_paged_attention_decode_shared_prefix(const void *q, const void *k_cache, const void *v_cache,
                                              const int32_t *block_tables, int max_blocks_per_seq,
-                                             const int32_t *context_lens, int num_seqs, int num_q_heads,
-                                             int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                                             const int32_t *context_lens, const int32_t *seq_order, int num_seqs,
+                                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                             int64_t num_blocks,
                                              float scale, int cache_dtype, const float *k_scale,
                                              const float *v_scale, int max_context_len,
                                              const int32_t *cu_group_seqs, const int32_t *group_prefix_tokens,
@@ -226,7 +227,7 @@ int pkv_paged_attention_decode_shared_prefix(const void *q, const void *k_cache,
         return PKV_ERR_INVALID_ARG;
     if (num_groups == 0 || head_dim != 128)  // nothing declared shared, or no prefix kernel for this head size
         return pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                                          nullptr, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                          seq_order, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                           num_blocks, scale, cache_dtype, k_scale, v_scale, max_context_len,
                                           partition_request, workspace, workspace_bytes, out, dev_err, stream);
     pkv_decode_plan plan;
@@ -251,7 +252,7 @@ int pkv_paged_attention_decode_shared_prefix(const void *q, const void *k_cache,
     a.block_tables = block_tables;
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.context_lens = context_lens;
-    a.seq_order = nullptr;
+    a.seq_order = seq_order;
     a.num_seqs = num_seqs;
     a.num_q_heads = num_q_heads;
     a.num_kv_heads = num_kv_heads;

@@ -90,9 +90,9 @@ def load_library(path: str):
     L.pkv_plan_decode.restype = i32
     L.pkv_plan_decode_shared_prefix.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, c.POINTER(_Plan)]
     L.pkv_plan_decode_shared_prefix.restype = i32
-    L.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i64,
-                                                           f32, i32, vp, vp, i32, vp, vp, i32, i32, i32, vp, sz, vp,
-                                                           vp, vp]
+    L.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
+                                                           i64, f32, i32, vp, vp, i32, vp, vp, i32, i32, i32, vp,
+                                                           sz, vp, vp, vp]
     L.pkv_paged_attention_decode_shared_prefix.restype = i32
     L.pkv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.pkv_decode_workspace_bytes.restype = sz
@@ -232,10 +232,11 @@ def plan_decode_shared_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim, blo
 def paged_attention_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale, cu_group_seqs,
                                          group_prefix_tokens, max_group_seqs, out=None, k_scale=None, v_scale=None,
                                          max_context_len=None, partition_request=0, workspace=None, dev_err=None,
-                                         stream=None):
+                                         stream=None, seq_order=None):
     """Decode of a batch whose consecutive groups of sequences share cached
     prefixes (int32 device tensors ``cu_group_seqs [G+1]`` and
-    ``group_prefix_tokens [G]``); same result as ``paged_attention_decode``."""
+    ``group_prefix_tokens [G]``); same result as ``paged_attention_decode``.
+    ``seq_order`` (optional, as there) orders the suffix decode."""
     S, nq, d = q.shape
     nblk, nkv, bs, d2 = k_cache.shape
     if d2 != d or v_cache.shape != k_cache.shape:
@@ -257,8 +258,11 @@ def paged_attention_decode_shared_prefix(q, k_cache, v_cache, block_tables, cont
     if plan["workspace_bytes"] and workspace is None:
         workspace = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if seq_order is not None and (seq_order.dtype != torch.int32 or seq_order.numel() != S):
+        raise ValueError("seq_order must be an int32 permutation of the sequences")
     st = lib().pkv_paged_attention_decode_shared_prefix(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), maxb, _ptr(context_lens), S, nq, nkv, d, bs, nblk,
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), maxb, _ptr(context_lens), _ptr(seq_order), S,
+        nq, nkv, d, bs, nblk,
         float(scale), dt, _ptr(k_scale), _ptr(v_scale), int(max_context_len), _ptr(cu_group_seqs),
         _ptr(group_prefix_tokens), G, int(max_group_seqs), int(partition_request), _ptr(workspace), ws_bytes,
         _ptr(out), _ptr(dev_err), _stream(stream))
@@ -507,7 +511,7 @@ class DecodeStep:
                 q, self.k_cache, self.v_cache, block_tables, context_lens, self.scale, cu, pre, mg, out=self.out,
                 k_scale=self.k_scale, v_scale=self.v_scale, max_context_len=self.max_context_len,
                 partition_request=self.partition_request, workspace=self.workspace, dev_err=self.dev_err,
-                stream=stream)
+                stream=stream, seq_order=seq_order)
         return paged_attention_decode(q, self.k_cache, self.v_cache, block_tables, context_lens, self.scale,
                                       out=self.out, k_scale=self.k_scale, v_scale=self.v_scale,
                                       max_context_len=self.max_context_len,

@@ -303,7 +303,7 @@ def test_shared_prefix_plan_and_host_checks(K):
                  ng=2, mg=3, part=0, ws=None, wsb=0, out=0x70000)
         a.update(kw)
         return L.pkv_paged_attention_decode_shared_prefix(
-            a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cl"], a["S"], a["nq"], a["nkv"], a["d"], a["bs"],
+            a["q"], a["kc"], a["vc"], a["bt"], a["maxb"], a["cl"], None, a["S"], a["nq"], a["nkv"], a["d"], a["bs"],
             a["nblk"], a["scale"], a["dt"], a["ks"], a["vs"], a["maxctx"], a["cu"], a["pre"], a["ng"], a["mg"],
             a["part"], a["ws"], a["wsb"], a["out"], None, None)
 

@@ -174,3 +174,35 @@ def test_cascade_is_ordered_on_the_callers_stream(dt):
     assert bool(torch.isfinite(first.float()).all())
     assert torch.equal(first.view(torch.int16), second.view(torch.int16))
     compare(first, oracle_of(wl_cpu), dt != W.CACHE_BF16, f"cascade on a side stream ({dt})")
+
+
+@pytest.mark.parametrize("dt", [W.CACHE_BF16, W.CACHE_FP8_TOKEN])
+def test_cascade_with_seq_order_is_bit_identical(dt):
+    """A visiting order (longest first, and a reversed one) changes when each
+    sequence's suffix runs, not what it computes: same bits as the natural
+    order; an order entry outside the batch is reported and its row skipped."""
+    wl_cpu = mixed_groups(dt, g=4, bs=16, seed=12)
+    wl = to_device(wl_cpu)
+    kp, vp = pools_for(wl)
+    cu, pre, mg = groups_of(wl)
+    c = wl.cfg
+    kw = dict(k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context)
+    base = K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                                  cu, pre, mg, **kw)
+    S = c.num_seqs
+    for order in (K.longest_first(wl_cpu.context_lens).cuda(), torch.arange(S - 1, -1, -1, dtype=torch.int32,
+                                                                            device="cuda")):
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                                                     c.softmax_scale, cu, pre, mg, dev_err=err, seq_order=order, **kw)
+        assert K.read_device_error(err) == K.PKV_OK
+        assert torch.equal(out.view(torch.int16), base.view(torch.int16))
+    bad = torch.arange(S, dtype=torch.int32, device="cuda")
+    bad[5] = S + 3  # sequence 5 is named by no valid entry
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full_like(base, 7.0)
+    K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, cu, pre,
+                                           mg, out=out, dev_err=err, seq_order=bad, **kw)
+    assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS
+    keep = [i for i in range(S) if i != 5]
+    assert torch.equal(out[keep].view(torch.int16), base[keep].view(torch.int16))
