@@ -35,3 +35,25 @@ def test_probe_follows_the_given_order():
     # the order decides which sequences are probed: the long one first stops the probe at one
     assert bench.probe_size(_wl(lens), [0, 1, 2, 3], threads=8) == 1
     assert bench.probe_size(_wl(lens), [1, 2, 3, 0], threads=8) == 3
+
+
+def _pwl(cu, ctx, fp8=False, token_scales=False, nq=8, nkv=2, d=128):
+    cfg = types.SimpleNamespace(num_q_heads=nq, num_kv_heads=nkv, head_dim=d)
+    return types.SimpleNamespace(cfg=cfg, cu_q_lens=torch.tensor(cu, dtype=torch.int32),
+                                 context_lens=torch.tensor(ctx, dtype=torch.int32), is_fp8=fp8,
+                                 token_scales=token_scales)
+
+
+def test_prefill_split_separates_chunks_from_decode_rows():
+    # chunk of 3 after a history of 2 (keys 3 + 4 + 5), two decode rows with contexts 10 and 7
+    wl = _pwl([0, 3, 4, 5], [5, 10, 7])
+    flops, kv = bench.prefill_split(wl)
+    assert flops == (3 + 4 + 5) * 8 * 4 * 128
+    assert kv == (10 + 7) * 2 * (2 * 128 * 2)  # bf16 K and V rows per KV head
+    # the FLOPs of every row together are the chunk FLOPs plus the decode rows' own
+    assert bench.prefill_flops(wl) == flops + (10 + 7) * 8 * 4 * 128
+    # E4M3: one byte per element; per-token scales add a K and a V scale per row
+    assert bench.prefill_split(_pwl([0, 1], [9], fp8=True))[1] == 9 * 2 * 2 * 128
+    assert bench.prefill_split(_pwl([0, 1], [9], fp8=True, token_scales=True))[1] == 9 * 2 * (2 * 128 + 8)
+    # no decode rows: nothing to stream
+    assert bench.prefill_split(_pwl([0, 4], [4]))[1] == 0
