@@ -1414,7 +1414,7 @@ def main():
                                                    step.groups[0], step.groups[1], step.groups[2], out=step.out,
                                                    k_scale=wl.k_scale, v_scale=wl.v_scale,
                                                    max_context_len=c.max_context, partition_request=args.partition,
-                                                   workspace=step.workspace, dev_err=step.dev_err, seq_order=order)
+                                                   workspace=step.workspace, dev_err=step.dev_err)
         else:
             K.paged_attention_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale, out=step.out,
                                      k_scale=wl.k_scale, v_scale=wl.v_scale, max_context_len=c.max_context,
@@ -1488,7 +1488,7 @@ def main():
                     f"{c.prefix_tokens}+U[{c.ctx_lo},{c.ctx_hi}]" if c.prefix_tokens else f"U[{c.ctx_lo},{c.ctx_hi}]"),
                 "kv_tokens": wl.kv_tokens(), "seed": args.seed, "partition_tokens": pt,
                 "schedule": ("shared-prefix cascade: each group's prefix once for all its members (tensor "
-                             "cores) beside the suffixes, longest first (order from host lengths)" if shared else
+                             "cores) beside the suffixes, in batch order" if shared else
                              "longest sequence first (order from host lengths)"),
                 "launch": "Python calls" if args.no_graph else "CUDA graphs of the store and of the decode, replayed",
                 "parallelism": f"replicas x{world} (independent batches, no collective)",

@@ -681,6 +681,26 @@ __global__ void __launch_bounds__(32 * kReduceWarps) paged_decode_reduce_kernel(
     const int seq_slot = (int)(row / p.num_q_heads);
     const int seq = p.seq_order ? __ldg(p.seq_order + seq_slot) : seq_slot;
     if (seq < 0 || seq >= p.num_seqs) return;  // the decode grid reported it
+    // the partials of slots 0 and 1 (every merged row has at least two slots),
+    // loaded before the length and the group are known
+    const long long base0 = ((long long)seq * p.num_q_heads + qh) * p.num_partitions;
+    float2 spec_ml[2];
+    float spec_o[2][DPL];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        spec_ml[i] = *reinterpret_cast<const float2 *>(p.part_ml + (base0 + i) * 2);
+        const float *po = p.part_o + (base0 + i) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(po);
+            spec_o[i][0] = v.x;
+            spec_o[i][1] = v.y;
+            spec_o[i][2] = v.z;
+            spec_o[i][3] = v.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) spec_o[i][k] = po[k];
+        }
+    }
     const int ctx = __ldg(p.context_lens + seq);
     const int table_cap = p.max_blocks_per_seq << p.log2_block_size;
     const bool bad_len = ctx < 1 || ctx > p.max_context_len || ctx > table_cap;
@@ -699,6 +719,41 @@ __global__ void __launch_bounds__(32 * kReduceWarps) paged_decode_reduce_kernel(
         if (n <= 1) return;  // decode wrote the output itself
     }
     const long long base = ((long long)seq * p.num_q_heads + qh) * p.num_partitions + first;
+    float acc[DPL];
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+    // Rows of at most two partials in slots 0 and 1 (a shared prefix and a
+    // short suffix, or a split in two) use the loads issued above, before the
+    // length and the group were known; the arithmetic is the general path's,
+    // operation for operation.
+    if (first + n <= 2 && !bad) {
+        // slot `first` (0, or 1 when there is no prefix), then slot 1 when n == 2;
+        // selects with constant indices keep the loaded values in registers
+        const float2 ml0 = first ? spec_ml[1] : spec_ml[0];
+        const float2 mla = lane == 0 ? ml0 : (lane == 1 && n == 2 ? spec_ml[1] : make_float2(-CUDART_INF_F, 1.f));
+        float M = lane < n ? mla.x : -CUDART_INF_F;
+        bool empty = lane < n && !(mla.y > 0.f);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        if (!__any_sync(0xffffffffu, empty)) {
+            float L = lane < n ? mla.y * exp2f(mla.x - M) : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            const float inv = 1.f / L;
+            const float w0 = ml0.y * exp2f(ml0.x - M) * inv;
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) acc[k] = fmaf(first ? spec_o[1][k] : spec_o[0][k], w0, acc[k]);
+            if (n == 2) {
+                const float w1 = spec_ml[1].y * exp2f(spec_ml[1].x - M) * inv;
+#pragma unroll
+                for (int k = 0; k < DPL; ++k) acc[k] = fmaf(spec_o[1][k], w1, acc[k]);
+            }
+        }
+        __nv_bfloat16 *dst = p.out + ((long long)seq * p.num_q_heads + qh) * D + lane * DPL;
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) dst[k] = __float2bfloat16_rn(acc[k]);
+        return;
+    }
     // maximum over the partitions, and whether any is empty (sum 0: a bad block)
     float M = -CUDART_INF_F;
     bool empty = false;
@@ -710,9 +765,6 @@ __global__ void __launch_bounds__(32 * kReduceWarps) paged_decode_reduce_kernel(
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     bad = __any_sync(0xffffffffu, bad || empty);
-    float acc[DPL];
-#pragma unroll
-    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
     if (!bad) {
         float L = 0.f;
         for (int i = lane; i < n; i += 32) {

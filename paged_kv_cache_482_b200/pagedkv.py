@@ -583,7 +583,10 @@ class DecodeStep:
                     keep = self.out
                     self.out = self._outs[i]
                     try:
-                        self.run(dq, dk, dv, ds, dbt, dcl, seq_order=dord)
+                        # the cascade's suffixes keep the batch order: longest first
+                        # measured slower there (the suffix blocks were allocated
+                        # in batch order, and sorting scatters their reads)
+                        self.run(dq, dk, dv, ds, dbt, dcl, seq_order=None if self.groups is not None else dord)
                     finally:
                         self.out = keep
 
