@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--out", default="", help="also append the JSON line to this file")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step's kernels from Python instead of replaying CUDA graphs of the step")
+    ap.add_argument("--natural-order", action="store_true",
+                    help="decode: visit the sequences in batch order instead of longest first")
     ap.add_argument("--no-staging", action="store_true",
                     help="E4M3 prefill: widen the codes in every CTA instead of once into a workspace")
     ap.add_argument("--no-shared-prefix", action="store_true",
@@ -1386,7 +1388,7 @@ def main():
     # store + decode (+ reduce when split); shared prefix: store + prefix + decode + merge
     launches_per_step = 4 if shared else 2 + (1 if step.plan["partition_tokens"] > 0 else 0)
     # The scheduler knows the lengths on the host: visit the longest sequences first.
-    order = K.longest_first(wl.context_lens.cpu()).cuda()
+    order = None if args.natural_order else K.longest_first(wl.context_lens.cpu()).cuda()
 
     stream = torch.cuda.current_stream()
     for _ in range(max(3, args.warmup)):
@@ -1489,7 +1491,8 @@ def main():
                 "kv_tokens": wl.kv_tokens(), "seed": args.seed, "partition_tokens": pt,
                 "schedule": ("shared-prefix cascade: each group's prefix once for all its members (tensor "
                              "cores) beside the suffixes, in batch order" if shared else
-                             "longest sequence first (order from host lengths)"),
+                             ("batch order" if args.natural_order else
+                              "longest sequence first (order from host lengths)")),
                 "launch": "Python calls" if args.no_graph else "CUDA graphs of the store and of the decode, replayed",
                 "parallelism": f"replicas x{world} (independent batches, no collective)",
                 "host_cores": host_cores,

@@ -584,8 +584,8 @@ class DecodeStep:
                     self.out = self._outs[i]
                     try:
                         # the cascade's suffixes keep the batch order: longest first
-                        # measured slower there (the suffix blocks were allocated
-                        # in batch order, and sorting scatters their reads)
+                        # measured slower there (short suffixes leave little tail to
+                        # remove)
                         self.run(dq, dk, dv, ds, dbt, dcl, seq_order=None if self.groups is not None else dord)
                     finally:
                         self.out = keep
