@@ -345,11 +345,11 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  * are widened exactly: chunks of more than 128 / group tokens use f16 for QK^T
  * (q scaled per row by a power of two into f16 range, exact for bf16 q) and,
  * with one scale per KV head, f16 for PV too; with per-token scales PV runs in
- * bf16; shorter chunks use bf16. The softmax weights are rounded to the PV
- * operand type and the normaliser sums those rounded weights, except with
- * per-token scales, where a weight is multiplied by its token's V scale
- * before rounding and the normaliser sums the unscaled weights. out is
- * rounded to bf16.
+ * bf16; shorter chunks use bf16. With per-token scales, scores are scaled
+ * by their token's K scale, and V is dequantised to bf16 before P V (each
+ * code times its token's V scale in fp32, rounded to bf16). The softmax
+ * weights are rounded to the PV operand type and the normaliser sums those
+ * rounded weights. out is rounded to bf16.
  *
  *  q             [total_q][num_q_heads][head_dim] bf16, contiguous
  *  block_tables  [num_seqs][max_blocks_per_seq] int32
@@ -362,9 +362,9 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  *                aligned, owned by the caller, contents not kept between
  *                calls. With it, the codes of the sequences whose chunks are
  *                longer than 128 / G tokens are widened once per call into
- *                dense 16-bit rows there (K f16; V f16, or bf16 with
- *                per-token scales; the per-token scales as fp32 rows; zeros
- *                past the context), and the warp-specialised kernel copies
+ *                dense 16-bit rows there (K f16; V f16, or with per-token
+ *                scales V dequantised to bf16 and the K scales as fp32 rows;
+ *                zeros past the context), and the warp-specialised kernel copies
  *                its tiles from there instead of widening the codes in every
  *                CTA: the same operand values, so the same result for finite
  *                cache contents. NULL: the CTAs widen the codes themselves.
@@ -400,7 +400,7 @@ PKV_API int pkv_paged_attention_prefill(const void *q, const void *k_cache, cons
 /*
  * pkv_prefill_workspace_bytes: size of the optional widening workspace of
  * pkv_paged_attention_prefill for an E4M3 cache:
- *   num_seqs * num_kv_heads * R * (4 * head_dim + (per-token scales ? 8 : 0))
+ *   num_seqs * num_kv_heads * R * (4 * head_dim + (per-token scales ? 4 : 0))
  * with R = max_blocks_per_seq * block_size rounded up to a multiple of 128
  * (the table's capacity: one run of R staging rows per sequence and KV
  * head). 0 for a bf16 cache, for arguments below 1, and when the staging

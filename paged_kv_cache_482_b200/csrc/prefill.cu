@@ -85,18 +85,18 @@ template <int D, bool FP8, bool TS = false>
 __device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const BlockIds &table, int kh, int j, int kv_end,
                                              int log2_bs, uint32_t sk, uint32_t sv, float *scales = nullptr) {
     if constexpr (TS) {
-        // K scales of the tile's tokens in scales[0..kBN), V scales in [kBN, 2 kBN); 0 past the end
-        if (threadIdx.x < 2 * kBN) {
-            const int t = threadIdx.x % kBN;
-            const bool is_v = threadIdx.x >= kBN;
+        // K scales of the tile's tokens in scales[0..kBN), 0 past the end (the
+        // V scales are applied to V as it is staged, below)
+        if (threadIdx.x < kBN) {
+            const int t = threadIdx.x;
             const int pos = j * kBN + t;
             float sc = 0.0f;
             if (pos < kv_end) {
                 const int64_t blk = table[pos >> log2_bs];
                 const int64_t idx = (blk * a.num_kv_heads + kh) * a.block_size + (pos & (a.block_size - 1));
-                sc = __ldg((is_v ? a.v_scale : a.k_scale) + idx);
+                sc = __ldg(a.k_scale + idx);
             }
-            scales[threadIdx.x] = sc;
+            scales[t] = sc;
         }
     }
     constexpr int kChunks = D / 8;             // 16-byte chunks per bf16 row
@@ -114,12 +114,15 @@ __device__ __forceinline__ void load_kv_tile(const PrefillArgs &a, const BlockId
         const uint32_t off = swz(kBN, t, c16);
         if constexpr (FP8) {
             uint2 kw = make_uint2(0, 0), vw = make_uint2(0, 0);
+            float vs = 0.0f;
             if (valid) {
                 kw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(a.k_cache) + elem));
                 vw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(a.v_cache) + elem));
+                if constexpr (TS) vs = __ldg(a.v_scale + elem / D);  // the row's V scale
             }
             st_shared16(sk + off, e4m3x8_to_bf16x8(kw));
-            st_shared16(sv + off, e4m3x8_to_bf16x8(vw));
+            // per-token scales: V is dequantised here (bf16 of code x scale), so P needs no scaling
+            st_shared16(sv + off, TS ? e4m3x8_scaled_bf16x8(vw, vs) : e4m3x8_to_bf16x8(vw));
         } else {
             const __nv_bfloat16 *kc = static_cast<const __nv_bfloat16 *>(a.k_cache);
             const __nv_bfloat16 *vc = static_cast<const __nv_bfloat16 *>(a.v_cache);
@@ -404,14 +407,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 const int i0 = c * 8 + 2 * h;
-                if constexpr (TS) {
-                    const float p0 = fast_exp2(x[i0] - m_run), p1 = fast_exp2(x[i0 + 1] - m_run);
-                    w[h] = pack_bf16(p0 * tsc[kBN + col0 + i0], p1 * tsc[kBN + col0 + i0 + 1]);
-                    l4[h] += p0 + p1;
-                } else {
-                    w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
-                    l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
-                }
+                w[h] = pack_bf16(fast_exp2(x[i0] - m_run), fast_exp2(x[i0 + 1] - m_run));
+                l4[h] += bf16lo(w[h]) + bf16hi(w[h]);
             }
             st_shared16(sp + swz(kRows, row, col0 / 8 + c), make_uint4(w[0], w[1], w[2], w[3]));
         }

@@ -38,10 +38,11 @@
 // Operand types: bf16 for a bf16 cache. For E4M3, f16: every E4M3 value is
 // an f16 value (one conversion per two codes), Q is scaled per row by a power
 // of two into f16 range (exact for bf16 input), and P is packed as f16. With
-// per-token scales, the converters also stage the tile's K and V scales;
-// scores are scaled by column, P is multiplied by the V scales before it is
-// rounded, and P V runs in bf16 (V widened to bf16), since P times a V scale
-// may leave f16 range.
+// per-token scales, the converters also stage the tile's K scales, scores are
+// scaled by column, and V is dequantised as it is widened (each code times its
+// row's scale in fp32, rounded to bf16), so P V runs in bf16 and P needs no
+// scaling: the weights are rounded to bf16 and the normaliser sums the
+// rounded weights, as for a bf16 cache.
 // With a workspace (E4M3 only), a widening kernel first expands the codes of
 // the sequences with long chunks once into dense 16-bit rows (K f16; V f16,
 // or bf16 with per-token scales; the per-token scales as fp32 rows), one
@@ -134,12 +135,12 @@ __device__ __forceinline__ void ws_kv_tile(const CUtensorMap *mk, const CUtensor
 
 // Dense staging of E4M3 K/V (workspace layout): rows of D 16-bit values,
 // row (s * num_kv_heads + kv head) * staging_stride + position; K rows, then V
-// rows, then (per-token scales) the K and V scales as fp32, one per row.
+// rows, then (per-token scales) the K scales as fp32, one per row (V is
+// staged dequantised, so its scales are not needed).
 struct Staging {
     uint16_t *k;
     uint16_t *v;
     float *k_scale;
-    float *v_scale;
 };
 
 template <int D>
@@ -149,7 +150,6 @@ __host__ __device__ __forceinline__ Staging staging_of(const PrefillArgs &a) {
     st.k = static_cast<uint16_t *>(a.staging);
     st.v = st.k + rows * D;
     st.k_scale = reinterpret_cast<float *>(st.v + rows * D);
-    st.v_scale = st.k_scale + rows;
     return st;
 }
 
@@ -203,15 +203,18 @@ __global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(PrefillArgs a, 
         }
         const int cc = threadIdx.x % kCPR;  // the same 16-code column in every chunk of this thread
         uint4 kc[kIt], vc[kIt];
+        float vs[kIt];
 #pragma unroll
         for (int u = 0; u < kIt; ++u) {
             kc[u] = make_uint4(0, 0, 0, 0);
             vc[u] = kc[u];
+            vs[u] = 0.0f;
             if (prow[u] >= 0) {
                 kc[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.k_cache) + prow[u] * D +
                                                             cc * 16));
                 vc[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.v_cache) + prow[u] * D +
                                                             cc * 16));
+                if constexpr (TS) vs[u] = __ldg(a.v_scale + prow[u]);
             }
         }
 #pragma unroll
@@ -222,9 +225,9 @@ __global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(PrefillArgs a, 
                 const uint2 h2 = e4m3x4_to_f16x4(kc[u].z), h3 = e4m3x4_to_f16x4(kc[u].w);
                 k0 = make_uint4(h0.x, h0.y, h1.x, h1.y);
                 k1 = make_uint4(h2.x, h2.y, h3.x, h3.y);
-                if constexpr (TS) {  // P V runs in bf16 with per-token scales
-                    v0 = e4m3x8_to_bf16x8(make_uint2(vc[u].x, vc[u].y));
-                    v1 = e4m3x8_to_bf16x8(make_uint2(vc[u].z, vc[u].w));
+                if constexpr (TS) {  // per-token scales: V dequantised (bf16 of code x scale), P V in bf16
+                    v0 = e4m3x8_scaled_bf16x8(make_uint2(vc[u].x, vc[u].y), vs[u]);
+                    v1 = e4m3x8_scaled_bf16x8(make_uint2(vc[u].z, vc[u].w), vs[u]);
                 } else {
                     const uint2 g0 = e4m3x4_to_f16x4(vc[u].x), g1 = e4m3x4_to_f16x4(vc[u].y);
                     const uint2 g2 = e4m3x4_to_f16x4(vc[u].z), g3 = e4m3x4_to_f16x4(vc[u].w);
@@ -242,18 +245,16 @@ __global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(PrefillArgs a, 
         if constexpr (TS) {
             for (int rr = threadIdx.x; rr < kBN; rr += blockDim.x) {
                 const int t = t0 + rr;
-                float ks = 0.0f, vs = 0.0f;
+                float ks = 0.0f;
                 if (t < ctx) {
                     const int b = __ldg(table + (t >> log2_bs));
                     if (b >= 0 && b < a.num_blocks) {
                         const long long prow = (static_cast<long long>(b) * a.num_kv_heads + kh) * a.block_size +
                                                (t & (a.block_size - 1));
                         ks = __ldg(a.k_scale + prow);
-                        vs = __ldg(a.v_scale + prow);
                     }
                 }
                 st.k_scale[drow0 + rr] = ks;
-                st.v_scale[drow0 + rr] = vs;
             }
         }
     }
@@ -279,8 +280,8 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
     constexpr int TQ = kRowsT / G;  // chunk tokens per query tile
     // bf16 cache: bf16 operands. E4M3 cache: f16 operands for S (one conversion
     // per two codes; Q is scaled into f16 range per row, see the staging below)
-    // and for P V with one scale per KV head. With one scale per token, P is
-    // multiplied by the V scales before it is rounded, which may leave f16
+    // and for P V with one scale per KV head. With one scale per token, V is
+    // dequantised to bf16 (code times its row's scale), which may leave f16
     // range: P V then runs in bf16 (P and V both bf16).
     constexpr uint32_t kIdescS = FP8 ? idesc_f16(kRowsT, kBN, false) : idesc_bf16(kRowsT, kBN, false);
     constexpr uint32_t kIdescPV = (FP8 && !TS) ? idesc_f16(kRowsT, D, true) : idesc_bf16(kRowsT, D, true);
@@ -543,12 +544,7 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
                 for (int i = 0; i < 32; ++i) {
                     const float2 t = __ffma2_rn(make_float2(x[hh * 64 + 2 * i], x[hh * 64 + 2 * i + 1]), sl2x2, nm2);
                     uint32_t w;
-                    if constexpr (TS) {  // P times the V scales of its columns, in bf16; l sums the unscaled weights
-                        const float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
-                        const float2 v2 = *reinterpret_cast<const float2 *>(tsc + kBN + hh * 64 + 2 * i);
-                        w = pack_bf16(p0 * v2.x, p1 * v2.y);
-                        l4[i & 3] += p0 + p1;
-                    } else if constexpr (FP8) {  // P in f16 (the E4M3 path's operand type)
+                    if constexpr (FP8 && !TS) {  // P in f16 (the E4M3 path's operand type)
                         w = pack_f16(fast_exp2(t.x), fast_exp2(t.y));
                         l4[i & 3] = fma_f16x2_acc(w, 0x3C003C00u, l4[i & 3]);
                     } else {
@@ -637,7 +633,7 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
                 if constexpr (STG) {
                     uint64_t *bar = &bars->kv_full[st];
                     const int row = srow0 + j * kBN;
-                    mbar_arrive_expect_tx(bar, 2u * (D / 64) * kBN * 128u + (TS ? 2u * kBN * 4u : 0u));
+                    mbar_arrive_expect_tx(bar, 2u * (D / 64) * kBN * 128u + (TS ? kBN * 4u : 0u));
 #pragma unroll
                     for (int h = 0; h < D / 64; ++h) {
                         tma_load_2d(kbuf(j) + h * kBN * 128, &map_k, h * 64, row, bar);
@@ -646,8 +642,7 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
                     if constexpr (TS) {
                         const Staging sg = staging_of<D>(a);
                         float *tsc = reinterpret_cast<float *>(sm + L::kScales) + st * 2 * kBN;
-                        bulk_g2s(tsc, sg.k_scale + row, kBN * 4, bar);
-                        bulk_g2s(tsc + kBN, sg.v_scale + row, kBN * 4, bar);
+                        bulk_g2s(tsc, sg.k_scale + row, kBN * 4, bar);  // V came dequantised
                     }
                 } else {
                     ws_kv_tile<D>(&map_k, &map_v, table, a.num_kv_heads, kh, a.block_size, log2_bs, j, kv_end,
@@ -697,28 +692,34 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
         constexpr int kPer = (kHalf + kCW - 1) / kCW;  // per thread and operand
         const int ct = (warp == kProducerWarp ? 0 : warp - kMmaWarp) * 32 + lane;
         uint4 wk[kPer], wv[kPer];
-        auto load = [&](uint4 (&w)[kPer], const void *pool, int j) {
+        // scl (V with per-token scales): also each chunk's row scale
+        auto load = [&](uint4 (&w)[kPer], const void *pool, int j, float *scl) {
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int idx = ct + u * kCW;
                 const int t = j * kBN + idx / kCPR;
                 w[u] = make_uint4(0, 0, 0, 0);
+                if (scl) scl[u] = 0.0f;
                 if (idx < kHalf && t < kv_end) {
-                    const int64_t off = ((static_cast<int64_t>(table[t >> log2_bs]) * a.num_kv_heads + kh) *
-                                             a.block_size + (t & (a.block_size - 1))) * D + (idx % kCPR) * 16;
-                    w[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(pool) + off));
+                    const int64_t row = (static_cast<int64_t>(table[t >> log2_bs]) * a.num_kv_heads + kh) *
+                                            a.block_size + (t & (a.block_size - 1));
+                    w[u] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(pool) + row * D +
+                                                               (idx % kCPR) * 16));
+                    if (scl) scl[u] = __ldg(a.v_scale + row);
                 }
             }
         };
-        auto store = [&](const uint4 (&w)[kPer], uint32_t dst, bool to_bf16) {
+        // scl: V with per-token scales, dequantised to bf16 (code x scale)
+        auto store = [&](const uint4 (&w)[kPer], uint32_t dst, const float *scl) {
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int idx = ct + u * kCW;
                 if (idx < kHalf) {
                     const int r = idx / kCPR, c16 = 2 * (idx % kCPR);
-                    if (to_bf16) {
-                        st_shared16(dst + swz(kBN, r, c16), e4m3x8_to_bf16x8(make_uint2(w[u].x, w[u].y)));
-                        st_shared16(dst + swz(kBN, r, c16 + 1), e4m3x8_to_bf16x8(make_uint2(w[u].z, w[u].w)));
+                    if (scl) {
+                        st_shared16(dst + swz(kBN, r, c16), e4m3x8_scaled_bf16x8(make_uint2(w[u].x, w[u].y), scl[u]));
+                        st_shared16(dst + swz(kBN, r, c16 + 1),
+                                    e4m3x8_scaled_bf16x8(make_uint2(w[u].z, w[u].w), scl[u]));
                     } else {
                         const uint2 h0 = e4m3x4_to_f16x4(w[u].x), h1 = e4m3x4_to_f16x4(w[u].y);
                         const uint2 h2 = e4m3x4_to_f16x4(w[u].z), h3 = e4m3x4_to_f16x4(w[u].w);
@@ -753,9 +754,11 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
                 if (i < 2 * kBN) dst[i] = sc[u];
             }
         };
+        float vsc[kPer];  // per-token scales: the V rows' scales of this thread's chunks
+        float *vs_ptr = TS ? vsc : nullptr;
         bool ok = true;
-        load(wk, a.k_cache, 0);
-        load(wv, a.v_cache, 0);
+        load(wk, a.k_cache, 0, nullptr);
+        load(wv, a.v_cache, 0, vs_ptr);
         if (TS) load_scales(0);
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages, use = j / kStages;
@@ -767,12 +770,12 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
             // K of tile j, then the next tile's K codes load while V is widened
             // (to bf16 with per-token scales, where P V runs in bf16)
             if (TS) store_scales(j);
-            store(wk, kbuf(j), false);
-            if (j + 1 < n_tiles) load(wk, a.k_cache, j + 1);
-            store(wv, vbuf(j), TS);
+            store(wk, kbuf(j), nullptr);
+            if (j + 1 < n_tiles) load(wk, a.k_cache, j + 1, nullptr);
+            store(wv, vbuf(j), vs_ptr);
             if (lane == 0) mbar_arrive(&bars->kv_full[st]);
             if (j + 1 < n_tiles) {
-                load(wv, a.v_cache, j + 1);
+                load(wv, a.v_cache, j + 1, vs_ptr);
                 if (TS) load_scales(j + 1);
             }
         }
@@ -1012,7 +1015,7 @@ size_t prefill_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int
     const long long stride = prefill_staging_stride(max_blocks_per_seq, block_size);
     const long long rows = static_cast<long long>(num_seqs) * num_kv_heads * stride;
     if (stride == 0 || rows > 0x7FFFFFFFLL) return 0;
-    return static_cast<size_t>(rows) * (4u * static_cast<size_t>(head_dim) + (token_scales ? 8u : 0u));
+    return static_cast<size_t>(rows) * (4u * static_cast<size_t>(head_dim) + (token_scales ? 4u : 0u));
 }
 
 cudaError_t launch_prefill_ws(const PrefillArgs &a, cudaStream_t stream) {

@@ -251,6 +251,22 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 w) {
     return o;
 }
 
+// Eight E4M3 codes times one fp32 scale -> eight bf16 values (each product
+// formed in fp32, then rounded to bf16): a V row of a per-token-scale cache,
+// dequantised for a bf16 P V.
+__device__ __forceinline__ uint4 e4m3x8_scaled_bf16x8(uint2 w, float s) {
+    uint4 o;
+    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w.x & 0xFFFFu));
+    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w.x >> 16));
+    float2 c = e4m3x2_to_float2(static_cast<uint16_t>(w.y & 0xFFFFu));
+    float2 d = e4m3x2_to_float2(static_cast<uint16_t>(w.y >> 16));
+    o.x = pack_bf16(a.x * s, a.y * s);
+    o.y = pack_bf16(b.x * s, b.y * s);
+    o.z = pack_bf16(c.x * s, c.y * s);
+    o.w = pack_bf16(d.x * s, d.y * s);
+    return o;
+}
+
 // Byte offset of 16-byte chunk c16 of row r in a swizzled operand of `rows` rows.
 __device__ __forceinline__ uint32_t swz(int rows, int r, int c16) {
     return static_cast<uint32_t>((c16 >> 3) * rows * 128 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));

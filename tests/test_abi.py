@@ -227,7 +227,7 @@ def test_prefill_workspace_bytes(K):
     wb = K.prefill_workspace_bytes
     # rows per (sequence, KV head): the table capacity rounded up to 128
     assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_FP8_E4M3) == 4 * 8 * 2048 * (4 * 128)
-    assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_FP8_E4M3_TOKEN) == 4 * 8 * 2048 * (4 * 128 + 8)
+    assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_FP8_E4M3_TOKEN) == 4 * 8 * 2048 * (4 * 128 + 4)
     assert wb(3, 2, 64, 3, 16, K.PKV_CACHE_FP8_E4M3) == 3 * 2 * 128 * (4 * 64)
     assert wb(1, 1, 128, 9, 16, K.PKV_CACHE_FP8_E4M3) == 256 * 512  # 144 -> 256 rows
     assert wb(4, 8, 128, 8, 256, K.PKV_CACHE_BF16) == 0
