@@ -489,20 +489,19 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
             tmem_ld128(tmem_s + lane_base, x);
             const float *tsc = reinterpret_cast<const float *>(sm + L::kScales) + (j % kStages) * 2 * kBN;
             if constexpr (TS) {
-                // the converters staged this tile's per-token scales with its codes:
-                // x = s * (sl2 * k_scale of the column). The stage is refilled only
-                // after both query tiles have released this tile, so this wait
-                // cannot see a later phase.
+                // the tile's per-token K scales were staged with its codes: x = s *
+                // k_scale of the column (the row's sl2 enters below, as without
+                // per-token scales). The stage is refilled only after both query
+                // tiles have released this tile, so this wait cannot see a later phase.
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_full[j % kStages],
                                                        static_cast<uint32_t>((j / kStages) & 1)))) {
                     ok = false;
                     break;
                 }
-                const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
                 for (int i = 0; i < kBN / 2; ++i) {
                     const float2 k2 = *reinterpret_cast<const float2 *>(tsc + 2 * i);
-                    const float2 v2 = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), __fmul2_rn(sl2x2, k2));
+                    const float2 v2 = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), k2);
                     x[2 * i] = v2.x;
                     x[2 * i + 1] = v2.y;
                 }
@@ -517,8 +516,8 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
             for (int k = 0; k < 8; ++k) m8[k] = x[k];
 #pragma unroll
             for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-            const float mx = (TS ? 1.0f : sl2) * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            const float mx = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             float alpha = 1.0f;
             bool rescale = false;
             if (j == 0) {
@@ -535,7 +534,7 @@ __global__ void __launch_bounds__(ws_threads<FP8 && !STG>(), 1)
             // P as 16-bit pairs (bf16, or f16 for E4M3 with per-head scales) over
             // columns 0..63 of S: scores 64 hh .. 64 hh + 63 go to columns
             // 32 hh .. 32 hh + 31 (all scores are in registers)
-            const float2 sl2x2 = make_float2(TS ? 1.0f : sl2, TS ? 1.0f : sl2), nm2 = make_float2(-m_run, -m_run);
+            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
             float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
