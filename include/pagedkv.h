@@ -360,7 +360,9 @@ PKV_API int pkv_paged_attention_decode_static_scratch(
  *  workspace     optional, E4M3 cache only (ignored for bf16; may be NULL):
  *                at least pkv_prefill_workspace_bytes(...) bytes, 16-byte
  *                aligned, owned by the caller, contents not kept between
- *                calls. With it, the codes of the sequences whose chunks are
+ *                calls (calls that may run at the same time, on different
+ *                streams, need separate workspaces). With it, the codes of
+ *                the sequences whose chunks are
  *                longer than 128 / G tokens are widened once per call into
  *                dense 16-bit rows there (K f16; V f16, or with per-token
  *                scales V dequantised to bf16 and the K scales as fp32 rows;
