@@ -280,7 +280,8 @@ PKV_API int pkv_paged_attention_decode(const void *q, const void *k_cache, const
  *
  * Device checks: a P_j that is not a multiple of block_size or exceeds a
  * member's context, a member whose shared block ids differ from the first
- * member's, or groups that do not lie inside the batch set
+ * member's, a group larger than max_group_seqs, or groups that do not lie
+ * inside the batch set
  * PKV_DEVERR_BOUNDS and the affected sequences' out rows are written as
  * zeros (where they can be located). head_dim 64, or num_groups == 0,
  * run the ordinary decode (same result).

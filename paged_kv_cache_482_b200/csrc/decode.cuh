@@ -115,11 +115,14 @@ __device__ __forceinline__ int group_of(const DecodeParams &p, int seq) {
 }
 
 // Prefix length of sequence seq in shared-prefix mode, or -1 when it is not
-// usable (negative, not a whole number of blocks, past the context, or the
-// sequence in no group).
+// usable (negative, not a whole number of blocks, past the context, the
+// sequence in no group, or a group larger than the host's bound
+// max_group_seqs, whose members past the bound no prefix kernel covers).
 __device__ __forceinline__ int prefix_of(const DecodeParams &p, int seq, int ctx) {
     const int j = group_of(p, seq);
-    if (j < 0 || seq >= __ldg(p.cu_group_seqs + j + 1)) return -1;
+    if (j < 0) return -1;
+    const int g1 = __ldg(p.cu_group_seqs + j + 1);
+    if (seq >= g1 || g1 - __ldg(p.cu_group_seqs + j) > p.max_group_seqs) return -1;
     const int P = __ldg(p.group_prefix + j);
     if (P < 0 || P > ctx || (P & (p.block_size - 1)) != 0) return -1;
     return P;

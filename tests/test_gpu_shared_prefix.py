@@ -206,3 +206,26 @@ def test_cascade_with_seq_order_is_bit_identical(dt):
     assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS
     keep = [i for i in range(S) if i != 5]
     assert torch.equal(out[keep].view(torch.int16), base[keep].view(torch.int16))
+
+
+def test_group_larger_than_the_stated_bound():
+    """max_group_seqs below the largest group: the prefix kernels' grid does not
+    cover that group's later members, so the whole group is reported
+    (PKV_DEVERR_BOUNDS) and written as zeros; the other groups are exact."""
+    wl_cpu = mixed_groups(W.CACHE_BF16, g=4, bs=16, seed=13)
+    wl = to_device(wl_cpu)
+    kp, vp = pools_for(wl)
+    cu, pre, _ = groups_of(wl)
+    sizes = [b - a for a, b in zip(wl.group_bounds[:-1], wl.group_bounds[1:])]
+    bound = sorted(sizes)[-2]  # below the largest group (40 members), at least the others
+    big = sizes.index(max(sizes))
+    c = wl.cfg
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = K.paged_attention_decode_shared_prefix(wl.q, kp, vp, wl.block_tables, wl.context_lens, c.softmax_scale,
+                                                 cu, pre, bound, k_scale=wl.k_scale, v_scale=wl.v_scale,
+                                                 max_context_len=c.max_context, dev_err=err)
+    assert K.read_device_error(err) == K.PKV_ERR_DEVICE_BOUNDS
+    zero = list(range(wl.group_bounds[big], wl.group_bounds[big + 1]))
+    assert bool((out[zero].float() == 0).all())
+    keep = [i for i in range(c.num_seqs) if i not in zero]
+    compare(out[keep], oracle_of(wl_cpu)[keep], False, "groups within the bound")
